@@ -1,0 +1,260 @@
+"""Pins for the CPU oracle, against things other than itself.
+
+The oracle restates RMS-Norm (Background, Equation 1 of "SwiftQK: Fast and
+Communication-Efficient Tensor Parallelism for Query-Key Normalization") and its
+Phase A shard decomposition in double precision.  Before any GPU result is
+compared with it, it is checked here against:
+
+* hand-derived closed forms (``tests/golden/closed_forms.json``);
+* a library routine that computes the same definition
+  (``torch.nn.functional.rms_norm`` in float64) and torch's own float32 ->
+  bfloat16 rounding;
+* invariants the mathematics fixes (output RMS with gamma = 1, scale
+  invariance, one-hot and power-of-two gamma, the shard-sum identity).
+
+Each plausible slip — a dropped eps, a sum instead of a mean, a shard width
+used as the divisor, a wrong sign, a stride or gamma index mix-up, truncation
+instead of round-to-nearest-even — fails at least one test below.
+"""
+from __future__ import annotations
+
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from tests.conftest import buffer_np, to_np
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "closed_forms.json")
+
+
+def _golden():
+    with open(GOLDEN) as f:
+        return json.load(f)
+
+
+def _parse_value(s):
+    if isinstance(s, (int, float)):
+        return float(s)
+    table = {"inf": math.inf, "-inf": -math.inf, "-0": -0.0}
+    if s in table:
+        return table[s]
+    # small closed-form expressions over powers of two, e.g. "1 + 3*2^-8"
+    return float(eval(s.replace("^", "**"), {"__builtins__": {}}, {}))
+
+
+# --------------------------------------------------------------------------- codec
+
+def test_bf16_decode_matches_field_definition():
+    for case in _golden()["bf16_decode"]:
+        got = oracle.bf16_decode([int(case["bits"], 16)])[0]
+        want = _parse_value(case["value"])
+        assert got == want and math.copysign(1, got) == math.copysign(1, want), case
+
+
+def test_bf16_encode_ties_to_even_fixtures():
+    for case in _golden()["bf16_encode_rne"]:
+        got = int(oracle.bf16_encode([_parse_value(case["value"])])[0])
+        assert got == int(case["bits"], 16), (case, hex(got))
+
+
+def test_bf16_encode_matches_torch_rounding_of_float32():
+    """torch rounds float32 -> bfloat16 to nearest, ties to even.  Every float32
+    is exact in double, so the oracle's single rounding must agree bit for bit.
+    Exact ties (low 16 bits == 0x8000) are included on purpose."""
+    g = torch.Generator().manual_seed(11)
+    raw = torch.randint(0, 2**31 - 1, (20000,), generator=g, dtype=torch.int64)
+    bits = raw.to(torch.int32)
+    ties = (bits & ~0xFFFF) | 0x8000
+    all_bits = torch.cat([bits, ties, -bits, -ties])
+    f = all_bits.view(torch.float32)
+    f = f[torch.isfinite(f)]
+    want = f.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    got = oracle.bf16_encode(f.double().numpy())
+    assert np.array_equal(got, want)
+
+
+def test_bf16_decode_matches_torch_for_every_finite_pattern():
+    bits = np.arange(0, 1 << 16, dtype=np.uint32).astype(np.uint16)
+    vals = torch.from_numpy(bits.view(np.int16).copy()).view(torch.bfloat16).double().numpy()
+    got = oracle.bf16_decode(bits)
+    finite = np.isfinite(vals)
+    assert np.array_equal(got[finite], vals[finite])
+    assert np.array_equal(np.isnan(got), np.isnan(vals))
+
+
+# --------------------------------------------------------------------------- closed forms
+
+def test_rmsnorm_closed_forms():
+    for case in _golden()["rmsnorm"]:
+        x = np.array(case["x"], dtype=np.float32)[None, :]
+        gm = np.array(case["gamma"], dtype=np.float32)
+        H = x.shape[1]
+        _, y, s = oracle.rmsnorm_rows(x, H, gm, case["eps"])
+        assert s[0] == case["sumsq"], case["name"]
+        np.testing.assert_allclose(y[0], case["y"], rtol=1e-15, atol=0, err_msg=case["name"])
+
+
+def test_sharded_closed_form_divides_by_full_width():
+    case = _golden()["sharded"][0]
+    x = np.array(case["x_full"], dtype=np.float32)
+    gm = np.array(case["gamma_full"], dtype=np.float32)
+    widths = case["shard_widths"]
+    H = int(sum(widths))
+    cols = np.cumsum([0] + widths)
+    parts = []
+    for p, w in enumerate(widths):
+        xs = np.ascontiguousarray(x[cols[p]:cols[p + 1]][None, :])
+        parts.append(oracle.partial_sumsq(xs, w, w, 1))
+    assert [float(v[0]) for v in parts] == case["partial_sumsq"]
+    stats = np.stack(parts)
+    for p, w in enumerate(widths):
+        xs = np.ascontiguousarray(x[cols[p]:cols[p + 1]][None, :])
+        gs = np.ascontiguousarray(gm[cols[p]:cols[p + 1]])
+        _, y = oracle.combine_apply(xs, w, w, 1, gs, stats, H, case["eps"])
+        np.testing.assert_allclose(y[0], case["y_shards"][p], rtol=1e-15, atol=0)
+
+
+# --------------------------------------------------------------------------- library routine
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("T,H,pad", [(1, 1, 0), (3, 7, 5), (17, 64, 3), (9, 513, 0), (4, 4096, 8)])
+def test_rmsnorm_matches_torch_rms_norm_float64(dtype, T, H, pad):
+    g = torch.Generator().manual_seed(1000 + T * 7 + H)
+    stride = H + pad
+    buf = (torch.randn((T, stride), generator=g) * 3.0).to(dtype)
+    view = buf[:, :H]
+    gm = (1.0 + 0.1 * torch.randn((H,), generator=g)).to(dtype)
+    eps = 1e-6
+    flat, st = buffer_np(view)
+    y_rounded, y, s = oracle.rmsnorm_rows(flat, H, to_np(gm), eps, stride=st, T=T)
+    ref = torch.nn.functional.rms_norm(view.double(), (H,), weight=gm.double(), eps=eps)
+    np.testing.assert_allclose(y, ref.numpy(), rtol=1e-13, atol=1e-300)
+    np.testing.assert_allclose(s, (view.double() ** 2).sum(dim=1).numpy(), rtol=1e-13)
+    # the stored output is one correct rounding of the double result
+    if dtype == torch.float32:
+        assert np.array_equal(y_rounded, y.astype(np.float32))
+    else:
+        assert np.array_equal(y_rounded, oracle.bf16_encode(y))
+
+
+def test_layerwise_treats_q_and_k_independently():
+    g = torch.Generator().manual_seed(5)
+    T, Hq, Hk = 6, 40, 24
+    q = torch.randn((T, Hq), generator=g)
+    k = torch.randn((T, Hk), generator=g) * 10
+    gq = 1 + 0.1 * torch.randn((Hq,), generator=g)
+    gk = 1 + 0.1 * torch.randn((Hk,), generator=g)
+    qo, ko = oracle.qknorm_layerwise(to_np(q), Hq, to_np(gq), Hq, to_np(k), Hk, to_np(gk), Hk, T, 1e-6)
+    rq = torch.nn.functional.rms_norm(q.double(), (Hq,), weight=gq.double(), eps=1e-6).float()
+    rk = torch.nn.functional.rms_norm(k.double(), (Hk,), weight=gk.double(), eps=1e-6).float()
+    np.testing.assert_allclose(qo, rq.numpy(), rtol=2e-7)
+    np.testing.assert_allclose(ko, rk.numpy(), rtol=2e-7)
+
+
+# --------------------------------------------------------------------------- invariants
+
+@pytest.mark.parametrize("eps_ratio", [0.0, 1e-6, 1.0, 37.0])
+def test_output_rms_with_unit_gamma(eps_ratio):
+    """gamma = 1: mean_j y_j^2 = m / (m + eps) exactly, m = mean_j x_j^2."""
+    g = torch.Generator().manual_seed(21)
+    T, H = 8, 300
+    x = torch.randn((T, H), generator=g, dtype=torch.float32)
+    m = (x.double() ** 2).mean(dim=1).numpy()
+    eps = float(eps_ratio * m.mean())
+    _, y, _ = oracle.rmsnorm_rows(to_np(x), H, np.ones(H, np.float32), eps)
+    got = (y ** 2).mean(axis=1)
+    np.testing.assert_allclose(got, m / (m + eps), rtol=1e-13)
+
+
+def test_scale_invariance_power_of_two():
+    """eps = 0 and c = 2^k: every step scales exactly, so y(c x) == y(x) bit for bit.
+    With eps small against mean(x^2) the two agree to about eps / mean(x^2)."""
+    g = torch.Generator().manual_seed(22)
+    T, H = 5, 256
+    x = torch.randn((T, H), generator=g, dtype=torch.float32)
+    gm = (1 + 0.1 * torch.randn((H,), generator=g)).float()
+    _, y0, _ = oracle.rmsnorm_rows(to_np(x), H, to_np(gm), 0.0)
+    for c in (2.0 ** -7, 2.0 ** 6):
+        _, yc, _ = oracle.rmsnorm_rows(to_np(x * c), H, to_np(gm), 0.0)
+        assert np.array_equal(yc, y0)
+    for c in (1e-2, 1e2):
+        _, yc, _ = oracle.rmsnorm_rows(to_np((x.double() * c).float()), H, to_np(gm), 1e-12)
+        np.testing.assert_allclose(yc, y0, rtol=1e-6)
+
+
+def test_one_hot_gamma_selects_one_column():
+    g = torch.Generator().manual_seed(23)
+    T, H, col = 4, 33, 17
+    x = torch.randn((T, H), generator=g, dtype=torch.float32)
+    gm = np.zeros(H, np.float32)
+    gm[col] = 1.0
+    _, y, s = oracle.rmsnorm_rows(to_np(x), H, gm, 1e-6)
+    assert np.count_nonzero(y[:, np.arange(H) != col]) == 0
+    r = 1.0 / np.sqrt(s / H + 1e-6)
+    np.testing.assert_allclose(y[:, col], x[:, col].double().numpy() * r, rtol=1e-15)
+
+
+def test_power_of_two_gamma_scales_exactly():
+    g = torch.Generator().manual_seed(24)
+    T, H = 3, 100
+    x = torch.randn((T, H), generator=g, dtype=torch.float32)
+    _, y1, _ = oracle.rmsnorm_rows(to_np(x), H, np.ones(H, np.float32), 1e-6)
+    _, y8, _ = oracle.rmsnorm_rows(to_np(x), H, np.full(H, 8.0, np.float32), 1e-6)
+    assert np.array_equal(y8, 8.0 * y1)
+
+
+def test_shard_sums_add_to_full_sum_exactly_for_integers():
+    """Small integers: every square and partial sum is exact in double, so
+    sum_p S_p == S_full with no rounding at all (Phase A identity)."""
+    g = torch.Generator().manual_seed(25)
+    T, H, P = 7, 96, 4
+    x = torch.randint(-50, 51, (T, H), generator=g).float()
+    _, _, s_full = oracle.rmsnorm_rows(to_np(x), H, np.ones(H, np.float32), 0.0)
+    w = H // P
+    parts = [oracle.partial_sumsq(to_np(x[:, p * w:(p + 1) * w]), w, w, T) for p in range(P)]
+    assert np.array_equal(np.sum(parts, axis=0), s_full)
+    assert np.array_equal(s_full, (x.double() ** 2).sum(dim=1).numpy())
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_shard_pipeline_matches_full_row(dtype):
+    """partial_sumsq per shard, then combine_apply per shard, reproduces the
+    unsharded normalization (same global semantics, Phase A)."""
+    g = torch.Generator().manual_seed(26)
+    T, Hq, P = 11, 160, 4
+    x = torch.randn((T, Hq), generator=g).to(dtype)
+    gm = (1 + 0.1 * torch.randn((Hq,), generator=g)).to(dtype)
+    _, y_full, _ = oracle.rmsnorm_rows(to_np(x), Hq, to_np(gm), 1e-6)
+    w = Hq // P
+    stats = np.stack([oracle.partial_sumsq(to_np(x[:, p * w:(p + 1) * w]), w, w, T) for p in range(P)])
+    for p in range(P):
+        _, yp = oracle.combine_apply(to_np(x[:, p * w:(p + 1) * w]), w, w, T,
+                                     to_np(gm[p * w:(p + 1) * w]), stats, Hq, 1e-6)
+        np.testing.assert_allclose(yp, y_full[:, p * w:(p + 1) * w], rtol=1e-14)
+
+
+def test_strided_rows_read_only_their_columns():
+    """Padding columns hold huge values; they must not leak into the result."""
+    T, H, stride = 4, 10, 16
+    buf = np.full((T, stride), 1e30, dtype=np.float32)
+    buf[:, :H] = np.arange(1, H + 1, dtype=np.float32)
+    _, y, s = oracle.rmsnorm_rows(buf, H, np.ones(H, np.float32), 0.0, stride=stride, T=T)
+    assert np.all(s == 385.0)  # 1^2 + ... + 10^2
+    np.testing.assert_allclose(y[0], np.arange(1, H + 1) / math.sqrt(38.5), rtol=1e-15)
+
+
+def test_empty_batch_and_bad_arguments():
+    y, ye, s = oracle.rmsnorm_rows(np.zeros((0, 8), np.float32), 8, np.ones(8, np.float32), 1e-6, T=0)
+    assert y.shape == (0, 8) and s.shape == (0,)
+    with pytest.raises(ValueError):
+        oracle.rmsnorm_rows(np.zeros((2, 8), np.float32), 8, np.ones(8, np.float32), -1.0)
+    with pytest.raises(ValueError):
+        oracle.rmsnorm_rows(np.zeros((2, 8), np.float32), 8, np.ones(8, np.float32), 1e-6, stride=4, T=2)
+    with pytest.raises(ValueError):
+        oracle.combine_apply(np.zeros((2, 8), np.float32), 8, 8, 2, np.ones(8, np.float32),
+                             np.zeros((1, 2)), 4, 1e-6)  # full width below shard width
