@@ -1,0 +1,218 @@
+"""Layerwise QK-RMSNorm for NVIDIA B200 (sm_100a).
+
+Python binding over the C-ABI library ``libqknorm.so`` (include/qknorm.h).  The
+functions here only marshal torch CUDA tensors into pointers, strides and a
+stream; every step of the computation runs in the library's CUDA kernels.  If
+the library is missing the call raises — there is no CPU path.
+
+RMS-Norm over the full projected Q and K rows of each token ("SwiftQK: Fast and
+Communication-Efficient Tensor Parallelism for Query-Key Normalization",
+Background, Equation 1):  y = x / sqrt(mean(x^2) + eps) * gamma, and its Phase A
+shard decomposition (per-shard squared sums, fp32 aggregation, then scaling).
+
+Tensors: 2-D ``[T, width]`` views whose rows may be strided (``stride(1) == 1``,
+``stride(0) >= width``), e.g. Q and K views into a packed ``[T, Hq+Hk+Hv]``
+buffer.  An output has the same row stride as its input (the C-ABI takes one
+stride per tensor); pass ``q_out=q_in`` to normalize in place.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import _clib
+from ._clib import QknLaunch, QKNormError
+
+__all__ = ["qknorm_layerwise", "qknorm_partial_stats", "qknorm_combine_apply",
+           "qknorm_layerwise_plan", "plan_shape", "plan_grid", "regions_overlap",
+           "capi", "version", "QknLaunch", "QKNormError"]
+
+_DTYPES = {torch.float32: _clib.QKN_F32, torch.bfloat16: _clib.QKN_BF16}
+
+
+def capi() -> ctypes.CDLL:
+    """The raw C-ABI (functions take pointers and sizes, as in include/qknorm.h)."""
+    return _clib.load()
+
+
+def version() -> int:
+    return capi().qknorm_version()
+
+
+# --------------------------------------------------------------------------- marshalling
+
+def _rows(t: torch.Tensor, name: str):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (this library has no CPU path)")
+    if t.dtype not in _DTYPES:
+        raise TypeError(f"{name}: dtype {t.dtype} unsupported (float32 or bfloat16)")
+    if t.dim() != 2:
+        raise ValueError(f"{name} must be 2-D [T, width]")
+    T, H = t.shape
+    if T > 0 and H > 1 and t.stride(1) != 1:
+        raise ValueError(f"{name} rows must be unit-stride along the width")
+    stride = t.stride(0) if T > 1 else max(t.stride(0), H)
+    return T, H, stride
+
+
+def _vec(t: torch.Tensor, name: str, n: int, dtype: torch.dtype, device):
+    if not (isinstance(t, torch.Tensor) and t.is_cuda and t.dtype == dtype and t.is_contiguous()
+            and t.numel() == n and t.device == device):
+        raise ValueError(f"{name} must be a contiguous CUDA {dtype} tensor of {n} elements on {device}")
+    return t.data_ptr()
+
+
+def _out_like(x: torch.Tensor, stride: int) -> torch.Tensor:
+    T, H = x.shape
+    return torch.empty_strided((T, H), (stride, 1), dtype=x.dtype, device=x.device)
+
+
+def _stream_handle(stream, device) -> int:
+    if stream is None:
+        return torch.cuda.current_stream(device).cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _same(dev_a, dtype_a, t: torch.Tensor, name: str):
+    if t.device != dev_a or t.dtype != dtype_a:
+        raise ValueError(f"{name} must be on {dev_a} with dtype {dtype_a}")
+
+
+def _layerwise_args(q_in, k_in, gamma_q, gamma_k, eps, q_out, k_out):
+    Tq, Hq, sq = _rows(q_in, "q_in")
+    Tk, Hk, sk = _rows(k_in, "k_in")
+    if Tq != Tk:
+        raise ValueError(f"q_in and k_in must have the same number of tokens ({Tq} != {Tk})")
+    dev, dt = q_in.device, q_in.dtype
+    _same(dev, dt, k_in, "k_in")
+    if q_out is None:
+        q_out = _out_like(q_in, sq)
+    if k_out is None:
+        k_out = _out_like(k_in, sk)
+    for t, name, (T, H, s) in ((q_out, "q_out", (Tq, Hq, sq)), (k_out, "k_out", (Tk, Hk, sk))):
+        _same(dev, dt, t, name)
+        To, Ho, so = _rows(t, name)
+        if (To, Ho) != (T, H) or (T > 1 and so != s):
+            raise ValueError(f"{name} must match its input's shape and row stride")
+    args = [q_in.data_ptr(), q_out.data_ptr(), _vec(gamma_q, "gamma_q", Hq, dt, dev), sq,
+            k_in.data_ptr(), k_out.data_ptr(), _vec(gamma_k, "gamma_k", Hk, dt, dev), sk,
+            Tq, Hq, Hk, float(eps), _DTYPES[dt]]
+    return args, q_out, k_out, dev
+
+
+# --------------------------------------------------------------------------- API
+
+def qknorm_layerwise(q_in: torch.Tensor, k_in: torch.Tensor, gamma_q: torch.Tensor,
+                     gamma_k: torch.Tensor, eps: float = 1e-6, *, q_out=None, k_out=None,
+                     stream=None, launch: QknLaunch | dict | None = None):
+    """Fused layerwise QK-Norm of all tokens in one launch; returns ``(q_out, k_out)``.
+
+    ``launch`` pins a launch shape (``qkn_launch``); results are identical for
+    every valid shape.  Asynchronous on ``stream`` (default: the current stream).
+    """
+    args, q_out, k_out, dev = _layerwise_args(q_in, k_in, gamma_q, gamma_k, eps, q_out, k_out)
+    lib = capi()
+    with torch.cuda.device(dev):
+        s = _stream_handle(stream, dev)
+        if launch is None:
+            st = lib.qknorm_layerwise(*args, s)
+        else:
+            L = launch if isinstance(launch, QknLaunch) else QknLaunch(**launch)
+            st = lib.qknorm_layerwise_launch(*args, s, ctypes.byref(L))
+    _clib.check(st, "qknorm_layerwise")
+    return q_out, k_out
+
+
+def qknorm_layerwise_plan(q_in, k_in, gamma_q, gamma_k, eps: float = 1e-6, *, q_out=None,
+                          k_out=None) -> dict:
+    """The launch ``qknorm_layerwise`` would use for these tensors."""
+    args, _, _, dev = _layerwise_args(q_in, k_in, gamma_q, gamma_k, eps, q_out, k_out)
+    L = QknLaunch()
+    with torch.cuda.device(dev):
+        st = capi().qknorm_layerwise_plan(*args, ctypes.byref(L))
+    _clib.check(st, "qknorm_layerwise_plan")
+    return L.as_dict()
+
+
+def qknorm_partial_stats(q_shard: torch.Tensor, k_shard: torch.Tensor, q_sumsq=None, k_sumsq=None,
+                         *, stream=None):
+    """Phase A local step: fp32 squared sum of every token's Q-shard and K-shard
+    row; returns ``(q_sumsq, k_sumsq)``, each ``[T]`` float32 (a row of a
+    caller-owned ``[P, T]`` array may be passed)."""
+    T, hq, sq = _rows(q_shard, "q_shard")
+    Tk, hk, sk = _rows(k_shard, "k_shard")
+    if T != Tk:
+        raise ValueError("q_shard and k_shard must have the same number of tokens")
+    dev, dt = q_shard.device, q_shard.dtype
+    _same(dev, dt, k_shard, "k_shard")
+    if q_sumsq is None:
+        q_sumsq = torch.empty((T,), dtype=torch.float32, device=dev)
+    if k_sumsq is None:
+        k_sumsq = torch.empty((T,), dtype=torch.float32, device=dev)
+    pq = _vec(q_sumsq, "q_sumsq", T, torch.float32, dev)
+    pk = _vec(k_sumsq, "k_sumsq", T, torch.float32, dev)
+    with torch.cuda.device(dev):
+        st = capi().qknorm_partial_stats(q_shard.data_ptr(), sq, hq, pq, k_shard.data_ptr(), sk, hk, pk,
+                                         T, _DTYPES[dt], _stream_handle(stream, dev))
+    _clib.check(st, "qknorm_partial_stats")
+    return q_sumsq, k_sumsq
+
+
+def qknorm_combine_apply(q_in: torch.Tensor, k_in: torch.Tensor, gamma_q_shard: torch.Tensor,
+                         gamma_k_shard: torch.Tensor, q_sumsq_all: torch.Tensor,
+                         k_sumsq_all: torch.Tensor, Hq_full: int, Hk_full: int, eps: float = 1e-6,
+                         *, q_out=None, k_out=None, stream=None):
+    """Phase A aggregation of the ``[P, T]`` fp32 partial sums (order p = 0..P-1),
+    factor over the FULL widths, then scale this shard; returns ``(q_out, k_out)``."""
+    T, hq, sq = _rows(q_in, "q_in")
+    Tk, hk, sk = _rows(k_in, "k_in")
+    if T != Tk:
+        raise ValueError("q_in and k_in must have the same number of tokens")
+    dev, dt = q_in.device, q_in.dtype
+    _same(dev, dt, k_in, "k_in")
+    if q_sumsq_all.dim() != 2 or k_sumsq_all.dim() != 2 or q_sumsq_all.shape != k_sumsq_all.shape \
+            or q_sumsq_all.shape[1] != T:
+        raise ValueError("q_sumsq_all and k_sumsq_all must both be [P, T]")
+    P = q_sumsq_all.shape[0]
+    ps_q = _vec(q_sumsq_all, "q_sumsq_all", P * T, torch.float32, dev)
+    ps_k = _vec(k_sumsq_all, "k_sumsq_all", P * T, torch.float32, dev)
+    if q_out is None:
+        q_out = _out_like(q_in, sq)
+    if k_out is None:
+        k_out = _out_like(k_in, sk)
+    for t, name, (H, s) in ((q_out, "q_out", (hq, sq)), (k_out, "k_out", (hk, sk))):
+        _same(dev, dt, t, name)
+        To, Ho, so = _rows(t, name)
+        if (To, Ho) != (T, H) or (T > 1 and so != s):
+            raise ValueError(f"{name} must match its input's shape and row stride")
+    with torch.cuda.device(dev):
+        st = capi().qknorm_combine_apply(
+            q_in.data_ptr(), q_out.data_ptr(), _vec(gamma_q_shard, "gamma_q_shard", hq, dt, dev), sq, hq,
+            ps_q, int(Hq_full),
+            k_in.data_ptr(), k_out.data_ptr(), _vec(gamma_k_shard, "gamma_k_shard", hk, dt, dev), sk, hk,
+            ps_k, int(Hk_full), P, T, float(eps), _DTYPES[dt], _stream_handle(stream, dev))
+    _clib.check(st, "qknorm_combine_apply")
+    return q_out, k_out
+
+
+# --------------------------------------------------------------------------- host planning (no GPU)
+
+def plan_shape(rows: int, units_max: int, vectorized: bool, sm_count: int) -> dict:
+    L = QknLaunch()
+    st = capi().qknorm_plan_shape(rows, units_max, 1 if vectorized else 0, sm_count, ctypes.byref(L))
+    _clib.check(st, "qknorm_plan_shape")
+    return L.as_dict()
+
+
+def plan_grid(rows: int, blocks_per_sm: int, sm_count: int) -> int:
+    return capi().qknorm_plan_grid(rows, blocks_per_sm, sm_count)
+
+
+def regions_overlap(a: tuple, b: tuple) -> bool:
+    """``a`` and ``b`` are ``(base, width_bytes, stride_bytes, rows)``."""
+    return bool(capi().qknorm_regions_overlap(*a, *b))

@@ -1,0 +1,584 @@
+// Host side of libqknorm.so: argument validation, overlap checks, launch
+// planning and the extern "C" entry points declared in include/qknorm.h and
+// include/qknorm_plan.h.
+//
+// Every entry point validates on the host before enqueueing anything, so a
+// rejected call never reaches the GPU.  Nothing here allocates device memory
+// or synchronizes.
+
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "qknorm.h"
+#include "qknorm_plan.h"
+#include "qknorm_kernels.cuh"
+
+#ifndef QKNORM_VERSION
+#define QKNORM_VERSION 100  // 0.1.0
+#endif
+
+namespace {
+
+// ---------------------------------------------------------------------------
+// Per-thread error message.
+thread_local char g_last_error[512] = "";
+
+qkn_status fail(qkn_status st, const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+    va_end(ap);
+    return st;
+}
+
+qkn_status ok() {
+    g_last_error[0] = '\0';
+    return QKN_OK;
+}
+
+int elem_bytes(qkn_dtype dt) { return dt == QKN_F32 ? 4 : 2; }
+
+bool dtype_valid(int dt) { return dt == QKN_F32 || dt == QKN_BF16; }
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ---------------------------------------------------------------------------
+// Overlap of two row sets.
+int64_t floor_div(int64_t a, int64_t b) {  // b > 0
+    int64_t q = a / b;
+    if ((a % b != 0) && (a < 0)) --q;
+    return q;
+}
+int64_t ceil_div_signed(int64_t a, int64_t b) {  // b > 0
+    return -floor_div(-a, b);
+}
+
+// Is there an integer k in [kmin, kmax] with lo < k * s < hi ?  (s > 0)
+bool multiple_in_open_interval(int64_t s, int64_t lo, int64_t hi, int64_t kmin, int64_t kmax) {
+    const int64_t k_lo = floor_div(lo, s) + 1;         // smallest k with k*s > lo
+    const int64_t k_hi = ceil_div_signed(hi, s) - 1;   // largest k with k*s < hi
+    const int64_t a = k_lo > kmin ? k_lo : kmin;
+    const int64_t b = k_hi < kmax ? k_hi : kmax;
+    return a <= b;
+}
+
+struct Region {
+    uint64_t base;
+    int64_t width;   // bytes per row
+    int64_t stride;  // bytes between rows
+    int64_t rows;
+};
+
+bool overlap(const Region &a, const Region &b) {
+    if (a.rows < 1 || b.rows < 1 || a.width < 1 || b.width < 1) return false;
+    const __int128 a_end = (__int128)a.base + (__int128)(a.rows - 1) * a.stride + a.width;
+    const __int128 b_end = (__int128)b.base + (__int128)(b.rows - 1) * b.stride + b.width;
+    if (a_end <= (__int128)b.base || b_end <= (__int128)a.base) return false;
+    if (a.rows == 1 && b.rows == 1) return true;
+    if (a.rows == 1 || b.rows == 1 || a.stride == b.stride) {
+        // Rows of `m` (multi-row, stride s) against rows of `o`.  Row pair
+        // (i, j) overlaps iff -w_m < (o + j*s_o) - (m + i*s) < w_o; with one
+        // row in `o` (j = 0) or a shared stride this depends on one integer k.
+        const Region &m = (a.rows == 1) ? b : a;
+        const Region &o = (a.rows == 1) ? a : b;
+        const int64_t s = m.stride;
+        const int64_t d = (int64_t)(o.base - m.base);  // wraps correctly for nearby addresses
+        int64_t kmin, kmax;
+        if (o.rows == 1) {
+            // i*s in (d - w_m, d + w_o), i in [0, rows_m - 1]
+            kmin = 0;
+            kmax = m.rows - 1;
+            return multiple_in_open_interval(s, d - m.width, d + o.width, kmin, kmax);
+        }
+        // shared stride: (i - j)*s in (d - w_m, d + w_o), i - j in [-(rows_o-1), rows_m-1]
+        kmin = -(o.rows - 1);
+        kmax = m.rows - 1;
+        return multiple_in_open_interval(s, d - m.width, d + o.width, kmin, kmax);
+    }
+    return true;  // different strides with intersecting ranges: conservative
+}
+
+// ---------------------------------------------------------------------------
+// Device facts, cached per device.
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+    int sm_count = 0;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+struct OccEntry {
+    const void *fn;
+    int device;
+    int threads;
+    int blocks;
+};
+constexpr int kOccSlots = 512;
+OccEntry g_occ[kOccSlots];
+int g_occ_n = 0;
+std::mutex g_occ_mu;
+
+qkn_status current_device(int *dev) {
+    cudaError_t e = cudaGetDevice(dev);
+    if (e != cudaSuccess) return fail(QKN_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    if (*dev < 0 || *dev >= kMaxDevices) return fail(QKN_ERR_UNSUPPORTED, "device ordinal %d too large", *dev);
+    return QKN_OK;
+}
+
+qkn_status sm_count(int dev, int *out) {
+    {
+        std::lock_guard<std::mutex> lk(g_dev_mu);
+        if (g_dev[dev].sm_count > 0) {
+            *out = g_dev[dev].sm_count;
+            return QKN_OK;
+        }
+    }
+    int n = 0;
+    cudaError_t e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess || n < 1)
+        return fail(QKN_ERR_CUDA, "cudaDeviceGetAttribute(SM count): %s", cudaGetErrorString(e));
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    g_dev[dev].sm_count = n;
+    *out = n;
+    return QKN_OK;
+}
+
+qkn_status blocks_per_sm(const void *fn, int dev, int threads, int *out) {
+    {
+        std::lock_guard<std::mutex> lk(g_occ_mu);
+        for (int i = 0; i < g_occ_n; ++i)
+            if (g_occ[i].fn == fn && g_occ[i].device == dev && g_occ[i].threads == threads) {
+                *out = g_occ[i].blocks;
+                return QKN_OK;
+            }
+    }
+    int n = 0;
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, threads, 0);
+    if (e != cudaSuccess)
+        return fail(QKN_ERR_CUDA, "cudaOccupancyMaxActiveBlocksPerMultiprocessor: %s", cudaGetErrorString(e));
+    if (n < 1) return fail(QKN_ERR_UNSUPPORTED, "kernel cannot run with %d threads per CTA", threads);
+    std::lock_guard<std::mutex> lk(g_occ_mu);
+    if (g_occ_n < kOccSlots) g_occ[g_occ_n++] = OccEntry{fn, dev, threads, n};
+    *out = n;
+    return QKN_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Kernel selection.
+template <typename E, int MODE>
+const void *register_kernel(int nv) {
+    switch (nv) {
+        case 1: return (const void *)qkn::rows_register_kernel<E, 1, MODE>;
+        case 2: return (const void *)qkn::rows_register_kernel<E, 2, MODE>;
+        case 4: return (const void *)qkn::rows_register_kernel<E, 4, MODE>;
+        case 8: return (const void *)qkn::rows_register_kernel<E, 8, MODE>;
+        default: return nullptr;
+    }
+}
+
+template <typename E, int MODE>
+const void *kernel_for(const qkn_launch &L) {
+    switch (L.kernel) {
+        case QKN_KERNEL_REGISTER: return register_kernel<E, MODE>(L.vec_per_thread);
+        case QKN_KERNEL_TWOPASS_VEC: return (const void *)qkn::rows_twopass_kernel<E, true, MODE>;
+        case QKN_KERNEL_TWOPASS_SCALAR: return (const void *)qkn::rows_twopass_kernel<E, false, MODE>;
+        default: return nullptr;
+    }
+}
+
+template <int MODE>
+const void *kernel_for(qkn_dtype dt, const qkn_launch &L) {
+    return dt == QKN_F32 ? kernel_for<float, MODE>(L) : kernel_for<__nv_bfloat16, MODE>(L);
+}
+
+// A prepared call: parameters plus the facts planning needs.
+struct Call {
+    qkn::Params p;
+    qkn_dtype dtype;
+    bool vectorized;
+    int64_t units_max;  // widest row in vectors (vectorized) or elements
+};
+
+void fill_rowset(qkn::RowSet &s, const void *in, void *out, const void *gamma, int64_t stride, int32_t width,
+                 int32_t div_width, int esz) {
+    const int per_vec = 16 / esz;
+    s.in = static_cast<const char *>(in);
+    s.out = static_cast<char *>(out);
+    s.gamma = static_cast<const char *>(gamma);
+    s.sumsq = nullptr;
+    s.sumsq_all = nullptr;
+    s.stride_bytes = stride * esz;
+    s.width = width;
+    s.nfull = width / per_vec;
+    s.tail = width % per_vec;
+    s.div = static_cast<float>(div_width);
+}
+
+void finish_call(Call &c, int esz, std::initializer_list<const void *> ptrs, int64_t q_stride, int64_t k_stride) {
+    bool v = ((q_stride * esz) % 16 == 0) && ((k_stride * esz) % 16 == 0);
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) v = false;
+    c.vectorized = v;
+    const int per_vec = 16 / esz;
+    int64_t wq = c.p.set[0].width, wk = c.p.set[1].width;
+    int64_t w = wq > wk ? wq : wk;
+    c.units_max = v ? (w + per_vec - 1) / per_vec : w;
+}
+
+bool eps_valid(float eps) { return std::isfinite(eps) && eps >= 0.0f; }
+
+// Rows of T must stay addressable: (T - 1) * stride + width elements in bytes below 2^62.
+bool extent_ok(int64_t T, int64_t stride, int64_t width, int esz) {
+    if (T <= 0) return true;
+    const __int128 bytes = ((__int128)(T - 1) * stride + width) * esz;
+    return bytes < ((__int128)1 << 62);
+}
+
+Region rows_region(const void *base, int64_t width, int64_t stride, int64_t T, int esz) {
+    return Region{(uint64_t)(uintptr_t)base, width * esz, stride * esz, T};
+}
+Region flat_region(const void *base, int64_t bytes) {
+    return Region{(uint64_t)(uintptr_t)base, bytes, bytes, 1};
+}
+
+// Written region `w` against a region `r` it must not touch, unless `r` is
+// the very same buffer (in place).
+bool bad_overlap(const Region &w, const Region &r, bool allow_identical) {
+    if (allow_identical && w.base == r.base && w.stride == r.stride && w.width == r.width) return false;
+    return overlap(w, r);
+}
+
+// Common checks of the fused and apply forms: outputs vs everything else.
+qkn_status check_outputs(const Region &oq, const Region &ok_, const Region &iq, const Region &ik,
+                         const Region *others, int n_others) {
+    if (overlap(oq, ok_)) return fail(QKN_ERR_INVALID_ARG, "q_out and k_out overlap");
+    if (bad_overlap(oq, iq, true)) return fail(QKN_ERR_INVALID_ARG, "q_out partly overlaps q_in (only out == in is allowed)");
+    if (bad_overlap(ok_, ik, true)) return fail(QKN_ERR_INVALID_ARG, "k_out partly overlaps k_in (only out == in is allowed)");
+    if (overlap(oq, ik)) return fail(QKN_ERR_INVALID_ARG, "q_out overlaps k_in");
+    if (overlap(ok_, iq)) return fail(QKN_ERR_INVALID_ARG, "k_out overlaps q_in");
+    for (int i = 0; i < n_others; ++i) {
+        if (overlap(oq, others[i])) return fail(QKN_ERR_INVALID_ARG, "q_out overlaps a read-only operand (gamma or sums)");
+        if (overlap(ok_, others[i])) return fail(QKN_ERR_INVALID_ARG, "k_out overlaps a read-only operand (gamma or sums)");
+    }
+    return QKN_OK;
+}
+
+qkn_status prepare_layerwise(const void *q_in, void *q_out, const void *gamma_q, int64_t q_stride,
+                             const void *k_in, void *k_out, const void *gamma_k, int64_t k_stride,
+                             int64_t T, int32_t Hq, int32_t Hk, float eps, qkn_dtype dtype, Call &c) {
+    if (!dtype_valid(dtype)) return fail(QKN_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
+    if (T < 0) return fail(QKN_ERR_INVALID_ARG, "T = %lld < 0", (long long)T);
+    if (Hq <= 0 || Hk <= 0) return fail(QKN_ERR_INVALID_ARG, "widths must be positive (Hq = %d, Hk = %d)", Hq, Hk);
+    if (q_stride < Hq || k_stride < Hk)
+        return fail(QKN_ERR_INVALID_ARG, "row stride below width (q: %lld < %d or k: %lld < %d)",
+                    (long long)q_stride, Hq, (long long)k_stride, Hk);
+    if (!eps_valid(eps)) return fail(QKN_ERR_INVALID_ARG, "eps must be finite and >= 0");
+    const int esz = elem_bytes(dtype);
+    if (!extent_ok(T, q_stride, Hq, esz) || !extent_ok(T, k_stride, Hk, esz))
+        return fail(QKN_ERR_INVALID_ARG, "buffer extent overflows");
+    if (T > 0 && (!q_in || !q_out || !gamma_q || !k_in || !k_out || !gamma_k))
+        return fail(QKN_ERR_INVALID_ARG, "null pointer");
+    if (T > 0) {
+        const Region iq = rows_region(q_in, Hq, q_stride, T, esz), oq = rows_region(q_out, Hq, q_stride, T, esz);
+        const Region ik = rows_region(k_in, Hk, k_stride, T, esz), ok_ = rows_region(k_out, Hk, k_stride, T, esz);
+        const Region others[2] = {flat_region(gamma_q, (int64_t)Hq * esz), flat_region(gamma_k, (int64_t)Hk * esz)};
+        qkn_status st = check_outputs(oq, ok_, iq, ik, others, 2);
+        if (st != QKN_OK) return st;
+    }
+    std::memset(&c, 0, sizeof(c));
+    c.dtype = dtype;
+    fill_rowset(c.p.set[0], q_in, q_out, gamma_q, q_stride, Hq, Hq, esz);
+    fill_rowset(c.p.set[1], k_in, k_out, gamma_k, k_stride, Hk, Hk, esz);
+    c.p.T = T;
+    c.p.rows = 2 * T;
+    c.p.eps = eps;
+    c.p.P = 1;
+    finish_call(c, esz, {q_in, q_out, gamma_q, k_in, k_out, gamma_k}, q_stride, k_stride);
+    return QKN_OK;
+}
+
+template <int MODE>
+qkn_status plan_call(const Call &c, qkn_launch &L) {
+    int dev = 0, sms = 0, bps = 0;
+    qkn_status st = current_device(&dev);
+    if (st != QKN_OK) return st;
+    if ((st = sm_count(dev, &sms)) != QKN_OK) return st;
+    if ((st = qknorm_plan_shape(c.p.rows, c.units_max, c.vectorized ? 1 : 0, sms, &L)) != QKN_OK)
+        return fail(st, "planning failed");
+    const void *fn = kernel_for<MODE>(c.dtype, L);
+    if (!fn) return fail(QKN_ERR_UNSUPPORTED, "no kernel for the planned launch");
+    if ((st = blocks_per_sm(fn, dev, L.threads, &bps)) != QKN_OK) return st;
+    L.grid = qknorm_plan_grid(c.p.rows, bps, sms);
+    return QKN_OK;
+}
+
+qkn_status check_launch(const Call &c, const qkn_launch &L) {
+    if (L.threads < 32 || L.threads > 1024 || (L.threads % 32) != 0)
+        return fail(QKN_ERR_INVALID_ARG, "threads must be a multiple of 32 in [32, 1024], got %d", L.threads);
+    if (L.grid < 1 || L.grid > 2147483647LL) return fail(QKN_ERR_INVALID_ARG, "grid out of range");
+    switch (L.kernel) {
+        case QKN_KERNEL_REGISTER: {
+            const int mt = qknorm_register_max_threads(L.vec_per_thread);
+            if (mt == 0) return fail(QKN_ERR_INVALID_ARG, "vec_per_thread must be 1, 2, 4 or 8");
+            if (L.threads > mt) return fail(QKN_ERR_INVALID_ARG, "threads above %d for vec_per_thread %d", mt, L.vec_per_thread);
+            if (!c.vectorized) return fail(QKN_ERR_INVALID_ARG, "register kernel needs 16-byte aligned buffers");
+            if ((int64_t)L.vec_per_thread * L.threads < c.units_max)
+                return fail(QKN_ERR_INVALID_ARG, "row of %lld vectors exceeds vec_per_thread * threads",
+                            (long long)c.units_max);
+            return QKN_OK;
+        }
+        case QKN_KERNEL_TWOPASS_VEC:
+            if (!c.vectorized) return fail(QKN_ERR_INVALID_ARG, "vector kernel needs 16-byte aligned buffers");
+            return QKN_OK;
+        case QKN_KERNEL_TWOPASS_SCALAR: return QKN_OK;
+        default: return fail(QKN_ERR_INVALID_ARG, "unknown kernel kind %d", L.kernel);
+    }
+}
+
+template <typename E, int MODE>
+cudaError_t launch_typed(const qkn_launch &L, const qkn::Params &p, cudaStream_t s) {
+    const dim3 grid((unsigned)L.grid), block((unsigned)L.threads);
+    switch (L.kernel) {
+        case QKN_KERNEL_REGISTER:
+            switch (L.vec_per_thread) {
+                case 1: qkn::rows_register_kernel<E, 1, MODE><<<grid, block, 0, s>>>(p); break;
+                case 2: qkn::rows_register_kernel<E, 2, MODE><<<grid, block, 0, s>>>(p); break;
+                case 4: qkn::rows_register_kernel<E, 4, MODE><<<grid, block, 0, s>>>(p); break;
+                case 8: qkn::rows_register_kernel<E, 8, MODE><<<grid, block, 0, s>>>(p); break;
+                default: return cudaErrorInvalidValue;
+            }
+            break;
+        case QKN_KERNEL_TWOPASS_VEC: qkn::rows_twopass_kernel<E, true, MODE><<<grid, block, 0, s>>>(p); break;
+        case QKN_KERNEL_TWOPASS_SCALAR: qkn::rows_twopass_kernel<E, false, MODE><<<grid, block, 0, s>>>(p); break;
+        default: return cudaErrorInvalidValue;
+    }
+    return cudaGetLastError();
+}
+
+template <int MODE>
+qkn_status launch(const Call &c, const qkn_launch &L, void *stream) {
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = c.dtype == QKN_F32 ? launch_typed<float, MODE>(L, c.p, s)
+                                        : launch_typed<__nv_bfloat16, MODE>(L, c.p, s);
+    if (e != cudaSuccess) return fail(QKN_ERR_CUDA, "kernel launch: %s", cudaGetErrorString(e));
+    return ok();
+}
+
+}  // namespace
+
+// ===========================================================================
+extern "C" {
+
+int32_t qknorm_register_max_threads(int32_t vec_per_thread) {
+    switch (vec_per_thread) {
+        case 1: return qkn::RegisterBounds<1>::kMaxThreads;
+        case 2: return qkn::RegisterBounds<2>::kMaxThreads;
+        case 4: return qkn::RegisterBounds<4>::kMaxThreads;
+        case 8: return qkn::RegisterBounds<8>::kMaxThreads;
+        default: return 0;
+    }
+}
+
+qkn_status qknorm_plan_shape(int64_t rows, int64_t units_max, int32_t vectorized, int32_t sm_count,
+                             qkn_launch *out) {
+    if (!out || rows < 1 || units_max < 1 || sm_count < 1) return QKN_ERR_INVALID_ARG;
+    qkn_launch L{};
+    L.grid = 0;
+    auto round32 = [](int64_t n) { return (int32_t)(((n + 31) / 32) * 32); };
+    if (!vectorized) {
+        L.kernel = QKN_KERNEL_TWOPASS_SCALAR;
+        L.vec_per_thread = 0;
+        L.threads = units_max >= 256 ? 256 : round32(units_max);
+        *out = L;
+        return QKN_OK;
+    }
+    if (units_max > 2048) {  // beyond 32 KB per row: two passes
+        L.kernel = QKN_KERNEL_TWOPASS_VEC;
+        L.vec_per_thread = 0;
+        L.threads = 512;
+        *out = L;
+        return QKN_OK;
+    }
+    L.kernel = QKN_KERNEL_REGISTER;
+    int nv;
+    if (rows <= sm_count) {
+        // Few rows (decode): spread each row over many threads so a row costs
+        // about one memory round trip.
+        nv = units_max <= 1024 ? 1 : 2;
+    } else {
+        // Many rows: moderate CTAs, several vectors in flight per thread.
+        nv = units_max >= 256 ? 4 : (units_max >= 64 ? 2 : 1);
+    }
+    int32_t threads = round32((units_max + nv - 1) / nv);
+    while (threads > qknorm_register_max_threads(nv)) {
+        nv *= 2;
+        threads = round32((units_max + nv - 1) / nv);
+    }
+    L.vec_per_thread = nv;
+    L.threads = threads;
+    *out = L;
+    return QKN_OK;
+}
+
+int64_t qknorm_plan_grid(int64_t rows, int32_t blocks_per_sm, int32_t sm_count) {
+    if (rows < 1) return 0;
+    const int64_t bps = blocks_per_sm > 0 ? blocks_per_sm : 1;
+    const int64_t sms = sm_count > 0 ? sm_count : 1;
+    const int64_t resident = bps * sms;
+    const int64_t trips = (rows + resident - 1) / resident;
+    return (rows + trips - 1) / trips;
+}
+
+int qknorm_regions_overlap(uint64_t a_base, int64_t a_width, int64_t a_stride, int64_t a_rows,
+                           uint64_t b_base, int64_t b_width, int64_t b_stride, int64_t b_rows) {
+    Region a{a_base, a_width, a_stride, a_rows}, b{b_base, b_width, b_stride, b_rows};
+    if (a.rows > 1 && a.stride < 1) return 1;
+    if (b.rows > 1 && b.stride < 1) return 1;
+    return overlap(a, b) ? 1 : 0;
+}
+
+qkn_status qknorm_layerwise(const void *q_in, void *q_out, const void *gamma_q, int64_t q_stride,
+                            const void *k_in, void *k_out, const void *gamma_k, int64_t k_stride,
+                            int64_t T, int32_t Hq, int32_t Hk, float eps, qkn_dtype dtype, void *stream) {
+    Call c;
+    qkn_status st = prepare_layerwise(q_in, q_out, gamma_q, q_stride, k_in, k_out, gamma_k, k_stride, T, Hq,
+                                      Hk, eps, dtype, c);
+    if (st != QKN_OK) return st;
+    if (T == 0) return ok();
+    qkn_launch L;
+    if ((st = plan_call<qkn::kFused>(c, L)) != QKN_OK) return st;
+    return launch<qkn::kFused>(c, L, stream);
+}
+
+qkn_status qknorm_layerwise_plan(const void *q_in, void *q_out, const void *gamma_q, int64_t q_stride,
+                                 const void *k_in, void *k_out, const void *gamma_k, int64_t k_stride,
+                                 int64_t T, int32_t Hq, int32_t Hk, float eps, qkn_dtype dtype,
+                                 qkn_launch *out) {
+    if (!out) return fail(QKN_ERR_INVALID_ARG, "null output");
+    Call c;
+    qkn_status st = prepare_layerwise(q_in, q_out, gamma_q, q_stride, k_in, k_out, gamma_k, k_stride, T, Hq,
+                                      Hk, eps, dtype, c);
+    if (st != QKN_OK) return st;
+    if (T == 0) {
+        std::memset(out, 0, sizeof(*out));
+        return ok();
+    }
+    if ((st = plan_call<qkn::kFused>(c, *out)) != QKN_OK) return st;
+    return ok();
+}
+
+qkn_status qknorm_layerwise_launch(const void *q_in, void *q_out, const void *gamma_q, int64_t q_stride,
+                                   const void *k_in, void *k_out, const void *gamma_k, int64_t k_stride,
+                                   int64_t T, int32_t Hq, int32_t Hk, float eps, qkn_dtype dtype, void *stream,
+                                   const qkn_launch *launch_cfg) {
+    if (!launch_cfg) return fail(QKN_ERR_INVALID_ARG, "null launch");
+    Call c;
+    qkn_status st = prepare_layerwise(q_in, q_out, gamma_q, q_stride, k_in, k_out, gamma_k, k_stride, T, Hq,
+                                      Hk, eps, dtype, c);
+    if (st != QKN_OK) return st;
+    if ((st = check_launch(c, *launch_cfg)) != QKN_OK) return st;
+    if (T == 0) return ok();
+    return launch<qkn::kFused>(c, *launch_cfg, stream);
+}
+
+qkn_status qknorm_partial_stats(const void *q_shard, int64_t q_stride, int32_t hq_shard, float *q_sumsq,
+                                const void *k_shard, int64_t k_stride, int32_t hk_shard, float *k_sumsq,
+                                int64_t T, qkn_dtype dtype, void *stream) {
+    if (!dtype_valid(dtype)) return fail(QKN_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
+    if (T < 0) return fail(QKN_ERR_INVALID_ARG, "T = %lld < 0", (long long)T);
+    if (hq_shard <= 0 || hk_shard <= 0) return fail(QKN_ERR_INVALID_ARG, "shard widths must be positive");
+    if (q_stride < hq_shard || k_stride < hk_shard) return fail(QKN_ERR_INVALID_ARG, "row stride below shard width");
+    const int esz = elem_bytes(dtype);
+    if (!extent_ok(T, q_stride, hq_shard, esz) || !extent_ok(T, k_stride, hk_shard, esz))
+        return fail(QKN_ERR_INVALID_ARG, "buffer extent overflows");
+    if (T > 0 && (!q_shard || !q_sumsq || !k_shard || !k_sumsq)) return fail(QKN_ERR_INVALID_ARG, "null pointer");
+    if (T == 0) return ok();
+    const Region iq = rows_region(q_shard, hq_shard, q_stride, T, esz);
+    const Region ik = rows_region(k_shard, hk_shard, k_stride, T, esz);
+    const Region sq = flat_region(q_sumsq, T * 4), sk = flat_region(k_sumsq, T * 4);
+    if (overlap(sq, sk)) return fail(QKN_ERR_INVALID_ARG, "q_sumsq and k_sumsq overlap");
+    if (overlap(sq, iq) || overlap(sq, ik) || overlap(sk, iq) || overlap(sk, ik))
+        return fail(QKN_ERR_INVALID_ARG, "a sum array overlaps an input");
+    Call c;
+    std::memset(&c, 0, sizeof(c));
+    c.dtype = dtype;
+    fill_rowset(c.p.set[0], q_shard, nullptr, nullptr, q_stride, hq_shard, hq_shard, esz);
+    fill_rowset(c.p.set[1], k_shard, nullptr, nullptr, k_stride, hk_shard, hk_shard, esz);
+    c.p.set[0].sumsq = q_sumsq;
+    c.p.set[1].sumsq = k_sumsq;
+    c.p.T = T;
+    c.p.rows = 2 * T;
+    c.p.eps = 0.0f;
+    c.p.P = 1;
+    finish_call(c, esz, {q_shard, k_shard}, q_stride, k_stride);
+    qkn_launch L;
+    qkn_status st = plan_call<qkn::kStats>(c, L);
+    if (st != QKN_OK) return st;
+    return launch<qkn::kStats>(c, L, stream);
+}
+
+qkn_status qknorm_combine_apply(const void *q_in, void *q_out, const void *gamma_q_shard, int64_t q_stride,
+                                int32_t hq_shard, const float *q_sumsq_all, int32_t Hq_full,
+                                const void *k_in, void *k_out, const void *gamma_k_shard, int64_t k_stride,
+                                int32_t hk_shard, const float *k_sumsq_all, int32_t Hk_full,
+                                int32_t P, int64_t T, float eps, qkn_dtype dtype, void *stream) {
+    if (!dtype_valid(dtype)) return fail(QKN_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
+    if (T < 0) return fail(QKN_ERR_INVALID_ARG, "T = %lld < 0", (long long)T);
+    if (P < 1) return fail(QKN_ERR_INVALID_ARG, "P = %d < 1", P);
+    if (hq_shard <= 0 || hk_shard <= 0) return fail(QKN_ERR_INVALID_ARG, "shard widths must be positive");
+    if (Hq_full < hq_shard || Hk_full < hk_shard) return fail(QKN_ERR_INVALID_ARG, "full width below shard width");
+    if (q_stride < hq_shard || k_stride < hk_shard) return fail(QKN_ERR_INVALID_ARG, "row stride below shard width");
+    if (!eps_valid(eps)) return fail(QKN_ERR_INVALID_ARG, "eps must be finite and >= 0");
+    const int esz = elem_bytes(dtype);
+    if (!extent_ok(T, q_stride, hq_shard, esz) || !extent_ok(T, k_stride, hk_shard, esz) ||
+        !extent_ok(1, 0, (int64_t)P * T, 4))
+        return fail(QKN_ERR_INVALID_ARG, "buffer extent overflows");
+    if (T > 0 && (!q_in || !q_out || !gamma_q_shard || !q_sumsq_all || !k_in || !k_out || !gamma_k_shard ||
+                  !k_sumsq_all))
+        return fail(QKN_ERR_INVALID_ARG, "null pointer");
+    if (T == 0) return ok();
+    const Region iq = rows_region(q_in, hq_shard, q_stride, T, esz), oq = rows_region(q_out, hq_shard, q_stride, T, esz);
+    const Region ik = rows_region(k_in, hk_shard, k_stride, T, esz), ok_ = rows_region(k_out, hk_shard, k_stride, T, esz);
+    const Region others[4] = {flat_region(gamma_q_shard, (int64_t)hq_shard * esz),
+                              flat_region(gamma_k_shard, (int64_t)hk_shard * esz),
+                              flat_region(q_sumsq_all, (int64_t)P * T * 4), flat_region(k_sumsq_all, (int64_t)P * T * 4)};
+    qkn_status st = check_outputs(oq, ok_, iq, ik, others, 4);
+    if (st != QKN_OK) return st;
+    Call c;
+    std::memset(&c, 0, sizeof(c));
+    c.dtype = dtype;
+    fill_rowset(c.p.set[0], q_in, q_out, gamma_q_shard, q_stride, hq_shard, Hq_full, esz);
+    fill_rowset(c.p.set[1], k_in, k_out, gamma_k_shard, k_stride, hk_shard, Hk_full, esz);
+    c.p.set[0].sumsq_all = q_sumsq_all;
+    c.p.set[1].sumsq_all = k_sumsq_all;
+    c.p.T = T;
+    c.p.rows = 2 * T;
+    c.p.eps = eps;
+    c.p.P = P;
+    finish_call(c, esz, {q_in, q_out, gamma_q_shard, k_in, k_out, gamma_k_shard}, q_stride, k_stride);
+    qkn_launch L;
+    if ((st = plan_call<qkn::kApply>(c, L)) != QKN_OK) return st;
+    return launch<qkn::kApply>(c, L, stream);
+}
+
+const char *qknorm_status_string(qkn_status s) {
+    switch (s) {
+        case QKN_OK: return "ok";
+        case QKN_ERR_INVALID_ARG: return "invalid argument";
+        case QKN_ERR_UNSUPPORTED: return "unsupported";
+        case QKN_ERR_CUDA: return "CUDA error";
+        default: return "unknown status";
+    }
+}
+
+const char *qknorm_last_error(void) { return g_last_error; }
+
+int qknorm_version(void) { return QKNORM_VERSION; }
+
+}  // extern "C"

@@ -1,0 +1,547 @@
+#!/usr/bin/env python
+"""Benchmark of fused layerwise QK-RMSNorm on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+                    [--workload prefill|decode|packed|gqa|tiny] [--tokens T]
+
+Prints ONE JSON line (rank 0).  A step is one pass of the whole path over one
+batch of synthetic input: for the default workload, one ``qknorm_layerwise``
+call normalizing the Q and K rows of a T=4096, Hq=Hk=4096 bf16 prefill batch
+(OLMo2-7B-shaped).  ``value`` is effective GB/s: the bytes the call must move
+(read + write of every Q and K element, plus gamma) divided by the time.
+
+Timing: W untimed warm-up steps, then exactly K steps captured in one CUDA
+graph (the C-ABI calls, replayed without host overhead) and timed with CUDA
+events on the launching stream, between a barrier and a device synchronize on
+both sides; the maximum over ranks is reported.  Consecutive steps rotate over
+several input/output sets whose total exceeds twice the L2 size, so no step
+finds its inputs in L2.  Under torchrun each rank normalizes its own batch
+(tokens are independent: no collective on the data path; weak scaling).
+
+``e2e`` times the same call through the public Python API with pinned host
+buffers: each step copies its inputs host->device, normalizes, and copies the
+outputs back.  ``cpu_baseline`` times the CPU oracle (double precision, one
+thread) on the same workload on this host.  ``--impl reference`` times that
+oracle alone, as the reference arm.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import glob
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+import torch
+
+import workloads
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+METRIC = "fused QK-RMSNorm effective HBM GB/s (% of B200 peak); µs per call"
+UNIT = "GB/s"
+FALLBACK_HBM_GBS = 6650.0  # used only when the measured peaks file is absent
+
+
+# --------------------------------------------------------------------------- plumbing
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--workload", choices=["prefill", "decode", "packed", "gqa", "tiny"], default="prefill")
+    ap.add_argument("--tokens", type=int, default=None, help="T for decode / packed workloads")
+    ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU baseline budget")
+    a = ap.parse_args(argv)
+    if a.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if a.steps < 1:
+        ap.error("--steps must be >= 1")
+    return a
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def load_peaks() -> dict:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return {"hbm_gbs": FALLBACK_HBM_GBS, "source": "fallback"}
+
+
+def source_digest() -> str:
+    """Digest of the CUDA sources and headers: profile counters apply only to
+    the build they were taken from."""
+    h = hashlib.sha256()
+    files = sorted(glob.glob(os.path.join(ROOT, "attention_normalization_b200", "csrc", "*"))
+                   + glob.glob(os.path.join(ROOT, "include", "*.h")))
+    for p in files:
+        h.update(os.path.basename(p).encode())
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: str, digest: str):
+    """DRAM bytes per launch from a committed ncu summary for this workload, if
+    it was taken from the current sources; else None."""
+    for p in sorted(glob.glob(os.path.join(ROOT, "profiles", "*.md"))):
+        text = open(p).read()
+        m_w = re.search(r"^workload:\s*(\S+)", text, re.M)
+        m_d = re.search(r"^source_digest:\s*(\S+)", text, re.M)
+        m_t = re.search(r"^dram_bytes_per_launch:\s*(\d+)", text, re.M)
+        if m_w and m_d and m_t and m_w.group(1) == workload and m_d.group(1) == digest:
+            return int(m_t.group(1))
+    return None
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML (read-only) while
+    ``active`` is set."""
+    REASONS = [(0x4, "sw_power_cap"), (0x8, "hw_slowdown"), (0x20, "sw_thermal_slowdown"),
+               (0x40, "hw_thermal_slowdown"), (0x80, "hw_power_brake_slowdown"),
+               (0x2, "applications_clocks_setting"), (0x10, "sync_boost")]
+
+    def __init__(self, cuda_index: int, period_s: float = 0.005):
+        self.period = period_s
+        self.samples = []
+        self.error = None
+        self.active = threading.Event()
+        self.stop_ev = threading.Event()
+        self.handle = None
+        self.max_mhz = None
+        try:
+            import pynvml
+            self.nv = pynvml
+            pynvml.nvmlInit()
+            self.handle = self._handle(cuda_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # NVML missing: report, do not fail the run
+            self.error = f"{type(e).__name__}: {e}"
+        self.thread = threading.Thread(target=self._run, daemon=True)
+
+    def _handle(self, cuda_index):
+        nv = self.nv
+        props = torch.cuda.get_device_properties(cuda_index)
+        try:
+            bus = "%08X:%02X:%02X.0" % (props.pci_domain_id, props.pci_bus_id, props.pci_device_id)
+            return nv.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            pass
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+        idx = int(vis.split(",")[cuda_index]) if vis and vis.split(",")[0].isdigit() else cuda_index
+        return nv.nvmlDeviceGetHandleByIndex(idx)
+
+    def _reasons(self):
+        nv = self.nv
+        for fn in ("nvmlDeviceGetCurrentClocksEventReasons", "nvmlDeviceGetCurrentClocksThrottleReasons"):
+            if hasattr(nv, fn):
+                return getattr(nv, fn)(self.handle)
+        return 0
+
+    def _run(self):
+        while not self.stop_ev.is_set():
+            if self.active.is_set() and self.handle is not None:
+                try:
+                    mhz = self.nv.nvmlDeviceGetClockInfo(self.handle, self.nv.NVML_CLOCK_SM)
+                    self.samples.append((mhz, int(self._reasons())))
+                except Exception as e:
+                    self.error = f"{type(e).__name__}: {e}"
+            time.sleep(self.period)
+
+    def start(self):
+        self.thread.start()
+
+    def summary(self) -> dict:
+        self.stop_ev.set()
+        self.thread.join(timeout=2)
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0,
+                    **({"error": self.error} if self.error else {})}
+        mask = 0
+        for _, r in self.samples:
+            mask |= r
+        return {"sm_mhz": statistics.median(m for m, _ in self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": [n for bit, n in self.REASONS if mask & bit], "samples": len(self.samples)}
+
+
+# --------------------------------------------------------------------------- workloads
+
+class Workload:
+    """A benchmark workload: CPU batch, effective bytes per step, and a step
+    function over a device-resident set."""
+
+    def __init__(self, kind: str, tokens: int | None, seed_offset: int):
+        self.kind = kind
+        if kind == "prefill":
+            self.batch = workloads.prefill_bf16(seed=1 + seed_offset)
+        elif kind == "tiny":
+            self.batch = workloads.tiny_fp32(seed=0 + seed_offset)
+        elif kind == "decode":
+            self.batch = workloads.decode_bf16(tokens or 1, seed=2 + seed_offset)
+        elif kind == "packed":
+            self.batch = workloads.packed_qkv(tokens or 16384, seed=4 + seed_offset)
+        elif kind == "gqa":
+            self.batch = workloads.gqa_sharded(seed=3 + seed_offset)
+        b = self.batch
+        self.esz = 4 if b.dtype == torch.float32 else 2
+        # bytes the method must move per step: read + write of every Q and K element, plus gamma
+        self.eff_bytes = 2 * self.esz * (b.Hq + b.Hk) * b.T + self.esz * (b.Hq + b.Hk)
+        self.name = b.name
+        self.launches_per_step = 2 * b.P if kind == "gqa" else 1
+
+    def config(self) -> dict:
+        b = self.batch
+        c = {"workload": self.name, "T": b.T, "Hq": b.Hq, "Hk": b.Hk, "io_dtype": str(b.dtype).replace("torch.", ""),
+             "eps": b.eps}
+        if self.kind == "packed":
+            c.update({"Hv": b.Hv, "row_stride": b.packed.shape[1], "in_place": True})
+        if self.kind == "gqa":
+            c.update({"P": b.P, "form": "partial_stats x P -> combine_apply x P"})
+        return c
+
+    # one device-resident set of buffers
+    def make_set(self, dev):
+        b = self.batch
+        if self.kind == "packed":
+            base = b.packed.to(dev)
+            return {"base": base, "q": base[:, :b.Hq], "k": base[:, b.Hq:b.Hq + b.Hk],
+                    "gq": b.gamma_q.to(dev), "gk": b.gamma_k.to(dev)}
+        if self.kind == "gqa":
+            P = b.P
+            wq, wk = b.Hq // P, b.Hk // P
+            gq, gk = b.gamma_q.to(dev), b.gamma_k.to(dev)
+            return {"qs": [s.to(dev) for s in b.q_shards], "ks": [s.to(dev) for s in b.k_shards],
+                    "qo": [torch.empty_like(s, device=dev) for s in b.q_shards],
+                    "ko": [torch.empty_like(s, device=dev) for s in b.k_shards],
+                    "gqs": [gq[p * wq:(p + 1) * wq].contiguous() for p in range(P)],
+                    "gks": [gk[p * wk:(p + 1) * wk].contiguous() for p in range(P)],
+                    "q_all": torch.empty((P, b.T), dtype=torch.float32, device=dev),
+                    "k_all": torch.empty((P, b.T), dtype=torch.float32, device=dev)}
+        q, k = b.q.to(dev), b.k.to(dev)
+        return {"q": q, "k": k, "qo": torch.empty_like(q), "ko": torch.empty_like(k),
+                "gq": b.gamma_q.to(dev), "gk": b.gamma_k.to(dev)}
+
+    def set_bytes(self) -> int:
+        b = self.batch
+        if self.kind == "packed":
+            return b.packed.numel() * self.esz
+        return 2 * self.esz * (b.Hq + b.Hk) * b.T
+
+    def step(self, qk, s):
+        b = self.batch
+        if self.kind == "packed":
+            qk.qknorm_layerwise(s["q"], s["k"], s["gq"], s["gk"], b.eps, q_out=s["q"], k_out=s["k"])
+        elif self.kind == "gqa":
+            for p in range(b.P):
+                qk.qknorm_partial_stats(s["qs"][p], s["ks"][p], s["q_all"][p], s["k_all"][p])
+            for p in range(b.P):
+                qk.qknorm_combine_apply(s["qs"][p], s["ks"][p], s["gqs"][p], s["gks"][p], s["q_all"], s["k_all"],
+                                        b.Hq, b.Hk, b.eps, q_out=s["qo"][p], k_out=s["ko"][p])
+        else:
+            qk.qknorm_layerwise(s["q"], s["k"], s["gq"], s["gk"], b.eps, q_out=s["qo"], k_out=s["ko"])
+
+
+def rotation_count(set_bytes: int, l2_bytes: int) -> int:
+    """Sets to rotate over so that the other sets touched between two uses of
+    one set exceed twice the L2 size."""
+    return max(2, math.ceil(2 * l2_bytes / max(1, set_bytes)) + 1)
+
+
+# --------------------------------------------------------------------------- CPU baseline (the oracle)
+
+def time_oracle(wl: Workload, budget_s: float, max_tokens: int | None = None) -> dict:
+    """Times the CPU oracle (double precision, one thread) on the workload's
+    own inputs: whole calls until the budget is spent, or, with max_tokens, a
+    prefix of that many tokens per call."""
+    import numpy as np
+
+    import oracle
+
+    b = wl.batch
+    T = b.T if max_tokens is None else max(1, min(b.T, max_tokens))
+
+    def np_rows(view):
+        view = view[:T]
+        t = view.contiguous()
+        a = t.view(torch.int16).numpy().view(np.uint16) if t.dtype == torch.bfloat16 else t.numpy()
+        return a, view.shape[1]
+
+    if wl.kind == "gqa":
+        qf, _ = np_rows(b.q_full)
+        kf, _ = np_rows(b.k_full)
+    else:
+        qf, _ = np_rows(b.q)
+        kf, _ = np_rows(b.k)
+    gq = np_rows(b.gamma_q[None, :])[0].ravel()
+    gk = np_rows(b.gamma_k[None, :])[0].ravel()
+
+    def one_call():
+        if wl.kind == "gqa":
+            P = b.P
+            wq, wk = b.Hq // P, b.Hk // P
+            sq = np.stack([oracle.partial_sumsq(np.ascontiguousarray(qf[:, p * wq:(p + 1) * wq]), wq, wq, T)
+                           for p in range(P)])
+            sk = np.stack([oracle.partial_sumsq(np.ascontiguousarray(kf[:, p * wk:(p + 1) * wk]), wk, wk, T)
+                           for p in range(P)])
+            for p in range(P):
+                oracle.combine_apply(np.ascontiguousarray(qf[:, p * wq:(p + 1) * wq]), wq, wq, T,
+                                     gq[p * wq:(p + 1) * wq], sq, b.Hq, b.eps)
+                oracle.combine_apply(np.ascontiguousarray(kf[:, p * wk:(p + 1) * wk]), wk, wk, T,
+                                     gk[p * wk:(p + 1) * wk], sk, b.Hk, b.eps)
+        else:
+            oracle.qknorm_layerwise(qf, b.Hq, gq, b.Hq, kf, b.Hk, gk, b.Hk, T, b.eps)
+
+    calls, t0 = 0, time.perf_counter()
+    while True:
+        one_call()
+        calls += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s or calls >= 1000:
+            break
+    per_call = el / calls
+    eff = 2 * wl.esz * (b.Hq + b.Hk) * T + wl.esz * (b.Hq + b.Hk)
+    return {"value": eff / per_call / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{calls} oracle call(s) on {T} of {b.T} tokens of {wl.name}, {el:.1f} s",
+            "us_per_call": per_call * 1e6, "tokens": T, "calls": calls}
+
+
+# --------------------------------------------------------------------------- native arm
+
+def native(args) -> int:
+    rank, world, local = dist_env()
+    if world != args.gpus and rank == 0:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}", file=sys.stderr)
+    if not torch.cuda.is_available():
+        print(json.dumps({"metric": METRIC, "error": "no CUDA device"}))
+        return 1
+    torch.cuda.set_device(local)
+    dev = torch.device(f"cuda:{local}")
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180), device_id=dev)
+
+    import attention_normalization_b200 as qk
+    qk.capi()  # fails loudly if the library is missing
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if dist is None:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    wl = Workload(args.workload, args.tokens, seed_offset=rank * 1000)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    R = rotating = rotation_count(wl.set_bytes(), l2)
+    sets = [wl.make_set(dev) for _ in range(R)]
+    torch.cuda.synchronize()
+
+    # eager warm-up (loads the library's per-device caches), then capture
+    for i in range(3):
+        wl.step(qk, sets[i % R])
+    torch.cuda.synchronize()
+    g_warm, g_timed = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_warm, capture_error_mode="thread_local"):
+        for i in range(args.warmup):
+            wl.step(qk, sets[i % R])
+    with torch.cuda.graph(g_timed, capture_error_mode="thread_local"):
+        for i in range(args.steps):
+            wl.step(qk, sets[(args.warmup + i) % R])
+    torch.cuda.synchronize()
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    g_warm.replay()  # W untimed warm-up steps
+    stream = torch.cuda.current_stream(dev)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    sampler.active.set()
+    ev0.record(stream)
+    g_timed.replay()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    sampler.active.clear()
+    barrier()
+    ms_rank = ev0.elapsed_time(ev1)
+    ms = max_over_ranks(ms_rank)
+    clocks = sampler.summary()
+
+    step_s = ms / 1e3 / args.steps
+    value = world * wl.eff_bytes / step_s / 1e9
+    per_rank_gbs = wl.eff_bytes / step_s / 1e9
+    peaks = load_peaks()
+    digest = source_digest()
+    kernel_s = step_s / wl.launches_per_step if wl.kind != "gqa" else step_s
+    roofline = {"bound": "hbm", "achieved": round(wl.eff_bytes / kernel_s / 1e9, 1), "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": round(wl.eff_bytes / kernel_s / 1e9 / peaks["hbm_gbs"], 4),
+                "traffic": profiled_traffic(wl.name, digest),
+                "peak_source": f"{peaks['source']} copy bandwidth",
+                "kernel": "qknorm rows kernel (the only kernel of the step)" if wl.kind != "gqa"
+                          else "whole step: partial_stats x P + combine_apply x P",
+                "algorithmic_bytes_per_launch": wl.eff_bytes if wl.kind != "gqa" else None,
+                "source_digest": digest}
+
+    # end to end through the public API with pinned host buffers
+    e2e = e2e_measure(qk, wl, dev, args, barrier, max_over_ranks)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = time_oracle(wl, args.cpu_seconds)
+
+    plan = None
+    if wl.kind in ("prefill", "tiny", "decode", "packed"):
+        s0 = sets[0]
+        if wl.kind == "packed":
+            plan = qk.qknorm_layerwise_plan(s0["q"], s0["k"], s0["gq"], s0["gk"], q_out=s0["q"], k_out=s0["k"])
+        else:
+            plan = qk.qknorm_layerwise_plan(s0["q"], s0["k"], s0["gq"], s0["gk"], q_out=s0["qo"], k_out=s0["ko"])
+
+    if rank == 0:
+        cfg = wl.config()
+        cfg.update({"parallelism": f"replicas x{world} (tokens independent, no collective)",
+                    "l2": f"rotating {R} input/output sets ({R * wl.set_bytes() / 1e6:.0f} MB; "
+                          f"{(R - 1) * wl.set_bytes() / 1e6:.0f} MB touched between reuses > 2 x {l2 / 1e6:.0f} MB L2)",
+                    "timing": "CUDA graph of K captured C-ABI calls, CUDA events on the launching stream",
+                    "launch_plan": plan})
+        line = {"metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 6),
+                "us_per_call": round(step_s * 1e6 / wl.launches_per_step, 3),
+                "pct_of_peak": round(100 * per_rank_gbs / peaks["hbm_gbs"], 2),
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+                "data": "synthetic (seeded; OLMo2-shaped activations, no dataset or weights)",
+                "config": cfg, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+                "gpu_launches": args.steps * wl.launches_per_step, "clocks": clocks,
+                "impl": "native"}
+        print(json.dumps(line))
+    del g_warm, g_timed
+    if dist is not None:
+        dist.destroy_process_group()
+    return 0
+
+
+def e2e_measure(qk, wl: Workload, dev, args, barrier, max_over_ranks) -> dict:
+    b = wl.batch
+    steps = max(1, min(args.e2e_steps, args.steps))
+    s = wl.make_set(dev)
+    if wl.kind == "packed":
+        h_in = [b.packed.clone().pin_memory()]
+        d_in = [s["base"]]
+        d_out = [s["base"]]
+    elif wl.kind == "gqa":
+        h_in = [t.clone().pin_memory() for t in b.q_shards + b.k_shards]
+        d_in = s["qs"] + s["ks"]
+        d_out = s["qo"] + s["ko"]
+    else:
+        h_in = [b.q.clone().pin_memory(), b.k.clone().pin_memory()]
+        d_in = [s["q"], s["k"]]
+        d_out = [s["qo"], s["ko"]]
+    h_g = [b.gamma_q.clone().pin_memory(), b.gamma_k.clone().pin_memory()]
+    d_g = [s["gq"], s["gk"]] if "gq" in s else [torch.empty_like(b.gamma_q, device=dev),
+                                                 torch.empty_like(b.gamma_k, device=dev)]
+    h_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in d_out]
+    h2d = sum(t.numel() * t.element_size() for t in h_in + h_g)
+    d2h = sum(t.numel() * t.element_size() for t in h_out)
+
+    def one():
+        for h, d in zip(h_in + h_g, d_in + d_g):
+            d.copy_(h, non_blocking=True)
+        if wl.kind == "gqa":
+            P = b.P
+            wq, wk = b.Hq // P, b.Hk // P
+            for p in range(P):
+                s["gqs"][p].copy_(d_g[0][p * wq:(p + 1) * wq])
+                s["gks"][p].copy_(d_g[1][p * wk:(p + 1) * wk])
+        wl.step(qk, s)
+        for h, d in zip(h_out, d_out):
+            h.copy_(d, non_blocking=True)
+
+    for _ in range(2):
+        one()
+    stream = torch.cuda.current_stream(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    barrier()
+    e0.record(stream)
+    for _ in range(steps):
+        one()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms = max_over_ranks(e0.elapsed_time(e1))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    return {"value": round(world * wl.eff_bytes / (ms / 1e3 / steps) / 1e9, 2), "unit": UNIT,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
+            "ms_per_step": round(ms / steps, 4),
+            "path": "pinned host -> device copies, qknorm_layerwise via the Python binding (eager), "
+                    "device -> pinned host copies, one stream"}
+
+
+# --------------------------------------------------------------------------- reference arm (the oracle)
+
+def reference(args) -> int:
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0  # the CPU oracle runs once, on rank 0
+    wl = Workload(args.workload, args.tokens, seed_offset=0)
+    b = wl.batch
+    # per-step sample: enough tokens that the whole run stays near a minute
+    probe = time_oracle(wl, 0.0, max_tokens=min(b.T, 8))
+    per_token_s = probe["us_per_call"] / 1e6 / probe["tokens"]
+    budget_s = 60.0
+    tokens = int(max(1, min(b.T, budget_s / ((args.steps + args.warmup) * per_token_s))))
+    for _ in range(args.warmup):
+        time_oracle(wl, 0.0, max_tokens=tokens)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        time_oracle(wl, 0.0, max_tokens=tokens)
+    el = time.perf_counter() - t0
+    eff = 2 * wl.esz * (b.Hq + b.Hk) * tokens + wl.esz * (b.Hq + b.Hk)
+    value = eff / (el / args.steps) / 1e9
+    cfg = wl.config()
+    cfg.update({"sample_tokens_per_step": tokens})
+    line = {"metric": METRIC, "value": round(value, 5), "unit": UNIT, "n_gpus": 0, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(el / args.steps * 1e3, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": cfg,
+            "impl": "reference",
+            "cpu_baseline": {"value": round(value, 5), "unit": UNIT, "cores": 1, "kind": "oracle",
+                             "sample": f"{tokens} of {b.T} tokens of {wl.name} per step, one thread"},
+            "e2e": {"value": round(value, 5), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+    return 0
+
+
+def main(argv=None) -> int:
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return reference(args)
+    return native(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,138 @@
+/*
+ * qknorm.h — C-ABI of libqknorm.so: layerwise QK-RMSNorm for NVIDIA B200 (sm_100a).
+ *
+ * What it computes ("SwiftQK: Fast and Communication-Efficient Tensor
+ * Parallelism for Query-Key Normalization", arXiv 2608.09160):
+ *
+ *   Background, RMS-Norm (Equation 1).  For the full projected Q row and the
+ *   full projected K row of every token, one factor per row:
+ *       S = sum_j x_j^2,   r = 1 / sqrt(S / H + eps),   y_j = (x_j * gamma_j) * r
+ *   with eps inside the square root and the mean over the full width H.  (The
+ *   page lost the typeset equation; this is the reading its surrounding text,
+ *   its RMSNorm citation and the phase descriptions support.)
+ *
+ *   Phase A.  The factor needs only the squared sum; a hidden-dimension shard
+ *   contributes its local squared sum, and the shard sums (fp32) add up to the
+ *   global one, with the same semantics as the unsharded form.
+ *
+ *   Phase B.  The weight multiplication x * gamma does not depend on the
+ *   reduction; the global factor r is applied to it and only the final
+ *   normalized values are written.
+ *
+ * Arithmetic: elements are widened to fp32; squared sums, the factor and the
+ * scaling are fp32 (squares accumulated with fused multiply-add); outputs are
+ * rounded once to the element type (round-to-nearest-even).  The factor uses
+ * the device's rsqrtf.  NaN/Inf inputs propagate as IEEE arithmetic does; a
+ * squared sum above FLT_MAX overflows to +inf (fp32 accumulation).
+ *
+ * Conventions shared by every entry point:
+ *   - Pointers are DEVICE pointers of the current CUDA device; the caller owns
+ *     every buffer.  The library allocates nothing and keeps no state besides a
+ *     per-device cache of launch occupancy and a per-thread error message.
+ *   - Layout: row-major.  Element (t, j) of a tensor with row stride `stride`
+ *     (in ELEMENTS, >= the row width) is at base[t * stride + j].  Packed
+ *     [Q | K | V] rows are addressed by passing base and base + Hq with the
+ *     packed stride; columns outside [0, width) (V, padding) are never read
+ *     or written.
+ *   - gamma vectors are contiguous, of the element type, one per tensor (or
+ *     per shard, for the shard entry points).
+ *   - out == in (same base, same stride) normalizes in place.  Any other
+ *     overlap between a written region and any other region is rejected with
+ *     QKN_ERR_INVALID_ARG.  Two strided regions with different strides whose
+ *     address ranges intersect are rejected even if their elements happen to
+ *     be disjoint.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Every
+ *     call only enqueues work: it is asynchronous and never synchronizes.
+ *   - T == 0 returns QKN_OK without launching anything.
+ *   - Arguments are validated on the host before any launch; a rejected call
+ *     enqueues nothing.  QKN_ERR_CUDA reports a launch failure (the message
+ *     is available from qknorm_last_error on the calling thread).
+ *   - Alignment is never an error: when every base pointer and every row
+ *     stride in bytes is a multiple of 16, rows move as 16-byte vectors;
+ *     otherwise a scalar-access kernel runs (still on the GPU).
+ *   - Thread safety: calls may be made from several host threads at once.
+ */
+#ifndef QKNORM_H
+#define QKNORM_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    QKN_F32 = 0,   /* IEEE binary32 elements */
+    QKN_BF16 = 1   /* bfloat16 elements */
+} qkn_dtype;
+
+typedef enum {
+    QKN_OK = 0,
+    QKN_ERR_INVALID_ARG = 1,   /* bad size, stride, eps, dtype, null pointer or overlap */
+    QKN_ERR_UNSUPPORTED = 2,   /* a launch shape this build cannot run */
+    QKN_ERR_CUDA = 3           /* the CUDA runtime reported an error */
+} qkn_status;
+
+/*
+ * Fused layerwise QK-Norm: normalizes the Q row and the K row of all T tokens
+ * in ONE kernel launch (Background, Equation 1; Phase B's fused weight
+ * multiplication and store).
+ *   q_in, q_out : [T rows, stride q_stride] elements; Q width Hq.
+ *   k_in, k_out : [T rows, stride k_stride] elements; K width Hk.
+ *   gamma_q [Hq], gamma_k [Hk].
+ *   eps >= 0 and finite.  dtype: element type of every buffer.
+ * Errors: QKN_ERR_INVALID_ARG for T < 0, Hq or Hk <= 0, a stride below its
+ * width, a bad eps or dtype, a null pointer with T > 0, or a forbidden overlap.
+ */
+qkn_status qknorm_layerwise(const void *q_in, void *q_out, const void *gamma_q, int64_t q_stride,
+                            const void *k_in, void *k_out, const void *gamma_k, int64_t k_stride,
+                            int64_t T, int32_t Hq, int32_t Hk, float eps, qkn_dtype dtype,
+                            void *stream);
+
+/*
+ * Phase A, local step, for one hidden-dimension shard of Q and of K: writes
+ * the fp32 squared sum of each token's shard row.
+ *   q_shard : [T rows, stride q_stride], shard width hq_shard; q_sumsq : [T] fp32 (written).
+ *   k_shard : [T rows, stride k_stride], shard width hk_shard; k_sumsq : [T] fp32 (written).
+ * For P shards the caller keeps a [P][T] fp32 array per tensor and passes
+ * sumsq_all + p * T for shard p.
+ * Errors: as qknorm_layerwise; the two sum arrays must not overlap each other
+ * or the inputs.
+ */
+qkn_status qknorm_partial_stats(const void *q_shard, int64_t q_stride, int32_t hq_shard, float *q_sumsq,
+                                const void *k_shard, int64_t k_stride, int32_t hk_shard, float *k_sumsq,
+                                int64_t T, qkn_dtype dtype, void *stream);
+
+/*
+ * Phase A aggregation followed by Phase B for one shard: for each token the P
+ * partial sums sumsq_all[p * T + t] are added in fp32 in the fixed order
+ * p = 0..P-1, r = 1 / sqrt(S / H_full + eps) divides by the FULL width
+ * (Hq_full / Hk_full, not the shard width), and the shard's elements are
+ * written as (x * gamma_shard) * r.
+ *   q_in, q_out : [T rows, stride q_stride], width hq_shard; gamma_q_shard [hq_shard].
+ *   q_sumsq_all : [P][T] fp32, contiguous.   Hq_full >= hq_shard.
+ *   (same for K.)   P >= 1.
+ * Errors: as qknorm_layerwise, plus P < 1 or a full width below its shard
+ * width; outputs must not overlap the sum arrays.
+ */
+qkn_status qknorm_combine_apply(const void *q_in, void *q_out, const void *gamma_q_shard, int64_t q_stride,
+                                int32_t hq_shard, const float *q_sumsq_all, int32_t Hq_full,
+                                const void *k_in, void *k_out, const void *gamma_k_shard, int64_t k_stride,
+                                int32_t hk_shard, const float *k_sumsq_all, int32_t Hk_full,
+                                int32_t P, int64_t T, float eps, qkn_dtype dtype, void *stream);
+
+/* Short English name of a status code (static storage). */
+const char *qknorm_status_string(qkn_status s);
+
+/* Message describing the last non-OK status returned on the calling thread
+ * ("" if none).  The pointer stays valid until the thread's next call. */
+const char *qknorm_last_error(void);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+int qknorm_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QKNORM_H */

@@ -1,0 +1,115 @@
+/*
+ * qknorm_plan.h — launch planning for libqknorm.so, exported so that the host
+ * logic can be tested without a GPU and so that a caller can pin a launch
+ * shape (benchmark sweeps, per-variant tests).  Include after qknorm.h.
+ *
+ * Execution model (the single-GPU form of the paper's "deadlock-safe
+ * persistent execution"): a kernel launches a bounded grid — at most as many
+ * CTAs as can be resident at once — and each CTA loops over row items
+ * blockIdx.x, blockIdx.x + grid, ...  Item i is row i / 2 of Q (i even) or of
+ * K (i odd), so the Q and K rows of a token are processed side by side.  A
+ * CTA works on one row at a time.
+ *
+ * Kernel kinds:
+ *   QKN_KERNEL_REGISTER  one pass; the row is held in registers, each thread
+ *                        owning up to vec_per_thread 16-byte vectors
+ *                        (vector v of a row belongs to thread v % threads);
+ *                        every element is read once and written once.
+ *                        Needs 16-byte alignment (see qknorm.h) and a row of
+ *                        at most vec_per_thread * threads vectors.
+ *   QKN_KERNEL_TWOPASS_VEC  two passes over the row with 16-byte vectors
+ *                        (the second pass re-reads x, mostly from L2); for
+ *                        rows too wide for registers.
+ *   QKN_KERNEL_TWOPASS_SCALAR  two passes with element-wise access; for
+ *                        buffers that are not 16-byte aligned.
+ */
+#ifndef QKNORM_PLAN_H
+#define QKNORM_PLAN_H
+
+#include <stdint.h>
+#include "qknorm.h"
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    QKN_KERNEL_REGISTER = 0,
+    QKN_KERNEL_TWOPASS_VEC = 1,
+    QKN_KERNEL_TWOPASS_SCALAR = 2
+} qkn_kernel_kind;
+
+typedef struct {
+    int32_t kernel;          /* qkn_kernel_kind */
+    int32_t vec_per_thread;  /* QKN_KERNEL_REGISTER only: 1, 2, 4 or 8 */
+    int32_t threads;         /* threads per CTA: a multiple of 32 in [32, 1024] */
+    int64_t grid;            /* number of CTAs, >= 1 */
+} qkn_launch;
+
+/* Largest CTA the register kernel accepts for a given vec_per_thread
+ * (1024 for 1 and 2, 512 for 4, 256 for 8); 0 for an unsupported value. */
+int32_t qknorm_register_max_threads(int32_t vec_per_thread);
+
+/*
+ * Chooses kernel kind, vec_per_thread and threads (grid is left 0) from:
+ *   rows       : row items in the launch (2 * T),
+ *   units_max  : the widest row, in 16-byte vectors if `vectorized`, else in elements,
+ *   vectorized : 1 if every pointer and row stride is 16-byte aligned,
+ *   sm_count   : streaming multiprocessors on the device.
+ * Pure function of its arguments; needs no GPU.  QKN_ERR_INVALID_ARG for
+ * rows < 1, units_max < 1 or sm_count < 1.
+ */
+qkn_status qknorm_plan_shape(int64_t rows, int64_t units_max, int32_t vectorized, int32_t sm_count,
+                             qkn_launch *out);
+
+/*
+ * CTAs for `rows` items when `blocks_per_sm` CTAs fit on each of `sm_count`
+ * SMs: never more than fit at once, and balanced so every CTA gets
+ * ceil(rows / grid) or one fewer items with as few loop trips as the resident
+ * limit allows.  Pure; returns 0 for rows < 1, and treats a non-positive
+ * blocks_per_sm or sm_count as 1.
+ */
+int64_t qknorm_plan_grid(int64_t rows, int32_t blocks_per_sm, int32_t sm_count);
+
+/*
+ * 1 if two row sets may share a byte, 0 if they are provably disjoint.  A row
+ * set is `rows` byte ranges [base + t * stride, base + t * stride + width).
+ * Exact when either set has one row or both strides are equal; otherwise any
+ * intersection of the address ranges counts as overlap (conservative).
+ * Empty sets (rows < 1 or width < 1) never overlap.
+ */
+int qknorm_regions_overlap(uint64_t a_base, int64_t a_width, int64_t a_stride, int64_t a_rows,
+                           uint64_t b_base, int64_t b_width, int64_t b_stride, int64_t b_rows);
+
+/*
+ * The launch qknorm_layerwise would use for these arguments on the current
+ * device (queries the SM count and the kernel's occupancy; needs a GPU).
+ * Validates its arguments exactly as qknorm_layerwise does.
+ */
+qkn_status qknorm_layerwise_plan(const void *q_in, void *q_out, const void *gamma_q, int64_t q_stride,
+                                 const void *k_in, void *k_out, const void *gamma_k, int64_t k_stride,
+                                 int64_t T, int32_t Hq, int32_t Hk, float eps, qkn_dtype dtype,
+                                 qkn_launch *out);
+
+/*
+ * qknorm_layerwise with a caller-chosen launch.  The squared sum is formed in
+ * an order fixed by the launch shape (per-thread sequential, then a warp
+ * butterfly, then warp partials in order), so a given shape is deterministic
+ * run to run, while two shapes may differ in the last bits of the sum and
+ * hence by one unit in the last place of an output.  Beyond the checks of
+ * qknorm_layerwise, QKN_ERR_INVALID_ARG when: threads is not a multiple of 32
+ * in [32, 1024]; grid < 1 or grid > 2^31 - 1; a vector kernel is asked for on
+ * unaligned buffers; for the register kernel, vec_per_thread is not 1, 2, 4
+ * or 8, threads exceeds qknorm_register_max_threads(vec_per_thread), or the
+ * widest row has more than vec_per_thread * threads vectors.
+ */
+qkn_status qknorm_layerwise_launch(const void *q_in, void *q_out, const void *gamma_q, int64_t q_stride,
+                                   const void *k_in, void *k_out, const void *gamma_k, int64_t k_stride,
+                                   int64_t T, int32_t Hq, int32_t Hk, float eps, qkn_dtype dtype,
+                                   void *stream, const qkn_launch *launch);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QKNORM_PLAN_H */

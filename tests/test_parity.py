@@ -1,0 +1,278 @@
+"""GPU parity: the CUDA path (through the C-ABI) against the CPU oracle on the
+same seeded input bytes.
+
+Tolerances (fp32 accumulation on the GPU, double in the oracle):
+  * fp32 outputs: max_j |y - o| / max(|o|, 1e-30) <= 1e-5, o the oracle's
+    unrounded double value;
+  * bf16 outputs: at most 1 unit in the last place between the GPU's bf16 and
+    the oracle's correctly rounded bf16, counted over ordered bit patterns;
+  * fp32 partial squared sums: relative error <= 1e-5.
+Why these hold: the GPU's squared sum of H terms carries a relative error of
+roughly (terms per thread + log2(threads)) * 2^-24 (well under 1e-5 for every
+shape here), rsqrtf adds at most 2 ulp and the two multiplies one ulp each, so
+an fp32 output is within ~1e-6 relative of the exact value; a bf16 output can
+then only differ from the correctly rounded one when the exact value lies that
+close to a rounding boundary, i.e. by one unit.
+
+Configurations are the five benchmark workloads (full sizes, the launch the
+library picks by default, which is what the benchmark times) plus small and
+ragged shapes, unaligned buffers, wide rows and every kernel variant.
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import attention_normalization_b200 as qk
+import oracle
+import workloads
+from tests.conftest import bf16_ulp_distance, buffer_np, to_np
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+
+
+# --------------------------------------------------------------------------- helpers
+
+def oracle_rows(view: torch.Tensor, gamma: torch.Tensor, eps: float):
+    """Oracle on a (possibly strided) CPU view: (rounded y, exact y, sumsq)."""
+    T, H = view.shape
+    if T == 0:
+        return (np.zeros((0, H), dtype=to_np(gamma).dtype), np.zeros((0, H)), np.zeros((0,)))
+    flat, stride = buffer_np(view)
+    return oracle.rmsnorm_rows(flat, H, to_np(gamma), eps, stride=stride, T=T)
+
+
+def assert_close(got: torch.Tensor, y_rounded: np.ndarray, y_exact: np.ndarray, what: str):
+    got = got.detach().cpu().contiguous()
+    if got.dtype == torch.bfloat16:
+        d = bf16_ulp_distance(to_np(got), y_rounded)
+        worst = int(d.max()) if d.size else 0
+        assert worst <= 1, f"{what}: {worst} bf16 ulp from the oracle (at {np.unravel_index(d.argmax(), d.shape)})"
+    else:
+        o = y_exact
+        rel = np.abs(got.double().numpy() - o) / np.maximum(np.abs(o), 1e-30)
+        worst = float(rel.max()) if rel.size else 0.0
+        assert worst <= 1e-5, f"{what}: relative error {worst:.3g} > 1e-5"
+
+
+def upload(batch: workloads.QKBatch):
+    """Device copies keeping every layout detail (strides, padding, packing)."""
+    if batch.packed is not None:
+        base = batch.packed.to(DEV)
+        q = base[:, :batch.Hq]
+        k = base[:, batch.Hq:batch.Hq + batch.Hk]
+        return q, k, base
+    qb = batch.meta.get("q_buffer")
+    kb = batch.meta.get("k_buffer")
+    if qb is not None:
+        qd, kd = qb.to(DEV), kb.to(DEV)
+        return qd[:batch.T, :batch.Hq], kd[:batch.T, :batch.Hk], (qd, kd)
+    return batch.q.to(DEV), batch.k.to(DEV), None
+
+
+def check_layerwise(batch: workloads.QKBatch, in_place: bool = False, launch=None):
+    q, k, keep = upload(batch)
+    gq, gk = batch.gamma_q.to(DEV), batch.gamma_k.to(DEV)
+    before = keep[0].clone() if isinstance(keep, tuple) else (keep.clone() if keep is not None else None)
+    if in_place:
+        qo, ko = qk.qknorm_layerwise(q, k, gq, gk, batch.eps, q_out=q, k_out=k, launch=launch)
+    else:
+        qo, ko = qk.qknorm_layerwise(q, k, gq, gk, batch.eps, launch=launch)
+    torch.cuda.synchronize()
+    yq, eq, _ = oracle_rows(batch.q, batch.gamma_q, batch.eps)
+    yk, ek, _ = oracle_rows(batch.k, batch.gamma_k, batch.eps)
+    assert_close(qo, yq, eq, f"{batch.name} Q")
+    assert_close(ko, yk, ek, f"{batch.name} K")
+    return q, k, qo, ko, keep, before
+
+
+# --------------------------------------------------------------------------- the five workloads
+
+def test_tiny_fp32_out_of_place_then_in_place_bitwise_equal():
+    b = workloads.tiny_fp32()
+    _, _, qo, ko, _, _ = check_layerwise(b)
+    q2, k2, qi, ki, _, _ = check_layerwise(b, in_place=True)
+    assert qi.data_ptr() == q2.data_ptr()
+    assert torch.equal(qo, qi) and torch.equal(ko, ki)
+
+
+def test_prefill_bf16_full_size():
+    b = workloads.prefill_bf16()
+    check_layerwise(b)
+
+
+@pytest.mark.parametrize("T", workloads.DECODE_TOKENS)
+def test_decode_bf16(T):
+    check_layerwise(workloads.decode_bf16(T))
+
+
+def test_gqa_shard_decomposed_full_size():
+    b = workloads.gqa_sharded()
+    P, T = b.P, b.T
+    qs = [s.to(DEV) for s in b.q_shards]
+    ks = [s.to(DEV) for s in b.k_shards]
+    wq, wk = b.Hq // P, b.Hk // P
+    q_all = torch.empty((P, T), dtype=torch.float32, device=DEV)
+    k_all = torch.empty((P, T), dtype=torch.float32, device=DEV)
+    for p in range(P):
+        qk.qknorm_partial_stats(qs[p], ks[p], q_all[p], k_all[p])
+    gq, gk = b.gamma_q.to(DEV), b.gamma_k.to(DEV)
+    outs = []
+    for p in range(P):
+        outs.append(qk.qknorm_combine_apply(qs[p], ks[p], gq[p * wq:(p + 1) * wq].contiguous(),
+                                            gk[p * wk:(p + 1) * wk].contiguous(), q_all, k_all,
+                                            b.Hq, b.Hk, b.eps))
+    torch.cuda.synchronize()
+    # Phase A partial sums against the oracle's double partial sums
+    for p in range(P):
+        oq = oracle.partial_sumsq(to_np(b.q_shards[p]), wq, wq, T)
+        ok_ = oracle.partial_sumsq(to_np(b.k_shards[p]), wk, wk, T)
+        np.testing.assert_allclose(q_all[p].cpu().double().numpy(), oq, rtol=1e-5, atol=0)
+        np.testing.assert_allclose(k_all[p].cpu().double().numpy(), ok_, rtol=1e-5, atol=0)
+    # outputs against the oracle over the FULL rows
+    yq, eq, _ = oracle_rows(b.q_full, b.gamma_q, b.eps)
+    yk, ek, _ = oracle_rows(b.k_full, b.gamma_k, b.eps)
+    got_q = torch.cat([o[0] for o in outs], dim=1)
+    got_k = torch.cat([o[1] for o in outs], dim=1)
+    assert_close(got_q, yq, eq, "gqa Q shards")
+    assert_close(got_k, yk, ek, "gqa K shards")
+    # ... and against the fused kernel on the unsplit rows (at most one ulp apart:
+    # the two forms add the same squares in different orders)
+    fq, fk = qk.qknorm_layerwise(b.q_full.to(DEV), b.k_full.to(DEV), gq, gk, b.eps)
+    assert int(bf16_ulp_distance(to_np(fq.cpu()), to_np(got_q.cpu())).max()) <= 1
+    assert int(bf16_ulp_distance(to_np(fk.cpu()), to_np(got_k.cpu())).max()) <= 1
+
+
+@pytest.mark.parametrize("T", workloads.PACKED_TOKENS)
+def test_packed_qkv_in_place_v_untouched(T):
+    b = workloads.packed_qkv(T)
+    _, _, _, _, base, before = check_layerwise(b, in_place=True)
+    v0 = b.Hq + b.Hk
+    assert torch.equal(base[:, v0:], before[:, v0:]), "V columns were modified"
+
+
+# --------------------------------------------------------------------------- edge cases
+
+def aligned_stride(H: int, dtype: torch.dtype, extra_vectors: int = 1) -> int:
+    """A row stride whose byte size is a multiple of 16, leaving padding after H."""
+    per = 16 // (4 if dtype == torch.float32 else 2)
+    return -(-H // per) * per + extra_vectors * per
+
+
+@pytest.mark.parametrize("layout", ["contiguous", "padded"])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("T,Hq,Hk", [(1, 1, 1), (2, 3, 7), (3, 8, 9), (17, 127, 129), (5, 513, 64),
+                                      (33, 4096, 1024), (7, 5120, 5120), (300, 1000, 24)])
+def test_small_and_ragged_shapes(layout, dtype, T, Hq, Hk):
+    """Layout "contiguous": strides equal the widths (unaligned whenever a width
+    is not a multiple of the vector).  Layout "padded": strides are 16-byte
+    multiples, so widths that are not run the vector kernels' ragged tail."""
+    kw = {}
+    if layout == "padded":
+        kw = dict(q_stride=aligned_stride(Hq, dtype), k_stride=aligned_stride(Hk, dtype))
+    check_layerwise(workloads.random_rows(T, Hq, Hk, dtype, seed=T * 131 + Hq + Hk, **kw))
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_padding_columns_untouched(dtype):
+    Hq, Hk = 203, 43  # ragged: neither is a whole number of 16-byte vectors
+    b = workloads.random_rows(9, Hq, Hk, dtype, seed=3, q_stride=aligned_stride(Hq, dtype, 3),
+                              k_stride=aligned_stride(Hk, dtype))
+    q, k, _ = upload(b)
+    assert qk.qknorm_layerwise_plan(q, k, b.gamma_q.to(DEV), b.gamma_k.to(DEV))["kernel"] == 0
+    q, k, qo, ko, keep, before = check_layerwise(b, in_place=True)
+    qd, kd = keep
+    assert torch.all(qd[:, Hq:].float() == -7.0) and torch.all(kd[:, Hk:].float() == -7.0)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_unaligned_buffers_use_the_scalar_kernel(dtype):
+    b = workloads.random_rows(13, 301, 77, dtype, seed=4, q_stride=301, k_stride=77)
+    q, k, _ = upload(b)
+    gq, gk = b.gamma_q.to(DEV), b.gamma_k.to(DEV)
+    plan = qk.qknorm_layerwise_plan(q, k, gq, gk)
+    assert plan["kernel"] == 2
+    check_layerwise(b)
+    # shift the start by one element: still correct
+    buf = torch.zeros((13 * 301 + 1,), dtype=dtype)
+    buf[1:] = b.q.reshape(-1)
+    bq = buf[1:].view(13, 301)
+    shifted = workloads.QKBatch("shifted", dtype, 13, 301, 77, bq, b.k, b.gamma_q, b.gamma_k)
+    qd = buf.to(DEV)[1:].view(13, 301)
+    qo, ko = qk.qknorm_layerwise(qd, k, gq, gk, b.eps)
+    yq, eq, _ = oracle_rows(shifted.q, b.gamma_q, b.eps)
+    assert_close(qo, yq, eq, "shifted Q")
+
+
+@pytest.mark.parametrize("dtype,H", [(torch.bfloat16, 20000), (torch.float32, 9000)])
+def test_rows_too_wide_for_registers(dtype, H):
+    b = workloads.random_rows(6, H, 64, dtype, seed=5)
+    q, k, _ = upload(b)
+    assert qk.qknorm_layerwise_plan(q, k, b.gamma_q.to(DEV), b.gamma_k.to(DEV))["kernel"] == 1
+    check_layerwise(b)
+
+
+def test_zero_rows_give_zero_and_empty_batch_is_a_no_op():
+    b = workloads.random_rows(4, 64, 32, torch.bfloat16, seed=6)
+    b.q[1].zero_()
+    b.meta["q_buffer"][1].zero_()
+    q, k, qo, ko, _, _ = check_layerwise(b)
+    assert torch.all(qo[1] == 0)
+    e = torch.empty((0, 64), dtype=torch.bfloat16, device=DEV)
+    g = torch.ones((64,), dtype=torch.bfloat16, device=DEV)
+    a, c = qk.qknorm_layerwise(e, e, g, g)
+    assert a.shape == (0, 64)
+
+
+@pytest.mark.parametrize("launch", [
+    {"kernel": 0, "vec_per_thread": 1, "threads": 1024, "grid": 7},
+    {"kernel": 0, "vec_per_thread": 2, "threads": 256, "grid": 148},
+    {"kernel": 0, "vec_per_thread": 4, "threads": 128, "grid": 1},
+    {"kernel": 0, "vec_per_thread": 8, "threads": 64, "grid": 1000},
+    {"kernel": 1, "vec_per_thread": 0, "threads": 96, "grid": 33},
+    {"kernel": 2, "vec_per_thread": 0, "threads": 1024, "grid": 5},
+])
+def test_every_kernel_variant_matches_the_oracle_and_is_deterministic(launch):
+    b = workloads.random_rows(67, 4096, 1000, torch.bfloat16, seed=7)
+    _, _, qo, ko, _, _ = check_layerwise(b, launch=launch)
+    _, _, qo2, ko2, _, _ = check_layerwise(b, launch=launch)
+    assert torch.equal(qo, qo2) and torch.equal(ko, ko2)
+
+
+def test_fp32_variants_and_apply_with_one_shard_equals_fused():
+    b = workloads.tiny_fp32()
+    q, k = b.q.to(DEV), b.k.to(DEV)
+    gq, gk = b.gamma_q.to(DEV), b.gamma_k.to(DEV)
+    sq, sk = qk.qknorm_partial_stats(q, k)
+    yq, eq, s_or = oracle_rows(b.q, b.gamma_q, b.eps)
+    np.testing.assert_allclose(sq.cpu().double().numpy(), s_or, rtol=1e-5)
+    aq, ak = qk.qknorm_combine_apply(q, k, gq, gk, sq[None, :], sk[None, :], b.Hq, b.Hk, b.eps)
+    assert_close(aq, yq, eq, "P=1 apply Q")
+    fq, fk = qk.qknorm_layerwise(q, k, gq, gk, b.eps)
+    # same launch shape, same squared sums: P = 1 apply reproduces the fused result bit for bit
+    assert torch.equal(aq, fq) and torch.equal(ak, fk)
+
+
+def test_runs_on_a_side_stream():
+    b = workloads.random_rows(64, 2048, 512, torch.bfloat16, seed=8)
+    q, k, _ = upload(b)
+    gq, gk = b.gamma_q.to(DEV), b.gamma_k.to(DEV)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        qo, ko = qk.qknorm_layerwise(q, k, gq, gk, b.eps)
+    s.synchronize()
+    yq, eq, _ = oracle_rows(b.q, b.gamma_q, b.eps)
+    assert_close(qo, yq, eq, "side stream Q")
+
+
+def test_invalid_call_on_gpu_raises_and_launches_nothing():
+    x = torch.zeros((4, 64), dtype=torch.bfloat16, device=DEV)
+    g = torch.ones((64,), dtype=torch.bfloat16, device=DEV)
+    with pytest.raises(qk.QKNormError, match="invalid argument"):
+        qk.qknorm_layerwise(x, x, g, g, -1.0)
+    big = torch.zeros((4, 128), dtype=torch.bfloat16, device=DEV)
+    with pytest.raises(qk.QKNormError, match="overlap"):
+        qk.qknorm_layerwise(big[:, :64], big[:, 32:96], g, g, q_out=big[:, :64], k_out=big[:, 32:96])
