@@ -77,6 +77,39 @@ def dist_env():
     return rank, world, local
 
 
+class Ranks:
+    """Barrier and max-over-ranks for the timing plumbing (no data-path
+    collective).  ``dist`` is torch.distributed or None (one process); NCCL
+    needs a CUDA ``device`` for its tensors, gloo takes the CPU."""
+
+    def __init__(self, dist=None, device=None):
+        self.dist = dist
+        self.device = device if device is not None else torch.device("cpu")
+
+    @property
+    def world(self) -> int:
+        return self.dist.get_world_size() if self.dist is not None else 1
+
+    def barrier(self):
+        if self.dist is not None:
+            self.dist.barrier()
+
+    def max(self, x: float) -> float:
+        if self.dist is None:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=self.device)
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
+        return float(t.item())
+
+
+def whole_job(eff_bytes_per_step: int, steps: int, max_ms: float, world: int) -> dict:
+    """Whole-job throughput: every rank processed `steps` steps of
+    `eff_bytes_per_step`; the job took the slowest rank's time."""
+    step_s = max_ms / 1e3 / steps
+    return {"value_gbs": world * eff_bytes_per_step / step_s / 1e9, "ms_per_step": max_ms / steps,
+            "per_rank_gbs": eff_bytes_per_step / step_s / 1e9}
+
+
 def load_peaks() -> dict:
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -343,16 +376,8 @@ def native(args) -> int:
     import attention_normalization_b200 as qk
     qk.capi()  # fails loudly if the library is missing
 
-    def barrier():
-        if dist is not None:
-            dist.barrier()
-
-    def max_over_ranks(x: float) -> float:
-        if dist is None:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    ranks = Ranks(dist, dev)
+    barrier, max_over_ranks = ranks.barrier, ranks.max
 
     wl = Workload(args.workload, args.tokens, seed_offset=rank * 1000)
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
@@ -392,9 +417,10 @@ def native(args) -> int:
     ms = max_over_ranks(ms_rank)
     clocks = sampler.summary()
 
-    step_s = ms / 1e3 / args.steps
-    value = world * wl.eff_bytes / step_s / 1e9
-    per_rank_gbs = wl.eff_bytes / step_s / 1e9
+    agg = whole_job(wl.eff_bytes, args.steps, ms, world)
+    step_s = agg["ms_per_step"] / 1e3
+    value = agg["value_gbs"]
+    per_rank_gbs = agg["per_rank_gbs"]
     peaks = load_peaks()
     digest = source_digest()
     kernel_s = step_s / wl.launches_per_step if wl.kind != "gqa" else step_s
