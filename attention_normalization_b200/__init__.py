@@ -40,6 +40,7 @@ def version() -> int:
     return capi().qknorm_version()
 
 
+
 # --------------------------------------------------------------------------- marshalling
 
 def _rows(t: torch.Tensor, name: str):
@@ -112,8 +113,10 @@ def qknorm_layerwise(q_in: torch.Tensor, k_in: torch.Tensor, gamma_q: torch.Tens
                      stream=None, launch: QknLaunch | dict | None = None):
     """Fused layerwise QK-Norm of all tokens in one launch; returns ``(q_out, k_out)``.
 
-    ``launch`` pins a launch shape (``qkn_launch``); results are identical for
-    every valid shape.  Asynchronous on ``stream`` (default: the current stream).
+    ``launch`` pins a launch shape (``qkn_launch``); every valid shape agrees
+    with the default within one unit in the last place (the squared sum is
+    added in a shape-dependent order) and is deterministic run to run.
+    Asynchronous on ``stream`` (default: the current stream).
     """
     args, q_out, k_out, dev = _layerwise_args(q_in, k_in, gamma_q, gamma_k, eps, q_out, k_out)
     lib = capi()

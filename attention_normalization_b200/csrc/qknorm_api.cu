@@ -47,6 +47,7 @@ bool dtype_valid(int dt) { return dt == QKN_F32 || dt == QKN_BF16; }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+
 // ---------------------------------------------------------------------------
 // Overlap of two row sets.
 int64_t floor_div(int64_t a, int64_t b) {  // b > 0
@@ -117,6 +118,7 @@ struct OccEntry {
     const void *fn;
     int device;
     int threads;
+    int64_t smem;
     int blocks;
 };
 constexpr int kOccSlots = 512;
@@ -149,43 +151,46 @@ qkn_status sm_count(int dev, int *out) {
     return QKN_OK;
 }
 
-qkn_status blocks_per_sm(const void *fn, int dev, int threads, int *out) {
+qkn_status blocks_per_sm(const void *fn, int dev, int threads, int64_t dyn_smem, int *out) {
     {
         std::lock_guard<std::mutex> lk(g_occ_mu);
         for (int i = 0; i < g_occ_n; ++i)
-            if (g_occ[i].fn == fn && g_occ[i].device == dev && g_occ[i].threads == threads) {
+            if (g_occ[i].fn == fn && g_occ[i].device == dev && g_occ[i].threads == threads &&
+                g_occ[i].smem == dyn_smem) {
                 *out = g_occ[i].blocks;
                 return QKN_OK;
             }
     }
     int n = 0;
-    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, threads, 0);
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, threads, (size_t)dyn_smem);
     if (e != cudaSuccess)
         return fail(QKN_ERR_CUDA, "cudaOccupancyMaxActiveBlocksPerMultiprocessor: %s", cudaGetErrorString(e));
     if (n < 1) return fail(QKN_ERR_UNSUPPORTED, "kernel cannot run with %d threads per CTA", threads);
     std::lock_guard<std::mutex> lk(g_occ_mu);
-    if (g_occ_n < kOccSlots) g_occ[g_occ_n++] = OccEntry{fn, dev, threads, n};
+    if (g_occ_n < kOccSlots) g_occ[g_occ_n++] = OccEntry{fn, dev, threads, dyn_smem, n};
     *out = n;
     return QKN_OK;
 }
 
 // ---------------------------------------------------------------------------
 // Kernel selection.
-template <typename E, int MODE>
+template <typename E, int MODE, bool TAIL>
 const void *register_kernel(int nv) {
     switch (nv) {
-        case 1: return (const void *)qkn::rows_register_kernel<E, 1, MODE>;
-        case 2: return (const void *)qkn::rows_register_kernel<E, 2, MODE>;
-        case 4: return (const void *)qkn::rows_register_kernel<E, 4, MODE>;
-        case 8: return (const void *)qkn::rows_register_kernel<E, 8, MODE>;
+        case 1: return (const void *)qkn::rows_register_kernel<E, 1, MODE, TAIL>;
+        case 2: return (const void *)qkn::rows_register_kernel<E, 2, MODE, TAIL>;
+        case 4: return (const void *)qkn::rows_register_kernel<E, 4, MODE, TAIL>;
+        case 8: return (const void *)qkn::rows_register_kernel<E, 8, MODE, TAIL>;
         default: return nullptr;
     }
 }
 
 template <typename E, int MODE>
-const void *kernel_for(const qkn_launch &L) {
+const void *kernel_for(const qkn_launch &L, bool tail) {
     switch (L.kernel) {
-        case QKN_KERNEL_REGISTER: return register_kernel<E, MODE>(L.vec_per_thread);
+        case QKN_KERNEL_REGISTER:
+            return tail ? register_kernel<E, MODE, true>(L.vec_per_thread)
+                        : register_kernel<E, MODE, false>(L.vec_per_thread);
         case QKN_KERNEL_TWOPASS_VEC: return (const void *)qkn::rows_twopass_kernel<E, true, MODE>;
         case QKN_KERNEL_TWOPASS_SCALAR: return (const void *)qkn::rows_twopass_kernel<E, false, MODE>;
         default: return nullptr;
@@ -193,8 +198,8 @@ const void *kernel_for(const qkn_launch &L) {
 }
 
 template <int MODE>
-const void *kernel_for(qkn_dtype dt, const qkn_launch &L) {
-    return dt == QKN_F32 ? kernel_for<float, MODE>(L) : kernel_for<__nv_bfloat16, MODE>(L);
+const void *kernel_for(qkn_dtype dt, const qkn_launch &L, bool tail) {
+    return dt == QKN_F32 ? kernel_for<float, MODE>(L, tail) : kernel_for<__nv_bfloat16, MODE>(L, tail);
 }
 
 // A prepared call: parameters plus the facts planning needs.
@@ -202,6 +207,7 @@ struct Call {
     qkn::Params p;
     qkn_dtype dtype;
     bool vectorized;
+    bool tail;          // some row ends in a partial 16-byte vector
     int64_t units_max;  // widest row in vectors (vectorized) or elements
 };
 
@@ -217,7 +223,7 @@ void fill_rowset(qkn::RowSet &s, const void *in, void *out, const void *gamma, i
     s.width = width;
     s.nfull = width / per_vec;
     s.tail = width % per_vec;
-    s.div = static_cast<float>(div_width);
+    s.inv_div = static_cast<float>(1.0 / static_cast<double>(div_width));
 }
 
 void finish_call(Call &c, int esz, std::initializer_list<const void *> ptrs, int64_t q_stride, int64_t k_stride) {
@@ -229,6 +235,26 @@ void finish_call(Call &c, int esz, std::initializer_list<const void *> ptrs, int
     int64_t wq = c.p.set[0].width, wk = c.p.set[1].width;
     int64_t w = wq > wk ? wq : wk;
     c.units_max = v ? (w + per_vec - 1) / per_vec : w;
+    c.tail = c.p.set[0].tail != 0 || c.p.set[1].tail != 0;
+}
+
+// Row groups of the register kernel for a launch of `threads` threads with
+// `nv` vectors each: the smallest group (a multiple of 32 dividing the CTA)
+// whose threads cover the tensor's row, and the items that follow.
+void set_groups(qkn::Params &p, int threads, int nv) {
+    for (int w = 0; w < 2; ++w) {
+        qkn::RowSet &d = p.set[w];
+        const int64_t units = (int64_t)d.nfull + (d.tail ? 1 : 0);
+        int group = threads;
+        for (int g = 32; g < threads; g += 32)
+            if (threads % g == 0 && (int64_t)g * nv >= units) {
+                group = g;
+                break;
+            }
+        d.group = group;
+        d.rows_per_item = threads / group;
+        d.items = (p.T + d.rows_per_item - 1) / d.rows_per_item;
+    }
 }
 
 bool eps_valid(float eps) { return std::isfinite(eps) && eps >= 0.0f; }
@@ -296,7 +322,6 @@ qkn_status prepare_layerwise(const void *q_in, void *q_out, const void *gamma_q,
     fill_rowset(c.p.set[0], q_in, q_out, gamma_q, q_stride, Hq, Hq, esz);
     fill_rowset(c.p.set[1], k_in, k_out, gamma_k, k_stride, Hk, Hk, esz);
     c.p.T = T;
-    c.p.rows = 2 * T;
     c.p.eps = eps;
     c.p.P = 1;
     finish_call(c, esz, {q_in, q_out, gamma_q, k_in, k_out, gamma_k}, q_stride, k_stride);
@@ -309,12 +334,19 @@ qkn_status plan_call(const Call &c, qkn_launch &L) {
     qkn_status st = current_device(&dev);
     if (st != QKN_OK) return st;
     if ((st = sm_count(dev, &sms)) != QKN_OK) return st;
-    if ((st = qknorm_plan_shape(c.p.rows, c.units_max, c.vectorized ? 1 : 0, sms, &L)) != QKN_OK)
+    const int64_t items = 2 * c.p.T;
+    if ((st = qknorm_plan_shape(items, c.units_max, c.vectorized ? 1 : 0, sms, &L)) != QKN_OK)
         return fail(st, "planning failed");
-    const void *fn = kernel_for<MODE>(c.dtype, L);
+    const void *fn = kernel_for<MODE>(c.dtype, L, c.tail);
     if (!fn) return fail(QKN_ERR_UNSUPPORTED, "no kernel for the planned launch");
-    if ((st = blocks_per_sm(fn, dev, L.threads, &bps)) != QKN_OK) return st;
-    L.grid = qknorm_plan_grid(c.p.rows, bps, sms);
+    if ((st = blocks_per_sm(fn, dev, L.threads, 0, &bps)) != QKN_OK) return st;
+    int64_t work = items;
+    if (L.kernel == QKN_KERNEL_REGISTER) {  // narrow rows share CTAs: count items, not rows
+        qkn::Params p = c.p;
+        set_groups(p, L.threads, L.vec_per_thread);
+        work = p.set[0].items + p.set[1].items;
+    }
+    L.grid = qknorm_plan_grid(work, bps, sms);
     return QKN_OK;
 }
 
@@ -341,21 +373,32 @@ qkn_status check_launch(const Call &c, const qkn_launch &L) {
     }
 }
 
+template <typename E, int MODE, bool TAIL>
+void launch_register(int nv, dim3 grid, dim3 block, cudaStream_t s, const qkn::Params &p) {
+    switch (nv) {
+        case 1: qkn::rows_register_kernel<E, 1, MODE, TAIL><<<grid, block, 0, s>>>(p); break;
+        case 2: qkn::rows_register_kernel<E, 2, MODE, TAIL><<<grid, block, 0, s>>>(p); break;
+        case 4: qkn::rows_register_kernel<E, 4, MODE, TAIL><<<grid, block, 0, s>>>(p); break;
+        case 8: qkn::rows_register_kernel<E, 8, MODE, TAIL><<<grid, block, 0, s>>>(p); break;
+        default: break;
+    }
+}
+
 template <typename E, int MODE>
-cudaError_t launch_typed(const qkn_launch &L, const qkn::Params &p, cudaStream_t s) {
+cudaError_t launch_typed(const qkn_launch &L, const Call &c, cudaStream_t s) {
     const dim3 grid((unsigned)L.grid), block((unsigned)L.threads);
     switch (L.kernel) {
-        case QKN_KERNEL_REGISTER:
-            switch (L.vec_per_thread) {
-                case 1: qkn::rows_register_kernel<E, 1, MODE><<<grid, block, 0, s>>>(p); break;
-                case 2: qkn::rows_register_kernel<E, 2, MODE><<<grid, block, 0, s>>>(p); break;
-                case 4: qkn::rows_register_kernel<E, 4, MODE><<<grid, block, 0, s>>>(p); break;
-                case 8: qkn::rows_register_kernel<E, 8, MODE><<<grid, block, 0, s>>>(p); break;
-                default: return cudaErrorInvalidValue;
-            }
+        case QKN_KERNEL_REGISTER: {
+            qkn::Params p = c.p;
+            set_groups(p, L.threads, L.vec_per_thread);
+            if (c.tail)
+                launch_register<E, MODE, true>(L.vec_per_thread, grid, block, s, p);
+            else
+                launch_register<E, MODE, false>(L.vec_per_thread, grid, block, s, p);
             break;
-        case QKN_KERNEL_TWOPASS_VEC: qkn::rows_twopass_kernel<E, true, MODE><<<grid, block, 0, s>>>(p); break;
-        case QKN_KERNEL_TWOPASS_SCALAR: qkn::rows_twopass_kernel<E, false, MODE><<<grid, block, 0, s>>>(p); break;
+        }
+        case QKN_KERNEL_TWOPASS_VEC: qkn::rows_twopass_kernel<E, true, MODE><<<grid, block, 0, s>>>(c.p); break;
+        case QKN_KERNEL_TWOPASS_SCALAR: qkn::rows_twopass_kernel<E, false, MODE><<<grid, block, 0, s>>>(c.p); break;
         default: return cudaErrorInvalidValue;
     }
     return cudaGetLastError();
@@ -364,8 +407,8 @@ cudaError_t launch_typed(const qkn_launch &L, const qkn::Params &p, cudaStream_t
 template <int MODE>
 qkn_status launch(const Call &c, const qkn_launch &L, void *stream) {
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    cudaError_t e = c.dtype == QKN_F32 ? launch_typed<float, MODE>(L, c.p, s)
-                                        : launch_typed<__nv_bfloat16, MODE>(L, c.p, s);
+    cudaError_t e = c.dtype == QKN_F32 ? launch_typed<float, MODE>(L, c, s)
+                                        : launch_typed<__nv_bfloat16, MODE>(L, c, s);
     if (e != cudaSuccess) return fail(QKN_ERR_CUDA, "kernel launch: %s", cudaGetErrorString(e));
     return ok();
 }
@@ -409,8 +452,8 @@ qkn_status qknorm_plan_shape(int64_t rows, int64_t units_max, int32_t vectorized
     int nv;
     if (rows <= sm_count) {
         // Few rows (decode): spread each row over many threads so a row costs
-        // about one memory round trip.
-        nv = units_max <= 1024 ? 1 : 2;
+        // about one memory round trip (two vectors per thread measured best).
+        nv = units_max < 128 ? 1 : 2;
     } else {
         // Many rows: moderate CTAs, several vectors in flight per thread.
         nv = units_max >= 256 ? 4 : (units_max >= 64 ? 2 : 1);
@@ -431,8 +474,7 @@ int64_t qknorm_plan_grid(int64_t rows, int32_t blocks_per_sm, int32_t sm_count) 
     const int64_t bps = blocks_per_sm > 0 ? blocks_per_sm : 1;
     const int64_t sms = sm_count > 0 ? sm_count : 1;
     const int64_t resident = bps * sms;
-    const int64_t trips = (rows + resident - 1) / resident;
-    return (rows + trips - 1) / trips;
+    return rows < resident ? rows : resident;
 }
 
 int qknorm_regions_overlap(uint64_t a_base, int64_t a_width, int64_t a_stride, int64_t a_rows,
@@ -513,7 +555,6 @@ qkn_status qknorm_partial_stats(const void *q_shard, int64_t q_stride, int32_t h
     c.p.set[0].sumsq = q_sumsq;
     c.p.set[1].sumsq = k_sumsq;
     c.p.T = T;
-    c.p.rows = 2 * T;
     c.p.eps = 0.0f;
     c.p.P = 1;
     finish_call(c, esz, {q_shard, k_shard}, q_stride, k_stride);
@@ -558,7 +599,6 @@ qkn_status qknorm_combine_apply(const void *q_in, void *q_out, const void *gamma
     c.p.set[0].sumsq_all = q_sumsq_all;
     c.p.set[1].sumsq_all = k_sumsq_all;
     c.p.T = T;
-    c.p.rows = 2 * T;
     c.p.eps = eps;
     c.p.P = P;
     finish_call(c, esz, {q_in, q_out, gamma_q_shard, k_in, k_out, gamma_k_shard}, q_stride, k_stride);

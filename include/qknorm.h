@@ -20,9 +20,10 @@
  *   normalized values are written.
  *
  * Arithmetic: elements are widened to fp32; squared sums, the factor and the
- * scaling are fp32 (squares accumulated with fused multiply-add); outputs are
- * rounded once to the element type (round-to-nearest-even).  The factor uses
- * the device's rsqrtf.  NaN/Inf inputs propagate as IEEE arithmetic does; a
+ * scaling are fp32 (squares accumulated with fused multiply-add); the mean is
+ * formed as S * fl(1/H), with 1/H rounded to fp32 once on the host (exact when
+ * H is a power of two); the factor uses the device's rsqrtf; outputs are
+ * rounded once to the element type (round-to-nearest-even).  NaN/Inf inputs propagate as IEEE arithmetic does; a
  * squared sum above FLT_MAX overflows to +inf (fp32 accumulation).
  *
  * Conventions shared by every entry point:

@@ -6,15 +6,18 @@
  * Execution model (the single-GPU form of the paper's "deadlock-safe
  * persistent execution"): a kernel launches a bounded grid — at most as many
  * CTAs as can be resident at once — and each CTA loops over row items
- * blockIdx.x, blockIdx.x + grid, ...  Item i is row i / 2 of Q (i even) or of
- * K (i odd), so the Q and K rows of a token are processed side by side.  A
- * CTA works on one row at a time.
+ * blockIdx.x, blockIdx.x + grid, ...  Items 0..T-1 are the Q rows and items
+ * T..2T-1 the K rows, so every CTA gets a near-equal share of each tensor's
+ * rows whatever the grid.  A CTA works on one row at a time.  No CTA ever
+ * waits on another, so any grid is safe.
  *
  * Kernel kinds:
  *   QKN_KERNEL_REGISTER  one pass; the row is held in registers, each thread
  *                        owning up to vec_per_thread 16-byte vectors
- *                        (vector v of a row belongs to thread v % threads);
- *                        every element is read once and written once.
+ *                        (vector v of a row belongs to thread v % threads, the
+ *                        same positions in every row, so a thread keeps its
+ *                        gamma vectors in registers across the rows of one
+ *                        tensor); every element is read once and written once.
  *                        Needs 16-byte alignment (see qknorm.h) and a row of
  *                        at most vec_per_thread * threads vectors.
  *   QKN_KERNEL_TWOPASS_VEC  two passes over the row with 16-byte vectors
@@ -64,10 +67,9 @@ qkn_status qknorm_plan_shape(int64_t rows, int64_t units_max, int32_t vectorized
 
 /*
  * CTAs for `rows` items when `blocks_per_sm` CTAs fit on each of `sm_count`
- * SMs: never more than fit at once, and balanced so every CTA gets
- * ceil(rows / grid) or one fewer items with as few loop trips as the resident
- * limit allows.  Pure; returns 0 for rows < 1, and treats a non-positive
- * blocks_per_sm or sm_count as 1.
+ * SMs: min(rows, blocks_per_sm * sm_count), i.e. every resident slot is
+ * filled and no CTA waits for a slot.  Pure; returns 0 for rows < 1, and
+ * treats a non-positive blocks_per_sm or sm_count as 1.
  */
 int64_t qknorm_plan_grid(int64_t rows, int32_t blocks_per_sm, int32_t sm_count);
 

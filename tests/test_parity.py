@@ -227,19 +227,54 @@ def test_zero_rows_give_zero_and_empty_batch_is_a_no_op():
     assert a.shape == (0, 64)
 
 
-@pytest.mark.parametrize("launch", [
+VARIANTS = [
     {"kernel": 0, "vec_per_thread": 1, "threads": 1024, "grid": 7},
     {"kernel": 0, "vec_per_thread": 2, "threads": 256, "grid": 148},
     {"kernel": 0, "vec_per_thread": 4, "threads": 128, "grid": 1},
+    {"kernel": 0, "vec_per_thread": 4, "threads": 128, "grid": 1184},
     {"kernel": 0, "vec_per_thread": 8, "threads": 64, "grid": 1000},
+    {"kernel": 0, "vec_per_thread": 8, "threads": 256, "grid": 134},
     {"kernel": 1, "vec_per_thread": 0, "threads": 96, "grid": 33},
     {"kernel": 2, "vec_per_thread": 0, "threads": 1024, "grid": 5},
-])
-def test_every_kernel_variant_matches_the_oracle_and_is_deterministic(launch):
-    b = workloads.random_rows(67, 4096, 1000, torch.bfloat16, seed=7)
+]
+
+
+def _cover(launch: dict, units: int) -> dict | None:
+    """Widen a register launch so that it covers `units` vectors, or None if
+    no CTA of its vec_per_thread can."""
+    if launch["kernel"] != 0:
+        return launch
+    nv = launch["vec_per_thread"]
+    if nv * launch["threads"] >= units:
+        return launch
+    limit = 1024 if nv <= 2 else (512 if nv == 4 else 256)
+    threads = -(-units // nv)
+    threads = -(-threads // 32) * 32
+    return None if threads > limit else dict(launch, threads=threads)
+
+
+@pytest.mark.parametrize("launch", VARIANTS, ids=lambda L: "k{kernel}_nv{vec_per_thread}_t{threads}_g{grid}".format(**L))
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("Hk", [1000, 1003])
+def test_every_kernel_variant_matches_the_oracle_and_is_deterministic(launch, dtype, Hk):
+    """Hk = 1003 leaves K rows with a ragged last vector (padded, aligned stride)."""
+    per = 4 if dtype == torch.float32 else 8
+    launch = _cover(launch, -(-4096 // per))
+    if launch is None:
+        pytest.skip("no CTA of this vec_per_thread covers the fp32 row")
+    b = workloads.random_rows(67, 4096, Hk, dtype, seed=7, k_stride=aligned_stride(Hk, dtype))
     _, _, qo, ko, _, _ = check_layerwise(b, launch=launch)
     _, _, qo2, ko2, _, _ = check_layerwise(b, launch=launch)
     assert torch.equal(qo, qo2) and torch.equal(ko, ko2)
+
+
+@pytest.mark.parametrize("T", [1, 3, 300])
+def test_register_kernel_in_place_on_packed_rows_any_grid(T):
+    """Q-first items with an even grid: both tensors' rows are covered."""
+    b = workloads.packed_qkv(T)
+    launch = {"kernel": 0, "vec_per_thread": 4, "threads": 128, "grid": 2 if T > 1 else 1}
+    _, _, _, _, base, before = check_layerwise(b, in_place=True, launch=launch)
+    assert torch.equal(base[:, b.Hq + b.Hk:], before[:, b.Hq + b.Hk:])
 
 
 def test_fp32_variants_and_apply_with_one_shard_equals_fused():
