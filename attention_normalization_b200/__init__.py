@@ -125,8 +125,7 @@ def qknorm_layerwise(q_in: torch.Tensor, k_in: torch.Tensor, gamma_q: torch.Tens
         if launch is None:
             st = lib.qknorm_layerwise(*args, s)
         else:
-            L = launch if isinstance(launch, QknLaunch) else QknLaunch(**launch)
-            st = lib.qknorm_layerwise_launch(*args, s, ctypes.byref(L))
+            st = lib.qknorm_layerwise_launch(*args, s, ctypes.byref(_launch_struct(launch)))
     _clib.check(st, "qknorm_layerwise")
     return q_out, k_out
 
@@ -142,8 +141,12 @@ def qknorm_layerwise_plan(q_in, k_in, gamma_q, gamma_k, eps: float = 1e-6, *, q_
     return L.as_dict()
 
 
+def _launch_struct(launch):
+    return launch if isinstance(launch, QknLaunch) else QknLaunch(**launch)
+
+
 def qknorm_partial_stats(q_shard: torch.Tensor, k_shard: torch.Tensor, q_sumsq=None, k_sumsq=None,
-                         *, stream=None):
+                         *, stream=None, launch: QknLaunch | dict | None = None):
     """Phase A local step: fp32 squared sum of every token's Q-shard and K-shard
     row; returns ``(q_sumsq, k_sumsq)``, each ``[T]`` float32 (a row of a
     caller-owned ``[P, T]`` array may be passed)."""
@@ -159,9 +162,13 @@ def qknorm_partial_stats(q_shard: torch.Tensor, k_shard: torch.Tensor, q_sumsq=N
         k_sumsq = torch.empty((T,), dtype=torch.float32, device=dev)
     pq = _vec(q_sumsq, "q_sumsq", T, torch.float32, dev)
     pk = _vec(k_sumsq, "k_sumsq", T, torch.float32, dev)
+    args = [q_shard.data_ptr(), sq, hq, pq, k_shard.data_ptr(), sk, hk, pk, T, _DTYPES[dt]]
     with torch.cuda.device(dev):
-        st = capi().qknorm_partial_stats(q_shard.data_ptr(), sq, hq, pq, k_shard.data_ptr(), sk, hk, pk,
-                                         T, _DTYPES[dt], _stream_handle(stream, dev))
+        s = _stream_handle(stream, dev)
+        if launch is None:
+            st = capi().qknorm_partial_stats(*args, s)
+        else:
+            st = capi().qknorm_partial_stats_launch(*args, s, ctypes.byref(_launch_struct(launch)))
     _clib.check(st, "qknorm_partial_stats")
     return q_sumsq, k_sumsq
 
@@ -169,7 +176,7 @@ def qknorm_partial_stats(q_shard: torch.Tensor, k_shard: torch.Tensor, q_sumsq=N
 def qknorm_combine_apply(q_in: torch.Tensor, k_in: torch.Tensor, gamma_q_shard: torch.Tensor,
                          gamma_k_shard: torch.Tensor, q_sumsq_all: torch.Tensor,
                          k_sumsq_all: torch.Tensor, Hq_full: int, Hk_full: int, eps: float = 1e-6,
-                         *, q_out=None, k_out=None, stream=None):
+                         *, q_out=None, k_out=None, stream=None, launch: QknLaunch | dict | None = None):
     """Phase A aggregation of the ``[P, T]`` fp32 partial sums (order p = 0..P-1),
     factor over the FULL widths, then scale this shard; returns ``(q_out, k_out)``."""
     T, hq, sq = _rows(q_in, "q_in")
@@ -193,12 +200,16 @@ def qknorm_combine_apply(q_in: torch.Tensor, k_in: torch.Tensor, gamma_q_shard: 
         To, Ho, so = _rows(t, name)
         if (To, Ho) != (T, H) or (T > 1 and so != s):
             raise ValueError(f"{name} must match its input's shape and row stride")
-    with torch.cuda.device(dev):
-        st = capi().qknorm_combine_apply(
-            q_in.data_ptr(), q_out.data_ptr(), _vec(gamma_q_shard, "gamma_q_shard", hq, dt, dev), sq, hq,
+    args = [q_in.data_ptr(), q_out.data_ptr(), _vec(gamma_q_shard, "gamma_q_shard", hq, dt, dev), sq, hq,
             ps_q, int(Hq_full),
             k_in.data_ptr(), k_out.data_ptr(), _vec(gamma_k_shard, "gamma_k_shard", hk, dt, dev), sk, hk,
-            ps_k, int(Hk_full), P, T, float(eps), _DTYPES[dt], _stream_handle(stream, dev))
+            ps_k, int(Hk_full), P, T, float(eps), _DTYPES[dt]]
+    with torch.cuda.device(dev):
+        s = _stream_handle(stream, dev)
+        if launch is None:
+            st = capi().qknorm_combine_apply(*args, s)
+        else:
+            st = capi().qknorm_combine_apply_launch(*args, s, ctypes.byref(_launch_struct(launch)))
     _clib.check(st, "qknorm_combine_apply")
     return q_out, k_out
 

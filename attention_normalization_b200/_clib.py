@@ -55,6 +55,11 @@ PROTOTYPES = {
     "qknorm_regions_overlap": (ctypes.c_int, [_u64, _i64, _i64, _i64, _u64, _i64, _i64, _i64]),
     "qknorm_layerwise_plan": (_st, _LAYERWISE_ARGS + [ctypes.POINTER(QknLaunch)]),
     "qknorm_layerwise_launch": (_st, _LAYERWISE_ARGS + [_vp, ctypes.POINTER(QknLaunch)]),
+    "qknorm_partial_stats_launch": (_st, [_vp, _i64, _i32, _vp, _vp, _i64, _i32, _vp, _i64, _dt, _vp,
+                                          ctypes.POINTER(QknLaunch)]),
+    "qknorm_combine_apply_launch": (_st, [_vp, _vp, _vp, _i64, _i32, _vp, _i32,
+                                          _vp, _vp, _vp, _i64, _i32, _vp, _i32,
+                                          _i32, _i64, _f32, _dt, _vp, ctypes.POINTER(QknLaunch)]),
 }
 
 _lib = None

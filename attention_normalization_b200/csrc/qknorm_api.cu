@@ -373,44 +373,114 @@ qkn_status check_launch(const Call &c, const qkn_launch &L) {
     }
 }
 
-template <typename E, int MODE, bool TAIL>
-void launch_register(int nv, dim3 grid, dim3 block, cudaStream_t s, const qkn::Params &p) {
-    switch (nv) {
-        case 1: qkn::rows_register_kernel<E, 1, MODE, TAIL><<<grid, block, 0, s>>>(p); break;
-        case 2: qkn::rows_register_kernel<E, 2, MODE, TAIL><<<grid, block, 0, s>>>(p); break;
-        case 4: qkn::rows_register_kernel<E, 4, MODE, TAIL><<<grid, block, 0, s>>>(p); break;
-        case 8: qkn::rows_register_kernel<E, 8, MODE, TAIL><<<grid, block, 0, s>>>(p); break;
-        default: break;
-    }
+// Every launch allows programmatic dependent launch: the kernel may be
+// dispatched while the previous kernel in the stream drains (see
+// pdl_wait_and_release in the kernels, which restores the ordering).
+cudaError_t launch_pdl(const void *fn, unsigned grid, unsigned block, cudaStream_t s, const qkn::Params &p) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    void *args[] = {const_cast<qkn::Params *>(&p)};
+    return cudaLaunchKernelExC(&cfg, fn, args);
 }
 
-template <typename E, int MODE>
-cudaError_t launch_typed(const qkn_launch &L, const Call &c, cudaStream_t s) {
-    const dim3 grid((unsigned)L.grid), block((unsigned)L.threads);
-    switch (L.kernel) {
-        case QKN_KERNEL_REGISTER: {
-            qkn::Params p = c.p;
-            set_groups(p, L.threads, L.vec_per_thread);
-            if (c.tail)
-                launch_register<E, MODE, true>(L.vec_per_thread, grid, block, s, p);
-            else
-                launch_register<E, MODE, false>(L.vec_per_thread, grid, block, s, p);
-            break;
-        }
-        case QKN_KERNEL_TWOPASS_VEC: qkn::rows_twopass_kernel<E, true, MODE><<<grid, block, 0, s>>>(c.p); break;
-        case QKN_KERNEL_TWOPASS_SCALAR: qkn::rows_twopass_kernel<E, false, MODE><<<grid, block, 0, s>>>(c.p); break;
-        default: return cudaErrorInvalidValue;
-    }
-    return cudaGetLastError();
+template <int MODE>
+cudaError_t launch_any(const qkn_launch &L, const Call &c, cudaStream_t s) {
+    const void *fn = kernel_for<MODE>(c.dtype, L, c.tail);
+    if (!fn) return cudaErrorInvalidValue;
+    qkn::Params p = c.p;
+    if (L.kernel == QKN_KERNEL_REGISTER) set_groups(p, L.threads, L.vec_per_thread);
+    return launch_pdl(fn, (unsigned)L.grid, (unsigned)L.threads, s, p);
 }
 
 template <int MODE>
 qkn_status launch(const Call &c, const qkn_launch &L, void *stream) {
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    cudaError_t e = c.dtype == QKN_F32 ? launch_typed<float, MODE>(L, c, s)
-                                        : launch_typed<__nv_bfloat16, MODE>(L, c, s);
+    cudaError_t e = launch_any<MODE>(L, c, static_cast<cudaStream_t>(stream));
+    if (e == cudaSuccess) e = cudaGetLastError();
     if (e != cudaSuccess) return fail(QKN_ERR_CUDA, "kernel launch: %s", cudaGetErrorString(e));
     return ok();
+}
+
+qkn_status prepare_stats(const void *q_shard, int64_t q_stride, int32_t hq_shard, float *q_sumsq,
+                         const void *k_shard, int64_t k_stride, int32_t hk_shard, float *k_sumsq, int64_t T,
+                         qkn_dtype dtype, Call &c) {
+    if (!dtype_valid(dtype)) return fail(QKN_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
+    if (T < 0) return fail(QKN_ERR_INVALID_ARG, "T = %lld < 0", (long long)T);
+    if (hq_shard <= 0 || hk_shard <= 0) return fail(QKN_ERR_INVALID_ARG, "shard widths must be positive");
+    if (q_stride < hq_shard || k_stride < hk_shard) return fail(QKN_ERR_INVALID_ARG, "row stride below shard width");
+    const int esz = elem_bytes(dtype);
+    if (!extent_ok(T, q_stride, hq_shard, esz) || !extent_ok(T, k_stride, hk_shard, esz))
+        return fail(QKN_ERR_INVALID_ARG, "buffer extent overflows");
+    if (T > 0 && (!q_shard || !q_sumsq || !k_shard || !k_sumsq)) return fail(QKN_ERR_INVALID_ARG, "null pointer");
+    if (T > 0) {
+        const Region iq = rows_region(q_shard, hq_shard, q_stride, T, esz);
+        const Region ik = rows_region(k_shard, hk_shard, k_stride, T, esz);
+        const Region sq = flat_region(q_sumsq, T * 4), sk = flat_region(k_sumsq, T * 4);
+        if (overlap(sq, sk)) return fail(QKN_ERR_INVALID_ARG, "q_sumsq and k_sumsq overlap");
+        if (overlap(sq, iq) || overlap(sq, ik) || overlap(sk, iq) || overlap(sk, ik))
+            return fail(QKN_ERR_INVALID_ARG, "a sum array overlaps an input");
+    }
+    std::memset(&c, 0, sizeof(c));
+    c.dtype = dtype;
+    fill_rowset(c.p.set[0], q_shard, nullptr, nullptr, q_stride, hq_shard, hq_shard, esz);
+    fill_rowset(c.p.set[1], k_shard, nullptr, nullptr, k_stride, hk_shard, hk_shard, esz);
+    c.p.set[0].sumsq = q_sumsq;
+    c.p.set[1].sumsq = k_sumsq;
+    c.p.T = T;
+    c.p.eps = 0.0f;
+    c.p.P = 1;
+    finish_call(c, esz, {q_shard, k_shard}, q_stride, k_stride);
+    return QKN_OK;
+}
+
+qkn_status prepare_apply(const void *q_in, void *q_out, const void *gamma_q_shard, int64_t q_stride,
+                         int32_t hq_shard, const float *q_sumsq_all, int32_t Hq_full, const void *k_in, void *k_out,
+                         const void *gamma_k_shard, int64_t k_stride, int32_t hk_shard, const float *k_sumsq_all,
+                         int32_t Hk_full, int32_t P, int64_t T, float eps, qkn_dtype dtype, Call &c) {
+    if (!dtype_valid(dtype)) return fail(QKN_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
+    if (T < 0) return fail(QKN_ERR_INVALID_ARG, "T = %lld < 0", (long long)T);
+    if (P < 1) return fail(QKN_ERR_INVALID_ARG, "P = %d < 1", P);
+    if (hq_shard <= 0 || hk_shard <= 0) return fail(QKN_ERR_INVALID_ARG, "shard widths must be positive");
+    if (Hq_full < hq_shard || Hk_full < hk_shard) return fail(QKN_ERR_INVALID_ARG, "full width below shard width");
+    if (q_stride < hq_shard || k_stride < hk_shard) return fail(QKN_ERR_INVALID_ARG, "row stride below shard width");
+    if (!eps_valid(eps)) return fail(QKN_ERR_INVALID_ARG, "eps must be finite and >= 0");
+    const int esz = elem_bytes(dtype);
+    if (!extent_ok(T, q_stride, hq_shard, esz) || !extent_ok(T, k_stride, hk_shard, esz) ||
+        !extent_ok(1, 0, (int64_t)P * T, 4))
+        return fail(QKN_ERR_INVALID_ARG, "buffer extent overflows");
+    if (T > 0 && (!q_in || !q_out || !gamma_q_shard || !q_sumsq_all || !k_in || !k_out || !gamma_k_shard ||
+                  !k_sumsq_all))
+        return fail(QKN_ERR_INVALID_ARG, "null pointer");
+    if (T > 0) {
+        const Region iq = rows_region(q_in, hq_shard, q_stride, T, esz);
+        const Region oq = rows_region(q_out, hq_shard, q_stride, T, esz);
+        const Region ik = rows_region(k_in, hk_shard, k_stride, T, esz);
+        const Region ok_ = rows_region(k_out, hk_shard, k_stride, T, esz);
+        const Region others[4] = {flat_region(gamma_q_shard, (int64_t)hq_shard * esz),
+                                  flat_region(gamma_k_shard, (int64_t)hk_shard * esz),
+                                  flat_region(q_sumsq_all, (int64_t)P * T * 4),
+                                  flat_region(k_sumsq_all, (int64_t)P * T * 4)};
+        qkn_status st = check_outputs(oq, ok_, iq, ik, others, 4);
+        if (st != QKN_OK) return st;
+    }
+    std::memset(&c, 0, sizeof(c));
+    c.dtype = dtype;
+    fill_rowset(c.p.set[0], q_in, q_out, gamma_q_shard, q_stride, hq_shard, Hq_full, esz);
+    fill_rowset(c.p.set[1], k_in, k_out, gamma_k_shard, k_stride, hk_shard, Hk_full, esz);
+    c.p.set[0].sumsq_all = q_sumsq_all;
+    c.p.set[1].sumsq_all = k_sumsq_all;
+    c.p.T = T;
+    c.p.eps = eps;
+    c.p.P = P;
+    finish_call(c, esz, {q_in, q_out, gamma_q_shard, k_in, k_out, gamma_k_shard}, q_stride, k_stride);
+    return QKN_OK;
 }
 
 }  // namespace
@@ -532,36 +602,27 @@ qkn_status qknorm_layerwise_launch(const void *q_in, void *q_out, const void *ga
 qkn_status qknorm_partial_stats(const void *q_shard, int64_t q_stride, int32_t hq_shard, float *q_sumsq,
                                 const void *k_shard, int64_t k_stride, int32_t hk_shard, float *k_sumsq,
                                 int64_t T, qkn_dtype dtype, void *stream) {
-    if (!dtype_valid(dtype)) return fail(QKN_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
-    if (T < 0) return fail(QKN_ERR_INVALID_ARG, "T = %lld < 0", (long long)T);
-    if (hq_shard <= 0 || hk_shard <= 0) return fail(QKN_ERR_INVALID_ARG, "shard widths must be positive");
-    if (q_stride < hq_shard || k_stride < hk_shard) return fail(QKN_ERR_INVALID_ARG, "row stride below shard width");
-    const int esz = elem_bytes(dtype);
-    if (!extent_ok(T, q_stride, hq_shard, esz) || !extent_ok(T, k_stride, hk_shard, esz))
-        return fail(QKN_ERR_INVALID_ARG, "buffer extent overflows");
-    if (T > 0 && (!q_shard || !q_sumsq || !k_shard || !k_sumsq)) return fail(QKN_ERR_INVALID_ARG, "null pointer");
-    if (T == 0) return ok();
-    const Region iq = rows_region(q_shard, hq_shard, q_stride, T, esz);
-    const Region ik = rows_region(k_shard, hk_shard, k_stride, T, esz);
-    const Region sq = flat_region(q_sumsq, T * 4), sk = flat_region(k_sumsq, T * 4);
-    if (overlap(sq, sk)) return fail(QKN_ERR_INVALID_ARG, "q_sumsq and k_sumsq overlap");
-    if (overlap(sq, iq) || overlap(sq, ik) || overlap(sk, iq) || overlap(sk, ik))
-        return fail(QKN_ERR_INVALID_ARG, "a sum array overlaps an input");
     Call c;
-    std::memset(&c, 0, sizeof(c));
-    c.dtype = dtype;
-    fill_rowset(c.p.set[0], q_shard, nullptr, nullptr, q_stride, hq_shard, hq_shard, esz);
-    fill_rowset(c.p.set[1], k_shard, nullptr, nullptr, k_stride, hk_shard, hk_shard, esz);
-    c.p.set[0].sumsq = q_sumsq;
-    c.p.set[1].sumsq = k_sumsq;
-    c.p.T = T;
-    c.p.eps = 0.0f;
-    c.p.P = 1;
-    finish_call(c, esz, {q_shard, k_shard}, q_stride, k_stride);
-    qkn_launch L;
-    qkn_status st = plan_call<qkn::kStats>(c, L);
+    qkn_status st = prepare_stats(q_shard, q_stride, hq_shard, q_sumsq, k_shard, k_stride, hk_shard, k_sumsq, T,
+                                  dtype, c);
     if (st != QKN_OK) return st;
+    if (T == 0) return ok();
+    qkn_launch L;
+    if ((st = plan_call<qkn::kStats>(c, L)) != QKN_OK) return st;
     return launch<qkn::kStats>(c, L, stream);
+}
+
+qkn_status qknorm_partial_stats_launch(const void *q_shard, int64_t q_stride, int32_t hq_shard, float *q_sumsq,
+                                       const void *k_shard, int64_t k_stride, int32_t hk_shard, float *k_sumsq,
+                                       int64_t T, qkn_dtype dtype, void *stream, const qkn_launch *launch_cfg) {
+    if (!launch_cfg) return fail(QKN_ERR_INVALID_ARG, "null launch");
+    Call c;
+    qkn_status st = prepare_stats(q_shard, q_stride, hq_shard, q_sumsq, k_shard, k_stride, hk_shard, k_sumsq, T,
+                                  dtype, c);
+    if (st != QKN_OK) return st;
+    if ((st = check_launch(c, *launch_cfg)) != QKN_OK) return st;
+    if (T == 0) return ok();
+    return launch<qkn::kStats>(c, *launch_cfg, stream);
 }
 
 qkn_status qknorm_combine_apply(const void *q_in, void *q_out, const void *gamma_q_shard, int64_t q_stride,
@@ -569,42 +630,30 @@ qkn_status qknorm_combine_apply(const void *q_in, void *q_out, const void *gamma
                                 const void *k_in, void *k_out, const void *gamma_k_shard, int64_t k_stride,
                                 int32_t hk_shard, const float *k_sumsq_all, int32_t Hk_full,
                                 int32_t P, int64_t T, float eps, qkn_dtype dtype, void *stream) {
-    if (!dtype_valid(dtype)) return fail(QKN_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
-    if (T < 0) return fail(QKN_ERR_INVALID_ARG, "T = %lld < 0", (long long)T);
-    if (P < 1) return fail(QKN_ERR_INVALID_ARG, "P = %d < 1", P);
-    if (hq_shard <= 0 || hk_shard <= 0) return fail(QKN_ERR_INVALID_ARG, "shard widths must be positive");
-    if (Hq_full < hq_shard || Hk_full < hk_shard) return fail(QKN_ERR_INVALID_ARG, "full width below shard width");
-    if (q_stride < hq_shard || k_stride < hk_shard) return fail(QKN_ERR_INVALID_ARG, "row stride below shard width");
-    if (!eps_valid(eps)) return fail(QKN_ERR_INVALID_ARG, "eps must be finite and >= 0");
-    const int esz = elem_bytes(dtype);
-    if (!extent_ok(T, q_stride, hq_shard, esz) || !extent_ok(T, k_stride, hk_shard, esz) ||
-        !extent_ok(1, 0, (int64_t)P * T, 4))
-        return fail(QKN_ERR_INVALID_ARG, "buffer extent overflows");
-    if (T > 0 && (!q_in || !q_out || !gamma_q_shard || !q_sumsq_all || !k_in || !k_out || !gamma_k_shard ||
-                  !k_sumsq_all))
-        return fail(QKN_ERR_INVALID_ARG, "null pointer");
-    if (T == 0) return ok();
-    const Region iq = rows_region(q_in, hq_shard, q_stride, T, esz), oq = rows_region(q_out, hq_shard, q_stride, T, esz);
-    const Region ik = rows_region(k_in, hk_shard, k_stride, T, esz), ok_ = rows_region(k_out, hk_shard, k_stride, T, esz);
-    const Region others[4] = {flat_region(gamma_q_shard, (int64_t)hq_shard * esz),
-                              flat_region(gamma_k_shard, (int64_t)hk_shard * esz),
-                              flat_region(q_sumsq_all, (int64_t)P * T * 4), flat_region(k_sumsq_all, (int64_t)P * T * 4)};
-    qkn_status st = check_outputs(oq, ok_, iq, ik, others, 4);
-    if (st != QKN_OK) return st;
     Call c;
-    std::memset(&c, 0, sizeof(c));
-    c.dtype = dtype;
-    fill_rowset(c.p.set[0], q_in, q_out, gamma_q_shard, q_stride, hq_shard, Hq_full, esz);
-    fill_rowset(c.p.set[1], k_in, k_out, gamma_k_shard, k_stride, hk_shard, Hk_full, esz);
-    c.p.set[0].sumsq_all = q_sumsq_all;
-    c.p.set[1].sumsq_all = k_sumsq_all;
-    c.p.T = T;
-    c.p.eps = eps;
-    c.p.P = P;
-    finish_call(c, esz, {q_in, q_out, gamma_q_shard, k_in, k_out, gamma_k_shard}, q_stride, k_stride);
+    qkn_status st = prepare_apply(q_in, q_out, gamma_q_shard, q_stride, hq_shard, q_sumsq_all, Hq_full, k_in, k_out,
+                                  gamma_k_shard, k_stride, hk_shard, k_sumsq_all, Hk_full, P, T, eps, dtype, c);
+    if (st != QKN_OK) return st;
+    if (T == 0) return ok();
     qkn_launch L;
     if ((st = plan_call<qkn::kApply>(c, L)) != QKN_OK) return st;
     return launch<qkn::kApply>(c, L, stream);
+}
+
+qkn_status qknorm_combine_apply_launch(const void *q_in, void *q_out, const void *gamma_q_shard, int64_t q_stride,
+                                       int32_t hq_shard, const float *q_sumsq_all, int32_t Hq_full,
+                                       const void *k_in, void *k_out, const void *gamma_k_shard, int64_t k_stride,
+                                       int32_t hk_shard, const float *k_sumsq_all, int32_t Hk_full,
+                                       int32_t P, int64_t T, float eps, qkn_dtype dtype, void *stream,
+                                       const qkn_launch *launch_cfg) {
+    if (!launch_cfg) return fail(QKN_ERR_INVALID_ARG, "null launch");
+    Call c;
+    qkn_status st = prepare_apply(q_in, q_out, gamma_q_shard, q_stride, hq_shard, q_sumsq_all, Hq_full, k_in, k_out,
+                                  gamma_k_shard, k_stride, hk_shard, k_sumsq_all, Hk_full, P, T, eps, dtype, c);
+    if (st != QKN_OK) return st;
+    if ((st = check_launch(c, *launch_cfg)) != QKN_OK) return st;
+    if (T == 0) return ok();
+    return launch<qkn::kApply>(c, *launch_cfg, stream);
 }
 
 const char *qknorm_status_string(qkn_status s) {

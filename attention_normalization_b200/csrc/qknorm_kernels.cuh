@@ -180,6 +180,18 @@ __device__ __forceinline__ float combine_partials(const float *all, int64_t T, i
 }
 
 // r = 1 / sqrt(S / H + eps), the mean formed as S * fl(1 / H).
+// Programmatic dependent launch (sm_90+).  Kernels here are launched with
+// programmatic stream serialization, so their CTAs may be dispatched while the
+// previous kernel in the stream is still draining.  Every kernel therefore
+// first waits until that kernel has completed and its memory operations are
+// visible (a no-op when launched without the attribute), and at once allows
+// the next kernel to be dispatched as its own CTAs retire; that kernel waits
+// for this one's completion in turn.
+__device__ __forceinline__ void pdl_wait_and_release() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ float rms_factor(float sumsq, float inv_div, float eps) {
     return rsqrtf(sumsq * inv_div + eps);
 }
@@ -301,6 +313,7 @@ template <typename E, int NV, int MODE, bool TAIL>
 __global__ void __launch_bounds__(RegisterBounds<NV>::kMaxThreads)
     rows_register_kernel(const __grid_constant__ Params p) {
     __shared__ float red[2][32];
+    pdl_wait_and_release();
     int slot = 0;
     const int tid = threadIdx.x;
     const int lane = tid & 31;
@@ -411,6 +424,7 @@ template <typename E, bool VEC, int MODE>
 __global__ void __launch_bounds__(1024) rows_twopass_kernel(const __grid_constant__ Params p) {
     using Pk = Pack<E>;
     __shared__ float red[2][32];
+    pdl_wait_and_release();
     int slot = 0;
     const int tid = threadIdx.x;
     const int nthr = blockDim.x;

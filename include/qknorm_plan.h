@@ -110,6 +110,21 @@ qkn_status qknorm_layerwise_launch(const void *q_in, void *q_out, const void *ga
                                    int64_t T, int32_t Hq, int32_t Hk, float eps, qkn_dtype dtype,
                                    void *stream, const qkn_launch *launch);
 
+/*
+ * qknorm_partial_stats / qknorm_combine_apply with a caller-chosen launch;
+ * the same launch rules and checks as qknorm_layerwise_launch apply.
+ */
+qkn_status qknorm_partial_stats_launch(const void *q_shard, int64_t q_stride, int32_t hq_shard, float *q_sumsq,
+                                       const void *k_shard, int64_t k_stride, int32_t hk_shard, float *k_sumsq,
+                                       int64_t T, qkn_dtype dtype, void *stream, const qkn_launch *launch);
+
+qkn_status qknorm_combine_apply_launch(const void *q_in, void *q_out, const void *gamma_q_shard, int64_t q_stride,
+                                       int32_t hq_shard, const float *q_sumsq_all, int32_t Hq_full,
+                                       const void *k_in, void *k_out, const void *gamma_k_shard, int64_t k_stride,
+                                       int32_t hk_shard, const float *k_sumsq_all, int32_t Hk_full,
+                                       int32_t P, int64_t T, float eps, qkn_dtype dtype, void *stream,
+                                       const qkn_launch *launch);
+
 #ifdef __cplusplus
 }
 #endif

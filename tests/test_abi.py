@@ -201,6 +201,24 @@ def test_launch_override_validation(lib):
     assert st(2, 0, 128, 1, a=unaligned) == OK
 
 
+def test_shard_launch_override_validation(lib):
+    T = 16384
+    stats = [BASE, 1280, 1280, BASE + (1 << 28), BASE + (2 << 28), 256, 256, BASE + (3 << 28), T, BF16, None]
+    apply = [BASE, BASE, BASE + (1 << 28), 1280, 1280, BASE + (2 << 28), 5120,
+             BASE + (3 << 28), BASE + (3 << 28), BASE + (4 << 28), 256, 256, BASE + (5 << 28), 1024,
+             4, T, 1e-6, BF16, None]
+    for f, args in ((lib.qknorm_partial_stats_launch, stats), (lib.qknorm_combine_apply_launch, apply)):
+        zero = list(args)
+        zero[8 if f is lib.qknorm_partial_stats_launch else 15] = 0  # T = 0: validated, nothing launched
+        assert f(*zero, ctypes.byref(_clib.QknLaunch(0, 2, 96, 10))) == OK
+        assert f(*zero, ctypes.byref(_clib.QknLaunch(0, 1, 96, 10))) == INVALID  # 96 < 160 vectors
+        assert f(*zero, ctypes.byref(_clib.QknLaunch(0, 2, 100, 10))) == INVALID
+        assert f(*zero, None) == INVALID
+        bad = list(args)
+        bad[1 if f is lib.qknorm_partial_stats_launch else 3] = 1279  # stride below width
+        assert f(*bad, ctypes.byref(_clib.QknLaunch(0, 2, 96, 10))) == INVALID
+
+
 # --------------------------------------------------------------------------- overlap
 
 def _brute(a, b):

@@ -277,6 +277,59 @@ def test_register_kernel_in_place_on_packed_rows_any_grid(T):
     assert torch.equal(base[:, b.Hq + b.Hk:], before[:, b.Hq + b.Hk:])
 
 
+SHARD_LAUNCHES = [
+    None,
+    {"kernel": 0, "vec_per_thread": 1, "threads": 160, "grid": 50},
+    {"kernel": 0, "vec_per_thread": 2, "threads": 96, "grid": 7},
+    {"kernel": 0, "vec_per_thread": 4, "threads": 128, "grid": 148},
+    {"kernel": 0, "vec_per_thread": 8, "threads": 128, "grid": 3},
+    {"kernel": 0, "vec_per_thread": 8, "threads": 32, "grid": 1},
+    {"kernel": 1, "vec_per_thread": 0, "threads": 64, "grid": 9},
+    {"kernel": 2, "vec_per_thread": 0, "threads": 256, "grid": 11},
+]
+
+
+@pytest.mark.parametrize("launch", SHARD_LAUNCHES, ids=lambda L: "default" if L is None else
+                         "k{kernel}_nv{vec_per_thread}_t{threads}_g{grid}".format(**L))
+@pytest.mark.parametrize("dtype,Hq,Hk,P", [(torch.bfloat16, 5120, 1024, 4), (torch.float32, 1200, 260, 4),
+                                           (torch.bfloat16, 1000, 200, 5)])
+def test_shard_pipeline_launch_variants(launch, dtype, Hq, Hk, P):
+    """partial_stats then combine_apply over P shards, each with a pinned
+    launch, against the oracle's full-row normalization."""
+    per = 4 if dtype == torch.float32 else 8
+    wq, wk = Hq // P, Hk // P
+    if launch is not None and launch["kernel"] == 0 and launch["vec_per_thread"] * launch["threads"] < -(-wq // per):
+        pytest.skip("launch does not cover a shard row")
+    if launch is not None and launch["kernel"] in (0, 1) and ((wq * (4 if dtype == torch.float32 else 2)) % 16
+                                                             or (wk * (4 if dtype == torch.float32 else 2)) % 16):
+        pytest.skip("vector kernels need 16-byte aligned shard strides")
+    T = 131
+    g = torch.Generator().manual_seed(Hq + Hk + P)
+    q = (torch.randn((T, Hq), generator=g) * 2).to(dtype)
+    k = (torch.randn((T, Hk), generator=g) * 0.5).to(dtype)
+    gq = workloads.gamma(Hq, 5, dtype)
+    gk = workloads.gamma(Hk, 6, dtype)
+    qs = [q[:, i * wq:(i + 1) * wq].contiguous().to(DEV) for i in range(P)]
+    ks = [k[:, i * wk:(i + 1) * wk].contiguous().to(DEV) for i in range(P)]
+    q_all = torch.empty((P, T), dtype=torch.float32, device=DEV)
+    k_all = torch.empty((P, T), dtype=torch.float32, device=DEV)
+    for i in range(P):
+        qk.qknorm_partial_stats(qs[i], ks[i], q_all[i], k_all[i], launch=launch)
+    outs = [qk.qknorm_combine_apply(qs[i], ks[i], gq[i * wq:(i + 1) * wq].contiguous().to(DEV),
+                                    gk[i * wk:(i + 1) * wk].contiguous().to(DEV), q_all, k_all, Hq, Hk, 1e-6,
+                                    launch=launch) for i in range(P)]
+    torch.cuda.synchronize()
+    for i in range(P):
+        np.testing.assert_allclose(q_all[i].cpu().double().numpy(),
+                                   oracle.partial_sumsq(to_np(q[:, i * wq:(i + 1) * wq]), wq, wq, T), rtol=1e-5)
+        np.testing.assert_allclose(k_all[i].cpu().double().numpy(),
+                                   oracle.partial_sumsq(to_np(k[:, i * wk:(i + 1) * wk]), wk, wk, T), rtol=1e-5)
+    yq, eq, _ = oracle_rows(q, gq, 1e-6)
+    yk, ek, _ = oracle_rows(k, gk, 1e-6)
+    assert_close(torch.cat([o[0] for o in outs], dim=1), yq, eq, "shards Q")
+    assert_close(torch.cat([o[1] for o in outs], dim=1), yk, ek, "shards K")
+
+
 def test_fp32_variants_and_apply_with_one_shard_equals_fused():
     b = workloads.tiny_fp32()
     q, k = b.q.to(DEV), b.k.to(DEV)
