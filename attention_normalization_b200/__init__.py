@@ -25,8 +25,8 @@ from . import _clib
 from ._clib import QknLaunch, QKNormError
 
 __all__ = ["qknorm_layerwise", "qknorm_partial_stats", "qknorm_combine_apply",
-           "qknorm_layerwise_plan", "plan_shape", "plan_grid", "regions_overlap",
-           "capi", "version", "QknLaunch", "QKNormError"]
+           "qknorm_layerwise_plan", "qknorm_layerwise_host", "qknorm_packed_host",
+           "plan_shape", "plan_grid", "regions_overlap", "capi", "version", "QknLaunch", "QKNormError"]
 
 _DTYPES = {torch.float32: _clib.QKN_F32, torch.bfloat16: _clib.QKN_BF16}
 
@@ -230,3 +230,6 @@ def plan_grid(rows: int, blocks_per_sm: int, sm_count: int) -> int:
 def regions_overlap(a: tuple, b: tuple) -> bool:
     """``a`` and ``b`` are ``(base, width_bytes, stride_bytes, rows)``."""
     return bool(capi().qknorm_regions_overlap(*a, *b))
+
+
+from .host_pipeline import qknorm_layerwise_host, qknorm_packed_host  # noqa: E402  (uses qknorm_layerwise)

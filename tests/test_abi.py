@@ -315,3 +315,14 @@ def test_binding_refuses_cpu_tensors():
         qk.qknorm_layerwise(x, x, g, g)
     with pytest.raises(ValueError, match="CUDA"):
         qk.qknorm_partial_stats(x, x)
+
+
+def test_host_pipeline_argument_checks():
+    x = torch.zeros((4, 8), dtype=torch.float32)
+    g = torch.ones((8,), dtype=torch.float32)
+    with pytest.raises(ValueError, match="same number of tokens"):
+        qk.qknorm_layerwise_host(x, torch.zeros((5, 8)), g, g)
+    with pytest.raises(ValueError, match="chunk_tokens"):
+        qk.qknorm_layerwise_host(x, x, g, g, chunk_tokens=0)
+    with pytest.raises(ValueError, match="inside the packed row"):
+        qk.qknorm_packed_host(torch.zeros((4, 16)), 0, 8, 8, 9, g, g)

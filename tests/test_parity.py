@@ -364,3 +364,39 @@ def test_invalid_call_on_gpu_raises_and_launches_nothing():
     big = torch.zeros((4, 128), dtype=torch.bfloat16, device=DEV)
     with pytest.raises(qk.QKNormError, match="overlap"):
         qk.qknorm_layerwise(big[:, :64], big[:, 32:96], g, g, q_out=big[:, :64], k_out=big[:, 32:96])
+
+
+# --------------------------------------------------------------------------- host pipeline
+
+@pytest.mark.parametrize("T,chunk", [(1, 512), (1000, 512), (1537, 256), (64, 7)])
+def test_host_pipeline_matches_the_oracle(T, chunk):
+    b = workloads.random_rows(T, 2048, 512, torch.bfloat16, seed=T + chunk)
+    hq, hk = b.q.contiguous().pin_memory(), b.k.contiguous().pin_memory()
+    qo, ko = qk.qknorm_layerwise_host(hq, hk, b.gamma_q, b.gamma_k, b.eps, chunk_tokens=chunk)
+    torch.cuda.current_stream().synchronize()
+    assert not qo.is_cuda and not ko.is_cuda
+    yq, eq, _ = oracle_rows(b.q, b.gamma_q, b.eps)
+    yk, ek, _ = oracle_rows(b.k, b.gamma_k, b.eps)
+    assert_close(qo, yq, eq, "host pipeline Q")
+    assert_close(ko, yk, ek, "host pipeline K")
+    # in place on the host buffers, fp32
+    bf = workloads.random_rows(T, 512, 96, torch.float32, seed=T)
+    hq2, hk2 = bf.q.contiguous().pin_memory(), bf.k.contiguous().pin_memory()
+    qk.qknorm_layerwise_host(hq2, hk2, bf.gamma_q, bf.gamma_k, bf.eps, q_out=hq2, k_out=hk2, chunk_tokens=chunk)
+    torch.cuda.current_stream().synchronize()
+    yq, eq, _ = oracle_rows(bf.q, bf.gamma_q, bf.eps)
+    assert_close(hq2, yq, eq, "host pipeline in place Q")
+
+
+@pytest.mark.parametrize("T", [3, 1500])
+def test_packed_host_pipeline_leaves_v_untouched(T):
+    b = workloads.packed_qkv(T)
+    host = b.packed.clone().pin_memory()
+    qk.qknorm_packed_host(host, 0, b.Hq, b.Hq, b.Hk, b.gamma_q, b.gamma_k, b.eps, chunk_tokens=512)
+    torch.cuda.current_stream().synchronize()
+    v0 = b.Hq + b.Hk
+    assert torch.equal(host[:, v0:], b.packed[:, v0:])
+    yq, eq, _ = oracle_rows(b.q, b.gamma_q, b.eps)
+    yk, ek, _ = oracle_rows(b.k, b.gamma_k, b.eps)
+    assert_close(host[:, :b.Hq], yq, eq, "packed host Q")
+    assert_close(host[:, b.Hq:v0], yk, ek, "packed host K")
