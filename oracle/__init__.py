@@ -15,8 +15,9 @@ This module only marshals numpy arrays into the plain C oracle
   weight multiplication and global RMS scaling of one shard.
 * ``bf16_decode`` / ``bf16_encode`` — the element codec.
 
-Arrays: fp32 data is passed as ``np.float32``; bfloat16 data is passed as its
-raw bit patterns in ``np.uint16``.  A 2-D input ``x`` of shape ``(T, stride)``
+Arrays: fp32 data is passed as ``np.float32``, IEEE half as ``np.float16``,
+bfloat16 as its raw bit patterns in ``np.uint16`` and FP8 E4M3 ("fn") as its
+raw bit patterns in ``np.uint8`` (with E4M3 data, gamma is bfloat16 bits).  A 2-D input ``x`` of shape ``(T, stride)``
 (or any C-contiguous array whose rows are ``stride`` elements apart) holds row
 ``t`` at element ``t * stride``; only its first ``H`` columns are read.
 """
@@ -31,6 +32,8 @@ from . import build as _build
 
 F32 = 0
 BF16 = 1
+F16 = 2
+E4M3 = 3
 
 _lib = None
 
@@ -49,6 +52,14 @@ def _load():
     lib.oracle_bf16_decode.restype = dbl
     lib.oracle_bf16_encode_rne.argtypes = [dbl]
     lib.oracle_bf16_encode_rne.restype = ctypes.c_uint16
+    lib.oracle_f16_decode.argtypes = [ctypes.c_uint16]
+    lib.oracle_f16_decode.restype = dbl
+    lib.oracle_f16_encode_rne.argtypes = [dbl]
+    lib.oracle_f16_encode_rne.restype = ctypes.c_uint16
+    lib.oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
+    lib.oracle_e4m3_decode.restype = dbl
+    lib.oracle_e4m3_encode_rne_sat.argtypes = [dbl]
+    lib.oracle_e4m3_encode_rne_sat.restype = ctypes.c_uint8
     lib.oracle_rmsnorm_rows.argtypes = [vp, i64, i64, i32, vp, dbl, ctypes.c_int,
                                         vp, i64, vp, vp]
     lib.oracle_rmsnorm_rows.restype = ctypes.c_int
@@ -69,7 +80,17 @@ def _dtype_code(arr: np.ndarray) -> int:
         return F32
     if arr.dtype == np.uint16:
         return BF16
-    raise TypeError(f"oracle takes float32 or uint16 (bfloat16 bits), got {arr.dtype}")
+    if arr.dtype == np.float16:
+        return F16
+    if arr.dtype == np.uint8:
+        return E4M3
+    raise TypeError(f"oracle takes float32, float16, uint16 (bfloat16 bits) or uint8 (E4M3 bits), "
+                    f"got {arr.dtype}")
+
+
+def _gamma_dtype(x_dtype):
+    """gamma has the element type of x, except bfloat16 bits with E4M3 data."""
+    return np.dtype(np.uint16) if x_dtype == np.uint8 else x_dtype
 
 
 def _ptr(arr):
@@ -97,6 +118,31 @@ def bf16_encode(values) -> np.ndarray:
                     dtype=np.uint16).reshape(v.shape)
 
 
+def f16_decode(bits) -> np.ndarray:
+    lib = _load()
+    b = np.asarray(bits, dtype=np.uint16)
+    return np.array([lib.oracle_f16_decode(int(v)) for v in b.ravel()], dtype=np.float64).reshape(b.shape)
+
+
+def f16_encode(values) -> np.ndarray:
+    """Bit patterns (uint16) of the IEEE half values nearest to `values`."""
+    lib = _load()
+    v = np.asarray(values, dtype=np.float64)
+    return np.array([lib.oracle_f16_encode_rne(float(a)) for a in v.ravel()], dtype=np.uint16).reshape(v.shape)
+
+
+def e4m3_decode(bits) -> np.ndarray:
+    lib = _load()
+    b = np.asarray(bits, dtype=np.uint8)
+    return np.array([lib.oracle_e4m3_decode(int(v)) for v in b.ravel()], dtype=np.float64).reshape(b.shape)
+
+
+def e4m3_encode(values) -> np.ndarray:
+    lib = _load()
+    v = np.asarray(values, dtype=np.float64)
+    return np.array([lib.oracle_e4m3_encode_rne_sat(float(a)) for a in v.ravel()], dtype=np.uint8).reshape(v.shape)
+
+
 def rmsnorm_rows(x: np.ndarray, H: int, gamma: np.ndarray, eps: float,
                  stride: int | None = None, T: int | None = None):
     """RMS-Norm of rows of width ``H``.
@@ -113,8 +159,8 @@ def rmsnorm_rows(x: np.ndarray, H: int, gamma: np.ndarray, eps: float,
         T = x.size // stride if x.ndim == 1 else int(np.prod(x.shape[:-1])) * x.shape[-1] // stride
     _check_rows(x, stride, T, H)
     g = np.ascontiguousarray(gamma)
-    if g.dtype != x.dtype or g.size < H:
-        raise ValueError("gamma must have the input's element type and at least H elements")
+    if g.dtype != _gamma_dtype(x.dtype) or g.size < H:
+        raise ValueError("gamma must have the gamma type of the input and at least H elements")
     y = np.zeros((T, H), dtype=x.dtype)
     y_exact = np.zeros((T, H), dtype=np.float64)
     sumsq = np.zeros((T,), dtype=np.float64)
@@ -182,5 +228,6 @@ def version() -> int:
     return _load().oracle_version()
 
 
-__all__ = ["F32", "BF16", "bf16_decode", "bf16_encode", "rmsnorm_rows", "qknorm_layerwise",
-           "partial_sumsq", "combine_apply", "version"]
+__all__ = ["F32", "BF16", "F16", "E4M3", "bf16_decode", "bf16_encode", "f16_decode", "f16_encode",
+           "e4m3_decode", "e4m3_encode", "rmsnorm_rows", "qknorm_layerwise", "partial_sumsq",
+           "combine_apply", "version"]

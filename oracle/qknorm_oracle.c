@@ -19,11 +19,22 @@
  *   - Evaluation, Fig. 2(b): the accuracy reference is RMSNorm in FP64 over the
  *     full vector.  This file is that reference.
  *
- * Element types: dtype 0 = IEEE binary32, dtype 1 = bfloat16 (1 sign bit,
- * 8 exponent bits with bias 127, 7 stored mantissa bits).  Inputs are decoded
- * exactly into double; all arithmetic is in double in plain left-to-right
- * order; an output of a narrow type is produced by one correctly rounded
- * (round-to-nearest, ties-to-even) conversion from the double result.
+ * Element types:
+ *   dtype 0 = IEEE binary32;
+ *   dtype 1 = bfloat16 (1 sign bit, 8 exponent bits with bias 127, 7 stored
+ *             mantissa bits);
+ *   dtype 2 = IEEE binary16 (1 sign, 5 exponent bits with bias 15, 10 stored
+ *             mantissa bits);
+ *   dtype 3 = FP8 E4M3 in its "fn" form (1 sign, 4 exponent bits with bias 7,
+ *             3 stored mantissa bits; no infinities; exponent 15 with mantissa
+ *             7 is NaN, so the largest finite value is 1.75 * 2^8 = 448).
+ *             With dtype 3 the gamma vector is bfloat16 (an E4M3 gamma near 1
+ *             would be spaced 0.125 apart); x and y are E4M3.
+ * Inputs are decoded exactly into double; all arithmetic is in double in
+ * plain left-to-right order; an output of a narrow type is produced by one
+ * correctly rounded (round-to-nearest, ties-to-even) conversion from the
+ * double result.  E4M3 outputs beyond the finite range saturate to +-448
+ * (the reading taken for an 8-bit format without infinities).
  *
  * Build: gcc -O2 -std=c11 -fno-fast-math -ffp-contract=off -shared -fPIC -lm
  * (FMA contraction is disabled so every product and sum is rounded on its own.)
@@ -34,6 +45,8 @@
 
 #define ORACLE_F32 0
 #define ORACLE_BF16 1
+#define ORACLE_F16 2
+#define ORACLE_E4M3 3
 
 #define ORACLE_OK 0
 #define ORACLE_BAD_ARG 1
@@ -100,30 +113,133 @@ uint16_t oracle_bf16_encode_rne(double y)
     return sign | (uint16_t)((expo << 7) | (int)frac);
 }
 
+/* binary16 bit pattern -> exact double, from the field definition. */
+double oracle_f16_decode(uint16_t b)
+{
+    int sign = (b >> 15) & 1;
+    int expo = (b >> 10) & 0x1F;
+    int mant = b & 0x3FF;
+    double v;
+    if (expo == 0x1F)
+        v = mant ? NAN : INFINITY;
+    else if (expo == 0)
+        v = ldexp((double)mant, -24);                 /* 0.mant * 2^-14 */
+    else
+        v = ldexp((double)(1024 + mant), expo - 25);  /* 1.mant * 2^(expo-15) */
+    return sign ? -v : v;
+}
+
+/* E4M3 ("fn") bit pattern -> exact double, from the field definition. */
+double oracle_e4m3_decode(uint8_t b)
+{
+    int sign = (b >> 7) & 1;
+    int expo = (b >> 3) & 0xF;
+    int mant = b & 0x7;
+    double v;
+    if (expo == 0xF && mant == 0x7)
+        v = NAN;
+    else if (expo == 0)
+        v = ldexp((double)mant, -9);                  /* 0.mant * 2^-6 */
+    else
+        v = ldexp((double)(8 + mant), expo - 10);     /* 1.mant * 2^(expo-7) */
+    return sign ? -v : v;
+}
+
+/*
+ * |y| rounded to nearest, ties to even, onto the grid of a binary format with
+ * `sig` significant bits whose smallest normal exponent is `emin`: spacing
+ * 2^(E - sig + 1) for |y| in [2^E, 2^(E+1)), never finer than the subnormal
+ * spacing 2^(emin - sig + 1).  Exact scaling by powers of two, nearbyint in
+ * the default (to-nearest-even) mode.  a > 0 and finite.
+ */
+static double round_to_grid(double a, int sig, int emin)
+{
+    int e;
+    (void)frexp(a, &e);               /* a = m * 2^e, m in [0.5, 1) */
+    int q = (e - 1) - (sig - 1);
+    if (q < emin - (sig - 1))
+        q = emin - (sig - 1);
+    return ldexp(nearbyint(ldexp(a, -q)), q);
+}
+
+/* double -> binary16, one rounding (RNE); beyond the largest finite value
+ * (65504) the rounded result is infinity. */
+uint16_t oracle_f16_encode_rne(double y)
+{
+    if (isnan(y))
+        return 0x7E00;
+    uint16_t sign = signbit(y) ? 0x8000 : 0;
+    double a = fabs(y);
+    if (isinf(a))
+        return sign | 0x7C00;
+    if (a == 0.0)
+        return sign;
+    double r = round_to_grid(a, 11, -14);
+    if (r >= 65536.0)
+        return sign | 0x7C00;
+    if (r < 0x1p-14)
+        return sign | (uint16_t)lrint(ldexp(r, 24));  /* subnormal */
+    int er;
+    double m = frexp(r, &er);
+    return sign | (uint16_t)(((er - 1 + 15) << 10) | (int)(lrint(ldexp(m, 11)) - 1024));
+}
+
+/* double -> E4M3 ("fn"), one rounding (RNE), saturating to +-448; NaN -> 0x7F. */
+uint8_t oracle_e4m3_encode_rne_sat(double y)
+{
+    if (isnan(y))
+        return 0x7F;
+    uint8_t sign = signbit(y) ? 0x80 : 0;
+    double a = fabs(y);
+    if (a == 0.0)
+        return sign;
+    double r = isinf(a) ? 448.0 : round_to_grid(a, 4, -6);
+    if (r > 448.0)
+        r = 448.0;
+    if (r < 0x1p-6)
+        return sign | (uint8_t)lrint(ldexp(r, 9));    /* subnormal */
+    int er;
+    double m = frexp(r, &er);
+    return sign | (uint8_t)(((er - 1 + 7) << 3) | (int)(lrint(ldexp(m, 4)) - 8));
+}
+
+static int elem_size(int dtype) { return dtype == ORACLE_F32 ? 4 : (dtype == ORACLE_E4M3 ? 1 : 2); }
+
+/* gamma is stored in the element type, except with E4M3 data, where it is bfloat16 */
+static int gamma_dtype(int dtype) { return dtype == ORACLE_E4M3 ? ORACLE_BF16 : dtype; }
+
 static double load_elem(const void *base, int dtype, int64_t idx)
 {
+    const char *p = (const char *)base + idx * elem_size(dtype);
     if (dtype == ORACLE_F32) {
         float f;
-        memcpy(&f, (const char *)base + idx * 4, 4);
+        memcpy(&f, p, 4);
         return (double)f;
     }
+    if (dtype == ORACLE_E4M3)
+        return oracle_e4m3_decode(*(const uint8_t *)p);
     uint16_t b;
-    memcpy(&b, (const char *)base + idx * 2, 2);
-    return oracle_bf16_decode(b);
+    memcpy(&b, p, 2);
+    return dtype == ORACLE_F16 ? oracle_f16_decode(b) : oracle_bf16_decode(b);
 }
 
 static void store_elem(void *base, int dtype, int64_t idx, double v)
 {
+    char *p = (char *)base + idx * elem_size(dtype);
     if (dtype == ORACLE_F32) {
         float f = (float)v;      /* C conversion: round to nearest, ties to even */
-        memcpy((char *)base + idx * 4, &f, 4);
+        memcpy(p, &f, 4);
         return;
     }
-    uint16_t b = oracle_bf16_encode_rne(v);
-    memcpy((char *)base + idx * 2, &b, 2);
+    if (dtype == ORACLE_E4M3) {
+        *(uint8_t *)p = oracle_e4m3_encode_rne_sat(v);
+        return;
+    }
+    uint16_t b = dtype == ORACLE_F16 ? oracle_f16_encode_rne(v) : oracle_bf16_encode_rne(v);
+    memcpy(p, &b, 2);
 }
 
-static int bad_dtype(int dtype) { return dtype != ORACLE_F32 && dtype != ORACLE_BF16; }
+static int bad_dtype(int dtype) { return dtype < ORACLE_F32 || dtype > ORACLE_E4M3; }
 
 /*
  * RMS-Norm of T rows of width H (Background, Equation 1):
@@ -152,7 +268,7 @@ int oracle_rmsnorm_rows(const void *x, int64_t x_stride, int64_t T, int32_t H,
         double r = 1.0 / sqrt(S / (double)H + eps);
         for (int32_t j = 0; j < H; ++j) {
             double v = load_elem(x, dtype, t * x_stride + j);
-            double g = load_elem(gamma, dtype, j);
+            double g = load_elem(gamma, gamma_dtype(dtype), j);
             double yv = (v * g) * r;
             if (y_exact)
                 y_exact[t * (int64_t)H + j] = yv;
@@ -229,7 +345,7 @@ int oracle_combine_apply(const void *x, int64_t x_stride, int64_t T, int32_t h_s
         double r = 1.0 / sqrt(S / (double)H_full + eps);
         for (int32_t j = 0; j < h_shard; ++j) {
             double v = load_elem(x, dtype, t * x_stride + j);
-            double g = load_elem(gamma_shard, dtype, j);
+            double g = load_elem(gamma_shard, gamma_dtype(dtype), j);
             double yv = (v * g) * r;
             if (y_exact)
                 y_exact[t * (int64_t)h_shard + j] = yv;

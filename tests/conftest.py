@@ -21,14 +21,17 @@ def pytest_collection_modifyitems(config, items):
 
 
 def to_np(t: torch.Tensor) -> np.ndarray:
-    """CPU tensor -> numpy array in the oracle's convention (bf16 as uint16 bits).
+    """CPU tensor -> numpy array in the oracle's convention (bf16 as uint16
+    bits, E4M3 as uint8 bits).
     The tensor is made contiguous first; a strided view keeps its values, not
     its layout."""
     t = t.detach().cpu().contiguous()
     if t.dtype == torch.bfloat16:
         return t.view(torch.int16).numpy().view(np.uint16)
-    if t.dtype == torch.float32:
+    if t.dtype in (torch.float32, torch.float16):
         return t.numpy()
+    if t.dtype == torch.float8_e4m3fn:
+        return t.view(torch.uint8).numpy()
     raise TypeError(f"unsupported dtype {t.dtype}")
 
 
@@ -54,3 +57,25 @@ def bf16_bits_to_ordered(bits: np.ndarray) -> np.ndarray:
 
 def bf16_ulp_distance(a_bits: np.ndarray, b_bits: np.ndarray) -> np.ndarray:
     return np.abs(bf16_bits_to_ordered(a_bits) - bf16_bits_to_ordered(b_bits))
+
+
+def ordered_bits(bits: np.ndarray, nbits: int) -> np.ndarray:
+    """Sign-magnitude bit patterns of an `nbits`-wide float format -> integers
+    whose difference counts representable values between two numbers (+0 and
+    -0 coincide)."""
+    b = bits.astype(np.int64)
+    sign = 1 << (nbits - 1)
+    mag = b & (sign - 1)
+    return np.where(b & sign, -mag, mag)
+
+
+def ulp_distance(a: np.ndarray, b: np.ndarray, dtype: torch.dtype) -> np.ndarray:
+    """Distance in units of the last place between two arrays of the same
+    narrow float type, given as the oracle's numpy arrays."""
+    if dtype == torch.bfloat16:
+        return np.abs(ordered_bits(a, 16) - ordered_bits(b, 16))
+    if dtype == torch.float16:
+        return np.abs(ordered_bits(a.view(np.uint16), 16) - ordered_bits(b.view(np.uint16), 16))
+    if dtype == torch.float8_e4m3fn:
+        return np.abs(ordered_bits(a, 8) - ordered_bits(b, 8))
+    raise TypeError(f"no ulp distance for {dtype}")

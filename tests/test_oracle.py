@@ -7,8 +7,8 @@ compared with it, it is checked here against:
 
 * hand-derived closed forms (``tests/golden/closed_forms.json``);
 * a library routine that computes the same definition
-  (``torch.nn.functional.rms_norm`` in float64) and torch's own float32 ->
-  bfloat16 rounding;
+  (``torch.nn.functional.rms_norm`` in float64) and torch's own conversions
+  between float32 and bfloat16, float16 and float8_e4m3fn (within its range);
 * invariants the mathematics fixes (output RMS with gamma = 1, scale
   invariance, one-hot and power-of-two gamma, the shard-sum identity).
 
@@ -87,6 +87,49 @@ def test_bf16_decode_matches_torch_for_every_finite_pattern():
     assert np.array_equal(np.isnan(got), np.isnan(vals))
 
 
+def test_f16_and_e4m3_fixtures():
+    g = _golden()
+    for case in g["f16_encode_rne"]:
+        got = int(oracle.f16_encode([_parse_value(case["value"])])[0])
+        assert got == int(case["bits"], 16), (case, hex(got))
+    for case in g["e4m3_decode"]:
+        assert oracle.e4m3_decode([int(case["bits"], 16)])[0] == case["value"], case
+    for case in g["e4m3_encode_rne_sat"]:
+        got = int(oracle.e4m3_encode([_parse_value(case["value"])])[0])
+        assert got == int(case["bits"], 16), (case, hex(got))
+
+
+def test_f16_codec_matches_torch():
+    bits = np.arange(0, 1 << 16, dtype=np.uint32).astype(np.uint16)
+    vals = torch.from_numpy(bits.view(np.int16).copy()).view(torch.float16).double().numpy()
+    got = oracle.f16_decode(bits)
+    fin = np.isfinite(vals)
+    assert np.array_equal(got[fin], vals[fin]) and np.array_equal(np.isinf(got), np.isinf(vals))
+    g = torch.Generator().manual_seed(12)
+    f = torch.randn((20000,), generator=g) * torch.exp(torch.randn((20000,), generator=g) * 4)
+    ties = (torch.from_numpy(bits[(bits & 0x7C00) != 0x7C00].astype(np.int16)).view(torch.float16).float()
+            * (1 + 2.0 ** -11))  # exact halfway points between neighbouring halves
+    f = torch.cat([f, ties[torch.isfinite(ties)]])
+    want = f.to(torch.float16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(oracle.f16_encode(f.double().numpy()), want)
+
+
+def test_e4m3_codec_matches_torch_within_range():
+    bits = np.arange(256, dtype=np.uint8)
+    vals = torch.from_numpy(bits.copy()).view(torch.float8_e4m3fn).double().numpy()
+    got = oracle.e4m3_decode(bits)
+    fin = np.isfinite(vals)
+    assert np.array_equal(got[fin], vals[fin]) and np.array_equal(np.isnan(got), np.isnan(vals))
+    g = torch.Generator().manual_seed(13)
+    f = torch.randn((20000,), generator=g) * torch.exp(torch.randn((20000,), generator=g) * 3)
+    f = f[f.abs() <= 448]
+    pos = np.sort(np.unique(np.abs(vals[fin])))  # midpoints between neighbours are exact ties
+    mids = torch.from_numpy((pos[:-1] + pos[1:]) / 2).float()
+    f = torch.cat([f, mids, -mids])
+    want = f.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(oracle.e4m3_encode(f.double().numpy()), want)
+
+
 # --------------------------------------------------------------------------- closed forms
 
 def test_rmsnorm_closed_forms():
@@ -121,14 +164,15 @@ def test_sharded_closed_form_divides_by_full_width():
 
 # --------------------------------------------------------------------------- library routine
 
-@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16, torch.float16, torch.float8_e4m3fn])
 @pytest.mark.parametrize("T,H,pad", [(1, 1, 0), (3, 7, 5), (17, 64, 3), (9, 513, 0), (4, 4096, 8)])
 def test_rmsnorm_matches_torch_rms_norm_float64(dtype, T, H, pad):
     g = torch.Generator().manual_seed(1000 + T * 7 + H)
     stride = H + pad
     buf = (torch.randn((T, stride), generator=g) * 3.0).to(dtype)
     view = buf[:, :H]
-    gm = (1.0 + 0.1 * torch.randn((H,), generator=g)).to(dtype)
+    gdt = torch.bfloat16 if dtype == torch.float8_e4m3fn else dtype
+    gm = (1.0 + 0.1 * torch.randn((H,), generator=g)).to(gdt)
     eps = 1e-6
     flat, st = buffer_np(view)
     y_rounded, y, s = oracle.rmsnorm_rows(flat, H, to_np(gm), eps, stride=st, T=T)
@@ -138,8 +182,12 @@ def test_rmsnorm_matches_torch_rms_norm_float64(dtype, T, H, pad):
     # the stored output is one correct rounding of the double result
     if dtype == torch.float32:
         assert np.array_equal(y_rounded, y.astype(np.float32))
-    else:
+    elif dtype == torch.bfloat16:
         assert np.array_equal(y_rounded, oracle.bf16_encode(y))
+    elif dtype == torch.float16:
+        assert np.array_equal(y_rounded.view(np.uint16), oracle.f16_encode(y))
+    else:
+        assert np.array_equal(y_rounded, oracle.e4m3_encode(y))
 
 
 def test_layerwise_treats_q_and_k_independently():

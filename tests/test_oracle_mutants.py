@@ -26,7 +26,14 @@ MUTANTS = [
     ("exponent_bias_off_by_one", "expo - 134", "expo - 133", None),
     ("truncate_not_rne", "double n = nearbyint(ldexp(a, -q));", "double n = trunc(ldexp(a, -q));", None),
     ("round_half_away", "double n = nearbyint(ldexp(a, -q));", "double n = round(ldexp(a, -q));", None),
-    ("gamma_indexed_by_token", "double g = load_elem(gamma, dtype, j);", "double g = load_elem(gamma, dtype, t);", None),
+    ("gamma_indexed_by_token", "double g = load_elem(gamma, gamma_dtype(dtype), j);",
+     "double g = load_elem(gamma, gamma_dtype(dtype), t);", None),
+    ("e4m3_exponent_bias", "ldexp((double)(8 + mant), expo - 10)", "ldexp((double)(8 + mant), expo - 9)", None),
+    ("e4m3_no_saturation", "    if (r > 448.0)\n        r = 448.0;\n", "", None),
+    ("f16_subnormal_scale", "ldexp((double)mant, -24);", "ldexp((double)mant, -25);", None),
+    ("f16_encode_bias", "((er - 1 + 15) << 10)", "((er - 1 + 14) << 10)", None),
+    ("f16_subnormal_threshold", "round_to_grid(a, 11, -14)", "round_to_grid(a, 11, -15)", None),
+    ("gamma_type_e4m3", "return dtype == ORACLE_E4M3 ? ORACLE_BF16 : dtype;", "return dtype;", None),
     ("stride_ignored", "double v = load_elem(x, dtype, t * x_stride + j);\n            double g",
      "double v = load_elem(x, dtype, t * (int64_t)H + j);\n            double g", 1),
     ("drop_last_shard", "for (int32_t p = 0; p < P; ++p)", "for (int32_t p = 0; p + 1 < P; ++p)", None),
