@@ -24,11 +24,17 @@ import torch
 from . import _clib
 from ._clib import QknLaunch, QKNormError
 
-__all__ = ["qknorm_layerwise", "qknorm_partial_stats", "qknorm_combine_apply",
+__all__ = ["qknorm_layerwise", "qknorm_partial_stats", "qknorm_combine_apply", "gamma_dtype",
            "qknorm_layerwise_plan", "qknorm_layerwise_host", "qknorm_packed_host",
            "plan_shape", "plan_grid", "regions_overlap", "capi", "version", "QknLaunch", "QKNormError"]
 
-_DTYPES = {torch.float32: _clib.QKN_F32, torch.bfloat16: _clib.QKN_BF16}
+_DTYPES = {torch.float32: _clib.QKN_F32, torch.bfloat16: _clib.QKN_BF16, torch.float16: _clib.QKN_F16,
+           torch.float8_e4m3fn: _clib.QKN_FP8_E4M3}
+
+
+def gamma_dtype(dtype: torch.dtype) -> torch.dtype:
+    """The gamma type that goes with activations of `dtype` (bf16 for E4M3)."""
+    return torch.bfloat16 if dtype == torch.float8_e4m3fn else dtype
 
 
 def capi() -> ctypes.CDLL:
@@ -49,7 +55,7 @@ def _rows(t: torch.Tensor, name: str):
     if not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor (this library has no CPU path)")
     if t.dtype not in _DTYPES:
-        raise TypeError(f"{name}: dtype {t.dtype} unsupported (float32 or bfloat16)")
+        raise TypeError(f"{name}: dtype {t.dtype} unsupported (float32, bfloat16, float16, float8_e4m3fn)")
     if t.dim() != 2:
         raise ValueError(f"{name} must be 2-D [T, width]")
     T, H = t.shape
@@ -100,8 +106,9 @@ def _layerwise_args(q_in, k_in, gamma_q, gamma_k, eps, q_out, k_out):
         To, Ho, so = _rows(t, name)
         if (To, Ho) != (T, H) or (T > 1 and so != s):
             raise ValueError(f"{name} must match its input's shape and row stride")
-    args = [q_in.data_ptr(), q_out.data_ptr(), _vec(gamma_q, "gamma_q", Hq, dt, dev), sq,
-            k_in.data_ptr(), k_out.data_ptr(), _vec(gamma_k, "gamma_k", Hk, dt, dev), sk,
+    gdt = gamma_dtype(dt)
+    args = [q_in.data_ptr(), q_out.data_ptr(), _vec(gamma_q, "gamma_q", Hq, gdt, dev), sq,
+            k_in.data_ptr(), k_out.data_ptr(), _vec(gamma_k, "gamma_k", Hk, gdt, dev), sk,
             Tq, Hq, Hk, float(eps), _DTYPES[dt]]
     return args, q_out, k_out, dev
 
@@ -200,9 +207,10 @@ def qknorm_combine_apply(q_in: torch.Tensor, k_in: torch.Tensor, gamma_q_shard: 
         To, Ho, so = _rows(t, name)
         if (To, Ho) != (T, H) or (T > 1 and so != s):
             raise ValueError(f"{name} must match its input's shape and row stride")
-    args = [q_in.data_ptr(), q_out.data_ptr(), _vec(gamma_q_shard, "gamma_q_shard", hq, dt, dev), sq, hq,
+    gdt = gamma_dtype(dt)
+    args = [q_in.data_ptr(), q_out.data_ptr(), _vec(gamma_q_shard, "gamma_q_shard", hq, gdt, dev), sq, hq,
             ps_q, int(Hq_full),
-            k_in.data_ptr(), k_out.data_ptr(), _vec(gamma_k_shard, "gamma_k_shard", hk, dt, dev), sk, hk,
+            k_in.data_ptr(), k_out.data_ptr(), _vec(gamma_k_shard, "gamma_k_shard", hk, gdt, dev), sk, hk,
             ps_k, int(Hk_full), P, T, float(eps), _DTYPES[dt]]
     with torch.cuda.device(dev):
         s = _stream_handle(stream, dev)
@@ -216,9 +224,10 @@ def qknorm_combine_apply(q_in: torch.Tensor, k_in: torch.Tensor, gamma_q_shard: 
 
 # --------------------------------------------------------------------------- host planning (no GPU)
 
-def plan_shape(rows: int, units_max: int, vectorized: bool, sm_count: int) -> dict:
+def plan_shape(rows: int, units_max: int, vectorized: bool, sm_count: int, elem_bytes: int = 2) -> dict:
     L = QknLaunch()
-    st = capi().qknorm_plan_shape(rows, units_max, 1 if vectorized else 0, sm_count, ctypes.byref(L))
+    st = capi().qknorm_plan_shape(rows, units_max, 1 if vectorized else 0, sm_count, elem_bytes,
+                                  ctypes.byref(L))
     _clib.check(st, "qknorm_plan_shape")
     return L.as_dict()
 

@@ -12,6 +12,8 @@ LIBRARY = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libqknorm.so
 
 QKN_F32 = 0
 QKN_BF16 = 1
+QKN_F16 = 2
+QKN_FP8_E4M3 = 3
 
 QKN_OK = 0
 QKN_ERR_INVALID_ARG = 1
@@ -50,7 +52,7 @@ PROTOTYPES = {
     "qknorm_last_error": (ctypes.c_char_p, []),
     "qknorm_version": (ctypes.c_int, []),
     "qknorm_register_max_threads": (_i32, [_i32]),
-    "qknorm_plan_shape": (_st, [_i64, _i64, _i32, _i32, ctypes.POINTER(QknLaunch)]),
+    "qknorm_plan_shape": (_st, [_i64, _i64, _i32, _i32, _i32, ctypes.POINTER(QknLaunch)]),
     "qknorm_plan_grid": (_i64, [_i64, _i32, _i32]),
     "qknorm_regions_overlap": (ctypes.c_int, [_u64, _i64, _i64, _i64, _u64, _i64, _i64, _i64]),
     "qknorm_layerwise_plan": (_st, _LAYERWISE_ARGS + [ctypes.POINTER(QknLaunch)]),

@@ -41,9 +41,11 @@ qkn_status ok() {
     return QKN_OK;
 }
 
-int elem_bytes(qkn_dtype dt) { return dt == QKN_F32 ? 4 : 2; }
+// Bytes of one element of x (and y), and of one element of gamma.
+int elem_bytes(qkn_dtype dt) { return dt == QKN_F32 ? 4 : (dt == QKN_FP8_E4M3 ? 1 : 2); }
+int gamma_bytes(qkn_dtype dt) { return dt == QKN_F32 ? 4 : 2; }
 
-bool dtype_valid(int dt) { return dt == QKN_F32 || dt == QKN_BF16; }
+bool dtype_valid(int dt) { return dt >= QKN_F32 && dt <= QKN_FP8_E4M3; }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -199,7 +201,13 @@ const void *kernel_for(const qkn_launch &L, bool tail) {
 
 template <int MODE>
 const void *kernel_for(qkn_dtype dt, const qkn_launch &L, bool tail) {
-    return dt == QKN_F32 ? kernel_for<float, MODE>(L, tail) : kernel_for<__nv_bfloat16, MODE>(L, tail);
+    switch (dt) {
+        case QKN_F32: return kernel_for<float, MODE>(L, tail);
+        case QKN_BF16: return kernel_for<__nv_bfloat16, MODE>(L, tail);
+        case QKN_F16: return kernel_for<__half, MODE>(L, tail);
+        case QKN_FP8_E4M3: return kernel_for<__nv_fp8_e4m3, MODE>(L, tail);
+        default: return nullptr;
+    }
 }
 
 // A prepared call: parameters plus the facts planning needs.
@@ -313,7 +321,8 @@ qkn_status prepare_layerwise(const void *q_in, void *q_out, const void *gamma_q,
     if (T > 0) {
         const Region iq = rows_region(q_in, Hq, q_stride, T, esz), oq = rows_region(q_out, Hq, q_stride, T, esz);
         const Region ik = rows_region(k_in, Hk, k_stride, T, esz), ok_ = rows_region(k_out, Hk, k_stride, T, esz);
-        const Region others[2] = {flat_region(gamma_q, (int64_t)Hq * esz), flat_region(gamma_k, (int64_t)Hk * esz)};
+        const int gsz = gamma_bytes(dtype);
+        const Region others[2] = {flat_region(gamma_q, (int64_t)Hq * gsz), flat_region(gamma_k, (int64_t)Hk * gsz)};
         qkn_status st = check_outputs(oq, ok_, iq, ik, others, 2);
         if (st != QKN_OK) return st;
     }
@@ -335,7 +344,8 @@ qkn_status plan_call(const Call &c, qkn_launch &L) {
     if (st != QKN_OK) return st;
     if ((st = sm_count(dev, &sms)) != QKN_OK) return st;
     const int64_t items = 2 * c.p.T;
-    if ((st = qknorm_plan_shape(items, c.units_max, c.vectorized ? 1 : 0, sms, &L)) != QKN_OK)
+    if ((st = qknorm_plan_shape(items, c.units_max, c.vectorized ? 1 : 0, sms, elem_bytes(c.dtype), &L)) !=
+        QKN_OK)
         return fail(st, "planning failed");
     const void *fn = kernel_for<MODE>(c.dtype, L, c.tail);
     if (!fn) return fail(QKN_ERR_UNSUPPORTED, "no kernel for the planned launch");
@@ -376,11 +386,12 @@ qkn_status check_launch(const Call &c, const qkn_launch &L) {
 // Every launch allows programmatic dependent launch: the kernel may be
 // dispatched while the previous kernel in the stream drains (see
 // pdl_wait_and_release in the kernels, which restores the ordering).
-cudaError_t launch_pdl(const void *fn, unsigned grid, unsigned block, cudaStream_t s, const qkn::Params &p) {
+cudaError_t launch_pdl(const void *fn, unsigned grid, unsigned block, size_t smem, cudaStream_t s,
+                       const qkn::Params &p) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(block);
-    cfg.dynamicSmemBytes = 0;
+    cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -397,7 +408,7 @@ cudaError_t launch_any(const qkn_launch &L, const Call &c, cudaStream_t s) {
     if (!fn) return cudaErrorInvalidValue;
     qkn::Params p = c.p;
     if (L.kernel == QKN_KERNEL_REGISTER) set_groups(p, L.threads, L.vec_per_thread);
-    return launch_pdl(fn, (unsigned)L.grid, (unsigned)L.threads, s, p);
+    return launch_pdl(fn, (unsigned)L.grid, (unsigned)L.threads, 0, s, p);
 }
 
 template <int MODE>
@@ -463,8 +474,9 @@ qkn_status prepare_apply(const void *q_in, void *q_out, const void *gamma_q_shar
         const Region oq = rows_region(q_out, hq_shard, q_stride, T, esz);
         const Region ik = rows_region(k_in, hk_shard, k_stride, T, esz);
         const Region ok_ = rows_region(k_out, hk_shard, k_stride, T, esz);
-        const Region others[4] = {flat_region(gamma_q_shard, (int64_t)hq_shard * esz),
-                                  flat_region(gamma_k_shard, (int64_t)hk_shard * esz),
+        const int gsz = gamma_bytes(dtype);
+        const Region others[4] = {flat_region(gamma_q_shard, (int64_t)hq_shard * gsz),
+                                  flat_region(gamma_k_shard, (int64_t)hk_shard * gsz),
                                   flat_region(q_sumsq_all, (int64_t)P * T * 4),
                                   flat_region(k_sumsq_all, (int64_t)P * T * 4)};
         qkn_status st = check_outputs(oq, ok_, iq, ik, others, 4);
@@ -499,8 +511,9 @@ int32_t qknorm_register_max_threads(int32_t vec_per_thread) {
 }
 
 qkn_status qknorm_plan_shape(int64_t rows, int64_t units_max, int32_t vectorized, int32_t sm_count,
-                             qkn_launch *out) {
+                             int32_t elem_bytes, qkn_launch *out) {
     if (!out || rows < 1 || units_max < 1 || sm_count < 1) return QKN_ERR_INVALID_ARG;
+    if (elem_bytes != 1 && elem_bytes != 2 && elem_bytes != 4) return QKN_ERR_INVALID_ARG;
     qkn_launch L{};
     L.grid = 0;
     auto round32 = [](int64_t n) { return (int32_t)(((n + 31) / 32) * 32); };
@@ -528,6 +541,9 @@ qkn_status qknorm_plan_shape(int64_t rows, int64_t units_max, int32_t vectorized
         // Many rows: moderate CTAs, several vectors in flight per thread.
         nv = units_max >= 256 ? 4 : (units_max >= 64 ? 2 : 1);
     }
+    // A 16-byte vector of 1-byte elements widens to twice the fp32 registers
+    // (and pairs with two gamma vectors): hold half as many per thread.
+    if (elem_bytes == 1 && nv > 1) nv /= 2;
     int32_t threads = round32((units_max + nv - 1) / nv);
     while (threads > qknorm_register_max_threads(nv)) {
         nv *= 2;

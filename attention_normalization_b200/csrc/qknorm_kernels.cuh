@@ -9,6 +9,8 @@
 //     way out and only the final values are written.
 //   Deadlock-safe persistent execution: a bounded grid of resident CTAs that
 //     loop over tokens (here: over the Q rows, then the K rows).
+//   Evaluation, Fig. 2(b): BF16 and FP8-E4M3 activations with FP32
+//     accumulation.
 //
 // The work is a read-once / write-once stream with a per-row reduction: no
 // contraction, so no tensor cores.  What matters on B200 is bytes in flight
@@ -17,6 +19,8 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -32,12 +36,12 @@ enum Mode : int {
 struct RowSet {
     const char *in;          // row t starts at in + t * stride_bytes
     char *out;               // kFused / kApply
-    const char *gamma;       // kFused / kApply, [width]
+    const char *gamma;       // kFused / kApply, [width] of the gamma type
     float *sumsq;            // kStats: [T]
     const float *sumsq_all;  // kApply: [P][T]
     int64_t stride_bytes;
     int32_t width;           // elements in this row (shard width for kStats / kApply)
-    int32_t nfull;           // full 16-byte vectors in the row
+    int32_t nfull;           // full 16-byte vectors of x in the row
     int32_t tail;            // elements after the last full vector
     float inv_div;           // 1 / (the FULL width), rounded to fp32 on the host
     int32_t group;           // register kernel: threads that share one row (a multiple of 32)
@@ -53,56 +57,149 @@ struct Params {
 };
 
 // ----------------------------------------------------------------------------
-// Element packing: 16-byte vectors <-> fp32 lanes.
+// Packed fp32 pairs.  sm_100 executes add/mul/fma on two fp32 lanes held in
+// one 64-bit register pair (PTX .f32x2); each lane is an ordinary IEEE
+// round-to-nearest operation, so results equal the scalar ones bit for bit
+// while the instruction count of the elementwise work halves.
+struct F2 {
+    unsigned long long v;
+};
+__device__ __forceinline__ F2 f2(float lo, float hi) {
+    return F2{static_cast<unsigned long long>(__float_as_uint(lo)) |
+              (static_cast<unsigned long long>(__float_as_uint(hi)) << 32)};
+}
+__device__ __forceinline__ F2 f2_bits(uint32_t lo_bits, uint32_t hi_bits) {
+    return F2{static_cast<unsigned long long>(lo_bits) | (static_cast<unsigned long long>(hi_bits) << 32)};
+}
+__device__ __forceinline__ float f2_lo(F2 a) { return __uint_as_float(static_cast<uint32_t>(a.v)); }
+__device__ __forceinline__ float f2_hi(F2 a) { return __uint_as_float(static_cast<uint32_t>(a.v >> 32)); }
+__device__ __forceinline__ F2 mul2(F2 a, F2 b) {
+    F2 d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d.v) : "l"(a.v), "l"(b.v));
+    return d;
+}
+__device__ __forceinline__ F2 fma2(F2 a, F2 b, F2 c) {
+    F2 d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d.v) : "l"(a.v), "l"(b.v), "l"(c.v));
+    return d;
+}
+
+// ----------------------------------------------------------------------------
+// Element types.  For each: the storage of one element (Bits), elements per
+// 16-byte vector (kPerVec), the gamma type (G) and how many 16-byte gamma
+// vectors cover the elements of one x vector (kGVecs); conversions of a whole
+// vector to / from fp32 pairs, and of one element.  Narrowing rounds to
+// nearest even (E4M3: and saturates to +-448, the format having no infinity).
 template <typename E>
-struct Pack;
+struct Elem;
 
 template <>
-struct Pack<float> {
-    static constexpr int N = 4;  // elements per 16-byte vector
+struct Elem<float> {
     using Bits = uint32_t;
-    __device__ __forceinline__ static void widen(const uint4 &v, float (&f)[N]) {
-        f[0] = __uint_as_float(v.x);
-        f[1] = __uint_as_float(v.y);
-        f[2] = __uint_as_float(v.z);
-        f[3] = __uint_as_float(v.w);
+    using G = float;
+    static constexpr int kPerVec = 4;
+    static constexpr int kGVecs = 1;
+    __device__ __forceinline__ static void widen(const uint4 &v, F2 (&p)[kPerVec / 2]) {
+        p[0] = f2_bits(v.x, v.y);
+        p[1] = f2_bits(v.z, v.w);
     }
-    __device__ __forceinline__ static uint4 narrow(const float (&f)[N]) {
-        return make_uint4(__float_as_uint(f[0]), __float_as_uint(f[1]), __float_as_uint(f[2]),
-                          __float_as_uint(f[3]));
+    __device__ __forceinline__ static uint4 narrow(const F2 (&p)[kPerVec / 2]) {
+        return make_uint4(static_cast<uint32_t>(p[0].v), static_cast<uint32_t>(p[0].v >> 32),
+                          static_cast<uint32_t>(p[1].v), static_cast<uint32_t>(p[1].v >> 32));
     }
-    __device__ __forceinline__ static float bits_to_float(Bits b) { return __uint_as_float(b); }
-    __device__ __forceinline__ static Bits float_to_bits(float f) { return __float_as_uint(f); }
+    __device__ __forceinline__ static float to_float(Bits b) { return __uint_as_float(b); }
+    __device__ __forceinline__ static Bits from_float(float f) { return __float_as_uint(f); }
 };
 
 template <>
-struct Pack<__nv_bfloat16> {
-    static constexpr int N = 8;
+struct Elem<__nv_bfloat16> {
     using Bits = uint16_t;
-    // A bf16 value is the upper half of the fp32 with the same bits: widening is exact.
-    __device__ __forceinline__ static void widen2(uint32_t u, float &lo, float &hi) {
-        lo = __uint_as_float(u << 16);
-        hi = __uint_as_float(u & 0xFFFF0000u);
-    }
-    __device__ __forceinline__ static uint32_t narrow2(float lo, float hi) {
-        __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);  // round to nearest even
+    using G = __nv_bfloat16;
+    static constexpr int kPerVec = 8;
+    static constexpr int kGVecs = 1;
+    // the bf16 in the low half of a word is the fp32 with those bits in the high half
+    __device__ __forceinline__ static F2 widen_word(uint32_t w) { return f2_bits(w << 16, w & 0xFFFF0000u); }
+    __device__ __forceinline__ static uint32_t narrow_word(F2 a) {
+        __nv_bfloat162 h = __floats2bfloat162_rn(f2_lo(a), f2_hi(a));
         return *reinterpret_cast<uint32_t *>(&h);
     }
-    __device__ __forceinline__ static void widen(const uint4 &v, float (&f)[N]) {
-        widen2(v.x, f[0], f[1]);
-        widen2(v.y, f[2], f[3]);
-        widen2(v.z, f[4], f[5]);
-        widen2(v.w, f[6], f[7]);
+    __device__ __forceinline__ static void widen(const uint4 &v, F2 (&p)[kPerVec / 2]) {
+        p[0] = widen_word(v.x);
+        p[1] = widen_word(v.y);
+        p[2] = widen_word(v.z);
+        p[3] = widen_word(v.w);
     }
-    __device__ __forceinline__ static uint4 narrow(const float (&f)[N]) {
-        return make_uint4(narrow2(f[0], f[1]), narrow2(f[2], f[3]), narrow2(f[4], f[5]),
-                          narrow2(f[6], f[7]));
+    __device__ __forceinline__ static uint4 narrow(const F2 (&p)[kPerVec / 2]) {
+        return make_uint4(narrow_word(p[0]), narrow_word(p[1]), narrow_word(p[2]), narrow_word(p[3]));
     }
-    __device__ __forceinline__ static float bits_to_float(Bits b) {
-        return __uint_as_float(static_cast<uint32_t>(b) << 16);
+    __device__ __forceinline__ static float to_float(Bits b) { return __uint_as_float(static_cast<uint32_t>(b) << 16); }
+    __device__ __forceinline__ static Bits from_float(float f) { return __bfloat16_as_ushort(__float2bfloat16_rn(f)); }
+};
+
+template <>
+struct Elem<__half> {
+    using Bits = uint16_t;
+    using G = __half;
+    static constexpr int kPerVec = 8;
+    static constexpr int kGVecs = 1;
+    __device__ __forceinline__ static F2 widen_word(uint32_t w) {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w));
+        return f2(f.x, f.y);
     }
-    __device__ __forceinline__ static Bits float_to_bits(float f) {
-        return __bfloat16_as_ushort(__float2bfloat16_rn(f));
+    __device__ __forceinline__ static uint32_t narrow_word(F2 a) {
+        __half2 h = __floats2half2_rn(f2_lo(a), f2_hi(a));
+        return *reinterpret_cast<uint32_t *>(&h);
+    }
+    __device__ __forceinline__ static void widen(const uint4 &v, F2 (&p)[kPerVec / 2]) {
+        p[0] = widen_word(v.x);
+        p[1] = widen_word(v.y);
+        p[2] = widen_word(v.z);
+        p[3] = widen_word(v.w);
+    }
+    __device__ __forceinline__ static uint4 narrow(const F2 (&p)[kPerVec / 2]) {
+        return make_uint4(narrow_word(p[0]), narrow_word(p[1]), narrow_word(p[2]), narrow_word(p[3]));
+    }
+    __device__ __forceinline__ static float to_float(Bits b) { return __half2float(__ushort_as_half(b)); }
+    __device__ __forceinline__ static Bits from_float(float f) { return __half_as_ushort(__float2half_rn(f)); }
+};
+
+template <>
+struct Elem<__nv_fp8_e4m3> {
+    using Bits = uint8_t;
+    using G = __nv_bfloat16;  // gamma is kept in bf16 next to E4M3 activations
+    static constexpr int kPerVec = 16;
+    static constexpr int kGVecs = 2;
+    // two E4M3 values (16 bits) -> exact half pair -> fp32 pair
+    __device__ __forceinline__ static F2 widen_half_word(uint32_t two) {
+        const __half2_raw hr =
+            __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two & 0xFFFFu), __NV_E4M3);
+        const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&hr));
+        return f2(f.x, f.y);
+    }
+    __device__ __forceinline__ static uint32_t narrow_pair(F2 a) {
+        return static_cast<uint32_t>(
+            __nv_cvt_float2_to_fp8x2(make_float2(f2_lo(a), f2_hi(a)), __NV_SATFINITE, __NV_E4M3));
+    }
+    __device__ __forceinline__ static void widen(const uint4 &v, F2 (&p)[kPerVec / 2]) {
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            p[2 * i] = widen_half_word(w[i]);
+            p[2 * i + 1] = widen_half_word(w[i] >> 16);
+        }
+    }
+    __device__ __forceinline__ static uint4 narrow(const F2 (&p)[kPerVec / 2]) {
+        uint32_t w[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) w[i] = narrow_pair(p[2 * i]) | (narrow_pair(p[2 * i + 1]) << 16);
+        return make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    __device__ __forceinline__ static float to_float(Bits b) {
+        const __half_raw hr = __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(b), __NV_E4M3);
+        return __half2float(*reinterpret_cast<const __half *>(&hr));
+    }
+    __device__ __forceinline__ static Bits from_float(float f) {
+        return static_cast<Bits>(__nv_cvt_float_to_fp8(f, __NV_SATFINITE, __NV_E4M3));
     }
 };
 
@@ -121,14 +218,15 @@ __device__ __forceinline__ uint4 ld_gamma(const char *p) {
     return __ldg(reinterpret_cast<const uint4 *>(p));
 }
 
-// The last, partial vector of a row: `n` (< N) elements, the rest zero.
+// The last, partial vector of a row: `n` (< kPerVec) elements, the rest zero.
 template <typename E>
 __device__ __forceinline__ uint4 ld_tail(const char *p, int n) {
-    using P = Pack<E>;
-    typename P::Bits b[P::N];
-    const typename P::Bits *src = reinterpret_cast<const typename P::Bits *>(p);
+    using B = typename Elem<E>::Bits;
+    constexpr int N = Elem<E>::kPerVec;
+    B b[N];
+    const B *src = reinterpret_cast<const B *>(p);
 #pragma unroll
-    for (int e = 0; e < P::N; ++e) b[e] = (e < n) ? src[e] : typename P::Bits(0);
+    for (int e = 0; e < N; ++e) b[e] = (e < n) ? src[e] : B(0);
     uint4 v;
     static_assert(sizeof(b) == sizeof(uint4), "vector size");
     memcpy(&v, b, sizeof(v));
@@ -136,13 +234,39 @@ __device__ __forceinline__ uint4 ld_tail(const char *p, int n) {
 }
 template <typename E>
 __device__ __forceinline__ void st_tail(char *p, const uint4 &v, int n) {
-    using P = Pack<E>;
-    typename P::Bits b[P::N];
+    using B = typename Elem<E>::Bits;
+    constexpr int N = Elem<E>::kPerVec;
+    B b[N];
     memcpy(b, &v, sizeof(v));
-    typename P::Bits *dst = reinterpret_cast<typename P::Bits *>(p);
+    B *dst = reinterpret_cast<B *>(p);
 #pragma unroll
-    for (int e = 0; e < P::N; ++e)
+    for (int e = 0; e < N; ++e)
         if (e < n) dst[e] = b[e];
+}
+
+// The gamma vectors covering x vector `vi` of a row of `nfull` full vectors
+// and `tail` trailing elements (zero past the row's end).
+template <typename E>
+__device__ __forceinline__ void ld_gamma_vec(const char *gamma, int vi, int nfull, int tail,
+                                             uint4 (&g)[Elem<E>::kGVecs]) {
+    using GB = typename Elem<typename Elem<E>::G>::Bits;
+    constexpr int KG = Elem<E>::kGVecs;
+    const char *p = gamma + static_cast<int64_t>(vi) * 16 * KG;
+    if (vi < nfull) {
+#pragma unroll
+        for (int j = 0; j < KG; ++j) g[j] = ld_gamma(p + 16 * j);
+    } else if (vi == nfull && tail) {
+        constexpr int N = Elem<E>::kPerVec;
+        GB b[N];
+        const GB *src = reinterpret_cast<const GB *>(p);
+#pragma unroll
+        for (int e = 0; e < N; ++e) b[e] = (e < tail) ? src[e] : GB(0);
+        static_assert(sizeof(b) == sizeof(g), "gamma vector size");
+        memcpy(g, b, sizeof(b));
+    } else {
+#pragma unroll
+        for (int j = 0; j < KG; ++j) g[j] = make_uint4(0u, 0u, 0u, 0u);
+    }
 }
 
 // ----------------------------------------------------------------------------
@@ -180,6 +304,10 @@ __device__ __forceinline__ float combine_partials(const float *all, int64_t T, i
 }
 
 // r = 1 / sqrt(S / H + eps), the mean formed as S * fl(1 / H).
+__device__ __forceinline__ float rms_factor(float sumsq, float inv_div, float eps) {
+    return rsqrtf(sumsq * inv_div + eps);
+}
+
 // Programmatic dependent launch (sm_90+).  Kernels here are launched with
 // programmatic stream serialization, so their CTAs may be dispatched while the
 // previous kernel in the stream is still draining.  Every kernel therefore
@@ -192,99 +320,40 @@ __device__ __forceinline__ void pdl_wait_and_release() {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
-__device__ __forceinline__ float rms_factor(float sumsq, float inv_div, float eps) {
-    return rsqrtf(sumsq * inv_div + eps);
-}
-
-// ----------------------------------------------------------------------------
-// Packed fp32 pairs.  sm_100 executes add/mul/fma on two fp32 lanes held in
-// one 64-bit register pair (PTX .f32x2); each lane is an ordinary IEEE
-// round-to-nearest operation, so results equal the scalar ones bit for bit
-// while the instruction count of the elementwise work halves.
-struct F2 {
-    unsigned long long v;
-};
-__device__ __forceinline__ F2 f2(float lo, float hi) {
-    return F2{static_cast<unsigned long long>(__float_as_uint(lo)) |
-              (static_cast<unsigned long long>(__float_as_uint(hi)) << 32)};
-}
-__device__ __forceinline__ F2 f2_bits(uint32_t lo_bits, uint32_t hi_bits) {
-    return F2{static_cast<unsigned long long>(lo_bits) | (static_cast<unsigned long long>(hi_bits) << 32)};
-}
-__device__ __forceinline__ float f2_lo(F2 a) { return __uint_as_float(static_cast<uint32_t>(a.v)); }
-__device__ __forceinline__ float f2_hi(F2 a) { return __uint_as_float(static_cast<uint32_t>(a.v >> 32)); }
-__device__ __forceinline__ F2 mul2(F2 a, F2 b) {
-    F2 d;
-    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d.v) : "l"(a.v), "l"(b.v));
-    return d;
-}
-__device__ __forceinline__ F2 fma2(F2 a, F2 b, F2 c) {
-    F2 d;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d.v) : "l"(a.v), "l"(b.v), "l"(c.v));
-    return d;
-}
-
-// A 16-byte vector as fp32 pairs: bf16 holds 4 pairs (one per 32-bit word),
-// fp32 holds 2.
-template <typename E>
-struct Pairs;
-template <>
-struct Pairs<__nv_bfloat16> {
-    static constexpr int K = 4;
-    __device__ __forceinline__ static void widen(const uint4 &v, F2 (&p)[K]) {
-        // the bf16 in the low half of a word is the fp32 with those bits in the high half
-        p[0] = f2_bits(v.x << 16, v.x & 0xFFFF0000u);
-        p[1] = f2_bits(v.y << 16, v.y & 0xFFFF0000u);
-        p[2] = f2_bits(v.z << 16, v.z & 0xFFFF0000u);
-        p[3] = f2_bits(v.w << 16, v.w & 0xFFFF0000u);
-    }
-    __device__ __forceinline__ static uint32_t narrow1(F2 a) {
-        __nv_bfloat162 h = __floats2bfloat162_rn(f2_lo(a), f2_hi(a));  // round to nearest even
-        return *reinterpret_cast<uint32_t *>(&h);
-    }
-    __device__ __forceinline__ static uint4 narrow(const F2 (&p)[K]) {
-        return make_uint4(narrow1(p[0]), narrow1(p[1]), narrow1(p[2]), narrow1(p[3]));
-    }
-};
-template <>
-struct Pairs<float> {
-    static constexpr int K = 2;
-    __device__ __forceinline__ static void widen(const uint4 &v, F2 (&p)[K]) {
-        p[0] = f2_bits(v.x, v.y);
-        p[1] = f2_bits(v.z, v.w);
-    }
-    __device__ __forceinline__ static uint4 narrow(const F2 (&p)[K]) {
-        return make_uint4(static_cast<uint32_t>(p[0].v), static_cast<uint32_t>(p[0].v >> 32),
-                          static_cast<uint32_t>(p[1].v), static_cast<uint32_t>(p[1].v >> 32));
-    }
-};
-
 // Squared sum of a thread's vectors (two fp32 lanes accumulate the even and
 // odd elements; they are added at the end).
 template <typename E, int NV>
 __device__ __forceinline__ float sumsq_pairs(const uint4 (&v)[NV]) {
-    using PP = Pairs<E>;
+    constexpr int K = Elem<E>::kPerVec / 2;
     F2 acc = f2(0.0f, 0.0f);
 #pragma unroll
     for (int i = 0; i < NV; ++i) {
-        F2 x[PP::K];
-        PP::widen(v[i], x);
+        F2 x[K];
+        Elem<E>::widen(v[i], x);
 #pragma unroll
-        for (int j = 0; j < PP::K; ++j) acc = fma2(x[j], x[j], acc);
+        for (int j = 0; j < K; ++j) acc = fma2(x[j], x[j], acc);
     }
     return f2_lo(acc) + f2_hi(acc);
 }
 
 // Phase B on the way out, one vector: y = (x * gamma) * r, rounded once.
 template <typename E>
-__device__ __forceinline__ uint4 scale_vec(const uint4 &xv, const uint4 &gv, F2 r2) {
-    using PP = Pairs<E>;
-    F2 x[PP::K], g[PP::K];
-    PP::widen(xv, x);
-    PP::widen(gv, g);
+__device__ __forceinline__ uint4 scale_vec(const uint4 &xv, const uint4 (&gv)[Elem<E>::kGVecs], F2 r2) {
+    using GT = typename Elem<E>::G;
+    constexpr int K = Elem<E>::kPerVec / 2;
+    constexpr int KG = Elem<GT>::kPerVec / 2;
+    F2 x[K], g[K];
+    Elem<E>::widen(xv, x);
 #pragma unroll
-    for (int j = 0; j < PP::K; ++j) x[j] = mul2(mul2(x[j], g[j]), r2);
-    return PP::narrow(x);
+    for (int j = 0; j < Elem<E>::kGVecs; ++j) {
+        F2 part[KG];
+        Elem<GT>::widen(gv[j], part);
+#pragma unroll
+        for (int k = 0; k < KG; ++k) g[j * KG + k] = part[k];
+    }
+#pragma unroll
+    for (int j = 0; j < K; ++j) x[j] = mul2(mul2(x[j], g[j]), r2);
+    return Elem<E>::narrow(x);
 }
 
 // ----------------------------------------------------------------------------
@@ -312,6 +381,7 @@ struct RegisterBounds {
 template <typename E, int NV, int MODE, bool TAIL>
 __global__ void __launch_bounds__(RegisterBounds<NV>::kMaxThreads)
     rows_register_kernel(const __grid_constant__ Params p) {
+    constexpr int KG = Elem<E>::kGVecs;
     __shared__ float red[2][32];
     pdl_wait_and_release();
     int slot = 0;
@@ -330,7 +400,7 @@ __global__ void __launch_bounds__(RegisterBounds<NV>::kMaxThreads)
     int64_t stride = 0;
     int nfull = 0, tail = 0, gsize = 32, rpi = 1, grp = 0, gl = 0, gwarps = 1;
     float inv_div = 0.0f;
-    uint4 g[NV];
+    uint4 g[NV][KG];
 
     for (int64_t item = blockIdx.x; item < n_items; item += gridDim.x) {
         const int w = item >= q_items ? 1 : 0;
@@ -353,16 +423,7 @@ __global__ void __launch_bounds__(RegisterBounds<NV>::kMaxThreads)
             gwarps = gsize >> 5;
             if (MODE != kStats) {
 #pragma unroll
-                for (int i = 0; i < NV; ++i) {
-                    const int vi = gl + i * gsize;
-                    const int64_t off = static_cast<int64_t>(vi) * 16;
-                    if (vi < nfull)
-                        g[i] = ld_gamma(d.gamma + off);
-                    else if (TAIL && vi == nfull && tail)
-                        g[i] = ld_tail<E>(d.gamma + off, tail);
-                    else
-                        g[i] = make_uint4(0u, 0u, 0u, 0u);
-                }
+                for (int i = 0; i < NV; ++i) ld_gamma_vec<E>(d.gamma, gl + i * gsize, nfull, tail, g[i]);
             }
         }
         const int64_t t = j * rpi + grp;
@@ -406,10 +467,15 @@ __global__ void __launch_bounds__(RegisterBounds<NV>::kMaxThreads)
         for (int i = 0; i < NV; ++i) {
             const int vi = gl + i * gsize;
             const int64_t off = static_cast<int64_t>(vi) * 16;
-            if (vi < nfull)
-                st_stream(orow + off, scale_vec<E>(v[i], g[i], r2));
-            else if (TAIL && vi == nfull && tail)
-                st_tail<E>(orow + off, scale_vec<E>(v[i], g[i], r2), tail);
+            const bool full = vi < nfull;
+            const bool part = TAIL && vi == nfull && tail;
+            if (full || part) {
+                const uint4 y = scale_vec<E>(v[i], g[i], r2);
+                if (full)
+                    st_stream(orow + off, y);
+                else
+                    st_tail<E>(orow + off, y, tail);
+            }
         }
     }
 }
@@ -419,10 +485,13 @@ __global__ void __launch_bounds__(RegisterBounds<NV>::kMaxThreads)
 // not 16-byte aligned (!VEC, element-wise).  Pass 1 forms the squared sum;
 // pass 2 re-reads x (largely from L2), scales and stores.  In place is safe:
 // pass 2 reads each element before the same thread writes it, and pass 1 has
-// finished for the whole row (block barrier) before pass 2 starts.
+// finished for the whole row (block barrier) before pass 2 starts.  Items are
+// whole rows, Q rows first, then K rows.
 template <typename E, bool VEC, int MODE>
 __global__ void __launch_bounds__(1024) rows_twopass_kernel(const __grid_constant__ Params p) {
-    using Pk = Pack<E>;
+    using EL = Elem<E>;
+    using GT = typename EL::G;
+    constexpr int K = EL::kPerVec / 2;
     __shared__ float red[2][32];
     pdl_wait_and_release();
     int slot = 0;
@@ -430,7 +499,7 @@ __global__ void __launch_bounds__(1024) rows_twopass_kernel(const __grid_constan
     const int nthr = blockDim.x;
 
     for (int64_t item = blockIdx.x; item < 2 * p.T; item += gridDim.x) {
-        const int w = item >= p.T ? 1 : 0;  // Q rows first, then K rows
+        const int w = item >= p.T ? 1 : 0;
         const RowSet &d = p.set[w];
         const int64_t t = w ? item - p.T : item;
         const char *row = d.in + t * d.stride_bytes;
@@ -445,13 +514,14 @@ __global__ void __launch_bounds__(1024) rows_twopass_kernel(const __grid_constan
                 if (VEC) {
                     const uint4 v = (u < d.nfull) ? ld_stream(row + static_cast<int64_t>(u) * 16)
                                                   : ld_tail<E>(row + static_cast<int64_t>(u) * 16, d.tail);
-                    float f[Pk::N];
-                    Pk::widen(v, f);
+                    F2 x[K];
+                    EL::widen(v, x);
+                    F2 a = f2(0.0f, 0.0f);
 #pragma unroll
-                    for (int e = 0; e < Pk::N; ++e) acc = fmaf(f[e], f[e], acc);
+                    for (int j = 0; j < K; ++j) a = fma2(x[j], x[j], a);
+                    acc += f2_lo(a) + f2_hi(a);
                 } else {
-                    const float f = Pk::bits_to_float(
-                        reinterpret_cast<const typename Pk::Bits *>(row)[u]);
+                    const float f = EL::to_float(reinterpret_cast<const typename EL::Bits *>(row)[u]);
                     acc = fmaf(f, f, acc);
                 }
             }
@@ -469,22 +539,17 @@ __global__ void __launch_bounds__(1024) rows_twopass_kernel(const __grid_constan
                 const bool full = u < d.nfull;
                 const int64_t off = static_cast<int64_t>(u) * 16;
                 const uint4 xv = full ? ld_stream(row + off) : ld_tail<E>(row + off, d.tail);
-                const uint4 gv = full ? ld_gamma(d.gamma + off) : ld_tail<E>(d.gamma + off, d.tail);
-                float f[Pk::N], g[Pk::N];
-                Pk::widen(xv, f);
-                Pk::widen(gv, g);
-#pragma unroll
-                for (int e = 0; e < Pk::N; ++e) f[e] = (f[e] * g[e]) * r;
-                const uint4 y = Pk::narrow(f);
+                uint4 gv[EL::kGVecs];
+                ld_gamma_vec<E>(d.gamma, u, d.nfull, d.tail, gv);
+                const uint4 y = scale_vec<E>(xv, gv, f2(r, r));
                 if (full)
                     st_stream(orow + off, y);
                 else
                     st_tail<E>(orow + off, y, d.tail);
             } else {
-                const float f = Pk::bits_to_float(reinterpret_cast<const typename Pk::Bits *>(row)[u]);
-                const float g =
-                    Pk::bits_to_float(reinterpret_cast<const typename Pk::Bits *>(d.gamma)[u]);
-                reinterpret_cast<typename Pk::Bits *>(orow)[u] = Pk::float_to_bits((f * g) * r);
+                const float f = EL::to_float(reinterpret_cast<const typename EL::Bits *>(row)[u]);
+                const float g = Elem<GT>::to_float(reinterpret_cast<const typename Elem<GT>::Bits *>(d.gamma)[u]);
+                reinterpret_cast<typename EL::Bits *>(orow)[u] = EL::from_float((f * g) * r);
             }
         }
     }

@@ -59,6 +59,8 @@ def parse_args(argv=None):
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--workload", choices=["prefill", "decode", "packed", "gqa", "tiny"], default="prefill")
     ap.add_argument("--tokens", type=int, default=None, help="T for decode / packed workloads")
+    ap.add_argument("--dtype", choices=["bf16", "f16", "e4m3"], default="bf16",
+                    help="element type of the prefill workload (gamma is bf16 with e4m3)")
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU baseline budget")
@@ -222,10 +224,12 @@ class Workload:
     """A benchmark workload: CPU batch, effective bytes per step, and a step
     function over a device-resident set."""
 
-    def __init__(self, kind: str, tokens: int | None, seed_offset: int):
+    DTYPES = {"bf16": torch.bfloat16, "f16": torch.float16, "e4m3": torch.float8_e4m3fn}
+
+    def __init__(self, kind: str, tokens: int | None, seed_offset: int, dtype: str = "bf16"):
         self.kind = kind
         if kind == "prefill":
-            self.batch = workloads.prefill_bf16(seed=1 + seed_offset)
+            self.batch = workloads.prefill_bf16(seed=1 + seed_offset, dtype=self.DTYPES[dtype])
         elif kind == "tiny":
             self.batch = workloads.tiny_fp32(seed=0 + seed_offset)
         elif kind == "decode":
@@ -235,9 +239,10 @@ class Workload:
         elif kind == "gqa":
             self.batch = workloads.gqa_sharded(seed=3 + seed_offset)
         b = self.batch
-        self.esz = 4 if b.dtype == torch.float32 else 2
+        self.esz = {torch.float32: 4, torch.float8_e4m3fn: 1}.get(b.dtype, 2)
+        gesz = 4 if b.dtype == torch.float32 else 2
         # bytes the method must move per step: read + write of every Q and K element, plus gamma
-        self.eff_bytes = 2 * self.esz * (b.Hq + b.Hk) * b.T + self.esz * (b.Hq + b.Hk)
+        self.eff_bytes = 2 * self.esz * (b.Hq + b.Hk) * b.T + gesz * (b.Hq + b.Hk)
         self.name = b.name
         self.launches_per_step = 2 * b.P if kind == "gqa" else 1
 
@@ -334,7 +339,12 @@ def time_oracle(wl: Workload, budget_s: float, max_tokens: int | None = None) ->
     def np_rows(view):
         view = view[:T]
         t = view.contiguous()
-        a = t.view(torch.int16).numpy().view(np.uint16) if t.dtype == torch.bfloat16 else t.numpy()
+        if t.dtype == torch.bfloat16:
+            a = t.view(torch.int16).numpy().view(np.uint16)
+        elif t.dtype == torch.float8_e4m3fn:
+            a = t.view(torch.uint8).numpy()
+        else:
+            a = t.numpy()
         return a, view.shape[1]
 
     if wl.kind == "gqa":
@@ -370,7 +380,7 @@ def time_oracle(wl: Workload, budget_s: float, max_tokens: int | None = None) ->
         if el >= budget_s or calls >= 1000:
             break
     per_call = el / calls
-    eff = 2 * wl.esz * (b.Hq + b.Hk) * T + wl.esz * (b.Hq + b.Hk)
+    eff = 2 * wl.esz * (b.Hq + b.Hk) * T + (4 if b.dtype == torch.float32 else 2) * (b.Hq + b.Hk)
     return {"value": eff / per_call / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle",
             "sample": f"{calls} oracle call(s) on {T} of {b.T} tokens of {wl.name}, {el:.1f} s",
             "us_per_call": per_call * 1e6, "tokens": T, "calls": calls}
@@ -398,7 +408,7 @@ def native(args) -> int:
     ranks = Ranks(dist, dev)
     barrier, max_over_ranks = ranks.barrier, ranks.max
 
-    wl = Workload(args.workload, args.tokens, seed_offset=rank * 1000)
+    wl = Workload(args.workload, args.tokens, seed_offset=rank * 1000, dtype=args.dtype)
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     R = rotating = rotation_count(wl.set_bytes(), l2)
     sets = [wl.make_set(dev) for _ in range(R)]
@@ -569,7 +579,7 @@ def reference(args) -> int:
     rank, world, _ = dist_env()
     if rank != 0:
         return 0  # the CPU oracle runs once, on rank 0
-    wl = Workload(args.workload, args.tokens, seed_offset=0)
+    wl = Workload(args.workload, args.tokens, seed_offset=0, dtype=args.dtype)
     b = wl.batch
     # per-step sample: enough tokens that the whole run stays near a minute
     probe = time_oracle(wl, 0.0, max_tokens=min(b.T, 8))
@@ -582,7 +592,7 @@ def reference(args) -> int:
     for _ in range(args.steps):
         time_oracle(wl, 0.0, max_tokens=tokens)
     el = time.perf_counter() - t0
-    eff = 2 * wl.esz * (b.Hq + b.Hk) * tokens + wl.esz * (b.Hq + b.Hk)
+    eff = 2 * wl.esz * (b.Hq + b.Hk) * tokens + (4 if b.dtype == torch.float32 else 2) * (b.Hq + b.Hk)
     value = eff / (el / args.steps) / 1e9
     cfg = wl.config()
     cfg.update({"sample_tokens_per_step": tokens})

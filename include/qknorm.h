@@ -19,6 +19,9 @@
  *   reduction; the global factor r is applied to it and only the final
  *   normalized values are written.
  *
+ * Paper, Evaluation, Fig. 2(b): BF16 and FP8-E4M3 activations, FP32
+ * accumulation.
+ *
  * Arithmetic: elements are widened to fp32; squared sums, the factor and the
  * scaling are fp32 (squares accumulated with fused multiply-add); the mean is
  * formed as S * fl(1/H), with 1/H rounded to fp32 once on the host (exact when
@@ -35,8 +38,8 @@
  *     [Q | K | V] rows are addressed by passing base and base + Hq with the
  *     packed stride; columns outside [0, width) (V, padding) are never read
  *     or written.
- *   - gamma vectors are contiguous, of the element type, one per tensor (or
- *     per shard, for the shard entry points).
+ *   - gamma vectors are contiguous, one per tensor (or per shard, for the
+ *     shard entry points), of the element type -- bfloat16 for E4M3 data.
  *   - out == in (same base, same stride) normalizes in place.  Any other
  *     overlap between a written region and any other region is rejected with
  *     QKN_ERR_INVALID_ARG.  Two strided regions with different strides whose
@@ -63,8 +66,12 @@ extern "C" {
 #endif
 
 typedef enum {
-    QKN_F32 = 0,   /* IEEE binary32 elements */
-    QKN_BF16 = 1   /* bfloat16 elements */
+    QKN_F32 = 0,      /* IEEE binary32 elements; gamma binary32 */
+    QKN_BF16 = 1,     /* bfloat16 elements; gamma bfloat16 */
+    QKN_F16 = 2,      /* IEEE binary16 elements; gamma binary16 */
+    QKN_FP8_E4M3 = 3  /* FP8 E4M3 ("fn": no infinities, largest finite 448)
+                         elements; gamma bfloat16.  Outputs round to nearest
+                         even and saturate to +-448. */
 } qkn_dtype;
 
 typedef enum {

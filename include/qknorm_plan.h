@@ -58,12 +58,13 @@ int32_t qknorm_register_max_threads(int32_t vec_per_thread);
  *   rows       : row items in the launch (2 * T),
  *   units_max  : the widest row, in 16-byte vectors if `vectorized`, else in elements,
  *   vectorized : 1 if every pointer and row stride is 16-byte aligned,
- *   sm_count   : streaming multiprocessors on the device.
+ *   sm_count   : streaming multiprocessors on the device,
+ *   elem_bytes : bytes per element of x (4, 2 or 1).
  * Pure function of its arguments; needs no GPU.  QKN_ERR_INVALID_ARG for
- * rows < 1, units_max < 1 or sm_count < 1.
+ * rows < 1, units_max < 1, sm_count < 1 or another elem_bytes.
  */
 qkn_status qknorm_plan_shape(int64_t rows, int64_t units_max, int32_t vectorized, int32_t sm_count,
-                             qkn_launch *out);
+                             int32_t elem_bytes, qkn_launch *out);
 
 /*
  * CTAs for `rows` items when `blocks_per_sm` CTAs fit on each of `sm_count`

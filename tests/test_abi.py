@@ -84,6 +84,8 @@ def test_well_formed_call_passes_validation(lib):
 
 @pytest.mark.parametrize("kw,why", [
     ({"dtype": 7}, "dtype"),
+    ({"dtype": 4}, "dtype past E4M3"),
+    ({"dtype": -1}, "negative dtype"),
     ({"T": -1}, "T < 0"),
     ({"Hq": 0}, "Hq = 0"),
     ({"Hk": -3}, "Hk < 0"),
@@ -274,6 +276,15 @@ def test_plan_shape_covers_the_row(rows, units):
     assert th % 32 == 0 and 32 <= th <= _clib.load().qknorm_register_max_threads(nv)
     assert nv * th >= units
     assert nv * (th - 32) < units  # no whole idle warp
+
+
+def test_plan_shape_one_byte_elements_hold_half_the_vectors():
+    two = qk.plan_shape(8192, 512, True, 148, 2)
+    one = qk.plan_shape(8192, 512, True, 148, 1)
+    assert one["vec_per_thread"] * 2 == two["vec_per_thread"]
+    assert one["vec_per_thread"] * one["threads"] >= 512
+    with pytest.raises(qk.QKNormError):
+        qk.plan_shape(10, 10, True, 148, 3)
 
 
 def test_plan_shape_wide_and_unaligned():

@@ -27,7 +27,7 @@ import torch
 import attention_normalization_b200 as qk
 import oracle
 import workloads
-from tests.conftest import bf16_ulp_distance, buffer_np, to_np
+from tests.conftest import bf16_ulp_distance, buffer_np, to_np, ulp_distance
 
 pytestmark = pytest.mark.gpu
 
@@ -45,12 +45,21 @@ def oracle_rows(view: torch.Tensor, gamma: torch.Tensor, eps: float):
     return oracle.rmsnorm_rows(flat, H, to_np(gamma), eps, stride=stride, T=T)
 
 
+ALL_DTYPES = [torch.float32, torch.bfloat16, torch.float16, torch.float8_e4m3fn]
+NARROW_DTYPES = [torch.bfloat16, torch.float16, torch.float8_e4m3fn]
+
+
+def esz(dtype: torch.dtype) -> int:
+    return {torch.float32: 4, torch.bfloat16: 2, torch.float16: 2, torch.float8_e4m3fn: 1}[dtype]
+
+
 def assert_close(got: torch.Tensor, y_rounded: np.ndarray, y_exact: np.ndarray, what: str):
     got = got.detach().cpu().contiguous()
-    if got.dtype == torch.bfloat16:
-        d = bf16_ulp_distance(to_np(got), y_rounded)
+    if got.dtype != torch.float32:
+        d = ulp_distance(to_np(got), y_rounded, got.dtype)
         worst = int(d.max()) if d.size else 0
-        assert worst <= 1, f"{what}: {worst} bf16 ulp from the oracle (at {np.unravel_index(d.argmax(), d.shape)})"
+        assert worst <= 1, (f"{what}: {worst} ulp of {got.dtype} from the oracle "
+                            f"(at {np.unravel_index(d.argmax(), d.shape)})")
     else:
         o = y_exact
         rel = np.abs(got.double().numpy() - o) / np.maximum(np.abs(o), 1e-30)
@@ -99,8 +108,9 @@ def test_tiny_fp32_out_of_place_then_in_place_bitwise_equal():
     assert torch.equal(qo, qi) and torch.equal(ko, ki)
 
 
-def test_prefill_bf16_full_size():
-    b = workloads.prefill_bf16()
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16, torch.float8_e4m3fn])
+def test_prefill_full_size(dtype):
+    b = workloads.prefill_bf16(dtype=dtype)
     check_layerwise(b)
 
 
@@ -158,12 +168,12 @@ def test_packed_qkv_in_place_v_untouched(T):
 
 def aligned_stride(H: int, dtype: torch.dtype, extra_vectors: int = 1) -> int:
     """A row stride whose byte size is a multiple of 16, leaving padding after H."""
-    per = 16 // (4 if dtype == torch.float32 else 2)
+    per = 16 // esz(dtype)
     return -(-H // per) * per + extra_vectors * per
 
 
 @pytest.mark.parametrize("layout", ["contiguous", "padded"])
-@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("dtype", ALL_DTYPES)
 @pytest.mark.parametrize("T,Hq,Hk", [(1, 1, 1), (2, 3, 7), (3, 8, 9), (17, 127, 129), (5, 513, 64),
                                       (33, 4096, 1024), (7, 5120, 5120), (300, 1000, 24)])
 def test_small_and_ragged_shapes(layout, dtype, T, Hq, Hk):
@@ -176,7 +186,7 @@ def test_small_and_ragged_shapes(layout, dtype, T, Hq, Hk):
     check_layerwise(workloads.random_rows(T, Hq, Hk, dtype, seed=T * 131 + Hq + Hk, **kw))
 
 
-@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("dtype", ALL_DTYPES)
 def test_padding_columns_untouched(dtype):
     Hq, Hk = 203, 43  # ragged: neither is a whole number of 16-byte vectors
     b = workloads.random_rows(9, Hq, Hk, dtype, seed=3, q_stride=aligned_stride(Hq, dtype, 3),
@@ -188,7 +198,7 @@ def test_padding_columns_untouched(dtype):
     assert torch.all(qd[:, Hq:].float() == -7.0) and torch.all(kd[:, Hk:].float() == -7.0)
 
 
-@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("dtype", ALL_DTYPES)
 def test_unaligned_buffers_use_the_scalar_kernel(dtype):
     b = workloads.random_rows(13, 301, 77, dtype, seed=4, q_stride=301, k_stride=77)
     q, k, _ = upload(b)
@@ -207,7 +217,8 @@ def test_unaligned_buffers_use_the_scalar_kernel(dtype):
     assert_close(qo, yq, eq, "shifted Q")
 
 
-@pytest.mark.parametrize("dtype,H", [(torch.bfloat16, 20000), (torch.float32, 9000)])
+@pytest.mark.parametrize("dtype,H", [(torch.bfloat16, 20000), (torch.float32, 9000), (torch.float16, 20000),
+                                     (torch.float8_e4m3fn, 40000)])
 def test_rows_too_wide_for_registers(dtype, H):
     b = workloads.random_rows(6, H, 64, dtype, seed=5)
     q, k, _ = upload(b)
@@ -254,11 +265,11 @@ def _cover(launch: dict, units: int) -> dict | None:
 
 
 @pytest.mark.parametrize("launch", VARIANTS, ids=lambda L: "k{kernel}_nv{vec_per_thread}_t{threads}_g{grid}".format(**L))
-@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("dtype", ALL_DTYPES)
 @pytest.mark.parametrize("Hk", [1000, 1003])
 def test_every_kernel_variant_matches_the_oracle_and_is_deterministic(launch, dtype, Hk):
     """Hk = 1003 leaves K rows with a ragged last vector (padded, aligned stride)."""
-    per = 4 if dtype == torch.float32 else 8
+    per = 16 // esz(dtype)
     launch = _cover(launch, -(-4096 // per))
     if launch is None:
         pytest.skip("no CTA of this vec_per_thread covers the fp32 row")
@@ -292,22 +303,22 @@ SHARD_LAUNCHES = [
 @pytest.mark.parametrize("launch", SHARD_LAUNCHES, ids=lambda L: "default" if L is None else
                          "k{kernel}_nv{vec_per_thread}_t{threads}_g{grid}".format(**L))
 @pytest.mark.parametrize("dtype,Hq,Hk,P", [(torch.bfloat16, 5120, 1024, 4), (torch.float32, 1200, 260, 4),
-                                           (torch.bfloat16, 1000, 200, 5)])
+                                           (torch.bfloat16, 1000, 200, 5), (torch.float16, 5120, 1024, 4),
+                                           (torch.float8_e4m3fn, 5120, 1024, 4)])
 def test_shard_pipeline_launch_variants(launch, dtype, Hq, Hk, P):
     """partial_stats then combine_apply over P shards, each with a pinned
     launch, against the oracle's full-row normalization."""
-    per = 4 if dtype == torch.float32 else 8
+    per = 16 // esz(dtype)
     wq, wk = Hq // P, Hk // P
     if launch is not None and launch["kernel"] == 0 and launch["vec_per_thread"] * launch["threads"] < -(-wq // per):
         pytest.skip("launch does not cover a shard row")
-    if launch is not None and launch["kernel"] in (0, 1) and ((wq * (4 if dtype == torch.float32 else 2)) % 16
-                                                             or (wk * (4 if dtype == torch.float32 else 2)) % 16):
+    if launch is not None and launch["kernel"] in (0, 1) and ((wq * esz(dtype)) % 16 or (wk * esz(dtype)) % 16):
         pytest.skip("vector kernels need 16-byte aligned shard strides")
     T = 131
     g = torch.Generator().manual_seed(Hq + Hk + P)
     q = (torch.randn((T, Hq), generator=g) * 2).to(dtype)
     k = (torch.randn((T, Hk), generator=g) * 0.5).to(dtype)
-    gq = workloads.gamma(Hq, 5, dtype)
+    gq = workloads.gamma(Hq, 5, dtype)  # bf16 for E4M3 activations
     gk = workloads.gamma(Hk, 6, dtype)
     qs = [q[:, i * wq:(i + 1) * wq].contiguous().to(DEV) for i in range(P)]
     ks = [k[:, i * wk:(i + 1) * wk].contiguous().to(DEV) for i in range(P)]

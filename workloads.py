@@ -49,9 +49,11 @@ def _normal_rows(gen: torch.Generator, T: int, H: int, dtype: torch.dtype,
 
 
 def gamma(H: int, seed: int, dtype: torch.dtype) -> torch.Tensor:
-    """Learnable-scale stand-in: 1 + 0.1 * N(0, 1), rounded once to ``dtype``."""
+    """Learnable-scale stand-in: 1 + 0.1 * N(0, 1), rounded once to the gamma
+    type that goes with activations of ``dtype`` (bfloat16 for FP8 E4M3)."""
     g = _gen(seed)
-    return (1.0 + 0.1 * torch.randn((H,), generator=g, dtype=torch.float32)).to(dtype)
+    gdt = torch.bfloat16 if dtype == torch.float8_e4m3fn else dtype
+    return (1.0 + 0.1 * torch.randn((H,), generator=g, dtype=torch.float32)).to(gdt)
 
 
 @dataclass
@@ -115,17 +117,20 @@ def tiny_fp32(seed: int = 0, T: int = 64, H: int = 512) -> QKBatch:
                    gamma(H, seed + 100, torch.float32), gamma(H, seed + 200, torch.float32))
 
 
-def prefill_bf16(seed: int = 1, T: int = 4096, H: int = 4096) -> QKBatch:
-    """OLMo2-7B-shaped prefill: T=4096, Hq=Hk=4096 (MHA), bf16.
-    x = N(0,1) * s_t with one scale per token s_t = exp(U(ln 0.1, ln 10)),
-    shared by the token's Q and K rows."""
+_DT_NAME = {torch.bfloat16: "bf16", torch.float16: "f16", torch.float32: "f32", torch.float8_e4m3fn: "e4m3"}
+
+
+def prefill_bf16(seed: int = 1, T: int = 4096, H: int = 4096, dtype: torch.dtype = torch.bfloat16) -> QKBatch:
+    """OLMo2-7B-shaped prefill: T=4096, Hq=Hk=4096 (MHA), bf16 (other element
+    types on request).  x = N(0,1) * s_t with one scale per token
+    s_t = exp(U(ln 0.1, ln 10)), shared by the token's Q and K rows."""
     g = _gen(seed)
     u = torch.rand((T,), generator=g, dtype=torch.float32)
     s = torch.exp(math.log(0.1) + u * (math.log(10.0) - math.log(0.1)))
-    q = _normal_rows(g, T, H, torch.bfloat16, row_scale=s)
-    k = _normal_rows(g, T, H, torch.bfloat16, row_scale=s)
-    return QKBatch(f"prefill_bf16_T{T}_H{H}", torch.bfloat16, T, H, H, q, k,
-                   gamma(H, seed + 100, torch.bfloat16), gamma(H, seed + 200, torch.bfloat16),
+    q = _normal_rows(g, T, H, dtype, row_scale=s)
+    k = _normal_rows(g, T, H, dtype, row_scale=s)
+    return QKBatch(f"prefill_{_DT_NAME[dtype]}_T{T}_H{H}", dtype, T, H, H, q, k,
+                   gamma(H, seed + 100, dtype), gamma(H, seed + 200, dtype),
                    meta={"row_scale": "LogUniform(0.1, 10) per token"})
 
 
