@@ -10,6 +10,8 @@ This module only marshals numpy arrays into the plain C oracle
 * ``rmsnorm_rows``   — RMS-Norm over full rows (Background, Equation 1 of
   "SwiftQK: Fast and Communication-Efficient Tensor Parallelism for Query-Key
   Normalization"); the FP64 gold of Fig. 2(b).
+* ``rmsnorm_heads``  — headwise RMS-Norm (one factor per attention head, the
+  other granularity the Background section names), gamma shared by the heads.
 * ``partial_sumsq``  — Phase A's per-shard squared sum.
 * ``combine_apply``  — Phase A's aggregation of the shard sums, then Phase B's
   weight multiplication and global RMS scaling of one shard.
@@ -66,6 +68,8 @@ def _load():
     lib.oracle_qknorm_layerwise.argtypes = [vp, i64, vp, i32, vp, i64, vp, i32,
                                             i64, dbl, ctypes.c_int, vp, vp]
     lib.oracle_qknorm_layerwise.restype = ctypes.c_int
+    lib.oracle_rmsnorm_heads.argtypes = [vp, i64, i64, i32, i32, vp, dbl, ctypes.c_int, vp, vp]
+    lib.oracle_rmsnorm_heads.restype = ctypes.c_int
     lib.oracle_partial_sumsq.argtypes = [vp, i64, i64, i32, ctypes.c_int, vp]
     lib.oracle_partial_sumsq.restype = ctypes.c_int
     lib.oracle_combine_apply.argtypes = [vp, i64, i64, i32, vp, vp, i32, i32, dbl,
@@ -192,6 +196,27 @@ def qknorm_layerwise(q: np.ndarray, q_stride: int, gamma_q: np.ndarray, Hq: int,
     return q_out, k_out
 
 
+def rmsnorm_heads(x: np.ndarray, n_heads: int, head_dim: int, gamma: np.ndarray, eps: float,
+                  stride: int, T: int):
+    """Headwise RMS-Norm: each of the n_heads heads of head_dim elements in a
+    row is normalized on its own with the shared gamma [head_dim].  Returns
+    ``(y, y_exact)`` of shape ``(T, n_heads * head_dim)``."""
+    lib = _load()
+    dt = _dtype_code(x)
+    W = n_heads * head_dim
+    _check_rows(x, stride, T, W)
+    g = np.ascontiguousarray(gamma)
+    if g.dtype != _gamma_dtype(x.dtype) or g.size < head_dim:
+        raise ValueError("gamma must have the gamma type of the input and head_dim elements")
+    y = np.zeros((T, W), dtype=x.dtype)
+    y_exact = np.zeros((T, W), dtype=np.float64)
+    st = lib.oracle_rmsnorm_heads(_ptr(x), stride, T, n_heads, head_dim, _ptr(g), float(eps), dt,
+                                  _ptr(y), _ptr(y_exact))
+    if st != 0:
+        raise ValueError(f"oracle_rmsnorm_heads rejected its arguments (status {st})")
+    return y, y_exact
+
+
 def partial_sumsq(x: np.ndarray, h_shard: int, stride: int, T: int) -> np.ndarray:
     """Phase A local step: float64 squared sum of each row's first ``h_shard`` columns."""
     lib = _load()
@@ -229,5 +254,5 @@ def version() -> int:
 
 
 __all__ = ["F32", "BF16", "F16", "E4M3", "bf16_decode", "bf16_encode", "f16_decode", "f16_encode",
-           "e4m3_decode", "e4m3_encode", "rmsnorm_rows", "qknorm_layerwise", "partial_sumsq",
+           "e4m3_decode", "e4m3_encode", "rmsnorm_rows", "rmsnorm_heads", "qknorm_layerwise", "partial_sumsq",
            "combine_apply", "version"]

@@ -297,6 +297,49 @@ int oracle_qknorm_layerwise(const void *q, int64_t q_stride, const void *gamma_q
 }
 
 /*
+ * Headwise QK-Norm (Background: "headwise QK-Norm computes an independent
+ * factor for each attention head"): token t's row of one tensor holds
+ * n_heads heads of head_dim elements each, head h at columns
+ * [h * head_dim, (h + 1) * head_dim).  Each head is RMS-normalized on its own
+ * over head_dim elements, with one gamma of length head_dim shared by every
+ * head (the reading taken: the pages do not say how gamma is laid out):
+ *   S_th = sum_{j < head_dim} x_t,h*hd+j ^2,  r_th = 1 / sqrt(S_th / head_dim + eps),
+ *   y_t,h*hd+j = (x_t,h*hd+j * gamma_j) * r_th.
+ * Output is contiguous [T][n_heads * head_dim].
+ */
+int oracle_rmsnorm_heads(const void *x, int64_t x_stride, int64_t T, int32_t n_heads, int32_t head_dim,
+                         const void *gamma, double eps, int dtype, void *y_out, double *y_exact)
+{
+    if (T < 0 || n_heads <= 0 || head_dim <= 0 || x_stride < (int64_t)n_heads * head_dim || bad_dtype(dtype) ||
+        !(eps >= 0.0))
+        return ORACLE_BAD_ARG;
+    if (T > 0 && (!x || !gamma))
+        return ORACLE_BAD_ARG;
+    const int64_t W = (int64_t)n_heads * head_dim;
+    for (int64_t t = 0; t < T; ++t) {
+        for (int32_t h = 0; h < n_heads; ++h) {
+            const int64_t c0 = (int64_t)h * head_dim;
+            double S = 0.0;
+            for (int32_t j = 0; j < head_dim; ++j) {
+                double v = load_elem(x, dtype, t * x_stride + c0 + j);
+                S += v * v;
+            }
+            double r = 1.0 / sqrt(S / (double)head_dim + eps);
+            for (int32_t j = 0; j < head_dim; ++j) {
+                double v = load_elem(x, dtype, t * x_stride + c0 + j);
+                double g = load_elem(gamma, gamma_dtype(dtype), j);
+                double yv = (v * g) * r;
+                if (y_exact)
+                    y_exact[t * W + c0 + j] = yv;
+                if (y_out)
+                    store_elem(y_out, dtype, t * W + c0 + j, yv);
+            }
+        }
+    }
+    return ORACLE_OK;
+}
+
+/*
  * Phase A, local step: the squared sum of each token's row restricted to one
  * hidden-dimension shard of width h_shard.  sumsq[t] = sum_{j < h_shard} x_tj^2.
  */

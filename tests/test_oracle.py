@@ -204,6 +204,46 @@ def test_layerwise_treats_q_and_k_independently():
     np.testing.assert_allclose(ko, rk.numpy(), rtol=2e-7)
 
 
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16, torch.float8_e4m3fn])
+@pytest.mark.parametrize("T,nh,hd,pad", [(1, 1, 1, 0), (5, 4, 8, 3), (3, 32, 128, 16), (7, 3, 7, 0)])
+def test_headwise_matches_torch_rms_norm_over_heads(dtype, T, nh, hd, pad):
+    """Headwise RMS-Norm is rms_norm over the last axis of the [T, n_heads,
+    head_dim] view, gamma [head_dim] broadcast over heads (a library routine)."""
+    g = torch.Generator().manual_seed(31 + T + nh + hd)
+    W = nh * hd
+    buf = (torch.randn((T, W + pad), generator=g) * 2).to(dtype)
+    view = buf[:, :W]
+    gdt = torch.bfloat16 if dtype == torch.float8_e4m3fn else dtype
+    gm = (1 + 0.1 * torch.randn((hd,), generator=g)).to(gdt)
+    flat, st = buffer_np(view)
+    y_r, y = oracle.rmsnorm_heads(flat, nh, hd, to_np(gm), 1e-6, stride=st, T=T)
+    ref = torch.nn.functional.rms_norm(view.double().reshape(T, nh, hd), (hd,), weight=gm.double(), eps=1e-6)
+    np.testing.assert_allclose(y, ref.reshape(T, W).numpy(), rtol=1e-13, atol=1e-300)
+
+
+def test_headwise_with_one_head_is_layerwise_and_heads_are_independent():
+    g = torch.Generator().manual_seed(32)
+    T, nh, hd = 4, 6, 16
+    x = torch.randn((T, nh * hd), generator=g)
+    gm = 1 + 0.1 * torch.randn((hd,), generator=g)
+    # one head spanning the row equals the layerwise form
+    _, y1 = oracle.rmsnorm_heads(to_np(x), 1, nh * hd, to_np(gm.repeat(nh)), 1e-6, stride=nh * hd, T=T)
+    _, yl, _ = oracle.rmsnorm_rows(to_np(x), nh * hd, to_np(gm.repeat(nh)), 1e-6)
+    np.testing.assert_allclose(y1, yl, rtol=1e-15)
+    # scaling one head leaves every other head's output unchanged (eps = 0: the scaled head is unchanged too)
+    x2 = x.clone()
+    x2[:, 2 * hd:3 * hd] *= 64.0
+    _, ya = oracle.rmsnorm_heads(to_np(x), nh, hd, to_np(gm), 0.0, stride=nh * hd, T=T)
+    _, yb = oracle.rmsnorm_heads(to_np(x2), nh, hd, to_np(gm), 0.0, stride=nh * hd, T=T)
+    assert np.array_equal(ya, yb)
+    # the per-head closed form: a head of constant c normalizes to gamma * c / sqrt(c^2 + eps)
+    x3 = torch.zeros((1, nh * hd))
+    x3[0, hd:2 * hd] = 0.5
+    _, y3 = oracle.rmsnorm_heads(to_np(x3), nh, hd, to_np(torch.ones(hd)), 0.25, stride=nh * hd, T=1)
+    np.testing.assert_allclose(y3[0, hd:2 * hd], 0.5 / math.sqrt(0.5), rtol=1e-15)
+    assert np.count_nonzero(y3[0, :hd]) == 0 and np.count_nonzero(y3[0, 2 * hd:]) == 0
+
+
 # --------------------------------------------------------------------------- invariants
 
 @pytest.mark.parametrize("eps_ratio", [0.0, 1e-6, 1.0, 37.0])

@@ -34,6 +34,9 @@ MUTANTS = [
     ("f16_encode_bias", "((er - 1 + 15) << 10)", "((er - 1 + 14) << 10)", None),
     ("f16_subnormal_threshold", "round_to_grid(a, 11, -14)", "round_to_grid(a, 11, -15)", None),
     ("gamma_type_e4m3", "return dtype == ORACLE_E4M3 ? ORACLE_BF16 : dtype;", "return dtype;", None),
+    ("heads_divide_by_row_width", "sqrt(S / (double)head_dim + eps)", "sqrt(S / (double)W + eps)", None),
+    ("heads_gamma_by_column", "double g = load_elem(gamma, gamma_dtype(dtype), j);\n                double yv",
+     "double g = load_elem(gamma, gamma_dtype(dtype), c0 + j);\n                double yv", None),
     ("stride_ignored", "double v = load_elem(x, dtype, t * x_stride + j);\n            double g",
      "double v = load_elem(x, dtype, t * (int64_t)H + j);\n            double g", 1),
     ("drop_last_shard", "for (int32_t p = 0; p < P; ++p)", "for (int32_t p = 0; p + 1 < P; ++p)", None),
