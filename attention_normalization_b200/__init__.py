@@ -24,7 +24,7 @@ import torch
 from . import _clib
 from ._clib import QknLaunch, QKNormError
 
-__all__ = ["qknorm_layerwise", "qknorm_partial_stats", "qknorm_combine_apply", "gamma_dtype",
+__all__ = ["qknorm_layerwise", "qknorm_headwise", "qknorm_partial_stats", "qknorm_combine_apply", "gamma_dtype",
            "qknorm_layerwise_plan", "qknorm_layerwise_host", "qknorm_packed_host",
            "plan_shape", "plan_grid", "regions_overlap", "capi", "version", "QknLaunch", "QKNormError"]
 
@@ -134,6 +134,44 @@ def qknorm_layerwise(q_in: torch.Tensor, k_in: torch.Tensor, gamma_q: torch.Tens
         else:
             st = lib.qknorm_layerwise_launch(*args, s, ctypes.byref(_launch_struct(launch)))
     _clib.check(st, "qknorm_layerwise")
+    return q_out, k_out
+
+
+def qknorm_headwise(q_in: torch.Tensor, k_in: torch.Tensor, gamma_q: torch.Tensor, gamma_k: torch.Tensor,
+                    head_dim: int, eps: float = 1e-6, *, q_out=None, k_out=None, stream=None,
+                    launch: QknLaunch | dict | None = None):
+    """Headwise QK-Norm: every head of ``head_dim`` elements in the Q rows
+    ``[T, q_heads * head_dim]`` and K rows ``[T, k_heads * head_dim]`` is
+    normalized on its own, gamma ``[head_dim]`` shared by a tensor's heads.
+    One launch for Q and K; returns ``(q_out, k_out)``."""
+    Tq, Wq, sq = _rows(q_in, "q_in")
+    Tk, Wk, sk = _rows(k_in, "k_in")
+    if Tq != Tk:
+        raise ValueError("q_in and k_in must have the same number of tokens")
+    if head_dim < 1 or Wq % head_dim or Wk % head_dim:
+        raise ValueError("row widths must be whole numbers of heads of head_dim elements")
+    dev, dt = q_in.device, q_in.dtype
+    _same(dev, dt, k_in, "k_in")
+    if q_out is None:
+        q_out = _out_like(q_in, sq)
+    if k_out is None:
+        k_out = _out_like(k_in, sk)
+    for t, name, (T, W, s) in ((q_out, "q_out", (Tq, Wq, sq)), (k_out, "k_out", (Tk, Wk, sk))):
+        _same(dev, dt, t, name)
+        To, Wo, so = _rows(t, name)
+        if (To, Wo) != (T, W) or (T > 1 and so != s):
+            raise ValueError(f"{name} must match its input's shape and row stride")
+    gdt = gamma_dtype(dt)
+    args = [q_in.data_ptr(), q_out.data_ptr(), _vec(gamma_q, "gamma_q", head_dim, gdt, dev), sq, Wq // head_dim,
+            k_in.data_ptr(), k_out.data_ptr(), _vec(gamma_k, "gamma_k", head_dim, gdt, dev), sk, Wk // head_dim,
+            Tq, int(head_dim), float(eps), _DTYPES[dt]]
+    with torch.cuda.device(dev):
+        s = _stream_handle(stream, dev)
+        if launch is None:
+            st = capi().qknorm_headwise(*args, s)
+        else:
+            st = capi().qknorm_headwise_launch(*args, s, ctypes.byref(_launch_struct(launch)))
+    _clib.check(st, "qknorm_headwise")
     return q_out, k_out
 
 

@@ -41,10 +41,13 @@ _vp, _i64, _i32, _u64, _f32 = (ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32,
 _dt = ctypes.c_int
 _st = ctypes.c_int
 _LAYERWISE_ARGS = [_vp, _vp, _vp, _i64, _vp, _vp, _vp, _i64, _i64, _i32, _i32, _f32, _dt]
+_HEADWISE_ARGS = [_vp, _vp, _vp, _i64, _i32, _vp, _vp, _vp, _i64, _i32, _i64, _i32, _f32, _dt]
 
 PROTOTYPES = {
     "qknorm_layerwise": (_st, _LAYERWISE_ARGS + [_vp]),
     "qknorm_partial_stats": (_st, [_vp, _i64, _i32, _vp, _vp, _i64, _i32, _vp, _i64, _dt, _vp]),
+    "qknorm_headwise": (_st, _HEADWISE_ARGS + [_vp]),
+    "qknorm_headwise_launch": (_st, _HEADWISE_ARGS + [_vp, ctypes.POINTER(QknLaunch)]),
     "qknorm_combine_apply": (_st, [_vp, _vp, _vp, _i64, _i32, _vp, _i32,
                                    _vp, _vp, _vp, _i64, _i32, _vp, _i32,
                                    _i32, _i64, _f32, _dt, _vp]),

@@ -232,12 +232,20 @@ void fill_rowset(qkn::RowSet &s, const void *in, void *out, const void *gamma, i
     s.nfull = width / per_vec;
     s.tail = width % per_vec;
     s.inv_div = static_cast<float>(1.0 / static_cast<double>(div_width));
+    s.heads = 1;
+    s.head_bytes = 0;
+    s.rows = 0;
 }
 
 void finish_call(Call &c, int esz, std::initializer_list<const void *> ptrs, int64_t q_stride, int64_t k_stride) {
     bool v = ((q_stride * esz) % 16 == 0) && ((k_stride * esz) % 16 == 0);
     for (const void *p : ptrs)
         if (p && !aligned16(p)) v = false;
+    for (int w = 0; w < 2; ++w) {
+        qkn::RowSet &d = c.p.set[w];
+        d.rows = c.p.T * d.heads;
+        if (d.heads > 1 && d.head_bytes % 16 != 0) v = false;  // every head must start on a vector
+    }
     c.vectorized = v;
     const int per_vec = 16 / esz;
     int64_t wq = c.p.set[0].width, wk = c.p.set[1].width;
@@ -254,14 +262,14 @@ void set_groups(qkn::Params &p, int threads, int nv) {
         qkn::RowSet &d = p.set[w];
         const int64_t units = (int64_t)d.nfull + (d.tail ? 1 : 0);
         int group = threads;
-        for (int g = 32; g < threads; g += 32)
+        for (int g = 1; g < threads; g = g < 32 ? g * 2 : g + 32)
             if (threads % g == 0 && (int64_t)g * nv >= units) {
                 group = g;
                 break;
             }
         d.group = group;
         d.rows_per_item = threads / group;
-        d.items = (p.T + d.rows_per_item - 1) / d.rows_per_item;
+        d.items = (d.rows + d.rows_per_item - 1) / d.rows_per_item;
     }
 }
 
@@ -343,7 +351,7 @@ qkn_status plan_call(const Call &c, qkn_launch &L) {
     qkn_status st = current_device(&dev);
     if (st != QKN_OK) return st;
     if ((st = sm_count(dev, &sms)) != QKN_OK) return st;
-    const int64_t items = 2 * c.p.T;
+    const int64_t items = c.p.set[0].rows + c.p.set[1].rows;
     if ((st = qknorm_plan_shape(items, c.units_max, c.vectorized ? 1 : 0, sms, elem_bytes(c.dtype), &L)) !=
         QKN_OK)
         return fail(st, "planning failed");
@@ -495,6 +503,50 @@ qkn_status prepare_apply(const void *q_in, void *q_out, const void *gamma_q_shar
     return QKN_OK;
 }
 
+qkn_status prepare_headwise(const void *q_in, void *q_out, const void *gamma_q, int64_t q_stride, int32_t q_heads,
+                            const void *k_in, void *k_out, const void *gamma_k, int64_t k_stride, int32_t k_heads,
+                            int64_t T, int32_t head_dim, float eps, qkn_dtype dtype, Call &c) {
+    if (q_heads <= 0 || k_heads <= 0 || head_dim <= 0)
+        return fail(QKN_ERR_INVALID_ARG, "heads and head_dim must be positive");
+    const int64_t wq = (int64_t)q_heads * head_dim, wk = (int64_t)k_heads * head_dim;
+    if (wq > INT32_MAX || wk > INT32_MAX) return fail(QKN_ERR_INVALID_ARG, "row width overflows");
+    if (T > 0 && ((int64_t)T * q_heads >= ((int64_t)1 << 31) || (int64_t)T * k_heads >= ((int64_t)1 << 31)))
+        return fail(QKN_ERR_INVALID_ARG, "T * heads must stay below 2^31");
+    // Validate the whole rows as the layerwise form does (sizes, strides, overlaps),
+    // with gamma regions of head_dim elements.
+    if (!dtype_valid(dtype)) return fail(QKN_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
+    if (T < 0) return fail(QKN_ERR_INVALID_ARG, "T = %lld < 0", (long long)T);
+    if (q_stride < wq || k_stride < wk) return fail(QKN_ERR_INVALID_ARG, "row stride below heads * head_dim");
+    if (!eps_valid(eps)) return fail(QKN_ERR_INVALID_ARG, "eps must be finite and >= 0");
+    const int esz = elem_bytes(dtype);
+    if (!extent_ok(T, q_stride, wq, esz) || !extent_ok(T, k_stride, wk, esz))
+        return fail(QKN_ERR_INVALID_ARG, "buffer extent overflows");
+    if (T > 0 && (!q_in || !q_out || !gamma_q || !k_in || !k_out || !gamma_k))
+        return fail(QKN_ERR_INVALID_ARG, "null pointer");
+    if (T > 0) {
+        const Region iq = rows_region(q_in, wq, q_stride, T, esz), oq = rows_region(q_out, wq, q_stride, T, esz);
+        const Region ik = rows_region(k_in, wk, k_stride, T, esz), ok_ = rows_region(k_out, wk, k_stride, T, esz);
+        const int gsz = gamma_bytes(dtype);
+        const Region others[2] = {flat_region(gamma_q, (int64_t)head_dim * gsz),
+                                  flat_region(gamma_k, (int64_t)head_dim * gsz)};
+        qkn_status st = check_outputs(oq, ok_, iq, ik, others, 2);
+        if (st != QKN_OK) return st;
+    }
+    std::memset(&c, 0, sizeof(c));
+    c.dtype = dtype;
+    fill_rowset(c.p.set[0], q_in, q_out, gamma_q, q_stride, head_dim, head_dim, esz);
+    fill_rowset(c.p.set[1], k_in, k_out, gamma_k, k_stride, head_dim, head_dim, esz);
+    c.p.set[0].heads = q_heads;
+    c.p.set[1].heads = k_heads;
+    c.p.set[0].head_bytes = (int64_t)head_dim * esz;
+    c.p.set[1].head_bytes = (int64_t)head_dim * esz;
+    c.p.T = T;
+    c.p.eps = eps;
+    c.p.P = 1;
+    finish_call(c, esz, {q_in, q_out, gamma_q, k_in, k_out, gamma_k}, q_stride, k_stride);
+    return QKN_OK;
+}
+
 }  // namespace
 
 // ===========================================================================
@@ -533,13 +585,21 @@ qkn_status qknorm_plan_shape(int64_t rows, int64_t units_max, int32_t vectorized
     }
     L.kernel = QKN_KERNEL_REGISTER;
     int nv;
+    bool narrow = false;
     if (rows <= sm_count) {
         // Few rows (decode): spread each row over many threads so a row costs
         // about one memory round trip (two vectors per thread measured best).
         nv = units_max < 128 ? 1 : 2;
+    } else if (units_max < 64) {
+        // Many narrow rows (attention heads, thin shards): a few lanes per row
+        // with up to four vectors each, so every thread keeps 64 bytes in
+        // flight, and several rows per warp.
+        narrow = true;
+        nv = 1;
+        while (nv < 4 && nv < units_max) nv *= 2;
     } else {
         // Many rows: moderate CTAs, several vectors in flight per thread.
-        nv = units_max >= 256 ? 4 : (units_max >= 64 ? 2 : 1);
+        nv = units_max >= 256 ? 4 : 2;
     }
     // A 16-byte vector of 1-byte elements widens to twice the fp32 registers
     // (and pairs with two gamma vectors): hold half as many per thread.
@@ -549,6 +609,7 @@ qkn_status qknorm_plan_shape(int64_t rows, int64_t units_max, int32_t vectorized
         nv *= 2;
         threads = round32((units_max + nv - 1) / nv);
     }
+    if (narrow) threads = 256;  // a CTA holds many row groups
     L.vec_per_thread = nv;
     L.threads = threads;
     *out = L;
@@ -609,6 +670,33 @@ qkn_status qknorm_layerwise_launch(const void *q_in, void *q_out, const void *ga
     Call c;
     qkn_status st = prepare_layerwise(q_in, q_out, gamma_q, q_stride, k_in, k_out, gamma_k, k_stride, T, Hq,
                                       Hk, eps, dtype, c);
+    if (st != QKN_OK) return st;
+    if ((st = check_launch(c, *launch_cfg)) != QKN_OK) return st;
+    if (T == 0) return ok();
+    return launch<qkn::kFused>(c, *launch_cfg, stream);
+}
+
+qkn_status qknorm_headwise(const void *q_in, void *q_out, const void *gamma_q, int64_t q_stride, int32_t q_heads,
+                           const void *k_in, void *k_out, const void *gamma_k, int64_t k_stride, int32_t k_heads,
+                           int64_t T, int32_t head_dim, float eps, qkn_dtype dtype, void *stream) {
+    Call c;
+    qkn_status st = prepare_headwise(q_in, q_out, gamma_q, q_stride, q_heads, k_in, k_out, gamma_k, k_stride,
+                                     k_heads, T, head_dim, eps, dtype, c);
+    if (st != QKN_OK) return st;
+    if (T == 0) return ok();
+    qkn_launch L;
+    if ((st = plan_call<qkn::kFused>(c, L)) != QKN_OK) return st;
+    return launch<qkn::kFused>(c, L, stream);
+}
+
+qkn_status qknorm_headwise_launch(const void *q_in, void *q_out, const void *gamma_q, int64_t q_stride,
+                                  int32_t q_heads, const void *k_in, void *k_out, const void *gamma_k,
+                                  int64_t k_stride, int32_t k_heads, int64_t T, int32_t head_dim, float eps,
+                                  qkn_dtype dtype, void *stream, const qkn_launch *launch_cfg) {
+    if (!launch_cfg) return fail(QKN_ERR_INVALID_ARG, "null launch");
+    Call c;
+    qkn_status st = prepare_headwise(q_in, q_out, gamma_q, q_stride, q_heads, k_in, k_out, gamma_k, k_stride,
+                                     k_heads, T, head_dim, eps, dtype, c);
     if (st != QKN_OK) return st;
     if ((st = check_launch(c, *launch_cfg)) != QKN_OK) return st;
     if (T == 0) return ok();

@@ -44,9 +44,12 @@ struct RowSet {
     int32_t nfull;           // full 16-byte vectors of x in the row
     int32_t tail;            // elements after the last full vector
     float inv_div;           // 1 / (the FULL width), rounded to fp32 on the host
-    int32_t group;           // register kernel: threads that share one row (a multiple of 32)
+    int32_t heads;           // rows per token: 1 (layerwise) or the number of heads (headwise)
+    int64_t head_bytes;      // headwise: bytes from one head to the next within a token's row
+    int64_t rows;            // T * heads
+    int32_t group;           // register kernel: threads that share one row (1..16, or a multiple of 32)
     int32_t rows_per_item;   // register kernel: blockDim / group rows handled per item
-    int64_t items;           // register kernel: ceil(T / rows_per_item)
+    int64_t items;           // register kernel: ceil(rows / rows_per_item)
 };
 
 struct Params {
@@ -279,6 +282,24 @@ __device__ __forceinline__ float warp_sum(float v) {
     return v;
 }
 
+// Sum over aligned groups of `g` lanes (g a power of two below 32): butterfly
+// with offsets g/2 .. 1 keeps the groups apart.
+__device__ __forceinline__ float segment_sum(float v, int g) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1)
+        if (off < g) v += __shfl_xor_sync(0xFFFFFFFFu, v, off);
+    return v;
+}
+
+// Row r of a tensor -> the byte offset of its first element: token r / heads,
+// head r % heads.
+__device__ __forceinline__ int64_t row_offset(int64_t r, int heads, int64_t stride, int64_t head_bytes) {
+    if (heads == 1) return r * stride;
+    const uint32_t rr = static_cast<uint32_t>(r);  // headwise rows are fewer than 2^31 (host check)
+    const uint32_t t = rr / static_cast<uint32_t>(heads);
+    return static_cast<int64_t>(t) * stride + static_cast<int64_t>(rr - t * heads) * head_bytes;
+}
+
 // `red` has two slots of 32 floats; alternating slots between consecutive rows
 // lets one barrier per row suffice: a thread can only overwrite slot s after
 // every thread has passed the barrier of the row in between, i.e. after all
@@ -359,8 +380,9 @@ __device__ __forceinline__ uint4 scale_vec(const uint4 &xv, const uint4 (&gv)[El
 // ----------------------------------------------------------------------------
 // One-pass register kernel.
 //
-// A row is handled by a group of `group` threads (a multiple of 32 that
-// divides the CTA); a CTA of blockDim threads therefore handles
+// A row (a token's Q or K row, or one head of it) is handled by a group of
+// `group` threads -- 1, 2, 4, 8 or 16 lanes of a warp, or a multiple of 32
+// that divides the CTA; a CTA of blockDim threads therefore handles
 // rows_per_item = blockDim / group consecutive rows of one tensor per item.
 // Items are the Q row-groups followed by the K row-groups, and CTA c takes
 // items c, c + grid, ...: every CTA gets a near-equal share of each tensor's
@@ -368,9 +390,10 @@ __device__ __forceinline__ uint4 scale_vec(const uint4 &xv, const uint4 (&gv)[El
 // (up to NV) of its row -- the same positions in every row -- so while
 // consecutive items belong to one tensor a thread keeps that tensor's
 // parameters and its gamma vectors in registers.  All loads of a row are
-// issued before any is used.  A one-warp group reduces with shuffles only;
-// wider groups add one CTA barrier per item.  Narrow rows (e.g. K beside a
-// wide Q) thus share a CTA instead of each paying for a whole one.
+// issued before any is used.  A group of up to one warp reduces with shuffles
+// only; wider groups add one CTA barrier per item.  Narrow rows (a K row
+// beside a wide Q row, an attention head) thus share a CTA -- or a warp --
+// instead of each paying for a whole one.
 // TAIL: some row ends in a partial vector (otherwise the tail code is
 // compiled out).
 template <int NV>
@@ -397,8 +420,8 @@ __global__ void __launch_bounds__(RegisterBounds<NV>::kMaxThreads)
     char *out = nullptr;
     float *sums = nullptr;
     const float *sums_all = nullptr;
-    int64_t stride = 0;
-    int nfull = 0, tail = 0, gsize = 32, rpi = 1, grp = 0, gl = 0, gwarps = 1;
+    int64_t stride = 0, head_bytes = 0, rows = 0;
+    int nfull = 0, tail = 0, gsize = 32, rpi = 1, grp = 0, gl = 0, gwarps = 1, heads = 1;
     float inv_div = 0.0f;
     uint4 g[NV][KG];
 
@@ -413,6 +436,9 @@ __global__ void __launch_bounds__(RegisterBounds<NV>::kMaxThreads)
             sums = d.sumsq;
             sums_all = d.sumsq_all;
             stride = d.stride_bytes;
+            head_bytes = d.head_bytes;
+            heads = d.heads;
+            rows = d.rows;
             nfull = d.nfull;
             tail = TAIL ? d.tail : 0;
             inv_div = d.inv_div;
@@ -426,9 +452,10 @@ __global__ void __launch_bounds__(RegisterBounds<NV>::kMaxThreads)
                 for (int i = 0; i < NV; ++i) ld_gamma_vec<E>(d.gamma, gl + i * gsize, nfull, tail, g[i]);
             }
         }
-        const int64_t t = j * rpi + grp;
-        const bool active = t < T;
-        const char *row = in + t * stride;
+        const int64_t t = j * rpi + grp;  // row index within the tensor (= token when heads == 1)
+        const bool active = t < rows;
+        const int64_t roff = active ? row_offset(t, heads, stride, head_bytes) : 0;
+        const char *row = in + roff;
         uint4 v[NV];
 #pragma unroll
         for (int i = 0; i < NV; ++i) {
@@ -446,7 +473,8 @@ __global__ void __launch_bounds__(RegisterBounds<NV>::kMaxThreads)
         if (MODE == kApply) {
             r = active ? rms_factor(combine_partials(sums_all, T, p.P, t), inv_div, p.eps) : 0.0f;
         } else {
-            float S = warp_sum(sumsq_pairs<E, NV>(v));
+            float S = sumsq_pairs<E, NV>(v);
+            S = gsize < 32 ? segment_sum(S, gsize) : warp_sum(S);
             if (gwarps > 1) {  // uniform: the whole CTA takes this branch
                 if (lane == 0) red[slot][warp] = S;
                 __syncthreads();
@@ -462,7 +490,7 @@ __global__ void __launch_bounds__(RegisterBounds<NV>::kMaxThreads)
         }
         if (!active) continue;
         const F2 r2 = f2(r, r);
-        char *orow = out + t * stride;
+        char *orow = out + roff;
 #pragma unroll
         for (int i = 0; i < NV; ++i) {
             const int vi = gl + i * gsize;
@@ -498,11 +526,13 @@ __global__ void __launch_bounds__(1024) rows_twopass_kernel(const __grid_constan
     const int tid = threadIdx.x;
     const int nthr = blockDim.x;
 
-    for (int64_t item = blockIdx.x; item < 2 * p.T; item += gridDim.x) {
-        const int w = item >= p.T ? 1 : 0;
+    const int64_t q_rows = p.set[0].rows;
+    for (int64_t item = blockIdx.x; item < q_rows + p.set[1].rows; item += gridDim.x) {
+        const int w = item >= q_rows ? 1 : 0;
         const RowSet &d = p.set[w];
-        const int64_t t = w ? item - p.T : item;
-        const char *row = d.in + t * d.stride_bytes;
+        const int64_t t = w ? item - q_rows : item;  // row index (= token when heads == 1)
+        const int64_t roff = row_offset(t, d.heads, d.stride_bytes, d.head_bytes);
+        const char *row = d.in + roff;
         const int units = VEC ? d.nfull + (d.tail ? 1 : 0) : d.width;
 
         float r;
@@ -533,7 +563,7 @@ __global__ void __launch_bounds__(1024) rows_twopass_kernel(const __grid_constan
             r = rms_factor(S, d.inv_div, p.eps);
         }
 
-        char *orow = d.out + t * d.stride_bytes;
+        char *orow = d.out + roff;
         for (int u = tid; u < units; u += nthr) {
             if (VEC) {
                 const bool full = u < d.nfull;

@@ -57,7 +57,7 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
-    ap.add_argument("--workload", choices=["prefill", "decode", "packed", "gqa", "tiny"], default="prefill")
+    ap.add_argument("--workload", choices=["prefill", "decode", "packed", "gqa", "tiny", "headwise"], default="prefill")
     ap.add_argument("--tokens", type=int, default=None, help="T for decode / packed workloads")
     ap.add_argument("--dtype", choices=["bf16", "f16", "e4m3"], default="bf16",
                     help="element type of the prefill workload (gamma is bf16 with e4m3)")
@@ -238,11 +238,14 @@ class Workload:
             self.batch = workloads.packed_qkv(tokens or 16384, seed=4 + seed_offset)
         elif kind == "gqa":
             self.batch = workloads.gqa_sharded(seed=3 + seed_offset)
+        elif kind == "headwise":
+            self.batch = workloads.headwise_bf16(seed=5 + seed_offset, T=tokens or 4096)
         b = self.batch
         self.esz = {torch.float32: 4, torch.float8_e4m3fn: 1}.get(b.dtype, 2)
         gesz = 4 if b.dtype == torch.float32 else 2
         # bytes the method must move per step: read + write of every Q and K element, plus gamma
-        self.eff_bytes = 2 * self.esz * (b.Hq + b.Hk) * b.T + gesz * (b.Hq + b.Hk)
+        gamma_elems = 2 * b.meta["head_dim"] if kind == "headwise" else b.Hq + b.Hk
+        self.eff_bytes = 2 * self.esz * (b.Hq + b.Hk) * b.T + gesz * gamma_elems
         self.name = b.name
         self.launches_per_step = 2 * b.P if kind == "gqa" else 1
 
@@ -254,6 +257,9 @@ class Workload:
             c.update({"Hv": b.Hv, "row_stride": b.packed.shape[1], "in_place": True})
         if self.kind == "gqa":
             c.update({"P": b.P, "form": "partial_stats x P -> combine_apply x P"})
+        if self.kind == "headwise":
+            c.update({"head_dim": b.meta["head_dim"], "q_heads": b.meta["q_heads"], "k_heads": b.meta["k_heads"],
+                      "form": "qknorm_headwise (one factor per head)"})
         return c
 
     # one device-resident set of buffers
@@ -294,6 +300,9 @@ class Workload:
             for p in range(b.P):
                 qk.qknorm_combine_apply(s["qs"][p], s["ks"][p], s["gqs"][p], s["gks"][p], s["q_all"], s["k_all"],
                                         b.Hq, b.Hk, b.eps, q_out=s["qo"][p], k_out=s["ko"][p])
+        elif self.kind == "headwise":
+            qk.qknorm_headwise(s["q"], s["k"], s["gq"], s["gk"], b.meta["head_dim"], b.eps,
+                               q_out=s["qo"], k_out=s["ko"])
         else:
             qk.qknorm_layerwise(s["q"], s["k"], s["gq"], s["gk"], b.eps, q_out=s["qo"], k_out=s["ko"])
 
@@ -357,7 +366,11 @@ def time_oracle(wl: Workload, budget_s: float, max_tokens: int | None = None) ->
     gk = np_rows(b.gamma_k[None, :])[0].ravel()
 
     def one_call():
-        if wl.kind == "gqa":
+        if wl.kind == "headwise":
+            hd = b.meta["head_dim"]
+            oracle.rmsnorm_heads(qf, b.Hq // hd, hd, gq, b.eps, stride=b.Hq, T=T)
+            oracle.rmsnorm_heads(kf, b.Hk // hd, hd, gk, b.eps, stride=b.Hk, T=T)
+        elif wl.kind == "gqa":
             P = b.P
             wq, wk = b.Hq // P, b.Hk // P
             sq = np.stack([oracle.partial_sumsq(np.ascontiguousarray(qf[:, p * wq:(p + 1) * wq]), wq, wq, T)
@@ -380,7 +393,7 @@ def time_oracle(wl: Workload, budget_s: float, max_tokens: int | None = None) ->
         if el >= budget_s or calls >= 1000:
             break
     per_call = el / calls
-    eff = 2 * wl.esz * (b.Hq + b.Hk) * T + (4 if b.dtype == torch.float32 else 2) * (b.Hq + b.Hk)
+    eff = wl.eff_bytes * T / b.T
     return {"value": eff / per_call / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle",
             "sample": f"{calls} oracle call(s) on {T} of {b.T} tokens of {wl.name}, {el:.1f} s",
             "us_per_call": per_call * 1e6, "tokens": T, "calls": calls}
@@ -542,6 +555,23 @@ def e2e_measure(qk, wl: Workload, dev, args, barrier, max_over_ranks) -> dict:
         h2d = sum(t.numel() * t.element_size() for t in h_in) + gbytes
         d2h = sum(t.numel() * t.element_size() for t in h_out)
         path = "per-shard pinned host -> device copies, partial_stats x P + combine_apply x P, device -> host copies"
+    elif wl.kind == "headwise":
+        s = wl.make_set(dev)
+        h_q, h_k = b.q.contiguous().pin_memory(), b.k.contiguous().pin_memory()
+        h_qo = torch.empty(h_q.shape, dtype=h_q.dtype, pin_memory=True)
+        h_ko = torch.empty(h_k.shape, dtype=h_k.dtype, pin_memory=True)
+
+        def one():
+            s["q"].copy_(h_q, non_blocking=True)
+            s["k"].copy_(h_k, non_blocking=True)
+            s["gq"].copy_(h_g[0], non_blocking=True)
+            s["gk"].copy_(h_g[1], non_blocking=True)
+            wl.step(qk, s)
+            h_qo.copy_(s["qo"], non_blocking=True)
+            h_ko.copy_(s["ko"], non_blocking=True)
+        h2d = sum(t.numel() * t.element_size() for t in (h_q, h_k)) + gbytes
+        d2h = sum(t.numel() * t.element_size() for t in (h_qo, h_ko))
+        path = "pinned host -> device copies, qknorm_headwise, device -> pinned host copies, one stream"
     else:
         h_q, h_k = b.q.contiguous().pin_memory(), b.k.contiguous().pin_memory()
         h_qo = torch.empty(h_q.shape, dtype=h_q.dtype, pin_memory=True)
@@ -592,7 +622,7 @@ def reference(args) -> int:
     for _ in range(args.steps):
         time_oracle(wl, 0.0, max_tokens=tokens)
     el = time.perf_counter() - t0
-    eff = 2 * wl.esz * (b.Hq + b.Hk) * tokens + (4 if b.dtype == torch.float32 else 2) * (b.Hq + b.Hk)
+    eff = wl.eff_bytes * tokens / b.T
     value = eff / (el / args.steps) / 1e9
     cfg = wl.config()
     cfg.update({"sample_tokens_per_step": tokens})

@@ -129,6 +129,26 @@ qkn_status qknorm_combine_apply(const void *q_in, void *q_out, const void *gamma
                                 int32_t hk_shard, const float *k_sumsq_all, int32_t Hk_full,
                                 int32_t P, int64_t T, float eps, qkn_dtype dtype, void *stream);
 
+/*
+ * Headwise QK-Norm (Background: the other granularity, "an independent factor
+ * for each attention head"): token t's Q row holds q_heads heads of head_dim
+ * elements, head h at columns [h * head_dim, (h + 1) * head_dim); K likewise
+ * with k_heads heads.  Each head is normalized on its own:
+ *       S = sum_j x_j^2 over the head,  r = 1 / sqrt(S / head_dim + eps),
+ *       y_j = (x_j * gamma_j) * r,
+ * with gamma_q [head_dim] shared by all Q heads and gamma_k [head_dim] by all K
+ * heads.  ONE launch for Q and K.  Strides as in qknorm_layerwise (stride >=
+ * heads * head_dim); out == in normalizes in place.  Heads move as 16-byte
+ * vectors when head_dim * element size is a multiple of 16 (and the usual
+ * pointer/stride alignment holds).  Under tensor parallelism whole heads live
+ * on one rank, so the headwise form needs no cross-shard statistics.
+ * Errors: as qknorm_layerwise, plus q_heads, k_heads or head_dim <= 0, or
+ * T * heads >= 2^31.
+ */
+qkn_status qknorm_headwise(const void *q_in, void *q_out, const void *gamma_q, int64_t q_stride, int32_t q_heads,
+                           const void *k_in, void *k_out, const void *gamma_k, int64_t k_stride, int32_t k_heads,
+                           int64_t T, int32_t head_dim, float eps, qkn_dtype dtype, void *stream);
+
 /* Short English name of a status code (static storage). */
 const char *qknorm_status_string(qkn_status s);
 

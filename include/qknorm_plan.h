@@ -12,12 +12,14 @@
  * waits on another, so any grid is safe.
  *
  * Kernel kinds:
- *   QKN_KERNEL_REGISTER  one pass; the row is held in registers, each thread
- *                        owning up to vec_per_thread 16-byte vectors
- *                        (vector v of a row belongs to thread v % threads, the
- *                        same positions in every row, so a thread keeps its
- *                        gamma vectors in registers across the rows of one
- *                        tensor); every element is read once and written once.
+ *   QKN_KERNEL_REGISTER  one pass; the row (or head) is held in registers by
+ *                        a group of threads -- 1, 2, 4, 8 or 16 lanes, or a
+ *                        multiple of 32 dividing the CTA, the smallest that
+ *                        covers the row with vec_per_thread 16-byte vectors
+ *                        each; lane l owns vectors l, l + group, ... of every
+ *                        row, so it keeps its gamma vectors in registers across
+ *                        the rows of one tensor; every element is read once and
+ *                        written once.
  *                        Needs 16-byte alignment (see qknorm.h) and a row of
  *                        at most vec_per_thread * threads vectors.
  *   QKN_KERNEL_TWOPASS_VEC  two passes over the row with 16-byte vectors
@@ -110,6 +112,12 @@ qkn_status qknorm_layerwise_launch(const void *q_in, void *q_out, const void *ga
                                    const void *k_in, void *k_out, const void *gamma_k, int64_t k_stride,
                                    int64_t T, int32_t Hq, int32_t Hk, float eps, qkn_dtype dtype,
                                    void *stream, const qkn_launch *launch);
+
+/* qknorm_headwise with a caller-chosen launch (rows are heads). */
+qkn_status qknorm_headwise_launch(const void *q_in, void *q_out, const void *gamma_q, int64_t q_stride,
+                                  int32_t q_heads, const void *k_in, void *k_out, const void *gamma_k,
+                                  int64_t k_stride, int32_t k_heads, int64_t T, int32_t head_dim, float eps,
+                                  qkn_dtype dtype, void *stream, const qkn_launch *launch);
 
 /*
  * qknorm_partial_stats / qknorm_combine_apply with a caller-chosen launch;

@@ -411,3 +411,87 @@ def test_packed_host_pipeline_leaves_v_untouched(T):
     yk, ek, _ = oracle_rows(b.k, b.gamma_k, b.eps)
     assert_close(host[:, :b.Hq], yq, eq, "packed host Q")
     assert_close(host[:, b.Hq:v0], yk, ek, "packed host K")
+
+
+# --------------------------------------------------------------------------- headwise
+
+def oracle_heads(view: torch.Tensor, n_heads: int, head_dim: int, gamma: torch.Tensor, eps: float):
+    T = view.shape[0]
+    flat, stride = buffer_np(view)
+    return oracle.rmsnorm_heads(flat, n_heads, head_dim, to_np(gamma), eps, stride=stride, T=T)
+
+
+def check_headwise(q, k, gq, gk, head_dim, eps=1e-6, in_place=False, launch=None, q_dev=None, k_dev=None):
+    """q, k: CPU views; q_dev/k_dev: device views with the same layout."""
+    qd = q.to(DEV) if q_dev is None else q_dev
+    kd = k.to(DEV) if k_dev is None else k_dev
+    kw = dict(q_out=qd, k_out=kd) if in_place else {}
+    qo, ko = qk.qknorm_headwise(qd, kd, gq.to(DEV), gk.to(DEV), head_dim, eps, launch=launch, **kw)
+    torch.cuda.synchronize()
+    yq, eq = oracle_heads(q, q.shape[1] // head_dim, head_dim, gq, eps)
+    yk, ek = oracle_heads(k, k.shape[1] // head_dim, head_dim, gk, eps)
+    assert_close(qo, yq, eq, "headwise Q")
+    assert_close(ko, yk, ek, "headwise K")
+    return qo, ko
+
+
+@pytest.mark.parametrize("dtype", ALL_DTYPES)
+@pytest.mark.parametrize("T,nq,nk,hd", [(1, 32, 8, 128), (37, 16, 4, 64), (300, 8, 8, 128), (5, 3, 2, 7),
+                                        (9, 4, 2, 32), (2, 1, 1, 256), (1000, 40, 8, 128)])
+def test_headwise_matches_the_oracle(dtype, T, nq, nk, hd):
+    g = torch.Generator().manual_seed(T + nq + nk + hd)
+    q = (torch.randn((T, nq * hd), generator=g) * 2).to(dtype)
+    k = (torch.randn((T, nk * hd), generator=g) * 0.5).to(dtype)
+    gq, gk = workloads.gamma(hd, 1, dtype), workloads.gamma(hd, 2, dtype)
+    check_headwise(q, k, gq, gk, hd)
+
+
+def test_headwise_in_place_on_packed_rows_v_untouched():
+    b = workloads.packed_qkv(333)
+    base = b.packed.to(DEV)
+    before = base.clone()
+    hd = 128
+    gq, gk = workloads.gamma(hd, 3, torch.bfloat16), workloads.gamma(hd, 4, torch.bfloat16)
+    qv, kv = base[:, :b.Hq], base[:, b.Hq:b.Hq + b.Hk]
+    check_headwise(b.q, b.k, gq, gk, hd, in_place=True, q_dev=qv, k_dev=kv)
+    assert torch.equal(base[:, b.Hq + b.Hk:], before[:, b.Hq + b.Hk:])
+
+
+@pytest.mark.parametrize("launch", [
+    {"kernel": 0, "vec_per_thread": 1, "threads": 128, "grid": 37},
+    {"kernel": 0, "vec_per_thread": 2, "threads": 256, "grid": 148},
+    {"kernel": 0, "vec_per_thread": 4, "threads": 128, "grid": 5},
+    {"kernel": 0, "vec_per_thread": 8, "threads": 64, "grid": 1000},
+    {"kernel": 0, "vec_per_thread": 1, "threads": 32, "grid": 1},
+    {"kernel": 1, "vec_per_thread": 0, "threads": 64, "grid": 77},
+    {"kernel": 2, "vec_per_thread": 0, "threads": 128, "grid": 9},
+], ids=lambda L: "k{kernel}_nv{vec_per_thread}_t{threads}_g{grid}".format(**L))
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float8_e4m3fn])
+def test_headwise_every_kernel_variant(launch, dtype):
+    g = torch.Generator().manual_seed(77)
+    T, nq, nk, hd = 131, 12, 4, 128
+    q = (torch.randn((T, nq * hd), generator=g)).to(dtype)
+    k = (torch.randn((T, nk * hd), generator=g) * 3).to(dtype)
+    gq, gk = workloads.gamma(hd, 5, dtype), workloads.gamma(hd, 6, dtype)
+    qo, ko = check_headwise(q, k, gq, gk, hd, launch=launch)
+    qo2, ko2 = check_headwise(q, k, gq, gk, hd, launch=launch)
+    assert torch.equal(qo, qo2) and torch.equal(ko, ko2)
+
+
+def test_layerwise_narrow_shards_use_sub_warp_groups():
+    """Rows of 2 and 4 vectors: several rows per warp, reduced by segments."""
+    for H, Hk in ((8, 8), (16, 8), (24, 12), (32, 16), (12, 20)):
+        # strides rounded up to whole 16-byte vectors; 12- and 20-wide rows end in a partial vector
+        b = workloads.random_rows(77, H, Hk, torch.bfloat16, seed=H, q_stride=-(-H // 8) * 8,
+                                  k_stride=-(-Hk // 8) * 8)
+        for launch in ({"kernel": 0, "vec_per_thread": 1, "threads": 128, "grid": 3},
+                       {"kernel": 0, "vec_per_thread": 2, "threads": 64, "grid": 150}):
+            check_layerwise(b, launch=launch)
+
+
+def test_headwise_full_size_bench_workload():
+    """The benchmarked headwise batch (T=4096, 32 Q heads and 8 K heads of 128,
+    bf16) with the planner's own launch, every element against the oracle."""
+    b = workloads.headwise_bf16()
+    hd = b.meta["head_dim"]
+    check_headwise(b.q, b.k, b.gamma_q, b.gamma_k, hd, eps=b.eps)

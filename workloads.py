@@ -163,6 +163,22 @@ def gqa_sharded(seed: int = 3, T: int = 16384, Hq: int = 5120, Hk: int = 1024,
                         gamma(Hq, seed + 100, torch.bfloat16), gamma(Hk, seed + 200, torch.bfloat16))
 
 
+def headwise_bf16(seed: int = 5, T: int = 4096, q_heads: int = 32, k_heads: int = 8,
+                  head_dim: int = 128) -> QKBatch:
+    """Headwise QK-Norm case (GQA-shaped: 32 query heads, 8 key heads of 128),
+    bf16, x ~ N(0,1) * s_t with s_t ~ LogUniform(0.1, 10) per token; gamma
+    [head_dim] per tensor.  ``meta['head_dim']`` holds the head size."""
+    g = _gen(seed)
+    u = torch.rand((T,), generator=g, dtype=torch.float32)
+    s = torch.exp(math.log(0.1) + u * (math.log(10.0) - math.log(0.1)))
+    q = _normal_rows(g, T, q_heads * head_dim, torch.bfloat16, row_scale=s)
+    k = _normal_rows(g, T, k_heads * head_dim, torch.bfloat16, row_scale=s)
+    return QKBatch(f"headwise_bf16_T{T}_q{q_heads}_k{k_heads}_d{head_dim}", torch.bfloat16, T,
+                   q_heads * head_dim, k_heads * head_dim, q, k,
+                   gamma(head_dim, seed + 100, torch.bfloat16), gamma(head_dim, seed + 200, torch.bfloat16),
+                   meta={"head_dim": head_dim, "q_heads": q_heads, "k_heads": k_heads})
+
+
 PACKED_TOKENS = (1024, 4096, 16384, 65536)
 
 
