@@ -15,6 +15,8 @@ This module only marshals numpy arrays into the plain C oracle
 * ``partial_sumsq``  — Phase A's per-shard squared sum.
 * ``combine_apply``  — Phase A's aggregation of the shard sums, then Phase B's
   weight multiplication and global RMS scaling of one shard.
+* ``project_rows``   — the linear projection that produces Q, K and V
+  (Background: Pre-LN layers), in double, rounded once to the element type.
 * ``bf16_decode`` / ``bf16_encode`` — the element codec.
 
 Arrays: fp32 data is passed as ``np.float32``, IEEE half as ``np.float16``,
@@ -69,6 +71,8 @@ def _load():
                                             i64, dbl, ctypes.c_int, vp, vp]
     lib.oracle_qknorm_layerwise.restype = ctypes.c_int
     lib.oracle_rmsnorm_heads.argtypes = [vp, i64, i64, i32, i32, vp, dbl, ctypes.c_int, vp, vp]
+    lib.oracle_project_rows.argtypes = [vp, i64, vp, i64, i64, i32, vp, i64, i32, ctypes.c_int, vp, vp]
+    lib.oracle_project_rows.restype = ctypes.c_int
     lib.oracle_rmsnorm_heads.restype = ctypes.c_int
     lib.oracle_partial_sumsq.argtypes = [vp, i64, i64, i32, ctypes.c_int, vp]
     lib.oracle_partial_sumsq.restype = ctypes.c_int
@@ -249,10 +253,45 @@ def combine_apply(x: np.ndarray, h_shard: int, stride: int, T: int, gamma_shard:
     return y, y_exact
 
 
+def project_rows(x: np.ndarray, w: np.ndarray, rows, D: int | None = None, N: int | None = None,
+                 x_stride: int | None = None, w_stride: int | None = None):
+    """The linear projection ``y[i][n] = sum_d x[rows[i]][d] * w[n][d]`` in
+    double, W stored ``[N][D]`` (one row per output column).
+
+    ``x`` is ``(T, x_stride)`` and ``w`` ``(N, w_stride)``, both of one element
+    type; only the first ``D`` columns are read.  Returns ``(y, y_exact)``:
+    ``y`` ``(n_rows, N)`` rounded once to the element type, ``y_exact`` the
+    float64 sums.
+    """
+    lib = _load()
+    dt = _dtype_code(x)
+    if _dtype_code(w) != dt:
+        raise TypeError("x and w must share an element type")
+    if x.ndim != 2 or w.ndim != 2:
+        raise ValueError("x and w must be 2-D")
+    x_stride = x.shape[1] if x_stride is None else x_stride
+    w_stride = w.shape[1] if w_stride is None else w_stride
+    D = x_stride if D is None else D
+    N = w.shape[0] if N is None else N
+    if not (x.flags.c_contiguous and w.flags.c_contiguous):
+        raise ValueError("oracle inputs must be C-contiguous")
+    if w.size < (N - 1) * w_stride + D:
+        raise ValueError("w too small for N rows of the given stride")
+    T = x.size // x_stride
+    r = np.ascontiguousarray(np.asarray(rows, dtype=np.int64).ravel())
+    y = np.zeros((r.size, N), dtype=x.dtype)
+    y_exact = np.zeros((r.size, N), dtype=np.float64)
+    st = lib.oracle_project_rows(_ptr(x), x_stride, _ptr(r), r.size, T, D, _ptr(w), w_stride, N, dt,
+                                 _ptr(y), _ptr(y_exact))
+    if st != 0:
+        raise ValueError(f"oracle_project_rows rejected its arguments (status {st})")
+    return y, y_exact
+
+
 def version() -> int:
     return _load().oracle_version()
 
 
 __all__ = ["F32", "BF16", "F16", "E4M3", "bf16_decode", "bf16_encode", "f16_decode", "f16_encode",
            "e4m3_decode", "e4m3_encode", "rmsnorm_rows", "rmsnorm_heads", "qknorm_layerwise", "partial_sumsq",
-           "combine_apply", "version"]
+           "combine_apply", "project_rows", "version"]

@@ -398,3 +398,40 @@ int oracle_combine_apply(const void *x, int64_t x_stride, int64_t T, int32_t h_s
     }
     return ORACLE_OK;
 }
+
+/*
+ * The linear projection that produces the tensors QK-Norm normalizes
+ * (Background: in a Pre-LN layer, linear projections of the hidden state give
+ * Q, K and V; QK-Norm runs between the Q/K projections and attention).
+ * W is stored one row per output column, [N][D] with row stride w_stride, so
+ * for each requested token t = rows[i]:
+ *   y_in = sum_{d < D} x_td * w_nd        (double, d from 0 to D-1 in order),
+ * and y_out[i][n] is y_in rounded once to the element type (the projection's
+ * output type).  y_exact (optional) receives the unrounded doubles, [n_rows][N].
+ * Products of two bfloat16 or binary16 values are exact in double; the sum is
+ * the only rounding before the final conversion.
+ */
+int oracle_project_rows(const void *x, int64_t x_stride, const int64_t *rows, int64_t n_rows, int64_t T,
+                        int32_t D, const void *w, int64_t w_stride, int32_t N, int dtype,
+                        void *y_out, double *y_exact)
+{
+    if (n_rows < 0 || T < 0 || D <= 0 || N <= 0 || x_stride < D || w_stride < D || bad_dtype(dtype))
+        return ORACLE_BAD_ARG;
+    if (n_rows > 0 && (!x || !w || !rows))
+        return ORACLE_BAD_ARG;
+    for (int64_t i = 0; i < n_rows; ++i) {
+        const int64_t t = rows[i];
+        if (t < 0 || t >= T)
+            return ORACLE_BAD_ARG;
+        for (int32_t n = 0; n < N; ++n) {
+            double acc = 0.0;
+            for (int32_t d = 0; d < D; ++d)
+                acc += load_elem(x, dtype, t * x_stride + d) * load_elem(w, dtype, (int64_t)n * w_stride + d);
+            if (y_exact)
+                y_exact[i * (int64_t)N + n] = acc;
+            if (y_out)
+                store_elem(y_out, dtype, i * (int64_t)N + n, acc);
+        }
+    }
+    return ORACLE_OK;
+}

@@ -346,3 +346,74 @@ def test_empty_batch_and_bad_arguments():
     with pytest.raises(ValueError):
         oracle.combine_apply(np.zeros((2, 8), np.float32), 8, 8, 2, np.ones(8, np.float32),
                              np.zeros((1, 2)), 4, 1e-6)  # full width below shard width
+
+
+# --------------------------------------------------------------------------- projection
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16, torch.float32])
+def test_projection_matches_numpy_matmul(dtype):
+    """The projection against a library matmul of the same decoded values
+    (float64 BLAS): W is [N][D], so y = x[rows] @ W^T."""
+    g = torch.Generator().manual_seed(41)
+    T, D, N = 9, 70, 33
+    x = torch.randn((T, D), generator=g).to(dtype)
+    w = (torch.randn((N, D), generator=g) * 0.1).to(dtype)
+    rows = [8, 0, 3, 3, 5]
+    y, y_exact = oracle.project_rows(to_np(x), to_np(w), rows)
+    ref = x.double().numpy()[rows] @ w.double().numpy().T
+    np.testing.assert_allclose(y_exact, ref, rtol=1e-12, atol=1e-12)
+    # the stored result is the exact sum rounded once to the element type
+    if dtype == torch.float32:
+        np.testing.assert_array_equal(y, ref.astype(np.float32))
+
+
+def test_projection_of_small_integers_is_exact_and_rounds_once():
+    """Integer inputs: every dot product is an exact integer (computed here in
+    Python integers); below 2^24 it converts to float32 exactly, and torch's
+    float32 -> bfloat16 rounding (pinned above) then gives the stored value."""
+    rng = np.random.default_rng(42)
+    T, D, N = 5, 48, 24
+    xi = rng.integers(-60, 61, size=(T, D))
+    wi = rng.integers(-60, 61, size=(N, D))
+    x = torch.tensor(xi, dtype=torch.bfloat16)
+    w = torch.tensor(wi, dtype=torch.bfloat16)
+    assert torch.equal(x.double(), torch.tensor(xi, dtype=torch.float64))  # |v| <= 60 is exact in bf16
+    y, y_exact = oracle.project_rows(to_np(x), to_np(w), list(range(T)))
+    exact = [[sum(int(xi[t, d]) * int(wi[n, d]) for d in range(D)) for n in range(N)] for t in range(T)]
+    assert y_exact.tolist() == [[float(v) for v in row] for row in exact]
+    expect = torch.tensor(exact, dtype=torch.float32).to(torch.bfloat16)
+    assert np.array_equal(y, to_np(expect))
+
+
+def test_projection_identity_weight_and_strides():
+    """W = I returns the selected rows bit for bit; padded row strides are
+    honoured on both operands; a one-hot W row selects one input column."""
+    g = torch.Generator().manual_seed(43)
+    T, D, pad = 6, 16, 8
+    xb = torch.randn((T, D + pad), generator=g).to(torch.bfloat16)
+    wb = torch.zeros((D, D + 4), dtype=torch.bfloat16)
+    wb[:, :D] = torch.eye(D)
+    wb[:, D:] = 99.0  # padding columns must not be read
+    y, _ = oracle.project_rows(to_np(xb), to_np(wb), [4, 1], D=D, N=D, x_stride=D + pad, w_stride=D + 4)
+    assert np.array_equal(y, to_np(xb[[4, 1], :D].contiguous()))
+    w1 = torch.zeros((3, D), dtype=torch.bfloat16)
+    w1[0, 5] = 1.0
+    w1[1, 0] = -2.0
+    w1[2, D - 1] = 0.5
+    _, ye = oracle.project_rows(to_np(xb), to_np(w1), [2], D=D, x_stride=D + pad)
+    xd = xb.double()
+    assert ye[0].tolist() == [xd[2, 5].item(), -2.0 * xd[2, 0].item(), 0.5 * xd[2, D - 1].item()]
+
+
+def test_projection_then_tile_sums_recover_the_row_sum():
+    """The projected Q row split into 256-column tiles: the tiles' squared sums
+    (Phase A's local step) add up to the full row's squared sum."""
+    g = torch.Generator().manual_seed(44)
+    T, D, N = 3, 64, 1024
+    x = torch.randn((T, D), generator=g).to(torch.bfloat16)
+    w = (torch.randn((N, D), generator=g) * 0.125).to(torch.bfloat16)
+    y, _ = oracle.project_rows(to_np(x), to_np(w), list(range(T)))
+    tiles = [oracle.partial_sumsq(np.ascontiguousarray(y[:, p * 256:(p + 1) * 256]), 256, 256, T)
+             for p in range(N // 256)]
+    _, _, full = oracle.rmsnorm_rows(y, N, np.full(N, 0x3F80, dtype=np.uint16), 0.0)
+    np.testing.assert_allclose(sum(tiles), full, rtol=1e-14)

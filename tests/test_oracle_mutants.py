@@ -41,6 +41,12 @@ MUTANTS = [
      "double v = load_elem(x, dtype, t * (int64_t)H + j);\n            double g", 1),
     ("drop_last_shard", "for (int32_t p = 0; p < P; ++p)", "for (int32_t p = 0; p + 1 < P; ++p)", None),
     ("square_missing", "S += v * v;", "S += v * fabs(v) * 0.5 + v * v * 0.5;", None),
+    ("proj_w_transposed", "load_elem(w, dtype, (int64_t)n * w_stride + d)",
+     "load_elem(w, dtype, (int64_t)(d % N) * w_stride + (n % D))", None),
+    ("proj_drop_last_term", "for (int32_t d = 0; d < D; ++d)", "for (int32_t d = 0; d + 1 < D; ++d)", None),
+    ("proj_row_index", "const int64_t t = rows[i];", "const int64_t t = i < T ? i : T - 1;", None),
+    ("proj_float_accumulation", "double acc = 0.0;\n            for (int32_t d",
+     "float acc = 0.0f;\n            for (int32_t d", None),
 ]
 
 
