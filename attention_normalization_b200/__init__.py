@@ -24,7 +24,8 @@ import torch
 from . import _clib
 from ._clib import QknLaunch, QKNormError
 
-__all__ = ["qknorm_layerwise", "qknorm_headwise", "qknorm_partial_stats", "qknorm_combine_apply", "gamma_dtype",
+__all__ = ["qknorm_layerwise", "qknorm_headwise", "qknorm_qkv_gemm_stats", "qknorm_qkv_projection",
+           "qkv_workspace_bytes", "device_timeouts", "qknorm_partial_stats", "qknorm_combine_apply", "gamma_dtype",
            "qknorm_layerwise_plan", "qknorm_layerwise_host", "qknorm_packed_host",
            "plan_shape", "plan_grid", "regions_overlap", "capi", "version", "QknLaunch", "QKNormError"]
 
@@ -173,6 +174,93 @@ def qknorm_headwise(q_in: torch.Tensor, k_in: torch.Tensor, gamma_q: torch.Tenso
             st = capi().qknorm_headwise_launch(*args, s, ctypes.byref(_launch_struct(launch)))
     _clib.check(st, "qknorm_headwise")
     return q_out, k_out
+
+
+# --------------------------------------------------------------------------- QKV projection
+
+QKV_TILE_N = 256  # output columns per GEMM tile = per partial sum
+
+
+def _projection_args(x, w, Hq, Hk, Hv, qkv):
+    T, D, xs = _rows(x, "x")
+    N, Dw, ws = _rows(w, "w")
+    if x.dtype != torch.bfloat16 or w.dtype != torch.bfloat16:
+        raise TypeError("the projection takes bfloat16 x and w")
+    if Dw != D:
+        raise ValueError(f"w must be [Hq + Hk + Hv, D] with D = {D}, got width {Dw}")
+    if N != Hq + Hk + Hv:
+        raise ValueError(f"w has {N} rows, Hq + Hk + Hv = {Hq + Hk + Hv}")
+    _same(x.device, x.dtype, w, "w")
+    if qkv is None:
+        qkv = torch.empty((T, N), dtype=x.dtype, device=x.device)
+    _same(x.device, x.dtype, qkv, "qkv")
+    To, No, qs = _rows(qkv, "qkv")
+    if (To, No) != (T, N):
+        raise ValueError(f"qkv must be [{T}, {N}]")
+    return T, D, xs, ws, qkv, qs
+
+
+def qkv_workspace_bytes(T: int, Hq: int, Hk: int) -> int:
+    """Workspace ``qknorm_qkv_projection`` needs (the per-tile partial sums)."""
+    n = capi().qknorm_qkv_projection_workspace_bytes(T, Hq, Hk)
+    if n < 0:
+        raise ValueError("invalid sizes for the projection workspace")
+    return n
+
+
+def qknorm_qkv_gemm_stats(x: torch.Tensor, w: torch.Tensor, Hq: int, Hk: int, Hv: int, *, qkv=None,
+                          q_sums=None, k_sums=None, stream=None):
+    """QKV projection ``qkv = bf16(x @ w.T)`` on the tensor cores, with the
+    squared sum of every 256-column Q and K tile of each token written by the
+    epilogue.  Returns ``(qkv, q_sums [Hq/256, T], k_sums [Hk/256, T])``."""
+    T, D, xs, ws, qkv, qs = _projection_args(x, w, Hq, Hk, Hv, qkv)
+    dev = x.device
+    if q_sums is None:
+        q_sums = torch.empty((Hq // QKV_TILE_N, T), dtype=torch.float32, device=dev)
+    if k_sums is None:
+        k_sums = torch.empty((Hk // QKV_TILE_N, T), dtype=torch.float32, device=dev)
+    for t, name, rows in ((q_sums, "q_sums", Hq // QKV_TILE_N), (k_sums, "k_sums", Hk // QKV_TILE_N)):
+        if not (t.is_cuda and t.device == dev and t.dtype == torch.float32 and t.is_contiguous()
+                and t.numel() == rows * T):
+            raise ValueError(f"{name} must be a contiguous float32 CUDA tensor of {rows} x {T}")
+    with torch.cuda.device(dev):
+        st = capi().qknorm_qkv_gemm_stats(x.data_ptr(), xs, w.data_ptr(), ws, qkv.data_ptr(), qs, T, D, Hq, Hk, Hv,
+                                          q_sums.data_ptr(), k_sums.data_ptr(), _clib.QKN_BF16,
+                                          _stream_handle(stream, dev))
+    _clib.check(st, "qknorm_qkv_gemm_stats")
+    return qkv, q_sums, k_sums
+
+
+def qknorm_qkv_projection(x: torch.Tensor, w: torch.Tensor, gamma_q: torch.Tensor, gamma_k: torch.Tensor,
+                          Hq: int, Hk: int, Hv: int, eps: float = 1e-6, *, qkv=None, workspace=None, stream=None):
+    """QKV projection followed by layerwise QK-Norm of its Q and K columns
+    (partial sums from the GEMM epilogue, then combine and scale in place).
+    Returns ``qkv [T, Hq + Hk + Hv]``."""
+    T, D, xs, ws, qkv, qs = _projection_args(x, w, Hq, Hk, Hv, qkv)
+    dev = x.device
+    need = qkv_workspace_bytes(T, Hq, Hk) if Hq % QKV_TILE_N == 0 and Hk % QKV_TILE_N == 0 else 0
+    if workspace is None:
+        workspace = torch.empty((max(need, 4) // 4,), dtype=torch.float32, device=dev)
+    if not (workspace.is_cuda and workspace.device == dev and workspace.is_contiguous()):
+        raise ValueError("workspace must be a contiguous CUDA tensor on the device of x")
+    gq = _vec(gamma_q, "gamma_q", Hq, torch.bfloat16, dev)
+    gk = _vec(gamma_k, "gamma_k", Hk, torch.bfloat16, dev)
+    with torch.cuda.device(dev):
+        st = capi().qknorm_qkv_projection(x.data_ptr(), xs, w.data_ptr(), ws, qkv.data_ptr(), qs, gq, gk, T, D,
+                                          Hq, Hk, Hv, float(eps), workspace.data_ptr(),
+                                          workspace.numel() * workspace.element_size(), _clib.QKN_BF16,
+                                          _stream_handle(stream, dev))
+    _clib.check(st, "qknorm_qkv_projection")
+    return qkv
+
+
+def device_timeouts(device=None) -> int:
+    """Synchronize ``device`` and return (and clear) the code a bounded wait in
+    the projection kernel recorded: 0 when none ran out."""
+    code = ctypes.c_int32(0)
+    with torch.cuda.device(device if device is not None else torch.cuda.current_device()):
+        _clib.check(capi().qknorm_device_timeouts(ctypes.byref(code)), "qknorm_device_timeouts")
+    return code.value
 
 
 def qknorm_layerwise_plan(q_in, k_in, gamma_q, gamma_k, eps: float = 1e-6, *, q_out=None,

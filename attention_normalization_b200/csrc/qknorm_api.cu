@@ -17,6 +17,7 @@
 #include "qknorm.h"
 #include "qknorm_plan.h"
 #include "qknorm_kernels.cuh"
+#include "qkv_gemm.cuh"
 
 #ifndef QKNORM_VERSION
 #define QKNORM_VERSION 100  // 0.1.0
@@ -340,7 +341,8 @@ qkn_status prepare_layerwise(const void *q_in, void *q_out, const void *gamma_q,
     fill_rowset(c.p.set[1], k_in, k_out, gamma_k, k_stride, Hk, Hk, esz);
     c.p.T = T;
     c.p.eps = eps;
-    c.p.P = 1;
+    c.p.set[0].P = 1;
+    c.p.set[1].P = 1;
     finish_call(c, esz, {q_in, q_out, gamma_q, k_in, k_out, gamma_k}, q_stride, k_stride);
     return QKN_OK;
 }
@@ -454,7 +456,8 @@ qkn_status prepare_stats(const void *q_shard, int64_t q_stride, int32_t hq_shard
     c.p.set[1].sumsq = k_sumsq;
     c.p.T = T;
     c.p.eps = 0.0f;
-    c.p.P = 1;
+    c.p.set[0].P = 1;
+    c.p.set[1].P = 1;
     finish_call(c, esz, {q_shard, k_shard}, q_stride, k_stride);
     return QKN_OK;
 }
@@ -498,7 +501,8 @@ qkn_status prepare_apply(const void *q_in, void *q_out, const void *gamma_q_shar
     c.p.set[1].sumsq_all = k_sumsq_all;
     c.p.T = T;
     c.p.eps = eps;
-    c.p.P = P;
+    c.p.set[0].P = P;
+    c.p.set[1].P = P;
     finish_call(c, esz, {q_in, q_out, gamma_q_shard, k_in, k_out, gamma_k_shard}, q_stride, k_stride);
     return QKN_OK;
 }
@@ -542,9 +546,87 @@ qkn_status prepare_headwise(const void *q_in, void *q_out, const void *gamma_q, 
     c.p.set[1].head_bytes = (int64_t)head_dim * esz;
     c.p.T = T;
     c.p.eps = eps;
-    c.p.P = 1;
+    c.p.set[0].P = 1;
+    c.p.set[1].P = 1;
     finish_call(c, esz, {q_in, q_out, gamma_q, k_in, k_out, gamma_k}, q_stride, k_stride);
     return QKN_OK;
+}
+
+// ---------------------------------------------------------------------------
+// QKV projection with Phase A sums in the epilogue.
+constexpr int kTileN = qkn::gemm::kBN;
+constexpr uint64_t kGemmTimeoutNs = 2000000000ull;  // 2 s per mbarrier wait
+
+struct Projection {
+    const void *x, *w;
+    void *qkv;
+    int64_t x_stride, w_stride, qkv_stride, T;
+    int32_t D, Hq, Hk, Hv, N;
+};
+
+qkn_status prepare_projection(const void *x, int64_t x_stride, const void *w, int64_t w_stride, void *qkv,
+                              int64_t qkv_stride, int64_t T, int32_t D, int32_t Hq, int32_t Hk, int32_t Hv,
+                              qkn_dtype dtype, Projection &pr) {
+    if (!dtype_valid(dtype)) return fail(QKN_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
+    if (dtype != QKN_BF16) return fail(QKN_ERR_UNSUPPORTED, "the projection runs on bfloat16 operands only");
+    if (T < 0) return fail(QKN_ERR_INVALID_ARG, "T = %lld < 0", (long long)T);
+    if (T >= ((int64_t)1 << 31)) return fail(QKN_ERR_INVALID_ARG, "T must stay below 2^31");
+    if (D <= 0 || Hq <= 0 || Hk <= 0 || Hv < 0) return fail(QKN_ERR_INVALID_ARG, "D, Hq, Hk must be positive, Hv >= 0");
+    if (Hq % kTileN || Hk % kTileN || Hv % kTileN)
+        return fail(QKN_ERR_UNSUPPORTED, "Hq, Hk and Hv must be multiples of %d (the output tile)", kTileN);
+    const int64_t N = (int64_t)Hq + Hk + Hv;
+    if (N > INT32_MAX) return fail(QKN_ERR_INVALID_ARG, "Hq + Hk + Hv overflows");
+    if (x_stride < D || w_stride < D || qkv_stride < N) return fail(QKN_ERR_INVALID_ARG, "row stride below width");
+    if (!extent_ok(T, x_stride, D, 2) || !extent_ok(N, w_stride, D, 2) || !extent_ok(T, qkv_stride, N, 2))
+        return fail(QKN_ERR_INVALID_ARG, "buffer extent overflows");
+    if (T > 0 && (!x || !w || !qkv)) return fail(QKN_ERR_INVALID_ARG, "null pointer");
+    if (T > 0 && (!aligned16(x) || !aligned16(w) || !aligned16(qkv) || (x_stride % 8) || (w_stride % 8) ||
+                  (qkv_stride % 8)))
+        return fail(QKN_ERR_INVALID_ARG, "x, w and qkv must be 16-byte aligned with strides a multiple of 8 elements");
+    pr = Projection{x, w, qkv, x_stride, w_stride, qkv_stride, T, D, Hq, Hk, Hv, (int32_t)N};
+    return QKN_OK;
+}
+
+// Regions the projection's outputs must not touch.
+qkn_status check_projection_overlaps(const Projection &pr, const float *q_sums, const float *k_sums,
+                                     const void *gamma_q, const void *gamma_k) {
+    const Region rx = rows_region(pr.x, pr.D, pr.x_stride, pr.T, 2);
+    const Region rw = rows_region(pr.w, pr.D, pr.w_stride, pr.N, 2);
+    const Region ro = rows_region(pr.qkv, pr.N, pr.qkv_stride, pr.T, 2);
+    const Region sq = flat_region(q_sums, (int64_t)(pr.Hq / kTileN) * pr.T * 4);
+    const Region sk = flat_region(k_sums, (int64_t)(pr.Hk / kTileN) * pr.T * 4);
+    if (overlap(ro, rx) || overlap(ro, rw)) return fail(QKN_ERR_INVALID_ARG, "qkv overlaps x or w");
+    if (overlap(ro, sq) || overlap(ro, sk)) return fail(QKN_ERR_INVALID_ARG, "qkv overlaps the partial sums");
+    if (overlap(sq, sk)) return fail(QKN_ERR_INVALID_ARG, "the Q and K partial sums overlap");
+    if (overlap(sq, rx) || overlap(sq, rw) || overlap(sk, rx) || overlap(sk, rw))
+        return fail(QKN_ERR_INVALID_ARG, "the partial sums overlap x or w");
+    if (gamma_q || gamma_k) {
+        const Region gq = flat_region(gamma_q, (int64_t)pr.Hq * 2), gk = flat_region(gamma_k, (int64_t)pr.Hk * 2);
+        if (overlap(ro, gq) || overlap(ro, gk)) return fail(QKN_ERR_INVALID_ARG, "qkv overlaps gamma");
+        if (overlap(sq, gq) || overlap(sq, gk) || overlap(sk, gq) || overlap(sk, gk))
+            return fail(QKN_ERR_INVALID_ARG, "the partial sums overlap gamma");
+    }
+    return QKN_OK;
+}
+
+qkn_status launch_projection_gemm(const Projection &pr, float *q_sums, float *k_sums, void *stream) {
+    qkn::gemm::GemmParams gp{};
+    gp.qkv = static_cast<char *>(pr.qkv);
+    gp.qkv_stride_bytes = pr.qkv_stride * 2;
+    gp.q_sumsq = q_sums;
+    gp.k_sumsq = k_sums;
+    gp.T = pr.T;
+    gp.k_blocks = (pr.D + qkn::gemm::kBK - 1) / qkn::gemm::kBK;
+    gp.q_tiles = pr.Hq / kTileN;
+    gp.k_tiles = pr.Hk / kTileN;
+    gp.n_tiles = pr.N / kTileN;
+    gp.timeout_ns = kGemmTimeoutNs;
+    const char *what = "";
+    cudaError_t e = qkn::gemm::launch_qkv_gemm(pr.x, pr.x_stride, pr.w, pr.w_stride, pr.D, pr.N, gp,
+                                               static_cast<cudaStream_t>(stream), &what);
+    if (e == cudaSuccess) e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(QKN_ERR_CUDA, "projection GEMM (%s): %s", what, cudaGetErrorString(e));
+    return ok();
 }
 
 }  // namespace
@@ -758,6 +840,73 @@ qkn_status qknorm_combine_apply_launch(const void *q_in, void *q_out, const void
     if ((st = check_launch(c, *launch_cfg)) != QKN_OK) return st;
     if (T == 0) return ok();
     return launch<qkn::kApply>(c, *launch_cfg, stream);
+}
+
+qkn_status qknorm_qkv_gemm_stats(const void *x, int64_t x_stride, const void *w, int64_t w_stride, void *qkv,
+                                 int64_t qkv_stride, int64_t T, int32_t D, int32_t Hq, int32_t Hk, int32_t Hv,
+                                 float *q_sumsq_all, float *k_sumsq_all, qkn_dtype dtype, void *stream) {
+    Projection pr;
+    qkn_status st = prepare_projection(x, x_stride, w, w_stride, qkv, qkv_stride, T, D, Hq, Hk, Hv, dtype, pr);
+    if (st != QKN_OK) return st;
+    if (T == 0) return ok();
+    if (!q_sumsq_all || !k_sumsq_all) return fail(QKN_ERR_INVALID_ARG, "null pointer");
+    if ((reinterpret_cast<uintptr_t>(q_sumsq_all) | reinterpret_cast<uintptr_t>(k_sumsq_all)) & 3u)
+        return fail(QKN_ERR_INVALID_ARG, "partial sums must be 4-byte aligned");
+    if ((st = check_projection_overlaps(pr, q_sumsq_all, k_sumsq_all, nullptr, nullptr)) != QKN_OK) return st;
+    return launch_projection_gemm(pr, q_sumsq_all, k_sumsq_all, stream);
+}
+
+int64_t qknorm_qkv_projection_workspace_bytes(int64_t T, int32_t Hq, int32_t Hk) {
+    if (T < 0 || Hq <= 0 || Hk <= 0 || Hq % kTileN || Hk % kTileN) return -1;
+    return (int64_t)(Hq / kTileN + Hk / kTileN) * T * 4;
+}
+
+qkn_status qknorm_qkv_projection(const void *x, int64_t x_stride, const void *w, int64_t w_stride, void *qkv,
+                                 int64_t qkv_stride, const void *gamma_q, const void *gamma_k, int64_t T, int32_t D,
+                                 int32_t Hq, int32_t Hk, int32_t Hv, float eps, void *workspace,
+                                 int64_t workspace_bytes, qkn_dtype dtype, void *stream) {
+    Projection pr;
+    qkn_status st = prepare_projection(x, x_stride, w, w_stride, qkv, qkv_stride, T, D, Hq, Hk, Hv, dtype, pr);
+    if (st != QKN_OK) return st;
+    if (!eps_valid(eps)) return fail(QKN_ERR_INVALID_ARG, "eps must be finite and >= 0");
+    if (T == 0) return ok();
+    const int64_t need = qknorm_qkv_projection_workspace_bytes(T, Hq, Hk);
+    if (!gamma_q || !gamma_k || !workspace) return fail(QKN_ERR_INVALID_ARG, "null pointer");
+    if (workspace_bytes < need)
+        return fail(QKN_ERR_INVALID_ARG, "workspace of %lld bytes, %lld needed", (long long)workspace_bytes,
+                    (long long)need);
+    if (reinterpret_cast<uintptr_t>(workspace) & 3u) return fail(QKN_ERR_INVALID_ARG, "workspace must be 4-byte aligned");
+    float *q_sums = static_cast<float *>(workspace);
+    float *k_sums = q_sums + (int64_t)(Hq / kTileN) * T;
+    if ((st = check_projection_overlaps(pr, q_sums, k_sums, gamma_q, gamma_k)) != QKN_OK) return st;
+
+    // Phase A aggregation + Phase B over the Q and K columns of qkv, in place.
+    Call c;
+    std::memset(&c, 0, sizeof(c));
+    c.dtype = dtype;
+    char *kcols = static_cast<char *>(qkv) + (int64_t)Hq * 2;
+    fill_rowset(c.p.set[0], qkv, qkv, gamma_q, qkv_stride, Hq, Hq, 2);
+    fill_rowset(c.p.set[1], kcols, kcols, gamma_k, qkv_stride, Hk, Hk, 2);
+    c.p.set[0].sumsq_all = q_sums;
+    c.p.set[1].sumsq_all = k_sums;
+    c.p.set[0].P = Hq / kTileN;
+    c.p.set[1].P = Hk / kTileN;
+    c.p.T = T;
+    c.p.eps = eps;
+    finish_call(c, 2, {qkv, kcols, gamma_q, gamma_k}, qkv_stride, qkv_stride);
+    qkn_launch L;
+    if ((st = plan_call<qkn::kApply>(c, L)) != QKN_OK) return st;
+    if ((st = launch_projection_gemm(pr, q_sums, k_sums, stream)) != QKN_OK) return st;
+    return launch<qkn::kApply>(c, L, stream);
+}
+
+qkn_status qknorm_device_timeouts(int32_t *code) {
+    if (!code) return fail(QKN_ERR_INVALID_ARG, "null pointer");
+    int v = 0;
+    cudaError_t e = qkn::gemm::read_and_clear_timeout(&v);
+    if (e != cudaSuccess) return fail(QKN_ERR_CUDA, "reading the timeout word: %s", cudaGetErrorString(e));
+    *code = v;
+    return ok();
 }
 
 const char *qknorm_status_string(qkn_status s) {

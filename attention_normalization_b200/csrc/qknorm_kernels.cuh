@@ -39,6 +39,7 @@ struct RowSet {
     const char *gamma;       // kFused / kApply, [width] of the gamma type
     float *sumsq;            // kStats: [T]
     const float *sumsq_all;  // kApply: [P][T]
+    int32_t P;               // kApply: partial sums per token in sumsq_all
     int64_t stride_bytes;
     int32_t width;           // elements in this row (shard width for kStats / kApply)
     int32_t nfull;           // full 16-byte vectors of x in the row
@@ -56,7 +57,6 @@ struct Params {
     RowSet set[2];           // 0 = Q, 1 = K
     int64_t T;
     float eps;
-    int32_t P;               // kApply: number of shards
 };
 
 // ----------------------------------------------------------------------------
@@ -421,7 +421,7 @@ __global__ void __launch_bounds__(RegisterBounds<NV>::kMaxThreads)
     float *sums = nullptr;
     const float *sums_all = nullptr;
     int64_t stride = 0, head_bytes = 0, rows = 0;
-    int nfull = 0, tail = 0, gsize = 32, rpi = 1, grp = 0, gl = 0, gwarps = 1, heads = 1;
+    int nfull = 0, tail = 0, gsize = 32, rpi = 1, grp = 0, gl = 0, gwarps = 1, heads = 1, nparts = 1;
     float inv_div = 0.0f;
     uint4 g[NV][KG];
 
@@ -435,6 +435,7 @@ __global__ void __launch_bounds__(RegisterBounds<NV>::kMaxThreads)
             out = d.out;
             sums = d.sumsq;
             sums_all = d.sumsq_all;
+            nparts = d.P;
             stride = d.stride_bytes;
             head_bytes = d.head_bytes;
             heads = d.heads;
@@ -471,7 +472,7 @@ __global__ void __launch_bounds__(RegisterBounds<NV>::kMaxThreads)
 
         float r;
         if (MODE == kApply) {
-            r = active ? rms_factor(combine_partials(sums_all, T, p.P, t), inv_div, p.eps) : 0.0f;
+            r = active ? rms_factor(combine_partials(sums_all, T, nparts, t), inv_div, p.eps) : 0.0f;
         } else {
             float S = sumsq_pairs<E, NV>(v);
             S = gsize < 32 ? segment_sum(S, gsize) : warp_sum(S);
@@ -537,7 +538,7 @@ __global__ void __launch_bounds__(1024) rows_twopass_kernel(const __grid_constan
 
         float r;
         if (MODE == kApply) {
-            r = rms_factor(combine_partials(d.sumsq_all, p.T, p.P, t), d.inv_div, p.eps);
+            r = rms_factor(combine_partials(d.sumsq_all, p.T, d.P, t), d.inv_div, p.eps);
         } else {
             float acc = 0.0f;
             for (int u = tid; u < units; u += nthr) {

@@ -1,0 +1,389 @@
+// QKV projection GEMM with Phase A partial squared sums in the epilogue
+// (tcgen05 + TMA + TMEM, sm_100a).  The kernel's structure is described in
+// qkv_gemm.cuh.
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "qkv_gemm.cuh"
+
+namespace qkn {
+namespace gemm {
+namespace {
+
+// Set by a wait that ran out; read and cleared by read_and_clear_timeout.
+__device__ int g_timeout_code = 0;
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// ---------------------------------------------------------------- mbarriers
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
+// True once the phase of parity `parity` has completed; false when
+// `timeout_ns` of global time passed first.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_t timeout_ns) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    for (;;) {
+        for (int i = 0; i < 32; ++i)
+            if (mbar_try_wait(bar, parity)) return true;
+        if (global_ns() - t0 > timeout_ns) return false;
+    }
+}
+
+// ---------------------------------------------------------------- TMA
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int32_t c0, int32_t c1,
+                                            uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+        "[%4];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar)
+        : "memory");
+}
+
+__device__ __forceinline__ void prefetch_map(const CUtensorMap *map) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// ---------------------------------------------------------------- tcgen05
+__device__ __forceinline__ void fence_before_sync() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void fence_after_sync() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor of a K-major operand tile stored as rows of
+// 128 bytes with the 128-byte swizzle (what a TMA box of 64 bf16 x rows with
+// CU_TENSOR_MAP_SWIZZLE_128B writes): start address >> 4 in bits 0-13,
+// leading-dimension offset 1 (unused by swizzled K-major layouts), stride
+// between 8-row groups 1024 bytes (>> 4 in bits 32-45), descriptor version 1
+// (bits 46-47), base offset 0 (atoms are 1024-byte aligned), layout type 2 =
+// 128-byte swizzle (bits 61-63).
+__device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t saddr) {
+    return static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4) | (static_cast<uint64_t>(1) << 16) |
+           (static_cast<uint64_t>(1024 >> 4) << 32) | (static_cast<uint64_t>(1) << 46) |
+           (static_cast<uint64_t>(2) << 61);
+}
+
+// Instruction descriptor of tcgen05.mma kind::f16: fp32 accumulator (bits
+// 4-5 = 1), A and B bf16 (bits 7-9 and 10-12 = 1), both K-major (bits 15, 16
+// = 0), N >> 3 in bits 17-22, M >> 4 in bits 24-28.
+constexpr uint32_t kIdescBf16 = (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(kBN >> 3) << 17) |
+                                (static_cast<uint32_t>(kBM >> 4) << 24);
+
+__device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// The mbarrier receives one arrival when every tcgen05.mma this thread issued
+// so far has completed.
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                 : "memory");
+}
+
+// 32 consecutive fp32 columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]),
+          "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]),
+          "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void record_timeout(int code, int *flag) {
+    atomicExch(&g_timeout_code, code);
+    *flag = 1;
+}
+
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+}  // namespace
+
+__global__ void __launch_bounds__(kThreads, 1)
+    qkv_gemm_stats_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
+                          const __grid_constant__ GemmParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ int s_abort;      // a wait in this CTA ran out
+    __shared__ int s_consumed;   // k-blocks whose MMAs were issued
+    __shared__ int s_issued;     // k-blocks whose TMA loads were issued
+
+    // 1024-byte aligned ring: A stages, then B stages, then the mbarriers.
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    const uint32_t a_base = base;
+    const uint32_t b_base = base + kStages * kABytes;
+    const uint32_t bars = base + kStages * kStageBytes;
+    auto full_bar = [&](int s) { return bars + 8u * s; };
+    auto empty_bar = [&](int s) { return bars + 8u * (kStages + s); };
+    const uint32_t acc_bar = bars + 16u * kStages;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem_raw + (bars - raw) + 8 * (2 * kStages + 1));
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int m_tile = blockIdx.x;  // tokens (fastest, so a wave shares W tiles and X stays in L2)
+    const int n_tile = blockIdx.y;  // output columns
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(full_bar(s), 1);
+            mbar_init(empty_bar(s), 1);
+        }
+        mbar_init(acc_bar, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        prefetch_map(&tmap_x);
+        prefetch_map(&tmap_w);
+        s_abort = 0;
+        s_consumed = 0;
+        s_issued = 0;
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                     "r"(kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+    pdl_wait();  // X may come from the previous kernel in the stream; qkv may still be read by it
+
+    if (warp == 0) {
+        if (lane == 0) {  // ---------------------------------------------- TMA producer
+            int issued = 0;
+            for (int kb = 0; kb < p.k_blocks; ++kb) {
+                const int s = kb % kStages;
+                const int round = kb / kStages;
+                if (round > 0 && !mbar_wait(empty_bar(s), (round - 1) & 1, p.timeout_ns)) {
+                    record_timeout(kErrProducer, &s_abort);
+                    break;
+                }
+                mbar_expect_tx(full_bar(s), kStageBytes);
+                tma_load_2d(a_base + s * kABytes, &tmap_x, kb * kBK, m_tile * kBM, full_bar(s));
+                tma_load_2d(b_base + s * kBBytes, &tmap_w, kb * kBK, n_tile * kBN, full_bar(s));
+                issued = kb + 1;
+            }
+            s_issued = issued;
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {  // ---------------------------------------------- MMA issuer
+            int kb = 0;
+            for (; kb < p.k_blocks; ++kb) {
+                const int s = kb % kStages;
+                if (!mbar_wait(full_bar(s), (kb / kStages) & 1, p.timeout_ns)) {
+                    record_timeout(kErrMma, &s_abort);
+                    break;
+                }
+                fence_after_sync();
+                const uint32_t a_s = a_base + s * kABytes;
+                const uint32_t b_s = b_base + s * kBBytes;
+#pragma unroll
+                for (int k = 0; k < kBK / kUmmaK; ++k)
+                    umma_bf16(tmem, sw128_kmajor_desc(a_s + k * kUmmaK * 2), sw128_kmajor_desc(b_s + k * kUmmaK * 2),
+                              kIdescBf16, (kb | k) != 0 ? 1u : 0u);
+                umma_commit(empty_bar(s));
+            }
+            s_consumed = kb;
+            umma_commit(acc_bar);  // also after a timeout, so the epilogue is not left waiting
+        }
+        __syncwarp();
+    } else {  // ------------------------------------------------------------ epilogue
+        bool ok = mbar_wait(acc_bar, 0, p.timeout_ns);
+        if (!ok) record_timeout(kErrEpilogue, &s_abort);
+        ok = __all_sync(0xFFFFFFFFu, ok) && p.k_blocks > 0;
+        fence_after_sync();
+        if (ok) {
+            const int quarter = warp & 3;  // TMEM lanes this warp may read
+            const int64_t row = static_cast<int64_t>(m_tile) * kBM + quarter * 32 + lane;
+            const bool live = row < p.T;
+            char *orow = p.qkv + (live ? row : 0) * p.qkv_stride_bytes + static_cast<int64_t>(n_tile) * kBN * 2;
+            const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+            float ss = 0.0f;
+#pragma unroll 1
+            for (int c = 0; c < kBN / 32; ++c) {
+                uint32_t r[32];
+                tmem_ld32(taddr + c * 32, r);
+                uint32_t packed[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const __nv_bfloat162 h =
+                        __float22bfloat162_rn(make_float2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])));
+                    const float lo = __low2float(h), hi = __high2float(h);
+                    ss = fmaf(lo, lo, ss);
+                    ss = fmaf(hi, hi, ss);
+                    packed[i] = *reinterpret_cast<const uint32_t *>(&h);
+                }
+                if (live) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(orow + c * 64);
+#pragma unroll
+                    for (int v = 0; v < 4; ++v)
+                        dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
+                }
+            }
+            if (live) {
+                if (n_tile < p.q_tiles) {
+                    if (p.q_sumsq) p.q_sumsq[static_cast<int64_t>(n_tile) * p.T + row] = ss;
+                } else if (n_tile < p.q_tiles + p.k_tiles) {
+                    if (p.k_sumsq) p.k_sumsq[static_cast<int64_t>(n_tile - p.q_tiles) * p.T + row] = ss;
+                }
+            }
+        }
+    }
+
+    fence_before_sync();
+    __syncthreads();
+    if (threadIdx.x == 0 && s_abort) {
+        // After a timeout, loads the MMA thread never consumed may still be in
+        // flight: let them land (bounded) before this CTA's shared memory is
+        // released.
+        for (int kb = s_consumed; kb < s_issued; ++kb)
+            (void)mbar_wait(full_bar(kb % kStages), (kb / kStages) & 1, p.timeout_ns);
+    }
+    if (warp == 1) {
+        fence_after_sync();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+    }
+}
+
+// ------------------------------------------------------------------ host side
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+cudaError_t g_encode_status = cudaSuccess;
+
+cudaError_t encoder(PFN_cuTensorMapEncodeTiled_v12000 *fn) {
+    std::call_once(g_encode_once, [] {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+        g_encode_status = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q);
+        if (g_encode_status == cudaSuccess && (q != cudaDriverEntryPointSuccess || !f))
+            g_encode_status = cudaErrorSymbolNotFound;
+        g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    });
+    *fn = g_encode;
+    return g_encode_status;
+}
+
+// A row-major bf16 matrix [outer][inner] with rows `stride_elems` apart, read
+// in boxes of box_outer rows x 64 columns with the 128-byte swizzle; reads
+// beyond the matrix return zeros.
+bool encode_bf16_rows(PFN_cuTensorMapEncodeTiled_v12000 fn, CUtensorMap *map, const void *base, int64_t inner,
+                      int64_t outer, int64_t stride_elems, uint32_t box_outer) {
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(outer)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(stride_elems) * 2};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(kBK), box_outer};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+constexpr int kMaxDevices = 64;
+bool g_smem_set[kMaxDevices] = {};
+std::mutex g_smem_mu;
+
+}  // namespace
+
+cudaError_t launch_qkv_gemm(const void *x, int64_t x_stride, const void *w, int64_t w_stride, int32_t D,
+                            int32_t N, const GemmParams &p, cudaStream_t stream, const char **what) {
+    PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    cudaError_t e = encoder(&fn);
+    if (e != cudaSuccess) {
+        *what = "cuTensorMapEncodeTiled entry point";
+        return e;
+    }
+    CUtensorMap tx, tw;
+    if (!encode_bf16_rows(fn, &tx, x, D, p.T, x_stride, kBM) || !encode_bf16_rows(fn, &tw, w, D, N, w_stride, kBN)) {
+        *what = "cuTensorMapEncodeTiled";
+        return cudaErrorInvalidValue;
+    }
+    int dev = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) {
+        *what = "cudaGetDevice";
+        return e;
+    }
+    {
+        std::lock_guard<std::mutex> lk(g_smem_mu);
+        if (dev < 0 || dev >= kMaxDevices || !g_smem_set[dev]) {
+            e = cudaFuncSetAttribute(qkv_gemm_stats_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+            if (e != cudaSuccess) {
+                *what = "cudaFuncSetAttribute(max dynamic shared memory)";
+                return e;
+            }
+            if (dev >= 0 && dev < kMaxDevices) g_smem_set[dev] = true;
+        }
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>((p.T + kBM - 1) / kBM), static_cast<unsigned>(p.n_tiles));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    void *args[] = {&tx, &tw, const_cast<GemmParams *>(&p)};
+    e = cudaLaunchKernelExC(&cfg, reinterpret_cast<const void *>(qkv_gemm_stats_kernel), args);
+    if (e != cudaSuccess) *what = "cudaLaunchKernelExC";
+    return e;
+}
+
+cudaError_t read_and_clear_timeout(int *code) {
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return e;
+    int v = 0;
+    if ((e = cudaMemcpyFromSymbol(&v, g_timeout_code, sizeof(int))) != cudaSuccess) return e;
+    const int zero = 0;
+    if ((e = cudaMemcpyToSymbol(g_timeout_code, &zero, sizeof(int))) != cudaSuccess) return e;
+    *code = v;
+    return cudaSuccess;
+}
+
+}  // namespace gemm
+}  // namespace qkn

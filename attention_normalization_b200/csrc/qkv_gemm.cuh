@@ -1,0 +1,92 @@
+// QKV projection on the sm_100a tensor cores with Phase A's partial squared
+// sums produced in the epilogue.
+//
+// Method: "SwiftQK: Fast and Communication-Efficient Tensor Parallelism for
+// Query-Key Normalization" (arXiv 2608.09160).
+//   Background: in a Pre-LN layer linear projections produce Q, K and V, and
+//     layerwise QK-Norm normalizes the full projected Q and K rows before
+//     attention.
+//   Phase A: the RMS factor needs only the squared sum of the row; each
+//     hidden-dimension shard contributes the squared sum of its own columns
+//     and the partial sums are added in fp32.
+// Here a shard is one 256-column output tile of the projection: the epilogue
+// that stores the tile's bf16 values also writes, per token, the squared sum
+// of those stored values.  The combine / factor / scale steps then run as the
+// usual apply pass (Phase A aggregation + Phase B).
+//
+// Kernel shape (one CTA per 128 x 256 output tile, 192 threads):
+//   warp 0, lane 0 : TMA producer.  X tile [128 x 64] and W tile [256 x 64]
+//                    per k-block into a 4-stage shared-memory ring, 128-byte
+//                    swizzle, completion counted on an mbarrier per stage.
+//   warp 1         : allocates 256 TMEM columns (the fp32 accumulator,
+//                    lane = tile row); lane 0 issues tcgen05.mma (M=128,
+//                    N=256, K=16, bf16 in, fp32 accumulate), four per
+//                    k-block, and tcgen05.commit frees the stage when the
+//                    MMAs have read it; a final commit signals the epilogue.
+//   warps 2..5     : epilogue.  Warp w reads TMEM lanes 32*(w%4) .. +31
+//                    (one tile row per thread) in 32-column chunks, rounds to
+//                    bf16 (nearest even), stores the row's 512 bytes and, for
+//                    Q and K tiles, sums the squares of the rounded values in
+//                    column order (fp32 fma) and writes one partial per row.
+// Every mbarrier wait is bounded by the global timer; on expiry the kernel
+// records a code in a device word, skips the rest of its work, frees its TMEM
+// and returns, so the context stays usable.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace qkn {
+namespace gemm {
+
+constexpr int kBM = 128;           // tile rows (tokens) = TMEM lanes
+constexpr int kBN = 256;           // tile columns = one partial-sum shard
+constexpr int kBK = 64;            // k-block: 64 bf16 = one 128-byte swizzle row
+constexpr int kStages = 4;
+constexpr int kUmmaK = 16;         // K of one tcgen05.mma kind::f16
+constexpr int kThreads = 192;
+constexpr int kABytes = kBM * kBK * 2;
+constexpr int kBBytes = kBN * kBK * 2;
+constexpr int kStageBytes = kABytes + kBBytes;
+constexpr int kTmemCols = 256;
+// ring + barriers (2 * kStages + 1 mbarriers) + TMEM address slot + 1 KB
+// alignment slack for the 128-byte-swizzle atoms
+constexpr int kSmemBytes = kStages * kStageBytes + 1024 + 256;
+
+struct GemmParams {
+    char *qkv;               // [T][qkv_stride] bf16, columns [0, N)
+    int64_t qkv_stride_bytes;
+    float *q_sumsq;          // [Hq / kBN][T] or null
+    float *k_sumsq;          // [Hk / kBN][T] or null
+    int64_t T;
+    int32_t k_blocks;        // ceil(D / kBK)
+    int32_t q_tiles;         // Hq / kBN
+    int32_t k_tiles;         // Hk / kBN
+    int32_t n_tiles;         // N / kBN
+    uint64_t timeout_ns;     // bound on every mbarrier wait
+};
+
+// Error codes written to the device word when a wait runs out.
+enum : int { kErrNone = 0, kErrProducer = 1, kErrMma = 2, kErrEpilogue = 3 };
+
+}  // namespace gemm
+}  // namespace qkn
+
+namespace qkn {
+namespace gemm {
+
+// Host side (qkv_gemm.cu).  Encodes the TMA maps for X [T][D] (row stride
+// x_stride elements) and W [N][D] (row stride w_stride) and launches one CTA
+// per output tile on `stream`.  Pointers must be 16-byte aligned and strides
+// multiples of 8 elements (the caller checks).  On failure *what names the
+// step that failed (static storage).
+cudaError_t launch_qkv_gemm(const void *x, int64_t x_stride, const void *w, int64_t w_stride, int32_t D,
+                            int32_t N, const GemmParams &p, cudaStream_t stream, const char **what);
+
+// The device word a bounded wait writes when it runs out (0 = none); reading
+// synchronizes the current device and clears the word.
+cudaError_t read_and_clear_timeout(int *code);
+
+}  // namespace gemm
+}  // namespace qkn

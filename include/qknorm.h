@@ -149,6 +149,63 @@ qkn_status qknorm_headwise(const void *q_in, void *q_out, const void *gamma_q, i
                            const void *k_in, void *k_out, const void *gamma_k, int64_t k_stride, int32_t k_heads,
                            int64_t T, int32_t head_dim, float eps, qkn_dtype dtype, void *stream);
 
+/*
+ * QKV projection with Phase A's partial sums in the GEMM epilogue (Background:
+ * in a Pre-LN layer linear projections of the hidden state produce Q, K and V,
+ * and QK-Norm sits between the Q/K projections and attention; Phase A: the
+ * RMS factor needs only each shard's squared sum).  Runs on the tensor cores
+ * (tcgen05, bf16 operands, fp32 accumulation).
+ *   x   : [T rows, stride x_stride] bfloat16, the hidden states, width D.
+ *   w   : [N rows, stride w_stride] bfloat16, N = Hq + Hk + Hv, one row per
+ *         output column (the linear layer's weight as stored): Q columns
+ *         first, then K, then V.
+ *   qkv : [T rows, stride qkv_stride] bfloat16 output,
+ *         qkv[t][n] = RNE_bf16( sum_d x[t][d] * w[n][d] ).
+ *   q_sumsq_all : [Hq / 256][T] fp32; entry [p][t] is the squared sum of the
+ *         stored (rounded) values qkv[t][256p .. 256p + 255], summed in column
+ *         order.  k_sumsq_all likewise for the K columns, [Hk / 256][T].
+ * These are exactly the inputs qknorm_combine_apply expects with 256-column
+ * shards; qknorm_qkv_projection below runs both steps.
+ * Requirements: dtype QKN_BF16 (else QKN_ERR_UNSUPPORTED); Hq, Hk > 0 and Hv
+ * >= 0 multiples of 256 (else QKN_ERR_UNSUPPORTED); D >= 1 (any D: the k
+ * loop reads zeros past it); x, w, qkv 16-byte aligned with strides a
+ * multiple of 8 elements; T < 2^31; qkv must not overlap x, w or the sums.
+ * Asynchronous on `stream`; allocates nothing.  T = 0 is a no-op.
+ */
+qkn_status qknorm_qkv_gemm_stats(const void *x, int64_t x_stride, const void *w, int64_t w_stride, void *qkv,
+                                 int64_t qkv_stride, int64_t T, int32_t D, int32_t Hq, int32_t Hk, int32_t Hv,
+                                 float *q_sumsq_all, float *k_sumsq_all, qkn_dtype dtype, void *stream);
+
+/* Bytes of workspace qknorm_qkv_projection needs: (Hq/256 + Hk/256) * T * 4,
+ * or -1 when the sizes are invalid. */
+int64_t qknorm_qkv_projection_workspace_bytes(int64_t T, int32_t Hq, int32_t Hk);
+
+/*
+ * Projection followed by layerwise QK-Norm of its Q and K columns, two
+ * launches on `stream`: qknorm_qkv_gemm_stats writing the partial sums into
+ * `workspace`, then Phase A's aggregation (partials added in order p = 0, 1,
+ * ..., fp32) and Phase B's scaling of the Q and K columns of qkv in place:
+ *   r = 1 / sqrt(S / H + eps),  qkv[t][j] = RNE_bf16( (qkv[t][j] * gamma_j) * r )
+ * with H = Hq for the Q columns (gamma_q [Hq]) and Hk for the K columns
+ * (gamma_k [Hk]); V columns keep the projection.  The caller owns
+ * `workspace` (>= qknorm_qkv_projection_workspace_bytes, 4-byte aligned); its
+ * contents on return are the partial sums.  Same requirements and errors as
+ * qknorm_qkv_gemm_stats, plus eps finite and >= 0 and non-null gamma.
+ */
+qkn_status qknorm_qkv_projection(const void *x, int64_t x_stride, const void *w, int64_t w_stride, void *qkv,
+                                 int64_t qkv_stride, const void *gamma_q, const void *gamma_k, int64_t T, int32_t D,
+                                 int32_t Hq, int32_t Hk, int32_t Hv, float eps, void *workspace,
+                                 int64_t workspace_bytes, qkn_dtype dtype, void *stream);
+
+/*
+ * Every wait inside the projection kernel is bounded (2 s); one that runs out
+ * records a non-zero code (1 = TMA producer, 2 = MMA issuer, 3 = epilogue)
+ * and the kernel returns early with its output incomplete.  This call
+ * synchronizes the current device, stores that code in *code (0 = none) and
+ * clears it.  No paper counterpart: a safety check of this library.
+ */
+qkn_status qknorm_device_timeouts(int32_t *code);
+
 /* Short English name of a status code (static storage). */
 const char *qknorm_status_string(qkn_status s);
 

@@ -340,3 +340,58 @@ def test_host_pipeline_argument_checks():
         qk.qknorm_layerwise_host(x, x, g, g, chunk_tokens=0)
     with pytest.raises(ValueError, match="inside the packed row"):
         qk.qknorm_packed_host(torch.zeros((4, 16)), 0, 8, 8, 9, g, g)
+
+
+def _proj_call(lib, **kw):
+    a = dict(x=0x10000, xs=4096, w=0x2000000, ws=4096, qkv=0x8000000, qs=12288, T=4096, D=4096, Hq=4096,
+             Hk=4096, Hv=4096, q_sums=0x20000000, k_sums=0x21000000, dtype=BF16)
+    a.update(kw)
+    return lib.qknorm_qkv_gemm_stats(a["x"], a["xs"], a["w"], a["ws"], a["qkv"], a["qs"], a["T"], a["D"], a["Hq"],
+                                     a["Hk"], a["Hv"], a["q_sums"], a["k_sums"], a["dtype"], None)
+
+
+@pytest.mark.parametrize("kw,want", [
+    ({}, CUDA),                                  # well formed: validation passes, the device query fails here
+    ({"T": 0}, OK),                              # empty batch: nothing enqueued
+    ({"dtype": F32}, UNSUPPORTED),
+    ({"dtype": 9}, INVALID),
+    ({"Hq": 4000}, UNSUPPORTED),                 # not a whole number of 256-column tiles
+    ({"Hv": 100}, UNSUPPORTED),
+    ({"Hk": 0}, INVALID),
+    ({"D": 0}, INVALID),
+    ({"T": -1}, INVALID),
+    ({"T": 1 << 31}, INVALID),
+    ({"xs": 4000}, INVALID),                     # stride below D
+    ({"qs": 12000}, INVALID),                    # stride below N
+    ({"xs": 4100}, INVALID),                     # stride not a multiple of 8 elements (TMA rows)
+    ({"x": 0x10008}, INVALID),                   # not 16-byte aligned
+    ({"w": 0}, INVALID),
+    ({"q_sums": 0}, INVALID),
+    ({"q_sums": 0x20000002}, INVALID),           # sums not 4-byte aligned
+    ({"qkv": 0x10000 + 2 * 4096 * 100}, INVALID),  # output overlaps x
+    ({"k_sums": 0x20000000 + 4 * 4096 * 3}, INVALID),  # K sums overlap the Q sums
+])
+def test_projection_validation(lib, kw, want):
+    assert _proj_call(lib, **kw) == want
+
+
+def test_projection_pipeline_validation(lib):
+    T, D, H = 4096, 4096, 4096
+    need = lib.qknorm_qkv_projection_workspace_bytes(T, H, H)
+    assert need == (H // 256 + H // 256) * T * 4
+    assert lib.qknorm_qkv_projection_workspace_bytes(T, 100, H) == -1
+    assert lib.qknorm_qkv_projection_workspace_bytes(-1, H, H) == -1
+
+    def call(**kw):
+        a = dict(gq=0x30000000, gk=0x30100000, eps=1e-6, ws=0x40000000, wsb=need)
+        a.update(kw)
+        return lib.qknorm_qkv_projection(0x10000, D, 0x2000000, D, 0x8000000, 3 * H, a["gq"], a["gk"], T, D, H, H,
+                                         H, a["eps"], a["ws"], a["wsb"], BF16, None)
+    assert call() == CUDA
+    assert call(wsb=need - 4) == INVALID
+    assert call(gq=0) == INVALID
+    assert call(eps=-1.0) == INVALID
+    assert call(eps=float("nan")) == INVALID
+    assert call(ws=0x8000000 + 64) == INVALID        # workspace inside qkv
+    assert call(gk=0x8000000) == INVALID             # gamma inside qkv
+    assert lib.qknorm_device_timeouts(None) == INVALID

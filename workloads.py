@@ -179,6 +179,45 @@ def headwise_bf16(seed: int = 5, T: int = 4096, q_heads: int = 32, k_heads: int 
                    meta={"head_dim": head_dim, "q_heads": q_heads, "k_heads": k_heads})
 
 
+@dataclass
+class ProjectionBatch:
+    """Hidden states and QKV projection weights (CPU tensors, bfloat16).
+
+    ``x`` is ``[T, D]``; ``w`` is ``[Hq + Hk + Hv, D]``, one row per output
+    column (Q columns first, then K, then V); ``gamma_q`` ``[Hq]`` and
+    ``gamma_k`` ``[Hk]`` are the QK-Norm scales."""
+    name: str
+    T: int
+    D: int
+    Hq: int
+    Hk: int
+    Hv: int
+    x: torch.Tensor
+    w: torch.Tensor
+    gamma_q: torch.Tensor
+    gamma_k: torch.Tensor
+    eps: float = 1e-6
+
+
+def qkv_projection(T: int = 4096, D: int = 4096, Hq: int = 4096, Hk: int = 4096, Hv: int = 4096,
+                   seed: int = 6) -> ProjectionBatch:
+    """Pre-LN hidden states and a QKV projection of OLMo2-7B's shape by
+    default (hidden 4096, 32 query / key / value heads of 128).  x ~ N(0,1) * s_t
+    with one s_t ~ LogUniform(0.1, 10) per token (the spread of per-token
+    scales the prefill workload uses); W ~ N(0, 1/D), the usual fan-in
+    scaling, so projected values are of order s_t.  gamma = 1 + 0.1 N(0,1).
+    Seeds: x uses ``seed``, W seed + 50, gamma_q seed + 100, gamma_k seed + 200."""
+    g = _gen(seed)
+    u = torch.rand((T,), generator=g, dtype=torch.float32)
+    s = torch.exp(math.log(0.1) + u * (math.log(10.0) - math.log(0.1)))
+    x = _normal_rows(g, T, D, torch.bfloat16, row_scale=s)
+    gw = _gen(seed + 50)
+    N = Hq + Hk + Hv
+    w = _normal_rows(gw, N, D, torch.bfloat16, row_scale=torch.full((N,), 1.0 / math.sqrt(D)))
+    return ProjectionBatch(f"qkv_projection_bf16_T{T}_D{D}_q{Hq}_k{Hk}_v{Hv}", T, D, Hq, Hk, Hv, x, w,
+                           gamma(Hq, seed + 100, torch.bfloat16), gamma(Hk, seed + 200, torch.bfloat16))
+
+
 PACKED_TOKENS = (1024, 4096, 16384, 65536)
 
 
