@@ -58,6 +58,9 @@ PROTOTYPES = {
     "qknorm_qkv_projection": (_st, [_vp, _i64, _vp, _i64, _vp, _i64, _vp, _vp, _i64, _i32, _i32, _i32, _i32,
                                     _f32, _vp, _i64, _dt, _vp]),
     "qknorm_device_timeouts": (_st, [ctypes.POINTER(ctypes.c_int32)]),
+    "qknorm_qkv_projection_noalloc": (_st, [_vp, _i64, _vp, _i64, _vp, _i64, _vp, _vp, _i64, _i32, _i32, _i32,
+                                            _i32, _f32, _dt, _vp]),
+    "qknorm_qkv_projection_noalloc_max_bytes": (_i64, []),
     "qknorm_last_error": (ctypes.c_char_p, []),
     "qknorm_version": (ctypes.c_int, []),
     "qknorm_register_max_threads": (_i32, [_i32]),

@@ -632,6 +632,40 @@ qkn_status launch_projection_gemm(const Projection &pr, float *q_sums, float *k_
 }  // namespace
 
 // ===========================================================================
+// ---------------------------------------------------------------------------
+// Scratch for qknorm_qkv_projection_noalloc: a fixed array in the library's
+// own device image, so that entry point never allocates.  Each GPU that loads
+// the library holds it until the process exits.  Host code must not pass the
+// array's name to a kernel (on the host it is only a stand-in for the symbol);
+// the device address comes from cudaGetSymbolAddress, once per device.
+constexpr int64_t kNoAllocScratchBytes = (int64_t)4 << 20;  // 4 MiB
+static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchBytes / 4];
+
+namespace {
+constexpr int kMaxScratchDevices = 64;
+std::mutex g_scratch_mu;
+void *g_scratch_addr[kMaxScratchDevices] = {};
+
+// Device address of g_noalloc_scratch on the current device (looked up on the
+// first call for that device, with the device current).
+qkn_status noalloc_scratch(void **out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return fail(QKN_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    if (dev < 0 || dev >= kMaxScratchDevices) return fail(QKN_ERR_UNSUPPORTED, "device index %d too large", dev);
+    std::lock_guard<std::mutex> lk(g_scratch_mu);
+    if (!g_scratch_addr[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess || !p)
+            return fail(QKN_ERR_CUDA, "cudaGetSymbolAddress(scratch): %s", cudaGetErrorString(e));
+        g_scratch_addr[dev] = p;
+    }
+    *out = g_scratch_addr[dev];
+    return QKN_OK;
+}
+}  // namespace
+
 extern "C" {
 
 int32_t qknorm_register_max_threads(int32_t vec_per_thread) {
@@ -899,6 +933,28 @@ qkn_status qknorm_qkv_projection(const void *x, int64_t x_stride, const void *w,
     if ((st = launch_projection_gemm(pr, q_sums, k_sums, stream)) != QKN_OK) return st;
     return launch<qkn::kApply>(c, L, stream);
 }
+
+qkn_status qknorm_qkv_projection_noalloc(const void *x, int64_t x_stride, const void *w, int64_t w_stride,
+                                         void *qkv, int64_t qkv_stride, const void *gamma_q, const void *gamma_k,
+                                         int64_t T, int32_t D, int32_t Hq, int32_t Hk, int32_t Hv, float eps,
+                                         qkn_dtype dtype, void *stream) {
+    const int64_t need = qknorm_qkv_projection_workspace_bytes(T, Hq, Hk);
+    if (T <= 0 || need < 0)  // empty or invalid: the checks below reject it or do nothing
+        return qknorm_qkv_projection(x, x_stride, w, w_stride, qkv, qkv_stride, gamma_q, gamma_k, T, D, Hq, Hk, Hv,
+                                     eps, nullptr, 0, dtype, stream);
+    if (need > kNoAllocScratchBytes)
+        return fail(QKN_ERR_INVALID_ARG,
+                    "needs %lld bytes of partial sums; the built-in scratch holds %lld "
+                    "((Hq/256 + Hk/256) * T must stay at or below %lld)",
+                    (long long)need, (long long)kNoAllocScratchBytes, (long long)(kNoAllocScratchBytes / 4));
+    void *ws = nullptr;
+    qkn_status st = noalloc_scratch(&ws);
+    if (st != QKN_OK) return st;
+    return qknorm_qkv_projection(x, x_stride, w, w_stride, qkv, qkv_stride, gamma_q, gamma_k, T, D, Hq, Hk, Hv, eps,
+                                 ws, kNoAllocScratchBytes, dtype, stream);
+}
+
+int64_t qknorm_qkv_projection_noalloc_max_bytes(void) { return kNoAllocScratchBytes; }
 
 qkn_status qknorm_device_timeouts(int32_t *code) {
     if (!code) return fail(QKN_ERR_INVALID_ARG, "null pointer");

@@ -198,6 +198,36 @@ qkn_status qknorm_qkv_projection(const void *x, int64_t x_stride, const void *w,
                                  int64_t workspace_bytes, qkn_dtype dtype, void *stream);
 
 /*
+ * qknorm_qkv_projection for callers that cannot allocate device memory: a
+ * host engine that owns every device allocation and forbids new ones once it
+ * is serving, or a latency-critical path on which a cudaMalloc (which may
+ * synchronize the device) is not acceptable.  Same arguments, results and
+ * errors as qknorm_qkv_projection, without the workspace: the partial sums go
+ * to a 4 MiB array built into this library (qknorm_qkv_projection_noalloc_max_bytes),
+ * which every GPU that loads the library holds until the process exits.
+ * Nothing is allocated: no cudaMalloc, no cudaFree, no allocating library
+ * call.  The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress, with that device current); make that first call
+ * before any stream capture.
+ * Limits: (Hq/256 + Hk/256) * T <= 1,048,576 (e.g. T = 32768 with Hq = Hk =
+ * 4096); larger calls return QKN_ERR_INVALID_ARG before any launch.
+ * Sharing: all calls on a device use the same array, and it keeps the last
+ * call's partial sums.  Every entry a call reads is written by that call's
+ * GEMM first, so nothing needs clearing; but two calls that can run at the
+ * same time on the GPU (different streams without ordering between them, or
+ * different host threads) race on the array and may corrupt each other's
+ * results.  Order such calls on one stream or with events.
+ * The paper has no counterpart: this is a deployment variant of this library.
+ */
+qkn_status qknorm_qkv_projection_noalloc(const void *x, int64_t x_stride, const void *w, int64_t w_stride,
+                                         void *qkv, int64_t qkv_stride, const void *gamma_q, const void *gamma_k,
+                                         int64_t T, int32_t D, int32_t Hq, int32_t Hk, int32_t Hv, float eps,
+                                         qkn_dtype dtype, void *stream);
+
+/* Bytes of the built-in scratch qknorm_qkv_projection_noalloc uses (4 MiB). */
+int64_t qknorm_qkv_projection_noalloc_max_bytes(void);
+
+/*
  * Every wait inside the projection kernel is bounded (2 s); one that runs out
  * records a non-zero code (1 = TMA producer, 2 = MMA issuer, 3 = epilogue)
  * and the kernel returns early with its output incomplete.  This call
