@@ -577,6 +577,8 @@ qkn_status prepare_projection(const void *x, int64_t x_stride, const void *w, in
     const int64_t N = (int64_t)Hq + Hk + Hv;
     if (N > INT32_MAX) return fail(QKN_ERR_INVALID_ARG, "Hq + Hk + Hv overflows");
     if (x_stride < D || w_stride < D || qkv_stride < N) return fail(QKN_ERR_INVALID_ARG, "row stride below width");
+    if (((T + 127) / 128) * (N / kTileN) > ((int64_t)1 << 30))
+        return fail(QKN_ERR_UNSUPPORTED, "more than 2^30 output tiles");
     if (!extent_ok(T, x_stride, D, 2) || !extent_ok(N, w_stride, D, 2) || !extent_ok(T, qkv_stride, N, 2))
         return fail(QKN_ERR_INVALID_ARG, "buffer extent overflows");
     if (T > 0 && (!x || !w || !qkv)) return fail(QKN_ERR_INVALID_ARG, "null pointer");
@@ -620,6 +622,8 @@ qkn_status launch_projection_gemm(const Projection &pr, float *q_sums, float *k_
     gp.q_tiles = pr.Hq / kTileN;
     gp.k_tiles = pr.Hk / kTileN;
     gp.n_tiles = pr.N / kTileN;
+    gp.m_tiles = (int32_t)((pr.T + qkn::gemm::kBM - 1) / qkn::gemm::kBM);
+    gp.num_tiles = gp.m_tiles * gp.n_tiles;
     gp.timeout_ns = kGemmTimeoutNs;
     const char *what = "";
     cudaError_t e = qkn::gemm::launch_qkv_gemm(pr.x, pr.x_stride, pr.w, pr.w_stride, pr.D, pr.N, gp,

@@ -148,10 +148,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                           const __grid_constant__ GemmParams p) {
     extern __shared__ uint8_t smem_raw[];
     __shared__ int s_abort;      // a wait in this CTA ran out
-    __shared__ int s_consumed;   // k-blocks whose MMAs were issued
-    __shared__ int s_issued;     // k-blocks whose TMA loads were issued
+    __shared__ int s_consumed;   // k-blocks (over all tiles) whose MMAs were issued
+    __shared__ int s_issued;     // k-blocks (over all tiles) whose TMA loads were issued
 
-    // 1024-byte aligned ring: A stages, then B stages, then the mbarriers.
+    // 1024-byte aligned ring: A stages, then B stages, then the mbarriers:
+    // full[kStages], empty[kStages], acc_full[2], acc_empty[2].
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     const uint32_t a_base = base;
@@ -159,20 +160,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t bars = base + kStages * kStageBytes;
     auto full_bar = [&](int s) { return bars + 8u * s; };
     auto empty_bar = [&](int s) { return bars + 8u * (kStages + s); };
-    const uint32_t acc_bar = bars + 16u * kStages;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem_raw + (bars - raw) + 8 * (2 * kStages + 1));
+    auto acc_full_bar = [&](int b) { return bars + 8u * (2 * kStages + b); };
+    auto acc_empty_bar = [&](int b) { return bars + 8u * (2 * kStages + 2 + b); };
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem_raw + (bars - raw) + 8 * (2 * kStages + 4));
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int m_tile = blockIdx.x;  // tokens (fastest, so a wave shares W tiles and X stays in L2)
-    const int n_tile = blockIdx.y;  // output columns
+    constexpr int kEpiWarps = 4;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(full_bar(s), 1);
             mbar_init(empty_bar(s), 1);
         }
-        mbar_init(acc_bar, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(acc_full_bar(b), 1);           // one tcgen05.commit per tile
+            mbar_init(acc_empty_bar(b), kEpiWarps);  // one arrival per epilogue warp
+        }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         prefetch_map(&tmap_x);
         prefetch_map(&tmap_w);
@@ -194,54 +198,76 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (warp == 0) {
         if (lane == 0) {  // ---------------------------------------------- TMA producer
-            int issued = 0;
-            for (int kb = 0; kb < p.k_blocks; ++kb) {
-                const int s = kb % kStages;
-                const int round = kb / kStages;
-                if (round > 0 && !mbar_wait(empty_bar(s), (round - 1) & 1, p.timeout_ns)) {
-                    record_timeout(kErrProducer, &s_abort);
-                    break;
+            int it = 0;   // k-blocks issued so far, over all of this CTA's tiles
+            for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
+                const int m_tile = tile % p.m_tiles;
+                const int n_tile = tile / p.m_tiles;
+                for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
+                    const int s = it % kStages;
+                    const int round = it / kStages;
+                    if (round > 0 && !mbar_wait(empty_bar(s), (round - 1) & 1, p.timeout_ns)) {
+                        record_timeout(kErrProducer, &s_abort);
+                        break;
+                    }
+                    mbar_expect_tx(full_bar(s), kStageBytes);
+                    tma_load_2d(a_base + s * kABytes, &tmap_x, kb * kBK, m_tile * kBM, full_bar(s));
+                    tma_load_2d(b_base + s * kBBytes, &tmap_w, kb * kBK, n_tile * kBN, full_bar(s));
                 }
-                mbar_expect_tx(full_bar(s), kStageBytes);
-                tma_load_2d(a_base + s * kABytes, &tmap_x, kb * kBK, m_tile * kBM, full_bar(s));
-                tma_load_2d(b_base + s * kBBytes, &tmap_w, kb * kBK, n_tile * kBN, full_bar(s));
-                issued = kb + 1;
             }
-            s_issued = issued;
+            s_issued = it;
         }
     } else if (warp == 1) {
         if (lane == 0) {  // ---------------------------------------------- MMA issuer
-            int kb = 0;
-            for (; kb < p.k_blocks; ++kb) {
-                const int s = kb % kStages;
-                if (!mbar_wait(full_bar(s), (kb / kStages) & 1, p.timeout_ns)) {
+            int it = 0;   // k-blocks consumed so far
+            int j = 0;    // tiles of this CTA so far
+            bool ok = true;
+            for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x, ++j) {
+                const int b = j & 1;
+                const int use = j >> 1;  // earlier uses of accumulator b
+                if (use > 0 && !mbar_wait(acc_empty_bar(b), (use - 1) & 1, p.timeout_ns)) {
                     record_timeout(kErrMma, &s_abort);
                     break;
                 }
                 fence_after_sync();
-                const uint32_t a_s = a_base + s * kABytes;
-                const uint32_t b_s = b_base + s * kBBytes;
+                const uint32_t acc = tmem + static_cast<uint32_t>(b * kAccCols);
+                for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
+                    const int s = it % kStages;
+                    if (!mbar_wait(full_bar(s), (it / kStages) & 1, p.timeout_ns)) {
+                        record_timeout(kErrMma, &s_abort);
+                        ok = false;
+                        break;
+                    }
+                    fence_after_sync();
+                    const uint32_t a_s = a_base + s * kABytes;
+                    const uint32_t b_s = b_base + s * kBBytes;
 #pragma unroll
-                for (int k = 0; k < kBK / kUmmaK; ++k)
-                    umma_bf16(tmem, sw128_kmajor_desc(a_s + k * kUmmaK * 2), sw128_kmajor_desc(b_s + k * kUmmaK * 2),
-                              kIdescBf16, (kb | k) != 0 ? 1u : 0u);
-                umma_commit(empty_bar(s));
+                    for (int k = 0; k < kBK / kUmmaK; ++k)
+                        umma_bf16(acc, sw128_kmajor_desc(a_s + k * kUmmaK * 2),
+                                  sw128_kmajor_desc(b_s + k * kUmmaK * 2), kIdescBf16, (kb | k) != 0 ? 1u : 0u);
+                    umma_commit(empty_bar(s));
+                }
+                umma_commit(acc_full_bar(b));  // also after a timeout, so the epilogue is not left waiting
             }
-            s_consumed = kb;
-            umma_commit(acc_bar);  // also after a timeout, so the epilogue is not left waiting
+            s_consumed = it;
         }
         __syncwarp();
     } else {  // ------------------------------------------------------------ epilogue
-        bool ok = mbar_wait(acc_bar, 0, p.timeout_ns);
-        if (!ok) record_timeout(kErrEpilogue, &s_abort);
-        ok = __all_sync(0xFFFFFFFFu, ok) && p.k_blocks > 0;
-        fence_after_sync();
-        if (ok) {
-            const int quarter = warp & 3;  // TMEM lanes this warp may read
+        const int quarter = warp & 3;  // TMEM lanes this warp may read
+        int j = 0;
+        for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++j) {
+            const int b = j & 1;
+            const int use = j >> 1;
+            bool ok = mbar_wait(acc_full_bar(b), use & 1, p.timeout_ns);
+            if (!ok) record_timeout(kErrEpilogue, &s_abort);
+            ok = __all_sync(0xFFFFFFFFu, ok) && p.k_blocks > 0;
+            if (!ok) break;
+            fence_after_sync();
+            const int m_tile = tile % p.m_tiles;
+            const int n_tile = tile / p.m_tiles;
             const int64_t row = static_cast<int64_t>(m_tile) * kBM + quarter * 32 + lane;
             const bool live = row < p.T;
             char *orow = p.qkv + (live ? row : 0) * p.qkv_stride_bytes + static_cast<int64_t>(n_tile) * kBN * 2;
-            const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+            const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(b * kAccCols);
             float ss = 0.0f;
 #pragma unroll 1
             for (int c = 0; c < kBN / 32; ++c) {
@@ -264,6 +290,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                         dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
                 }
             }
+            // The accumulator has been read: hand it back to the MMA thread.
+            fence_before_sync();
+            __syncwarp();
+            if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(acc_empty_bar(b)) : "memory");
             if (live) {
                 if (n_tile < p.q_tiles) {
                     if (p.q_sumsq) p.q_sumsq[static_cast<int64_t>(n_tile) * p.T + row] = ss;
@@ -280,8 +310,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // After a timeout, loads the MMA thread never consumed may still be in
         // flight: let them land (bounded) before this CTA's shared memory is
         // released.
-        for (int kb = s_consumed; kb < s_issued; ++kb)
-            (void)mbar_wait(full_bar(kb % kStages), (kb / kStages) & 1, p.timeout_ns);
+        for (int it = s_consumed; it < s_issued; ++it)
+            (void)mbar_wait(full_bar(it % kStages), (it / kStages) & 1, p.timeout_ns);
     }
     if (warp == 1) {
         fence_after_sync();
@@ -359,7 +389,14 @@ cudaError_t launch_qkv_gemm(const void *x, int64_t x_stride, const void *w, int6
         }
     }
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>((p.T + kBM - 1) / kBM), static_cast<unsigned>(p.n_tiles));
+    int sms = 0;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) {
+        *what = "cudaDeviceGetAttribute(multiprocessor count)";
+        return e;
+    }
+    // Persistent: one CTA per SM (its shared memory allows no second one).
+    const int grid = p.num_tiles < sms ? p.num_tiles : sms;
+    cfg.gridDim = dim3(static_cast<unsigned>(grid > 0 ? grid : 1));
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = kSmemBytes;
     cfg.stream = stream;

@@ -14,23 +14,33 @@
 // of those stored values.  The combine / factor / scale steps then run as the
 // usual apply pass (Phase A aggregation + Phase B).
 //
-// Kernel shape (one CTA per 128 x 256 output tile, 192 threads):
+// Kernel shape: persistent, one CTA of 192 threads per SM, each taking the
+// 128 x 256 output tiles blockIdx.x, blockIdx.x + gridDim.x, ... (tile index
+// = n_tile * m_tiles + m_tile, token tiles fastest, so the CTAs running at one
+// time share W tiles and X stays in L2):
 //   warp 0, lane 0 : TMA producer.  X tile [128 x 64] and W tile [256 x 64]
 //                    per k-block into a 4-stage shared-memory ring, 128-byte
-//                    swizzle, completion counted on an mbarrier per stage.
-//   warp 1         : allocates 256 TMEM columns (the fp32 accumulator,
-//                    lane = tile row); lane 0 issues tcgen05.mma (M=128,
-//                    N=256, K=16, bf16 in, fp32 accumulate), four per
-//                    k-block, and tcgen05.commit frees the stage when the
-//                    MMAs have read it; a final commit signals the epilogue.
+//                    swizzle, completion counted on an mbarrier per stage; the
+//                    ring runs on across tiles.
+//   warp 1         : allocates 512 TMEM columns, two fp32 accumulators of
+//                    128 lanes x 256 columns (lane = tile row); lane 0 issues
+//                    tcgen05.mma (M=128, N=256, K=16, bf16 in, fp32
+//                    accumulate), four per k-block, into the accumulator of
+//                    the tile's parity, frees each stage with tcgen05.commit
+//                    when its MMAs have read it, and signals the epilogue when
+//                    a tile's accumulator is complete.
 //   warps 2..5     : epilogue.  Warp w reads TMEM lanes 32*(w%4) .. +31
 //                    (one tile row per thread) in 32-column chunks, rounds to
 //                    bf16 (nearest even), stores the row's 512 bytes and, for
 //                    Q and K tiles, sums the squares of the rounded values in
-//                    column order (fp32 fma) and writes one partial per row.
+//                    column order (fp32 fma) and writes one partial per row;
+//                    then hands the accumulator back to the MMA thread.  With
+//                    two accumulators the epilogue of one tile overlaps the
+//                    MMAs of the next.
 // Every mbarrier wait is bounded by the global timer; on expiry the kernel
-// records a code in a device word, skips the rest of its work, frees its TMEM
-// and returns, so the context stays usable.
+// records a code in a device word, skips the rest of its work, lets its
+// in-flight loads land, frees its TMEM and returns, so the context stays
+// usable.
 #pragma once
 
 #include <cuda.h>
@@ -49,8 +59,9 @@ constexpr int kThreads = 192;
 constexpr int kABytes = kBM * kBK * 2;
 constexpr int kBBytes = kBN * kBK * 2;
 constexpr int kStageBytes = kABytes + kBBytes;
-constexpr int kTmemCols = 256;
-// ring + barriers (2 * kStages + 1 mbarriers) + TMEM address slot + 1 KB
+constexpr int kAccCols = kBN;      // fp32 columns of one accumulator
+constexpr int kTmemCols = 2 * kAccCols;
+// ring + barriers (2 * kStages + 4 mbarriers) + TMEM address slot + 1 KB
 // alignment slack for the 128-byte-swizzle atoms
 constexpr int kSmemBytes = kStages * kStageBytes + 1024 + 256;
 
@@ -64,6 +75,8 @@ struct GemmParams {
     int32_t q_tiles;         // Hq / kBN
     int32_t k_tiles;         // Hk / kBN
     int32_t n_tiles;         // N / kBN
+    int32_t m_tiles;         // ceil(T / kBM)
+    int32_t num_tiles;       // m_tiles * n_tiles
     uint64_t timeout_ns;     // bound on every mbarrier wait
 };
 

@@ -2,7 +2,7 @@
 """Benchmark of fused layerwise QK-RMSNorm on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
-                    [--workload prefill|decode|packed|gqa|tiny] [--tokens T]
+                    [--workload prefill|decode|packed|gqa|tiny|headwise|projection] [--tokens T]
 
 Prints ONE JSON line (rank 0).  A step is one pass of the whole path over one
 batch of synthetic input: for the default workload, one ``qknorm_layerwise``
@@ -57,7 +57,8 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
-    ap.add_argument("--workload", choices=["prefill", "decode", "packed", "gqa", "tiny", "headwise"], default="prefill")
+    ap.add_argument("--workload", choices=["prefill", "decode", "packed", "gqa", "tiny", "headwise", "projection"],
+                    default="prefill")
     ap.add_argument("--tokens", type=int, default=None, help="T for decode / packed workloads")
     ap.add_argument("--dtype", choices=["bf16", "f16", "e4m3"], default="bf16",
                     help="element type of the prefill workload (gamma is bf16 with e4m3)")
@@ -637,8 +638,235 @@ def reference(args) -> int:
     return 0
 
 
+# --------------------------------------------------------------------------- QKV projection workload
+
+PROJ_METRIC = "QKV projection + layerwise QK-Norm TFLOP/s (tensor-core roofline); µs per call"
+PROJ_UNIT = "TFLOP/s"
+
+
+def load_tensor_peak() -> dict:
+    """Measured dense bf16 tensor throughput (burst: the projection kernel is
+    timed on its own, not inside a seconds-long loop)."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {"tflops": float(d["bf16_tflops"]), "sustained": float(d.get("bf16_tflops_sustained", 0.0)),
+                "source": "measured cuBLAS bf16 GEMM (burst)"}
+    except (OSError, KeyError, ValueError):
+        return {"tflops": 1590.0, "sustained": 1400.0, "source": "fallback bf16 GEMM"}
+
+
+def _proj_flops(b) -> float:
+    return 2.0 * b.T * b.D * (b.Hq + b.Hk + b.Hv)
+
+
+def time_oracle_projection(b, budget_s: float, rows: int = 1) -> dict:
+    """The CPU oracle on `rows` tokens per call (projection of those rows in
+    double, then RMS-Norm of their Q and K columns), repeated until the budget
+    is spent; reported in the workload's unit (TFLOP/s of projection work)."""
+    import numpy as np
+
+    import oracle
+    xs = b.x.contiguous().view(torch.int16).numpy().view(np.uint16)
+    ws = b.w.contiguous().view(torch.int16).numpy().view(np.uint16)
+    gq = b.gamma_q.view(torch.int16).numpy().view(np.uint16)
+    gk = b.gamma_k.view(torch.int16).numpy().view(np.uint16)
+    calls, t0 = 0, time.perf_counter()
+    while True:
+        sel = [(calls * rows + i) % b.T for i in range(rows)]
+        y, _ = oracle.project_rows(xs, ws, sel)
+        oracle.rmsnorm_rows(np.ascontiguousarray(y[:, :b.Hq]), b.Hq, gq, b.eps)
+        oracle.rmsnorm_rows(np.ascontiguousarray(y[:, b.Hq:b.Hq + b.Hk]), b.Hk, gk, b.eps)
+        calls += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+    per_row = el / (calls * rows)
+    flops_per_row = _proj_flops(b) / b.T
+    return {"value": round(flops_per_row / per_row / 1e12, 9), "unit": PROJ_UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{calls * rows} token rows of {b.name} ({calls} calls), {el:.1f} s",
+            "us_per_token": per_row * 1e6}
+
+
+def native_projection(args) -> int:
+    rank, world, local = dist_env()
+    if not torch.cuda.is_available():
+        print(json.dumps({"metric": PROJ_METRIC, "error": "no CUDA device"}))
+        return 1
+    torch.cuda.set_device(local)
+    dev = torch.device(f"cuda:{local}")
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180), device_id=dev)
+    import attention_normalization_b200 as qk
+    qk.capi()
+    ranks = Ranks(dist, dev)
+
+    b = workloads.qkv_projection(T=args.tokens or 4096, seed=6 + rank * 1000)
+    N = b.Hq + b.Hk + b.Hv
+    flops = _proj_flops(b)
+    ws_bytes = qk.qkv_workspace_bytes(b.T, b.Hq, b.Hk)
+    set_bytes = 2 * (b.T * b.D + N * b.D + b.T * N) + ws_bytes
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    R = rotation_count(set_bytes, l2)
+    gq, gk = b.gamma_q.to(dev), b.gamma_k.to(dev)
+    sets = [{"x": b.x.to(dev), "w": b.w.to(dev), "qkv": torch.empty((b.T, N), dtype=torch.bfloat16, device=dev),
+             "ws": torch.empty((ws_bytes // 4,), dtype=torch.float32, device=dev),
+             "qs": torch.empty((b.Hq // 256, b.T), dtype=torch.float32, device=dev),
+             "ks": torch.empty((b.Hk // 256, b.T), dtype=torch.float32, device=dev)} for _ in range(R)]
+
+    def step(s):
+        qk.qknorm_qkv_projection(s["x"], s["w"], gq, gk, b.Hq, b.Hk, b.Hv, b.eps, qkv=s["qkv"], workspace=s["ws"])
+
+    def gemm_only(s):
+        qk.qknorm_qkv_gemm_stats(s["x"], s["w"], b.Hq, b.Hk, b.Hv, qkv=s["qkv"], q_sums=s["qs"], k_sums=s["ks"])
+
+    def cublas_unfused(s):  # library baseline: cuBLAS GEMM, then the fused layerwise kernel in place
+        torch.matmul(s["x"], s["w"].t(), out=s["qkv"])
+        q, k = s["qkv"][:, :b.Hq], s["qkv"][:, b.Hq:b.Hq + b.Hk]
+        qk.qknorm_layerwise(q, k, gq, gk, b.eps, q_out=q, k_out=k)
+
+    stream = torch.cuda.current_stream(dev)
+
+    def graph_time(fn, steps, warm):
+        for i in range(3):
+            fn(sets[i % R])
+        torch.cuda.synchronize()
+        gw, gt = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gw, capture_error_mode="thread_local"):
+            for i in range(warm):
+                fn(sets[i % R])
+        with torch.cuda.graph(gt, capture_error_mode="thread_local"):
+            for i in range(steps):
+                fn(sets[(warm + i) % R])
+        torch.cuda.synchronize()
+        graph_upload(gt, stream)
+        gw.replay()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        ranks.barrier()
+        torch.cuda.synchronize()
+        sampler.active.set()
+        e0.record(stream)
+        gt.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        sampler.active.clear()
+        ranks.barrier()
+        ms = ranks.max(e0.elapsed_time(e1))
+        del gw, gt
+        return ms
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    ms = graph_time(step, args.steps, args.warmup)
+    clocks = sampler.summary()
+    side_steps = max(3, min(args.steps, 200))
+    sampler = ClockSampler(local)  # the comparison runs get their own (unreported) sampler
+    sampler.start()
+    ms_gemm = graph_time(gemm_only, side_steps, args.warmup)
+    ms_cublas = graph_time(cublas_unfused, side_steps, args.warmup)
+    sampler.summary()
+    timeouts = qk.device_timeouts()
+
+    step_s = ms / 1e3 / args.steps
+    gemm_s = ms_gemm / 1e3 / side_steps
+    value = world * flops / step_s / 1e12
+    peak = load_tensor_peak()
+
+    # end to end: hidden states in from pinned host memory, the normalized QKV back out
+    h_x = b.x.contiguous().pin_memory()
+    h_qkv = torch.empty((b.T, N), dtype=torch.bfloat16, pin_memory=True)
+    s0 = sets[0]
+
+    def one():
+        s0["x"].copy_(h_x, non_blocking=True)
+        step(s0)
+        h_qkv.copy_(s0["qkv"], non_blocking=True)
+    for _ in range(2):
+        one()
+    e2e_steps = max(1, min(args.e2e_steps, args.steps))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    ranks.barrier()
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        one()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ranks.barrier()
+    ms_e2e = ranks.max(e0.elapsed_time(e1))
+    e2e = {"value": round(world * flops / (ms_e2e / 1e3 / e2e_steps) / 1e12, 2), "unit": PROJ_UNIT,
+           "h2d_bytes_per_step": h_x.numel() * 2, "d2h_bytes_per_step": h_qkv.numel() * 2, "steps": e2e_steps,
+           "ms_per_step": round(ms_e2e / e2e_steps, 4),
+           "path": "pinned host -> device copy of x, qknorm_qkv_projection (weights and gamma resident), "
+                   "device -> pinned host copy of qkv, one stream"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = time_oracle_projection(b, args.cpu_seconds)
+
+    if rank == 0:
+        between = (R - 1) * set_bytes
+        cfg = {"workload": b.name, "T": b.T, "D": b.D, "Hq": b.Hq, "Hk": b.Hk, "Hv": b.Hv, "io_dtype": "bfloat16",
+               "eps": b.eps, "form": "qknorm_qkv_projection: tcgen05 GEMM with per-tile squared sums in the "
+                                     "epilogue, then combine + scale of the Q and K columns in place",
+               "parallelism": f"replicas x{world} (tokens independent, no collective)",
+               "l2": f"rotating {R} sets of x, w, qkv, workspace ({R * set_bytes / 1e6:.1f} MB; "
+                     f"{between / 1e6:.1f} MB touched between reuses "
+                     + ("> 2 x" if between > 2 * l2 else "< 2 x") + f" {l2 / 1e6:.0f} MB L2)",
+               "timing": "CUDA graph of K captured C-ABI calls, CUDA events on the launching stream"}
+        gemm_tflops = flops / gemm_s / 1e12
+        line = {"metric": PROJ_METRIC, "value": round(value, 1), "unit": PROJ_UNIT, "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 6),
+                "us_per_call": round(step_s * 1e6, 2), "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded; OLMo2-7B-shaped projection, "
+                                                             "random weights)",
+                "config": cfg,
+                "roofline": {"bound": "tensor", "achieved": round(gemm_tflops, 1), "peak": peak["tflops"],
+                             "unit": "TFLOP/s", "frac": round(gemm_tflops / peak["tflops"], 4), "traffic": None,
+                             "peak_source": peak["source"], "kernel": "qkv_gemm_stats_kernel (timed alone)",
+                             "algorithmic_flops_per_launch": flops, "source_digest": source_digest()},
+                "breakdown_us": {"gemm_stats": round(gemm_s * 1e6, 2),
+                                 "combine_apply": round(step_s * 1e6 - gemm_s * 1e6, 2),
+                                 "cublas_matmul_plus_qknorm_layerwise": round(ms_cublas / side_steps * 1e3, 2)},
+                "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 2 * args.steps, "clocks": clocks,
+                "device_timeouts": timeouts, "impl": "native"}
+        print(json.dumps(line))
+    if dist is not None:
+        dist.destroy_process_group()
+    return 0
+
+
+def projection_reference(args) -> int:
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    b = workloads.qkv_projection(T=args.tokens or 4096, seed=6)
+    for _ in range(args.warmup):
+        time_oracle_projection(b, 0.0)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        time_oracle_projection(b, 0.0)
+    el = time.perf_counter() - t0
+    value = _proj_flops(b) / b.T / (el / args.steps) / 1e12
+    line = {"metric": PROJ_METRIC, "value": round(value, 9), "unit": PROJ_UNIT, "n_gpus": 0, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(el / args.steps * 1e3, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": b.name, "sample_tokens_per_step": 1}, "impl": "reference",
+            "cpu_baseline": {"value": round(value, 9), "unit": PROJ_UNIT, "cores": 1, "kind": "oracle",
+                             "sample": f"1 of {b.T} token rows of {b.name} per step, one thread"},
+            "e2e": {"value": round(value, 9), "unit": PROJ_UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+    return 0
+
+
 def main(argv=None) -> int:
     args = parse_args(argv)
+    if args.workload == "projection":
+        return projection_reference(args) if args.impl == "reference" else native_projection(args)
     if args.impl == "reference":
         return reference(args)
     return native(args)
