@@ -611,7 +611,18 @@ qkn_status check_projection_overlaps(const Projection &pr, const float *q_sums, 
     return QKN_OK;
 }
 
-qkn_status launch_projection_gemm(const Projection &pr, float *q_sums, float *k_sums, void *stream) {
+// Fused QK-Norm inside the GEMM: per-strip completion counters (zeroed on
+// the stream before the launch) and the Q / K scales.
+struct FusedNorm {
+    int *counters;
+    const void *gamma_q, *gamma_k;
+    float eps;
+};
+
+int64_t projection_m_tiles(int64_t T) { return (T + qkn::gemm::kBM - 1) / qkn::gemm::kBM; }
+
+qkn_status launch_projection_gemm(const Projection &pr, float *q_sums, float *k_sums, void *stream,
+                                  const FusedNorm *fuse = nullptr) {
     qkn::gemm::GemmParams gp{};
     gp.qkv = static_cast<char *>(pr.qkv);
     gp.qkv_stride_bytes = pr.qkv_stride * 2;
@@ -625,6 +636,17 @@ qkn_status launch_projection_gemm(const Projection &pr, float *q_sums, float *k_
     gp.m_tiles = (int32_t)((pr.T + qkn::gemm::kBM - 1) / qkn::gemm::kBM);
     gp.num_tiles = gp.m_tiles * gp.n_tiles;
     gp.timeout_ns = kGemmTimeoutNs;
+    if (fuse) {
+        gp.counters = fuse->counters;
+        gp.gamma_q = static_cast<const char *>(fuse->gamma_q);
+        gp.gamma_k = static_cast<const char *>(fuse->gamma_k);
+        gp.inv_hq = static_cast<float>(1.0 / static_cast<double>(pr.Hq));
+        gp.inv_hk = static_cast<float>(1.0 / static_cast<double>(pr.Hk));
+        gp.eps = fuse->eps;
+        cudaError_t me = cudaMemsetAsync(fuse->counters, 0, (size_t)(2 * gp.m_tiles) * sizeof(int),
+                                         static_cast<cudaStream_t>(stream));
+        if (me != cudaSuccess) return fail(QKN_ERR_CUDA, "clearing the strip counters: %s", cudaGetErrorString(me));
+    }
     const char *what = "";
     cudaError_t e = qkn::gemm::launch_qkv_gemm(pr.x, pr.x_stride, pr.w, pr.w_stride, pr.D, pr.N, gp,
                                                static_cast<cudaStream_t>(stream), &what);
@@ -896,7 +918,8 @@ qkn_status qknorm_qkv_gemm_stats(const void *x, int64_t x_stride, const void *w,
 
 int64_t qknorm_qkv_projection_workspace_bytes(int64_t T, int32_t Hq, int32_t Hk) {
     if (T < 0 || Hq <= 0 || Hk <= 0 || Hq % kTileN || Hk % kTileN) return -1;
-    return (int64_t)(Hq / kTileN + Hk / kTileN) * T * 4;
+    // partial sums [Hq/256][T] and [Hk/256][T], then two strip counters per 128 tokens
+    return (int64_t)(Hq / kTileN + Hk / kTileN) * T * 4 + 2 * projection_m_tiles(T) * 4;
 }
 
 qkn_status qknorm_qkv_projection(const void *x, int64_t x_stride, const void *w, int64_t w_stride, void *qkv,
@@ -917,8 +940,23 @@ qkn_status qknorm_qkv_projection(const void *x, int64_t x_stride, const void *w,
     float *q_sums = static_cast<float *>(workspace);
     float *k_sums = q_sums + (int64_t)(Hq / kTileN) * T;
     if ((st = check_projection_overlaps(pr, q_sums, k_sums, gamma_q, gamma_k)) != QKN_OK) return st;
+    {
+        const Region wsr = flat_region(workspace, need);
+        if (overlap(wsr, rows_region(qkv, pr.N, qkv_stride, T, 2)) || overlap(wsr, rows_region(x, D, x_stride, T, 2)) ||
+            overlap(wsr, rows_region(w, D, w_stride, pr.N, 2)) || overlap(wsr, flat_region(gamma_q, (int64_t)Hq * 2)) ||
+            overlap(wsr, flat_region(gamma_k, (int64_t)Hk * 2)))
+            return fail(QKN_ERR_INVALID_ARG, "the workspace overlaps an operand");
+    }
 
-    // Phase A aggregation + Phase B over the Q and K columns of qkv, in place.
+    // 16-byte aligned gamma: QK-Norm runs inside the GEMM (the CTA that stores
+    // a strip's last Q or K tile combines the strip's partial sums and scales
+    // it in place).
+    if (aligned16(gamma_q) && aligned16(gamma_k)) {
+        FusedNorm fz{reinterpret_cast<int *>(k_sums + (int64_t)(Hk / kTileN) * T), gamma_q, gamma_k, eps};
+        return launch_projection_gemm(pr, q_sums, k_sums, stream, &fz);
+    }
+    // Otherwise a second launch: Phase A aggregation + Phase B over the Q and
+    // K columns of qkv, in place.
     Call c;
     std::memset(&c, 0, sizeof(c));
     c.dtype = dtype;

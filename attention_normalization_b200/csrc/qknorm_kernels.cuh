@@ -324,9 +324,10 @@ __device__ __forceinline__ float combine_partials(const float *all, int64_t T, i
     return s;
 }
 
-// r = 1 / sqrt(S / H + eps), the mean formed as S * fl(1 / H).
+// r = 1 / sqrt(S / H + eps), the mean formed as S * fl(1 / H); the product
+// and the sum are one fused multiply-add (rounded once).
 __device__ __forceinline__ float rms_factor(float sumsq, float inv_div, float eps) {
-    return rsqrtf(sumsq * inv_div + eps);
+    return rsqrtf(__fmaf_rn(sumsq, inv_div, eps));
 }
 
 // Programmatic dependent launch (sm_90+).  Kernels here are launched with

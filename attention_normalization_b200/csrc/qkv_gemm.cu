@@ -141,6 +141,162 @@ __device__ __forceinline__ void record_timeout(int code, int *flag) {
 
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
+// Barrier among the epilogue warps only (named barrier 1; 0 is __syncthreads).
+__device__ __forceinline__ void epilogue_sync() {
+    asm volatile("bar.sync 1, %0;" ::"n"(kEpiWarps * 32) : "memory");
+}
+
+// True on every epilogue thread iff `ok` holds on all of them (a named
+// barrier with an AND reduction), so all epilogue warps take the same branch.
+__device__ __forceinline__ bool epilogue_all(bool ok) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.and.pred q, 1, %2, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"(static_cast<uint32_t>(ok)), "n"(kEpiWarps * 32)
+        : "memory");
+    return r != 0;
+}
+
+// Tile index -> (token tile, column tile): token tile fastest (within
+// groups of kGroupM token tiles when kGroupM > 0).
+__device__ __forceinline__ void tile_coords(int tile, int m_tiles, int n_tiles, int &m, int &n) {
+    if (kGroupM == 0) {
+        m = tile % m_tiles;
+        n = tile / m_tiles;
+        return;
+    }
+    const int per_group = kGroupM * n_tiles;
+    const int g = tile / per_group;
+    const int first = g * kGroupM;
+    const int gm = min(kGroupM, m_tiles - first);
+    const int r = tile - g * per_group;
+    m = first + r % gm;
+    n = r / gm;
+}
+
+// 8 bf16 (one 16-byte vector) -> (x * gamma) * r rounded to bf16, each
+// product in fp32 round-to-nearest.
+__device__ __forceinline__ uint4 scale8(uint4 x, uint4 g, float r) {
+    uint32_t xs[4] = {x.x, x.y, x.z, x.w}, gs[4] = {g.x, g.y, g.z, g.w}, ys[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float x0 = __uint_as_float(xs[i] << 16), x1 = __uint_as_float(xs[i] & 0xFFFF0000u);
+        const float g0 = __uint_as_float(gs[i] << 16), g1 = __uint_as_float(gs[i] & 0xFFFF0000u);
+        const __nv_bfloat162 h = __floats2bfloat162_rn(__fmul_rn(__fmul_rn(x0, g0), r), __fmul_rn(__fmul_rn(x1, g1), r));
+        ys[i] = *reinterpret_cast<const uint32_t *>(&h);
+    }
+    return make_uint4(ys[0], ys[1], ys[2], ys[3]);
+}
+
+__device__ __forceinline__ int ld_acquire(const int *p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Phase A aggregation + Phase B for one stored Q (tensor 0) or K (tensor 1)
+// tile, run by the 256 epilogue threads once every tile of its 128-token
+// strip has been counted: r = rsqrt(S / H + eps) with S the strip's partial
+// sums added in order p = 0, 1, ...; then (x * gamma) * r over the tile, in
+// place.  Partial sums written by other CTAs are read through L2 (.cg).
+__device__ __noinline__ void scale_tile(const GemmParams &p, int tensor, int m_tile, int n_tile, float *s_r) {
+    const int et = threadIdx.x - 64;  // 0 .. 255
+    const int P = tensor ? p.k_tiles : p.q_tiles;
+    const int first = tensor ? p.q_tiles : 0;  // the tensor's first column tile
+    const float *sums = tensor ? p.k_sumsq : p.q_sumsq;
+    const float inv = tensor ? p.inv_hk : p.inv_hq;
+    const int64_t row0 = static_cast<int64_t>(m_tile) * kBM;
+    const int rows = static_cast<int>(p.T - row0 < kBM ? p.T - row0 : kBM);
+    if (et < kBM) {
+        float r = 0.0f;
+        if (et < rows) {
+            // eight loads in flight at a time, added strictly in order p = 0, 1, ...
+            const float *col = sums + row0 + et;
+            float S = 0.0f;
+            for (int q0 = 0; q0 < P; q0 += 8) {
+                float v[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) v[i] = q0 + i < P ? __ldcg(col + static_cast<int64_t>(q0 + i) * p.T) : 0.0f;
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    if (q0 + i < P) S += v[i];
+            }
+            r = rsqrtf(__fmaf_rn(S, inv, p.eps));
+        }
+        s_r[et] = r;
+    }
+    epilogue_sync();
+    // warp e takes rows e, e + 8, ...; lane l the l-th 16-byte vector of each
+    // (a tile row is 32 vectors), so every load and store is one whole row
+    const int e = et >> 5, lane = et & 31;
+    const uint4 *gamma = reinterpret_cast<const uint4 *>(tensor ? p.gamma_k : p.gamma_q);
+    const uint4 g = __ldg(gamma + (n_tile - first) * (kBN / 8) + lane);
+    char *base = p.qkv + row0 * p.qkv_stride_bytes + static_cast<int64_t>(n_tile) * kBN * 2 + lane * 16;
+    constexpr int kBatch = 16;  // rows in flight per warp
+#pragma unroll 1
+    for (int r0 = e; r0 < rows; r0 += kEpiWarps * kBatch) {
+        uint4 xv[kBatch];
+#pragma unroll
+        for (int i = 0; i < kBatch; ++i) {
+            const int rr = r0 + kEpiWarps * i;
+            xv[i] = rr < rows ? __ldcg(reinterpret_cast<const uint4 *>(base + rr * p.qkv_stride_bytes))
+                              : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int i = 0; i < kBatch; ++i) {
+            const int rr = r0 + kEpiWarps * i;
+            if (rr < rows) *reinterpret_cast<uint4 *>(base + rr * p.qkv_stride_bytes) = scale8(xv[i], g, s_r[rr]);
+        }
+    }
+    epilogue_sync();  // s_r is reused by the next tile
+}
+
+// Scales this CTA's stored Q / K tiles from sequence index `from` up to (not
+// including) `upto`, in order, while their strips are complete.  Without
+// `wait` it stops at the first incomplete strip or after `budget` tiles; with
+// `wait` (only once all of this CTA's own tiles are stored and counted, so
+// it never waits on itself) it waits, bounded, for each strip.  Returns the
+// next index to scale.
+__device__ int scale_ready_tiles(const GemmParams &p, int from, int upto, bool wait, int budget, float *s_r,
+                                 int *abort_flag) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    while (from < upto && budget > 0) {
+        const int tile = blockIdx.x + from * gridDim.x;
+        int m_tile, n_tile;
+        tile_coords(tile, p.m_tiles, p.n_tiles, m_tile, n_tile);
+        const int tensor = n_tile < p.q_tiles ? 0 : (n_tile < p.q_tiles + p.k_tiles ? 1 : -1);
+        if (tensor < 0) {  // V tile: nothing to scale
+            ++from;
+            continue;
+        }
+        bool ready = true;
+        if (warp == 2 && lane == 0) {
+            const int *cnt = p.counters + tensor * p.m_tiles + m_tile;
+            const int P = tensor ? p.k_tiles : p.q_tiles;
+            ready = ld_acquire(cnt) >= P;
+            if (!ready && wait) {
+                const uint64_t t0 = global_ns();
+                while (!(ready = ld_acquire(cnt) >= P)) {
+                    if (global_ns() - t0 > p.timeout_ns) {
+                        record_timeout(kErrEpilogue, abort_flag);
+                        break;
+                    }
+                    __nanosleep(256);
+                }
+            }
+        }
+        if (!epilogue_all(ready)) break;  // the leader's answer, in every epilogue thread;
+                                          // with `wait` a timeout (reported) leaves the rest unscaled
+        scale_tile(p, tensor, m_tile, n_tile, s_r);
+        ++from;
+        --budget;
+    }
+    return from;
+}
 }  // namespace
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -150,6 +306,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     __shared__ int s_abort;      // a wait in this CTA ran out
     __shared__ int s_consumed;   // k-blocks (over all tiles) whose MMAs were issued
     __shared__ int s_issued;     // k-blocks (over all tiles) whose TMA loads were issued
+    __shared__ float s_half[2][kBM];  // second-half squared sums, by tile parity
+    __shared__ float s_r[kBM];        // RMS factors of the strip being scaled
 
     // 1024-byte aligned ring: A stages, then B stages, then the mbarriers:
     // full[kStages], empty[kStages], acc_full[2], acc_empty[2].
@@ -166,7 +324,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    constexpr int kEpiWarps = 4;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
@@ -200,8 +357,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {  // ---------------------------------------------- TMA producer
             int it = 0;   // k-blocks issued so far, over all of this CTA's tiles
             for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
-                const int m_tile = tile % p.m_tiles;
-                const int n_tile = tile / p.m_tiles;
+                int m_tile, n_tile;
+                tile_coords(tile, p.m_tiles, p.n_tiles, m_tile, n_tile);
                 for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
                     const int s = it % kStages;
                     const int round = it / kStages;
@@ -252,25 +409,35 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __syncwarp();
     } else {  // ------------------------------------------------------------ epilogue
-        const int quarter = warp & 3;  // TMEM lanes this warp may read
+        const int quarter = warp & 3;          // TMEM lanes this warp may read
+        const int half = (warp - 2) >> 2;      // which column range of the tile (0 with 4 warps)
+        const int rl = quarter * 32 + lane;    // row within the tile
+        const bool fused = p.counters != nullptr;
+        int norm_next = 0;  // next of this CTA's tiles to scale (fused QK-Norm)
+        bool timed_out = false;
         int j = 0;
         for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++j) {
             const int b = j & 1;
             const int use = j >> 1;
             bool ok = mbar_wait(acc_full_bar(b), use & 1, p.timeout_ns);
             if (!ok) record_timeout(kErrEpilogue, &s_abort);
-            ok = __all_sync(0xFFFFFFFFu, ok) && p.k_blocks > 0;
-            if (!ok) break;
+            // the same decision in every epilogue warp, so the named barriers below always match
+            if (!epilogue_all(ok && p.k_blocks > 0)) {
+                timed_out = true;
+                break;
+            }
             fence_after_sync();
-            const int m_tile = tile % p.m_tiles;
-            const int n_tile = tile / p.m_tiles;
-            const int64_t row = static_cast<int64_t>(m_tile) * kBM + quarter * 32 + lane;
+            int m_tile, n_tile;
+            tile_coords(tile, p.m_tiles, p.n_tiles, m_tile, n_tile);
+            const int64_t row = static_cast<int64_t>(m_tile) * kBM + rl;
             const bool live = row < p.T;
-            char *orow = p.qkv + (live ? row : 0) * p.qkv_stride_bytes + static_cast<int64_t>(n_tile) * kBN * 2;
-            const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(b * kAccCols);
+            const int col0 = half * kEpiCols;
+            char *orow = p.qkv + (live ? row : 0) * p.qkv_stride_bytes + (static_cast<int64_t>(n_tile) * kBN + col0) * 2;
+            const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) +
+                                   static_cast<uint32_t>(b * kAccCols + col0);
             float ss = 0.0f;
 #pragma unroll 1
-            for (int c = 0; c < kBN / 32; ++c) {
+            for (int c = 0; c < kEpiCols / 32; ++c) {
                 uint32_t r[32];
                 tmem_ld32(taddr + c * 32, r);
                 uint32_t packed[16];
@@ -294,14 +461,30 @@ __global__ void __launch_bounds__(kThreads, 1)
             fence_before_sync();
             __syncwarp();
             if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(acc_empty_bar(b)) : "memory");
-            if (live) {
-                if (n_tile < p.q_tiles) {
-                    if (p.q_sumsq) p.q_sumsq[static_cast<int64_t>(n_tile) * p.T + row] = ss;
-                } else if (n_tile < p.q_tiles + p.k_tiles) {
-                    if (p.k_sumsq) p.k_sumsq[static_cast<int64_t>(n_tile - p.q_tiles) * p.T + row] = ss;
+
+            const int tensor = n_tile < p.q_tiles ? 0 : (n_tile < p.q_tiles + p.k_tiles ? 1 : -1);
+            if (tensor >= 0) {  // Q or K tile: its partial sums (V columns have none)
+                if (kEpiSplit == 2 && half == 1) s_half[b][rl] = ss;
+                if (kEpiSplit == 2) epilogue_sync();
+                if (half == 0 && live) {
+                    const float total = kEpiSplit == 2 ? ss + s_half[b][rl] : ss;
+                    if (tensor == 0) {
+                        if (p.q_sumsq) p.q_sumsq[static_cast<int64_t>(n_tile) * p.T + row] = total;
+                    } else {
+                        if (p.k_sumsq) p.k_sumsq[static_cast<int64_t>(n_tile - p.q_tiles) * p.T + row] = total;
+                    }
                 }
+                if (fused) __threadfence();  // this thread's stores of the tile, before the count
+                epilogue_sync();             // s_half[b] has been read
+                // Count the tile on its strip (after every thread's fence above).
+                if (fused && warp == 2 && lane == 0) atomicAdd(p.counters + tensor * p.m_tiles + m_tile, 1);
             }
+            // Scale earlier tiles of this CTA whose strips are complete (at
+            // most two per tile, inside the MMAs' slack).
+            if (fused) norm_next = scale_ready_tiles(p, norm_next, j + 1, false, 2, s_r, &s_abort);
         }
+        if (fused && !timed_out)
+            scale_ready_tiles(p, norm_next, j, true, 1 << 30, s_r, &s_abort);
     }
 
     fence_before_sync();

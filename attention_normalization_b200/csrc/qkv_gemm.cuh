@@ -14,10 +14,12 @@
 // of those stored values.  The combine / factor / scale steps then run as the
 // usual apply pass (Phase A aggregation + Phase B).
 //
-// Kernel shape: persistent, one CTA of 192 threads per SM, each taking the
-// 128 x 256 output tiles blockIdx.x, blockIdx.x + gridDim.x, ... (tile index
-// = n_tile * m_tiles + m_tile, token tiles fastest, so the CTAs running at one
-// time share W tiles and X stays in L2):
+// Kernel shape: persistent, one CTA of 320 threads per SM, each taking the
+// 128 x 256 output tiles blockIdx.x, blockIdx.x + gridDim.x, ...  The token
+// tile runs fastest (tile = column tile * token tiles + token tile), so the
+// CTAs running at one time share a few W tiles while X stays in L2.
+// (Groups of kGroupM token tiles, column tile next, were measured 6% slower
+// at the OLMo2-7B shape and are off by default.)  Roles:
 //   warp 0, lane 0 : TMA producer.  X tile [128 x 64] and W tile [256 x 64]
 //                    per k-block into a 4-stage shared-memory ring, 128-byte
 //                    swizzle, completion counted on an mbarrier per stage; the
@@ -29,14 +31,28 @@
 //                    the tile's parity, frees each stage with tcgen05.commit
 //                    when its MMAs have read it, and signals the epilogue when
 //                    a tile's accumulator is complete.
-//   warps 2..5     : epilogue.  Warp w reads TMEM lanes 32*(w%4) .. +31
-//                    (one tile row per thread) in 32-column chunks, rounds to
-//                    bf16 (nearest even), stores the row's 512 bytes and, for
-//                    Q and K tiles, sums the squares of the rounded values in
-//                    column order (fp32 fma) and writes one partial per row;
-//                    then hands the accumulator back to the MMA thread.  With
+//   warps 2..9     : epilogue, two warps per TMEM lane quarter.  Warp w
+//                    reads TMEM lanes 32*(w%4) .. +31 (one tile row per
+//                    thread); warps 2..5 take columns 0..127 of the tile and
+//                    warps 6..9 columns 128..255, in 32-column chunks.  Each
+//                    value is rounded to bf16 (nearest even) and stored; for
+//                    Q and K tiles each half sums the squares of its rounded
+//                    values in column order (fp32 fma), and the tile's
+//                    partial for the row is (first half) + (second half).
+//                    Then the accumulator goes back to the MMA thread.  With
 //                    two accumulators the epilogue of one tile overlaps the
 //                    MMAs of the next.
+// Fused QK-Norm (when `counters` is set): after storing a Q or K tile and its
+// partial sums, the epilogue makes its writes visible (fence) and counts the
+// tile on its strip's counter (one per 128-token strip and tensor).  Between
+// tiles it scales, in order, those of its own earlier Q / K tiles whose strips
+// are complete (counter = the tensor's tile count, read with acquire): the
+// strip's partial sums are added in order p = 0, 1, ... (fp32), r = rsqrt(S /
+// H + eps) per token, and the tile is rewritten in place as (x * gamma) * r
+// rounded to bf16, read back through L2 -- Phase A's aggregation and Phase B's
+// scaling without a second pass over HBM.  Once all of its own tiles are
+// counted it waits (bounded) for its remaining strips; it never waits while
+// it still owes tiles, so no CTA waits on one that waits on it.
 // Every mbarrier wait is bounded by the global timer; on expiry the kernel
 // records a code in a device word, skips the rest of its work, lets its
 // in-flight loads land, frees its TMEM and returns, so the context stays
@@ -55,7 +71,18 @@ constexpr int kBN = 256;           // tile columns = one partial-sum shard
 constexpr int kBK = 64;            // k-block: 64 bf16 = one 128-byte swizzle row
 constexpr int kStages = 4;
 constexpr int kUmmaK = 16;         // K of one tcgen05.mma kind::f16
-constexpr int kThreads = 192;
+#ifndef QKN_GEMM_EPI_WARPS
+#define QKN_GEMM_EPI_WARPS 8
+#endif
+#ifndef QKN_GEMM_GROUP_M
+#define QKN_GEMM_GROUP_M 0
+#endif
+constexpr int kEpiWarps = QKN_GEMM_EPI_WARPS;  // 4 or 8: one or two per TMEM lane quarter
+static_assert(kEpiWarps == 4 || kEpiWarps == 8, "the epilogue has 4 or 8 warps");
+constexpr int kEpiSplit = kEpiWarps / 4;       // warps sharing one lane quarter (column split)
+constexpr int kEpiCols = kBN / kEpiSplit;      // tile columns per epilogue warp
+constexpr int kThreads = 64 + 32 * kEpiWarps;
+constexpr int kGroupM = QKN_GEMM_GROUP_M;      // token tiles per raster group; 0 = one group
 constexpr int kABytes = kBM * kBK * 2;
 constexpr int kBBytes = kBN * kBK * 2;
 constexpr int kStageBytes = kABytes + kBBytes;
@@ -78,6 +105,13 @@ struct GemmParams {
     int32_t m_tiles;         // ceil(T / kBM)
     int32_t num_tiles;       // m_tiles * n_tiles
     uint64_t timeout_ns;     // bound on every mbarrier wait
+    // Fused QK-Norm (all null / unused when counters is null).
+    int *counters;           // [2][m_tiles] tiles stored per strip, zero at launch
+    const char *gamma_q;     // [Hq] bf16
+    const char *gamma_k;     // [Hk] bf16
+    float inv_hq;            // fl(1 / Hq)
+    float inv_hk;            // fl(1 / Hk)
+    float eps;
 };
 
 // Error codes written to the device word when a wait runs out.

@@ -830,7 +830,7 @@ def native_projection(args) -> int:
                              "peak_source": peak["source"], "kernel": "qkv_gemm_stats_kernel (timed alone)",
                              "algorithmic_flops_per_launch": flops, "source_digest": source_digest()},
                 "breakdown_us": {"gemm_stats": round(gemm_s * 1e6, 2),
-                                 "combine_apply": round(step_s * 1e6 - gemm_s * 1e6, 2),
+                                 "norm_in_epilogue_extra": round(step_s * 1e6 - gemm_s * 1e6, 2),
                                  "cublas_matmul_plus_qknorm_layerwise": round(ms_cublas / side_steps * 1e3, 2)},
                 "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 2 * args.steps, "clocks": clocks,
                 "device_timeouts": timeouts, "impl": "native"}

@@ -189,3 +189,37 @@ def test_projection_is_deterministic_and_matches_combine_apply():
     torch.cuda.synchronize()
     assert torch.equal(a, c)
     assert torch.equal(a[:, :b.Hq], qo) and torch.equal(a[:, b.Hq:b.Hq + b.Hk], ko)
+
+
+def _unaligned_copy(t: torch.Tensor) -> torch.Tensor:
+    """The same values in a buffer whose start is not 16-byte aligned."""
+    buf = torch.empty(t.numel() + 8, dtype=t.dtype, device=t.device)
+    v = buf[1:t.numel() + 1]
+    v.copy_(t)
+    assert v.data_ptr() % 16 != 0
+    return v
+
+
+@pytest.mark.parametrize("T,D,Hq,Hk,Hv", [
+    (1000, 136, 1024, 512, 512),    # ragged last strip; Q and K with different tile counts
+    (4096, 64, 2048, 512, 512),     # many strips finishing at once
+    (129, 64, 256, 256, 0),         # one tile per strip and tensor
+    (2048, 320, 512, 1536, 256),    # K wider than Q
+])
+def test_fused_norm_equals_the_two_launch_path(T, D, Hq, Hk, Hv):
+    """With 16-byte aligned gamma the strip that stores its last tile scales
+    itself inside the GEMM; with unaligned gamma a second kernel does it.
+    Both combine the same partial sums in the same order, so they agree bit
+    for bit; sampled rows are also checked against the oracle."""
+    b = workloads.qkv_projection(T=T, D=D, Hq=Hq, Hk=Hk, Hv=Hv, seed=T + Hk)
+    x, w = b.x.to(DEV), b.w.to(DEV)
+    gq, gk = b.gamma_q.to(DEV), b.gamma_k.to(DEV)
+    fused = qk.qknorm_qkv_projection(x, w, gq, gk, Hq, Hk, Hv, b.eps)
+    two = qk.qknorm_qkv_projection(x, w, _unaligned_copy(gq), _unaligned_copy(gk), Hq, Hk, Hv, b.eps)
+    plain, _, _ = qk.qknorm_qkv_gemm_stats(x, w, Hq, Hk, Hv)
+    torch.cuda.synchronize()
+    assert torch.equal(fused, two)
+    rows = _sample_rows(T, 12, T + 1)
+    proj = check_projection(b, plain, rows)
+    check_normalized(b, proj, fused, rows)
+    assert qk.device_timeouts() == 0
