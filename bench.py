@@ -123,11 +123,17 @@ def load_peaks() -> dict:
         return {"hbm_gbs": FALLBACK_HBM_GBS, "source": "fallback"}
 
 
-def source_digest() -> str:
-    """Digest of the CUDA sources and headers: profile counters apply only to
-    the build they were taken from."""
+KERNEL_SOURCES = {
+    "rows": ["qknorm_kernels.cuh", "qknorm_api.cu"],
+    "projection": ["qkv_gemm.cu", "qkv_gemm.cuh", "qknorm_api.cu"],
+}
+
+
+def source_digest(kind: str = "rows") -> str:
+    """Digest of the sources of one kernel family and the public headers:
+    profile counters apply only to the build they were taken from."""
     h = hashlib.sha256()
-    files = sorted(glob.glob(os.path.join(ROOT, "attention_normalization_b200", "csrc", "*"))
+    files = sorted([os.path.join(ROOT, "attention_normalization_b200", "csrc", f) for f in KERNEL_SOURCES[kind]]
                    + glob.glob(os.path.join(ROOT, "include", "*.h")))
     for p in files:
         h.update(os.path.basename(p).encode())
@@ -826,9 +832,10 @@ def native_projection(args) -> int:
                                                              "random weights)",
                 "config": cfg,
                 "roofline": {"bound": "tensor", "achieved": round(gemm_tflops, 1), "peak": peak["tflops"],
-                             "unit": "TFLOP/s", "frac": round(gemm_tflops / peak["tflops"], 4), "traffic": None,
+                             "unit": "TFLOP/s", "frac": round(gemm_tflops / peak["tflops"], 4),
+                             "traffic": profiled_traffic(b.name, source_digest("projection")),
                              "peak_source": peak["source"], "kernel": "qkv_gemm_stats_kernel (timed alone)",
-                             "algorithmic_flops_per_launch": flops, "source_digest": source_digest()},
+                             "algorithmic_flops_per_launch": flops, "source_digest": source_digest("projection")},
                 "breakdown_us": {"gemm_stats": round(gemm_s * 1e6, 2),
                                  "norm_in_epilogue_extra": round(step_s * 1e6 - gemm_s * 1e6, 2),
                                  "cublas_matmul_plus_qknorm_layerwise": round(ms_cublas / side_steps * 1e3, 2)},
