@@ -986,9 +986,9 @@ qkn_status qknorm_qkv_projection_noalloc(const void *x, int64_t x_stride, const 
                                      eps, nullptr, 0, dtype, stream);
     if (need > kNoAllocScratchBytes)
         return fail(QKN_ERR_INVALID_ARG,
-                    "needs %lld bytes of partial sums; the built-in scratch holds %lld "
-                    "((Hq/256 + Hk/256) * T must stay at or below %lld)",
-                    (long long)need, (long long)kNoAllocScratchBytes, (long long)(kNoAllocScratchBytes / 4));
+                    "needs %lld bytes of workspace (partial sums and strip counters); the built-in scratch "
+                    "holds %lld",
+                    (long long)need, (long long)kNoAllocScratchBytes);
     void *ws = nullptr;
     qkn_status st = noalloc_scratch(&ws);
     if (st != QKN_OK) return st;

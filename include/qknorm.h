@@ -209,14 +209,17 @@ qkn_status qknorm_qkv_projection(const void *x, int64_t x_stride, const void *w,
  * call.  The first call on a device looks up the array's device address
  * (cudaGetSymbolAddress, with that device current); make that first call
  * before any stream capture.
- * Limits: (Hq/256 + Hk/256) * T <= 1,048,576 (e.g. T = 32768 with Hq = Hk =
- * 4096); larger calls return QKN_ERR_INVALID_ARG before any launch.
+ * Limits: the call's workspace, qknorm_qkv_projection_workspace_bytes(T, Hq,
+ * Hk) = (Hq/256 + Hk/256) * T * 4 + 8 * ceil(T / 128) bytes, must fit in the
+ * 4 MiB (e.g. T = 32000 with Hq = Hk = 4096); larger calls return
+ * QKN_ERR_INVALID_ARG before any launch.
  * Sharing: all calls on a device use the same array, and it keeps the last
- * call's partial sums.  Every entry a call reads is written by that call's
- * GEMM first, so nothing needs clearing; but two calls that can run at the
- * same time on the GPU (different streams without ordering between them, or
- * different host threads) race on the array and may corrupt each other's
- * results.  Order such calls on one stream or with events.
+ * call's contents.  Each call clears the strip counters it uses on its
+ * stream (cudaMemsetAsync, which allocates nothing) and writes every partial
+ * sum before reading it; but two calls that can run at the same time on the
+ * GPU (different streams without ordering between them, or different host
+ * threads) race on the array and may corrupt each other's results.  Order
+ * such calls on one stream or with events.
  * The paper has no counterpart: this is a deployment variant of this library.
  */
 qkn_status qknorm_qkv_projection_noalloc(const void *x, int64_t x_stride, const void *w, int64_t w_stride,

@@ -53,7 +53,7 @@ def test_noalloc_matches_the_workspace_entry_point_on_two_calls():
 
 
 def test_noalloc_rejects_a_call_beyond_its_scratch():
-    """(Hq/256 + Hk/256) * T above 1,048,576 is refused before any launch."""
+    """A workspace beyond the 4 MiB scratch is refused before any launch."""
     b = workloads.ProjectionBatch("too_big", 32769, 64, 4096, 4096, 0, None, None, None, None)
     lib = qk.capi()
     st = lib.qknorm_qkv_projection_noalloc(0x10000, 64, 0x20000000, 64, 0x40000000, 8192, 0x60000000, 0x60010000,
