@@ -357,6 +357,18 @@ qkn_status plan_call(const Call &c, qkn_launch &L) {
     if ((st = qknorm_plan_shape(items, c.units_max, c.vectorized ? 1 : 0, sms, elem_bytes(c.dtype), &L)) !=
         QKN_OK)
         return fail(st, "planning failed");
+    if (MODE == qkn::kStats && L.kernel == QKN_KERNEL_REGISTER && items > sms) {
+        // The partial-sum pass only reads and holds no gamma: more vectors per
+        // lane (up to 8; 4 for 1-byte elements) keep more bytes in flight,
+        // one warp (or fewer lanes) per row, 128-thread CTAs.
+        const int cap = elem_bytes(c.dtype) == 1 ? 4 : 8;
+        int nv = 1;
+        while (nv < cap && (int64_t)nv * 32 < c.units_max) nv *= 2;
+        if ((int64_t)nv * 128 >= c.units_max) {
+            L.vec_per_thread = nv;
+            L.threads = 128;
+        }
+    }
     const void *fn = kernel_for<MODE>(c.dtype, L, c.tail);
     if (!fn) return fail(QKN_ERR_UNSUPPORTED, "no kernel for the planned launch");
     if ((st = blocks_per_sm(fn, dev, L.threads, 0, &bps)) != QKN_OK) return st;

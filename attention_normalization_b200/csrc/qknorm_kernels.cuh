@@ -317,10 +317,22 @@ __device__ __forceinline__ float block_sum(float v, float (*red)[32], int &slot)
     return s;
 }
 
-// Phase A aggregation: the P partial sums of token t, added in order p = 0..P-1.
-__device__ __forceinline__ float combine_partials(const float *all, int64_t T, int P, int64_t t) {
+// Phase A aggregation: the P partial sums of token t (all[p * T + t]) added
+// in order p = 0, 1, ..., P-1 in fp32.  The lanes of a warp that share row t
+// split the loads: lane li (< width, a power of two <= 32, the lane's index
+// within its row group) loads partials li, li + width, ..., and every lane
+// adds all P values in order from shuffles, so each gets the same sequential
+// sum with one load instead of P.  Every lane of the warp must call it
+// (inactive rows pass active = false and load nothing).
+__device__ __forceinline__ float combine_partials_lanes(const float *all, int64_t T, int P, int64_t t, bool active,
+                                                        int li, int width) {
     float s = 0.0f;
-    for (int p = 0; p < P; ++p) s += __ldg(all + static_cast<int64_t>(p) * T + t);
+    for (int p0 = 0; p0 < P; p0 += width) {
+        const int q = p0 + li;
+        const float v = (active && q < P) ? __ldg(all + static_cast<int64_t>(q) * T + t) : 0.0f;
+        const int n = P - p0 < width ? P - p0 : width;
+        for (int i = 0; i < n; ++i) s += __shfl_sync(0xFFFFFFFFu, v, i, width);
+    }
     return s;
 }
 
@@ -473,7 +485,9 @@ __global__ void __launch_bounds__(RegisterBounds<NV>::kMaxThreads)
 
         float r;
         if (MODE == kApply) {
-            r = active ? rms_factor(combine_partials(sums_all, T, nparts, t), inv_div, p.eps) : 0.0f;
+            const float S = gsize < 32 ? combine_partials_lanes(sums_all, T, nparts, t, active, gl, gsize)
+                                       : combine_partials_lanes(sums_all, T, nparts, t, active, lane, 32);
+            r = active ? rms_factor(S, inv_div, p.eps) : 0.0f;
         } else {
             float S = sumsq_pairs<E, NV>(v);
             S = gsize < 32 ? segment_sum(S, gsize) : warp_sum(S);
@@ -539,7 +553,7 @@ __global__ void __launch_bounds__(1024) rows_twopass_kernel(const __grid_constan
 
         float r;
         if (MODE == kApply) {
-            r = rms_factor(combine_partials(d.sumsq_all, p.T, d.P, t), d.inv_div, p.eps);
+            r = rms_factor(combine_partials_lanes(d.sumsq_all, p.T, d.P, t, true, tid & 31, 32), d.inv_div, p.eps);
         } else {
             float acc = 0.0f;
             for (int u = tid; u < units; u += nthr) {
