@@ -646,7 +646,8 @@ qkn_status launch_projection_gemm(const Projection &pr, float *q_sums, float *k_
     gp.k_tiles = pr.Hk / kTileN;
     gp.n_tiles = pr.N / kTileN;
     gp.m_tiles = (int32_t)((pr.T + qkn::gemm::kBM - 1) / qkn::gemm::kBM);
-    gp.num_tiles = gp.m_tiles * gp.n_tiles;
+    gp.m_units = (int32_t)((pr.T + qkn::gemm::kBM * qkn::gemm::kCta - 1) / (qkn::gemm::kBM * qkn::gemm::kCta));
+    gp.num_units = gp.m_units * gp.n_tiles;
     gp.timeout_ns = kGemmTimeoutNs;
     if (fuse) {
         gp.counters = fuse->counters;

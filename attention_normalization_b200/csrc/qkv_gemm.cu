@@ -71,6 +71,41 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map
         : "memory");
 }
 
+// With a CTA pair the load lands in this CTA's shared memory and its bytes are
+// counted on `bar`, the leader CTA's barrier (a shared::cluster address).
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap *map, int32_t c0, int32_t c1,
+                                                 uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, "
+        "%3}], [%4];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar)
+        : "memory");
+}
+
+// ---------------------------------------------------------------- clusters
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+// The shared::cluster address of the variable at shared::cta address `addr`
+// in the cluster's CTA `rank`.
+__device__ __forceinline__ uint32_t map_to_cta(uint32_t addr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+    return r;
+}
+
+// All threads of both CTAs of the pair.
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
 __device__ __forceinline__ void prefetch_map(const CUtensorMap *map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -100,23 +135,32 @@ __device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t saddr) {
 // 4-5 = 1), A and B bf16 (bits 7-9 and 10-12 = 1), both K-major (bits 15, 16
 // = 0), N >> 3 in bits 17-22, M >> 4 in bits 24-28.
 constexpr uint32_t kIdescBf16 = (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(kBN >> 3) << 17) |
-                                (static_cast<uint32_t>(kBM >> 4) << 24);
+                                (static_cast<uint32_t>((kBM * kCta) >> 4) << 24);
 
 __device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                           uint32_t accumulate) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        "tcgen05.mma.cta_group::%5.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "n"(kCta)
         : "memory");
 }
 
 // The mbarrier receives one arrival when every tcgen05.mma this thread issued
-// so far has completed.
+// so far has completed; with a CTA pair, the barrier at the same offset in
+// both CTAs does.
 __device__ __forceinline__ void umma_commit(uint32_t bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
-                 : "memory");
+    if constexpr (kCta == 1) {
+        asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                     : "memory");
+    } else {
+        asm volatile(
+            "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+                bar),
+            "h"(static_cast<uint16_t>(0x3))
+            : "memory");
+    }
 }
 
 // 32 consecutive fp32 columns of this thread's TMEM lane.
@@ -161,21 +205,22 @@ __device__ __forceinline__ bool epilogue_all(bool ok) {
     return r != 0;
 }
 
-// Tile index -> (token tile, column tile): token tile fastest (within
-// groups of kGroupM token tiles when kGroupM > 0).
-__device__ __forceinline__ void tile_coords(int tile, int m_tiles, int n_tiles, int &m, int &n) {
-    if (kGroupM == 0) {
-        m = tile % m_tiles;
-        n = tile / m_tiles;
-        return;
-    }
-    const int per_group = kGroupM * n_tiles;
-    const int g = tile / per_group;
-    const int first = g * kGroupM;
-    const int gm = min(kGroupM, m_tiles - first);
-    const int r = tile - g * per_group;
-    m = first + r % gm;
-    n = r / gm;
+// This CTA's j-th tile: work unit u = cluster + j * clusters (a unit is one
+// MMA's 128 * kCta tokens x 256 columns; token blocks fastest, so the units
+// running at one time share a few W tiles while X stays in L2); the CTA takes
+// token tile m_unit * kCta + rank of it.
+struct TileRef {
+    int m_tile, n_tile;
+};
+__device__ __forceinline__ TileRef cta_tile(const GemmParams &p, int j, int rank) {
+    const int clusters = static_cast<int>(gridDim.x) / kCta;
+    const int u = static_cast<int>(blockIdx.x) / kCta + j * clusters;
+    return TileRef{(u % p.m_units) * kCta + rank, u / p.m_units};
+}
+__device__ __forceinline__ int cta_tile_count(const GemmParams &p) {
+    const int clusters = static_cast<int>(gridDim.x) / kCta;
+    const int c = static_cast<int>(blockIdx.x) / kCta;
+    return c < p.num_units ? (p.num_units - c + clusters - 1) / clusters : 0;
 }
 
 // 8 bf16 (one 16-byte vector) -> (x * gamma) * r rounded to bf16, each
@@ -262,12 +307,15 @@ __device__ __noinline__ void scale_tile(const GemmParams &p, int tensor, int m_t
 // it never waits on itself) it waits, bounded, for each strip.  Returns the
 // next index to scale.
 __device__ int scale_ready_tiles(const GemmParams &p, int from, int upto, bool wait, int budget, float *s_r,
-                                 int *abort_flag) {
+                                 int *abort_flag, int rank) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     while (from < upto && budget > 0) {
-        const int tile = blockIdx.x + from * gridDim.x;
-        int m_tile, n_tile;
-        tile_coords(tile, p.m_tiles, p.n_tiles, m_tile, n_tile);
+        const TileRef tr = cta_tile(p, from, rank);
+        const int m_tile = tr.m_tile, n_tile = tr.n_tile;
+        if (m_tile >= p.m_tiles) {  // the pair's second token tile lies past T
+            ++from;
+            continue;
+        }
         const int tensor = n_tile < p.q_tiles ? 0 : (n_tile < p.q_tiles + p.k_tiles ? 1 : -1);
         if (tensor < 0) {  // V tile: nothing to scale
             ++from;
@@ -307,10 +355,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     __shared__ int s_consumed;   // k-blocks (over all tiles) whose MMAs were issued
     __shared__ int s_issued;     // k-blocks (over all tiles) whose TMA loads were issued
     __shared__ float s_half[2][kBM];  // second-half squared sums, by tile parity
-    __shared__ float s_r[kBM];        // RMS factors of the strip being scaled
+    __shared__ float s_r[kBM];        // RMS factors of the tile being scaled
 
     // 1024-byte aligned ring: A stages, then B stages, then the mbarriers:
-    // full[kStages], empty[kStages], acc_full[2], acc_empty[2].
+    // full[kStages], empty[kStages], acc_full[2], acc_empty[2].  The layout
+    // is the same in both CTAs of a pair, so one offset names a barrier in
+    // either.
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     const uint32_t a_base = base;
@@ -324,15 +374,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    const int rank = kCta == 2 ? static_cast<int>(cluster_rank()) : 0;
+    const bool leader = rank == 0;  // issues the MMAs and owns the barriers they wait on
+    const int n_tiles_cta = cta_tile_count(p);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
-            mbar_init(full_bar(s), 1);
-            mbar_init(empty_bar(s), 1);
+            mbar_init(full_bar(s), 1);   // the leader's expect-tx arrival; bytes of both CTAs
+            mbar_init(empty_bar(s), 1);  // one tcgen05.commit
         }
         for (int b = 0; b < 2; ++b) {
-            mbar_init(acc_full_bar(b), 1);           // one tcgen05.commit per tile
-            mbar_init(acc_empty_bar(b), kEpiWarps);  // one arrival per epilogue warp
+            mbar_init(acc_full_bar(b), 1);                   // one tcgen05.commit per tile
+            mbar_init(acc_empty_bar(b), kEpiWarps * kCta);   // every epilogue warp of the group
         }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         prefetch_map(&tmap_x);
@@ -341,24 +394,33 @@ __global__ void __launch_bounds__(kThreads, 1)
         s_consumed = 0;
         s_issued = 0;
     }
-    if (warp == 1) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
-                     "r"(kTmemCols)
-                     : "memory");
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    if (warp == 1) {  // both CTAs of a pair allocate, with the same warp and address
+        if constexpr (kCta == 1) {
+            asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                             smem_u32(tmem_slot)),
+                         "r"(kTmemCols)
+                         : "memory");
+            asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+        } else {
+            asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                             smem_u32(tmem_slot)),
+                         "r"(kTmemCols)
+                         : "memory");
+            asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+        }
     }
     fence_before_sync();
     __syncthreads();
+    if constexpr (kCta == 2) cluster_sync();  // the peer's barriers are initialized before any remote use
     fence_after_sync();
     const uint32_t tmem = *tmem_slot;
     pdl_wait();  // X may come from the previous kernel in the stream; qkv may still be read by it
 
     if (warp == 0) {
-        if (lane == 0) {  // ---------------------------------------------- TMA producer
+        if (lane == 0) {  // ---------------------------------------------- TMA producer (each CTA)
             int it = 0;   // k-blocks issued so far, over all of this CTA's tiles
-            for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
-                int m_tile, n_tile;
-                tile_coords(tile, p.m_tiles, p.n_tiles, m_tile, n_tile);
+            for (int j = 0; j < n_tiles_cta; ++j) {
+                const TileRef tr = cta_tile(p, j, rank);
                 for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
                     const int s = it % kStages;
                     const int round = it / kStages;
@@ -366,19 +428,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                         record_timeout(kErrProducer, &s_abort);
                         break;
                     }
-                    mbar_expect_tx(full_bar(s), kStageBytes);
-                    tma_load_2d(a_base + s * kABytes, &tmap_x, kb * kBK, m_tile * kBM, full_bar(s));
-                    tma_load_2d(b_base + s * kBBytes, &tmap_w, kb * kBK, n_tile * kBN, full_bar(s));
+                    if (leader) mbar_expect_tx(full_bar(s), kTxBytes);
+                    const int ax = kb * kBK, ay = tr.m_tile * kBM;
+                    const int by = tr.n_tile * kBN + rank * kBNLocal;
+                    if constexpr (kCta == 1) {
+                        tma_load_2d(a_base + s * kABytes, &tmap_x, ax, ay, full_bar(s));
+                        tma_load_2d(b_base + s * kBBytes, &tmap_w, ax, by, full_bar(s));
+                    } else {
+                        const uint32_t lbar = map_to_cta(full_bar(s), 0);
+                        tma_load_2d_pair(a_base + s * kABytes, &tmap_x, ax, ay, lbar);
+                        tma_load_2d_pair(b_base + s * kBBytes, &tmap_w, ax, by, lbar);
+                    }
                 }
             }
             s_issued = it;
         }
     } else if (warp == 1) {
-        if (lane == 0) {  // ---------------------------------------------- MMA issuer
+        if (leader && lane == 0) {  // ------------------------------------ MMA issuer (leader CTA)
             int it = 0;   // k-blocks consumed so far
-            int j = 0;    // tiles of this CTA so far
             bool ok = true;
-            for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x, ++j) {
+            for (int j = 0; ok && j < n_tiles_cta; ++j) {
                 const int b = j & 1;
                 const int use = j >> 1;  // earlier uses of accumulator b
                 if (use > 0 && !mbar_wait(acc_empty_bar(b), (use - 1) & 1, p.timeout_ns)) {
@@ -403,20 +472,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                                   sw128_kmajor_desc(b_s + k * kUmmaK * 2), kIdescBf16, (kb | k) != 0 ? 1u : 0u);
                     umma_commit(empty_bar(s));
                 }
-                umma_commit(acc_full_bar(b));  // also after a timeout, so the epilogue is not left waiting
+                umma_commit(acc_full_bar(b));  // also after a timeout, so the epilogues are not left waiting
             }
             s_consumed = it;
         }
         __syncwarp();
-    } else {  // ------------------------------------------------------------ epilogue
+    } else {  // ------------------------------------------------------------ epilogue (each CTA)
         const int quarter = warp & 3;          // TMEM lanes this warp may read
         const int half = (warp - 2) >> 2;      // which column range of the tile (0 with 4 warps)
         const int rl = quarter * 32 + lane;    // row within the tile
         const bool fused = p.counters != nullptr;
+        // the leader's acc_empty barriers: every epilogue warp of the group arrives there
+        const uint32_t acc_empty_leader[2] = {kCta == 2 ? map_to_cta(acc_empty_bar(0), 0) : acc_empty_bar(0),
+                                              kCta == 2 ? map_to_cta(acc_empty_bar(1), 0) : acc_empty_bar(1)};
         int norm_next = 0;  // next of this CTA's tiles to scale (fused QK-Norm)
         bool timed_out = false;
         int j = 0;
-        for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++j) {
+        for (; j < n_tiles_cta; ++j) {
             const int b = j & 1;
             const int use = j >> 1;
             bool ok = mbar_wait(acc_full_bar(b), use & 1, p.timeout_ns);
@@ -427,8 +499,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
             }
             fence_after_sync();
-            int m_tile, n_tile;
-            tile_coords(tile, p.m_tiles, p.n_tiles, m_tile, n_tile);
+            const TileRef tr = cta_tile(p, j, rank);
+            const int m_tile = tr.m_tile, n_tile = tr.n_tile;
+            const bool tile_live = m_tile < p.m_tiles;  // the pair's second token tile may lie past T
             const int64_t row = static_cast<int64_t>(m_tile) * kBM + rl;
             const bool live = row < p.T;
             const int col0 = half * kEpiCols;
@@ -460,10 +533,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             // The accumulator has been read: hand it back to the MMA thread.
             fence_before_sync();
             __syncwarp();
-            if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(acc_empty_bar(b)) : "memory");
+            if (lane == 0) {
+                if constexpr (kCta == 1)
+                    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(acc_empty_bar(b)) : "memory");
+                else
+                    mbar_arrive_cluster(acc_empty_leader[b]);
+            }
 
             const int tensor = n_tile < p.q_tiles ? 0 : (n_tile < p.q_tiles + p.k_tiles ? 1 : -1);
-            if (tensor >= 0) {  // Q or K tile: its partial sums (V columns have none)
+            if (tensor >= 0 && tile_live) {  // Q or K tile: its partial sums (V columns have none)
                 if (kEpiSplit == 2 && half == 1) s_half[b][rl] = ss;
                 if (kEpiSplit == 2) epilogue_sync();
                 if (half == 0 && live) {
@@ -481,24 +559,30 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             // Scale earlier tiles of this CTA whose strips are complete (at
             // most two per tile, inside the MMAs' slack).
-            if (fused) norm_next = scale_ready_tiles(p, norm_next, j + 1, false, 2, s_r, &s_abort);
+            if (fused) norm_next = scale_ready_tiles(p, norm_next, j + 1, false, 2, s_r, &s_abort, rank);
         }
         if (fused && !timed_out)
-            scale_ready_tiles(p, norm_next, j, true, 1 << 30, s_r, &s_abort);
+            scale_ready_tiles(p, norm_next, j, true, 1 << 30, s_r, &s_abort, rank);
     }
 
     fence_before_sync();
     __syncthreads();
-    if (threadIdx.x == 0 && s_abort) {
+    if (threadIdx.x == 0 && s_abort && leader) {
         // After a timeout, loads the MMA thread never consumed may still be in
-        // flight: let them land (bounded) before this CTA's shared memory is
-        // released.
+        // flight (both CTAs' bytes count on the leader's barriers): let them
+        // land, bounded, before shared memory is released.
         for (int it = s_consumed; it < s_issued; ++it)
             (void)mbar_wait(full_bar(it % kStages), (it / kStages) & 1, p.timeout_ns);
     }
+    if constexpr (kCta == 2) cluster_sync();  // no CTA leaves while its peer may still use its memory
     if (warp == 1) {
         fence_after_sync();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+        if constexpr (kCta == 1)
+            asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
+                         : "memory");
+        else
+            asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
+                         : "memory");
     }
 }
 
@@ -538,6 +622,7 @@ bool encode_bf16_rows(PFN_cuTensorMapEncodeTiled_v12000 fn, CUtensorMap *map, co
 
 constexpr int kMaxDevices = 64;
 bool g_smem_set[kMaxDevices] = {};
+int g_groups[kMaxDevices] = {};  // resident CTA groups per device
 std::mutex g_smem_mu;
 
 }  // namespace
@@ -551,7 +636,8 @@ cudaError_t launch_qkv_gemm(const void *x, int64_t x_stride, const void *w, int6
         return e;
     }
     CUtensorMap tx, tw;
-    if (!encode_bf16_rows(fn, &tx, x, D, p.T, x_stride, kBM) || !encode_bf16_rows(fn, &tw, w, D, N, w_stride, kBN)) {
+    if (!encode_bf16_rows(fn, &tx, x, D, p.T, x_stride, kBM) ||
+        !encode_bf16_rows(fn, &tw, w, D, N, w_stride, kBNLocal)) {  // each CTA stages kBNLocal W rows
         *what = "cuTensorMapEncodeTiled";
         return cudaErrorInvalidValue;
     }
@@ -572,22 +658,50 @@ cudaError_t launch_qkv_gemm(const void *x, int64_t x_stride, const void *w, int6
         }
     }
     cudaLaunchConfig_t cfg = {};
-    int sms = 0;
-    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) {
-        *what = "cudaDeviceGetAttribute(multiprocessor count)";
-        return e;
-    }
-    // Persistent: one CTA per SM (its shared memory allows no second one).
-    const int grid = p.num_tiles < sms ? p.num_tiles : sms;
-    cfg.gridDim = dim3(static_cast<unsigned>(grid > 0 ? grid : 1));
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = kSmemBytes;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = kCta;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = kCta == 2 ? 2 : 1;
+    // Persistent: one CTA per SM (its shared memory allows no second one), as
+    // many CTA groups as can be resident at once, so every group runs from
+    // the start (a group that waited for a free SM would finish last).
+    int groups = 0;
+    {
+        std::lock_guard<std::mutex> lk(g_smem_mu);
+        if (dev >= 0 && dev < kMaxDevices && g_groups[dev] > 0) groups = g_groups[dev];
+    }
+    if (groups == 0) {
+        if constexpr (kCta == 1) {
+            e = cudaDeviceGetAttribute(&groups, cudaDevAttrMultiProcessorCount, dev);
+            if (e != cudaSuccess) {
+                *what = "cudaDeviceGetAttribute(multiprocessor count)";
+                return e;
+            }
+        } else {
+            cfg.gridDim = dim3(kCta);
+            e = cudaOccupancyMaxActiveClusters(&groups, reinterpret_cast<const void *>(qkv_gemm_stats_kernel), &cfg);
+            if (e != cudaSuccess) {
+                *what = "cudaOccupancyMaxActiveClusters";
+                return e;
+            }
+        }
+        if (groups < 1) {
+            *what = "no resident CTA group";
+            return cudaErrorInvalidConfiguration;
+        }
+        std::lock_guard<std::mutex> lk(g_smem_mu);
+        if (dev >= 0 && dev < kMaxDevices) g_groups[dev] = groups;
+    }
+    const int units = p.num_units < groups ? p.num_units : groups;
+    cfg.gridDim = dim3(static_cast<unsigned>((units > 0 ? units : 1) * kCta));
     void *args[] = {&tx, &tw, const_cast<GemmParams *>(&p)};
     e = cudaLaunchKernelExC(&cfg, reinterpret_cast<const void *>(qkv_gemm_stats_kernel), args);
     if (e != cudaSuccess) *what = "cudaLaunchKernelExC";

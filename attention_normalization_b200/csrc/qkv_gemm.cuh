@@ -69,8 +69,17 @@ namespace gemm {
 constexpr int kBM = 128;           // tile rows (tokens) = TMEM lanes
 constexpr int kBN = 256;           // tile columns = one partial-sum shard
 constexpr int kBK = 64;            // k-block: 64 bf16 = one 128-byte swizzle row
-constexpr int kStages = 4;
 constexpr int kUmmaK = 16;         // K of one tcgen05.mma kind::f16
+#ifndef QKN_GEMM_CTA_GROUP
+#define QKN_GEMM_CTA_GROUP 2
+#endif
+// CTAs per MMA: 2 = a cluster of two CTAs on two SMs runs one 256 x 256 tile
+// with tcgen05 cta_group::2 (each CTA holds 128 rows of X and 128 rows of W
+// per k-block and receives 128 x 256 of the result); 1 = one CTA per 128 x 256
+// tile.
+constexpr int kCta = QKN_GEMM_CTA_GROUP;
+static_assert(kCta == 1 || kCta == 2, "one or two CTAs per MMA");
+constexpr int kStages = kCta == 2 ? 6 : 4;
 #ifndef QKN_GEMM_EPI_WARPS
 #define QKN_GEMM_EPI_WARPS 8
 #endif
@@ -83,9 +92,11 @@ constexpr int kEpiSplit = kEpiWarps / 4;       // warps sharing one lane quarter
 constexpr int kEpiCols = kBN / kEpiSplit;      // tile columns per epilogue warp
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr int kGroupM = QKN_GEMM_GROUP_M;      // token tiles per raster group; 0 = one group
+constexpr int kBNLocal = kBN / kCta;           // W rows (output columns) each CTA stages
 constexpr int kABytes = kBM * kBK * 2;
-constexpr int kBBytes = kBN * kBK * 2;
-constexpr int kStageBytes = kABytes + kBBytes;
+constexpr int kBBytes = kBNLocal * kBK * 2;
+constexpr int kStageBytes = kABytes + kBBytes;    // per CTA and stage
+constexpr int kTxBytes = kStageBytes * kCta;      // bytes one full barrier phase counts
 constexpr int kAccCols = kBN;      // fp32 columns of one accumulator
 constexpr int kTmemCols = 2 * kAccCols;
 // ring + barriers (2 * kStages + 4 mbarriers) + TMEM address slot + 1 KB
@@ -102,8 +113,9 @@ struct GemmParams {
     int32_t q_tiles;         // Hq / kBN
     int32_t k_tiles;         // Hk / kBN
     int32_t n_tiles;         // N / kBN
-    int32_t m_tiles;         // ceil(T / kBM)
-    int32_t num_tiles;       // m_tiles * n_tiles
+    int32_t m_tiles;         // ceil(T / kBM): 128-token tiles (= strips)
+    int32_t m_units;         // ceil(T / (kBM * kCta)): token blocks of one MMA
+    int32_t num_units;       // m_units * n_tiles: work units (one per CTA group)
     uint64_t timeout_ns;     // bound on every mbarrier wait
     // Fused QK-Norm (all null / unused when counters is null).
     int *counters;           // [2][m_tiles] tiles stored per strip, zero at launch
