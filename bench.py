@@ -769,16 +769,22 @@ def native_projection(args) -> int:
     sampler.start()
     ms = graph_time(step, args.steps, args.warmup)
     clocks = sampler.summary()
-    side_steps = max(3, min(args.steps, 200))
+    # Comparison (informational): short graphs of the pipeline, the GEMM with
+    # partial sums alone and cuBLAS + qknorm_layerwise, interleaved round by
+    # round so that clock and power drift hits all three alike; medians.
+    side_steps = max(3, min(args.steps, 20))
     sampler = ClockSampler(local)  # the comparison runs get their own (unreported) sampler
     sampler.start()
-    ms_gemm = graph_time(gemm_only, side_steps, args.warmup)
-    ms_cublas = graph_time(cublas_unfused, side_steps, args.warmup)
+    side = {"pipeline": [], "gemm": [], "cublas": []}
+    for _ in range(5):
+        side["pipeline"].append(graph_time(step, side_steps, 3) / side_steps)
+        side["gemm"].append(graph_time(gemm_only, side_steps, 3) / side_steps)
+        side["cublas"].append(graph_time(cublas_unfused, side_steps, 3) / side_steps)
     sampler.summary()
+    side = {k: statistics.median(v) for k, v in side.items()}
     timeouts = qk.device_timeouts()
 
     step_s = ms / 1e3 / args.steps
-    gemm_s = ms_gemm / 1e3 / side_steps
     value = world * flops / step_s / 1e12
     peak = load_tensor_peak()
 
@@ -824,21 +830,24 @@ def native_projection(args) -> int:
                      f"{between / 1e6:.1f} MB touched between reuses "
                      + ("> 2 x" if between > 2 * l2 else "< 2 x") + f" {l2 / 1e6:.0f} MB L2)",
                "timing": "CUDA graph of K captured C-ABI calls, CUDA events on the launching stream"}
-        gemm_tflops = flops / gemm_s / 1e12
+        # the fused kernel is the step's only kernel (beside a 256-byte memset)
+        kernel_tflops = flops / step_s / 1e12
         line = {"metric": PROJ_METRIC, "value": round(value, 1), "unit": PROJ_UNIT, "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 6),
                 "us_per_call": round(step_s * 1e6, 2), "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded; OLMo2-7B-shaped projection, "
                                                              "random weights)",
                 "config": cfg,
-                "roofline": {"bound": "tensor", "achieved": round(gemm_tflops, 1), "peak": peak["tflops"],
-                             "unit": "TFLOP/s", "frac": round(gemm_tflops / peak["tflops"], 4),
+                "roofline": {"bound": "tensor", "achieved": round(kernel_tflops, 1), "peak": peak["tflops"],
+                             "unit": "TFLOP/s", "frac": round(kernel_tflops / peak["tflops"], 4),
                              "traffic": profiled_traffic(b.name, source_digest("projection")),
-                             "peak_source": peak["source"], "kernel": "qkv_gemm_stats_kernel (timed alone)",
+                             "peak_source": peak["source"],
+                             "kernel": "qkv_gemm_stats_kernel with the fused QK-Norm (the step's one kernel)",
                              "algorithmic_flops_per_launch": flops, "source_digest": source_digest("projection")},
-                "breakdown_us": {"gemm_stats": round(gemm_s * 1e6, 2),
-                                 "norm_in_epilogue_extra": round(step_s * 1e6 - gemm_s * 1e6, 2),
-                                 "cublas_matmul_plus_qknorm_layerwise": round(ms_cublas / side_steps * 1e3, 2)},
+                "comparison_us": {"how": f"medians of 5 interleaved rounds of {side_steps}-call graphs",
+                                  "projection_with_qk_norm": round(side["pipeline"] * 1e3, 2),
+                                  "gemm_with_partial_sums_only": round(side["gemm"] * 1e3, 2),
+                                  "cublas_matmul_plus_qknorm_layerwise": round(side["cublas"] * 1e3, 2)},
                 "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 2 * args.steps, "clocks": clocks,
                 "device_timeouts": timeouts, "impl": "native"}
         print(json.dumps(line))
