@@ -25,7 +25,7 @@ from . import _clib
 from ._clib import QknLaunch, QKNormError
 
 __all__ = ["qknorm_layerwise", "qknorm_headwise", "qknorm_qkv_gemm_stats", "qknorm_qkv_projection",
-           "qkv_workspace_bytes", "device_timeouts", "qknorm_partial_stats", "qknorm_combine_apply", "gamma_dtype",
+           "qkv_workspace_bytes", "device_timeouts", "qknorm_tp_layerwise", "TpExchange", "qknorm_partial_stats", "qknorm_combine_apply", "gamma_dtype",
            "qknorm_layerwise_plan", "qknorm_layerwise_host", "qknorm_packed_host",
            "plan_shape", "plan_grid", "regions_overlap", "capi", "version", "QknLaunch", "QKNormError"]
 
@@ -261,6 +261,85 @@ def device_timeouts(device=None) -> int:
     with torch.cuda.device(device if device is not None else torch.cuda.current_device()):
         _clib.check(capi().qknorm_device_timeouts(ctypes.byref(code)), "qknorm_device_timeouts")
     return code.value
+
+
+# --------------------------------------------------------------------------- tensor-parallel form
+
+class TpExchange:
+    """Receive buffers of an R-rank tensor-parallel group, all on one device
+    (the single-GPU form, where one call runs every rank), and the call epoch.
+    Each buffer holds [R][T][2] 64-bit words; they start zeroed and every call
+    takes the next epoch, so they are never cleared again."""
+
+    def __init__(self, R: int, T: int, device):
+        n = capi().qknorm_tp_recv_bytes(R, T)
+        if n < 0:
+            raise ValueError(f"invalid R={R} or T={T} for the exchange")
+        self.R, self.T = R, T
+        self.buffers = [torch.zeros((max(n, 8) // 8,), dtype=torch.int64, device=device) for _ in range(R)]
+        self.epoch = 0
+
+    def pointers(self):
+        return [b.data_ptr() for b in self.buffers]
+
+    def next_epoch(self) -> int:
+        self.epoch += 1
+        if self.epoch >= 2 ** 32:
+            raise RuntimeError("exchange epochs exhausted; make a new TpExchange")
+        return self.epoch
+
+
+def qknorm_tp_layerwise(q_shards, k_shards, gamma_q_shards, gamma_k_shards, Hq_full: int, Hk_full: int,
+                        eps: float = 1e-6, *, exchange: TpExchange | None = None, recv=None, epoch: int | None = None,
+                        R: int | None = None, first_rank: int = 0, q_out=None, k_out=None, in_place: bool = False,
+                        blocks_per_rank: int = 0, timeout_ns: int = 0, stream=None):
+    """Tensor-parallel layerwise QK-Norm: runs ranks first_rank ..
+    first_rank + len(q_shards) - 1 of an R-rank group; shard j holds Q columns
+    of rank first_rank + j for all T tokens.  The ranks exchange only their
+    scalar partial sums (through ``exchange`` / ``recv``).  Returns the lists
+    ``(q_out, k_out)``."""
+    n_local = len(q_shards)
+    if not (n_local == len(k_shards) == len(gamma_q_shards) == len(gamma_k_shards)) or n_local < 1:
+        raise ValueError("one Q shard, K shard and gamma slice each per local rank")
+    T, hq, sq = _rows(q_shards[0], "q_shards[0]")
+    _, hk, sk = _rows(k_shards[0], "k_shards[0]")
+    dev, dt = q_shards[0].device, q_shards[0].dtype
+    for j in range(n_local):
+        for t, name, (H, s) in ((q_shards[j], f"q_shards[{j}]", (hq, sq)), (k_shards[j], f"k_shards[{j}]", (hk, sk))):
+            _same(dev, dt, t, name)
+            Tj, Hj, sj = _rows(t, name)
+            if (Tj, Hj) != (T, H) or (T > 1 and sj != s):
+                raise ValueError(f"{name}: every local shard must have the same shape and row stride")
+    if exchange is not None:
+        recv = exchange.pointers()
+        R = exchange.R if R is None else R
+        epoch = exchange.next_epoch() if epoch is None else epoch
+    if recv is None or epoch is None:
+        raise ValueError("pass an exchange, or recv pointers and an epoch")
+    R = n_local if R is None else R
+    if len(recv) != R:
+        raise ValueError(f"{len(recv)} receive buffers for R={R}")
+    if in_place:
+        q_out, k_out = list(q_shards), list(k_shards)
+    if q_out is None:
+        q_out = [_out_like(q, sq) for q in q_shards]
+    if k_out is None:
+        k_out = [_out_like(k, sk) for k in k_shards]
+    gdt = gamma_dtype(dt)
+    gq = [_vec(g, f"gamma_q_shards[{j}]", hq, gdt, dev) for j, g in enumerate(gamma_q_shards)]
+    gk = [_vec(g, f"gamma_k_shards[{j}]", hk, gdt, dev) for j, g in enumerate(gamma_k_shards)]
+    P = ctypes.c_void_p
+
+    def arr(xs):
+        return (P * len(xs))(*[int(x) for x in xs])
+    with torch.cuda.device(dev):
+        st = capi().qknorm_tp_layerwise(R, first_rank, n_local, arr([q.data_ptr() for q in q_shards]),
+                                        arr([q.data_ptr() for q in q_out]), arr(gq), sq, hq, int(Hq_full),
+                                        arr([k.data_ptr() for k in k_shards]), arr([k.data_ptr() for k in k_out]),
+                                        arr(gk), sk, hk, int(Hk_full), T, float(eps), _DTYPES[dt], arr(recv),
+                                        int(epoch), int(blocks_per_rank), int(timeout_ns), _stream_handle(stream, dev))
+    _clib.check(st, "qknorm_tp_layerwise")
+    return q_out, k_out
 
 
 def qknorm_layerwise_plan(q_in, k_in, gamma_q, gamma_k, eps: float = 1e-6, *, q_out=None,

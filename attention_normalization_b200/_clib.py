@@ -61,6 +61,9 @@ PROTOTYPES = {
     "qknorm_qkv_projection_noalloc": (_st, [_vp, _i64, _vp, _i64, _vp, _i64, _vp, _vp, _i64, _i32, _i32, _i32,
                                             _i32, _f32, _dt, _vp]),
     "qknorm_qkv_projection_noalloc_max_bytes": (_i64, []),
+    "qknorm_tp_recv_bytes": (_i64, [_i32, _i64]),
+    "qknorm_tp_layerwise": (_st, [_i32, _i32, _i32, _vp, _vp, _vp, _i64, _i32, _i32, _vp, _vp, _vp, _i64, _i32, _i32,
+                                  _i64, _f32, _dt, _vp, ctypes.c_uint32, _i32, _u64, _vp]),
     "qknorm_last_error": (ctypes.c_char_p, []),
     "qknorm_version": (ctypes.c_int, []),
     "qknorm_register_max_threads": (_i32, [_i32]),

@@ -51,7 +51,8 @@ def build(force: bool = False, ptxas_verbose: bool = False, quiet: bool = False)
     cmd = [_nvcc(), *ARCH_FLAGS, "-O3", "-lineinfo", "-std=c++17", "--expt-relaxed-constexpr",
            "-Xcompiler", "-fPIC,-Wall", "-shared", "-cudart", "static",
            "-I", INCLUDE, "-I", CSRC,
-           os.path.join(CSRC, "qknorm_api.cu"), os.path.join(CSRC, "qkv_gemm.cu"), "-o", tmp]
+           os.path.join(CSRC, "qknorm_api.cu"), os.path.join(CSRC, "qkv_gemm.cu"), os.path.join(CSRC, "qknorm_tp.cu"),
+           "-o", tmp]
     if ptxas_verbose:
         cmd[1:1] = ["-Xptxas", "-v"]
     r = subprocess.run(cmd, capture_output=True, text=True)

@@ -18,6 +18,7 @@
 #include "qknorm_plan.h"
 #include "qknorm_kernels.cuh"
 #include "qkv_gemm.cuh"
+#include "qknorm_tp.cuh"
 
 #ifndef QKNORM_VERSION
 #define QKNORM_VERSION 100  // 0.1.0
@@ -1013,10 +1014,118 @@ int64_t qknorm_qkv_projection_noalloc_max_bytes(void) { return kNoAllocScratchBy
 
 qkn_status qknorm_device_timeouts(int32_t *code) {
     if (!code) return fail(QKN_ERR_INVALID_ARG, "null pointer");
-    int v = 0;
+    int v = 0, w = 0;
     cudaError_t e = qkn::gemm::read_and_clear_timeout(&v);
+    if (e == cudaSuccess) e = qkn::tp::tp_read_and_clear_timeout(&w);
     if (e != cudaSuccess) return fail(QKN_ERR_CUDA, "reading the timeout word: %s", cudaGetErrorString(e));
-    *code = v;
+    *code = v ? v : w;
+    return ok();
+}
+
+int64_t qknorm_tp_recv_bytes(int32_t R, int64_t T) {
+    if (R < 1 || R > qkn::tp::kMaxRanks || T < 0) return -1;
+    return (int64_t)R * T * 2 * 8;
+}
+
+qkn_status qknorm_tp_layerwise(int32_t R, int32_t first_rank, int32_t n_local, const void *const *q_in,
+                               void *const *q_out, const void *const *gamma_q, int64_t q_stride, int32_t hq_shard,
+                               int32_t Hq_full, const void *const *k_in, void *const *k_out,
+                               const void *const *gamma_k, int64_t k_stride, int32_t hk_shard, int32_t Hk_full,
+                               int64_t T, float eps, qkn_dtype dtype, void *const *recv, uint32_t epoch,
+                               int32_t blocks_per_rank, uint64_t timeout_ns, void *stream) {
+    using qkn::tp::kMaxLocal;
+    using qkn::tp::kMaxRanks;
+    if (!dtype_valid(dtype)) return fail(QKN_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
+    if (R < 1 || R > kMaxRanks) return fail(QKN_ERR_INVALID_ARG, "R = %d outside [1, %d]", R, kMaxRanks);
+    if (n_local < 1 || n_local > kMaxLocal || first_rank < 0 || first_rank + n_local > R)
+        return fail(QKN_ERR_INVALID_ARG, "local ranks [%d, %d) outside [0, %d)", first_rank, first_rank + n_local, R);
+    if (T < 0 || T >= ((int64_t)1 << 31)) return fail(QKN_ERR_INVALID_ARG, "T must be in [0, 2^31)");
+    if (hq_shard <= 0 || hk_shard <= 0) return fail(QKN_ERR_INVALID_ARG, "shard widths must be positive");
+    if (Hq_full < hq_shard || Hk_full < hk_shard) return fail(QKN_ERR_INVALID_ARG, "full width below shard width");
+    if (q_stride < hq_shard || k_stride < hk_shard) return fail(QKN_ERR_INVALID_ARG, "row stride below shard width");
+    if (!eps_valid(eps)) return fail(QKN_ERR_INVALID_ARG, "eps must be finite and >= 0");
+    if (epoch == 0) return fail(QKN_ERR_INVALID_ARG, "epoch 0 is reserved (receive buffers start zeroed)");
+    if (blocks_per_rank < 0) return fail(QKN_ERR_INVALID_ARG, "blocks_per_rank < 0");
+    const int esz = elem_bytes(dtype);
+    if (!extent_ok(T, q_stride, hq_shard, esz) || !extent_ok(T, k_stride, hk_shard, esz))
+        return fail(QKN_ERR_INVALID_ARG, "buffer extent overflows");
+    if (T == 0) return ok();
+    if (!q_in || !q_out || !gamma_q || !k_in || !k_out || !gamma_k || !recv)
+        return fail(QKN_ERR_INVALID_ARG, "null pointer array");
+    for (int r = 0; r < R; ++r)
+        if (!recv[r] || (reinterpret_cast<uintptr_t>(recv[r]) & 7u))
+            return fail(QKN_ERR_INVALID_ARG, "receive buffer %d null or not 8-byte aligned", r);
+    const int per_vec = 16 / esz;
+    if (hq_shard % per_vec || hk_shard % per_vec || (q_stride * esz) % 16 || (k_stride * esz) % 16)
+        return fail(QKN_ERR_UNSUPPORTED, "shard widths and strides must be whole 16-byte vectors");
+    const int gsz = gamma_bytes(dtype);
+    for (int j = 0; j < n_local; ++j) {
+        const void *ptrs[6] = {q_in[j], q_out[j], gamma_q[j], k_in[j], k_out[j], gamma_k[j]};
+        for (const void *pp : ptrs)
+            if (!pp) return fail(QKN_ERR_INVALID_ARG, "null pointer for local rank %d", j);
+            else if (!aligned16(pp)) return fail(QKN_ERR_UNSUPPORTED, "local rank %d: buffers must be 16-byte aligned", j);
+        const Region iq = rows_region(q_in[j], hq_shard, q_stride, T, esz), oq = rows_region(q_out[j], hq_shard, q_stride, T, esz);
+        const Region ik = rows_region(k_in[j], hk_shard, k_stride, T, esz), ok_ = rows_region(k_out[j], hk_shard, k_stride, T, esz);
+        const Region others[3] = {flat_region(gamma_q[j], (int64_t)hq_shard * gsz),
+                                  flat_region(gamma_k[j], (int64_t)hk_shard * gsz),
+                                  flat_region(recv[first_rank + j], qknorm_tp_recv_bytes(R, T))};
+        qkn_status st = check_outputs(oq, ok_, iq, ik, others, 3);
+        if (st != QKN_OK) return st;
+    }
+    for (int j = 0; j < n_local; ++j)  // no rank's output may touch another local rank's buffers
+        for (int jj = 0; jj < n_local; ++jj) {
+            if (jj == j) continue;
+            const Region outs[2] = {rows_region(q_out[j], hq_shard, q_stride, T, esz),
+                                    rows_region(k_out[j], hk_shard, k_stride, T, esz)};
+            const Region theirs[4] = {rows_region(q_in[jj], hq_shard, q_stride, T, esz),
+                                      rows_region(k_in[jj], hk_shard, k_stride, T, esz),
+                                      rows_region(q_out[jj], hq_shard, q_stride, T, esz),
+                                      rows_region(k_out[jj], hk_shard, k_stride, T, esz)};
+            for (const Region &o : outs)
+                for (const Region &t : theirs)
+                    if (overlap(o, t)) return fail(QKN_ERR_INVALID_ARG, "rank %d's output overlaps rank %d's rows", j, jj);
+        }
+    // launch shape: one block per token at a time, NV vectors per thread
+    const int64_t vq = hq_shard / per_vec, vk = hk_shard / per_vec, vmax = vq > vk ? vq : vk;
+    int nv = vmax <= 32 ? 1 : (vmax <= 512 ? 2 : 4);
+    int threads = (int)(((vmax + nv - 1) / nv + 31) / 32 * 32);
+    if (threads > 256) return fail(QKN_ERR_UNSUPPORTED, "shard rows above 1024 vectors");
+    int dev = 0, sms = 0, bps = 0;
+    qkn_status st = current_device(&dev);
+    if (st != QKN_OK) return st;
+    if ((st = sm_count(dev, &sms)) != QKN_OK) return st;
+    cudaError_t e = qkn::tp::tp_blocks_per_sm((int)dtype, nv, threads, &bps);
+    if (e != cudaSuccess || bps < 1) return fail(QKN_ERR_CUDA, "occupancy query: %s", cudaGetErrorString(e));
+    const int64_t resident = (int64_t)bps * sms;
+    int64_t G = blocks_per_rank > 0 ? blocks_per_rank : resident / n_local;
+    if (G > T) G = T;
+    if (G < 1 || G * n_local > resident)
+        return fail(QKN_ERR_UNSUPPORTED, "%lld blocks per rank x %d ranks exceed the %lld resident blocks",
+                    (long long)G, n_local, (long long)resident);
+    qkn::tp::TpParams tp{};
+    for (int j = 0; j < n_local; ++j)
+        tp.local[j] = qkn::tp::RankPtrs{static_cast<const char *>(q_in[j]), static_cast<char *>(q_out[j]),
+                                        static_cast<const char *>(gamma_q[j]), static_cast<const char *>(k_in[j]),
+                                        static_cast<char *>(k_out[j]), static_cast<const char *>(gamma_k[j])};
+    for (int r = 0; r < R; ++r) tp.recv[r] = static_cast<unsigned long long *>(recv[r]);
+    tp.q_stride_bytes = q_stride * esz;
+    tp.k_stride_bytes = k_stride * esz;
+    tp.T = T;
+    tp.R = R;
+    tp.first_rank = first_rank;
+    tp.n_local = n_local;
+    tp.blocks_per_rank = (int32_t)G;
+    tp.q_vecs = (int32_t)vq;
+    tp.k_vecs = (int32_t)vk;
+    tp.inv_hq = static_cast<float>(1.0 / static_cast<double>(Hq_full));
+    tp.inv_hk = static_cast<float>(1.0 / static_cast<double>(Hk_full));
+    tp.eps = eps;
+    tp.epoch = epoch;
+    tp.timeout_ns = timeout_ns ? timeout_ns : kGemmTimeoutNs;
+    const char *what = "";
+    e = qkn::tp::launch_tp(tp, (int)dtype, nv, threads, static_cast<cudaStream_t>(stream), &what);
+    if (e == cudaSuccess) e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(QKN_ERR_CUDA, "tensor-parallel kernel (%s): %s", what, cudaGetErrorString(e));
     return ok();
 }
 

@@ -1,0 +1,264 @@
+// Tensor-parallel layerwise QK-Norm with the scalar partial sums exchanged
+// through memory (structure and protocol in qknorm_tp.cuh).
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+#include <cuda_runtime.h>
+
+#include "qknorm_kernels.cuh"
+#include "qknorm_tp.cuh"
+
+namespace qkn {
+namespace tp {
+namespace {
+
+// Set by a wait that ran out (code 4); read and cleared by the host.
+__device__ int g_tp_timeout = 0;
+// The epoch of a call in which a wait ran out: every other wait of that call
+// gives up at once instead of running out in turn.
+__device__ unsigned int g_tp_aborted_epoch = 0;
+
+__device__ __forceinline__ void st_release_sys(unsigned long long *p, unsigned long long v) {
+    asm volatile("st.release.sys.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+__device__ __forceinline__ unsigned long long ld_acquire_sys(const unsigned long long *p) {
+    unsigned long long v;
+    asm volatile("ld.acquire.sys.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ uint64_t now_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ unsigned long long pack(uint32_t epoch, float v) {
+    return (static_cast<unsigned long long>(epoch) << 32) | __float_as_uint(v);
+}
+
+__device__ __forceinline__ bool aborted(uint32_t epoch) {
+    return *reinterpret_cast<volatile unsigned int *>(&g_tp_aborted_epoch) == epoch;
+}
+
+// Waits (bounded) until the word at `src` carries `epoch`; its value, or
+// false after a timeout or an abort of this call.
+__device__ __forceinline__ bool wait_word(const unsigned long long *src, uint32_t epoch, uint64_t timeout_ns,
+                                          float &v) {
+    unsigned long long w = ld_acquire_sys(src);
+    if (static_cast<uint32_t>(w >> 32) != epoch) {
+        const uint64_t t0 = now_ns();
+        for (;;) {
+            __nanosleep(64);
+            w = ld_acquire_sys(src);
+            if (static_cast<uint32_t>(w >> 32) == epoch) break;
+            if (aborted(epoch)) return false;
+            if (now_ns() - t0 > timeout_ns) {
+                atomicExch(&g_tp_timeout, 4);
+                atomicExch(&g_tp_aborted_epoch, epoch);
+                return false;
+            }
+        }
+    }
+    v = __uint_as_float(static_cast<uint32_t>(w));
+    return true;
+}
+
+// x * gamma for one vector, kept in fp32 pairs until the factor is known.
+template <typename E>
+__device__ __forceinline__ void mul_gamma(const uint4 &xv, const uint4 (&gv)[Elem<E>::kGVecs],
+                                          F2 (&u)[Elem<E>::kPerVec / 2]) {
+    using GT = typename Elem<E>::G;
+    constexpr int KG = Elem<GT>::kPerVec / 2;
+    Elem<E>::widen(xv, u);
+#pragma unroll
+    for (int j = 0; j < Elem<E>::kGVecs; ++j) {
+        F2 part[KG];
+        Elem<GT>::widen(gv[j], part);
+#pragma unroll
+        for (int k = 0; k < KG; ++k) u[j * KG + k] = mul2(u[j * KG + k], part[k]);
+    }
+}
+
+template <typename E>
+__device__ __forceinline__ uint4 times_r(const F2 (&u)[Elem<E>::kPerVec / 2], F2 r2) {
+    constexpr int K = Elem<E>::kPerVec / 2;
+    F2 y[K];
+#pragma unroll
+    for (int j = 0; j < K; ++j) y[j] = mul2(u[j], r2);
+    return Elem<E>::narrow(y);
+}
+
+}  // namespace
+
+// One block handles one token at a time: the rank's Q shard row and K shard
+// row, thread i holding 16-byte vectors i, i + blockDim, ... of each.
+constexpr int kTpMaxThreads = 256;
+
+template <typename E, int NV>
+__global__ void __launch_bounds__(kTpMaxThreads) tp_rows_kernel(const __grid_constant__ TpParams p) {
+    constexpr int KG = Elem<E>::kGVecs;
+    constexpr int K2 = Elem<E>::kPerVec / 2;
+    __shared__ float red[2][2][32];  // [slot][tensor][warp]
+    __shared__ float s_r[2];         // the token's factors (Q, K)
+    __shared__ int s_ok;
+    pdl_wait_and_release();
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
+    const int local = blockIdx.x / p.blocks_per_rank;
+    const int c = blockIdx.x - local * p.blocks_per_rank;
+    const int rank = p.first_rank + local;
+    const RankPtrs rp = p.local[local];
+
+    uint4 gq[NV][KG], gk[NV][KG];  // this rank's gamma slices, for the whole launch
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+        ld_gamma_vec<E>(rp.gamma_q, tid + i * blockDim.x, p.q_vecs, 0, gq[i]);
+        ld_gamma_vec<E>(rp.gamma_k, tid + i * blockDim.x, p.k_vecs, 0, gk[i]);
+    }
+    int slot = 0;
+    for (int64_t t = c; t < p.T; t += p.blocks_per_rank) {
+        const char *qrow = rp.q_in + t * p.q_stride_bytes;
+        const char *krow = rp.k_in + t * p.k_stride_bytes;
+        uint4 xq[NV], xk[NV];
+#pragma unroll
+        for (int i = 0; i < NV; ++i) {
+            const int vi = tid + i * blockDim.x;
+            xq[i] = vi < p.q_vecs ? ld_stream(qrow + static_cast<int64_t>(vi) * 16) : make_uint4(0u, 0u, 0u, 0u);
+            xk[i] = vi < p.k_vecs ? ld_stream(krow + static_cast<int64_t>(vi) * 16) : make_uint4(0u, 0u, 0u, 0u);
+        }
+        // Phase A, local step: the shard's squared sums (fixed order: warp
+        // butterfly, then warps 0, 1, ...).
+        float sq = warp_sum(sumsq_pairs<E, NV>(xq));
+        float sk = warp_sum(sumsq_pairs<E, NV>(xk));
+        if (lane == 0) {
+            red[slot][0][warp] = sq;
+            red[slot][1][warp] = sk;
+        }
+        __syncthreads();
+        float Sq = 0.0f, Sk = 0.0f;
+        for (int w = 0; w < nwarps; ++w) {
+            Sq += red[slot][0][w];
+            Sk += red[slot][1][w];
+        }
+        slot ^= 1;
+
+        if (warp == 0) {
+            // Exchange: lane i writes this rank's partials into rank i's
+            // buffer, then waits for rank i's partials in this rank's buffer.
+            float vq = 0.0f, vk = 0.0f;
+            bool ok = true;
+            if (lane < p.R) {
+                unsigned long long *dst = p.recv[lane] + (static_cast<int64_t>(rank) * p.T + t) * 2;
+                st_release_sys(dst, pack(p.epoch, Sq));
+                st_release_sys(dst + 1, pack(p.epoch, Sk));
+                const unsigned long long *src = p.recv[rank] + (static_cast<int64_t>(lane) * p.T + t) * 2;
+                ok = wait_word(src, p.epoch, p.timeout_ns, vq) && wait_word(src + 1, p.epoch, p.timeout_ns, vk);
+            }
+            ok = __all_sync(0xFFFFFFFFu, ok);
+            // Phase A aggregation: the R partials added in rank order, fp32.
+            float Aq = 0.0f, Ak = 0.0f;
+            for (int i = 0; i < p.R; ++i) {
+                Aq += __shfl_sync(0xFFFFFFFFu, vq, i);
+                Ak += __shfl_sync(0xFFFFFFFFu, vk, i);
+            }
+            if (lane == 0) {
+                s_r[0] = rms_factor(Aq, p.inv_hq, p.eps);
+                s_r[1] = rms_factor(Ak, p.inv_hk, p.eps);
+                s_ok = ok;
+            }
+        }
+        // Phase B: x * gamma does not depend on the reduction (the other
+        // warps form it while warp 0 waits).
+        F2 uq[NV][K2], uk[NV][K2];
+#pragma unroll
+        for (int i = 0; i < NV; ++i) {
+            mul_gamma<E>(xq[i], gq[i], uq[i]);
+            mul_gamma<E>(xk[i], gk[i], uk[i]);
+        }
+        __syncthreads();
+        if (!s_ok) continue;  // a wait gave up: this token is left unwritten (the timeout is reported)
+        const F2 rq = f2(s_r[0], s_r[0]), rk = f2(s_r[1], s_r[1]);
+        char *qo = rp.q_out + t * p.q_stride_bytes;
+        char *ko = rp.k_out + t * p.k_stride_bytes;
+#pragma unroll
+        for (int i = 0; i < NV; ++i) {
+            const int vi = tid + i * blockDim.x;
+            if (vi < p.q_vecs) st_stream(qo + static_cast<int64_t>(vi) * 16, times_r<E>(uq[i], rq));
+            if (vi < p.k_vecs) st_stream(ko + static_cast<int64_t>(vi) * 16, times_r<E>(uk[i], rk));
+        }
+    }
+}
+
+namespace {
+
+template <typename E>
+const void *tp_kernel(int nv) {
+    switch (nv) {
+        case 1: return (const void *)tp_rows_kernel<E, 1>;
+        case 2: return (const void *)tp_rows_kernel<E, 2>;
+        case 4: return (const void *)tp_rows_kernel<E, 4>;
+        default: return nullptr;
+    }
+}
+
+const void *tp_kernel(int dtype, int nv) {
+    switch (dtype) {
+        case 0: return tp_kernel<float>(nv);
+        case 1: return tp_kernel<__nv_bfloat16>(nv);
+        case 2: return tp_kernel<__half>(nv);
+        case 3: return tp_kernel<__nv_fp8_e4m3>(nv);
+        default: return nullptr;
+    }
+}
+
+}  // namespace
+
+cudaError_t tp_blocks_per_sm(int dtype, int nv, int threads, int *out) {
+    const void *fn = tp_kernel(dtype, nv);
+    if (!fn) return cudaErrorInvalidValue;
+    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(out, fn, threads, 0);
+}
+
+cudaError_t launch_tp(const TpParams &p, int dtype, int nv, int threads, cudaStream_t stream, const char **what) {
+    const void *fn = tp_kernel(dtype, nv);
+    if (!fn) {
+        *what = "kernel selection";
+        return cudaErrorInvalidValue;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(p.blocks_per_rank * p.n_local));
+    cfg.blockDim = dim3(static_cast<unsigned>(threads));
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    int n = 0;
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+    if (p.n_local > 1) {  // blocks of different ranks wait on one another: all must be resident
+        attr[n].id = cudaLaunchAttributeCooperative;
+        attr[n].val.cooperative = 1;
+        ++n;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = n;
+    void *args[] = {const_cast<TpParams *>(&p)};
+    cudaError_t e = cudaLaunchKernelExC(&cfg, fn, args);
+    if (e != cudaSuccess) *what = "cudaLaunchKernelExC";
+    return e;
+}
+
+cudaError_t tp_read_and_clear_timeout(int *code) {
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return e;
+    int v = 0;
+    if ((e = cudaMemcpyFromSymbol(&v, g_tp_timeout, sizeof(int))) != cudaSuccess) return e;
+    const int zero = 0;
+    if ((e = cudaMemcpyToSymbol(g_tp_timeout, &zero, sizeof(int))) != cudaSuccess) return e;
+    *code = v;
+    return cudaSuccess;
+}
+
+}  // namespace tp
+}  // namespace qkn

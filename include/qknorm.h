@@ -231,9 +231,48 @@ qkn_status qknorm_qkv_projection_noalloc(const void *x, int64_t x_stride, const 
 int64_t qknorm_qkv_projection_noalloc_max_bytes(void);
 
 /*
+ * Tensor-parallel layerwise QK-Norm: the paper's multi-GPU kernel (Phase A:
+ * each rank squares and sums its hidden-dimension shard and the ranks add
+ * their scalar partial sums in fp32; Phase B: warp 0 of each block carries
+ * that exchange while the other warps multiply the shard by gamma, then the
+ * global factor scales it; deadlock-safe persistent blocks).
+ *   R ranks each hold a shard of every token's Q row (hq_shard columns of
+ *   Hq_full) and K row (hk_shard of Hk_full).  This call runs the n_local
+ *   ranks first_rank .. first_rank + n_local - 1; local rank j's rows are
+ *   q_in[j] / q_out[j] ([T rows, stride q_stride]), gamma slice gamma_q[j]
+ *   [hq_shard], and likewise for K.  out == in normalizes in place.
+ *   recv[r] (r < R) is rank r's receive buffer, qknorm_tp_recv_bytes(R, T)
+ *   bytes: a device pointer valid on this GPU -- its own memory for local
+ *   ranks, a peer mapping (cudaIpcOpenMemHandle or similar) for ranks on other
+ *   GPUs.  Buffers start zeroed; each call on the same buffers passes a new
+ *   epoch (> 0), and all ranks of one call pass the same epoch.
+ *   Result: y = (x * gamma) * r with r = 1 / sqrt(S / H_full + eps) and S the
+ *   ranks' partial sums added in rank order 0 .. R-1, identical on every rank.
+ * Deployments: one GPU per rank (n_local = 1, each GPU calls with its own
+ * rank; pass the same blocks_per_rank on every rank, or 0 on identical GPUs),
+ * or several ranks in one call on one GPU (their blocks wait on one another,
+ * so the launch is cooperative and must fit on the GPU at once).
+ * Waits are bounded by timeout_ns (0 = 2 s); one that runs out reports code 4
+ * through qknorm_device_timeouts, every other wait of the call gives up, and
+ * the tokens concerned are left unwritten.
+ * Requirements: 1 <= R <= 8, n_local <= 8; dtype any of qkn_dtype; 16-byte
+ * aligned buffers and shard widths / strides that are whole 16-byte vectors
+ * (else QKN_ERR_UNSUPPORTED); shard rows of at most 1024 vectors.  T = 0 is a
+ * no-op.  Asynchronous on `stream`; allocates nothing.
+ */
+int64_t qknorm_tp_recv_bytes(int32_t R, int64_t T);
+qkn_status qknorm_tp_layerwise(int32_t R, int32_t first_rank, int32_t n_local, const void *const *q_in,
+                               void *const *q_out, const void *const *gamma_q, int64_t q_stride, int32_t hq_shard,
+                               int32_t Hq_full, const void *const *k_in, void *const *k_out,
+                               const void *const *gamma_k, int64_t k_stride, int32_t hk_shard, int32_t Hk_full,
+                               int64_t T, float eps, qkn_dtype dtype, void *const *recv, uint32_t epoch,
+                               int32_t blocks_per_rank, uint64_t timeout_ns, void *stream);
+
+/*
  * Every wait inside the projection kernel is bounded (2 s); one that runs out
- * records a non-zero code (1 = TMA producer, 2 = MMA issuer, 3 = epilogue)
- * and the kernel returns early with its output incomplete.  This call
+ * records a non-zero code (1 = TMA producer, 2 = MMA issuer, 3 = epilogue;
+ * 4 = a tensor-parallel exchange wait) and the kernel returns early with its
+ * output incomplete.  This call
  * synchronizes the current device, stores that code in *code (0 = none) and
  * clears it.  No paper counterpart: a safety check of this library.
  */

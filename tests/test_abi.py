@@ -395,3 +395,41 @@ def test_projection_pipeline_validation(lib):
     assert call(ws=0x8000000 + 64) == INVALID        # workspace inside qkv
     assert call(gk=0x8000000) == INVALID             # gamma inside qkv
     assert lib.qknorm_device_timeouts(None) == INVALID
+
+
+def _tp_call(lib, **kw):
+    P = ctypes.c_void_p
+    a = dict(R=4, first=0, n=4, T=128, hq=256, Hq=1024, hk=128, Hk=512, qs=256, ks=128, eps=1e-6, dtype=BF16,
+             epoch=1, G=0, recv=[0x40000000 + r * 0x100000 for r in range(4)])
+    a.update(kw)
+    n = a["n"]
+    base = lambda off: (P * max(n, 1))(*[0x10000000 + off + j * 0x1000000 for j in range(max(n, 1))])
+    recv = (P * len(a["recv"]))(*a["recv"])
+    return lib.qknorm_tp_layerwise(a["R"], a["first"], n, base(0), base(0x400000), base(0x800000), a["qs"], a["hq"],
+                                   a["Hq"], base(0x900000), base(0xB00000), base(0xD00000), a["ks"], a["hk"], a["Hk"],
+                                   a["T"], a["eps"], a["dtype"], recv, a["epoch"], a["G"], 0, None)
+
+
+@pytest.mark.parametrize("kw,want", [
+    ({}, CUDA),                                    # well formed: validation passes, the device query fails here
+    ({"T": 0}, OK),
+    ({"R": 0}, INVALID),
+    ({"R": 9}, INVALID),
+    ({"first": 2, "n": 3}, INVALID),               # ranks beyond R
+    ({"epoch": 0}, INVALID),                       # reserved
+    ({"G": -1}, INVALID),
+    ({"dtype": 7}, INVALID),
+    ({"eps": -1.0}, INVALID),
+    ({"Hq": 100}, INVALID),                        # full width below the shard width
+    ({"qs": 200}, INVALID),                        # stride below the shard width
+    ({"hq": 252, "qs": 256}, UNSUPPORTED),         # shard width not whole 16-byte vectors
+    ({"recv": [0x40000000, 0, 0x40200000, 0x40300000]}, INVALID),
+    ({"recv": [0x40000004, 0x40100000, 0x40200000, 0x40300000]}, INVALID),  # not 8-byte aligned
+])
+def test_tp_validation(lib, kw, want):
+    assert _tp_call(lib, **kw) == want
+
+
+def test_tp_recv_bytes(lib):
+    assert lib.qknorm_tp_recv_bytes(4, 4096) == 4 * 4096 * 16
+    assert lib.qknorm_tp_recv_bytes(0, 10) == -1 and lib.qknorm_tp_recv_bytes(9, 10) == -1

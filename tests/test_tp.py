@@ -1,0 +1,114 @@
+"""The tensor-parallel form (the paper's multi-GPU kernel) on one GPU.
+
+``qknorm_tp_layerwise`` runs R ranks, each holding a hidden-dimension shard
+of every token's Q and K rows; the ranks exchange only their scalar partial
+sums through receive buffers (Phase A) while the shards are multiplied by
+gamma (Phase B).  Here all ranks run in one cooperative launch on one GPU,
+their receive buffers in that GPU's memory -- the same kernel and protocol a
+one-rank-per-GPU deployment uses with peer-mapped buffers.
+
+Every output shard is compared with the oracle's RMS-Norm of the full,
+unsharded row (the definition), within the tolerances of the other parity
+tests: 1 ulp of the element type, or 1e-5 relative for fp32.  A launch that
+leaves one rank out makes the exchange waits run out: the kernel must return,
+report the timeout and leave the context usable.
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import attention_normalization_b200 as qk
+import workloads
+from tests.test_parity import ALL_DTYPES, assert_close, oracle_rows
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+
+
+def _batch(T, Hq, Hk, dtype, seed):
+    return workloads.random_rows(T, Hq, Hk, dtype, seed=seed, scale=1.5)
+
+
+def _shards(full: torch.Tensor, R: int):
+    w = full.shape[1] // R
+    return [full[:, r * w:(r + 1) * w].contiguous().to(DEV) for r in range(R)]
+
+
+def _gamma_shards(g: torch.Tensor, R: int):
+    w = g.numel() // R
+    return [g[r * w:(r + 1) * w].contiguous().to(DEV) for r in range(R)]
+
+
+def run_tp(b, R, ex=None, **kw):
+    ex = ex or qk.TpExchange(R, b.T, DEV)
+    qo, ko = qk.qknorm_tp_layerwise(_shards(b.q, R), _shards(b.k, R), _gamma_shards(b.gamma_q, R),
+                                    _gamma_shards(b.gamma_k, R), b.Hq, b.Hk, b.eps, exchange=ex, **kw)
+    torch.cuda.synchronize()
+    return torch.cat([q.cpu() for q in qo], dim=1), torch.cat([k.cpu() for k in ko], dim=1)
+
+
+def check_full(b, q, k):
+    yq, eq, _ = oracle_rows(b.q, b.gamma_q, b.eps)
+    yk, ek, _ = oracle_rows(b.k, b.gamma_k, b.eps)
+    assert_close(q, yq, eq, f"{b.name} TP Q")
+    assert_close(k, yk, ek, f"{b.name} TP K")
+
+
+@pytest.mark.parametrize("dtype", ALL_DTYPES)
+@pytest.mark.parametrize("R", [1, 2, 4, 8])
+def test_tp_matches_the_full_row_oracle(R, dtype):
+    b = _batch(300, 2048, 512, dtype, seed=R)
+    q, k = run_tp(b, R)
+    check_full(b, q, k)
+    assert qk.device_timeouts() == 0
+
+
+def test_tp_prefill_full_size():
+    """The prefill batch (T=4096, Hq=Hk=4096 bf16) split over 4 ranks."""
+    b = workloads.prefill_bf16()
+    q, k = run_tp(b, 4)
+    check_full(b, q, k)
+    assert qk.device_timeouts() == 0
+
+
+def test_tp_any_block_count_gives_the_same_bits_and_buffers_are_reused():
+    """The result does not depend on how many blocks each rank runs; one
+    exchange serves consecutive calls (a new epoch each), in place too."""
+    b = _batch(257, 1024, 256, torch.bfloat16, seed=11)
+    ex = qk.TpExchange(4, b.T, DEV)
+    ref_q, ref_k = run_tp(b, 4, ex)
+    for G in (1, 7, 64):
+        q, k = run_tp(b, 4, ex, blocks_per_rank=G)
+        assert torch.equal(q, ref_q) and torch.equal(k, ref_k)
+    qs, ks = _shards(b.q, 4), _shards(b.k, 4)
+    qk.qknorm_tp_layerwise(qs, ks, _gamma_shards(b.gamma_q, 4), _gamma_shards(b.gamma_k, 4), b.Hq, b.Hk, b.eps,
+                           exchange=ex, in_place=True)
+    torch.cuda.synchronize()
+    assert torch.equal(torch.cat([q.cpu() for q in qs], 1), ref_q)
+    assert torch.equal(torch.cat([k.cpu() for k in ks], 1), ref_k)
+    check_full(b, ref_q, ref_k)
+    assert qk.device_timeouts() == 0
+
+
+def test_tp_missing_rank_times_out_and_the_context_stays_usable():
+    """Ranks 0..2 of a 4-rank group run; rank 3 never publishes, so every
+    exchange wait runs out (50 ms): the kernel returns, reports code 4, and
+    writes none of the tokens.  A complete call afterwards is correct."""
+    R = 4
+    b = _batch(64, 1024, 512, torch.bfloat16, seed=12)
+    ex = qk.TpExchange(R, b.T, DEV)
+    qs, ks = _shards(b.q, R), _shards(b.k, R)
+    gq, gk = _gamma_shards(b.gamma_q, R), _gamma_shards(b.gamma_k, R)
+    sentinel = [torch.full_like(q, 3.0) for q in qs[:3]]
+    qo, _ = qk.qknorm_tp_layerwise(qs[:3], ks[:3], gq[:3], gk[:3], b.Hq, b.Hk, b.eps, exchange=ex, R=R,
+                                   first_rank=0, q_out=sentinel, timeout_ns=50_000_000)
+    torch.cuda.synchronize()
+    assert qk.device_timeouts() == 4
+    assert all(torch.all(q == 3.0) for q in qo)
+    assert qk.device_timeouts() == 0  # reading cleared it
+    q, k = run_tp(b, R, ex)
+    check_full(b, q, k)
+    assert qk.device_timeouts() == 0
