@@ -19,13 +19,41 @@ __device__ int g_tp_timeout = 0;
 // gives up at once instead of running out in turn.
 __device__ unsigned int g_tp_aborted_epoch = 0;
 
-__device__ __forceinline__ void st_release_sys(unsigned long long *p, unsigned long long v) {
-    asm volatile("st.release.sys.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+// Memory scope of the exchange: system when some ranks are on other GPUs
+// (peer memory), GPU when every rank runs in this launch.
+template <bool SYS>
+__device__ __forceinline__ void st_relaxed(unsigned long long *p, unsigned long long v) {
+    if constexpr (SYS)
+        asm volatile("st.relaxed.sys.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+    else
+        asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
 
-__device__ __forceinline__ unsigned long long ld_acquire_sys(const unsigned long long *p) {
+template <bool SYS>
+__device__ __forceinline__ void st_release(unsigned long long *p, unsigned long long v) {
+    if constexpr (SYS)
+        asm volatile("st.release.sys.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+    else
+        asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+template <bool SYS>
+__device__ __forceinline__ unsigned long long ld_acquire(const unsigned long long *p) {
     unsigned long long v;
-    asm volatile("ld.acquire.sys.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    if constexpr (SYS)
+        asm volatile("ld.acquire.sys.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    else
+        asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+
+template <bool SYS>
+__device__ __forceinline__ unsigned long long ld_relaxed(const unsigned long long *p) {
+    unsigned long long v;
+    if constexpr (SYS)
+        asm volatile("ld.relaxed.sys.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    else
+        asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
     return v;
 }
 
@@ -45,14 +73,15 @@ __device__ __forceinline__ bool aborted(uint32_t epoch) {
 
 // Waits (bounded) until the word at `src` carries `epoch`; its value, or
 // false after a timeout or an abort of this call.
+template <bool SYS>
 __device__ __forceinline__ bool wait_word(const unsigned long long *src, uint32_t epoch, uint64_t timeout_ns,
                                           float &v) {
-    unsigned long long w = ld_acquire_sys(src);
+    unsigned long long w = ld_acquire<SYS>(src);
     if (static_cast<uint32_t>(w >> 32) != epoch) {
         const uint64_t t0 = now_ns();
         for (;;) {
-            __nanosleep(64);
-            w = ld_acquire_sys(src);
+            __nanosleep(32);
+            w = ld_acquire<SYS>(src);
             if (static_cast<uint32_t>(w >> 32) == epoch) break;
             if (aborted(epoch)) return false;
             if (now_ns() - t0 > timeout_ns) {
@@ -97,7 +126,7 @@ __device__ __forceinline__ uint4 times_r(const F2 (&u)[Elem<E>::kPerVec / 2], F2
 // row, thread i holding 16-byte vectors i, i + blockDim, ... of each.
 constexpr int kTpMaxThreads = 256;
 
-template <typename E, int NV>
+template <typename E, int NV, bool SYS>
 __global__ void __launch_bounds__(kTpMaxThreads) tp_rows_kernel(const __grid_constant__ TpParams p) {
     constexpr int KG = Elem<E>::kGVecs;
     constexpr int K2 = Elem<E>::kPerVec / 2;
@@ -150,11 +179,18 @@ __global__ void __launch_bounds__(kTpMaxThreads) tp_rows_kernel(const __grid_con
             float vq = 0.0f, vk = 0.0f;
             bool ok = true;
             if (lane < p.R) {
+                // the Q word, then the K word with release: a reader that
+                // sees the K word's epoch (acquire) sees the Q word too
                 unsigned long long *dst = p.recv[lane] + (static_cast<int64_t>(rank) * p.T + t) * 2;
-                st_release_sys(dst, pack(p.epoch, Sq));
-                st_release_sys(dst + 1, pack(p.epoch, Sk));
+                st_relaxed<SYS>(dst, pack(p.epoch, Sq));
+                st_release<SYS>(dst + 1, pack(p.epoch, Sk));
                 const unsigned long long *src = p.recv[rank] + (static_cast<int64_t>(lane) * p.T + t) * 2;
-                ok = wait_word(src, p.epoch, p.timeout_ns, vq) && wait_word(src + 1, p.epoch, p.timeout_ns, vk);
+                ok = wait_word<SYS>(src + 1, p.epoch, p.timeout_ns, vk);
+                if (ok) {
+                    const unsigned long long wq = ld_relaxed<SYS>(src);
+                    ok = static_cast<uint32_t>(wq >> 32) == p.epoch;
+                    vq = __uint_as_float(static_cast<uint32_t>(wq));
+                }
             }
             ok = __all_sync(0xFFFFFFFFu, ok);
             // Phase A aggregation: the R partials added in rank order, fp32.
@@ -193,36 +229,42 @@ __global__ void __launch_bounds__(kTpMaxThreads) tp_rows_kernel(const __grid_con
 
 namespace {
 
-template <typename E>
+template <typename E, bool SYS>
 const void *tp_kernel(int nv) {
     switch (nv) {
-        case 1: return (const void *)tp_rows_kernel<E, 1>;
-        case 2: return (const void *)tp_rows_kernel<E, 2>;
-        case 4: return (const void *)tp_rows_kernel<E, 4>;
+        case 1: return (const void *)tp_rows_kernel<E, 1, SYS>;
+        case 2: return (const void *)tp_rows_kernel<E, 2, SYS>;
+        case 4: return (const void *)tp_rows_kernel<E, 4, SYS>;
         default: return nullptr;
     }
 }
 
+template <bool SYS>
 const void *tp_kernel(int dtype, int nv) {
     switch (dtype) {
-        case 0: return tp_kernel<float>(nv);
-        case 1: return tp_kernel<__nv_bfloat16>(nv);
-        case 2: return tp_kernel<__half>(nv);
-        case 3: return tp_kernel<__nv_fp8_e4m3>(nv);
+        case 0: return tp_kernel<float, SYS>(nv);
+        case 1: return tp_kernel<__nv_bfloat16, SYS>(nv);
+        case 2: return tp_kernel<__half, SYS>(nv);
+        case 3: return tp_kernel<__nv_fp8_e4m3, SYS>(nv);
         default: return nullptr;
     }
+}
+
+// System scope when some rank of the group runs elsewhere (peer memory).
+const void *tp_kernel(int dtype, int nv, bool all_local) {
+    return all_local ? tp_kernel<false>(dtype, nv) : tp_kernel<true>(dtype, nv);
 }
 
 }  // namespace
 
 cudaError_t tp_blocks_per_sm(int dtype, int nv, int threads, int *out) {
-    const void *fn = tp_kernel(dtype, nv);
+    const void *fn = tp_kernel(dtype, nv, false);
     if (!fn) return cudaErrorInvalidValue;
     return cudaOccupancyMaxActiveBlocksPerMultiprocessor(out, fn, threads, 0);
 }
 
 cudaError_t launch_tp(const TpParams &p, int dtype, int nv, int threads, cudaStream_t stream, const char **what) {
-    const void *fn = tp_kernel(dtype, nv);
+    const void *fn = tp_kernel(dtype, nv, p.n_local == p.R);
     if (!fn) {
         *what = "kernel selection";
         return cudaErrorInvalidValue;

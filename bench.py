@@ -57,8 +57,9 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
-    ap.add_argument("--workload", choices=["prefill", "decode", "packed", "gqa", "tiny", "headwise", "projection"],
+    ap.add_argument("--workload", choices=["prefill", "decode", "packed", "gqa", "tiny", "headwise", "projection", "tp"],
                     default="prefill")
+    ap.add_argument("--ranks", type=int, default=4, help="tensor-parallel ranks of the tp workload")
     ap.add_argument("--tokens", type=int, default=None, help="T for decode / packed workloads")
     ap.add_argument("--dtype", choices=["bf16", "f16", "e4m3"], default="bf16",
                     help="element type of the prefill workload (gamma is bf16 with e4m3)")
@@ -233,7 +234,7 @@ class Workload:
 
     DTYPES = {"bf16": torch.bfloat16, "f16": torch.float16, "e4m3": torch.float8_e4m3fn}
 
-    def __init__(self, kind: str, tokens: int | None, seed_offset: int, dtype: str = "bf16"):
+    def __init__(self, kind: str, tokens: int | None, seed_offset: int, dtype: str = "bf16", ranks: int = 4):
         self.kind = kind
         if kind == "prefill":
             self.batch = workloads.prefill_bf16(seed=1 + seed_offset, dtype=self.DTYPES[dtype])
@@ -247,6 +248,9 @@ class Workload:
             self.batch = workloads.gqa_sharded(seed=3 + seed_offset)
         elif kind == "headwise":
             self.batch = workloads.headwise_bf16(seed=5 + seed_offset, T=tokens or 4096)
+        elif kind == "tp":
+            self.batch = workloads.prefill_bf16(seed=1 + seed_offset)
+        self.ranks = ranks
         b = self.batch
         self.esz = {torch.float32: 4, torch.float8_e4m3fn: 1}.get(b.dtype, 2)
         gesz = 4 if b.dtype == torch.float32 else 2
@@ -267,6 +271,10 @@ class Workload:
         if self.kind == "headwise":
             c.update({"head_dim": b.meta["head_dim"], "q_heads": b.meta["q_heads"], "k_heads": b.meta["k_heads"],
                       "form": "qknorm_headwise (one factor per head)"})
+        if self.kind == "tp":
+            c.update({"R": self.ranks, "form": f"qknorm_tp_layerwise: {self.ranks} tensor-parallel ranks, each with "
+                                               "1/R of every Q and K row, exchanging scalar partial sums; all ranks "
+                                               "in one cooperative launch on one GPU"})
         return c
 
     # one device-resident set of buffers
@@ -287,6 +295,16 @@ class Workload:
                     "gks": [gk[p * wk:(p + 1) * wk].contiguous() for p in range(P)],
                     "q_all": torch.empty((P, b.T), dtype=torch.float32, device=dev),
                     "k_all": torch.empty((P, b.T), dtype=torch.float32, device=dev)}
+        if self.kind == "tp":
+            import attention_normalization_b200 as qk
+            R = self.ranks
+            wq, wk = b.Hq // R, b.Hk // R
+            qs = [b.q[:, r * wq:(r + 1) * wq].contiguous().to(dev) for r in range(R)]
+            ks = [b.k[:, r * wk:(r + 1) * wk].contiguous().to(dev) for r in range(R)]
+            return {"qs": qs, "ks": ks, "qo": [torch.empty_like(t) for t in qs], "ko": [torch.empty_like(t) for t in ks],
+                    "gqs": [b.gamma_q[r * wq:(r + 1) * wq].contiguous().to(dev) for r in range(R)],
+                    "gks": [b.gamma_k[r * wk:(r + 1) * wk].contiguous().to(dev) for r in range(R)],
+                    "ex": qk.TpExchange(R, b.T, dev)}
         q, k = b.q.to(dev), b.k.to(dev)
         return {"q": q, "k": k, "qo": torch.empty_like(q), "ko": torch.empty_like(k),
                 "gq": b.gamma_q.to(dev), "gk": b.gamma_k.to(dev)}
@@ -310,6 +328,10 @@ class Workload:
         elif self.kind == "headwise":
             qk.qknorm_headwise(s["q"], s["k"], s["gq"], s["gk"], b.meta["head_dim"], b.eps,
                                q_out=s["qo"], k_out=s["ko"])
+        elif self.kind == "tp":
+            # each call takes the exchange's next epoch: a captured graph is replayed once
+            qk.qknorm_tp_layerwise(s["qs"], s["ks"], s["gqs"], s["gks"], b.Hq, b.Hk, b.eps, exchange=s["ex"],
+                                   q_out=s["qo"], k_out=s["ko"])
         else:
             qk.qknorm_layerwise(s["q"], s["k"], s["gq"], s["gk"], b.eps, q_out=s["qo"], k_out=s["ko"])
 
@@ -428,7 +450,7 @@ def native(args) -> int:
     ranks = Ranks(dist, dev)
     barrier, max_over_ranks = ranks.barrier, ranks.max
 
-    wl = Workload(args.workload, args.tokens, seed_offset=rank * 1000, dtype=args.dtype)
+    wl = Workload(args.workload, args.tokens, seed_offset=rank * 1000, dtype=args.dtype, ranks=args.ranks)
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     R = rotating = rotation_count(wl.set_bytes(), l2)
     sets = [wl.make_set(dev) for _ in range(R)]
@@ -479,10 +501,13 @@ def native(args) -> int:
                 "unit": "GB/s", "frac": round(wl.eff_bytes / kernel_s / 1e9 / peaks["hbm_gbs"], 4),
                 "traffic": profiled_traffic(wl.name, digest),
                 "peak_source": f"{peaks['source']} copy bandwidth",
-                "kernel": "qknorm rows kernel (the only kernel of the step)" if wl.kind != "gqa"
-                          else "whole step: partial_stats x P + combine_apply x P",
+                "kernel": {"gqa": "whole step: partial_stats x P + combine_apply x P",
+                           "tp": "tp_rows_kernel, all ranks in one launch (the only kernel of the step)"}.get(
+                               wl.kind, "qknorm rows kernel (the only kernel of the step)"),
                 "algorithmic_bytes_per_launch": wl.eff_bytes if wl.kind != "gqa" else None,
                 "source_digest": digest}
+
+    timeouts = qk.device_timeouts()  # any bounded wait that ran out (tensor-parallel exchange)
 
     # end to end through the public API with pinned host buffers
     e2e = e2e_measure(qk, wl, dev, args, barrier, max_over_ranks)
@@ -517,7 +542,7 @@ def native(args) -> int:
                 "data": "synthetic (seeded; OLMo2-shaped activations, no dataset or weights)",
                 "config": cfg, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": args.steps * wl.launches_per_step, "clocks": clocks,
-                "impl": "native"}
+                "device_timeouts": timeouts, "impl": "native"}
         print(json.dumps(line))
     del g_warm, g_timed
     if dist is not None:
@@ -562,6 +587,20 @@ def e2e_measure(qk, wl: Workload, dev, args, barrier, max_over_ranks) -> dict:
         h2d = sum(t.numel() * t.element_size() for t in h_in) + gbytes
         d2h = sum(t.numel() * t.element_size() for t in h_out)
         path = "per-shard pinned host -> device copies, partial_stats x P + combine_apply x P, device -> host copies"
+    elif wl.kind == "tp":
+        s = wl.make_set(dev)
+        h_in = [t.cpu().pin_memory() for t in s["qs"] + s["ks"]]
+        h_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in s["qo"] + s["ko"]]
+
+        def one():
+            for h, d in zip(h_in, s["qs"] + s["ks"]):
+                d.copy_(h, non_blocking=True)
+            wl.step(qk, s)
+            for h, d in zip(h_out, s["qo"] + s["ko"]):
+                h.copy_(d, non_blocking=True)
+        h2d = sum(t.numel() * t.element_size() for t in h_in)
+        d2h = sum(t.numel() * t.element_size() for t in h_out)
+        path = "per-rank shards pinned host -> device, qknorm_tp_layerwise (all ranks, one launch), device -> host"
     elif wl.kind == "headwise":
         s = wl.make_set(dev)
         h_q, h_k = b.q.contiguous().pin_memory(), b.k.contiguous().pin_memory()
