@@ -1087,9 +1087,17 @@ qkn_status qknorm_tp_layerwise(int32_t R, int32_t first_rank, int32_t n_local, c
         }
     // launch shape: one block per token at a time, NV vectors per thread
     const int64_t vq = hq_shard / per_vec, vk = hk_shard / per_vec, vmax = vq > vk ? vq : vk;
-    int nv = vmax <= 32 ? 1 : (vmax <= 512 ? 2 : 4);
-    int threads = (int)(((vmax + nv - 1) / nv + 31) / 32 * 32);
-    if (threads > 256) return fail(QKN_ERR_UNSUPPORTED, "shard rows above 1024 vectors");
+    int nv, threads;
+    int64_t tokens_per_block = 1;
+    if (vmax <= 128) {  // one token per warp, four warps per block
+        nv = vmax <= 32 ? -1 : (vmax <= 64 ? -2 : -4);
+        threads = 128;
+        tokens_per_block = 4;
+    } else {
+        nv = vmax <= 512 ? 2 : 4;
+        threads = (int)(((vmax + nv - 1) / nv + 31) / 32 * 32);
+        if (threads > 256) return fail(QKN_ERR_UNSUPPORTED, "shard rows above 1024 vectors");
+    }
     int dev = 0, sms = 0, bps = 0;
     qkn_status st = current_device(&dev);
     if (st != QKN_OK) return st;
@@ -1098,7 +1106,8 @@ qkn_status qknorm_tp_layerwise(int32_t R, int32_t first_rank, int32_t n_local, c
     if (e != cudaSuccess || bps < 1) return fail(QKN_ERR_CUDA, "occupancy query: %s", cudaGetErrorString(e));
     const int64_t resident = (int64_t)bps * sms;
     int64_t G = blocks_per_rank > 0 ? blocks_per_rank : resident / n_local;
-    if (G > T) G = T;
+    const int64_t needed = (T + tokens_per_block - 1) / tokens_per_block;
+    if (G > needed) G = needed;
     if (G < 1 || G * n_local > resident)
         return fail(QKN_ERR_UNSUPPORTED, "%lld blocks per rank x %d ranks exceed the %lld resident blocks",
                     (long long)G, n_local, (long long)resident);

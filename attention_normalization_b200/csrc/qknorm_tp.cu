@@ -227,14 +227,91 @@ __global__ void __launch_bounds__(kTpMaxThreads) tp_rows_kernel(const __grid_con
     }
 }
 
+// Narrow shard rows (at most 32 * NV vectors): one warp per token, kTpWarps
+// warps per block, no block barrier.  Warp w of block b of a rank takes
+// tokens (b * kTpWarps + w), + G * kTpWarps, ...; lane i exchanges with rank
+// i as in the block form, every lane gets the sums by shuffles, and the warp
+// then scales its row as (x * gamma) * r (the same products as the block
+// form, formed after the wait to keep registers for more warps in flight).
+constexpr int kTpWarps = 4;
+
+template <typename E, int NV, bool SYS>
+__global__ void __launch_bounds__(32 * kTpWarps) tp_warp_kernel(const __grid_constant__ TpParams p) {
+    constexpr int KG = Elem<E>::kGVecs;
+    pdl_wait_and_release();
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int local = blockIdx.x / p.blocks_per_rank;
+    const int c = blockIdx.x - local * p.blocks_per_rank;
+    const int rank = p.first_rank + local;
+    const RankPtrs rp = p.local[local];
+    const int64_t step = static_cast<int64_t>(p.blocks_per_rank) * kTpWarps;
+
+    uint4 gq[NV][KG], gk[NV][KG];
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+        ld_gamma_vec<E>(rp.gamma_q, lane + 32 * i, p.q_vecs, 0, gq[i]);
+        ld_gamma_vec<E>(rp.gamma_k, lane + 32 * i, p.k_vecs, 0, gk[i]);
+    }
+    for (int64_t t = static_cast<int64_t>(c) * kTpWarps + warp; t < p.T; t += step) {
+        const char *qrow = rp.q_in + t * p.q_stride_bytes;
+        const char *krow = rp.k_in + t * p.k_stride_bytes;
+        uint4 xq[NV], xk[NV];
+#pragma unroll
+        for (int i = 0; i < NV; ++i) {
+            const int vi = lane + 32 * i;
+            xq[i] = vi < p.q_vecs ? ld_stream(qrow + static_cast<int64_t>(vi) * 16) : make_uint4(0u, 0u, 0u, 0u);
+            xk[i] = vi < p.k_vecs ? ld_stream(krow + static_cast<int64_t>(vi) * 16) : make_uint4(0u, 0u, 0u, 0u);
+        }
+        const float Sq = warp_sum(sumsq_pairs<E, NV>(xq));  // Phase A, local step
+        const float Sk = warp_sum(sumsq_pairs<E, NV>(xk));
+        if (lane < p.R) {
+            unsigned long long *dst = p.recv[lane] + (static_cast<int64_t>(rank) * p.T + t) * 2;
+            st_relaxed<SYS>(dst, pack(p.epoch, Sq));
+            st_release<SYS>(dst + 1, pack(p.epoch, Sk));
+        }
+        float vq = 0.0f, vk = 0.0f;
+        bool ok = true;
+        if (lane < p.R) {
+            const unsigned long long *src = p.recv[rank] + (static_cast<int64_t>(lane) * p.T + t) * 2;
+            ok = wait_word<SYS>(src + 1, p.epoch, p.timeout_ns, vk);
+            if (ok) {
+                const unsigned long long wq = ld_relaxed<SYS>(src);
+                ok = static_cast<uint32_t>(wq >> 32) == p.epoch;
+                vq = __uint_as_float(static_cast<uint32_t>(wq));
+            }
+        }
+        if (!__all_sync(0xFFFFFFFFu, ok)) continue;  // a wait gave up: token left unwritten (reported)
+        float Aq = 0.0f, Ak = 0.0f;  // Phase A aggregation, in rank order
+        for (int i = 0; i < p.R; ++i) {
+            Aq += __shfl_sync(0xFFFFFFFFu, vq, i);
+            Ak += __shfl_sync(0xFFFFFFFFu, vk, i);
+        }
+        const float rq1 = rms_factor(Aq, p.inv_hq, p.eps), rk1 = rms_factor(Ak, p.inv_hk, p.eps);
+        const F2 rq = f2(rq1, rq1), rk = f2(rk1, rk1);
+        char *qo = rp.q_out + t * p.q_stride_bytes;
+        char *ko = rp.k_out + t * p.k_stride_bytes;
+#pragma unroll
+        for (int i = 0; i < NV; ++i) {
+            const int vi = lane + 32 * i;
+            if (vi < p.q_vecs) st_stream(qo + static_cast<int64_t>(vi) * 16, scale_vec<E>(xq[i], gq[i], rq));
+            if (vi < p.k_vecs) st_stream(ko + static_cast<int64_t>(vi) * 16, scale_vec<E>(xk[i], gk[i], rk));
+        }
+    }
+}
+
 namespace {
 
+// nv > 0: the block-per-token kernel with nv vectors per thread; nv < 0: the
+// warp-per-token kernel with -nv vectors per lane.
 template <typename E, bool SYS>
 const void *tp_kernel(int nv) {
     switch (nv) {
         case 1: return (const void *)tp_rows_kernel<E, 1, SYS>;
         case 2: return (const void *)tp_rows_kernel<E, 2, SYS>;
         case 4: return (const void *)tp_rows_kernel<E, 4, SYS>;
+        case -1: return (const void *)tp_warp_kernel<E, 1, SYS>;
+        case -2: return (const void *)tp_warp_kernel<E, 2, SYS>;
+        case -4: return (const void *)tp_warp_kernel<E, 4, SYS>;
         default: return nullptr;
     }
 }

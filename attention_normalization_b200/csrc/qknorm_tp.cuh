@@ -15,6 +15,9 @@
 //   Deadlock-safe persistent execution: the grid is bounded by the resident
 //     blocks and each block loops over tokens.
 //
+// Shard rows of at most 128 vectors run one token per warp (four per block,
+// no block barrier), wider ones one token per block.
+//
 // One kernel serves two deployments:
 //   * one rank per GPU: each GPU launches its own rank; receive buffers of the
 //     other ranks are reached through peer mappings (P2P stores and loads,
@@ -71,8 +74,10 @@ struct TpParams {
 };
 
 // Host side (qknorm_tp.cu): launch `p` on `stream` with `threads` threads per
-// block and NV vectors per thread for element type `dtype` (1 = bf16, 2 =
-// fp16, 0 = fp32, 3 = E4M3); cooperative when n_local > 1.
+// block for element type `dtype` (1 = bf16, 2 = fp16, 0 = fp32, 3 = E4M3);
+// nv > 0 selects the block-per-token kernel with nv vectors per thread, nv < 0
+// the warp-per-token kernel (128-thread blocks of 4 warps) with -nv vectors
+// per lane.  Cooperative when n_local > 1.
 cudaError_t launch_tp(const TpParams &p, int dtype, int nv, int threads, cudaStream_t stream, const char **what);
 
 // Blocks of the kernel for (dtype, nv, threads) resident per SM.
