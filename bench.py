@@ -125,17 +125,17 @@ def load_peaks() -> dict:
 
 
 KERNEL_SOURCES = {
-    "rows": ["qknorm_kernels.cuh", "qknorm_api.cu"],
-    "projection": ["qkv_gemm.cu", "qkv_gemm.cuh", "qknorm_api.cu"],
+    "rows": ["qknorm_kernels.cuh"],
+    "projection": ["qkv_gemm.cu", "qkv_gemm.cuh"],
 }
 
 
 def source_digest(kind: str = "rows") -> str:
-    """Digest of the sources of one kernel family and the public headers:
-    profile counters apply only to the build they were taken from."""
+    """Digest of one kernel family's device sources: profile counters apply
+    only to the kernel they were taken from (the launch shape is checked
+    separately, see profiled_traffic)."""
     h = hashlib.sha256()
-    files = sorted([os.path.join(ROOT, "attention_normalization_b200", "csrc", f) for f in KERNEL_SOURCES[kind]]
-                   + glob.glob(os.path.join(ROOT, "include", "*.h")))
+    files = sorted(os.path.join(ROOT, "attention_normalization_b200", "csrc", f) for f in KERNEL_SOURCES[kind])
     for p in files:
         h.update(os.path.basename(p).encode())
         with open(p, "rb") as f:
@@ -143,17 +143,29 @@ def source_digest(kind: str = "rows") -> str:
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(workload: str, digest: str):
+def profiled_traffic(workload: str, digest: str, launch: str | None = None):
     """DRAM bytes per launch from a committed ncu summary for this workload, if
-    it was taken from the current sources; else None."""
+    it was taken from the current kernel sources (and, when the summary names
+    one, the same launch shape); else None."""
     for p in sorted(glob.glob(os.path.join(ROOT, "profiles", "*.md"))):
         text = open(p).read()
         m_w = re.search(r"^workload:\s*(\S+)", text, re.M)
         m_d = re.search(r"^source_digest:\s*(\S+)", text, re.M)
         m_t = re.search(r"^dram_bytes_per_launch:\s*(\d+)", text, re.M)
-        if m_w and m_d and m_t and m_w.group(1) == workload and m_d.group(1) == digest:
-            return int(m_t.group(1))
+        m_l = re.search(r"^launch:\s*(.+)$", text, re.M)
+        if not (m_w and m_d and m_t) or m_w.group(1) != workload or m_d.group(1) != digest:
+            continue
+        if m_l and launch is not None and m_l.group(1).strip() != launch:
+            continue
+        return int(m_t.group(1))
     return None
+
+
+def launch_text(plan) -> str | None:
+    """A launch plan as the profile summaries record it."""
+    if not plan:
+        return None
+    return "kernel={kernel} vec_per_thread={vec_per_thread} threads={threads} grid={grid}".format(**plan)
 
 
 class ClockSampler:
@@ -497,9 +509,17 @@ def native(args) -> int:
     peaks = load_peaks()
     digest = source_digest()
     kernel_s = step_s / wl.launches_per_step if wl.kind != "gqa" else step_s
+    plan = None
+    if wl.kind in ("prefill", "tiny", "decode", "packed"):
+        s0 = sets[0]
+        if wl.kind == "packed":
+            plan = qk.qknorm_layerwise_plan(s0["q"], s0["k"], s0["gq"], s0["gk"], q_out=s0["q"], k_out=s0["k"])
+        else:
+            plan = qk.qknorm_layerwise_plan(s0["q"], s0["k"], s0["gq"], s0["gk"], q_out=s0["qo"], k_out=s0["ko"])
+
     roofline = {"bound": "hbm", "achieved": round(wl.eff_bytes / kernel_s / 1e9, 1), "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "frac": round(wl.eff_bytes / kernel_s / 1e9 / peaks["hbm_gbs"], 4),
-                "traffic": profiled_traffic(wl.name, digest),
+                "traffic": profiled_traffic(wl.name, digest, launch_text(plan)),
                 "peak_source": f"{peaks['source']} copy bandwidth",
                 "kernel": {"gqa": "whole step: partial_stats x P + combine_apply x P",
                            "tp": "tp_rows_kernel, all ranks in one launch (the only kernel of the step)"}.get(
@@ -515,14 +535,6 @@ def native(args) -> int:
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = time_oracle(wl, args.cpu_seconds)
-
-    plan = None
-    if wl.kind in ("prefill", "tiny", "decode", "packed"):
-        s0 = sets[0]
-        if wl.kind == "packed":
-            plan = qk.qknorm_layerwise_plan(s0["q"], s0["k"], s0["gq"], s0["gk"], q_out=s0["q"], k_out=s0["k"])
-        else:
-            plan = qk.qknorm_layerwise_plan(s0["q"], s0["k"], s0["gq"], s0["gk"], q_out=s0["qo"], k_out=s0["ko"])
 
     if rank == 0:
         cfg = wl.config()
