@@ -1090,7 +1090,10 @@ qkn_status qknorm_tp_layerwise(int32_t R, int32_t first_rank, int32_t n_local, c
     int nv, threads;
     int64_t tokens_per_block = 1;
     if (vmax <= 128) {  // one token per warp, four warps per block
-        nv = vmax <= 32 ? -1 : (vmax <= 64 ? -2 : -4);
+        auto lanes_nv = [](int64_t v) { return v <= 32 ? 1 : (v <= 64 ? 2 : 4); };
+        int nvq = lanes_nv(vq), nvk = lanes_nv(vk);
+        if (nvk > nvq) nvq = nvk;  // instantiated with NVK <= NVQ
+        nv = -(8 * nvq + nvk);
         threads = 128;
         tokens_per_block = 4;
     } else {

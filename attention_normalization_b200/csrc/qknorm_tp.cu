@@ -227,7 +227,7 @@ __global__ void __launch_bounds__(kTpMaxThreads) tp_rows_kernel(const __grid_con
     }
 }
 
-// Narrow shard rows (at most 32 * NV vectors): one warp per token, kTpWarps
+// Narrow shard rows (at most 32 * NVQ vectors of Q, 32 * NVK of K): one warp per token, kTpWarps
 // warps per block, no block barrier.  Warp w of block b of a rank takes
 // tokens (b * kTpWarps + w), + G * kTpWarps, ...; lane i exchanges with rank
 // i as in the block form, every lane gets the sums by shuffles, and the warp
@@ -235,7 +235,7 @@ __global__ void __launch_bounds__(kTpMaxThreads) tp_rows_kernel(const __grid_con
 // form, formed after the wait to keep registers for more warps in flight).
 constexpr int kTpWarps = 4;
 
-template <typename E, int NV, bool SYS>
+template <typename E, int NVQ, int NVK, bool SYS>
 __global__ void __launch_bounds__(32 * kTpWarps) tp_warp_kernel(const __grid_constant__ TpParams p) {
     constexpr int KG = Elem<E>::kGVecs;
     pdl_wait_and_release();
@@ -246,24 +246,27 @@ __global__ void __launch_bounds__(32 * kTpWarps) tp_warp_kernel(const __grid_con
     const RankPtrs rp = p.local[local];
     const int64_t step = static_cast<int64_t>(p.blocks_per_rank) * kTpWarps;
 
-    uint4 gq[NV][KG], gk[NV][KG];
+    uint4 gq[NVQ][KG], gk[NVK][KG];
 #pragma unroll
-    for (int i = 0; i < NV; ++i) {
-        ld_gamma_vec<E>(rp.gamma_q, lane + 32 * i, p.q_vecs, 0, gq[i]);
-        ld_gamma_vec<E>(rp.gamma_k, lane + 32 * i, p.k_vecs, 0, gk[i]);
-    }
+    for (int i = 0; i < NVQ; ++i) ld_gamma_vec<E>(rp.gamma_q, lane + 32 * i, p.q_vecs, 0, gq[i]);
+#pragma unroll
+    for (int i = 0; i < NVK; ++i) ld_gamma_vec<E>(rp.gamma_k, lane + 32 * i, p.k_vecs, 0, gk[i]);
     for (int64_t t = static_cast<int64_t>(c) * kTpWarps + warp; t < p.T; t += step) {
         const char *qrow = rp.q_in + t * p.q_stride_bytes;
         const char *krow = rp.k_in + t * p.k_stride_bytes;
-        uint4 xq[NV], xk[NV];
+        uint4 xq[NVQ], xk[NVK];
 #pragma unroll
-        for (int i = 0; i < NV; ++i) {
+        for (int i = 0; i < NVQ; ++i) {
             const int vi = lane + 32 * i;
             xq[i] = vi < p.q_vecs ? ld_stream(qrow + static_cast<int64_t>(vi) * 16) : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int i = 0; i < NVK; ++i) {
+            const int vi = lane + 32 * i;
             xk[i] = vi < p.k_vecs ? ld_stream(krow + static_cast<int64_t>(vi) * 16) : make_uint4(0u, 0u, 0u, 0u);
         }
-        const float Sq = warp_sum(sumsq_pairs<E, NV>(xq));  // Phase A, local step
-        const float Sk = warp_sum(sumsq_pairs<E, NV>(xk));
+        const float Sq = warp_sum(sumsq_pairs<E, NVQ>(xq));  // Phase A, local step
+        const float Sk = warp_sum(sumsq_pairs<E, NVK>(xk));
         if (lane < p.R) {
             unsigned long long *dst = p.recv[lane] + (static_cast<int64_t>(rank) * p.T + t) * 2;
             st_relaxed<SYS>(dst, pack(p.epoch, Sq));
@@ -291,9 +294,13 @@ __global__ void __launch_bounds__(32 * kTpWarps) tp_warp_kernel(const __grid_con
         char *qo = rp.q_out + t * p.q_stride_bytes;
         char *ko = rp.k_out + t * p.k_stride_bytes;
 #pragma unroll
-        for (int i = 0; i < NV; ++i) {
+        for (int i = 0; i < NVQ; ++i) {
             const int vi = lane + 32 * i;
             if (vi < p.q_vecs) st_stream(qo + static_cast<int64_t>(vi) * 16, scale_vec<E>(xq[i], gq[i], rq));
+        }
+#pragma unroll
+        for (int i = 0; i < NVK; ++i) {
+            const int vi = lane + 32 * i;
             if (vi < p.k_vecs) st_stream(ko + static_cast<int64_t>(vi) * 16, scale_vec<E>(xk[i], gk[i], rk));
         }
     }
@@ -302,16 +309,20 @@ __global__ void __launch_bounds__(32 * kTpWarps) tp_warp_kernel(const __grid_con
 namespace {
 
 // nv > 0: the block-per-token kernel with nv vectors per thread; nv < 0: the
-// warp-per-token kernel with -nv vectors per lane.
+// warp-per-token kernel with NVQ and NVK vectors per lane, nv = -(8 NVQ + NVK).
 template <typename E, bool SYS>
 const void *tp_kernel(int nv) {
     switch (nv) {
         case 1: return (const void *)tp_rows_kernel<E, 1, SYS>;
         case 2: return (const void *)tp_rows_kernel<E, 2, SYS>;
         case 4: return (const void *)tp_rows_kernel<E, 4, SYS>;
-        case -1: return (const void *)tp_warp_kernel<E, 1, SYS>;
-        case -2: return (const void *)tp_warp_kernel<E, 2, SYS>;
-        case -4: return (const void *)tp_warp_kernel<E, 4, SYS>;
+        // warp form: nv = -(8 * NVQ + NVK), NVK <= NVQ (wider K rows take NVQ = NVK)
+        case -(8 * 1 + 1): return (const void *)tp_warp_kernel<E, 1, 1, SYS>;
+        case -(8 * 2 + 1): return (const void *)tp_warp_kernel<E, 2, 1, SYS>;
+        case -(8 * 2 + 2): return (const void *)tp_warp_kernel<E, 2, 2, SYS>;
+        case -(8 * 4 + 1): return (const void *)tp_warp_kernel<E, 4, 1, SYS>;
+        case -(8 * 4 + 2): return (const void *)tp_warp_kernel<E, 4, 2, SYS>;
+        case -(8 * 4 + 4): return (const void *)tp_warp_kernel<E, 4, 4, SYS>;
         default: return nullptr;
     }
 }

@@ -76,8 +76,9 @@ struct TpParams {
 // Host side (qknorm_tp.cu): launch `p` on `stream` with `threads` threads per
 // block for element type `dtype` (1 = bf16, 2 = fp16, 0 = fp32, 3 = E4M3);
 // nv > 0 selects the block-per-token kernel with nv vectors per thread, nv < 0
-// the warp-per-token kernel (128-thread blocks of 4 warps) with -nv vectors
-// per lane.  Cooperative when n_local > 1.
+// the warp-per-token kernel (128-thread blocks of 4 warps) with NVQ vectors
+// per lane for Q and NVK for K, nv = -(8 NVQ + NVK).  Cooperative when
+// n_local > 1.
 cudaError_t launch_tp(const TpParams &p, int dtype, int nv, int threads, cudaStream_t stream, const char **what);
 
 // Blocks of the kernel for (dtype, nv, threads) resident per SM.
