@@ -356,18 +356,67 @@ __device__ __forceinline__ void pdl_wait_and_release() {
 
 // Squared sum of a thread's vectors (two fp32 lanes accumulate the even and
 // odd elements; they are added at the end).
+// Squares of the two halves of an f16x2 word added to the even and odd
+// accumulators with sm_100's mixed-precision fma (f16 inputs, fp32 addend and
+// result).  An f16 x f16 product is exact in fp32, so each step equals the
+// fp32 fma of the widened values -- the same sums as widening first, without
+// the two conversions.
+__device__ __forceinline__ void fma_sq_half2(uint32_t w, float &even, float &odd) {
+    asm("{\n\t.reg .f16 lo, hi;\n\t"
+        "mov.b32 {lo, hi}, %2;\n\t"
+        "fma.rn.f32.f16 %0, lo, lo, %0;\n\t"
+        "fma.rn.f32.f16 %1, hi, hi, %1;\n\t}"
+        : "+f"(even), "+f"(odd)
+        : "r"(w));
+}
+
+template <typename E>
+struct HalfSquares {  // element types whose squares take fma_sq_half2
+    static constexpr bool value = false;
+};
+template <>
+struct HalfSquares<__half> {
+    static constexpr bool value = true;
+};
+template <>
+struct HalfSquares<__nv_fp8_e4m3> {
+    static constexpr bool value = true;
+};
+
 template <typename E, int NV>
 __device__ __forceinline__ float sumsq_pairs(const uint4 (&v)[NV]) {
     constexpr int K = Elem<E>::kPerVec / 2;
-    F2 acc = f2(0.0f, 0.0f);
+    if constexpr (HalfSquares<E>::value) {
+        float even = 0.0f, odd = 0.0f;  // the two lanes of the f32x2 form below
 #pragma unroll
-    for (int i = 0; i < NV; ++i) {
-        F2 x[K];
-        Elem<E>::widen(v[i], x);
+        for (int i = 0; i < NV; ++i) {
+            const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
 #pragma unroll
-        for (int j = 0; j < K; ++j) acc = fma2(x[j], x[j], acc);
+            for (int j = 0; j < 4; ++j) {
+                if constexpr (sizeof(typename Elem<E>::Bits) == 2) {
+                    fma_sq_half2(w[j], even, odd);
+                } else {  // two E4M3 pairs per word, each widened exactly to f16x2
+                    const __half2_raw lo =
+                        __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w[j] & 0xFFFFu), __NV_E4M3);
+                    const __half2_raw hi =
+                        __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w[j] >> 16), __NV_E4M3);
+                    fma_sq_half2(*reinterpret_cast<const uint32_t *>(&lo), even, odd);
+                    fma_sq_half2(*reinterpret_cast<const uint32_t *>(&hi), even, odd);
+                }
+            }
+        }
+        return even + odd;
+    } else {
+        F2 acc = f2(0.0f, 0.0f);
+#pragma unroll
+        for (int i = 0; i < NV; ++i) {
+            F2 x[K];
+            Elem<E>::widen(v[i], x);
+#pragma unroll
+            for (int j = 0; j < K; ++j) acc = fma2(x[j], x[j], acc);
+        }
+        return f2_lo(acc) + f2_hi(acc);
     }
-    return f2_lo(acc) + f2_hi(acc);
 }
 
 // Phase B on the way out, one vector: y = (x * gamma) * r, rounded once.
