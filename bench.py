@@ -375,6 +375,59 @@ def rotation_count(set_bytes: int, l2_bytes: int) -> int:
 
 # --------------------------------------------------------------------------- CPU baseline (the oracle)
 
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def time_oracle_parallel(wl: Workload, budget_s: float) -> dict:
+    """The same oracle calls split over the host's cores: one thread per core,
+    each normalizing a contiguous block of tokens (the C oracle runs outside
+    the Python lock).  Whole calls until the budget is spent."""
+    import concurrent.futures
+
+    import numpy as np
+
+    import oracle
+    b = wl.batch
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else (os.cpu_count() or 1)
+
+    def bits(view):
+        t = view.contiguous()
+        if t.dtype == torch.bfloat16:
+            return t.view(torch.int16).numpy().view(np.uint16)
+        if t.dtype == torch.float8_e4m3fn:
+            return t.view(torch.uint8).numpy()
+        return t.numpy()
+    q, k = bits(b.q), bits(b.k)
+    gq, gk = bits(b.gamma_q[None, :]).ravel(), bits(b.gamma_k[None, :]).ravel()
+    edges = np.linspace(0, b.T, min(cores, b.T) + 1).astype(int)
+    blocks = [(lo, hi) for lo, hi in zip(edges[:-1], edges[1:]) if hi > lo]
+
+    def part(lo_hi):
+        lo, hi = lo_hi
+        oracle.qknorm_layerwise(np.ascontiguousarray(q[lo:hi]), b.Hq, gq, b.Hq, np.ascontiguousarray(k[lo:hi]), b.Hk,
+                                gk, b.Hk, hi - lo, b.eps)
+    with concurrent.futures.ThreadPoolExecutor(max_workers=len(blocks)) as ex:
+        calls, t0 = 0, time.perf_counter()
+        while True:
+            list(ex.map(part, blocks))
+            calls += 1
+            el = time.perf_counter() - t0
+            if el >= budget_s or calls >= 1000:
+                break
+    per_call = el / calls
+    return {"value": wl.eff_bytes / per_call / 1e9, "unit": UNIT, "cores": len(blocks), "cpu": cpu_model(),
+            "sample": f"{calls} whole oracle call(s) of {wl.name} over {len(blocks)} threads, {el:.1f} s",
+            "us_per_call": per_call * 1e6}
+
+
 def time_oracle(wl: Workload, budget_s: float, max_tokens: int | None = None) -> dict:
     """Times the CPU oracle (double precision, one thread) on the workload's
     own inputs: whole calls until the budget is spent, or, with max_tokens, a
@@ -501,6 +554,37 @@ def native(args) -> int:
     ms_rank = ev0.elapsed_time(ev1)
     ms = max_over_ranks(ms_rank)
     clocks = sampler.summary()
+    del g_warm, g_timed
+
+    # Spread (informational): 20 replays of a short graph, each timed on its
+    # own, give per-call p10 / p50 / p90; and the same calls launched eagerly,
+    # back to back, for the latency-bound shapes.
+    spread = None
+    if rank == 0 and wl.kind != "tp":  # tp captures take fresh epochs: not replayed twice
+        m = max(1, min(100, args.steps))
+        g_short = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_short, capture_error_mode="thread_local"):
+            for i in range(m):
+                wl.step(qk, sets[i % R])
+        g_short.replay()
+        torch.cuda.synchronize()
+        per_call = []
+        for _ in range(20):
+            ev0.record(stream)
+            g_short.replay()
+            ev1.record(stream)
+            torch.cuda.synchronize()
+            per_call.append(ev0.elapsed_time(ev1) * 1e3 / m / wl.launches_per_step)
+        del g_short
+        per_call.sort()
+        spread = {"us_per_call_p10": round(per_call[2], 3), "us_per_call_p50": round(statistics.median(per_call), 3),
+                  "us_per_call_p90": round(per_call[17], 3), "replays": 20, "calls_per_replay": m}
+        ev0.record(stream)
+        for i in range(m):
+            wl.step(qk, sets[i % R])
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        spread["eager_us_per_call"] = round(ev0.elapsed_time(ev1) * 1e3 / m / wl.launches_per_step, 3)
 
     agg = whole_job(wl.eff_bytes, args.steps, ms, world)
     step_s = agg["ms_per_step"] / 1e3
@@ -535,6 +619,8 @@ def native(args) -> int:
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = time_oracle(wl, args.cpu_seconds)
+        if wl.kind in ("prefill", "packed", "tiny", "decode", "tp"):
+            cpu["all_cores"] = time_oracle_parallel(wl, args.cpu_seconds)
 
     if rank == 0:
         cfg = wl.config()
@@ -554,9 +640,8 @@ def native(args) -> int:
                 "data": "synthetic (seeded; OLMo2-shaped activations, no dataset or weights)",
                 "config": cfg, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": args.steps * wl.launches_per_step, "clocks": clocks,
-                "device_timeouts": timeouts, "impl": "native"}
+                "spread": spread, "device_timeouts": timeouts, "impl": "native"}
         print(json.dumps(line))
-    del g_warm, g_timed
     if dist is not None:
         dist.destroy_process_group()
     return 0
