@@ -1105,7 +1105,7 @@ qkn_status qknorm_tp_layerwise(int32_t R, int32_t first_rank, int32_t n_local, c
     qkn_status st = current_device(&dev);
     if (st != QKN_OK) return st;
     if ((st = sm_count(dev, &sms)) != QKN_OK) return st;
-    cudaError_t e = qkn::tp::tp_blocks_per_sm((int)dtype, nv, threads, &bps);
+    cudaError_t e = qkn::tp::tp_blocks_per_sm((int)dtype, nv, threads, n_local == R, &bps);
     if (e != cudaSuccess || bps < 1) return fail(QKN_ERR_CUDA, "occupancy query: %s", cudaGetErrorString(e));
     const int64_t resident = (int64_t)bps * sms;
     int64_t G = blocks_per_rank > 0 ? blocks_per_rank : resident / n_local;

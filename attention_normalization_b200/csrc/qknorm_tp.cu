@@ -345,8 +345,8 @@ const void *tp_kernel(int dtype, int nv, bool all_local) {
 
 }  // namespace
 
-cudaError_t tp_blocks_per_sm(int dtype, int nv, int threads, int *out) {
-    const void *fn = tp_kernel(dtype, nv, false);
+cudaError_t tp_blocks_per_sm(int dtype, int nv, int threads, bool all_local, int *out) {
+    const void *fn = tp_kernel(dtype, nv, all_local);
     if (!fn) return cudaErrorInvalidValue;
     return cudaOccupancyMaxActiveBlocksPerMultiprocessor(out, fn, threads, 0);
 }

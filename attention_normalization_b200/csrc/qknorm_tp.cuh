@@ -81,8 +81,9 @@ struct TpParams {
 // n_local > 1.
 cudaError_t launch_tp(const TpParams &p, int dtype, int nv, int threads, cudaStream_t stream, const char **what);
 
-// Blocks of the kernel for (dtype, nv, threads) resident per SM.
-cudaError_t tp_blocks_per_sm(int dtype, int nv, int threads, int *out);
+// Blocks of the kernel for (dtype, nv, threads) resident per SM; all_local
+// selects the GPU-scope form (every rank in the launch), else system scope.
+cudaError_t tp_blocks_per_sm(int dtype, int nv, int threads, bool all_local, int *out);
 
 // The code a timed-out wait recorded (0 = none); synchronizes the device and
 // clears it.
