@@ -495,3 +495,28 @@ def test_headwise_full_size_bench_workload():
     b = workloads.headwise_bf16()
     hd = b.meta["head_dim"]
     check_headwise(b.q, b.k, b.gamma_q, b.gamma_k, hd, eps=b.eps)
+
+
+@pytest.mark.parametrize("dtype,bound,floor", [(torch.bfloat16, 2.0 ** -8, 2.0 ** -134),
+                                               (torch.float8_e4m3fn, 2.0 ** -3, 2.0 ** -10)])
+def test_prefill_error_band_against_fp64_gold(dtype, bound, floor):
+    """Fig. 2(b) context: max / mean / RMS absolute error of the GPU output
+    against the unrounded double oracle on the prefill batch (the paper reports
+    5.0e-2 / 2.1e-3 / 3.4e-3 for BF16 and 5.0e-1 / 2.5e-2 / 3.9e-2 for FP8-E4M3
+    on inputs it does not describe).  The error here is the output rounding
+    alone, so it stays within half an ulp plus the fp32 work:
+    |err| <= bound * |y| + floor, bound = 2^-8 (bf16) / 2^-3 (E4M3), floor =
+    half the subnormal spacing (2^-134 / 2^-10)."""
+    b = workloads.prefill_bf16(dtype=dtype)
+    q, k, _ = upload(b)
+    qo, ko = qk.qknorm_layerwise(q, k, b.gamma_q.to(DEV), b.gamma_k.to(DEV), b.eps)
+    torch.cuda.synchronize()
+    errs = []
+    for got, view, g in ((qo, b.q, b.gamma_q), (ko, b.k, b.gamma_k)):
+        _, exact, _ = oracle_rows(view, g, b.eps)
+        y = got.float().cpu().double().numpy()
+        err = np.abs(y - exact)
+        assert np.all(err <= bound * np.abs(exact) + floor), "error beyond half an ulp of the type"
+        errs.append(err.ravel())
+    e = np.concatenate(errs)
+    print(f"\nerror band {dtype}: max {e.max():.3e}  mean {e.mean():.3e}  rms {np.sqrt((e * e).mean()):.3e}")
