@@ -60,6 +60,8 @@ def parse_args(argv=None):
     ap.add_argument("--workload", choices=["prefill", "decode", "packed", "gqa", "tiny", "headwise", "projection", "tp"],
                     default="prefill")
     ap.add_argument("--ranks", type=int, default=4, help="tensor-parallel ranks of the tp workload")
+    ap.add_argument("--proj", default="4096,4096,4096,4096",
+                    help="D,Hq,Hk,Hv of the projection workload (T from --tokens, default 4096)")
     ap.add_argument("--tokens", type=int, default=None, help="T for decode / packed workloads")
     ap.add_argument("--dtype", choices=["bf16", "f16", "e4m3"], default="bf16",
                     help="element type of the prefill workload (gamma is bf16 with e4m3)")
@@ -846,7 +848,8 @@ def native_projection(args) -> int:
     qk.capi()
     ranks = Ranks(dist, dev)
 
-    b = workloads.qkv_projection(T=args.tokens or 4096, seed=6 + rank * 1000)
+    D, Hq, Hk, Hv = (int(v) for v in args.proj.split(","))
+    b = workloads.qkv_projection(T=args.tokens or 4096, D=D, Hq=Hq, Hk=Hk, Hv=Hv, seed=6 + rank * 1000)
     N = b.Hq + b.Hk + b.Hv
     flops = _proj_flops(b)
     ws_bytes = qk.qkv_workspace_bytes(b.T, b.Hq, b.Hk)
@@ -996,7 +999,8 @@ def projection_reference(args) -> int:
     rank, world, _ = dist_env()
     if rank != 0:
         return 0
-    b = workloads.qkv_projection(T=args.tokens or 4096, seed=6)
+    D, Hq, Hk, Hv = (int(v) for v in args.proj.split(","))
+    b = workloads.qkv_projection(T=args.tokens or 4096, D=D, Hq=Hq, Hk=Hk, Hv=Hv, seed=6)
     for _ in range(args.warmup):
         time_oracle_projection(b, 0.0)
     t0 = time.perf_counter()
