@@ -14,23 +14,26 @@
 // of those stored values.  The combine / factor / scale steps then run as the
 // usual apply pass (Phase A aggregation + Phase B).
 //
-// Kernel shape: persistent, one CTA of 320 threads per SM, each taking the
-// 128 x 256 output tiles blockIdx.x, blockIdx.x + gridDim.x, ...  The token
-// tile runs fastest (tile = column tile * token tiles + token tile), so the
-// CTAs running at one time share a few W tiles while X stays in L2.
-// (Groups of kGroupM token tiles, column tile next, were measured 6% slower
-// at the OLMo2-7B shape and are off by default.)  Roles:
-//   warp 0, lane 0 : TMA producer.  X tile [128 x 64] and W tile [256 x 64]
-//                    per k-block into a 4-stage shared-memory ring, 128-byte
-//                    swizzle, completion counted on an mbarrier per stage; the
-//                    ring runs on across tiles.
+// Kernel shape: persistent, clusters of kCta CTAs (320 threads each, one per
+// SM), as many as are resident at once.  A work unit is one MMA tile of
+// 128 * kCta tokens x 256 columns; cluster c takes units c, c + clusters, ...
+// in a grouped raster (token block fastest within a group of group_units
+// token blocks, then the column tile, then the group; the host sizes the
+// group by what fits in L2).  With kCta = 2 the pair's leader issues
+// tcgen05.mma cta_group::2 (M = 256) and each CTA receives its 128 rows of
+// the 128 x 256 result in its own TMEM.  Roles, per CTA:
+//   warp 0, lane 0 : TMA producer.  X tile [128 x 64] and this CTA's half of
+//                    the W tile [256 / kCta x 64] per k-block into a kStages
+//                    shared-memory ring, 128-byte swizzle, completion counted
+//                    on the leader's mbarrier per stage; the ring runs on
+//                    across tiles.
 //   warp 1         : allocates 512 TMEM columns, two fp32 accumulators of
-//                    128 lanes x 256 columns (lane = tile row); lane 0 issues
-//                    tcgen05.mma (M=128, N=256, K=16, bf16 in, fp32
+//                    128 lanes x 256 columns (lane = tile row); in the leader
+//                    lane 0 issues the MMAs (K = 16, bf16 in, fp32
 //                    accumulate), four per k-block, into the accumulator of
-//                    the tile's parity, frees each stage with tcgen05.commit
-//                    when its MMAs have read it, and signals the epilogue when
-//                    a tile's accumulator is complete.
+//                    the tile's parity, frees each stage in both CTAs with
+//                    tcgen05.commit when its MMAs have read it, and signals
+//                    both epilogues when a tile's accumulator is complete.
 //   warps 2..9     : epilogue, two warps per TMEM lane quarter.  Warp w
 //                    reads TMEM lanes 32*(w%4) .. +31 (one tile row per
 //                    thread); warps 2..5 take columns 0..127 of the tile and
@@ -84,14 +87,14 @@ constexpr int kStages = kCta == 2 ? 6 : 4;
 #define QKN_GEMM_EPI_WARPS 8
 #endif
 #ifndef QKN_GEMM_GROUP_M
-#define QKN_GEMM_GROUP_M 0
+#define QKN_GEMM_GROUP_M -1
 #endif
 constexpr int kEpiWarps = QKN_GEMM_EPI_WARPS;  // 4 or 8: one or two per TMEM lane quarter
 static_assert(kEpiWarps == 4 || kEpiWarps == 8, "the epilogue has 4 or 8 warps");
 constexpr int kEpiSplit = kEpiWarps / 4;       // warps sharing one lane quarter (column split)
 constexpr int kEpiCols = kBN / kEpiSplit;      // tile columns per epilogue warp
 constexpr int kThreads = 64 + 32 * kEpiWarps;
-constexpr int kGroupM = QKN_GEMM_GROUP_M;      // token tiles per raster group; 0 = one group
+constexpr int kGroupM = QKN_GEMM_GROUP_M;      // token blocks per raster group: -1 = the host's choice, 0 = one group
 constexpr int kBNLocal = kBN / kCta;           // W rows (output columns) each CTA stages
 constexpr int kABytes = kBM * kBK * 2;
 constexpr int kBBytes = kBNLocal * kBK * 2;
@@ -116,6 +119,7 @@ struct GemmParams {
     int32_t m_tiles;         // ceil(T / kBM): 128-token tiles (= strips)
     int32_t m_units;         // ceil(T / (kBM * kCta)): token blocks of one MMA
     int32_t num_units;       // m_units * n_tiles: work units (one per CTA group)
+    int32_t group_units;     // token blocks per raster group, 1 .. m_units
     uint64_t timeout_ns;     // bound on every mbarrier wait
     // Fused QK-Norm (all null / unused when counters is null).
     int *counters;           // [2][m_tiles] tiles stored per strip, zero at launch

@@ -174,6 +174,32 @@ def test_projection_full_size_sampled_rows():
     assert qk.device_timeouts() == 0
 
 
+@pytest.mark.parametrize("T,D,Hq,Hk,Hv", [
+    (16284, 3072, 2048, 512, 512),     # X (100 MB) beyond half of L2, W (19 MB) within: one token block per group
+    (12000, 4096, 4096, 4096, 2048),   # X (99 MB) and W (84 MB) beyond: groups of ~sqrt(clusters), ragged last
+])
+def test_projection_rasters_beyond_l2(T, D, Hq, Hk, Hv):
+    """Shapes whose operands do not fit in half of L2 run the GEMM in smaller
+    raster groups (on a B200: 148 SMs, 126 MB L2); the tiles, their sums and
+    the fused rescale must not depend on the order.  Checked on sampled rows
+    against the oracle, with the ragged last strip among them, and bit for bit
+    against the two-launch path."""
+    b = workloads.qkv_projection(T=T, D=D, Hq=Hq, Hk=Hk, Hv=Hv, seed=T + D)
+    x, w = b.x.to(DEV), b.w.to(DEV)
+    gq, gk = b.gamma_q.to(DEV), b.gamma_k.to(DEV)
+    plain, qs, ks = qk.qknorm_qkv_gemm_stats(x, w, Hq, Hk, Hv)
+    fused = qk.qknorm_qkv_projection(x, w, gq, gk, Hq, Hk, Hv, b.eps)
+    two = qk.qknorm_qkv_projection(x, w, _unaligned_copy(gq), _unaligned_copy(gk), Hq, Hk, Hv, b.eps)
+    torch.cuda.synchronize()
+    assert torch.equal(fused, two)
+    rows = _sample_rows(T, 16, T + 2)
+    proj = check_projection(b, plain, rows)
+    check_tile_sums(proj, qs, rows, 0, Hq // TILE)
+    check_tile_sums(proj, ks, rows, Hq, Hk // TILE)
+    check_normalized(b, proj, fused, rows)
+    assert qk.device_timeouts() == 0
+
+
 def test_projection_is_deterministic_and_matches_combine_apply():
     """Two runs agree bit for bit, and the pipeline equals gemm_stats followed
     by the public qknorm_combine_apply with 256-column shards (Hq == Hk)."""
