@@ -1053,8 +1053,8 @@ qkn_status qknorm_tp_layerwise(int32_t R, int32_t first_rank, int32_t n_local, c
     if (!q_in || !q_out || !gamma_q || !k_in || !k_out || !gamma_k || !recv)
         return fail(QKN_ERR_INVALID_ARG, "null pointer array");
     for (int r = 0; r < R; ++r)
-        if (!recv[r] || (reinterpret_cast<uintptr_t>(recv[r]) & 7u))
-            return fail(QKN_ERR_INVALID_ARG, "receive buffer %d null or not 8-byte aligned", r);
+        if (!recv[r] || (reinterpret_cast<uintptr_t>(recv[r]) & 15u))
+            return fail(QKN_ERR_INVALID_ARG, "receive buffer %d null or not 16-byte aligned", r);
     const int per_vec = 16 / esz;
     if (hq_shard % per_vec || hk_shard % per_vec || (q_stride * esz) % 16 || (k_stride * esz) % 16)
         return fail(QKN_ERR_UNSUPPORTED, "shard widths and strides must be whole 16-byte vectors");
@@ -1089,8 +1089,8 @@ qkn_status qknorm_tp_layerwise(int32_t R, int32_t first_rank, int32_t n_local, c
     const int64_t vq = hq_shard / per_vec, vk = hk_shard / per_vec, vmax = vq > vk ? vq : vk;
     int nv, threads;
     int64_t tokens_per_block = 1;
-    if (vmax <= 128) {  // one token per warp, four warps per block
-        auto lanes_nv = [](int64_t v) { return v <= 32 ? 1 : (v <= 64 ? 2 : 4); };
+    if (vmax <= 256) {  // one token per warp, four warps per block
+        auto lanes_nv = [](int64_t v) { return v <= 32 ? 1 : (v <= 64 ? 2 : (v <= 128 ? 4 : 8)); };
         int nvq = lanes_nv(vq), nvk = lanes_nv(vk);
         if (nvk > nvq) nvq = nvk;  // instantiated with NVK <= NVQ
         nv = -(8 * nvq + nvk);

@@ -21,41 +21,6 @@ __device__ unsigned int g_tp_aborted_epoch = 0;
 
 // Memory scope of the exchange: system when some ranks are on other GPUs
 // (peer memory), GPU when every rank runs in this launch.
-template <bool SYS>
-__device__ __forceinline__ void st_relaxed(unsigned long long *p, unsigned long long v) {
-    if constexpr (SYS)
-        asm volatile("st.relaxed.sys.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
-    else
-        asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
-}
-
-template <bool SYS>
-__device__ __forceinline__ void st_release(unsigned long long *p, unsigned long long v) {
-    if constexpr (SYS)
-        asm volatile("st.release.sys.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
-    else
-        asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
-}
-
-template <bool SYS>
-__device__ __forceinline__ unsigned long long ld_acquire(const unsigned long long *p) {
-    unsigned long long v;
-    if constexpr (SYS)
-        asm volatile("ld.acquire.sys.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-    else
-        asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-    return v;
-}
-
-template <bool SYS>
-__device__ __forceinline__ unsigned long long ld_relaxed(const unsigned long long *p) {
-    unsigned long long v;
-    if constexpr (SYS)
-        asm volatile("ld.relaxed.sys.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-    else
-        asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-    return v;
-}
 
 __device__ __forceinline__ uint64_t now_ns() {
     uint64_t t;
@@ -71,27 +36,56 @@ __device__ __forceinline__ bool aborted(uint32_t epoch) {
     return *reinterpret_cast<volatile unsigned int *>(&g_tp_aborted_epoch) == epoch;
 }
 
-// Waits (bounded) until the word at `src` carries `epoch`; its value, or
+// Publishes this rank's partial sums for one token (the Q word, then the K
+// word, one 16-byte store).  Each word carries the call's epoch beside its
+// value, so a reader that sees the epoch in a word has that word's value:
+// nothing else is communicated, so no ordering between the words or with
+// other memory is needed and relaxed stores suffice.
+template <bool SYS>
+__device__ __forceinline__ void publish_pair(unsigned long long *dst, uint32_t epoch, float sq, float sk) {
+    const unsigned long long wq = pack(epoch, sq), wk = pack(epoch, sk);
+    if constexpr (SYS)
+        asm volatile("st.relaxed.sys.global.v2.u64 [%0], {%1, %2};" ::"l"(dst), "l"(wq), "l"(wk) : "memory");
+    else
+        asm volatile("st.relaxed.gpu.global.v2.u64 [%0], {%1, %2};" ::"l"(dst), "l"(wq), "l"(wk) : "memory");
+}
+
+template <bool SYS>
+__device__ __forceinline__ void load_pair(const unsigned long long *src, unsigned long long &wq,
+                                          unsigned long long &wk) {
+    if constexpr (SYS)
+        asm volatile("ld.relaxed.sys.global.v2.u64 {%0, %1}, [%2];" : "=l"(wq), "=l"(wk) : "l"(src) : "memory");
+    else
+        asm volatile("ld.relaxed.gpu.global.v2.u64 {%0, %1}, [%2];" : "=l"(wq), "=l"(wk) : "l"(src) : "memory");
+}
+
+// Waits (bounded) until both words at `src` carry `epoch`; their values, or
 // false after a timeout or an abort of this call.
 template <bool SYS>
-__device__ __forceinline__ bool wait_word(const unsigned long long *src, uint32_t epoch, uint64_t timeout_ns,
-                                          float &v) {
-    unsigned long long w = ld_acquire<SYS>(src);
-    if (static_cast<uint32_t>(w >> 32) != epoch) {
+__device__ __forceinline__ bool wait_pair(const unsigned long long *src, uint32_t epoch, uint64_t timeout_ns,
+                                          float &vq, float &vk) {
+    unsigned long long wq, wk;
+    load_pair<SYS>(src, wq, wk);
+    if (static_cast<uint32_t>(wq >> 32) != epoch || static_cast<uint32_t>(wk >> 32) != epoch) {
         const uint64_t t0 = now_ns();
-        for (;;) {
+        for (uint32_t it = 1;; ++it) {
             __nanosleep(32);
-            w = ld_acquire<SYS>(src);
-            if (static_cast<uint32_t>(w >> 32) == epoch) break;
-            if (aborted(epoch)) return false;
-            if (now_ns() - t0 > timeout_ns) {
-                atomicExch(&g_tp_timeout, 4);
-                atomicExch(&g_tp_aborted_epoch, epoch);
-                return false;
+            load_pair<SYS>(src, wq, wk);
+            if (static_cast<uint32_t>(wq >> 32) == epoch && static_cast<uint32_t>(wk >> 32) == epoch) break;
+            // every waiting lane of the GPU would read the same abort word:
+            // look at it (and the clock) every 64 polls only
+            if ((it & 63u) == 0) {
+                if (aborted(epoch)) return false;
+                if (now_ns() - t0 > timeout_ns) {
+                    atomicExch(&g_tp_timeout, 4);
+                    atomicExch(&g_tp_aborted_epoch, epoch);
+                    return false;
+                }
             }
         }
     }
-    v = __uint_as_float(static_cast<uint32_t>(w));
+    vq = __uint_as_float(static_cast<uint32_t>(wq));
+    vk = __uint_as_float(static_cast<uint32_t>(wk));
     return true;
 }
 
@@ -179,18 +173,9 @@ __global__ void __launch_bounds__(kTpMaxThreads) tp_rows_kernel(const __grid_con
             float vq = 0.0f, vk = 0.0f;
             bool ok = true;
             if (lane < p.R) {
-                // the Q word, then the K word with release: a reader that
-                // sees the K word's epoch (acquire) sees the Q word too
-                unsigned long long *dst = p.recv[lane] + (static_cast<int64_t>(rank) * p.T + t) * 2;
-                st_relaxed<SYS>(dst, pack(p.epoch, Sq));
-                st_release<SYS>(dst + 1, pack(p.epoch, Sk));
-                const unsigned long long *src = p.recv[rank] + (static_cast<int64_t>(lane) * p.T + t) * 2;
-                ok = wait_word<SYS>(src + 1, p.epoch, p.timeout_ns, vk);
-                if (ok) {
-                    const unsigned long long wq = ld_relaxed<SYS>(src);
-                    ok = static_cast<uint32_t>(wq >> 32) == p.epoch;
-                    vq = __uint_as_float(static_cast<uint32_t>(wq));
-                }
+                publish_pair<SYS>(p.recv[lane] + (static_cast<int64_t>(rank) * p.T + t) * 2, p.epoch, Sq, Sk);
+                ok = wait_pair<SYS>(p.recv[rank] + (static_cast<int64_t>(lane) * p.T + t) * 2, p.epoch,
+                                    p.timeout_ns, vq, vk);
             }
             ok = __all_sync(0xFFFFFFFFu, ok);
             // Phase A aggregation: the R partials added in rank order, fp32.
@@ -227,17 +212,116 @@ __global__ void __launch_bounds__(kTpMaxThreads) tp_rows_kernel(const __grid_con
     }
 }
 
-// Narrow shard rows (at most 32 * NVQ vectors of Q, 32 * NVK of K): one warp per token, kTpWarps
-// warps per block, no block barrier.  Warp w of block b of a rank takes
-// tokens (b * kTpWarps + w), + G * kTpWarps, ...; lane i exchanges with rank
-// i as in the block form, every lane gets the sums by shuffles, and the warp
-// then scales its row as (x * gamma) * r (the same products as the block
-// form, formed after the wait to keep registers for more warps in flight).
+// Narrow shard rows (at most 32 * NVQ vectors of Q, 32 * NVK of K): one warp
+// per token, kTpWarps warps per block, no block barrier.  Warp w of block b
+// of a rank takes tokens (b * kTpWarps + w), + G * kTpWarps, ...; lane i
+// exchanges with rank i as in the block form, every lane gets the sums by
+// shuffles, and the warp then scales its row as (x * gamma) * r (the same
+// products as the block form).  The exchange is a round trip through memory,
+// so throughput comes from the number of tokens in flight: the warp holds
+// only its row (gamma is re-read from L1 when the row is scaled) and the
+// register cap below fits as many warps on an SM as the row's registers
+// allow.
 constexpr int kTpWarps = 4;
 
+#ifndef QKN_TP_PIPE
+#define QKN_TP_PIPE 1
+#endif
+constexpr int kTpPipe = QKN_TP_PIPE;  // tokens a warp has in flight at once
+
+#ifndef QKN_TP_REGS_PER_VEC
+#define QKN_TP_REGS_PER_VEC 4
+#endif
+template <int NVQ, int NVK>
+constexpr int tp_warp_min_blocks() {
+    // registers per 16-byte vector held, plus ~40 for the rest
+    constexpr int regs = QKN_TP_REGS_PER_VEC * (NVQ + NVK) * kTpPipe + 40;
+    return 65536 / (32 * kTpWarps * regs) < 16 ? 65536 / (32 * kTpWarps * regs) : 16;
+}
+
+// One token's rows of this rank, held in registers.
+template <typename E, int NVQ, int NVK>
+struct TpRow {
+    uint4 xq[NVQ], xk[NVK];
+    float sq, sk;
+};
+
+template <typename E, int NVQ, int NVK>
+__device__ __forceinline__ void tp_load(const TpParams &p, const RankPtrs &rp, int64_t t, int lane,
+                                        TpRow<E, NVQ, NVK> &row) {
+    const char *qrow = rp.q_in + t * p.q_stride_bytes;
+    const char *krow = rp.k_in + t * p.k_stride_bytes;
+#pragma unroll
+    for (int i = 0; i < NVQ; ++i) {
+        const int vi = lane + 32 * i;
+        row.xq[i] = vi < p.q_vecs ? ld_stream(qrow + static_cast<int64_t>(vi) * 16) : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int i = 0; i < NVK; ++i) {
+        const int vi = lane + 32 * i;
+        row.xk[i] = vi < p.k_vecs ? ld_stream(krow + static_cast<int64_t>(vi) * 16) : make_uint4(0u, 0u, 0u, 0u);
+    }
+}
+
+// Phase A, local step and publication: the shard's squared sums, written to
+// every rank's receive buffer (lane i to rank i).
 template <typename E, int NVQ, int NVK, bool SYS>
-__global__ void __launch_bounds__(32 * kTpWarps) tp_warp_kernel(const __grid_constant__ TpParams p) {
+__device__ __forceinline__ void tp_publish(const TpParams &p, int rank, int64_t t, int lane,
+                                           TpRow<E, NVQ, NVK> &row) {
+    row.sq = warp_sum(sumsq_pairs<E, NVQ>(row.xq));
+    row.sk = warp_sum(sumsq_pairs<E, NVK>(row.xk));
+    if (lane < p.R) publish_pair<SYS>(p.recv[lane] + (static_cast<int64_t>(rank) * p.T + t) * 2, p.epoch, row.sq, row.sk);
+}
+
+// Waits for the other ranks' partials of token t, adds them in rank order
+// and stores (x * gamma) * r; a wait that gave up leaves the token unwritten
+// (the timeout is reported).
+template <typename E, int NVQ, int NVK, bool SYS>
+__device__ __forceinline__ void tp_finish(const TpParams &p, const RankPtrs &rp, int rank, int64_t t, int lane,
+                                          const TpRow<E, NVQ, NVK> &row) {
     constexpr int KG = Elem<E>::kGVecs;
+    float vq = 0.0f, vk = 0.0f;
+    bool ok = true;
+    if (lane < p.R)
+        ok = wait_pair<SYS>(p.recv[rank] + (static_cast<int64_t>(lane) * p.T + t) * 2, p.epoch, p.timeout_ns, vq, vk);
+    if (!__all_sync(0xFFFFFFFFu, ok)) return;  // a wait gave up: token left unwritten (reported)
+    float Aq = 0.0f, Ak = 0.0f;  // Phase A aggregation, in rank order
+    for (int i = 0; i < p.R; ++i) {
+        Aq += __shfl_sync(0xFFFFFFFFu, vq, i);
+        Ak += __shfl_sync(0xFFFFFFFFu, vk, i);
+    }
+    const float rq1 = rms_factor(Aq, p.inv_hq, p.eps), rk1 = rms_factor(Ak, p.inv_hk, p.eps);
+    const F2 rq = f2(rq1, rq1), rk = f2(rk1, rk1);
+    char *qo = rp.q_out + t * p.q_stride_bytes;
+    char *ko = rp.k_out + t * p.k_stride_bytes;
+#pragma unroll
+    for (int i = 0; i < NVQ; ++i) {
+        const int vi = lane + 32 * i;
+        if (vi < p.q_vecs) {
+            uint4 g[KG];
+            ld_gamma_vec<E>(rp.gamma_q, vi, p.q_vecs, 0, g);
+            st_stream(qo + static_cast<int64_t>(vi) * 16, scale_vec<E>(row.xq[i], g, rq));
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < NVK; ++i) {
+        const int vi = lane + 32 * i;
+        if (vi < p.k_vecs) {
+            uint4 g[KG];
+            ld_gamma_vec<E>(rp.gamma_k, vi, p.k_vecs, 0, g);
+            st_stream(ko + static_cast<int64_t>(vi) * 16, scale_vec<E>(row.xk[i], g, rk));
+        }
+    }
+}
+
+// Warp w of block c takes tokens s, s + step, s + 2 step, ... (s = c * 4 + w,
+// step = G * 4), kTpPipe at a time: it loads and publishes all of them
+// before it waits for the first, so the exchange of one overlaps the loads of
+// the next.  Every rank's warp (c, w) has the same sequence, and publishes a
+// group before waiting on it, so no wait depends on a warp that waits on it.
+template <typename E, int NVQ, int NVK, bool SYS>
+__global__ void __launch_bounds__(32 * kTpWarps, tp_warp_min_blocks<NVQ, NVK>())
+    tp_warp_kernel(const __grid_constant__ TpParams p) {
     pdl_wait_and_release();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int local = blockIdx.x / p.blocks_per_rank;
@@ -246,63 +330,17 @@ __global__ void __launch_bounds__(32 * kTpWarps) tp_warp_kernel(const __grid_con
     const RankPtrs rp = p.local[local];
     const int64_t step = static_cast<int64_t>(p.blocks_per_rank) * kTpWarps;
 
-    uint4 gq[NVQ][KG], gk[NVK][KG];
+    for (int64_t t0 = static_cast<int64_t>(c) * kTpWarps + warp; t0 < p.T; t0 += kTpPipe * step) {
+        TpRow<E, NVQ, NVK> row[kTpPipe];
 #pragma unroll
-    for (int i = 0; i < NVQ; ++i) ld_gamma_vec<E>(rp.gamma_q, lane + 32 * i, p.q_vecs, 0, gq[i]);
+        for (int j = 0; j < kTpPipe; ++j)
+            if (t0 + j * step < p.T) tp_load<E, NVQ, NVK>(p, rp, t0 + j * step, lane, row[j]);
 #pragma unroll
-    for (int i = 0; i < NVK; ++i) ld_gamma_vec<E>(rp.gamma_k, lane + 32 * i, p.k_vecs, 0, gk[i]);
-    for (int64_t t = static_cast<int64_t>(c) * kTpWarps + warp; t < p.T; t += step) {
-        const char *qrow = rp.q_in + t * p.q_stride_bytes;
-        const char *krow = rp.k_in + t * p.k_stride_bytes;
-        uint4 xq[NVQ], xk[NVK];
+        for (int j = 0; j < kTpPipe; ++j)
+            if (t0 + j * step < p.T) tp_publish<E, NVQ, NVK, SYS>(p, rank, t0 + j * step, lane, row[j]);
 #pragma unroll
-        for (int i = 0; i < NVQ; ++i) {
-            const int vi = lane + 32 * i;
-            xq[i] = vi < p.q_vecs ? ld_stream(qrow + static_cast<int64_t>(vi) * 16) : make_uint4(0u, 0u, 0u, 0u);
-        }
-#pragma unroll
-        for (int i = 0; i < NVK; ++i) {
-            const int vi = lane + 32 * i;
-            xk[i] = vi < p.k_vecs ? ld_stream(krow + static_cast<int64_t>(vi) * 16) : make_uint4(0u, 0u, 0u, 0u);
-        }
-        const float Sq = warp_sum(sumsq_pairs<E, NVQ>(xq));  // Phase A, local step
-        const float Sk = warp_sum(sumsq_pairs<E, NVK>(xk));
-        if (lane < p.R) {
-            unsigned long long *dst = p.recv[lane] + (static_cast<int64_t>(rank) * p.T + t) * 2;
-            st_relaxed<SYS>(dst, pack(p.epoch, Sq));
-            st_release<SYS>(dst + 1, pack(p.epoch, Sk));
-        }
-        float vq = 0.0f, vk = 0.0f;
-        bool ok = true;
-        if (lane < p.R) {
-            const unsigned long long *src = p.recv[rank] + (static_cast<int64_t>(lane) * p.T + t) * 2;
-            ok = wait_word<SYS>(src + 1, p.epoch, p.timeout_ns, vk);
-            if (ok) {
-                const unsigned long long wq = ld_relaxed<SYS>(src);
-                ok = static_cast<uint32_t>(wq >> 32) == p.epoch;
-                vq = __uint_as_float(static_cast<uint32_t>(wq));
-            }
-        }
-        if (!__all_sync(0xFFFFFFFFu, ok)) continue;  // a wait gave up: token left unwritten (reported)
-        float Aq = 0.0f, Ak = 0.0f;  // Phase A aggregation, in rank order
-        for (int i = 0; i < p.R; ++i) {
-            Aq += __shfl_sync(0xFFFFFFFFu, vq, i);
-            Ak += __shfl_sync(0xFFFFFFFFu, vk, i);
-        }
-        const float rq1 = rms_factor(Aq, p.inv_hq, p.eps), rk1 = rms_factor(Ak, p.inv_hk, p.eps);
-        const F2 rq = f2(rq1, rq1), rk = f2(rk1, rk1);
-        char *qo = rp.q_out + t * p.q_stride_bytes;
-        char *ko = rp.k_out + t * p.k_stride_bytes;
-#pragma unroll
-        for (int i = 0; i < NVQ; ++i) {
-            const int vi = lane + 32 * i;
-            if (vi < p.q_vecs) st_stream(qo + static_cast<int64_t>(vi) * 16, scale_vec<E>(xq[i], gq[i], rq));
-        }
-#pragma unroll
-        for (int i = 0; i < NVK; ++i) {
-            const int vi = lane + 32 * i;
-            if (vi < p.k_vecs) st_stream(ko + static_cast<int64_t>(vi) * 16, scale_vec<E>(xk[i], gk[i], rk));
-        }
+        for (int j = 0; j < kTpPipe; ++j)
+            if (t0 + j * step < p.T) tp_finish<E, NVQ, NVK, SYS>(p, rp, rank, t0 + j * step, lane, row[j]);
     }
 }
 
@@ -323,6 +361,10 @@ const void *tp_kernel(int nv) {
         case -(8 * 4 + 1): return (const void *)tp_warp_kernel<E, 4, 1, SYS>;
         case -(8 * 4 + 2): return (const void *)tp_warp_kernel<E, 4, 2, SYS>;
         case -(8 * 4 + 4): return (const void *)tp_warp_kernel<E, 4, 4, SYS>;
+        case -(8 * 8 + 1): return (const void *)tp_warp_kernel<E, 8, 1, SYS>;
+        case -(8 * 8 + 2): return (const void *)tp_warp_kernel<E, 8, 2, SYS>;
+        case -(8 * 8 + 4): return (const void *)tp_warp_kernel<E, 8, 4, SYS>;
+        case -(8 * 8 + 8): return (const void *)tp_warp_kernel<E, 8, 8, SYS>;
         default: return nullptr;
     }
 }

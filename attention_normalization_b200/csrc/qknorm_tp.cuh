@@ -7,21 +7,21 @@
 //     K rows; it computes the shard's squared sums and the ranks add their
 //     partial sums (fp32) to get the global sums -- a scalar per token and
 //     tensor crosses between ranks instead of the activations.
-//   Phase B: warp 0 carries the exchange (it writes this rank's partials into
-//     every rank's receive buffer and waits for the others') while the other
-//     warps multiply the shard by gamma, which does not depend on the
-//     reduction; then the global factor scales the products and only the
-//     final values are stored.
+//   Phase B: the shard times gamma is scaled by the global factor and only
+//     the final values are stored.  For shard rows above 256 vectors warp 0
+//     carries the exchange (it writes this rank's partials into every rank's
+//     receive buffer and waits for the others') while the other warps
+//     multiply the shard by gamma, which does not depend on the reduction;
+//     narrower rows run one token per warp (four per block, no block
+//     barrier), the multiply after the wait, so that the warp holds only its
+//     row and more tokens are in flight per SM.
 //   Deadlock-safe persistent execution: the grid is bounded by the resident
 //     blocks and each block loops over tokens.
 //
-// Shard rows of at most 128 vectors run one token per warp (four per block,
-// no block barrier), wider ones one token per block.
-//
 // One kernel serves two deployments:
 //   * one rank per GPU: each GPU launches its own rank; receive buffers of the
-//     other ranks are reached through peer mappings (P2P stores and loads,
-//     release / acquire at system scope);
+//     other ranks are reached through peer mappings (P2P stores and loads at
+//     system scope);
 //   * several ranks in one launch on one GPU (the test form here): the ranks'
 //     blocks wait on one another, so the launch is cooperative (all blocks
 //     resident at once).
@@ -34,6 +34,9 @@
 // (0 = Q, 1 = K)).  A word counts as arrived when its epoch field equals the
 // call's epoch, so buffers are never cleared between calls: each call on the
 // same buffers uses a new epoch (buffers start zeroed, epoch 0 is never used).
+// Each word validates itself and carries the only data exchanged, so the two
+// words of a token are written with one relaxed 16-byte store and polled with
+// relaxed loads: no fence or release/acquire pair on the exchange path.
 // Every wait is bounded by the global timer; on expiry the kernel records a
 // code, marks the epoch aborted so every other wait of the call gives up at
 // once, and skips the affected tokens (their outputs are not written).

@@ -233,16 +233,17 @@ int64_t qknorm_qkv_projection_noalloc_max_bytes(void);
 /*
  * Tensor-parallel layerwise QK-Norm: the paper's multi-GPU kernel (Phase A:
  * each rank squares and sums its hidden-dimension shard and the ranks add
- * their scalar partial sums in fp32; Phase B: warp 0 of each block carries
- * that exchange while the other warps multiply the shard by gamma, then the
- * global factor scales it; deadlock-safe persistent blocks).
+ * their scalar partial sums in fp32; Phase B: the global factor scales the
+ * shard times gamma -- for shard rows above 256 vectors warp 0 of each block
+ * carries the exchange while the other warps multiply the shard by gamma,
+ * narrower rows run one token per warp; deadlock-safe persistent blocks).
  *   R ranks each hold a shard of every token's Q row (hq_shard columns of
  *   Hq_full) and K row (hk_shard of Hk_full).  This call runs the n_local
  *   ranks first_rank .. first_rank + n_local - 1; local rank j's rows are
  *   q_in[j] / q_out[j] ([T rows, stride q_stride]), gamma slice gamma_q[j]
  *   [hq_shard], and likewise for K.  out == in normalizes in place.
  *   recv[r] (r < R) is rank r's receive buffer, qknorm_tp_recv_bytes(R, T)
- *   bytes: a device pointer valid on this GPU -- its own memory for local
+ *   bytes, 16-byte aligned: a device pointer valid on this GPU -- its own memory for local
  *   ranks, a peer mapping (cudaIpcOpenMemHandle or similar) for ranks on other
  *   GPUs.  Buffers start zeroed; each call on the same buffers passes a new
  *   epoch (> 0), and all ranks of one call pass the same epoch.

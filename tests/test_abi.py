@@ -424,7 +424,8 @@ def _tp_call(lib, **kw):
     ({"qs": 200}, INVALID),                        # stride below the shard width
     ({"hq": 252, "qs": 256}, UNSUPPORTED),         # shard width not whole 16-byte vectors
     ({"recv": [0x40000000, 0, 0x40200000, 0x40300000]}, INVALID),
-    ({"recv": [0x40000004, 0x40100000, 0x40200000, 0x40300000]}, INVALID),  # not 8-byte aligned
+    ({"recv": [0x40000004, 0x40100000, 0x40200000, 0x40300000]}, INVALID),  # not 16-byte aligned
+    ({"recv": [0x40000000, 0x40100008, 0x40200000, 0x40300000]}, INVALID),
 ])
 def test_tp_validation(lib, kw, want):
     assert _tp_call(lib, **kw) == want
