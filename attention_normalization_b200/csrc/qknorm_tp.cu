@@ -224,10 +224,10 @@ __global__ void __launch_bounds__(kTpMaxThreads) tp_rows_kernel(const __grid_con
 // allow.
 constexpr int kTpWarps = 4;
 
-#ifndef QKN_TP_PIPE
-#define QKN_TP_PIPE 1
+#ifndef QKN_TP_AHEAD
+#define QKN_TP_AHEAD 2
 #endif
-constexpr int kTpPipe = QKN_TP_PIPE;  // tokens a warp has in flight at once
+constexpr int kTpAhead = QKN_TP_AHEAD;  // tokens a warp publishes ahead of the one it finishes
 
 #ifndef QKN_TP_REGS_PER_VEC
 #define QKN_TP_REGS_PER_VEC 4
@@ -235,7 +235,7 @@ constexpr int kTpPipe = QKN_TP_PIPE;  // tokens a warp has in flight at once
 template <int NVQ, int NVK>
 constexpr int tp_warp_min_blocks() {
     // registers per 16-byte vector held, plus ~40 for the rest
-    constexpr int regs = QKN_TP_REGS_PER_VEC * (NVQ + NVK) * kTpPipe + 40;
+    constexpr int regs = QKN_TP_REGS_PER_VEC * (NVQ + NVK) + 40;
     return 65536 / (32 * kTpWarps * regs) < 16 ? 65536 / (32 * kTpWarps * regs) : 16;
 }
 
@@ -246,7 +246,17 @@ struct TpRow {
     float sq, sk;
 };
 
-template <typename E, int NVQ, int NVK>
+// KEEP: the row will be read again soon (kept in L2 at normal priority);
+// else its last read (streaming).
+template <bool KEEP>
+__device__ __forceinline__ uint4 tp_ld(const char *p) {
+    if constexpr (KEEP)
+        return __ldcg(reinterpret_cast<const uint4 *>(p));
+    else
+        return ld_stream(p);
+}
+
+template <typename E, int NVQ, int NVK, bool KEEP = false>
 __device__ __forceinline__ void tp_load(const TpParams &p, const RankPtrs &rp, int64_t t, int lane,
                                         TpRow<E, NVQ, NVK> &row) {
     const char *qrow = rp.q_in + t * p.q_stride_bytes;
@@ -254,12 +264,12 @@ __device__ __forceinline__ void tp_load(const TpParams &p, const RankPtrs &rp, i
 #pragma unroll
     for (int i = 0; i < NVQ; ++i) {
         const int vi = lane + 32 * i;
-        row.xq[i] = vi < p.q_vecs ? ld_stream(qrow + static_cast<int64_t>(vi) * 16) : make_uint4(0u, 0u, 0u, 0u);
+        row.xq[i] = vi < p.q_vecs ? tp_ld<KEEP>(qrow + static_cast<int64_t>(vi) * 16) : make_uint4(0u, 0u, 0u, 0u);
     }
 #pragma unroll
     for (int i = 0; i < NVK; ++i) {
         const int vi = lane + 32 * i;
-        row.xk[i] = vi < p.k_vecs ? ld_stream(krow + static_cast<int64_t>(vi) * 16) : make_uint4(0u, 0u, 0u, 0u);
+        row.xk[i] = vi < p.k_vecs ? tp_ld<KEEP>(krow + static_cast<int64_t>(vi) * 16) : make_uint4(0u, 0u, 0u, 0u);
     }
 }
 
@@ -315,10 +325,14 @@ __device__ __forceinline__ void tp_finish(const TpParams &p, const RankPtrs &rp,
 }
 
 // Warp w of block c takes tokens s, s + step, s + 2 step, ... (s = c * 4 + w,
-// step = G * 4), kTpPipe at a time: it loads and publishes all of them
-// before it waits for the first, so the exchange of one overlaps the loads of
-// the next.  Every rank's warp (c, w) has the same sequence, and publishes a
-// group before waiting on it, so no wait depends on a warp that waits on it.
+// step = G * 4) and publishes kTpAhead tokens ahead of the one it finishes:
+// iteration k loads token k (kept in L2), publishes its partial sums, then
+// re-reads token k - kTpAhead (an L2 hit, read kTpAhead tokens earlier),
+// waits for that token's exchange (by now mostly complete) and stores it.
+// No row is held across a wait on the exchange, so the warp's registers stay
+// those of one row.  Every rank's warp (c, w) has the same sequence and
+// publishes a token before it waits on it, so no wait depends on a warp that
+// waits on it.
 template <typename E, int NVQ, int NVK, bool SYS>
 __global__ void __launch_bounds__(32 * kTpWarps, tp_warp_min_blocks<NVQ, NVK>())
     tp_warp_kernel(const __grid_constant__ TpParams p) {
@@ -329,18 +343,19 @@ __global__ void __launch_bounds__(32 * kTpWarps, tp_warp_min_blocks<NVQ, NVK>())
     const int rank = p.first_rank + local;
     const RankPtrs rp = p.local[local];
     const int64_t step = static_cast<int64_t>(p.blocks_per_rank) * kTpWarps;
-
-    for (int64_t t0 = static_cast<int64_t>(c) * kTpWarps + warp; t0 < p.T; t0 += kTpPipe * step) {
-        TpRow<E, NVQ, NVK> row[kTpPipe];
-#pragma unroll
-        for (int j = 0; j < kTpPipe; ++j)
-            if (t0 + j * step < p.T) tp_load<E, NVQ, NVK>(p, rp, t0 + j * step, lane, row[j]);
-#pragma unroll
-        for (int j = 0; j < kTpPipe; ++j)
-            if (t0 + j * step < p.T) tp_publish<E, NVQ, NVK, SYS>(p, rank, t0 + j * step, lane, row[j]);
-#pragma unroll
-        for (int j = 0; j < kTpPipe; ++j)
-            if (t0 + j * step < p.T) tp_finish<E, NVQ, NVK, SYS>(p, rp, rank, t0 + j * step, lane, row[j]);
+    const int64_t first = static_cast<int64_t>(c) * kTpWarps + warp;
+    const int64_t n = first < p.T ? (p.T - 1 - first) / step + 1 : 0;  // tokens of this warp
+    for (int64_t k = 0; k < n + kTpAhead; ++k) {
+        if (k < n) {
+            TpRow<E, NVQ, NVK> row;
+            tp_load<E, NVQ, NVK, true>(p, rp, first + k * step, lane, row);
+            tp_publish<E, NVQ, NVK, SYS>(p, rank, first + k * step, lane, row);
+        }
+        if (k >= kTpAhead) {
+            TpRow<E, NVQ, NVK> row;
+            tp_load<E, NVQ, NVK>(p, rp, first + (k - kTpAhead) * step, lane, row);
+            tp_finish<E, NVQ, NVK, SYS>(p, rp, rank, first + (k - kTpAhead) * step, lane, row);
+        }
     }
 }
 

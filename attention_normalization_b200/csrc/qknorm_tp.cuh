@@ -13,8 +13,10 @@
 //     receive buffer and waits for the others') while the other warps
 //     multiply the shard by gamma, which does not depend on the reduction;
 //     narrower rows run one token per warp (four per block, no block
-//     barrier), the multiply after the wait, so that the warp holds only its
-//     row and more tokens are in flight per SM.
+//     barrier), the multiply after the wait.  There a warp publishes two
+//     tokens ahead of the one it finishes and re-reads that one's row from
+//     L2, so its exchange is mostly complete when the warp waits on it and no
+//     row is held across a wait.
 //   Deadlock-safe persistent execution: the grid is bounded by the resident
 //     blocks and each block loops over tokens.
 //
