@@ -218,10 +218,10 @@ __global__ void __launch_bounds__(kTpMaxThreads) tp_rows_kernel(const __grid_con
 // exchanges with rank i as in the block form, every lane gets the sums by
 // shuffles, and the warp then scales its row as (x * gamma) * r (the same
 // products as the block form).  The exchange is a round trip through memory,
-// so throughput comes from the number of tokens in flight: the warp holds
-// only its row (gamma is re-read from L1 when the row is scaled) and the
-// register cap below fits as many warps on an SM as the row's registers
-// allow.
+// so throughput comes from the number of tokens in flight: a warp passes its
+// row through registers in batches (gamma re-read from L1 when the row is
+// scaled) and publishes ahead, and the register cap below fits as many warps
+// on an SM as one batch's registers allow.
 constexpr int kTpWarps = 4;
 
 #ifndef QKN_TP_AHEAD
@@ -229,22 +229,24 @@ constexpr int kTpWarps = 4;
 #endif
 constexpr int kTpAhead = QKN_TP_AHEAD;  // tokens a warp publishes ahead of the one it finishes
 
+#ifndef QKN_TP_BATCH
+#define QKN_TP_BATCH 4
+#endif
+// 16-byte vectors per lane a warp loads at once: a row passes through the
+// warp in batches, so registers depend on the batch, not on the row width.
+constexpr int kTpBatch = QKN_TP_BATCH;
+
 #ifndef QKN_TP_REGS_PER_VEC
 #define QKN_TP_REGS_PER_VEC 4
 #endif
 template <int NVQ, int NVK>
 constexpr int tp_warp_min_blocks() {
-    // registers per 16-byte vector held, plus ~40 for the rest
-    constexpr int regs = QKN_TP_REGS_PER_VEC * (NVQ + NVK) + 40;
+    // registers per 16-byte vector held (a batch of Q or K vectors, NVK <=
+    // NVQ, and their gamma vectors), plus ~40 for the rest
+    constexpr int held = 2 * (NVQ < kTpBatch ? NVQ : kTpBatch);
+    constexpr int regs = QKN_TP_REGS_PER_VEC * held + 40;
     return 65536 / (32 * kTpWarps * regs) < 16 ? 65536 / (32 * kTpWarps * regs) : 16;
 }
-
-// One token's rows of this rank, held in registers.
-template <typename E, int NVQ, int NVK>
-struct TpRow {
-    uint4 xq[NVQ], xk[NVK];
-    float sq, sk;
-};
 
 // KEEP: the row will be read again soon (kept in L2 at normal priority);
 // else its last read (streaming).
@@ -256,40 +258,72 @@ __device__ __forceinline__ uint4 tp_ld(const char *p) {
         return ld_stream(p);
 }
 
-template <typename E, int NVQ, int NVK, bool KEEP = false>
-__device__ __forceinline__ void tp_load(const TpParams &p, const RankPtrs &rp, int64_t t, int lane,
-                                        TpRow<E, NVQ, NVK> &row) {
-    const char *qrow = rp.q_in + t * p.q_stride_bytes;
-    const char *krow = rp.k_in + t * p.k_stride_bytes;
+template <int NV, bool KEEP, int B>
+__device__ __forceinline__ void tp_load_batch(const char *row, int nvecs, int lane, int b, uint4 (&x)[B]) {
 #pragma unroll
-    for (int i = 0; i < NVQ; ++i) {
-        const int vi = lane + 32 * i;
-        row.xq[i] = vi < p.q_vecs ? tp_ld<KEEP>(qrow + static_cast<int64_t>(vi) * 16) : make_uint4(0u, 0u, 0u, 0u);
-    }
-#pragma unroll
-    for (int i = 0; i < NVK; ++i) {
-        const int vi = lane + 32 * i;
-        row.xk[i] = vi < p.k_vecs ? tp_ld<KEEP>(krow + static_cast<int64_t>(vi) * 16) : make_uint4(0u, 0u, 0u, 0u);
+    for (int i = 0; i < B; ++i) {
+        const int vi = lane + 32 * (b + i);
+        x[i] = vi < nvecs ? tp_ld<KEEP>(row + static_cast<int64_t>(vi) * 16) : make_uint4(0u, 0u, 0u, 0u);
     }
 }
 
-// Phase A, local step and publication: the shard's squared sums, written to
-// every rank's receive buffer (lane i to rank i).
+// Phase A, local step and publication: the shard's squared sums, Q and K
+// batches loaded side by side, written to every rank's receive buffer (lane
+// i to rank i).
 template <typename E, int NVQ, int NVK, bool SYS>
-__device__ __forceinline__ void tp_publish(const TpParams &p, int rank, int64_t t, int lane,
-                                           TpRow<E, NVQ, NVK> &row) {
-    row.sq = warp_sum(sumsq_pairs<E, NVQ>(row.xq));
-    row.sk = warp_sum(sumsq_pairs<E, NVK>(row.xk));
-    if (lane < p.R) publish_pair<SYS>(p.recv[lane] + (static_cast<int64_t>(rank) * p.T + t) * 2, p.epoch, row.sq, row.sk);
+__device__ __forceinline__ void tp_publish(const TpParams &p, const RankPtrs &rp, int rank, int64_t t, int lane) {
+    constexpr int BQ = NVQ < kTpBatch ? NVQ : kTpBatch;
+    constexpr int BK = NVK < kTpBatch ? NVK : kTpBatch;
+    const char *qrow = rp.q_in + t * p.q_stride_bytes;
+    const char *krow = rp.k_in + t * p.k_stride_bytes;
+    float sq = 0.0f, sk = 0.0f;
+#pragma unroll
+    for (int b = 0; b < NVQ; b += BQ) {  // NVK <= NVQ
+        uint4 xq[BQ], xk[BK];
+        tp_load_batch<NVQ, true, BQ>(qrow, p.q_vecs, lane, b, xq);
+        if (b < NVK) tp_load_batch<NVK, true, BK>(krow, p.k_vecs, lane, b, xk);
+        sq += sumsq_pairs<E, BQ>(xq);
+        if (b < NVK) sk += sumsq_pairs<E, BK>(xk);
+    }
+    sq = warp_sum(sq);
+    sk = warp_sum(sk);
+    if (lane < p.R) publish_pair<SYS>(p.recv[lane] + (static_cast<int64_t>(rank) * p.T + t) * 2, p.epoch, sq, sk);
+}
+
+// Phase B for one shard row, from its first batch (already loaded) on:
+// (x * gamma) * r, batch by batch.
+template <typename E, int NV, int B>
+__device__ __forceinline__ void tp_scale_row(const char *in, char *out, const char *gamma, int nvecs, int lane,
+                                             F2 r, uint4 (&x)[B]) {
+    constexpr int KG = Elem<E>::kGVecs;
+#pragma unroll
+    for (int b = 0; b < NV; b += B) {
+        if (b > 0) tp_load_batch<NV, false, B>(in, nvecs, lane, b, x);
+#pragma unroll
+        for (int i = 0; i < B; ++i) {
+            const int vi = lane + 32 * (b + i);
+            if (vi < nvecs) {
+                uint4 g[KG];
+                ld_gamma_vec<E>(gamma, vi, nvecs, 0, g);
+                st_stream(out + static_cast<int64_t>(vi) * 16, scale_vec<E>(x[i], g, r));
+            }
+        }
+    }
 }
 
 // Waits for the other ranks' partials of token t, adds them in rank order
-// and stores (x * gamma) * r; a wait that gave up leaves the token unwritten
+// and stores (x * gamma) * r, re-reading the rows (the first batches of Q and
+// K while the exchange completes); a wait that gave up leaves the token unwritten
 // (the timeout is reported).
 template <typename E, int NVQ, int NVK, bool SYS>
-__device__ __forceinline__ void tp_finish(const TpParams &p, const RankPtrs &rp, int rank, int64_t t, int lane,
-                                          const TpRow<E, NVQ, NVK> &row) {
-    constexpr int KG = Elem<E>::kGVecs;
+__device__ __forceinline__ void tp_finish(const TpParams &p, const RankPtrs &rp, int rank, int64_t t, int lane) {
+    constexpr int BQ = NVQ < kTpBatch ? NVQ : kTpBatch;
+    constexpr int BK = NVK < kTpBatch ? NVK : kTpBatch;
+    const char *qrow = rp.q_in + t * p.q_stride_bytes;
+    const char *krow = rp.k_in + t * p.k_stride_bytes;
+    uint4 xq[BQ], xk[BK];
+    tp_load_batch<NVQ, false, BQ>(qrow, p.q_vecs, lane, 0, xq);
+    tp_load_batch<NVK, false, BK>(krow, p.k_vecs, lane, 0, xk);
     float vq = 0.0f, vk = 0.0f;
     bool ok = true;
     if (lane < p.R)
@@ -300,39 +334,19 @@ __device__ __forceinline__ void tp_finish(const TpParams &p, const RankPtrs &rp,
         Aq += __shfl_sync(0xFFFFFFFFu, vq, i);
         Ak += __shfl_sync(0xFFFFFFFFu, vk, i);
     }
-    const float rq1 = rms_factor(Aq, p.inv_hq, p.eps), rk1 = rms_factor(Ak, p.inv_hk, p.eps);
-    const F2 rq = f2(rq1, rq1), rk = f2(rk1, rk1);
-    char *qo = rp.q_out + t * p.q_stride_bytes;
-    char *ko = rp.k_out + t * p.k_stride_bytes;
-#pragma unroll
-    for (int i = 0; i < NVQ; ++i) {
-        const int vi = lane + 32 * i;
-        if (vi < p.q_vecs) {
-            uint4 g[KG];
-            ld_gamma_vec<E>(rp.gamma_q, vi, p.q_vecs, 0, g);
-            st_stream(qo + static_cast<int64_t>(vi) * 16, scale_vec<E>(row.xq[i], g, rq));
-        }
-    }
-#pragma unroll
-    for (int i = 0; i < NVK; ++i) {
-        const int vi = lane + 32 * i;
-        if (vi < p.k_vecs) {
-            uint4 g[KG];
-            ld_gamma_vec<E>(rp.gamma_k, vi, p.k_vecs, 0, g);
-            st_stream(ko + static_cast<int64_t>(vi) * 16, scale_vec<E>(row.xk[i], g, rk));
-        }
-    }
+    const float rq = rms_factor(Aq, p.inv_hq, p.eps), rk = rms_factor(Ak, p.inv_hk, p.eps);
+    tp_scale_row<E, NVQ, BQ>(qrow, rp.q_out + t * p.q_stride_bytes, rp.gamma_q, p.q_vecs, lane, f2(rq, rq), xq);
+    tp_scale_row<E, NVK, BK>(krow, rp.k_out + t * p.k_stride_bytes, rp.gamma_k, p.k_vecs, lane, f2(rk, rk), xk);
 }
 
 // Warp w of block c takes tokens s, s + step, s + 2 step, ... (s = c * 4 + w,
 // step = G * 4) and publishes kTpAhead tokens ahead of the one it finishes:
-// iteration k loads token k (kept in L2), publishes its partial sums, then
+// iteration k reads token k (kept in L2) and publishes its partial sums, then
 // re-reads token k - kTpAhead (an L2 hit, read kTpAhead tokens earlier),
 // waits for that token's exchange (by now mostly complete) and stores it.
-// No row is held across a wait on the exchange, so the warp's registers stay
-// those of one row.  Every rank's warp (c, w) has the same sequence and
-// publishes a token before it waits on it, so no wait depends on a warp that
-// waits on it.
+// No row is held across a wait on the exchange beyond one batch.  Every
+// rank's warp (c, w) has the same sequence and publishes a token before it
+// waits on it, so no wait depends on a warp that waits on it.
 template <typename E, int NVQ, int NVK, bool SYS>
 __global__ void __launch_bounds__(32 * kTpWarps, tp_warp_min_blocks<NVQ, NVK>())
     tp_warp_kernel(const __grid_constant__ TpParams p) {
@@ -346,16 +360,8 @@ __global__ void __launch_bounds__(32 * kTpWarps, tp_warp_min_blocks<NVQ, NVK>())
     const int64_t first = static_cast<int64_t>(c) * kTpWarps + warp;
     const int64_t n = first < p.T ? (p.T - 1 - first) / step + 1 : 0;  // tokens of this warp
     for (int64_t k = 0; k < n + kTpAhead; ++k) {
-        if (k < n) {
-            TpRow<E, NVQ, NVK> row;
-            tp_load<E, NVQ, NVK, true>(p, rp, first + k * step, lane, row);
-            tp_publish<E, NVQ, NVK, SYS>(p, rank, first + k * step, lane, row);
-        }
-        if (k >= kTpAhead) {
-            TpRow<E, NVQ, NVK> row;
-            tp_load<E, NVQ, NVK>(p, rp, first + (k - kTpAhead) * step, lane, row);
-            tp_finish<E, NVQ, NVK, SYS>(p, rp, rank, first + (k - kTpAhead) * step, lane, row);
-        }
+        if (k < n) tp_publish<E, NVQ, NVK, SYS>(p, rp, rank, first + k * step, lane);
+        if (k >= kTpAhead) tp_finish<E, NVQ, NVK, SYS>(p, rp, rank, first + (k - kTpAhead) * step, lane);
     }
 }
 
