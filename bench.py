@@ -129,6 +129,7 @@ def load_peaks() -> dict:
 KERNEL_SOURCES = {
     "rows": ["qknorm_kernels.cuh"],
     "projection": ["qkv_gemm.cu", "qkv_gemm.cuh"],
+    "tp": ["qknorm_tp.cu", "qknorm_tp.cuh", "qknorm_kernels.cuh"],
 }
 
 
@@ -161,6 +162,13 @@ def profiled_traffic(workload: str, digest: str, launch: str | None = None):
             continue
         return int(m_t.group(1))
     return None
+
+
+def tp_warp_form(wl) -> bool:
+    """Whether the tensor-parallel call runs one token per warp: shard rows of
+    at most 256 16-byte vectors (the library's own rule)."""
+    b = wl.batch
+    return max(b.Hq, b.Hk) // wl.ranks * wl.esz // 16 <= 256
 
 
 def launch_text(plan) -> str | None:
@@ -271,7 +279,7 @@ class Workload:
         # bytes the method must move per step: read + write of every Q and K element, plus gamma
         gamma_elems = 2 * b.meta["head_dim"] if kind == "headwise" else b.Hq + b.Hk
         self.eff_bytes = 2 * self.esz * (b.Hq + b.Hk) * b.T + gesz * gamma_elems
-        self.name = b.name
+        self.name = f"tp_R{ranks}_{b.name}" if kind == "tp" else b.name
         self.launches_per_step = 2 * b.P if kind == "gqa" else 1
 
     def config(self) -> dict:
@@ -593,7 +601,7 @@ def native(args) -> int:
     value = agg["value_gbs"]
     per_rank_gbs = agg["per_rank_gbs"]
     peaks = load_peaks()
-    digest = source_digest()
+    digest = source_digest("tp" if wl.kind == "tp" else "rows")
     kernel_s = step_s / wl.launches_per_step if wl.kind != "gqa" else step_s
     plan = None
     if wl.kind in ("prefill", "tiny", "decode", "packed"):
@@ -608,7 +616,9 @@ def native(args) -> int:
                 "traffic": profiled_traffic(wl.name, digest, launch_text(plan)),
                 "peak_source": f"{peaks['source']} copy bandwidth",
                 "kernel": {"gqa": "whole step: partial_stats x P + combine_apply x P",
-                           "tp": "tp_rows_kernel, all ranks in one launch (the only kernel of the step)"}.get(
+                           "tp": ("tp_warp_kernel (one token per warp)" if tp_warp_form(wl) else
+                                  "tp_rows_kernel (one token per block)")
+                           + ", all ranks in one launch (the only kernel of the step)"}.get(
                                wl.kind, "qknorm rows kernel (the only kernel of the step)"),
                 "algorithmic_bytes_per_launch": wl.eff_bytes if wl.kind != "gqa" else None,
                 "source_digest": digest}
