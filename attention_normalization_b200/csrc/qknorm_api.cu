@@ -1085,21 +1085,17 @@ qkn_status qknorm_tp_layerwise(int32_t R, int32_t first_rank, int32_t n_local, c
                 for (const Region &t : theirs)
                     if (overlap(o, t)) return fail(QKN_ERR_INVALID_ARG, "rank %d's output overlaps rank %d's rows", j, jj);
         }
-    // launch shape: one block per token at a time, NV vectors per thread
+    // launch shape: one token per warp, four warps per block; rows of up to 8
+    // vectors per lane unrolled, wider ones in a batch loop
     const int64_t vq = hq_shard / per_vec, vk = hk_shard / per_vec, vmax = vq > vk ? vq : vk;
-    int nv, threads;
-    int64_t tokens_per_block = 1;
-    if (vmax <= 256) {  // one token per warp, four warps per block
+    int nv = 0;
+    const int threads = 128;
+    const int64_t tokens_per_block = 4;
+    if (vmax <= 256) {
         auto lanes_nv = [](int64_t v) { return v <= 32 ? 1 : (v <= 64 ? 2 : (v <= 128 ? 4 : 8)); };
         int nvq = lanes_nv(vq), nvk = lanes_nv(vk);
         if (nvk > nvq) nvq = nvk;  // instantiated with NVK <= NVQ
         nv = -(8 * nvq + nvk);
-        threads = 128;
-        tokens_per_block = 4;
-    } else {
-        nv = vmax <= 512 ? 2 : 4;
-        threads = (int)(((vmax + nv - 1) / nv + 31) / 32 * 32);
-        if (threads > 256) return fail(QKN_ERR_UNSUPPORTED, "shard rows above 1024 vectors");
     }
     int dev = 0, sms = 0, bps = 0;
     qkn_status st = current_device(&dev);

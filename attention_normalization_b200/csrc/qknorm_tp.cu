@@ -89,139 +89,19 @@ __device__ __forceinline__ bool wait_pair(const unsigned long long *src, uint32_
     return true;
 }
 
-// x * gamma for one vector, kept in fp32 pairs until the factor is known.
-template <typename E>
-__device__ __forceinline__ void mul_gamma(const uint4 &xv, const uint4 (&gv)[Elem<E>::kGVecs],
-                                          F2 (&u)[Elem<E>::kPerVec / 2]) {
-    using GT = typename Elem<E>::G;
-    constexpr int KG = Elem<GT>::kPerVec / 2;
-    Elem<E>::widen(xv, u);
-#pragma unroll
-    for (int j = 0; j < Elem<E>::kGVecs; ++j) {
-        F2 part[KG];
-        Elem<GT>::widen(gv[j], part);
-#pragma unroll
-        for (int k = 0; k < KG; ++k) u[j * KG + k] = mul2(u[j * KG + k], part[k]);
-    }
-}
-
-template <typename E>
-__device__ __forceinline__ uint4 times_r(const F2 (&u)[Elem<E>::kPerVec / 2], F2 r2) {
-    constexpr int K = Elem<E>::kPerVec / 2;
-    F2 y[K];
-#pragma unroll
-    for (int j = 0; j < K; ++j) y[j] = mul2(u[j], r2);
-    return Elem<E>::narrow(y);
-}
-
 }  // namespace
 
-// One block handles one token at a time: the rank's Q shard row and K shard
-// row, thread i holding 16-byte vectors i, i + blockDim, ... of each.
-constexpr int kTpMaxThreads = 256;
-
-template <typename E, int NV, bool SYS>
-__global__ void __launch_bounds__(kTpMaxThreads) tp_rows_kernel(const __grid_constant__ TpParams p) {
-    constexpr int KG = Elem<E>::kGVecs;
-    constexpr int K2 = Elem<E>::kPerVec / 2;
-    __shared__ float red[2][2][32];  // [slot][tensor][warp]
-    __shared__ float s_r[2];         // the token's factors (Q, K)
-    __shared__ int s_ok;
-    pdl_wait_and_release();
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
-    const int local = blockIdx.x / p.blocks_per_rank;
-    const int c = blockIdx.x - local * p.blocks_per_rank;
-    const int rank = p.first_rank + local;
-    const RankPtrs rp = p.local[local];
-
-    uint4 gq[NV][KG], gk[NV][KG];  // this rank's gamma slices, for the whole launch
-#pragma unroll
-    for (int i = 0; i < NV; ++i) {
-        ld_gamma_vec<E>(rp.gamma_q, tid + i * blockDim.x, p.q_vecs, 0, gq[i]);
-        ld_gamma_vec<E>(rp.gamma_k, tid + i * blockDim.x, p.k_vecs, 0, gk[i]);
-    }
-    int slot = 0;
-    for (int64_t t = c; t < p.T; t += p.blocks_per_rank) {
-        const char *qrow = rp.q_in + t * p.q_stride_bytes;
-        const char *krow = rp.k_in + t * p.k_stride_bytes;
-        uint4 xq[NV], xk[NV];
-#pragma unroll
-        for (int i = 0; i < NV; ++i) {
-            const int vi = tid + i * blockDim.x;
-            xq[i] = vi < p.q_vecs ? ld_stream(qrow + static_cast<int64_t>(vi) * 16) : make_uint4(0u, 0u, 0u, 0u);
-            xk[i] = vi < p.k_vecs ? ld_stream(krow + static_cast<int64_t>(vi) * 16) : make_uint4(0u, 0u, 0u, 0u);
-        }
-        // Phase A, local step: the shard's squared sums (fixed order: warp
-        // butterfly, then warps 0, 1, ...).
-        float sq = warp_sum(sumsq_pairs<E, NV>(xq));
-        float sk = warp_sum(sumsq_pairs<E, NV>(xk));
-        if (lane == 0) {
-            red[slot][0][warp] = sq;
-            red[slot][1][warp] = sk;
-        }
-        __syncthreads();
-        float Sq = 0.0f, Sk = 0.0f;
-        for (int w = 0; w < nwarps; ++w) {
-            Sq += red[slot][0][w];
-            Sk += red[slot][1][w];
-        }
-        slot ^= 1;
-
-        if (warp == 0) {
-            // Exchange: lane i writes this rank's partials into rank i's
-            // buffer, then waits for rank i's partials in this rank's buffer.
-            float vq = 0.0f, vk = 0.0f;
-            bool ok = true;
-            if (lane < p.R) {
-                publish_pair<SYS>(p.recv[lane] + (static_cast<int64_t>(rank) * p.T + t) * 2, p.epoch, Sq, Sk);
-                ok = wait_pair<SYS>(p.recv[rank] + (static_cast<int64_t>(lane) * p.T + t) * 2, p.epoch,
-                                    p.timeout_ns, vq, vk);
-            }
-            ok = __all_sync(0xFFFFFFFFu, ok);
-            // Phase A aggregation: the R partials added in rank order, fp32.
-            float Aq = 0.0f, Ak = 0.0f;
-            for (int i = 0; i < p.R; ++i) {
-                Aq += __shfl_sync(0xFFFFFFFFu, vq, i);
-                Ak += __shfl_sync(0xFFFFFFFFu, vk, i);
-            }
-            if (lane == 0) {
-                s_r[0] = rms_factor(Aq, p.inv_hq, p.eps);
-                s_r[1] = rms_factor(Ak, p.inv_hk, p.eps);
-                s_ok = ok;
-            }
-        }
-        // Phase B: x * gamma does not depend on the reduction (the other
-        // warps form it while warp 0 waits).
-        F2 uq[NV][K2], uk[NV][K2];
-#pragma unroll
-        for (int i = 0; i < NV; ++i) {
-            mul_gamma<E>(xq[i], gq[i], uq[i]);
-            mul_gamma<E>(xk[i], gk[i], uk[i]);
-        }
-        __syncthreads();
-        if (!s_ok) continue;  // a wait gave up: this token is left unwritten (the timeout is reported)
-        const F2 rq = f2(s_r[0], s_r[0]), rk = f2(s_r[1], s_r[1]);
-        char *qo = rp.q_out + t * p.q_stride_bytes;
-        char *ko = rp.k_out + t * p.k_stride_bytes;
-#pragma unroll
-        for (int i = 0; i < NV; ++i) {
-            const int vi = tid + i * blockDim.x;
-            if (vi < p.q_vecs) st_stream(qo + static_cast<int64_t>(vi) * 16, times_r<E>(uq[i], rq));
-            if (vi < p.k_vecs) st_stream(ko + static_cast<int64_t>(vi) * 16, times_r<E>(uk[i], rk));
-        }
-    }
-}
-
-// Narrow shard rows (at most 32 * NVQ vectors of Q, 32 * NVK of K): one warp
-// per token, kTpWarps warps per block, no block barrier.  Warp w of block b
-// of a rank takes tokens (b * kTpWarps + w), + G * kTpWarps, ...; lane i
-// exchanges with rank i as in the block form, every lane gets the sums by
-// shuffles, and the warp then scales its row as (x * gamma) * r (the same
-// products as the block form).  The exchange is a round trip through memory,
-// so throughput comes from the number of tokens in flight: a warp passes its
-// row through registers in batches (gamma re-read from L1 when the row is
-// scaled) and publishes ahead, and the register cap below fits as many warps
-// on an SM as one batch's registers allow.
+// One warp per token, kTpWarps warps per block, no block barrier.  Warp w of
+// block c of a rank takes tokens (c * kTpWarps + w), + G * kTpWarps, ...;
+// lane i exchanges with rank i, every lane gets the sums by shuffles, and
+// the warp scales its row as (x * gamma) * r.  The exchange is a round trip
+// through memory, so throughput comes from the number of tokens in flight: a
+// warp passes its row through registers in batches of at most kTpBatch
+// 16-byte vectors per lane (gamma re-read from L1 when the row is scaled)
+// and publishes ahead, and the register cap below fits as many warps on an
+// SM as one batch's registers allow.  Shard rows of up to 8 vectors per lane
+// (NVQ for Q, NVK <= NVQ for K) run fully unrolled; wider rows take the
+// kTpWide instantiation, whose batch loop runs over the row at run time.
 constexpr int kTpWarps = 4;
 
 #ifndef QKN_TP_AHEAD
@@ -239,11 +119,13 @@ constexpr int kTpBatch = QKN_TP_BATCH;
 #ifndef QKN_TP_REGS_PER_VEC
 #define QKN_TP_REGS_PER_VEC 4
 #endif
+constexpr int kTpWide = 0;  // NVQ = NVK = kTpWide: any width, batches of kTpBatch
+
 template <int NVQ, int NVK>
 constexpr int tp_warp_min_blocks() {
     // registers per 16-byte vector held (a batch of Q or K vectors, NVK <=
     // NVQ, and their gamma vectors), plus ~40 for the rest
-    constexpr int held = 2 * (NVQ < kTpBatch ? NVQ : kTpBatch);
+    constexpr int held = 2 * (NVQ == kTpWide || NVQ > kTpBatch ? kTpBatch : NVQ);
     constexpr int regs = QKN_TP_REGS_PER_VEC * held + 40;
     return 65536 / (32 * kTpWarps * regs) < 16 ? 65536 / (32 * kTpWarps * regs) : 16;
 }
@@ -272,18 +154,20 @@ __device__ __forceinline__ void tp_load_batch(const char *row, int nvecs, int la
 // i to rank i).
 template <typename E, int NVQ, int NVK, bool SYS>
 __device__ __forceinline__ void tp_publish(const TpParams &p, const RankPtrs &rp, int rank, int64_t t, int lane) {
-    constexpr int BQ = NVQ < kTpBatch ? NVQ : kTpBatch;
-    constexpr int BK = NVK < kTpBatch ? NVK : kTpBatch;
+    constexpr int BQ = NVQ == kTpWide || NVQ > kTpBatch ? kTpBatch : NVQ;
+    constexpr int BK = NVK == kTpWide || NVK > kTpBatch ? kTpBatch : NVK;
     const char *qrow = rp.q_in + t * p.q_stride_bytes;
     const char *krow = rp.k_in + t * p.k_stride_bytes;
+    // vectors per lane of the wider row (Q; either for the wide form)
+    const int nq = NVQ != kTpWide ? NVQ : ((p.q_vecs > p.k_vecs ? p.q_vecs : p.k_vecs) + 31) >> 5;
     float sq = 0.0f, sk = 0.0f;
 #pragma unroll
-    for (int b = 0; b < NVQ; b += BQ) {  // NVK <= NVQ
+    for (int b = 0; b < nq; b += BQ) {  // NVK <= NVQ
         uint4 xq[BQ], xk[BK];
         tp_load_batch<NVQ, true, BQ>(qrow, p.q_vecs, lane, b, xq);
-        if (b < NVK) tp_load_batch<NVK, true, BK>(krow, p.k_vecs, lane, b, xk);
+        if (NVK == kTpWide || b < NVK) tp_load_batch<NVK, true, BK>(krow, p.k_vecs, lane, b, xk);
         sq += sumsq_pairs<E, BQ>(xq);
-        if (b < NVK) sk += sumsq_pairs<E, BK>(xk);
+        if (NVK == kTpWide || b < NVK) sk += sumsq_pairs<E, BK>(xk);
     }
     sq = warp_sum(sq);
     sk = warp_sum(sk);
@@ -296,8 +180,9 @@ template <typename E, int NV, int B>
 __device__ __forceinline__ void tp_scale_row(const char *in, char *out, const char *gamma, int nvecs, int lane,
                                              F2 r, uint4 (&x)[B]) {
     constexpr int KG = Elem<E>::kGVecs;
+    const int nv = NV != kTpWide ? NV : (nvecs + 31) >> 5;
 #pragma unroll
-    for (int b = 0; b < NV; b += B) {
+    for (int b = 0; b < nv; b += B) {
         if (b > 0) tp_load_batch<NV, false, B>(in, nvecs, lane, b, x);
 #pragma unroll
         for (int i = 0; i < B; ++i) {
@@ -317,8 +202,8 @@ __device__ __forceinline__ void tp_scale_row(const char *in, char *out, const ch
 // (the timeout is reported).
 template <typename E, int NVQ, int NVK, bool SYS>
 __device__ __forceinline__ void tp_finish(const TpParams &p, const RankPtrs &rp, int rank, int64_t t, int lane) {
-    constexpr int BQ = NVQ < kTpBatch ? NVQ : kTpBatch;
-    constexpr int BK = NVK < kTpBatch ? NVK : kTpBatch;
+    constexpr int BQ = NVQ == kTpWide || NVQ > kTpBatch ? kTpBatch : NVQ;
+    constexpr int BK = NVK == kTpWide || NVK > kTpBatch ? kTpBatch : NVK;
     const char *qrow = rp.q_in + t * p.q_stride_bytes;
     const char *krow = rp.k_in + t * p.k_stride_bytes;
     uint4 xq[BQ], xk[BK];
@@ -367,15 +252,13 @@ __global__ void __launch_bounds__(32 * kTpWarps, tp_warp_min_blocks<NVQ, NVK>())
 
 namespace {
 
-// nv > 0: the block-per-token kernel with nv vectors per thread; nv < 0: the
-// warp-per-token kernel with NVQ and NVK vectors per lane, nv = -(8 NVQ + NVK).
+// nv < 0: the warp kernel with NVQ and NVK vectors per lane, nv = -(8 NVQ +
+// NVK); nv == 0: the warp kernel for rows of any width.
 template <typename E, bool SYS>
 const void *tp_kernel(int nv) {
     switch (nv) {
-        case 1: return (const void *)tp_rows_kernel<E, 1, SYS>;
-        case 2: return (const void *)tp_rows_kernel<E, 2, SYS>;
-        case 4: return (const void *)tp_rows_kernel<E, 4, SYS>;
-        // warp form: nv = -(8 * NVQ + NVK), NVK <= NVQ (wider K rows take NVQ = NVK)
+        case 0: return (const void *)tp_warp_kernel<E, kTpWide, kTpWide, SYS>;
+        // nv = -(8 * NVQ + NVK), NVK <= NVQ (wider K rows take NVQ = NVK)
         case -(8 * 1 + 1): return (const void *)tp_warp_kernel<E, 1, 1, SYS>;
         case -(8 * 2 + 1): return (const void *)tp_warp_kernel<E, 2, 1, SYS>;
         case -(8 * 2 + 2): return (const void *)tp_warp_kernel<E, 2, 2, SYS>;

@@ -8,15 +8,13 @@
 //     partial sums (fp32) to get the global sums -- a scalar per token and
 //     tensor crosses between ranks instead of the activations.
 //   Phase B: the shard times gamma is scaled by the global factor and only
-//     the final values are stored.  For shard rows above 256 vectors warp 0
-//     carries the exchange (it writes this rank's partials into every rank's
-//     receive buffer and waits for the others') while the other warps
-//     multiply the shard by gamma, which does not depend on the reduction;
-//     narrower rows run one token per warp (four per block, no block
-//     barrier), the multiply after the wait.  There a warp publishes two
-//     tokens ahead of the one it finishes and re-reads that one's row from
-//     L2, so its exchange is mostly complete when the warp waits on it and no
-//     row is held across a wait.
+//     the final values are stored.  The pages overlap the exchange with the
+//     gamma multiply (warp 0 exchanges while the other warps multiply); here
+//     one warp carries a token (four per block, no block barrier) and the
+//     overlap is deeper: a warp publishes two tokens ahead of the one it
+//     finishes and re-reads that one's rows from L2, so its exchange is
+//     mostly complete when the warp waits on it, and no row is held across a
+//     wait (rows pass through registers in batches, so any shard width fits).
 //   Deadlock-safe persistent execution: the grid is bounded by the resident
 //     blocks and each block loops over tokens.
 //
@@ -79,11 +77,10 @@ struct TpParams {
 };
 
 // Host side (qknorm_tp.cu): launch `p` on `stream` with `threads` threads per
-// block for element type `dtype` (1 = bf16, 2 = fp16, 0 = fp32, 3 = E4M3);
-// nv > 0 selects the block-per-token kernel with nv vectors per thread, nv < 0
-// the warp-per-token kernel (128-thread blocks of 4 warps) with NVQ vectors
-// per lane for Q and NVK for K, nv = -(8 NVQ + NVK).  Cooperative when
-// n_local > 1.
+// block (128: four warps, one token each) for element type `dtype` (1 = bf16,
+// 2 = fp16, 0 = fp32, 3 = E4M3); nv < 0 selects the kernel with NVQ vectors
+// per lane for Q and NVK for K, nv = -(8 NVQ + NVK), nv == 0 the kernel for
+// rows of any width.  Cooperative when n_local > 1.
 cudaError_t launch_tp(const TpParams &p, int dtype, int nv, int threads, cudaStream_t stream, const char **what);
 
 // Blocks of the kernel for (dtype, nv, threads) resident per SM; all_local

@@ -164,13 +164,6 @@ def profiled_traffic(workload: str, digest: str, launch: str | None = None):
     return None
 
 
-def tp_warp_form(wl) -> bool:
-    """Whether the tensor-parallel call runs one token per warp: shard rows of
-    at most 256 16-byte vectors (the library's own rule)."""
-    b = wl.batch
-    return max(b.Hq, b.Hk) // wl.ranks * wl.esz // 16 <= 256
-
-
 def launch_text(plan) -> str | None:
     """A launch plan as the profile summaries record it."""
     if not plan:
@@ -616,9 +609,8 @@ def native(args) -> int:
                 "traffic": profiled_traffic(wl.name, digest, launch_text(plan)),
                 "peak_source": f"{peaks['source']} copy bandwidth",
                 "kernel": {"gqa": "whole step: partial_stats x P + combine_apply x P",
-                           "tp": ("tp_warp_kernel (one token per warp)" if tp_warp_form(wl) else
-                                  "tp_rows_kernel (one token per block)")
-                           + ", all ranks in one launch (the only kernel of the step)"}.get(
+                           "tp": "tp_warp_kernel (one token per warp), all ranks in one launch "
+                                 "(the only kernel of the step)"}.get(
                                wl.kind, "qknorm rows kernel (the only kernel of the step)"),
                 "algorithmic_bytes_per_launch": wl.eff_bytes if wl.kind != "gqa" else None,
                 "source_digest": digest}

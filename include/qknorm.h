@@ -234,18 +234,18 @@ int64_t qknorm_qkv_projection_noalloc_max_bytes(void);
  * Tensor-parallel layerwise QK-Norm: the paper's multi-GPU kernel (Phase A:
  * each rank squares and sums its hidden-dimension shard and the ranks add
  * their scalar partial sums in fp32; Phase B: the global factor scales the
- * shard times gamma -- for shard rows above 256 vectors warp 0 of each block
- * carries the exchange while the other warps multiply the shard by gamma,
- * narrower rows run one token per warp; deadlock-safe persistent blocks).
+ * shard times gamma; deadlock-safe persistent blocks).  One warp carries a
+ * token, publishing two tokens ahead of the one it finishes so that the
+ * exchange overlaps the loads of later tokens.
  *   R ranks each hold a shard of every token's Q row (hq_shard columns of
  *   Hq_full) and K row (hk_shard of Hk_full).  This call runs the n_local
  *   ranks first_rank .. first_rank + n_local - 1; local rank j's rows are
  *   q_in[j] / q_out[j] ([T rows, stride q_stride]), gamma slice gamma_q[j]
  *   [hq_shard], and likewise for K.  out == in normalizes in place.
  *   recv[r] (r < R) is rank r's receive buffer, qknorm_tp_recv_bytes(R, T)
- *   bytes, 16-byte aligned: a device pointer valid on this GPU -- its own memory for local
- *   ranks, a peer mapping (cudaIpcOpenMemHandle or similar) for ranks on other
- *   GPUs.  Buffers start zeroed; each call on the same buffers passes a new
+ *   bytes, 16-byte aligned: a device pointer valid on this GPU -- its own
+ *   memory for local ranks, a peer mapping (cudaIpcOpenMemHandle or similar)
+ *   for ranks on other GPUs.  Buffers start zeroed; each call on the same buffers passes a new
  *   epoch (> 0), and all ranks of one call pass the same epoch.
  *   Result: y = (x * gamma) * r with r = 1 / sqrt(S / H_full + eps) and S the
  *   ranks' partial sums added in rank order 0 .. R-1, identical on every rank.
@@ -258,8 +258,8 @@ int64_t qknorm_qkv_projection_noalloc_max_bytes(void);
  * the tokens concerned are left unwritten.
  * Requirements: 1 <= R <= 8, n_local <= 8; dtype any of qkn_dtype; 16-byte
  * aligned buffers and shard widths / strides that are whole 16-byte vectors
- * (else QKN_ERR_UNSUPPORTED); shard rows of at most 1024 vectors.  T = 0 is a
- * no-op.  Asynchronous on `stream`; allocates nothing.
+ * (else QKN_ERR_UNSUPPORTED).  T = 0 is a no-op.  Asynchronous on `stream`;
+ * allocates nothing.
  */
 int64_t qknorm_tp_recv_bytes(int32_t R, int64_t T);
 qkn_status qknorm_tp_layerwise(int32_t R, int32_t first_rank, int32_t n_local, const void *const *q_in,

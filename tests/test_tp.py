@@ -66,6 +66,19 @@ def test_tp_matches_the_full_row_oracle(R, dtype):
     assert qk.device_timeouts() == 0
 
 
+@pytest.mark.parametrize("R,Hq,Hk,dtype", [
+    (1, 16384, 2048, torch.bfloat16),   # 2048 + 256 vectors per shard row: 64 per lane, in 16 batches
+    (2, 8192, 1024, torch.float32),     # 2048 + 256 vectors per shard row
+    (4, 5120, 1024, torch.float8_e4m3fn),
+])
+def test_tp_wide_shards(R, Hq, Hk, dtype):
+    """Shard rows of any width pass through a warp in batches."""
+    b = _batch(67, Hq, Hk, dtype, seed=40 + R)
+    q, k = run_tp(b, R)
+    check_full(b, q, k)
+    assert qk.device_timeouts() == 0
+
+
 def test_tp_prefill_full_size():
     """The prefill batch (T=4096, Hq=Hk=4096 bf16) split over 4 ranks."""
     b = workloads.prefill_bf16()
