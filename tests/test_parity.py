@@ -226,6 +226,24 @@ def test_rows_too_wide_for_registers(dtype, H):
     check_layerwise(b)
 
 
+def test_prefill_rows_beyond_2gib():
+    """Q and K of 2.16 GB each (T = 2^31 / 8192 + 1000 rows of 4096 bf16):
+    rows on both sides of the 2^31-byte offset, and the first and last rows,
+    against the oracle (64-bit row offsets in every address)."""
+    T = (1 << 31) // (4096 * 2) + 1000
+    b = workloads.large_rows_on_device(T, 4096, 4096, torch.bfloat16, seed=77, device=DEV)
+    gq, gk = b.gamma_q.to(DEV), b.gamma_k.to(DEV)
+    qo, ko = qk.qknorm_layerwise(b.q, b.k, gq, gk, b.eps)
+    torch.cuda.synchronize()
+    edge = (1 << 31) // (4096 * 2)
+    rows = torch.tensor([0, 1, edge - 1, edge, edge + 1, T // 2, T - 2, T - 1], device=DEV)
+    for x, out, g, name in ((b.q, qo, b.gamma_q, "Q"), (b.k, ko, b.gamma_k, "K")):
+        y, e, _ = oracle_rows(x[rows].cpu(), g, b.eps)
+        assert_close(out[rows].cpu(), y, e, f"{b.name} {name}")
+    del qo, ko, b
+    torch.cuda.empty_cache()
+
+
 def test_zero_rows_give_zero_and_empty_batch_is_a_no_op():
     b = workloads.random_rows(4, 64, 32, torch.bfloat16, seed=6)
     b.q[1].zero_()

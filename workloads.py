@@ -270,6 +270,19 @@ def random_rows(T: int, Hq: int, Hk: int, dtype: torch.dtype, seed: int,
                    meta={"q_buffer": qb, "k_buffer": kb})
 
 
+def large_rows_on_device(T: int, Hq: int, Hk: int, dtype: torch.dtype, seed: int, device) -> QKBatch:
+    """Q and K batches too large to build on the host (several GB), drawn on
+    the device: x ~ N(0, 1) from a CUDA generator seeded with ``seed`` (Q
+    first, then K), rounded once to ``dtype``; gamma as elsewhere, on the
+    host.  The oracle reads back the rows it checks."""
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed))
+    q = torch.randn((T, Hq), generator=g, dtype=torch.float32, device=device).to(dtype)
+    k = torch.randn((T, Hk), generator=g, dtype=torch.float32, device=device).to(dtype)
+    return QKBatch(f"large_T{T}_Hq{Hq}_Hk{Hk}", dtype, T, Hq, Hk, q, k,
+                   gamma(Hq, seed + 100, dtype), gamma(Hk, seed + 200, dtype))
+
+
 def effective_bytes(T: int, Hq: int, Hk: int, esz: int) -> int:
     """Bytes a layerwise QK-Norm call must move: read + write of every Q and K
     element, plus one read of gamma_q and gamma_k."""
