@@ -25,7 +25,7 @@ from . import _clib
 from ._clib import QknLaunch, QKNormError
 
 __all__ = ["qknorm_layerwise", "qknorm_headwise", "qknorm_qkv_gemm_stats", "qknorm_qkv_projection",
-           "qkv_workspace_bytes", "device_timeouts", "qknorm_tp_layerwise", "TpExchange", "qknorm_partial_stats", "qknorm_combine_apply", "gamma_dtype",
+           "qkv_workspace_bytes", "device_timeouts", "qknorm_tp_layerwise", "TpExchange", "TpPeerExchange", "qknorm_partial_stats", "qknorm_combine_apply", "gamma_dtype",
            "qknorm_layerwise_plan", "qknorm_layerwise_host", "qknorm_packed_host",
            "plan_shape", "plan_grid", "regions_overlap", "capi", "version", "QknLaunch", "QKNormError"]
 
@@ -289,15 +289,21 @@ class TpExchange:
         return self.epoch
 
 
+from .tp_peer import TpPeerExchange  # noqa: E402  (one rank per GPU: receive buffers over CUDA IPC)
+
+
 def qknorm_tp_layerwise(q_shards, k_shards, gamma_q_shards, gamma_k_shards, Hq_full: int, Hk_full: int,
-                        eps: float = 1e-6, *, exchange: TpExchange | None = None, recv=None, epoch: int | None = None,
+                        eps: float = 1e-6, *, exchange: TpExchange | TpPeerExchange | None = None, recv=None,
+                        epoch: int | None = None,
                         R: int | None = None, first_rank: int = 0, q_out=None, k_out=None, in_place: bool = False,
                         blocks_per_rank: int = 0, timeout_ns: int = 0, stream=None):
     """Tensor-parallel layerwise QK-Norm: runs ranks first_rank ..
     first_rank + len(q_shards) - 1 of an R-rank group; shard j holds Q columns
     of rank first_rank + j for all T tokens.  The ranks exchange only their
-    scalar partial sums (through ``exchange`` / ``recv``).  Returns the lists
-    ``(q_out, k_out)``."""
+    scalar partial sums (through ``exchange`` / ``recv``): a ``TpExchange``
+    when every rank runs in this call on this GPU, a ``TpPeerExchange`` when
+    each process runs its own rank on its own GPU (pass ``first_rank`` = that
+    rank and one shard).  Returns the lists ``(q_out, k_out)``."""
     n_local = len(q_shards)
     if not (n_local == len(k_shards) == len(gamma_q_shards) == len(gamma_k_shards)) or n_local < 1:
         raise ValueError("one Q shard, K shard and gamma slice each per local rank")

@@ -84,3 +84,102 @@ def test_reference_arm_line_on_rank_zero():
     assert d["impl"] == "reference" and d["unit"] == "GB/s" and d["value"] > 0
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] == 1
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
+
+
+# --------------------------------------------------------------------------- one rank per GPU: receive buffers
+
+class FakeIpc:
+    """Stands in for CUDA IPC on CPU: a rank's buffer is a made-up address, a
+    handle names the exporting address, and opening maps it to an address of
+    its own; every call is recorded."""
+
+    def __init__(self, rank):
+        self.rank = rank
+        self.log = []
+
+    def alloc_zeroed(self, nbytes):
+        self.log.append(("alloc", nbytes))
+        return 0x10000000 * (self.rank + 1)
+
+    def free(self, ptr):
+        self.log.append(("free", ptr))
+
+    def export(self, ptr):
+        self.log.append(("export", ptr))
+        return ptr.to_bytes(8, "little") + bytes(56)
+
+    def open(self, handle):
+        ptr = int.from_bytes(handle[:8], "little")
+        self.log.append(("open", ptr))
+        return ptr + 0x700000000000
+
+    def close(self, ptr):
+        self.log.append(("close", ptr))
+
+
+def _peer_worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        from attention_normalization_b200.tp_peer import TpPeerExchange
+        ipc = FakeIpc(rank)
+        ex = TpPeerExchange(world, 4096, ipc=ipc)
+        ptrs = ex.pointers()
+        epochs = [ex.next_epoch(), ex.next_epoch()]
+        ex.close()
+        out.put((rank, ptrs, epochs, ipc.log))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_peer_exchange_handles_gloo():
+    """Each rank allocates and exports its buffer, opens every other rank's
+    handle in rank order, keeps its own at its rank; epochs step from 1 on
+    every rank; close unmaps the peers and frees its own buffer."""
+    world, port = 3, _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_peer_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    got = sorted(q.get(timeout=120) for _ in range(world))
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    own = [0x10000000 * (r + 1) for r in range(world)]
+    for rank, ptrs, epochs, log in got:
+        assert epochs == [1, 2]
+        assert ptrs == [own[r] if r == rank else own[r] + 0x700000000000 for r in range(world)]
+        assert log[0] == ("alloc", world * 4096 * 16) and log[1] == ("export", own[rank])
+        assert [e for e in log if e[0] == "open"] == [("open", own[r]) for r in range(world) if r != rank]
+        assert [e for e in log if e[0] == "close"] == [("close", own[r] + 0x700000000000)
+                                                      for r in range(world) if r != rank]
+        assert log[-1] == ("free", own[rank])
+
+
+def _peer_bad_worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        from attention_normalization_b200.tp_peer import TpPeerExchange
+        try:
+            TpPeerExchange(world + 1, 16, ipc=FakeIpc(rank))
+            out.put((rank, "accepted"))
+        except ValueError as e:
+            out.put((rank, str(e)))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_peer_exchange_rejects_a_group_of_another_size_gloo():
+    world, port = 2, _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_peer_bad_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    got = [q.get(timeout=120) for _ in range(world)]
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    assert all("R = 3" in msg for _, msg in got)
