@@ -125,3 +125,30 @@ def test_tp_missing_rank_times_out_and_the_context_stays_usable():
     q, k = run_tp(b, R, ex)
     check_full(b, q, k)
     assert qk.device_timeouts() == 0
+
+
+def test_peer_exchange_single_rank_on_the_gpu():
+    """TpPeerExchange's CUDA side on one GPU: a one-rank group allocates,
+    zeroes and exports its receive buffer through the runtime's IPC calls, and
+    a call through it normalizes like the oracle.  (Groups of several ranks
+    need one GPU each.)"""
+    import socket
+
+    import torch.distributed as dist
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1)
+    try:
+        b = _batch(64, 1024, 512, torch.bfloat16, seed=31)
+        ex = qk.TpPeerExchange(1, b.T)
+        assert len(ex.pointers()) == 1
+        q, k = run_tp(b, 1, ex)
+        check_full(b, q, k)
+        q2, k2 = run_tp(b, 1, ex)  # the next epoch on the same buffer
+        assert torch.equal(q, q2) and torch.equal(k, k2)
+        assert ex.epoch == 2
+        ex.close()
+        assert qk.device_timeouts() == 0
+    finally:
+        dist.destroy_process_group()
