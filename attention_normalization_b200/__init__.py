@@ -57,13 +57,14 @@ def _rows(t: torch.Tensor, name: str):
         raise ValueError(f"{name} must be a CUDA tensor (this library has no CPU path)")
     if t.dtype not in _DTYPES:
         raise TypeError(f"{name}: dtype {t.dtype} unsupported (float32, bfloat16, float16, float8_e4m3fn)")
-    if t.dim() != 2:
+    shape = t.shape
+    if len(shape) != 2:
         raise ValueError(f"{name} must be 2-D [T, width]")
-    T, H = t.shape
-    if T > 0 and H > 1 and t.stride(1) != 1:
+    T, H = shape
+    s0, s1 = t.stride()
+    if T > 0 and H > 1 and s1 != 1:
         raise ValueError(f"{name} rows must be unit-stride along the width")
-    stride = t.stride(0) if T > 1 else max(t.stride(0), H)
-    return T, H, stride
+    return T, H, (s0 if T > 1 else max(s0, H))
 
 
 def _vec(t: torch.Tensor, name: str, n: int, dtype: torch.dtype, device):
@@ -78,12 +79,38 @@ def _out_like(x: torch.Tensor, stride: int) -> torch.Tensor:
     return torch.empty_strided((T, H), (stride, 1), dtype=x.dtype, device=x.device)
 
 
+# The current stream's raw handle without building a Stream object (a
+# fraction of a microsecond instead of about two per call), where torch has it.
+_raw_current_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+
+
 def _stream_handle(stream, device) -> int:
     if stream is None:
+        if _raw_current_stream is not None:
+            return _raw_current_stream(device.index if device.index is not None else torch.cuda.current_device())
         return torch.cuda.current_stream(device).cuda_stream
     if isinstance(stream, torch.cuda.Stream):
         return stream.cuda_stream
     return int(stream)
+
+
+class _NoSwitch:
+    def __enter__(self):
+        return None
+
+    def __exit__(self, *exc):
+        return False
+
+
+_NO_SWITCH = _NoSwitch()
+
+
+def _on(device):
+    """Makes `device` current for a call: a no-op when it already is (the
+    usual case), else torch.cuda.device."""
+    if device.index is None or device.index == torch.cuda.current_device():
+        return _NO_SWITCH
+    return torch.cuda.device(device)
 
 
 def _same(dev_a, dtype_a, t: torch.Tensor, name: str):
@@ -128,7 +155,7 @@ def qknorm_layerwise(q_in: torch.Tensor, k_in: torch.Tensor, gamma_q: torch.Tens
     """
     args, q_out, k_out, dev = _layerwise_args(q_in, k_in, gamma_q, gamma_k, eps, q_out, k_out)
     lib = capi()
-    with torch.cuda.device(dev):
+    with _on(dev):
         s = _stream_handle(stream, dev)
         if launch is None:
             st = lib.qknorm_layerwise(*args, s)
@@ -166,7 +193,7 @@ def qknorm_headwise(q_in: torch.Tensor, k_in: torch.Tensor, gamma_q: torch.Tenso
     args = [q_in.data_ptr(), q_out.data_ptr(), _vec(gamma_q, "gamma_q", head_dim, gdt, dev), sq, Wq // head_dim,
             k_in.data_ptr(), k_out.data_ptr(), _vec(gamma_k, "gamma_k", head_dim, gdt, dev), sk, Wk // head_dim,
             Tq, int(head_dim), float(eps), _DTYPES[dt]]
-    with torch.cuda.device(dev):
+    with _on(dev):
         s = _stream_handle(stream, dev)
         if launch is None:
             st = capi().qknorm_headwise(*args, s)
@@ -223,7 +250,7 @@ def qknorm_qkv_gemm_stats(x: torch.Tensor, w: torch.Tensor, Hq: int, Hk: int, Hv
         if not (t.is_cuda and t.device == dev and t.dtype == torch.float32 and t.is_contiguous()
                 and t.numel() == rows * T):
             raise ValueError(f"{name} must be a contiguous float32 CUDA tensor of {rows} x {T}")
-    with torch.cuda.device(dev):
+    with _on(dev):
         st = capi().qknorm_qkv_gemm_stats(x.data_ptr(), xs, w.data_ptr(), ws, qkv.data_ptr(), qs, T, D, Hq, Hk, Hv,
                                           q_sums.data_ptr(), k_sums.data_ptr(), _clib.QKN_BF16,
                                           _stream_handle(stream, dev))
@@ -245,7 +272,7 @@ def qknorm_qkv_projection(x: torch.Tensor, w: torch.Tensor, gamma_q: torch.Tenso
         raise ValueError("workspace must be a contiguous CUDA tensor on the device of x")
     gq = _vec(gamma_q, "gamma_q", Hq, torch.bfloat16, dev)
     gk = _vec(gamma_k, "gamma_k", Hk, torch.bfloat16, dev)
-    with torch.cuda.device(dev):
+    with _on(dev):
         st = capi().qknorm_qkv_projection(x.data_ptr(), xs, w.data_ptr(), ws, qkv.data_ptr(), qs, gq, gk, T, D,
                                           Hq, Hk, Hv, float(eps), workspace.data_ptr(),
                                           workspace.numel() * workspace.element_size(), _clib.QKN_BF16,
@@ -338,7 +365,7 @@ def qknorm_tp_layerwise(q_shards, k_shards, gamma_q_shards, gamma_k_shards, Hq_f
 
     def arr(xs):
         return (P * len(xs))(*[int(x) for x in xs])
-    with torch.cuda.device(dev):
+    with _on(dev):
         st = capi().qknorm_tp_layerwise(R, first_rank, n_local, arr([q.data_ptr() for q in q_shards]),
                                         arr([q.data_ptr() for q in q_out]), arr(gq), sq, hq, int(Hq_full),
                                         arr([k.data_ptr() for k in k_shards]), arr([k.data_ptr() for k in k_out]),
@@ -353,7 +380,7 @@ def qknorm_layerwise_plan(q_in, k_in, gamma_q, gamma_k, eps: float = 1e-6, *, q_
     """The launch ``qknorm_layerwise`` would use for these tensors."""
     args, _, _, dev = _layerwise_args(q_in, k_in, gamma_q, gamma_k, eps, q_out, k_out)
     L = QknLaunch()
-    with torch.cuda.device(dev):
+    with _on(dev):
         st = capi().qknorm_layerwise_plan(*args, ctypes.byref(L))
     _clib.check(st, "qknorm_layerwise_plan")
     return L.as_dict()
@@ -381,7 +408,7 @@ def qknorm_partial_stats(q_shard: torch.Tensor, k_shard: torch.Tensor, q_sumsq=N
     pq = _vec(q_sumsq, "q_sumsq", T, torch.float32, dev)
     pk = _vec(k_sumsq, "k_sumsq", T, torch.float32, dev)
     args = [q_shard.data_ptr(), sq, hq, pq, k_shard.data_ptr(), sk, hk, pk, T, _DTYPES[dt]]
-    with torch.cuda.device(dev):
+    with _on(dev):
         s = _stream_handle(stream, dev)
         if launch is None:
             st = capi().qknorm_partial_stats(*args, s)
@@ -423,7 +450,7 @@ def qknorm_combine_apply(q_in: torch.Tensor, k_in: torch.Tensor, gamma_q_shard: 
             ps_q, int(Hq_full),
             k_in.data_ptr(), k_out.data_ptr(), _vec(gamma_k_shard, "gamma_k_shard", hk, gdt, dev), sk, hk,
             ps_k, int(Hk_full), P, T, float(eps), _DTYPES[dt]]
-    with torch.cuda.device(dev):
+    with _on(dev):
         s = _stream_handle(stream, dev)
         if launch is None:
             st = capi().qknorm_combine_apply(*args, s)
