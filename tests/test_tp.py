@@ -152,3 +152,52 @@ def test_peer_exchange_single_rank_on_the_gpu():
         assert qk.device_timeouts() == 0
     finally:
         dist.destroy_process_group()
+
+
+def _ipc_pair_worker(rank, port, out):
+    import numpy as np
+    import torch.distributed as dist
+    from cuda.bindings import runtime as rt
+    torch.cuda.set_device(0)
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=2)
+    try:
+        ex = qk.TpPeerExchange(2, 64)
+        ptrs = ex.pointers()
+        # write a marker into the other rank's buffer through its mapping
+        mark = np.array([0x1234 + rank], dtype=np.uint64)
+        (err,) = rt.cudaMemcpy(ptrs[1 - rank] + 8 * rank, mark.ctypes.data, 8, rt.cudaMemcpyKind.cudaMemcpyHostToDevice)
+        assert err == rt.cudaError_t.cudaSuccess
+        (err,) = rt.cudaDeviceSynchronize()
+        dist.barrier()
+        got = np.zeros(2, dtype=np.uint64)
+        (err,) = rt.cudaMemcpy(got.ctypes.data, ptrs[rank], 16, rt.cudaMemcpyKind.cudaMemcpyDeviceToHost)
+        assert err == rt.cudaError_t.cudaSuccess
+        dist.barrier()  # no rank unmaps while the other may still write
+        ex.close()
+        out.put((rank, [int(v) for v in got]))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_peer_exchange_maps_another_process_buffer():
+    """Two processes on this GPU exchange IPC handles through a gloo group and
+    each writes a marker into the other's receive buffer through its mapping
+    (plain copies; no kernel waits on another process)."""
+    import socket
+
+    import torch.multiprocessing as mp
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_ipc_pair_worker, args=(r, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    got = dict(q.get(timeout=180) for _ in range(2))
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    # rank r's buffer holds the other rank's marker at that rank's slot, zero elsewhere
+    assert got[0] == [0, 0x1234 + 1]
+    assert got[1] == [0x1234 + 0, 0]
