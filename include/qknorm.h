@@ -77,7 +77,7 @@ typedef enum {
 typedef enum {
     QKN_OK = 0,
     QKN_ERR_INVALID_ARG = 1,   /* bad size, stride, eps, dtype, null pointer or overlap */
-    QKN_ERR_UNSUPPORTED = 2,   /* a launch shape this build cannot run */
+    QKN_ERR_UNSUPPORTED = 2,   /* a launch shape the library cannot run */
     QKN_ERR_CUDA = 3           /* the CUDA runtime reported an error */
 } qkn_status;
 
