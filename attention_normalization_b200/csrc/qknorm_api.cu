@@ -1066,12 +1066,23 @@ qkn_status qknorm_tp_layerwise(int32_t R, int32_t first_rank, int32_t n_local, c
             else if (!aligned16(pp)) return fail(QKN_ERR_UNSUPPORTED, "local rank %d: buffers must be 16-byte aligned", j);
         const Region iq = rows_region(q_in[j], hq_shard, q_stride, T, esz), oq = rows_region(q_out[j], hq_shard, q_stride, T, esz);
         const Region ik = rows_region(k_in[j], hk_shard, k_stride, T, esz), ok_ = rows_region(k_out[j], hk_shard, k_stride, T, esz);
-        const Region others[3] = {flat_region(gamma_q[j], (int64_t)hq_shard * gsz),
-                                  flat_region(gamma_k[j], (int64_t)hk_shard * gsz),
-                                  flat_region(recv[first_rank + j], qknorm_tp_recv_bytes(R, T))};
-        qkn_status st = check_outputs(oq, ok_, iq, ik, others, 3);
+        const Region others[2] = {flat_region(gamma_q[j], (int64_t)hq_shard * gsz),
+                                  flat_region(gamma_k[j], (int64_t)hk_shard * gsz)};
+        qkn_status st = check_outputs(oq, ok_, iq, ik, others, 2);
         if (st != QKN_OK) return st;
+        // the kernel writes every rank's receive buffer: none may share a byte
+        // with this rank's rows or gamma slices
+        for (int r = 0; r < R; ++r) {
+            const Region rb = flat_region(recv[r], qknorm_tp_recv_bytes(R, T));
+            if (overlap(rb, oq) || overlap(rb, ok_) || overlap(rb, iq) || overlap(rb, ik) || overlap(rb, others[0]) ||
+                overlap(rb, others[1]))
+                return fail(QKN_ERR_INVALID_ARG, "receive buffer %d overlaps local rank %d's rows or gamma", r, j);
+        }
     }
+    for (int r = 0; r < R; ++r)  // nor one another
+        for (int r2 = r + 1; r2 < R; ++r2)
+            if (overlap(flat_region(recv[r], qknorm_tp_recv_bytes(R, T)), flat_region(recv[r2], qknorm_tp_recv_bytes(R, T))))
+                return fail(QKN_ERR_INVALID_ARG, "receive buffers %d and %d overlap", r, r2);
     for (int j = 0; j < n_local; ++j)  // no rank's output may touch another local rank's buffers
         for (int jj = 0; jj < n_local; ++jj) {
             if (jj == j) continue;

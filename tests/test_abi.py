@@ -426,6 +426,10 @@ def _tp_call(lib, **kw):
     ({"recv": [0x40000000, 0, 0x40200000, 0x40300000]}, INVALID),
     ({"recv": [0x40000004, 0x40100000, 0x40200000, 0x40300000]}, INVALID),  # not 16-byte aligned
     ({"recv": [0x40000000, 0x40100008, 0x40200000, 0x40300000]}, INVALID),
+    ({"recv": [0x40000000, 0x40001000, 0x40200000, 0x40300000]}, INVALID),  # two receive buffers overlap
+    ({"recv": [0x40000000, 0x40100000, 0x40200000, 0x11400000]}, INVALID),  # rank 3's buffer on rank 1's q_out
+    ({"recv": [0x40000000, 0x40100000, 0x10000000, 0x40300000]}, INVALID),  # rank 2's buffer on rank 0's q_in
+    ({"recv": [0x40000000, 0x40100000, 0x40200000, 0x10800000]}, INVALID),  # on rank 0's gamma_q slice
 ])
 def test_tp_validation(lib, kw, want):
     assert _tp_call(lib, **kw) == want
