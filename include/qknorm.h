@@ -258,7 +258,9 @@ int64_t qknorm_qkv_projection_noalloc_max_bytes(void);
  * the tokens concerned are left unwritten.
  * Requirements: 1 <= R <= 8, n_local <= 8; dtype any of qkn_dtype; 16-byte
  * aligned buffers and shard widths / strides that are whole 16-byte vectors
- * (else QKN_ERR_UNSUPPORTED).  T = 0 is a no-op.  Asynchronous on `stream`;
+ * (else QKN_ERR_UNSUPPORTED); no output overlapping another operand, and no
+ * receive buffer overlapping another or any local rank's rows or gamma
+ * (else QKN_ERR_INVALID_ARG).  T = 0 is a no-op.  Asynchronous on `stream`;
  * allocates nothing.
  */
 int64_t qknorm_tp_recv_bytes(int32_t R, int64_t T);
