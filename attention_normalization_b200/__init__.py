@@ -323,14 +323,16 @@ def qknorm_tp_layerwise(q_shards, k_shards, gamma_q_shards, gamma_k_shards, Hq_f
                         eps: float = 1e-6, *, exchange: TpExchange | TpPeerExchange | None = None, recv=None,
                         epoch: int | None = None,
                         R: int | None = None, first_rank: int = 0, q_out=None, k_out=None, in_place: bool = False,
-                        blocks_per_rank: int = 0, timeout_ns: int = 0, stream=None):
+                        blocks_per_rank: int = 0, timeout_ns: int = 0, system_scope: bool = False, stream=None):
     """Tensor-parallel layerwise QK-Norm: runs ranks first_rank ..
     first_rank + len(q_shards) - 1 of an R-rank group; shard j holds Q columns
     of rank first_rank + j for all T tokens.  The ranks exchange only their
     scalar partial sums (through ``exchange`` / ``recv``): a ``TpExchange``
     when every rank runs in this call on this GPU, a ``TpPeerExchange`` when
     each process runs its own rank on its own GPU (pass ``first_rank`` = that
-    rank and one shard).  Returns the lists ``(q_out, k_out)``."""
+    rank and one shard).  ``system_scope`` runs the exchange with system-scope
+    loads and stores (the peer-memory form) even when every rank is in this
+    call.  Returns the lists ``(q_out, k_out)``."""
     n_local = len(q_shards)
     if not (n_local == len(k_shards) == len(gamma_q_shards) == len(gamma_k_shards)) or n_local < 1:
         raise ValueError("one Q shard, K shard and gamma slice each per local rank")
@@ -366,11 +368,12 @@ def qknorm_tp_layerwise(q_shards, k_shards, gamma_q_shards, gamma_k_shards, Hq_f
     def arr(xs):
         return (P * len(xs))(*[int(x) for x in xs])
     with _on(dev):
-        st = capi().qknorm_tp_layerwise(R, first_rank, n_local, arr([q.data_ptr() for q in q_shards]),
-                                        arr([q.data_ptr() for q in q_out]), arr(gq), sq, hq, int(Hq_full),
-                                        arr([k.data_ptr() for k in k_shards]), arr([k.data_ptr() for k in k_out]),
-                                        arr(gk), sk, hk, int(Hk_full), T, float(eps), _DTYPES[dt], arr(recv),
-                                        int(epoch), int(blocks_per_rank), int(timeout_ns), _stream_handle(stream, dev))
+        st = capi().qknorm_tp_layerwise_scope(R, first_rank, n_local, arr([q.data_ptr() for q in q_shards]),
+                                              arr([q.data_ptr() for q in q_out]), arr(gq), sq, hq, int(Hq_full),
+                                              arr([k.data_ptr() for k in k_shards]),
+                                              arr([k.data_ptr() for k in k_out]), arr(gk), sk, hk, int(Hk_full), T,
+                                              float(eps), _DTYPES[dt], arr(recv), int(epoch), int(blocks_per_rank),
+                                              int(timeout_ns), 1 if system_scope else 0, _stream_handle(stream, dev))
     _clib.check(st, "qknorm_tp_layerwise")
     return q_out, k_out
 

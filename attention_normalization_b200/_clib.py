@@ -17,8 +17,9 @@ QKN_FP8_E4M3 = 3
 
 QKN_OK = 0
 QKN_ERR_INVALID_ARG = 1
-QKN_ERR_UNSUPPORTED = 2
-QKN_ERR_CUDA = 3
+QKN_ERR_MISALIGNED = 2  # reserved: never returned (unaligned buffers take a scalar-access kernel)
+QKN_ERR_UNSUPPORTED = 3
+QKN_ERR_CUDA = 4
 
 QKN_KERNEL_REGISTER = 0
 QKN_KERNEL_TWOPASS_VEC = 1
@@ -64,6 +65,10 @@ PROTOTYPES = {
     "qknorm_tp_recv_bytes": (_i64, [_i32, _i64]),
     "qknorm_tp_layerwise": (_st, [_i32, _i32, _i32, _vp, _vp, _vp, _i64, _i32, _i32, _vp, _vp, _vp, _i64, _i32, _i32,
                                   _i64, _f32, _dt, _vp, ctypes.c_uint32, _i32, _u64, _vp]),
+    "qknorm_tp_layerwise_scope": (_st, [_i32, _i32, _i32, _vp, _vp, _vp, _i64, _i32, _i32, _vp, _vp, _vp, _i64, _i32,
+                                        _i32, _i64, _f32, _dt, _vp, ctypes.c_uint32, _i32, _u64, _i32, _vp]),
+    "qknorm_layerwise_host": (_st, _LAYERWISE_ARGS + [_vp, _i64, _i64, _vp, _vp, _vp]),
+    "qknorm_layerwise_host_ring_bytes": (_i64, [_i64, _i32, _i32, _dt, _i32]),
     "qknorm_last_error": (ctypes.c_char_p, []),
     "qknorm_version": (ctypes.c_int, []),
     "qknorm_register_max_threads": (_i32, [_i32]),

@@ -52,7 +52,7 @@ def build(force: bool = False, ptxas_verbose: bool = False, quiet: bool = False)
            "-Xcompiler", "-fPIC,-Wall", "-shared", "-cudart", "static",
            "-I", INCLUDE, "-I", CSRC,
            os.path.join(CSRC, "qknorm_api.cu"), os.path.join(CSRC, "qkv_gemm.cu"), os.path.join(CSRC, "qknorm_tp.cu"),
-           "-o", tmp]
+           os.path.join(CSRC, "qknorm_host.cu"), "-o", tmp]
     if ptxas_verbose:
         cmd[1:1] = ["-Xptxas", "-v"]
     r = subprocess.run(cmd, capture_output=True, text=True)

@@ -6,6 +6,7 @@
 // rejected call never reaches the GPU.  Nothing here allocates device memory
 // or synchronizes.
 
+#include <cuda.h>  // CUcontext / CUresult types only: driver entry points are fetched at run time
 #include <cuda_runtime.h>
 
 #include <cmath>
@@ -21,7 +22,7 @@
 #include "qknorm_tp.cuh"
 
 #ifndef QKNORM_VERSION
-#define QKNORM_VERSION 100  // 0.1.0
+#define QKNORM_VERSION 200  // 0.2.0: status codes of the boundary contract (UNSUPPORTED 3, CUDA 4)
 #endif
 
 namespace {
@@ -42,6 +43,16 @@ qkn_status ok() {
     g_last_error[0] = '\0';
     return QKN_OK;
 }
+
+}  // namespace
+
+namespace qkn {
+// The calling thread's message for qknorm_last_error, for the library's other
+// translation units (the host-buffer pipeline).
+void set_last_error(const char *msg) { snprintf(g_last_error, sizeof(g_last_error), "%s", msg); }
+}  // namespace qkn
+
+namespace {
 
 // Bytes of one element of x (and y), and of one element of gamma.
 int elem_bytes(qkn_dtype dt) { return dt == QKN_F32 ? 4 : (dt == QKN_FP8_E4M3 ? 1 : 2); }
@@ -677,31 +688,70 @@ qkn_status launch_projection_gemm(const Projection &pr, float *q_sums, float *k_
 // own device image, so that entry point never allocates.  Each GPU that loads
 // the library holds it until the process exits.  Host code must not pass the
 // array's name to a kernel (on the host it is only a stand-in for the symbol);
-// the device address comes from cudaGetSymbolAddress, once per device.
+// the device address comes from cudaGetSymbolAddress, looked up once per
+// device and context.
 constexpr int64_t kNoAllocScratchBytes = (int64_t)4 << 20;  // 4 MiB
 static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchBytes / 4];
 
 namespace {
 constexpr int kMaxScratchDevices = 64;
 std::mutex g_scratch_mu;
-void *g_scratch_addr[kMaxScratchDevices] = {};
 
-// Device address of g_noalloc_scratch on the current device (looked up on the
-// first call for that device, with the device current).
+struct ScratchAddr {
+    unsigned long long ctx_id;  // the context the address belongs to (0: unknown)
+    void *addr;
+};
+ScratchAddr g_scratch_addr[kMaxScratchDevices] = {};
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext *);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long *);
+
+// The unique id of the calling thread's current CUDA context, or 0 when there
+// is none yet or the driver cannot tell.  A device reset (cudaDeviceReset)
+// ends the primary context, and the next one gets a new id -- and a new
+// address for the scratch array.
+unsigned long long current_context_id() {
+    static CtxGetCurrentFn get_current = nullptr;
+    static CtxGetIdFn get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &f, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<CtxGetCurrentFn>(f);
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &f, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<CtxGetIdFn>(f);
+    });
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS)
+        return 0;
+    return id;
+}
+
+// Device address of g_noalloc_scratch on the current device: looked up with
+// that device current on the first call, and again whenever the current
+// context is not the one the cached address came from (after a device reset),
+// or on every call when the context's id cannot be read.
 qkn_status noalloc_scratch(void **out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return fail(QKN_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
     if (dev < 0 || dev >= kMaxScratchDevices) return fail(QKN_ERR_UNSUPPORTED, "device index %d too large", dev);
+    const unsigned long long ctx = current_context_id();
     std::lock_guard<std::mutex> lk(g_scratch_mu);
-    if (!g_scratch_addr[dev]) {
+    ScratchAddr &slot = g_scratch_addr[dev];
+    if (!slot.addr || ctx == 0 || slot.ctx_id != ctx) {
         void *p = nullptr;
         e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
         if (e != cudaSuccess || !p)
             return fail(QKN_ERR_CUDA, "cudaGetSymbolAddress(scratch): %s", cudaGetErrorString(e));
-        g_scratch_addr[dev] = p;
+        // the lookup makes the device's primary context current if none was
+        slot = ScratchAddr{ctx ? ctx : current_context_id(), p};
     }
-    *out = g_scratch_addr[dev];
+    *out = slot.addr;
     return QKN_OK;
 }
 }  // namespace
@@ -1023,18 +1073,26 @@ qkn_status qknorm_device_timeouts(int32_t *code) {
 }
 
 int64_t qknorm_tp_recv_bytes(int32_t R, int64_t T) {
-    if (R < 1 || R > qkn::tp::kMaxRanks || T < 0) return -1;
-    return (int64_t)R * T * 2 * 8;
+    if (R < 1 || R > qkn::tp::kMaxRanks || T < 0 || T >= ((int64_t)1 << 31)) return -1;
+    return (int64_t)R * T * 2 * 8 + 16;  // exchange words, then the 16-byte trailer (abort word)
 }
 
-qkn_status qknorm_tp_layerwise(int32_t R, int32_t first_rank, int32_t n_local, const void *const *q_in,
-                               void *const *q_out, const void *const *gamma_q, int64_t q_stride, int32_t hq_shard,
-                               int32_t Hq_full, const void *const *k_in, void *const *k_out,
-                               const void *const *gamma_k, int64_t k_stride, int32_t hk_shard, int32_t Hk_full,
-                               int64_t T, float eps, qkn_dtype dtype, void *const *recv, uint32_t epoch,
-                               int32_t blocks_per_rank, uint64_t timeout_ns, void *stream) {
+}  // extern "C"
+
+namespace {
+
+// qknorm_tp_layerwise with the exchange scope: scope 0 picks GPU scope when
+// every rank of the group runs in the call and system scope otherwise; scope 1
+// takes system scope whatever runs where.
+qkn_status tp_layerwise(int32_t R, int32_t first_rank, int32_t n_local, const void *const *q_in,
+                        void *const *q_out, const void *const *gamma_q, int64_t q_stride, int32_t hq_shard,
+                        int32_t Hq_full, const void *const *k_in, void *const *k_out, const void *const *gamma_k,
+                        int64_t k_stride, int32_t hk_shard, int32_t Hk_full, int64_t T, float eps, qkn_dtype dtype,
+                        void *const *recv, uint32_t epoch, int32_t blocks_per_rank, uint64_t timeout_ns,
+                        int32_t scope, void *stream) {
     using qkn::tp::kMaxLocal;
     using qkn::tp::kMaxRanks;
+    if (scope != 0 && scope != 1) return fail(QKN_ERR_INVALID_ARG, "scope must be 0 (automatic) or 1 (system)");
     if (!dtype_valid(dtype)) return fail(QKN_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
     if (R < 1 || R > kMaxRanks) return fail(QKN_ERR_INVALID_ARG, "R = %d outside [1, %d]", R, kMaxRanks);
     if (n_local < 1 || n_local > kMaxLocal || first_rank < 0 || first_rank + n_local > R)
@@ -1112,7 +1170,8 @@ qkn_status qknorm_tp_layerwise(int32_t R, int32_t first_rank, int32_t n_local, c
     qkn_status st = current_device(&dev);
     if (st != QKN_OK) return st;
     if ((st = sm_count(dev, &sms)) != QKN_OK) return st;
-    cudaError_t e = qkn::tp::tp_blocks_per_sm((int)dtype, nv, threads, n_local == R, &bps);
+    const bool gpu_scope = n_local == R && scope == 0;
+    cudaError_t e = qkn::tp::tp_blocks_per_sm((int)dtype, nv, threads, gpu_scope, &bps);
     if (e != cudaSuccess || bps < 1) return fail(QKN_ERR_CUDA, "occupancy query: %s", cudaGetErrorString(e));
     const int64_t resident = (int64_t)bps * sms;
     int64_t G = blocks_per_rank > 0 ? blocks_per_rank : resident / n_local;
@@ -1142,16 +1201,43 @@ qkn_status qknorm_tp_layerwise(int32_t R, int32_t first_rank, int32_t n_local, c
     tp.epoch = epoch;
     tp.timeout_ns = timeout_ns ? timeout_ns : kGemmTimeoutNs;
     const char *what = "";
-    e = qkn::tp::launch_tp(tp, (int)dtype, nv, threads, static_cast<cudaStream_t>(stream), &what);
+    e = qkn::tp::launch_tp(tp, (int)dtype, nv, threads, gpu_scope, static_cast<cudaStream_t>(stream), &what);
     if (e == cudaSuccess) e = cudaGetLastError();
     if (e != cudaSuccess) return fail(QKN_ERR_CUDA, "tensor-parallel kernel (%s): %s", what, cudaGetErrorString(e));
     return ok();
+}
+
+}  // namespace
+
+extern "C" {
+
+qkn_status qknorm_tp_layerwise(int32_t R, int32_t first_rank, int32_t n_local, const void *const *q_in,
+                               void *const *q_out, const void *const *gamma_q, int64_t q_stride, int32_t hq_shard,
+                               int32_t Hq_full, const void *const *k_in, void *const *k_out,
+                               const void *const *gamma_k, int64_t k_stride, int32_t hk_shard, int32_t Hk_full,
+                               int64_t T, float eps, qkn_dtype dtype, void *const *recv, uint32_t epoch,
+                               int32_t blocks_per_rank, uint64_t timeout_ns, void *stream) {
+    return tp_layerwise(R, first_rank, n_local, q_in, q_out, gamma_q, q_stride, hq_shard, Hq_full, k_in, k_out,
+                        gamma_k, k_stride, hk_shard, Hk_full, T, eps, dtype, recv, epoch, blocks_per_rank, timeout_ns,
+                        0, stream);
+}
+
+qkn_status qknorm_tp_layerwise_scope(int32_t R, int32_t first_rank, int32_t n_local, const void *const *q_in,
+                                     void *const *q_out, const void *const *gamma_q, int64_t q_stride,
+                                     int32_t hq_shard, int32_t Hq_full, const void *const *k_in, void *const *k_out,
+                                     const void *const *gamma_k, int64_t k_stride, int32_t hk_shard, int32_t Hk_full,
+                                     int64_t T, float eps, qkn_dtype dtype, void *const *recv, uint32_t epoch,
+                                     int32_t blocks_per_rank, uint64_t timeout_ns, int32_t scope, void *stream) {
+    return tp_layerwise(R, first_rank, n_local, q_in, q_out, gamma_q, q_stride, hq_shard, Hq_full, k_in, k_out,
+                        gamma_k, k_stride, hk_shard, Hk_full, T, eps, dtype, recv, epoch, blocks_per_rank, timeout_ns,
+                        scope, stream);
 }
 
 const char *qknorm_status_string(qkn_status s) {
     switch (s) {
         case QKN_OK: return "ok";
         case QKN_ERR_INVALID_ARG: return "invalid argument";
+        case QKN_ERR_MISALIGNED: return "misaligned (reserved; not returned)";
         case QKN_ERR_UNSUPPORTED: return "unsupported";
         case QKN_ERR_CUDA: return "CUDA error";
         default: return "unknown status";

@@ -13,11 +13,9 @@ namespace qkn {
 namespace tp {
 namespace {
 
-// Set by a wait that ran out (code 4); read and cleared by the host.
+// Set to 4 by a wait that ran out or gave up (every wait that returns without
+// its partial sums sets it); read and cleared by the host.
 __device__ int g_tp_timeout = 0;
-// The epoch of a call in which a wait ran out: every other wait of that call
-// gives up at once instead of running out in turn.
-__device__ unsigned int g_tp_aborted_epoch = 0;
 
 // Memory scope of the exchange: system when some ranks are on other GPUs
 // (peer memory), GPU when every rank runs in this launch.
@@ -32,8 +30,37 @@ __device__ __forceinline__ unsigned long long pack(uint32_t epoch, float v) {
     return (static_cast<unsigned long long>(epoch) << 32) | __float_as_uint(v);
 }
 
-__device__ __forceinline__ bool aborted(uint32_t epoch) {
-    return *reinterpret_cast<volatile unsigned int *>(&g_tp_aborted_epoch) == epoch;
+// The abort word of a receive buffer: the 64-bit word after its [R][T][2]
+// exchange words.  A wait that runs out stores the call's epoch there, in the
+// buffer of every rank of its launch, and the other waits of that call give
+// up when they see it.  It belongs to the buffer set and the epoch together,
+// so a later call -- a later epoch on these buffers, or any epoch on another
+// (zeroed) set -- never mistakes an old abort for its own.
+__device__ __forceinline__ unsigned long long *abort_word(const TpParams &p, int rank) {
+    return p.recv[rank] + static_cast<int64_t>(p.R) * p.T * 2;
+}
+
+template <bool SYS>
+__device__ __forceinline__ bool aborted(const unsigned long long *word, uint32_t epoch) {
+    unsigned long long v;
+    if constexpr (SYS)
+        asm volatile("ld.relaxed.sys.global.u64 %0, [%1];" : "=l"(v) : "l"(word) : "memory");
+    else
+        asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(word) : "memory");
+    return v == epoch;
+}
+
+// Marks the call aborted in the abort word of every rank this launch runs.
+template <bool SYS>
+__device__ __forceinline__ void mark_aborted(const TpParams &p, uint32_t epoch) {
+    for (int j = 0; j < p.n_local; ++j) {
+        unsigned long long *w = abort_word(p, p.first_rank + j);
+        const unsigned long long v = epoch;
+        if constexpr (SYS)
+            asm volatile("st.relaxed.sys.global.u64 [%0], %1;" ::"l"(w), "l"(v) : "memory");
+        else
+            asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(w), "l"(v) : "memory");
+    }
 }
 
 // Publishes this rank's partial sums for one token (the Q word, then the K
@@ -59,26 +86,30 @@ __device__ __forceinline__ void load_pair(const unsigned long long *src, unsigne
         asm volatile("ld.relaxed.gpu.global.v2.u64 {%0, %1}, [%2];" : "=l"(wq), "=l"(wk) : "l"(src) : "memory");
 }
 
-// Waits (bounded) until both words at `src` carry `epoch`; their values, or
-// false after a timeout or an abort of this call.
+// Waits (bounded) until both words at `src` carry the call's epoch; their
+// values, or false after a timeout or an abort of this call (`rank` is the
+// waiting rank, whose buffer holds the abort word it watches).  Every false
+// return records code 4.
 template <bool SYS>
-__device__ __forceinline__ bool wait_pair(const unsigned long long *src, uint32_t epoch, uint64_t timeout_ns,
-                                          float &vq, float &vk) {
+__device__ __forceinline__ bool wait_pair(const TpParams &p, int rank, const unsigned long long *src, float &vq,
+                                          float &vk) {
+    const uint32_t epoch = p.epoch;
     unsigned long long wq, wk;
     load_pair<SYS>(src, wq, wk);
     if (static_cast<uint32_t>(wq >> 32) != epoch || static_cast<uint32_t>(wk >> 32) != epoch) {
         const uint64_t t0 = now_ns();
+        const unsigned long long *abort = abort_word(p, rank);
         for (uint32_t it = 1;; ++it) {
             __nanosleep(32);
             load_pair<SYS>(src, wq, wk);
             if (static_cast<uint32_t>(wq >> 32) == epoch && static_cast<uint32_t>(wk >> 32) == epoch) break;
-            // every waiting lane of the GPU would read the same abort word:
+            // every waiting lane of a rank would read the same abort word:
             // look at it (and the clock) every 64 polls only
             if ((it & 63u) == 0) {
-                if (aborted(epoch)) return false;
-                if (now_ns() - t0 > timeout_ns) {
+                const bool gave_up = aborted<SYS>(abort, epoch);
+                if (gave_up || now_ns() - t0 > p.timeout_ns) {
                     atomicExch(&g_tp_timeout, 4);
-                    atomicExch(&g_tp_aborted_epoch, epoch);
+                    if (!gave_up) mark_aborted<SYS>(p, epoch);
                     return false;
                 }
             }
@@ -212,7 +243,7 @@ __device__ __forceinline__ void tp_finish(const TpParams &p, const RankPtrs &rp,
     float vq = 0.0f, vk = 0.0f;
     bool ok = true;
     if (lane < p.R)
-        ok = wait_pair<SYS>(p.recv[rank] + (static_cast<int64_t>(lane) * p.T + t) * 2, p.epoch, p.timeout_ns, vq, vk);
+        ok = wait_pair<SYS>(p, rank, p.recv[rank] + (static_cast<int64_t>(lane) * p.T + t) * 2, vq, vk);
     if (!__all_sync(0xFFFFFFFFu, ok)) return;  // a wait gave up: token left unwritten (reported)
     float Aq = 0.0f, Ak = 0.0f;  // Phase A aggregation, in rank order
     for (int i = 0; i < p.R; ++i) {
@@ -284,21 +315,27 @@ const void *tp_kernel(int dtype, int nv) {
     }
 }
 
-// System scope when some rank of the group runs elsewhere (peer memory).
-const void *tp_kernel(int dtype, int nv, bool all_local) {
-    return all_local ? tp_kernel<false>(dtype, nv) : tp_kernel<true>(dtype, nv);
+// GPU scope when every rank of the group runs in the launch, system scope
+// when some rank runs elsewhere (peer memory).
+const void *tp_kernel(int dtype, int nv, bool gpu_scope) {
+    return gpu_scope ? tp_kernel<false>(dtype, nv) : tp_kernel<true>(dtype, nv);
 }
 
 }  // namespace
 
-cudaError_t tp_blocks_per_sm(int dtype, int nv, int threads, bool all_local, int *out) {
-    const void *fn = tp_kernel(dtype, nv, all_local);
+cudaError_t tp_blocks_per_sm(int dtype, int nv, int threads, bool gpu_scope, int *out) {
+    const void *fn = tp_kernel(dtype, nv, gpu_scope);
     if (!fn) return cudaErrorInvalidValue;
     return cudaOccupancyMaxActiveBlocksPerMultiprocessor(out, fn, threads, 0);
 }
 
-cudaError_t launch_tp(const TpParams &p, int dtype, int nv, int threads, cudaStream_t stream, const char **what) {
-    const void *fn = tp_kernel(dtype, nv, p.n_local == p.R);
+cudaError_t launch_tp(const TpParams &p, int dtype, int nv, int threads, bool gpu_scope, cudaStream_t stream,
+                      const char **what) {
+    if (gpu_scope && p.n_local != p.R) {
+        *what = "GPU-scope exchange with ranks outside the launch";
+        return cudaErrorInvalidValue;
+    }
+    const void *fn = tp_kernel(dtype, nv, gpu_scope);
     if (!fn) {
         *what = "kernel selection";
         return cudaErrorInvalidValue;

@@ -34,12 +34,16 @@
 // (0 = Q, 1 = K)).  A word counts as arrived when its epoch field equals the
 // call's epoch, so buffers are never cleared between calls: each call on the
 // same buffers uses a new epoch (buffers start zeroed, epoch 0 is never used).
+// After the exchange words comes one 16-byte trailer whose first word is the
+// buffer's abort word: the epoch of the last call in which a wait of this
+// rank ran out.
 // Each word validates itself and carries the only data exchanged, so the two
 // words of a token are written with one relaxed 16-byte store and polled with
 // relaxed loads: no fence or release/acquire pair on the exchange path.
 // Every wait is bounded by the global timer; on expiry the kernel records a
-// code, marks the epoch aborted so every other wait of the call gives up at
-// once, and skips the affected tokens (their outputs are not written).
+// code, marks the epoch aborted in the abort word of every rank the launch
+// runs so every other wait of the call gives up at once (recording the code
+// too), and skips the affected tokens (their outputs are not written).
 #pragma once
 
 #include <cuda_runtime.h>
@@ -62,7 +66,7 @@ struct RankPtrs {
 
 struct TpParams {
     RankPtrs local[kMaxLocal];            // the ranks this launch runs
-    unsigned long long *recv[kMaxRanks];  // rank i's receive buffer [R][T][2] (peer-mapped when remote)
+    unsigned long long *recv[kMaxRanks];  // rank i's receive buffer [R][T][2] + abort word (peer-mapped when remote)
     int64_t q_stride_bytes, k_stride_bytes;
     int64_t T;
     int32_t R;                            // ranks in the group
@@ -80,12 +84,14 @@ struct TpParams {
 // block (128: four warps, one token each) for element type `dtype` (1 = bf16,
 // 2 = fp16, 0 = fp32, 3 = E4M3); nv < 0 selects the kernel with NVQ vectors
 // per lane for Q and NVK for K, nv = -(8 NVQ + NVK), nv == 0 the kernel for
-// rows of any width.  Cooperative when n_local > 1.
-cudaError_t launch_tp(const TpParams &p, int dtype, int nv, int threads, cudaStream_t stream, const char **what);
+// rows of any width.  gpu_scope selects the exchange at GPU scope (valid only
+// when every rank of the group runs in this launch), else system scope (peer
+// memory).  Cooperative when n_local > 1.
+cudaError_t launch_tp(const TpParams &p, int dtype, int nv, int threads, bool gpu_scope, cudaStream_t stream,
+                      const char **what);
 
-// Blocks of the kernel for (dtype, nv, threads) resident per SM; all_local
-// selects the GPU-scope form (every rank in the launch), else system scope.
-cudaError_t tp_blocks_per_sm(int dtype, int nv, int threads, bool all_local, int *out);
+// Blocks of the kernel for (dtype, nv, threads, scope) resident per SM.
+cudaError_t tp_blocks_per_sm(int dtype, int nv, int threads, bool gpu_scope, int *out);
 
 // The code a timed-out wait recorded (0 = none); synchronizes the device and
 // clears it.

@@ -66,6 +66,8 @@ def parse_args(argv=None):
     ap.add_argument("--dtype", choices=["bf16", "f16", "e4m3"], default="bf16",
                     help="element type of the prefill workload (gamma is bf16 with e4m3)")
     ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--e2e-chunk", type=int, default=512, help="tokens per chunk of the host-buffer pipeline")
+    ap.add_argument("--e2e-slots", type=int, default=3, help="device ring slots of the host-buffer pipeline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU baseline budget")
     a = ap.parse_args(argv)
@@ -106,6 +108,10 @@ class Ranks:
         t = torch.tensor([x], dtype=torch.float64, device=self.device)
         self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
         return float(t.item())
+
+
+def parallelism(world: int) -> str:
+    return f"replicas x{world} (tokens independent, no collective)"
 
 
 def whole_job(eff_bytes_per_step: int, steps: int, max_ms: float, world: int) -> dict:
@@ -215,14 +221,20 @@ class ClockSampler:
                 return getattr(nv, fn)(self.handle)
         return 0
 
+    def sample_now(self):
+        """One sample, taken on the calling thread (read-only NVML queries)."""
+        if self.handle is None:
+            return
+        try:
+            mhz = self.nv.nvmlDeviceGetClockInfo(self.handle, self.nv.NVML_CLOCK_SM)
+            self.samples.append((mhz, int(self._reasons())))
+        except Exception as e:
+            self.error = f"{type(e).__name__}: {e}"
+
     def _run(self):
         while not self.stop_ev.is_set():
-            if self.active.is_set() and self.handle is not None:
-                try:
-                    mhz = self.nv.nvmlDeviceGetClockInfo(self.handle, self.nv.NVML_CLOCK_SM)
-                    self.samples.append((mhz, int(self._reasons())))
-                except Exception as e:
-                    self.error = f"{type(e).__name__}: {e}"
+            if self.active.is_set():
+                self.sample_now()
             time.sleep(self.period)
 
     def start(self):
@@ -547,12 +559,17 @@ def native(args) -> int:
     torch.cuda.synchronize()
     barrier()
     torch.cuda.synchronize()
+    # the timed region can be far shorter than the sampling period: samples
+    # are also taken at its edges and while the replay is in flight
+    sampler.sample_now()
     sampler.active.set()
     ev0.record(stream)
     g_timed.replay()
     ev1.record(stream)
+    sampler.sample_now()
     torch.cuda.synchronize()
     sampler.active.clear()
+    sampler.sample_now()
     barrier()
     ms_rank = ev0.elapsed_time(ev1)
     ms = max_over_ranks(ms_rank)
@@ -628,21 +645,21 @@ def native(args) -> int:
 
     if rank == 0:
         cfg = wl.config()
+        cfg["parallelism"] = parallelism(world)
         between = (R - 1) * wl.set_bytes()
-        cfg.update({"parallelism": f"replicas x{world} (tokens independent, no collective)",
-                    "l2": f"rotating {R} input/output sets ({R * wl.set_bytes() / 1e6:.1f} MB; "
-                          f"{between / 1e6:.1f} MB touched between reuses "
-                          + ("> 2 x" if between > 2 * l2 else "< 2 x (L2-warm)") + f" {l2 / 1e6:.0f} MB L2)",
-                    "timing": "CUDA graph of K captured C-ABI calls (uploaded before timing: %s), "
-                              "CUDA events on the launching stream" % ("yes" if uploaded else "no"),
-                    "launch_plan": plan})
+        measurement = {"l2": f"rotating {R} input/output sets ({R * wl.set_bytes() / 1e6:.1f} MB; "
+                             f"{between / 1e6:.1f} MB touched between reuses "
+                             + ("> 2 x" if between > 2 * l2 else "< 2 x (L2-warm)") + f" {l2 / 1e6:.0f} MB L2)",
+                       "timing": "CUDA graph of K captured C-ABI calls (uploaded before timing: %s), "
+                                 "CUDA events on the launching stream" % ("yes" if uploaded else "no"),
+                       "launch_plan": plan}
         line = {"metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 6),
                 "us_per_call": round(step_s * 1e6 / wl.launches_per_step, 3),
                 "pct_of_peak": round(100 * per_rank_gbs / peaks["hbm_gbs"], 2),
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
                 "data": "synthetic (seeded; OLMo2-shaped activations, no dataset or weights)",
-                "config": cfg, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+                "config": cfg, "measurement": measurement, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": args.steps * wl.launches_per_step, "clocks": clocks,
                 "spread": spread, "device_timeouts": timeouts, "impl": "native"}
         print(json.dumps(line))
@@ -663,11 +680,15 @@ def e2e_measure(qk, wl: Workload, dev, args, barrier, max_over_ranks) -> dict:
         h_packed = b.packed.clone().pin_memory()
 
         def one():
-            qk.qknorm_packed_host(h_packed, 0, b.Hq, b.Hq, b.Hk, h_g[0], h_g[1], b.eps, device=dev)
-        h2d = h_packed.numel() * h_packed.element_size() + gbytes
-        d2h = h_packed.numel() * h_packed.element_size()
-        path = ("qknorm_packed_host: whole packed rows pinned host -> device in 512-token chunks, Q and K "
-                "normalized in place, rows device -> host; copies and kernel overlap on three streams")
+            qk.qknorm_packed_host(h_packed, 0, b.Hq, b.Hq, b.Hk, h_g[0], h_g[1], b.eps, device=dev,
+                                  chunk_tokens=args.e2e_chunk, slots=args.e2e_slots)
+        qk_bytes = b.T * (b.Hq + b.Hk) * wl.esz
+        h2d = qk_bytes + gbytes
+        d2h = qk_bytes
+        path = (f"C-ABI qknorm_layerwise_host: the Q and K columns of the pinned packed host rows -> device in "
+                f"{args.e2e_chunk}-token chunks (pitched copies; V never moves), normalized in place, back into "
+                f"the same host columns; {args.e2e_slots}-slot device ring, copies and kernel overlap on three "
+                "streams")
     elif wl.kind == "gqa":
         s = wl.make_set(dev)
         h_in = [t.clone().pin_memory() for t in b.q_shards + b.k_shards]
@@ -725,11 +746,13 @@ def e2e_measure(qk, wl: Workload, dev, args, barrier, max_over_ranks) -> dict:
         h_ko = torch.empty(h_k.shape, dtype=h_k.dtype, pin_memory=True)
 
         def one():
-            qk.qknorm_layerwise_host(h_q, h_k, h_g[0], h_g[1], b.eps, q_out=h_qo, k_out=h_ko, device=dev)
+            qk.qknorm_layerwise_host(h_q, h_k, h_g[0], h_g[1], b.eps, q_out=h_qo, k_out=h_ko, device=dev,
+                                     chunk_tokens=args.e2e_chunk, slots=args.e2e_slots)
         h2d = sum(t.numel() * t.element_size() for t in (h_q, h_k)) + gbytes
         d2h = sum(t.numel() * t.element_size() for t in (h_qo, h_ko))
-        path = ("qknorm_layerwise_host: pinned host -> device in 512-token chunks, normalized on the device, "
-                "device -> pinned host; copies and kernel overlap on three streams")
+        path = (f"C-ABI qknorm_layerwise_host: pinned host -> device in {args.e2e_chunk}-token chunks, normalized "
+                f"on the device, device -> pinned host; {args.e2e_slots}-slot device ring, copies and kernel "
+                "overlap on three streams")
 
     for _ in range(2):
         one()
@@ -771,8 +794,8 @@ def reference(args) -> int:
     el = time.perf_counter() - t0
     eff = wl.eff_bytes * tokens / b.T
     value = eff / (el / args.steps) / 1e9
-    cfg = wl.config()
-    cfg.update({"sample_tokens_per_step": tokens})
+    cfg = wl.config()  # the native arm's config, so both lines name the same workload
+    cfg["parallelism"] = parallelism(world)
     line = {"metric": METRIC, "value": round(value, 5), "unit": UNIT, "n_gpus": 0, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(el / args.steps * 1e3, 4), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": cfg,

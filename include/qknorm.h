@@ -77,8 +77,10 @@ typedef enum {
 typedef enum {
     QKN_OK = 0,
     QKN_ERR_INVALID_ARG = 1,   /* bad size, stride, eps, dtype, null pointer or overlap */
-    QKN_ERR_UNSUPPORTED = 2,   /* a launch shape the library cannot run */
-    QKN_ERR_CUDA = 3           /* the CUDA runtime reported an error */
+    QKN_ERR_MISALIGNED = 2,    /* reserved: never returned -- unaligned buffers take a
+                                  scalar-access kernel instead (see Alignment above) */
+    QKN_ERR_UNSUPPORTED = 3,   /* a shape or launch the library cannot run */
+    QKN_ERR_CUDA = 4           /* the CUDA runtime reported an error */
 } qkn_status;
 
 /*
@@ -128,6 +130,58 @@ qkn_status qknorm_combine_apply(const void *q_in, void *q_out, const void *gamma
                                 const void *k_in, void *k_out, const void *gamma_k_shard, int64_t k_stride,
                                 int32_t hk_shard, const float *k_sumsq_all, int32_t Hk_full,
                                 int32_t P, int64_t T, float eps, qkn_dtype dtype, void *stream);
+
+/*
+ * Fused layerwise QK-Norm of rows held in HOST memory, end to end: the T
+ * tokens flow in chunks of chunk_tokens through a ring of device buffers, and
+ * for each chunk the Q and K rows are copied host->device, normalized in
+ * place on the device by the same kernel as qknorm_layerwise (Background,
+ * Equation 1; Phase B), and copied device->host.  The host->device copy of
+ * one chunk, the kernel on the previous one and the device->host copy of the
+ * one before that overlap on three streams.
+ *   q_in, q_out, k_in, k_out : HOST pointers, rows as in qknorm_layerwise
+ *       ([T rows, stride q_stride] / [T rows, stride k_stride] elements).
+ *       Page-locked memory (cudaHostAlloc / cudaHostRegister) lets the copies
+ *       run asynchronously at full speed; pageable memory works but the copies
+ *       then stage through the driver.  out == in normalizes in place; for
+ *       packed [Q | K | V] host rows pass base and base + Hq with the packed
+ *       stride: only the Q and K columns travel, V is neither read nor written.
+ *   gamma_q [Hq], gamma_k [Hk] : DEVICE pointers (resident weights).
+ *   ring : DEVICE buffer owned by the caller, 256-byte aligned, of ring_bytes
+ *       bytes; it holds floor(ring_bytes / slot) slots (at most
+ *       QKN_HOST_MAX_SLOTS), a slot being chunk_tokens rows of Q then of K.
+ *       qknorm_layerwise_host_ring_bytes gives the size for a slot count; two
+ *       slots overlap copies in both directions with the kernel, three also
+ *       let a copy-in run ahead.
+ *   stream : the call's stream -- the kernels run on it, the copies start
+ *       after everything queued on it before the call, and the call is
+ *       complete (every output row back in host memory) once `stream`
+ *       reaches the point where the call returns.  copy_in_stream and
+ *       copy_out_stream carry the two copy directions; three different
+ *       streams give the overlap (equal streams are correct, only serial).
+ *       Calls that share a ring must be ordered through `stream`.
+ * Host memory must stay valid and unmodified until the call is complete.
+ * Errors: as qknorm_layerwise (arguments validated before anything is
+ * enqueued; host regions checked for overlap by address), plus
+ * QKN_ERR_INVALID_ARG for chunk_tokens < 1, a null or unaligned ring, a ring
+ * smaller than one slot, or a ring overlapping gamma.  A QKN_ERR_CUDA from a
+ * failed copy or launch may leave earlier chunks enqueued.
+ * No paper counterpart beyond the kernel: this is the library's end-to-end
+ * path for callers whose activations live in host memory.
+ */
+#define QKN_HOST_MAX_SLOTS 8
+qkn_status qknorm_layerwise_host(const void *q_in, void *q_out, const void *gamma_q, int64_t q_stride,
+                                 const void *k_in, void *k_out, const void *gamma_k, int64_t k_stride,
+                                 int64_t T, int32_t Hq, int32_t Hk, float eps, qkn_dtype dtype, void *ring,
+                                 int64_t ring_bytes, int64_t chunk_tokens, void *stream, void *copy_in_stream,
+                                 void *copy_out_stream);
+
+/* Bytes of a ring of `slots` slots for qknorm_layerwise_host: slots *
+ * (round_up(chunk_tokens * Hq * esz, 256) + round_up(chunk_tokens * Hk * esz,
+ * 256)), esz the element size; -1 for chunk_tokens < 1 or > 2^31, Hq or Hk <
+ * 1, slots outside [1, QKN_HOST_MAX_SLOTS] or an unknown dtype. */
+int64_t qknorm_layerwise_host_ring_bytes(int64_t chunk_tokens, int32_t Hq, int32_t Hk, qkn_dtype dtype,
+                                         int32_t slots);
 
 /*
  * Headwise QK-Norm (Background: the other granularity, "an independent factor
@@ -208,7 +262,10 @@ qkn_status qknorm_qkv_projection(const void *x, int64_t x_stride, const void *w,
  * Nothing is allocated: no cudaMalloc, no cudaFree, no allocating library
  * call.  The first call on a device looks up the array's device address
  * (cudaGetSymbolAddress, with that device current); make that first call
- * before any stream capture.
+ * before any stream capture.  The address is kept with the id of the context
+ * it belongs to and looked up again when the calling thread's context is
+ * another one (after cudaDeviceReset, say): the first call after such a
+ * change should also come before any capture.
  * Limits: the call's workspace, qknorm_qkv_projection_workspace_bytes(T, Hq,
  * Hk) = (Hq/256 + Hk/256) * T * 4 + 8 * ceil(T / 128) bytes, must fit in the
  * 4 MiB (e.g. T = 32000 with Hq = Hk = 4096); larger calls return
@@ -245,8 +302,10 @@ int64_t qknorm_qkv_projection_noalloc_max_bytes(void);
  *   recv[r] (r < R) is rank r's receive buffer, qknorm_tp_recv_bytes(R, T)
  *   bytes, 16-byte aligned: a device pointer valid on this GPU -- its own
  *   memory for local ranks, a peer mapping (cudaIpcOpenMemHandle or similar)
- *   for ranks on other GPUs.  Buffers start zeroed; each call on the same buffers passes a new
- *   epoch (> 0), and all ranks of one call pass the same epoch.
+ *   for ranks on other GPUs.  A buffer holds R * T pairs of 64-bit exchange
+ *   words and a 16-byte trailer (its abort word).  Buffers start zeroed and
+ *   are never cleared by the library; each call on the same buffers passes a
+ *   new epoch (> 0), and all ranks of one call pass the same epoch.
  *   Result: y = (x * gamma) * r with r = 1 / sqrt(S / H_full + eps) and S the
  *   ranks' partial sums added in rank order 0 .. R-1, identical on every rank.
  * Deployments: one GPU per rank (n_local = 1, each GPU calls with its own
@@ -254,8 +313,11 @@ int64_t qknorm_qkv_projection_noalloc_max_bytes(void);
  * or several ranks in one call on one GPU (their blocks wait on one another,
  * so the launch is cooperative and must fit on the GPU at once).
  * Waits are bounded by timeout_ns (0 = 2 s); one that runs out reports code 4
- * through qknorm_device_timeouts, every other wait of the call gives up, and
- * the tokens concerned are left unwritten.
+ * through qknorm_device_timeouts and writes the call's epoch into the abort
+ * word of every rank the call runs; every other wait of that call on those
+ * buffers then gives up and reports code 4 as well, and the tokens concerned
+ * are left unwritten.  The abort belongs to those buffers and that epoch:
+ * later epochs, and other buffers, are not affected.
  * Requirements: 1 <= R <= 8, n_local <= 8; dtype any of qkn_dtype; 16-byte
  * aligned buffers and shard widths / strides that are whole 16-byte vectors
  * (else QKN_ERR_UNSUPPORTED); no output overlapping another operand, and no
@@ -263,6 +325,8 @@ int64_t qknorm_qkv_projection_noalloc_max_bytes(void);
  * (else QKN_ERR_INVALID_ARG).  T = 0 is a no-op.  Asynchronous on `stream`;
  * allocates nothing.
  */
+/* Bytes of one receive buffer: R * T * 16 + 16; -1 for R outside [1, 8],
+ * T < 0 or T >= 2^31. */
 int64_t qknorm_tp_recv_bytes(int32_t R, int64_t T);
 qkn_status qknorm_tp_layerwise(int32_t R, int32_t first_rank, int32_t n_local, const void *const *q_in,
                                void *const *q_out, const void *const *gamma_q, int64_t q_stride, int32_t hq_shard,

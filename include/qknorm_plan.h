@@ -134,6 +134,22 @@ qkn_status qknorm_combine_apply_launch(const void *q_in, void *q_out, const void
                                        int32_t P, int64_t T, float eps, qkn_dtype dtype, void *stream,
                                        const qkn_launch *launch);
 
+/*
+ * qknorm_tp_layerwise with the memory scope of the exchange chosen by the
+ * caller.  scope 0: as qknorm_tp_layerwise (GPU-scope loads and stores when
+ * every rank of the group runs in this call, system scope otherwise); scope
+ * 1: system scope always -- the instantiation a one-rank-per-GPU deployment
+ * runs over peer memory -- so that it can be checked with every rank in one
+ * call on one GPU.  Same arguments, results and errors as
+ * qknorm_tp_layerwise, plus QKN_ERR_INVALID_ARG for another scope.
+ */
+qkn_status qknorm_tp_layerwise_scope(int32_t R, int32_t first_rank, int32_t n_local, const void *const *q_in,
+                                     void *const *q_out, const void *const *gamma_q, int64_t q_stride,
+                                     int32_t hq_shard, int32_t Hq_full, const void *const *k_in, void *const *k_out,
+                                     const void *const *gamma_k, int64_t k_stride, int32_t hk_shard, int32_t Hk_full,
+                                     int64_t T, float eps, qkn_dtype dtype, void *const *recv, uint32_t epoch,
+                                     int32_t blocks_per_rank, uint64_t timeout_ns, int32_t scope, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

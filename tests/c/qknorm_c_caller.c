@@ -1,9 +1,13 @@
 /*
  * A plain C caller of libqknorm.so: no Python, no torch.  Reads Q, K and the
  * two gamma vectors (bfloat16 bits) from files, normalizes them on the GPU
- * with qknorm_layerwise through the C ABI, and writes the outputs back.
+ * through the C ABI twice, and writes both results:
+ *   - qknorm_layerwise on device buffers -> qo.bin, ko.bin;
+ *   - qknorm_layerwise_host on page-locked host buffers, in place, in chunks
+ *     of `chunk` tokens through a two-slot device ring on three streams ->
+ *     qo_host.bin, ko_host.bin.
  *
- *   qknorm_c_caller T Hq Hk eps q.bin k.bin gq.bin gk.bin qo.bin ko.bin
+ *   qknorm_c_caller T Hq Hk eps chunk q.bin k.bin gq.bin gk.bin qo.bin ko.bin qo_host.bin ko_host.bin
  *
  * Exit status 0 on success; any CUDA or library error is printed with the
  * library's own message.
@@ -12,6 +16,7 @@
 #include <stdint.h>
 #include <stdio.h>
 #include <stdlib.h>
+#include <string.h>
 
 #include "qknorm.h"
 
@@ -46,16 +51,17 @@ static int write_file(const char *path, const void *buf, size_t bytes) {
     } while (0)
 
 int main(int argc, char **argv) {
-    if (argc != 11) {
-        fprintf(stderr, "usage: %s T Hq Hk eps q k gq gk qo ko\n", argv[0]);
+    if (argc != 14) {
+        fprintf(stderr, "usage: %s T Hq Hk eps chunk q k gq gk qo ko qo_host ko_host\n", argv[0]);
         return 1;
     }
     const long long T = atoll(argv[1]);
     const int Hq = atoi(argv[2]), Hk = atoi(argv[3]);
     const float eps = (float)atof(argv[4]);
+    const long long chunk = atoll(argv[5]);
     const size_t qb = (size_t)T * Hq * 2, kb = (size_t)T * Hk * 2;
-    void *hq = read_file(argv[5], qb), *hk = read_file(argv[6], kb);
-    void *hgq = read_file(argv[7], (size_t)Hq * 2), *hgk = read_file(argv[8], (size_t)Hk * 2);
+    void *hq = read_file(argv[6], qb), *hk = read_file(argv[7], kb);
+    void *hgq = read_file(argv[8], (size_t)Hq * 2), *hgk = read_file(argv[9], (size_t)Hk * 2);
     if (!hq || !hk || !hgq || !hgk) {
         fprintf(stderr, "could not read the inputs\n");
         return 1;
@@ -87,12 +93,43 @@ int main(int argc, char **argv) {
         return 4;
     }
     CHECK_CUDA(cudaStreamSynchronize(s));
+
+    /* the same rows from page-locked host memory, normalized in place */
+    void *pq, *pk;
+    CHECK_CUDA(cudaHostAlloc(&pq, qb, cudaHostAllocDefault));
+    CHECK_CUDA(cudaHostAlloc(&pk, kb, cudaHostAllocDefault));
+    memcpy(pq, hq, qb);
+    memcpy(pk, hk, kb);
+    const int64_t ring_bytes = qknorm_layerwise_host_ring_bytes(chunk, Hq, Hk, QKN_BF16, 2);
+    if (ring_bytes < 0) {
+        fprintf(stderr, "qknorm_layerwise_host_ring_bytes refused chunk %lld\n", chunk);
+        return 5;
+    }
+    void *ring;
+    CHECK_CUDA(cudaMalloc(&ring, (size_t)ring_bytes));
+    cudaStream_t s_in, s_out;
+    CHECK_CUDA(cudaStreamCreate(&s_in));
+    CHECK_CUDA(cudaStreamCreate(&s_out));
+    st = qknorm_layerwise_host(pq, pq, dgq, Hq, pk, pk, dgk, Hk, T, Hq, Hk, eps, QKN_BF16, ring, ring_bytes, chunk,
+                               (void *)s, (void *)s_in, (void *)s_out);
+    if (st != QKN_OK) {
+        fprintf(stderr, "qknorm_layerwise_host: %s: %s\n", qknorm_status_string(st), qknorm_last_error());
+        return 6;
+    }
+    CHECK_CUDA(cudaStreamSynchronize(s)); /* the call is complete once `s` passes it */
+
     CHECK_CUDA(cudaMemcpy(hq, dqo, qb, cudaMemcpyDeviceToHost));
     CHECK_CUDA(cudaMemcpy(hk, dko, kb, cudaMemcpyDeviceToHost));
-    if (write_file(argv[9], hq, qb) || write_file(argv[10], hk, kb)) {
+    if (write_file(argv[10], hq, qb) || write_file(argv[11], hk, kb) || write_file(argv[12], pq, qb) ||
+        write_file(argv[13], pk, kb)) {
         fprintf(stderr, "could not write the outputs\n");
         return 1;
     }
+    cudaStreamDestroy(s_in);
+    cudaStreamDestroy(s_out);
+    cudaFree(ring);
+    cudaFreeHost(pq);
+    cudaFreeHost(pk);
     cudaStreamDestroy(s);
     cudaFree(dq);
     cudaFree(dk);

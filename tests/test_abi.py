@@ -24,7 +24,7 @@ from attention_normalization_b200 import build as qbuild
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADERS = [os.path.join(ROOT, "include", h) for h in ("qknorm.h", "qknorm_plan.h")]
 
-OK, INVALID, UNSUPPORTED, CUDA = 0, 1, 2, 3
+OK, INVALID, MISALIGNED, UNSUPPORTED, CUDA = 0, 1, 2, 3, 4  # the status codes of the boundary contract
 F32, BF16 = 0, 1
 
 
@@ -57,6 +57,8 @@ def test_version_and_status_strings(lib):
     assert lib.qknorm_status_string(OK) == b"ok"
     assert lib.qknorm_status_string(INVALID) == b"invalid argument"
     assert lib.qknorm_status_string(CUDA) == b"CUDA error"
+    assert lib.qknorm_status_string(UNSUPPORTED) == b"unsupported"
+    assert lib.qknorm_status_string(MISALIGNED).startswith(b"misaligned")
     assert lib.qknorm_status_string(99) == b"unknown status"
 
 
@@ -435,6 +437,88 @@ def test_tp_validation(lib, kw, want):
     assert _tp_call(lib, **kw) == want
 
 
+def test_status_codes_in_the_header_are_the_contract():
+    """The enumerators' values as include/qknorm.h spells them (0..4, with 2
+    reserved for misaligned buffers, which the library never reports)."""
+    import re
+    text = open(os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "qknorm.h")).read()
+    got = {m.group(1): int(m.group(2)) for m in re.finditer(r"\b(QKN_(?:OK|ERR_[A-Z_]+))\s*=\s*(\d+)", text)}
+    assert got == {"QKN_OK": 0, "QKN_ERR_INVALID_ARG": 1, "QKN_ERR_MISALIGNED": 2, "QKN_ERR_UNSUPPORTED": 3,
+                   "QKN_ERR_CUDA": 4}
+    assert (_clib.QKN_OK, _clib.QKN_ERR_INVALID_ARG, _clib.QKN_ERR_MISALIGNED, _clib.QKN_ERR_UNSUPPORTED,
+            _clib.QKN_ERR_CUDA) == (0, 1, 2, 3, 4)
+
+
 def test_tp_recv_bytes(lib):
-    assert lib.qknorm_tp_recv_bytes(4, 4096) == 4 * 4096 * 16
+    assert lib.qknorm_tp_recv_bytes(4, 4096) == 4 * 4096 * 16 + 16  # exchange words, then the abort-word trailer
     assert lib.qknorm_tp_recv_bytes(0, 10) == -1 and lib.qknorm_tp_recv_bytes(9, 10) == -1
+
+
+def test_tp_scope_validation(lib):
+    """qknorm_tp_layerwise_scope: scope 0 or 1 pass validation (the device
+    query then fails here), any other scope is refused."""
+    P = ctypes.c_void_p
+    n = 4
+    base = lambda off: (P * n)(*[0x10000000 + off + j * 0x1000000 for j in range(n)])
+    recv = (P * 4)(*[0x40000000 + r * 0x100000 for r in range(4)])
+
+    def call(scope):
+        return lib.qknorm_tp_layerwise_scope(4, 0, n, base(0), base(0x400000), base(0x800000), 256, 256, 1024,
+                                             base(0x900000), base(0xB00000), base(0xD00000), 128, 128, 512, 128,
+                                             1e-6, BF16, recv, 1, 0, 0, scope, None)
+    assert call(0) == CUDA and call(1) == CUDA
+    assert call(2) == INVALID and call(-1) == INVALID
+
+
+# --------------------------------------------------------------------------- host-buffer entry point
+
+HOST = 0x7F0000000000  # fake host addresses: validation never dereferences them
+
+
+def _host_call(lib, **kw):
+    a = dict(q_in=HOST, q_out=HOST + (1 << 30), k_in=HOST + (2 << 30), k_out=HOST + (3 << 30), gq=BASE,
+             gk=BASE + 4096, qs=512, ks=256, T=1000, Hq=512, Hk=256, eps=1e-6, dtype=BF16, ring=BASE + (1 << 20),
+             chunk=128, slots=2, ring_bytes=None)
+    a.update(kw)
+    rb = a["ring_bytes"]
+    if rb is None:
+        rb = lib.qknorm_layerwise_host_ring_bytes(a["chunk"], a["Hq"], a["Hk"], BF16, a["slots"])
+    return lib.qknorm_layerwise_host(a["q_in"], a["q_out"], a["gq"], a["qs"], a["k_in"], a["k_out"], a["gk"], a["ks"],
+                                     a["T"], a["Hq"], a["Hk"], a["eps"], a["dtype"], a["ring"], rb, a["chunk"], None,
+                                     None, None)
+
+
+@pytest.mark.parametrize("kw,want", [
+    ({}, CUDA),                                        # well formed: validation passes, event creation fails here
+    ({"T": 0}, OK),
+    ({"T": -1}, INVALID),
+    ({"chunk": 0}, INVALID),
+    ({"ring": 0}, INVALID),
+    ({"ring": BASE + (1 << 20) + 16}, INVALID),        # ring not 256-byte aligned
+    ({"ring_bytes": 1000}, INVALID),                   # smaller than one slot
+    ({"gq": BASE + (1 << 20) + 256}, INVALID),         # gamma inside the ring
+    ({"q_out": HOST + 2}, INVALID),                    # partly overlaps q_in
+    ({"q_out": HOST, "k_out": HOST + (2 << 30)}, CUDA),  # in place: allowed
+    ({"k_out": HOST + 512}, INVALID),                  # k_out on q_in's rows (q_in rows are 1024 B)
+    ({"qs": 500}, INVALID),                            # stride below width
+    ({"eps": float("nan")}, INVALID),
+    ({"dtype": 7}, INVALID),
+    ({"gk": 0}, INVALID),
+    # packed [Q | K | V] host rows in place: Q at the base, K at +Hq, shared stride 6144
+    ({"q_in": HOST, "q_out": HOST, "k_in": HOST + 8192, "k_out": HOST + 8192, "Hq": 4096, "Hk": 1024, "qs": 6144,
+      "ks": 6144}, CUDA),
+])
+def test_host_entry_point_validation(lib, kw, want):
+    assert _host_call(lib, **kw) == want
+
+
+def test_host_ring_bytes(lib):
+    # two 256-byte aligned parts per slot
+    assert lib.qknorm_layerwise_host_ring_bytes(512, 4096, 4096, BF16, 3) == 3 * 2 * 512 * 4096 * 2
+    assert lib.qknorm_layerwise_host_ring_bytes(3, 8, 8, BF16, 1) == 256 + 256
+    assert lib.qknorm_layerwise_host_ring_bytes(1, 4, 4, 3, 8) == 8 * 512  # E4M3
+    assert lib.qknorm_layerwise_host_ring_bytes(0, 8, 8, BF16, 1) == -1
+    assert lib.qknorm_layerwise_host_ring_bytes(8, 8, 8, BF16, 0) == -1
+    assert lib.qknorm_layerwise_host_ring_bytes(8, 8, 8, BF16, 9) == -1
+    assert lib.qknorm_layerwise_host_ring_bytes(8, 0, 8, BF16, 1) == -1
+    assert lib.qknorm_layerwise_host_ring_bytes(8, 8, 8, 9, 1) == -1

@@ -150,7 +150,7 @@ def test_peer_exchange_handles_gloo():
     for rank, ptrs, epochs, log in got:
         assert epochs == [1, 2]
         assert ptrs == [own[r] if r == rank else own[r] + 0x700000000000 for r in range(world)]
-        assert log[0] == ("alloc", world * 4096 * 16) and log[1] == ("export", own[rank])
+        assert log[0] == ("alloc", world * 4096 * 16 + 16) and log[1] == ("export", own[rank])  # + abort-word trailer
         assert [e for e in log if e[0] == "open"] == [("open", own[r]) for r in range(world) if r != rank]
         assert [e for e in log if e[0] == "close"] == [("close", own[r] + 0x700000000000)
                                                       for r in range(world) if r != rank]

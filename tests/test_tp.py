@@ -66,6 +66,31 @@ def test_tp_matches_the_full_row_oracle(R, dtype):
     assert qk.device_timeouts() == 0
 
 
+@pytest.mark.parametrize("dtype", ALL_DTYPES)
+@pytest.mark.parametrize("R", [2, 4, 8])
+def test_tp_system_scope_matches_the_full_row_oracle(R, dtype):
+    """The system-scope instantiation -- the one a one-rank-per-GPU deployment
+    runs, with system-scope stores and loads on peer memory -- here with every
+    rank in one cooperative launch on one GPU, against the oracle."""
+    b = _batch(300, 2048, 512, dtype, seed=60 + R)
+    q, k = run_tp(b, R, system_scope=True)
+    check_full(b, q, k)
+    assert qk.device_timeouts() == 0
+    gq, gk = run_tp(b, R)  # the GPU-scope instantiation gives the same bits
+    assert torch.equal(q, gq) and torch.equal(k, gk)
+
+
+@pytest.mark.parametrize("R,Hq,Hk,dtype", [
+    (2, 8192, 1024, torch.bfloat16),    # 512 + 64 vectors per shard row: the batch-loop form
+    (8, 5120, 1024, torch.float32),
+])
+def test_tp_system_scope_wide_shards(R, Hq, Hk, dtype):
+    b = _batch(67, Hq, Hk, dtype, seed=70 + R)
+    q, k = run_tp(b, R, system_scope=True)
+    check_full(b, q, k)
+    assert qk.device_timeouts() == 0
+
+
 @pytest.mark.parametrize("R,Hq,Hk,dtype", [
     (1, 16384, 2048, torch.bfloat16),   # 2048 + 256 vectors per shard row: 64 per lane, in 16 batches
     (2, 8192, 1024, torch.float32),     # 2048 + 256 vectors per shard row
@@ -123,6 +148,43 @@ def test_tp_missing_rank_times_out_and_the_context_stays_usable():
     assert all(torch.all(q == 3.0) for q in qo)
     assert qk.device_timeouts() == 0  # reading cleared it
     q, k = run_tp(b, R, ex)
+    check_full(b, q, k)
+    assert qk.device_timeouts() == 0
+
+
+def test_tp_timeout_on_fresh_buffers_is_reported_again():
+    """An abort belongs to the receive buffers it happened on and that call's
+    epoch.  Ranks 0..2 of 4 time out at epoch 1 (code 4); a fresh exchange,
+    whose first call is epoch 1 again, repeats that incomplete call: its waits
+    must run out and report code 4 in turn -- not give up at once on the
+    earlier abort and report nothing.  A complete call on another fresh
+    exchange then matches the oracle, and one on the first exchange's next
+    epoch too."""
+    R = 4
+    b = _batch(64, 1024, 512, torch.bfloat16, seed=13)
+    qs, ks = _shards(b.q, R), _shards(b.k, R)
+    gq, gk = _gamma_shards(b.gamma_q, R), _gamma_shards(b.gamma_k, R)
+
+    def incomplete(ex):
+        sentinel = [torch.full_like(q, 3.0) for q in qs[:3]]
+        qo, _ = qk.qknorm_tp_layerwise(qs[:3], ks[:3], gq[:3], gk[:3], b.Hq, b.Hk, b.eps, exchange=ex, R=R,
+                                       first_rank=0, q_out=sentinel, timeout_ns=50_000_000)
+        torch.cuda.synchronize()
+        return qo
+
+    first = qk.TpExchange(R, b.T, DEV)
+    qo = incomplete(first)
+    assert first.epoch == 1 and qk.device_timeouts() == 4
+    assert all(torch.all(q == 3.0) for q in qo)
+    second = qk.TpExchange(R, b.T, DEV)
+    qo = incomplete(second)
+    assert second.epoch == 1
+    assert qk.device_timeouts() == 4, "the second exchange's waits gave up without reporting"
+    assert all(torch.all(q == 3.0) for q in qo)
+    assert qk.device_timeouts() == 0
+    q, k = run_tp(b, R, qk.TpExchange(R, b.T, DEV))
+    check_full(b, q, k)
+    q, k = run_tp(b, R, first)  # epoch 2 on the buffers that saw the abort
     check_full(b, q, k)
     assert qk.device_timeouts() == 0
 

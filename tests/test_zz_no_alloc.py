@@ -1,29 +1,46 @@
 """The allocation-free projection entry point, through the C-ABI.
 
-``qknorm_qkv_projection_noalloc`` serves callers that cannot allocate device
-memory (a host engine that owns every allocation, or a path that cannot take
-cudaMalloc's possible device synchronization): it keeps its partial sums in a
-fixed array inside the library instead of a caller-supplied workspace.  Its
-results must match ``qknorm_qkv_projection`` (same kernels, same order of
-operations), checked here within the 1-ulp tolerance the bf16 parity tests use
-on two calls in a row, the second smaller than the first so stale partial sums
-from the first call are still in the shared array.
+``qknorm_qkv_projection_noalloc`` is for callers that cannot allocate device
+memory: a serving engine that owns every device allocation and refuses new
+ones once it runs, or a latency-critical path on which cudaMalloc's possible
+device synchronization is not acceptable.  It keeps the partial sums in a
+fixed array inside the library instead of a caller-supplied workspace, and
+otherwise runs the same kernels in the same order as
+``qknorm_qkv_projection``.  So its output must equal that entry point's bit
+for bit.
 
-This file is named to be collected last.
+Two calls run in a row, the second smaller than the first, so the first
+call's partial sums are still in the shared array when the second runs.  The
+workspace entry point gets a workspace filled with NaN, so a partial sum that
+either path reads without having written it shows up as a difference.  Both
+calls are also checked against the oracle on sampled rows (projection and
+RMS-Norm, with the bounds of the projection tests).  The checks run twice: in
+this process, after whatever ran before, and in a fresh Python process whose
+first library call is this one.
+
+This file is collected last, so a run that stops at its first failure has
+run every other test first.
 """
 from __future__ import annotations
 
+import os
+import subprocess
+import sys
+
+import numpy as np
 import pytest
 import torch
 
 import attention_normalization_b200 as qk
 import workloads
 from attention_normalization_b200 import _clib
-from tests.conftest import bf16_ulp_distance, to_np
+from tests.conftest import to_np
+from tests.test_projection import _sample_rows, check_normalized, check_projection
 
 pytestmark = pytest.mark.gpu
 
 DEV = "cuda:0"
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
 def _noalloc(b: workloads.ProjectionBatch, x: torch.Tensor, w: torch.Tensor, qkv: torch.Tensor) -> int:
@@ -36,20 +53,41 @@ def _noalloc(b: workloads.ProjectionBatch, x: torch.Tensor, w: torch.Tensor, qkv
     return st
 
 
-def test_noalloc_matches_the_workspace_entry_point_on_two_calls():
+def run_two_calls() -> None:
+    """Two calls in a row, each bit-equal to qknorm_qkv_projection and within
+    the projection tests' bounds of the oracle on sampled rows."""
     lib = qk.capi()
     assert lib.qknorm_qkv_projection_noalloc_max_bytes() == 4 << 20
-    for b in (workloads.qkv_projection(T=2048, D=512, Hq=4096, Hk=1024, Hv=1024, seed=21),
-              workloads.qkv_projection(T=300, D=384, Hq=1024, Hk=512, Hv=256, seed=22)):
+    batches = (workloads.qkv_projection(T=2048, D=512, Hq=4096, Hk=1024, Hv=1024, seed=21),
+               workloads.qkv_projection(T=300, D=384, Hq=1024, Hk=512, Hv=256, seed=22))
+    for i, b in enumerate(batches):
         x, w = b.x.to(DEV), b.w.to(DEV)
         N = b.Hq + b.Hk + b.Hv
-        got = torch.empty((b.T, N), dtype=torch.bfloat16, device=DEV)
+        got = torch.full((b.T, N), float("nan"), dtype=torch.bfloat16, device=DEV)
         assert _noalloc(b, x, w, got) == _clib.QKN_OK, lib.qknorm_last_error().decode()
-        ref = qk.qknorm_qkv_projection(x, w, b.gamma_q.to(DEV), b.gamma_k.to(DEV), b.Hq, b.Hk, b.Hv, b.eps)
+        need = qk.qkv_workspace_bytes(b.T, b.Hq, b.Hk)
+        ws = torch.full(((need + 3) // 4,), float("nan"), dtype=torch.float32, device=DEV)
+        ref = qk.qknorm_qkv_projection(x, w, b.gamma_q.to(DEV), b.gamma_k.to(DEV), b.Hq, b.Hk, b.Hv, b.eps,
+                                       workspace=ws)
         torch.cuda.synchronize()
-        d = bf16_ulp_distance(to_np(got.cpu()), to_np(ref.cpu()))
-        assert d.max() <= 1, f"{b.name}: {int(d.max())} ulp from qknorm_qkv_projection"
-    assert qk.device_timeouts() == 0
+        assert qk.device_timeouts() == 0
+        g, r = to_np(got.cpu()), to_np(ref.cpu())
+        assert np.array_equal(g, r), (f"call {i + 1} ({b.name}): {int(np.sum(g != r))} elements differ from "
+                                      "qknorm_qkv_projection")
+        rows = _sample_rows(b.T, 24, seed=300 + i)
+        proj = check_projection(b, got, rows)
+        check_normalized(b, proj, got, rows)
+
+
+def test_noalloc_matches_the_workspace_entry_point_and_the_oracle_on_two_calls():
+    run_two_calls()
+
+
+def test_noalloc_in_a_fresh_process():
+    """The same two calls as the first library calls of a new process."""
+    r = subprocess.run([sys.executable, "-c", "import tests.test_zz_no_alloc as t; t.run_two_calls()"],
+                       cwd=ROOT, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stdout[-4000:] + r.stderr[-4000:]
 
 
 def test_noalloc_rejects_a_call_beyond_its_scratch():
