@@ -25,7 +25,9 @@ from . import _clib
 from ._clib import QknLaunch, QKNormError
 
 __all__ = ["qknorm_layerwise", "qknorm_headwise", "qknorm_qkv_gemm_stats", "qknorm_qkv_projection",
-           "qkv_workspace_bytes", "device_timeouts", "qknorm_tp_layerwise", "TpExchange", "TpPeerExchange", "qknorm_partial_stats", "qknorm_combine_apply", "gamma_dtype",
+           "qkv_workspace_bytes", "device_timeouts", "qknorm_tp_layerwise", "TpExchange", "TpPeerExchange",
+           "qknorm_partial_stats", "qknorm_combine_apply", "qknorm_partial_stats_shards",
+           "qknorm_combine_apply_shards", "gamma_dtype",
            "qknorm_layerwise_plan", "qknorm_layerwise_host", "qknorm_packed_host",
            "plan_shape", "plan_grid", "regions_overlap", "capi", "version", "QknLaunch", "QKNormError"]
 
@@ -460,6 +462,101 @@ def qknorm_combine_apply(q_in: torch.Tensor, k_in: torch.Tensor, gamma_q_shard: 
         else:
             st = capi().qknorm_combine_apply_launch(*args, s, ctypes.byref(_launch_struct(launch)))
     _clib.check(st, "qknorm_combine_apply")
+    return q_out, k_out
+
+
+def _ptr_array(xs):
+    P = ctypes.c_void_p
+    return (P * len(xs))(*[int(x) for x in xs])
+
+
+def _shard_list(ts, name):
+    if not isinstance(ts, (list, tuple)) or not ts:
+        raise ValueError(f"{name} must be a non-empty list of tensors, one per shard")
+    T, H, s = _rows(ts[0], f"{name}[0]")
+    for j, t in enumerate(ts):
+        _same(ts[0].device, ts[0].dtype, t, f"{name}[{j}]")
+        Tj, Hj, sj = _rows(t, f"{name}[{j}]")
+        if (Tj, Hj) != (T, H) or (T > 1 and sj != s):
+            raise ValueError(f"{name}: every shard must have the same shape and row stride")
+    return T, H, s
+
+
+def _sums_all(t, name, P, T, dev):
+    if t is None:
+        return torch.empty((P, T), dtype=torch.float32, device=dev)
+    if not (isinstance(t, torch.Tensor) and t.is_cuda and t.device == dev and t.dtype == torch.float32
+            and t.is_contiguous() and tuple(t.shape) == (P, T)):
+        raise ValueError(f"{name} must be a contiguous float32 CUDA tensor of shape [{P}, {T}]")
+    return t
+
+
+def qknorm_partial_stats_shards(q_shards, k_shards, q_sumsq_all=None, k_sumsq_all=None, *, stream=None):
+    """Phase A local step for P shards of Q and of K in one launch: row p of
+    the returned ``[P, T]`` float32 arrays ``(q_sumsq_all, k_sumsq_all)``
+    holds the squared sums of shard p, exactly what P calls of
+    ``qknorm_partial_stats`` would write."""
+    P = len(q_shards)
+    if len(k_shards) != P:
+        raise ValueError("one K shard per Q shard")
+    T, hq, sq = _shard_list(q_shards, "q_shards")
+    Tk, hk, sk = _shard_list(k_shards, "k_shards")
+    dev, dt = q_shards[0].device, q_shards[0].dtype
+    _same(dev, dt, k_shards[0], "k_shards[0]")
+    if T != Tk:
+        raise ValueError("Q and K shards must have the same number of tokens")
+    q_sumsq_all = _sums_all(q_sumsq_all, "q_sumsq_all", P, T, dev)
+    k_sumsq_all = _sums_all(k_sumsq_all, "k_sumsq_all", P, T, dev)
+    with _on(dev):
+        st = capi().qknorm_partial_stats_shards(P, _ptr_array([t.data_ptr() for t in q_shards]), sq, hq,
+                                                q_sumsq_all.data_ptr(), _ptr_array([t.data_ptr() for t in k_shards]),
+                                                sk, hk, k_sumsq_all.data_ptr(), T, _DTYPES[dt],
+                                                _stream_handle(stream, dev))
+    _clib.check(st, "qknorm_partial_stats_shards")
+    return q_sumsq_all, k_sumsq_all
+
+
+def qknorm_combine_apply_shards(q_in, k_in, gamma_q_shards, gamma_k_shards, q_sumsq_all: torch.Tensor,
+                                k_sumsq_all: torch.Tensor, Hq_full: int, Hk_full: int, eps: float = 1e-6, *,
+                                q_out=None, k_out=None, stream=None):
+    """Phase A aggregation and Phase B for P shards of Q and of K in one
+    launch: the same results as P calls of ``qknorm_combine_apply`` with the
+    same ``[P, T]`` partial sums.  Returns the lists ``(q_out, k_out)``."""
+    P = len(q_in)
+    if not (len(k_in) == len(gamma_q_shards) == len(gamma_k_shards) == P):
+        raise ValueError("one K shard and one gamma slice of each tensor per Q shard")
+    T, hq, sq = _shard_list(q_in, "q_in")
+    Tk, hk, sk = _shard_list(k_in, "k_in")
+    dev, dt = q_in[0].device, q_in[0].dtype
+    _same(dev, dt, k_in[0], "k_in[0]")
+    if T != Tk:
+        raise ValueError("Q and K shards must have the same number of tokens")
+    for t, name in ((q_sumsq_all, "q_sumsq_all"), (k_sumsq_all, "k_sumsq_all")):
+        _sums_all(t, name, P, T, dev)
+    if q_out is None:
+        q_out = [_out_like(t, sq) for t in q_in]
+    if k_out is None:
+        k_out = [_out_like(t, sk) for t in k_in]
+    if len(q_out) != P or len(k_out) != P:
+        raise ValueError("one output per shard")
+    for outs, name, (H, s) in ((q_out, "q_out", (hq, sq)), (k_out, "k_out", (hk, sk))):
+        for j, t in enumerate(outs):
+            _same(dev, dt, t, f"{name}[{j}]")
+            To, Ho, so = _rows(t, f"{name}[{j}]")
+            if (To, Ho) != (T, H) or (T > 1 and so != s):
+                raise ValueError(f"{name}[{j}] must match its input's shape and row stride")
+    gdt = gamma_dtype(dt)
+    gq = [_vec(g, f"gamma_q_shards[{j}]", hq, gdt, dev) for j, g in enumerate(gamma_q_shards)]
+    gk = [_vec(g, f"gamma_k_shards[{j}]", hk, gdt, dev) for j, g in enumerate(gamma_k_shards)]
+    with _on(dev):
+        st = capi().qknorm_combine_apply_shards(P, _ptr_array([t.data_ptr() for t in q_in]),
+                                                _ptr_array([t.data_ptr() for t in q_out]), _ptr_array(gq), sq, hq,
+                                                q_sumsq_all.data_ptr(), int(Hq_full),
+                                                _ptr_array([t.data_ptr() for t in k_in]),
+                                                _ptr_array([t.data_ptr() for t in k_out]), _ptr_array(gk), sk, hk,
+                                                k_sumsq_all.data_ptr(), int(Hk_full), T, float(eps), _DTYPES[dt],
+                                                _stream_handle(stream, dev))
+    _clib.check(st, "qknorm_combine_apply_shards")
     return q_out, k_out
 
 

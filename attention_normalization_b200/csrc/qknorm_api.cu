@@ -189,48 +189,65 @@ qkn_status blocks_per_sm(const void *fn, int dev, int threads, int64_t dyn_smem,
 
 // ---------------------------------------------------------------------------
 // Kernel selection.
-template <typename E, int MODE, bool TAIL>
+template <typename E, int MODE, bool TAIL, int SETS>
 const void *register_kernel(int nv) {
     switch (nv) {
-        case 1: return (const void *)qkn::rows_register_kernel<E, 1, MODE, TAIL>;
-        case 2: return (const void *)qkn::rows_register_kernel<E, 2, MODE, TAIL>;
-        case 4: return (const void *)qkn::rows_register_kernel<E, 4, MODE, TAIL>;
-        case 8: return (const void *)qkn::rows_register_kernel<E, 8, MODE, TAIL>;
+        case 1: return (const void *)qkn::rows_register_kernel<E, 1, MODE, TAIL, SETS>;
+        case 2: return (const void *)qkn::rows_register_kernel<E, 2, MODE, TAIL, SETS>;
+        case 4: return (const void *)qkn::rows_register_kernel<E, 4, MODE, TAIL, SETS>;
+        case 8: return (const void *)qkn::rows_register_kernel<E, 8, MODE, TAIL, SETS>;
         default: return nullptr;
     }
 }
 
-template <typename E, int MODE>
+// The two-pass kernels take one Q and one K row set only; multi-shard calls
+// (SETS > 2) run the register kernel.
+template <typename E, int MODE, int SETS>
 const void *kernel_for(const qkn_launch &L, bool tail) {
     switch (L.kernel) {
         case QKN_KERNEL_REGISTER:
-            return tail ? register_kernel<E, MODE, true>(L.vec_per_thread)
-                        : register_kernel<E, MODE, false>(L.vec_per_thread);
-        case QKN_KERNEL_TWOPASS_VEC: return (const void *)qkn::rows_twopass_kernel<E, true, MODE>;
-        case QKN_KERNEL_TWOPASS_SCALAR: return (const void *)qkn::rows_twopass_kernel<E, false, MODE>;
+            return tail ? register_kernel<E, MODE, true, SETS>(L.vec_per_thread)
+                        : register_kernel<E, MODE, false, SETS>(L.vec_per_thread);
+        case QKN_KERNEL_TWOPASS_VEC:
+            if constexpr (SETS == 2) return (const void *)qkn::rows_twopass_kernel<E, true, MODE>;
+            return nullptr;
+        case QKN_KERNEL_TWOPASS_SCALAR:
+            if constexpr (SETS == 2) return (const void *)qkn::rows_twopass_kernel<E, false, MODE>;
+            return nullptr;
         default: return nullptr;
     }
 }
 
-template <int MODE>
+template <int MODE, int SETS = 2>
 const void *kernel_for(qkn_dtype dt, const qkn_launch &L, bool tail) {
     switch (dt) {
-        case QKN_F32: return kernel_for<float, MODE>(L, tail);
-        case QKN_BF16: return kernel_for<__nv_bfloat16, MODE>(L, tail);
-        case QKN_F16: return kernel_for<__half, MODE>(L, tail);
-        case QKN_FP8_E4M3: return kernel_for<__nv_fp8_e4m3, MODE>(L, tail);
+        case QKN_F32: return kernel_for<float, MODE, SETS>(L, tail);
+        case QKN_BF16: return kernel_for<__nv_bfloat16, MODE, SETS>(L, tail);
+        case QKN_F16: return kernel_for<__half, MODE, SETS>(L, tail);
+        case QKN_FP8_E4M3: return kernel_for<__nv_fp8_e4m3, MODE, SETS>(L, tail);
         default: return nullptr;
     }
 }
 
 // A prepared call: parameters plus the facts planning needs.
-struct Call {
-    qkn::Params p;
+template <int SETS>
+struct CallT {
+    qkn::ParamsT<SETS> p;
     qkn_dtype dtype;
     bool vectorized;
     bool tail;          // some row ends in a partial 16-byte vector
     int64_t units_max;  // widest row in vectors (vectorized) or elements
 };
+using Call = CallT<2>;
+using ShardCall = CallT<qkn::kMaxShardSets>;
+
+// Zeroed call with `nsets` row sets in use.
+template <int SETS>
+void init_call(CallT<SETS> &c, qkn_dtype dtype, int nsets) {
+    std::memset(&c, 0, sizeof(c));
+    c.dtype = dtype;
+    c.p.nsets = nsets;
+}
 
 void fill_rowset(qkn::RowSet &s, const void *in, void *out, const void *gamma, int64_t stride, int32_t width,
                  int32_t div_width, int esz) {
@@ -250,28 +267,39 @@ void fill_rowset(qkn::RowSet &s, const void *in, void *out, const void *gamma, i
     s.rows = 0;
 }
 
+// Rows per set, and whether every set moves as 16-byte vectors (`aligned`:
+// the caller's pointers and strides allow it), the widest row, any tail.
+template <int SETS>
+void finish_sets(CallT<SETS> &c, int esz, bool aligned) {
+    bool v = aligned;
+    int64_t w = 0;
+    c.tail = false;
+    for (int i = 0; i < c.p.nsets; ++i) {
+        qkn::RowSet &d = c.p.set[i];
+        d.rows = c.p.T * d.heads;
+        if (d.heads > 1 && d.head_bytes % 16 != 0) v = false;  // every head must start on a vector
+        if (d.width > w) w = d.width;
+        if (d.tail) c.tail = true;
+    }
+    c.vectorized = v;
+    const int per_vec = 16 / esz;
+    c.units_max = v ? (w + per_vec - 1) / per_vec : w;
+}
+
 void finish_call(Call &c, int esz, std::initializer_list<const void *> ptrs, int64_t q_stride, int64_t k_stride) {
     bool v = ((q_stride * esz) % 16 == 0) && ((k_stride * esz) % 16 == 0);
     for (const void *p : ptrs)
         if (p && !aligned16(p)) v = false;
-    for (int w = 0; w < 2; ++w) {
-        qkn::RowSet &d = c.p.set[w];
-        d.rows = c.p.T * d.heads;
-        if (d.heads > 1 && d.head_bytes % 16 != 0) v = false;  // every head must start on a vector
-    }
-    c.vectorized = v;
-    const int per_vec = 16 / esz;
-    int64_t wq = c.p.set[0].width, wk = c.p.set[1].width;
-    int64_t w = wq > wk ? wq : wk;
-    c.units_max = v ? (w + per_vec - 1) / per_vec : w;
-    c.tail = c.p.set[0].tail != 0 || c.p.set[1].tail != 0;
+    finish_sets(c, esz, v);
 }
 
 // Row groups of the register kernel for a launch of `threads` threads with
 // `nv` vectors each: the smallest group (a multiple of 32 dividing the CTA)
-// whose threads cover the tensor's row, and the items that follow.
-void set_groups(qkn::Params &p, int threads, int nv) {
-    for (int w = 0; w < 2; ++w) {
+// whose threads cover the set's row, and the items that follow.
+template <int SETS>
+void set_groups(qkn::ParamsT<SETS> &p, int threads, int nv) {
+    int64_t end = 0;
+    for (int w = 0; w < p.nsets; ++w) {
         qkn::RowSet &d = p.set[w];
         const int64_t units = (int64_t)d.nfull + (d.tail ? 1 : 0);
         int group = threads;
@@ -283,7 +311,10 @@ void set_groups(qkn::Params &p, int threads, int nv) {
         d.group = group;
         d.rows_per_item = threads / group;
         d.items = (d.rows + d.rows_per_item - 1) / d.rows_per_item;
+        end += d.items;
+        d.item_end = end;
     }
+    p.n_items = end;
 }
 
 bool eps_valid(float eps) { return std::isfinite(eps) && eps >= 0.0f; }
@@ -347,8 +378,7 @@ qkn_status prepare_layerwise(const void *q_in, void *q_out, const void *gamma_q,
         qkn_status st = check_outputs(oq, ok_, iq, ik, others, 2);
         if (st != QKN_OK) return st;
     }
-    std::memset(&c, 0, sizeof(c));
-    c.dtype = dtype;
+    init_call(c, dtype, 2);
     fill_rowset(c.p.set[0], q_in, q_out, gamma_q, q_stride, Hq, Hq, esz);
     fill_rowset(c.p.set[1], k_in, k_out, gamma_k, k_stride, Hk, Hk, esz);
     c.p.T = T;
@@ -359,13 +389,14 @@ qkn_status prepare_layerwise(const void *q_in, void *q_out, const void *gamma_q,
     return QKN_OK;
 }
 
-template <int MODE>
-qkn_status plan_call(const Call &c, qkn_launch &L) {
+template <int MODE, int SETS>
+qkn_status plan_call(const CallT<SETS> &c, qkn_launch &L) {
     int dev = 0, sms = 0, bps = 0;
     qkn_status st = current_device(&dev);
     if (st != QKN_OK) return st;
     if ((st = sm_count(dev, &sms)) != QKN_OK) return st;
-    const int64_t items = c.p.set[0].rows + c.p.set[1].rows;
+    int64_t items = 0;
+    for (int i = 0; i < c.p.nsets; ++i) items += c.p.set[i].rows;
     if ((st = qknorm_plan_shape(items, c.units_max, c.vectorized ? 1 : 0, sms, elem_bytes(c.dtype), &L)) !=
         QKN_OK)
         return fail(st, "planning failed");
@@ -381,20 +412,21 @@ qkn_status plan_call(const Call &c, qkn_launch &L) {
             L.threads = 128;
         }
     }
-    const void *fn = kernel_for<MODE>(c.dtype, L, c.tail);
+    const void *fn = kernel_for<MODE, SETS>(c.dtype, L, c.tail);
     if (!fn) return fail(QKN_ERR_UNSUPPORTED, "no kernel for the planned launch");
     if ((st = blocks_per_sm(fn, dev, L.threads, 0, &bps)) != QKN_OK) return st;
     int64_t work = items;
     if (L.kernel == QKN_KERNEL_REGISTER) {  // narrow rows share CTAs: count items, not rows
-        qkn::Params p = c.p;
+        qkn::ParamsT<SETS> p = c.p;
         set_groups(p, L.threads, L.vec_per_thread);
-        work = p.set[0].items + p.set[1].items;
+        work = p.n_items;
     }
     L.grid = qknorm_plan_grid(work, bps, sms);
     return QKN_OK;
 }
 
-qkn_status check_launch(const Call &c, const qkn_launch &L) {
+template <int SETS>
+qkn_status check_launch(const CallT<SETS> &c, const qkn_launch &L) {
     if (L.threads < 32 || L.threads > 1024 || (L.threads % 32) != 0)
         return fail(QKN_ERR_INVALID_ARG, "threads must be a multiple of 32 in [32, 1024], got %d", L.threads);
     if (L.grid < 1 || L.grid > 2147483647LL) return fail(QKN_ERR_INVALID_ARG, "grid out of range");
@@ -420,8 +452,8 @@ qkn_status check_launch(const Call &c, const qkn_launch &L) {
 // Every launch allows programmatic dependent launch: the kernel may be
 // dispatched while the previous kernel in the stream drains (see
 // pdl_wait_and_release in the kernels, which restores the ordering).
-cudaError_t launch_pdl(const void *fn, unsigned grid, unsigned block, size_t smem, cudaStream_t s,
-                       const qkn::Params &p) {
+template <typename P>
+cudaError_t launch_pdl(const void *fn, unsigned grid, unsigned block, size_t smem, cudaStream_t s, const P &p) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(block);
@@ -432,22 +464,22 @@ cudaError_t launch_pdl(const void *fn, unsigned grid, unsigned block, size_t sme
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    void *args[] = {const_cast<qkn::Params *>(&p)};
+    void *args[] = {const_cast<P *>(&p)};
     return cudaLaunchKernelExC(&cfg, fn, args);
 }
 
-template <int MODE>
-cudaError_t launch_any(const qkn_launch &L, const Call &c, cudaStream_t s) {
-    const void *fn = kernel_for<MODE>(c.dtype, L, c.tail);
+template <int MODE, int SETS>
+cudaError_t launch_any(const qkn_launch &L, const CallT<SETS> &c, cudaStream_t s) {
+    const void *fn = kernel_for<MODE, SETS>(c.dtype, L, c.tail);
     if (!fn) return cudaErrorInvalidValue;
-    qkn::Params p = c.p;
+    qkn::ParamsT<SETS> p = c.p;
     if (L.kernel == QKN_KERNEL_REGISTER) set_groups(p, L.threads, L.vec_per_thread);
     return launch_pdl(fn, (unsigned)L.grid, (unsigned)L.threads, 0, s, p);
 }
 
-template <int MODE>
-qkn_status launch(const Call &c, const qkn_launch &L, void *stream) {
-    cudaError_t e = launch_any<MODE>(L, c, static_cast<cudaStream_t>(stream));
+template <int MODE, int SETS>
+qkn_status launch(const CallT<SETS> &c, const qkn_launch &L, void *stream) {
+    cudaError_t e = launch_any<MODE, SETS>(L, c, static_cast<cudaStream_t>(stream));
     if (e == cudaSuccess) e = cudaGetLastError();
     if (e != cudaSuccess) return fail(QKN_ERR_CUDA, "kernel launch: %s", cudaGetErrorString(e));
     return ok();
@@ -472,8 +504,7 @@ qkn_status prepare_stats(const void *q_shard, int64_t q_stride, int32_t hq_shard
         if (overlap(sq, iq) || overlap(sq, ik) || overlap(sk, iq) || overlap(sk, ik))
             return fail(QKN_ERR_INVALID_ARG, "a sum array overlaps an input");
     }
-    std::memset(&c, 0, sizeof(c));
-    c.dtype = dtype;
+    init_call(c, dtype, 2);
     fill_rowset(c.p.set[0], q_shard, nullptr, nullptr, q_stride, hq_shard, hq_shard, esz);
     fill_rowset(c.p.set[1], k_shard, nullptr, nullptr, k_stride, hk_shard, hk_shard, esz);
     c.p.set[0].sumsq = q_sumsq;
@@ -517,8 +548,7 @@ qkn_status prepare_apply(const void *q_in, void *q_out, const void *gamma_q_shar
         qkn_status st = check_outputs(oq, ok_, iq, ik, others, 4);
         if (st != QKN_OK) return st;
     }
-    std::memset(&c, 0, sizeof(c));
-    c.dtype = dtype;
+    init_call(c, dtype, 2);
     fill_rowset(c.p.set[0], q_in, q_out, gamma_q_shard, q_stride, hq_shard, Hq_full, esz);
     fill_rowset(c.p.set[1], k_in, k_out, gamma_k_shard, k_stride, hk_shard, Hk_full, esz);
     c.p.set[0].sumsq_all = q_sumsq_all;
@@ -530,6 +560,132 @@ qkn_status prepare_apply(const void *q_in, void *q_out, const void *gamma_q_shar
     finish_call(c, esz, {q_in, q_out, gamma_q_shard, k_in, k_out, gamma_k_shard}, q_stride, k_stride);
     return QKN_OK;
 }
+
+// Multi-shard forms: P shards of Q and P of K, each shard's rows in its own
+// buffer (same width and stride for every shard of a tensor), in one launch.
+qkn_status check_shard_common(int32_t P, int64_t T, int32_t hq_shard, int32_t hk_shard, int64_t q_stride,
+                              int64_t k_stride, qkn_dtype dtype) {
+    if (!dtype_valid(dtype)) return fail(QKN_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
+    if (P < 1 || P > qkn::kMaxShards) return fail(QKN_ERR_INVALID_ARG, "P = %d outside [1, %d]", P, qkn::kMaxShards);
+    if (T < 0) return fail(QKN_ERR_INVALID_ARG, "T = %lld < 0", (long long)T);
+    if (hq_shard <= 0 || hk_shard <= 0) return fail(QKN_ERR_INVALID_ARG, "shard widths must be positive");
+    if (q_stride < hq_shard || k_stride < hk_shard) return fail(QKN_ERR_INVALID_ARG, "row stride below shard width");
+    const int esz = elem_bytes(dtype);
+    if (!extent_ok(T, q_stride, hq_shard, esz) || !extent_ok(T, k_stride, hk_shard, esz) ||
+        !extent_ok(1, 0, (int64_t)P * T, 4))
+        return fail(QKN_ERR_INVALID_ARG, "buffer extent overflows");
+    return QKN_OK;
+}
+
+bool shard_ptrs_aligned(const void *const *a, int P) {
+    for (int p = 0; p < P; ++p)
+        if (!aligned16(a[p])) return false;
+    return true;
+}
+
+qkn_status prepare_stats_shards(int32_t P, const void *const *q_shards, int64_t q_stride, int32_t hq_shard,
+                                float *q_sumsq_all, const void *const *k_shards, int64_t k_stride, int32_t hk_shard,
+                                float *k_sumsq_all, int64_t T, qkn_dtype dtype, ShardCall &c) {
+    qkn_status st = check_shard_common(P, T, hq_shard, hk_shard, q_stride, k_stride, dtype);
+    if (st != QKN_OK) return st;
+    const int esz = elem_bytes(dtype);
+    if (T > 0) {
+        if (!q_shards || !k_shards || !q_sumsq_all || !k_sumsq_all) return fail(QKN_ERR_INVALID_ARG, "null pointer");
+        for (int p = 0; p < P; ++p)
+            if (!q_shards[p] || !k_shards[p]) return fail(QKN_ERR_INVALID_ARG, "null shard pointer %d", p);
+        const Region sq = flat_region(q_sumsq_all, (int64_t)P * T * 4), sk = flat_region(k_sumsq_all, (int64_t)P * T * 4);
+        if (overlap(sq, sk)) return fail(QKN_ERR_INVALID_ARG, "q_sumsq_all and k_sumsq_all overlap");
+        for (int p = 0; p < P; ++p) {
+            const Region iq = rows_region(q_shards[p], hq_shard, q_stride, T, esz);
+            const Region ik = rows_region(k_shards[p], hk_shard, k_stride, T, esz);
+            if (overlap(sq, iq) || overlap(sq, ik) || overlap(sk, iq) || overlap(sk, ik))
+                return fail(QKN_ERR_INVALID_ARG, "a sum array overlaps shard %d", p);
+        }
+    }
+    init_call(c, dtype, 2 * P);
+    for (int p = 0; p < P && T > 0; ++p) {
+        qkn::RowSet &dq = c.p.set[p], &dk = c.p.set[P + p];
+        fill_rowset(dq, q_shards[p], nullptr, nullptr, q_stride, hq_shard, hq_shard, esz);
+        fill_rowset(dk, k_shards[p], nullptr, nullptr, k_stride, hk_shard, hk_shard, esz);
+        dq.sumsq = q_sumsq_all + (int64_t)p * T;
+        dk.sumsq = k_sumsq_all + (int64_t)p * T;
+        dq.P = dk.P = 1;
+    }
+    c.p.T = T;
+    c.p.eps = 0.0f;
+    if (T > 0)
+        finish_sets(c, esz, (q_stride * esz) % 16 == 0 && (k_stride * esz) % 16 == 0 &&
+                                shard_ptrs_aligned(q_shards, P) && shard_ptrs_aligned(k_shards, P));
+    return QKN_OK;
+}
+
+qkn_status prepare_apply_shards(int32_t P, const void *const *q_in, void *const *q_out,
+                                const void *const *gamma_q_shards, int64_t q_stride, int32_t hq_shard,
+                                const float *q_sumsq_all, int32_t Hq_full, const void *const *k_in,
+                                void *const *k_out, const void *const *gamma_k_shards, int64_t k_stride,
+                                int32_t hk_shard, const float *k_sumsq_all, int32_t Hk_full, int64_t T, float eps,
+                                qkn_dtype dtype, ShardCall &c) {
+    qkn_status st = check_shard_common(P, T, hq_shard, hk_shard, q_stride, k_stride, dtype);
+    if (st != QKN_OK) return st;
+    if (Hq_full < hq_shard || Hk_full < hk_shard) return fail(QKN_ERR_INVALID_ARG, "full width below shard width");
+    if (!eps_valid(eps)) return fail(QKN_ERR_INVALID_ARG, "eps must be finite and >= 0");
+    const int esz = elem_bytes(dtype);
+    const int gsz = gamma_bytes(dtype);
+    if (T > 0) {
+        if (!q_in || !q_out || !gamma_q_shards || !k_in || !k_out || !gamma_k_shards || !q_sumsq_all || !k_sumsq_all)
+            return fail(QKN_ERR_INVALID_ARG, "null pointer");
+        for (int p = 0; p < P; ++p)
+            if (!q_in[p] || !q_out[p] || !gamma_q_shards[p] || !k_in[p] || !k_out[p] || !gamma_k_shards[p])
+                return fail(QKN_ERR_INVALID_ARG, "null pointer for shard %d", p);
+        // every output against everything else of every shard (its own input
+        // only when identical: in place)
+        for (int p = 0; p < P; ++p) {
+            const Region oq = rows_region(q_out[p], hq_shard, q_stride, T, esz);
+            const Region ok_ = rows_region(k_out[p], hk_shard, k_stride, T, esz);
+            for (int o = 0; o < P; ++o) {
+                const Region iq = rows_region(q_in[o], hq_shard, q_stride, T, esz);
+                const Region ik = rows_region(k_in[o], hk_shard, k_stride, T, esz);
+                const Region others[4] = {flat_region(gamma_q_shards[o], (int64_t)hq_shard * gsz),
+                                          flat_region(gamma_k_shards[o], (int64_t)hk_shard * gsz),
+                                          flat_region(q_sumsq_all, (int64_t)P * T * 4),
+                                          flat_region(k_sumsq_all, (int64_t)P * T * 4)};
+                if (o == p) {
+                    if ((st = check_outputs(oq, ok_, iq, ik, others, 4)) != QKN_OK) return st;
+                    continue;
+                }
+                const Region oq2 = rows_region(q_out[o], hq_shard, q_stride, T, esz);
+                const Region ok2 = rows_region(k_out[o], hk_shard, k_stride, T, esz);
+                const Region all[8] = {iq, ik, oq2, ok2, others[0], others[1], others[2], others[3]};
+                for (const Region &r : all)
+                    if (overlap(oq, r) || overlap(ok_, r))
+                        return fail(QKN_ERR_INVALID_ARG, "an output of shard %d overlaps an operand of shard %d", p, o);
+            }
+        }
+    }
+    init_call(c, dtype, 2 * P);
+    for (int p = 0; p < P && T > 0; ++p) {
+        qkn::RowSet &dq = c.p.set[p], &dk = c.p.set[P + p];
+        fill_rowset(dq, q_in[p], q_out[p], gamma_q_shards[p], q_stride, hq_shard, Hq_full, esz);
+        fill_rowset(dk, k_in[p], k_out[p], gamma_k_shards[p], k_stride, hk_shard, Hk_full, esz);
+        dq.sumsq_all = q_sumsq_all;
+        dk.sumsq_all = k_sumsq_all;
+        dq.P = dk.P = P;
+    }
+    c.p.T = T;
+    c.p.eps = eps;
+    if (T > 0) {
+        bool v = (q_stride * esz) % 16 == 0 && (k_stride * esz) % 16 == 0;
+        for (const void *const *a : {q_in, (const void *const *)q_out, gamma_q_shards, k_in,
+                                     (const void *const *)k_out, gamma_k_shards})
+            v = v && shard_ptrs_aligned(a, P);
+        finish_sets(c, esz, v);
+    }
+    return QKN_OK;
+}
+
+// A multi-shard call runs as one launch of the register kernel when its rows
+// allow it (16-byte aligned, at most 32 KB); otherwise shard by shard.
+bool one_launch(const ShardCall &c) { return c.vectorized && c.units_max <= 2048; }
 
 qkn_status prepare_headwise(const void *q_in, void *q_out, const void *gamma_q, int64_t q_stride, int32_t q_heads,
                             const void *k_in, void *k_out, const void *gamma_k, int64_t k_stride, int32_t k_heads,
@@ -560,8 +716,7 @@ qkn_status prepare_headwise(const void *q_in, void *q_out, const void *gamma_q, 
         qkn_status st = check_outputs(oq, ok_, iq, ik, others, 2);
         if (st != QKN_OK) return st;
     }
-    std::memset(&c, 0, sizeof(c));
-    c.dtype = dtype;
+    init_call(c, dtype, 2);
     fill_rowset(c.p.set[0], q_in, q_out, gamma_q, q_stride, head_dim, head_dim, esz);
     fill_rowset(c.p.set[1], k_in, k_out, gamma_k, k_stride, head_dim, head_dim, esz);
     c.p.set[0].heads = q_heads;
@@ -966,6 +1121,53 @@ qkn_status qknorm_combine_apply_launch(const void *q_in, void *q_out, const void
     return launch<qkn::kApply>(c, *launch_cfg, stream);
 }
 
+qkn_status qknorm_partial_stats_shards(int32_t P, const void *const *q_shards, int64_t q_stride, int32_t hq_shard,
+                                       float *q_sumsq_all, const void *const *k_shards, int64_t k_stride,
+                                       int32_t hk_shard, float *k_sumsq_all, int64_t T, qkn_dtype dtype,
+                                       void *stream) {
+    ShardCall c;
+    qkn_status st = prepare_stats_shards(P, q_shards, q_stride, hq_shard, q_sumsq_all, k_shards, k_stride, hk_shard,
+                                         k_sumsq_all, T, dtype, c);
+    if (st != QKN_OK) return st;
+    if (T == 0) return ok();
+    if (!one_launch(c)) {
+        for (int p = 0; p < P; ++p)
+            if ((st = qknorm_partial_stats(q_shards[p], q_stride, hq_shard, q_sumsq_all + (int64_t)p * T, k_shards[p],
+                                           k_stride, hk_shard, k_sumsq_all + (int64_t)p * T, T, dtype, stream)) !=
+                QKN_OK)
+                return st;
+        return ok();
+    }
+    qkn_launch L;
+    if ((st = plan_call<qkn::kStats>(c, L)) != QKN_OK) return st;
+    return launch<qkn::kStats>(c, L, stream);
+}
+
+qkn_status qknorm_combine_apply_shards(int32_t P, const void *const *q_in, void *const *q_out,
+                                       const void *const *gamma_q_shards, int64_t q_stride, int32_t hq_shard,
+                                       const float *q_sumsq_all, int32_t Hq_full, const void *const *k_in,
+                                       void *const *k_out, const void *const *gamma_k_shards, int64_t k_stride,
+                                       int32_t hk_shard, const float *k_sumsq_all, int32_t Hk_full, int64_t T,
+                                       float eps, qkn_dtype dtype, void *stream) {
+    ShardCall c;
+    qkn_status st = prepare_apply_shards(P, q_in, q_out, gamma_q_shards, q_stride, hq_shard, q_sumsq_all, Hq_full,
+                                         k_in, k_out, gamma_k_shards, k_stride, hk_shard, k_sumsq_all, Hk_full, T, eps,
+                                         dtype, c);
+    if (st != QKN_OK) return st;
+    if (T == 0) return ok();
+    if (!one_launch(c)) {
+        for (int p = 0; p < P; ++p)
+            if ((st = qknorm_combine_apply(q_in[p], q_out[p], gamma_q_shards[p], q_stride, hq_shard, q_sumsq_all,
+                                           Hq_full, k_in[p], k_out[p], gamma_k_shards[p], k_stride, hk_shard,
+                                           k_sumsq_all, Hk_full, P, T, eps, dtype, stream)) != QKN_OK)
+                return st;
+        return ok();
+    }
+    qkn_launch L;
+    if ((st = plan_call<qkn::kApply>(c, L)) != QKN_OK) return st;
+    return launch<qkn::kApply>(c, L, stream);
+}
+
 qkn_status qknorm_qkv_gemm_stats(const void *x, int64_t x_stride, const void *w, int64_t w_stride, void *qkv,
                                  int64_t qkv_stride, int64_t T, int32_t D, int32_t Hq, int32_t Hk, int32_t Hv,
                                  float *q_sumsq_all, float *k_sumsq_all, qkn_dtype dtype, void *stream) {
@@ -1022,8 +1224,7 @@ qkn_status qknorm_qkv_projection(const void *x, int64_t x_stride, const void *w,
     // Otherwise a second launch: Phase A aggregation + Phase B over the Q and
     // K columns of qkv, in place.
     Call c;
-    std::memset(&c, 0, sizeof(c));
-    c.dtype = dtype;
+    init_call(c, dtype, 2);
     char *kcols = static_cast<char *>(qkv) + (int64_t)Hq * 2;
     fill_rowset(c.p.set[0], qkv, qkv, gamma_q, qkv_stride, Hq, Hq, 2);
     fill_rowset(c.p.set[1], kcols, kcols, gamma_k, qkv_stride, Hk, Hk, 2);

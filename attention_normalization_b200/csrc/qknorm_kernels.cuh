@@ -51,13 +51,24 @@ struct RowSet {
     int32_t group;           // register kernel: threads that share one row (1..16, or a multiple of 32)
     int32_t rows_per_item;   // register kernel: blockDim / group rows handled per item
     int64_t items;           // register kernel: ceil(rows / rows_per_item)
+    int64_t item_end;        // register kernel: items of this set and of every set before it
 };
 
-struct Params {
-    RowSet set[2];           // 0 = Q, 1 = K
+// The row sets of one launch: Q then K (SETS = 2), or -- for the multi-shard
+// forms of Phase A's local step and of the combine/apply -- the P Q shards
+// then the P K shards (SETS = kMaxShardSets, nsets = 2P of them in use).
+template <int SETS>
+struct ParamsT {
+    RowSet set[SETS];
+    int32_t nsets;           // sets in use
+    int64_t n_items;         // register kernel: items over all sets in use
     int64_t T;
     float eps;
 };
+using Params = ParamsT<2>;   // 0 = Q, 1 = K
+constexpr int kMaxShards = 8;
+constexpr int kMaxShardSets = 2 * kMaxShards;
+using ShardParams = ParamsT<kMaxShardSets>;
 
 // ----------------------------------------------------------------------------
 // Packed fp32 pairs.  sm_100 executes add/mul/fma on two fp32 lanes held in
@@ -446,9 +457,10 @@ __device__ __forceinline__ uint4 scale_vec(const uint4 &xv, const uint4 (&gv)[El
 // `group` threads -- 1, 2, 4, 8 or 16 lanes of a warp, or a multiple of 32
 // that divides the CTA; a CTA of blockDim threads therefore handles
 // rows_per_item = blockDim / group consecutive rows of one tensor per item.
-// Items are the Q row-groups followed by the K row-groups, and CTA c takes
-// items c, c + grid, ...: every CTA gets a near-equal share of each tensor's
-// rows whatever the grid.  Lane l of a group owns vectors l, l + group, ...
+// Items are the Q row-groups followed by the K row-groups (in a multi-shard
+// launch: the row-groups of each Q shard, then of each K shard), and CTA c
+// takes items c, c + grid, ...: every CTA gets a near-equal share of each
+// tensor's rows whatever the grid.  Lane l of a group owns vectors l, l + group, ...
 // (up to NV) of its row -- the same positions in every row -- so while
 // consecutive items belong to one tensor a thread keeps that tensor's
 // parameters and its gamma vectors in registers.  All loads of a row are
@@ -463,9 +475,9 @@ struct RegisterBounds {
     static constexpr int kMaxThreads = NV <= 2 ? 1024 : (NV == 4 ? 512 : 256);
 };
 
-template <typename E, int NV, int MODE, bool TAIL>
+template <typename E, int NV, int MODE, bool TAIL, int SETS>
 __global__ void __launch_bounds__(RegisterBounds<NV>::kMaxThreads)
-    rows_register_kernel(const __grid_constant__ Params p) {
+    rows_register_kernel(const __grid_constant__ ParamsT<SETS> p) {
     constexpr int KG = Elem<E>::kGVecs;
     __shared__ float red[2][32];
     pdl_wait_and_release();
@@ -474,10 +486,10 @@ __global__ void __launch_bounds__(RegisterBounds<NV>::kMaxThreads)
     const int lane = tid & 31;
     const int warp = tid >> 5;
     const int64_t T = p.T;
-    const int64_t q_items = p.set[0].items;
-    const int64_t n_items = q_items + p.set[1].items;
+    const int64_t n_items = p.n_items;
 
     int which = -1;
+    int64_t set_begin = 0, set_end = 0;  // items of the current set: [set_begin, set_end)
     const char *in = nullptr;
     char *out = nullptr;
     float *sums = nullptr;
@@ -488,11 +500,13 @@ __global__ void __launch_bounds__(RegisterBounds<NV>::kMaxThreads)
     uint4 g[NV][KG];
 
     for (int64_t item = blockIdx.x; item < n_items; item += gridDim.x) {
-        const int w = item >= q_items ? 1 : 0;
-        const int64_t j = w ? item - q_items : item;
-        if (w != which) {  // uniform across the CTA
-            which = w;
-            const RowSet &d = p.set[w];
+        if (item >= set_end) {  // uniform across the CTA: on to the set holding this item
+            do {
+                ++which;
+                set_begin = set_end;
+                set_end = p.set[which].item_end;
+            } while (item >= set_end);
+            const RowSet &d = p.set[which];
             in = d.in;
             out = d.out;
             sums = d.sumsq;
@@ -515,7 +529,7 @@ __global__ void __launch_bounds__(RegisterBounds<NV>::kMaxThreads)
                 for (int i = 0; i < NV; ++i) ld_gamma_vec<E>(d.gamma, gl + i * gsize, nfull, tail, g[i]);
             }
         }
-        const int64_t t = j * rpi + grp;  // row index within the tensor (= token when heads == 1)
+        const int64_t t = (item - set_begin) * rpi + grp;  // row index within the set (= token when heads == 1)
         const bool active = t < rows;
         const int64_t roff = active ? row_offset(t, heads, stride, head_bytes) : 0;
         const char *row = in + roff;

@@ -60,6 +60,8 @@ def parse_args(argv=None):
     ap.add_argument("--workload", choices=["prefill", "decode", "packed", "gqa", "tiny", "headwise", "projection", "tp"],
                     default="prefill")
     ap.add_argument("--ranks", type=int, default=4, help="tensor-parallel ranks of the tp workload")
+    ap.add_argument("--gqa-form", choices=["multi", "per-shard"], default="multi",
+                    help="gqa workload: the two multi-shard calls (2 launches) or P calls of each phase (2P)")
     ap.add_argument("--proj", default="4096,4096,4096,4096",
                     help="D,Hq,Hk,Hv of the projection workload (T from --tokens, default 4096)")
     ap.add_argument("--tokens", type=int, default=None, help="T for decode / packed workloads")
@@ -261,8 +263,10 @@ class Workload:
 
     DTYPES = {"bf16": torch.bfloat16, "f16": torch.float16, "e4m3": torch.float8_e4m3fn}
 
-    def __init__(self, kind: str, tokens: int | None, seed_offset: int, dtype: str = "bf16", ranks: int = 4):
+    def __init__(self, kind: str, tokens: int | None, seed_offset: int, dtype: str = "bf16", ranks: int = 4,
+                 gqa_form: str = "multi"):
         self.kind = kind
+        self.gqa_form = gqa_form
         if kind == "prefill":
             self.batch = workloads.prefill_bf16(seed=1 + seed_offset, dtype=self.DTYPES[dtype])
         elif kind == "tiny":
@@ -285,7 +289,7 @@ class Workload:
         gamma_elems = 2 * b.meta["head_dim"] if kind == "headwise" else b.Hq + b.Hk
         self.eff_bytes = 2 * self.esz * (b.Hq + b.Hk) * b.T + gesz * gamma_elems
         self.name = f"tp_R{ranks}_{b.name}" if kind == "tp" else b.name
-        self.launches_per_step = 2 * b.P if kind == "gqa" else 1
+        self.launches_per_step = (2 * b.P if gqa_form == "per-shard" else 2) if kind == "gqa" else 1
 
     def config(self) -> dict:
         b = self.batch
@@ -294,7 +298,8 @@ class Workload:
         if self.kind == "packed":
             c.update({"Hv": b.Hv, "row_stride": b.packed.shape[1], "in_place": True})
         if self.kind == "gqa":
-            c.update({"P": b.P, "form": "partial_stats x P -> combine_apply x P"})
+            c.update({"P": b.P, "form": "partial_stats x P -> combine_apply x P" if self.gqa_form == "per-shard" else
+                      "partial_stats_shards (P shards, one launch) -> combine_apply_shards (P shards, one launch)"})
         if self.kind == "headwise":
             c.update({"head_dim": b.meta["head_dim"], "q_heads": b.meta["q_heads"], "k_heads": b.meta["k_heads"],
                       "form": "qknorm_headwise (one factor per head)"})
@@ -346,12 +351,16 @@ class Workload:
         b = self.batch
         if self.kind == "packed":
             qk.qknorm_layerwise(s["q"], s["k"], s["gq"], s["gk"], b.eps, q_out=s["q"], k_out=s["k"])
-        elif self.kind == "gqa":
+        elif self.kind == "gqa" and self.gqa_form == "per-shard":
             for p in range(b.P):
                 qk.qknorm_partial_stats(s["qs"][p], s["ks"][p], s["q_all"][p], s["k_all"][p])
             for p in range(b.P):
                 qk.qknorm_combine_apply(s["qs"][p], s["ks"][p], s["gqs"][p], s["gks"][p], s["q_all"], s["k_all"],
                                         b.Hq, b.Hk, b.eps, q_out=s["qo"][p], k_out=s["ko"][p])
+        elif self.kind == "gqa":
+            qk.qknorm_partial_stats_shards(s["qs"], s["ks"], s["q_all"], s["k_all"])
+            qk.qknorm_combine_apply_shards(s["qs"], s["ks"], s["gqs"], s["gks"], s["q_all"], s["k_all"], b.Hq, b.Hk,
+                                           b.eps, q_out=s["qo"], k_out=s["ko"])
         elif self.kind == "headwise":
             qk.qknorm_headwise(s["q"], s["k"], s["gq"], s["gk"], b.meta["head_dim"], b.eps,
                                q_out=s["qo"], k_out=s["ko"])
@@ -530,7 +539,8 @@ def native(args) -> int:
     ranks = Ranks(dist, dev)
     barrier, max_over_ranks = ranks.barrier, ranks.max
 
-    wl = Workload(args.workload, args.tokens, seed_offset=rank * 1000, dtype=args.dtype, ranks=args.ranks)
+    wl = Workload(args.workload, args.tokens, seed_offset=rank * 1000, dtype=args.dtype, ranks=args.ranks,
+                  gqa_form=args.gqa_form)
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     R = rotating = rotation_count(wl.set_bytes(), l2)
     sets = [wl.make_set(dev) for _ in range(R)]
@@ -625,12 +635,20 @@ def native(args) -> int:
                 "unit": "GB/s", "frac": round(wl.eff_bytes / kernel_s / 1e9 / peaks["hbm_gbs"], 4),
                 "traffic": profiled_traffic(wl.name, digest, launch_text(plan)),
                 "peak_source": f"{peaks['source']} copy bandwidth",
-                "kernel": {"gqa": "whole step: partial_stats x P + combine_apply x P",
+                "kernel": {"gqa": "whole step: " + wl.config()["form"],
                            "tp": "tp_warp_kernel (one token per warp), all ranks in one launch "
                                  "(the only kernel of the step)"}.get(
                                wl.kind, "qknorm rows kernel (the only kernel of the step)"),
                 "algorithmic_bytes_per_launch": wl.eff_bytes if wl.kind != "gqa" else None,
                 "source_digest": digest}
+    if wl.kind == "gqa":
+        # the decomposed form must read every shard twice (partial sums, then
+        # apply): its floor is 2 reads + 1 write of Q and K, gamma, and the
+        # [P][T] sums written once and read once
+        b = wl.batch
+        floor = 3 * wl.esz * (b.Hq + b.Hk) * b.T + 2 * (b.Hq + b.Hk) + 2 * 2 * b.P * b.T * 4
+        roofline.update({"floor_bytes_per_step": floor, "floor_achieved": round(floor / step_s / 1e9, 1),
+                         "floor_frac": round(floor / step_s / 1e9 / peaks["hbm_gbs"], 4)})
 
     timeouts = qk.device_timeouts()  # any bounded wait that ran out (tensor-parallel exchange)
 
@@ -666,6 +684,36 @@ def native(args) -> int:
     if dist is not None:
         dist.destroy_process_group()
     return 0
+
+
+def link_calibration(dev, h2d_bytes: int, d2h_bytes: int, eff_bytes: int, reps: int = 5) -> dict:
+    """The host link on its own: pinned copies of one step's bytes, each
+    direction alone and both at once on two streams (best of `reps`), and the
+    end-to-end value those copies alone would allow."""
+    src_h = torch.empty(h2d_bytes, dtype=torch.uint8, pin_memory=True)
+    dst_d = torch.empty(h2d_bytes, dtype=torch.uint8, device=dev)
+    src_d = torch.empty(d2h_bytes, dtype=torch.uint8, device=dev)
+    dst_h = torch.empty(d2h_bytes, dtype=torch.uint8, pin_memory=True)
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+
+    def timed(h2d: bool, d2h: bool) -> float:
+        best = float("inf")
+        for _ in range(reps):
+            torch.cuda.synchronize(dev)
+            t0 = time.perf_counter()
+            if h2d:
+                with torch.cuda.stream(s_in):
+                    dst_d.copy_(src_h, non_blocking=True)
+            if d2h:
+                with torch.cuda.stream(s_out):
+                    dst_h.copy_(src_d, non_blocking=True)
+            torch.cuda.synchronize(dev)
+            best = min(best, time.perf_counter() - t0)
+        return best
+    t_in, t_out, t_both = timed(True, False), timed(False, True), timed(True, True)
+    return {"h2d_gbs": round(h2d_bytes / t_in / 1e9, 2), "d2h_gbs": round(d2h_bytes / t_out / 1e9, 2),
+            "both_ms": round(t_both * 1e3, 4), "e2e_copy_limit": round(eff_bytes / t_both / 1e9, 2),
+            "how": "pinned torch copies of the step's bytes, host clock, best of %d" % reps}
 
 
 def e2e_measure(qk, wl: Workload, dev, args, barrier, max_over_ranks) -> dict:
@@ -754,7 +802,7 @@ def e2e_measure(qk, wl: Workload, dev, args, barrier, max_over_ranks) -> dict:
                 f"on the device, device -> pinned host; {args.e2e_slots}-slot device ring, copies and kernel "
                 "overlap on three streams")
 
-    for _ in range(2):
+    for _ in range(3):
         one()
     stream = torch.cuda.current_stream(dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -768,9 +816,10 @@ def e2e_measure(qk, wl: Workload, dev, args, barrier, max_over_ranks) -> dict:
     barrier()
     ms = max_over_ranks(e0.elapsed_time(e1))
     world = int(os.environ.get("WORLD_SIZE", "1"))
+    link = link_calibration(dev, h2d, d2h, wl.eff_bytes)
     return {"value": round(world * wl.eff_bytes / (ms / 1e3 / steps) / 1e9, 2), "unit": UNIT,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
-            "ms_per_step": round(ms / steps, 4), "path": path}
+            "ms_per_step": round(ms / steps, 4), "path": path, "link": link}
 
 
 # --------------------------------------------------------------------------- reference arm (the oracle)

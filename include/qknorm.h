@@ -132,6 +132,39 @@ qkn_status qknorm_combine_apply(const void *q_in, void *q_out, const void *gamma
                                 int32_t P, int64_t T, float eps, qkn_dtype dtype, void *stream);
 
 /*
+ * Multi-shard forms of the two calls above, for P hidden-dimension shards of Q
+ * and of K held in separate buffers on this GPU (Phase A: every shard's local
+ * squared sum; its aggregation in the fixed order p = 0..P-1; Phase B: each
+ * shard scaled by the global factor).  Each covers all P shards in ONE kernel
+ * launch instead of P, with the same results as the per-shard calls:
+ *   qknorm_partial_stats_shards  ==  for p in 0..P-1:
+ *       qknorm_partial_stats(q_shards[p], ..., q_sumsq_all + p * T,
+ *                            k_shards[p], ..., k_sumsq_all + p * T, ...)
+ *   qknorm_combine_apply_shards  ==  for p in 0..P-1:
+ *       qknorm_combine_apply(q_in[p], q_out[p], gamma_q_shards[p], ..., q_sumsq_all, Hq_full,
+ *                            k_in[p], k_out[p], gamma_k_shards[p], ..., k_sumsq_all, Hk_full, P, ...)
+ * (a squared sum may differ in its last bit from the per-shard call's where
+ * the two launches group the shard's row differently; both are within the
+ * parity tolerances).
+ *   P in [1, 8].  Every Q shard has width hq_shard and row stride q_stride;
+ *   likewise for K.  q_sumsq_all / k_sumsq_all: [P][T] fp32, contiguous.
+ *   q_out[p] == q_in[p] normalizes shard p in place.
+ * Errors: as the per-shard calls, plus P outside [1, 8]; no output may
+ * overlap any other shard's operands.  When the rows cannot move as 16-byte
+ * vectors (unaligned) or are wider than 32 KB, the call runs shard by shard.
+ */
+qkn_status qknorm_partial_stats_shards(int32_t P, const void *const *q_shards, int64_t q_stride, int32_t hq_shard,
+                                       float *q_sumsq_all, const void *const *k_shards, int64_t k_stride,
+                                       int32_t hk_shard, float *k_sumsq_all, int64_t T, qkn_dtype dtype,
+                                       void *stream);
+qkn_status qknorm_combine_apply_shards(int32_t P, const void *const *q_in, void *const *q_out,
+                                       const void *const *gamma_q_shards, int64_t q_stride, int32_t hq_shard,
+                                       const float *q_sumsq_all, int32_t Hq_full, const void *const *k_in,
+                                       void *const *k_out, const void *const *gamma_k_shards, int64_t k_stride,
+                                       int32_t hk_shard, const float *k_sumsq_all, int32_t Hk_full, int64_t T,
+                                       float eps, qkn_dtype dtype, void *stream);
+
+/*
  * Fused layerwise QK-Norm of rows held in HOST memory, end to end: the T
  * tokens flow in chunks of chunk_tokens through a ring of device buffers, and
  * for each chunk the Q and K rows are copied host->device, normalized in

@@ -522,3 +522,57 @@ def test_host_ring_bytes(lib):
     assert lib.qknorm_layerwise_host_ring_bytes(8, 8, 8, BF16, 9) == -1
     assert lib.qknorm_layerwise_host_ring_bytes(8, 0, 8, BF16, 1) == -1
     assert lib.qknorm_layerwise_host_ring_bytes(8, 8, 8, 9, 1) == -1
+
+
+# --------------------------------------------------------------------------- multi-shard calls
+
+def _shards_call(lib, which, **kw):
+    P_ = ctypes.c_void_p
+    a = dict(P=4, T=256, hq=256, hk=128, qs=256, ks=128, eps=1e-6, dtype=BF16, Hq=1024, Hk=512,
+             q_all=0x60000000, k_all=0x61000000, q_out=None, k_out=None)
+    a.update(kw)
+    n = max(a["P"], 1)
+    arr = lambda base, step=0x100000: (P_ * n)(*[base + j * step for j in range(n)])
+    q_in, k_in = arr(0x10000000), arr(0x20000000)
+    if which == "stats":
+        return lib.qknorm_partial_stats_shards(a["P"], q_in, a["qs"], a["hq"], a["q_all"], k_in, a["ks"], a["hk"],
+                                               a["k_all"], a["T"], a["dtype"], None)
+    q_out = a["q_out"] if a["q_out"] is not None else arr(0x30000000)
+    k_out = arr(0x40000000)
+    return lib.qknorm_combine_apply_shards(a["P"], q_in, q_out, arr(0x50000000, 0x1000), a["qs"], a["hq"], a["q_all"],
+                                           a["Hq"], k_in, k_out, arr(0x50800000, 0x1000), a["ks"], a["hk"],
+                                           a["k_all"], a["Hk"], a["T"], a["eps"], a["dtype"], None)
+
+
+@pytest.mark.parametrize("which", ["stats", "apply"])
+@pytest.mark.parametrize("kw,want", [
+    ({}, CUDA),                                 # well formed: validation passes, the device query fails here
+    ({"T": 0}, OK),
+    ({"P": 0}, INVALID),
+    ({"P": 9}, INVALID),
+    ({"T": -1}, INVALID),
+    ({"hq": 0}, INVALID),
+    ({"qs": 100}, INVALID),                     # stride below the shard width
+    ({"dtype": 7}, INVALID),
+    ({"q_all": 0}, INVALID),
+])
+def test_multi_shard_validation(lib, which, kw, want):
+    assert _shards_call(lib, which, **kw) == want
+
+
+def test_multi_shard_stats_sums_must_not_overlap(lib):
+    """The stats call writes the sums: they may not touch a shard or each
+    other.  The apply call only reads them, beside inputs it only reads."""
+    assert _shards_call(lib, "stats", q_all=0x10000000 + 512) == INVALID   # sums on shard 0's rows
+    assert _shards_call(lib, "stats", k_all=0x60000000 + 8) == INVALID     # the two sum arrays overlap
+    assert _shards_call(lib, "apply", q_all=0x10000000 + 512) == CUDA
+
+
+def test_multi_shard_apply_outputs_checked_across_shards(lib):
+    P_ = ctypes.c_void_p
+    # shard 1's Q output lands on shard 0's Q input
+    q_out = (P_ * 4)(0x30000000, 0x10000000, 0x30200000, 0x30300000)
+    assert _shards_call(lib, "apply", q_out=q_out) == INVALID
+    assert b"shard" in lib.qknorm_last_error()
+    assert _shards_call(lib, "apply", Hq=100) == INVALID        # full width below the shard width
+    assert _shards_call(lib, "apply", eps=-1.0) == INVALID

@@ -156,6 +156,96 @@ def test_gqa_shard_decomposed_full_size():
     assert int(bf16_ulp_distance(to_np(fk.cpu()), to_np(got_k.cpu())).max()) <= 1
 
 
+def _split(full: torch.Tensor, P: int, stride_pad: int = 0):
+    """P column shards of `full` in separate device buffers, each with
+    `stride_pad` padding elements after its row."""
+    w = full.shape[1] // P
+    out = []
+    for p in range(P):
+        buf = torch.full((full.shape[0], w + stride_pad), 7.0, dtype=full.dtype).to(DEV)
+        buf[:, :w] = full[:, p * w:(p + 1) * w].to(DEV)
+        out.append(buf[:, :w])
+    return out
+
+
+def test_gqa_multi_shard_calls_full_size_equal_the_per_shard_calls():
+    """The GQA step through the two multi-shard calls (one launch per phase):
+    partial sums and outputs bit-equal to the per-shard calls at this shape
+    (same row groups), and against the oracle over the full rows."""
+    b = workloads.gqa_sharded()
+    P, T = b.P, b.T
+    wq, wk = b.Hq // P, b.Hk // P
+    qs = [s.to(DEV) for s in b.q_shards]
+    ks = [s.to(DEV) for s in b.k_shards]
+    gq, gk = b.gamma_q.to(DEV), b.gamma_k.to(DEV)
+    gqs = [gq[p * wq:(p + 1) * wq].contiguous() for p in range(P)]
+    gks = [gk[p * wk:(p + 1) * wk].contiguous() for p in range(P)]
+    q_all, k_all = qk.qknorm_partial_stats_shards(qs, ks)
+    qo, ko = qk.qknorm_combine_apply_shards(qs, ks, gqs, gks, q_all, k_all, b.Hq, b.Hk, b.eps)
+    ref_q = torch.empty((P, T), dtype=torch.float32, device=DEV)
+    ref_k = torch.empty((P, T), dtype=torch.float32, device=DEV)
+    for p in range(P):
+        qk.qknorm_partial_stats(qs[p], ks[p], ref_q[p], ref_k[p])
+    per = [qk.qknorm_combine_apply(qs[p], ks[p], gqs[p], gks[p], ref_q, ref_k, b.Hq, b.Hk, b.eps) for p in range(P)]
+    torch.cuda.synchronize()
+    assert torch.equal(q_all, ref_q) and torch.equal(k_all, ref_k)
+    for p in range(P):
+        assert torch.equal(qo[p], per[p][0]) and torch.equal(ko[p], per[p][1])
+    yq, eq, _ = oracle_rows(b.q_full, b.gamma_q, b.eps)
+    yk, ek, _ = oracle_rows(b.k_full, b.gamma_k, b.eps)
+    assert_close(torch.cat([o.cpu() for o in qo], dim=1), yq, eq, "gqa multi-shard Q")
+    assert_close(torch.cat([o.cpu() for o in ko], dim=1), yk, ek, "gqa multi-shard K")
+
+
+@pytest.mark.parametrize("dtype", ALL_DTYPES)
+@pytest.mark.parametrize("P,T,Hq,Hk,pad", [
+    (1, 100, 1024, 256, 0),
+    (2, 37, 2048, 512, 8),      # padded rows
+    (4, 1, 5120, 1024, 0),      # one token: few rows, the latency plan
+    (8, 300, 4096, 1024, 0),    # eight shards: sixteen row sets
+    (3, 129, 768, 384, 0),      # shard rows whose width is not a power of two
+    (4, 64, 1000, 200, 0),      # unaligned shard widths: shard by shard, scalar kernels
+])
+def test_multi_shard_calls_match_the_oracle(dtype, P, T, Hq, Hk, pad):
+    b = workloads.random_rows(T, Hq, Hk, dtype, seed=P * 1000 + T, scale=1.5)
+    qs, ks = _split(b.q, P, pad), _split(b.k, P, pad)
+    wq, wk = Hq // P, Hk // P
+    gq, gk = b.gamma_q.to(DEV), b.gamma_k.to(DEV)
+    gqs = [gq[p * wq:(p + 1) * wq].contiguous() for p in range(P)]
+    gks = [gk[p * wk:(p + 1) * wk].contiguous() for p in range(P)]
+    q_all, k_all = qk.qknorm_partial_stats_shards(qs, ks)
+    torch.cuda.synchronize()
+    for p in range(P):
+        oq = oracle.partial_sumsq(to_np(b.q[:, p * wq:(p + 1) * wq]), wq, wq, T)
+        ok_ = oracle.partial_sumsq(to_np(b.k[:, p * wk:(p + 1) * wk]), wk, wk, T)
+        np.testing.assert_allclose(q_all[p].cpu().double().numpy(), oq, rtol=1e-5, atol=0)
+        np.testing.assert_allclose(k_all[p].cpu().double().numpy(), ok_, rtol=1e-5, atol=0)
+    # out of place, then in place: bit for bit the same
+    qo, ko = qk.qknorm_combine_apply_shards(qs, ks, gqs, gks, q_all, k_all, Hq, Hk, b.eps)
+    torch.cuda.synchronize()
+    yq, eq, _ = oracle_rows(b.q, b.gamma_q, b.eps)
+    yk, ek, _ = oracle_rows(b.k, b.gamma_k, b.eps)
+    assert_close(torch.cat([o.cpu() for o in qo], dim=1), yq, eq, "multi-shard Q")
+    assert_close(torch.cat([o.cpu() for o in ko], dim=1), yk, ek, "multi-shard K")
+    qk.qknorm_combine_apply_shards(qs, ks, gqs, gks, q_all, k_all, Hq, Hk, b.eps, q_out=qs, k_out=ks)
+    torch.cuda.synchronize()
+    for p in range(P):
+        assert torch.equal(qs[p], qo[p]) and torch.equal(ks[p], ko[p])
+        if pad:  # padding after each shard row untouched
+            base_q = qs[p].as_strided((T, wq + pad), (wq + pad, 1))
+            assert torch.all(base_q[:, wq:].float() == 7.0)
+
+
+def test_multi_shard_calls_reject_overlapping_shards():
+    x = torch.zeros((8, 256), dtype=torch.bfloat16, device=DEV)
+    g = torch.ones((128,), dtype=torch.bfloat16, device=DEV)
+    qa, ka = qk.qknorm_partial_stats_shards([x[:, :128], x[:, 128:]], [x[:, :128], x[:, 128:]])
+    out = torch.empty((8, 256), dtype=torch.bfloat16, device=DEV)
+    with pytest.raises(qk.QKNormError, match="overlap"):  # shard 1's output on shard 0's input
+        qk.qknorm_combine_apply_shards([x[:, :128], x[:, 128:]], [x[:, :128], x[:, 128:]], [g, g], [g, g], qa, ka,
+                                       256, 256, q_out=[out[:, :128], x[:, :128]], k_out=[out[:, 128:], x[:, 128:]])
+
+
 @pytest.mark.parametrize("T", workloads.PACKED_TOKENS)
 def test_packed_qkv_in_place_v_untouched(T):
     b = workloads.packed_qkv(T)

@@ -14,7 +14,8 @@ call's partial sums are still in the shared array when the second runs.  The
 workspace entry point gets a workspace filled with NaN, so a partial sum that
 either path reads without having written it shows up as a difference.  Both
 calls are also checked against the oracle on sampled rows (projection and
-RMS-Norm, with the bounds of the projection tests).  The checks run twice: in
+RMS-Norm of the projection, with the bounds of the projection tests; V
+columns equal to the plain projection).  The checks run twice: in
 this process, after whatever ran before, and in a fresh Python process whose
 first library call is this one.
 
@@ -74,9 +75,15 @@ def run_two_calls() -> None:
         g, r = to_np(got.cpu()), to_np(ref.cpu())
         assert np.array_equal(g, r), (f"call {i + 1} ({b.name}): {int(np.sum(g != r))} elements differ from "
                                       "qknorm_qkv_projection")
+        # the oracle: its projection checked against the GEMM's stored values
+        # (the call rescales Q and K in place, V keeps the projection), its
+        # RMS-Norm against the call's Q and K columns
+        plain, _, _ = qk.qknorm_qkv_gemm_stats(x, w, b.Hq, b.Hk, b.Hv)
+        torch.cuda.synchronize()
         rows = _sample_rows(b.T, 24, seed=300 + i)
-        proj = check_projection(b, got, rows)
+        proj = check_projection(b, plain, rows)
         check_normalized(b, proj, got, rows)
+        assert torch.equal(got[:, b.Hq + b.Hk:], plain[:, b.Hq + b.Hk:])
 
 
 def test_noalloc_matches_the_workspace_entry_point_and_the_oracle_on_two_calls():
