@@ -491,7 +491,8 @@ def _sums_all(t, name, P, T, dev):
     return t
 
 
-def qknorm_partial_stats_shards(q_shards, k_shards, q_sumsq_all=None, k_sumsq_all=None, *, stream=None):
+def qknorm_partial_stats_shards(q_shards, k_shards, q_sumsq_all=None, k_sumsq_all=None, *, stream=None,
+                                launch: QknLaunch | dict | None = None):
     """Phase A local step for P shards of Q and of K in one launch: row p of
     the returned ``[P, T]`` float32 arrays ``(q_sumsq_all, k_sumsq_all)``
     holds the squared sums of shard p, exactly what P calls of
@@ -507,18 +508,21 @@ def qknorm_partial_stats_shards(q_shards, k_shards, q_sumsq_all=None, k_sumsq_al
         raise ValueError("Q and K shards must have the same number of tokens")
     q_sumsq_all = _sums_all(q_sumsq_all, "q_sumsq_all", P, T, dev)
     k_sumsq_all = _sums_all(k_sumsq_all, "k_sumsq_all", P, T, dev)
+    args = [P, _ptr_array([t.data_ptr() for t in q_shards]), sq, hq, q_sumsq_all.data_ptr(),
+            _ptr_array([t.data_ptr() for t in k_shards]), sk, hk, k_sumsq_all.data_ptr(), T, _DTYPES[dt]]
     with _on(dev):
-        st = capi().qknorm_partial_stats_shards(P, _ptr_array([t.data_ptr() for t in q_shards]), sq, hq,
-                                                q_sumsq_all.data_ptr(), _ptr_array([t.data_ptr() for t in k_shards]),
-                                                sk, hk, k_sumsq_all.data_ptr(), T, _DTYPES[dt],
-                                                _stream_handle(stream, dev))
+        s = _stream_handle(stream, dev)
+        if launch is None:
+            st = capi().qknorm_partial_stats_shards(*args, s)
+        else:
+            st = capi().qknorm_partial_stats_shards_launch(*args, s, ctypes.byref(_launch_struct(launch)))
     _clib.check(st, "qknorm_partial_stats_shards")
     return q_sumsq_all, k_sumsq_all
 
 
 def qknorm_combine_apply_shards(q_in, k_in, gamma_q_shards, gamma_k_shards, q_sumsq_all: torch.Tensor,
                                 k_sumsq_all: torch.Tensor, Hq_full: int, Hk_full: int, eps: float = 1e-6, *,
-                                q_out=None, k_out=None, stream=None):
+                                q_out=None, k_out=None, stream=None, launch: QknLaunch | dict | None = None):
     """Phase A aggregation and Phase B for P shards of Q and of K in one
     launch: the same results as P calls of ``qknorm_combine_apply`` with the
     same ``[P, T]`` partial sums.  Returns the lists ``(q_out, k_out)``."""
@@ -548,14 +552,16 @@ def qknorm_combine_apply_shards(q_in, k_in, gamma_q_shards, gamma_k_shards, q_su
     gdt = gamma_dtype(dt)
     gq = [_vec(g, f"gamma_q_shards[{j}]", hq, gdt, dev) for j, g in enumerate(gamma_q_shards)]
     gk = [_vec(g, f"gamma_k_shards[{j}]", hk, gdt, dev) for j, g in enumerate(gamma_k_shards)]
+    args = [P, _ptr_array([t.data_ptr() for t in q_in]), _ptr_array([t.data_ptr() for t in q_out]),
+            _ptr_array(gq), sq, hq, q_sumsq_all.data_ptr(), int(Hq_full), _ptr_array([t.data_ptr() for t in k_in]),
+            _ptr_array([t.data_ptr() for t in k_out]), _ptr_array(gk), sk, hk, k_sumsq_all.data_ptr(), int(Hk_full),
+            T, float(eps), _DTYPES[dt]]
     with _on(dev):
-        st = capi().qknorm_combine_apply_shards(P, _ptr_array([t.data_ptr() for t in q_in]),
-                                                _ptr_array([t.data_ptr() for t in q_out]), _ptr_array(gq), sq, hq,
-                                                q_sumsq_all.data_ptr(), int(Hq_full),
-                                                _ptr_array([t.data_ptr() for t in k_in]),
-                                                _ptr_array([t.data_ptr() for t in k_out]), _ptr_array(gk), sk, hk,
-                                                k_sumsq_all.data_ptr(), int(Hk_full), T, float(eps), _DTYPES[dt],
-                                                _stream_handle(stream, dev))
+        s = _stream_handle(stream, dev)
+        if launch is None:
+            st = capi().qknorm_combine_apply_shards(*args, s)
+        else:
+            st = capi().qknorm_combine_apply_shards_launch(*args, s, ctypes.byref(_launch_struct(launch)))
     _clib.check(st, "qknorm_combine_apply_shards")
     return q_out, k_out
 

@@ -55,6 +55,11 @@ PROTOTYPES = {
     "qknorm_partial_stats_shards": (_st, [_i32, _vp, _i64, _i32, _vp, _vp, _i64, _i32, _vp, _i64, _dt, _vp]),
     "qknorm_combine_apply_shards": (_st, [_i32, _vp, _vp, _vp, _i64, _i32, _vp, _i32,
                                           _vp, _vp, _vp, _i64, _i32, _vp, _i32, _i64, _f32, _dt, _vp]),
+    "qknorm_partial_stats_shards_launch": (_st, [_i32, _vp, _i64, _i32, _vp, _vp, _i64, _i32, _vp, _i64, _dt, _vp,
+                                                 ctypes.POINTER(QknLaunch)]),
+    "qknorm_combine_apply_shards_launch": (_st, [_i32, _vp, _vp, _vp, _i64, _i32, _vp, _i32,
+                                                 _vp, _vp, _vp, _i64, _i32, _vp, _i32, _i64, _f32, _dt, _vp,
+                                                 ctypes.POINTER(QknLaunch)]),
     "qknorm_status_string": (ctypes.c_char_p, [_st]),
     "qknorm_qkv_gemm_stats": (_st, [_vp, _i64, _vp, _i64, _vp, _i64, _i64, _i32, _i32, _i32, _i32,
                                     _vp, _vp, _dt, _vp]),

@@ -946,7 +946,7 @@ qkn_status qknorm_plan_shape(int64_t rows, int64_t units_max, int32_t vectorized
     }
     L.kernel = QKN_KERNEL_REGISTER;
     int nv;
-    bool narrow = false;
+    bool narrow = false, many = false;
     if (rows <= sm_count) {
         // Few rows (decode): spread each row over many threads so a row costs
         // about one memory round trip (two vectors per thread measured best).
@@ -961,10 +961,13 @@ qkn_status qknorm_plan_shape(int64_t rows, int64_t units_max, int32_t vectorized
     } else {
         // Many rows: moderate CTAs, several vectors in flight per thread.
         nv = units_max >= 256 ? 4 : 2;
+        many = true;
     }
-    // A 16-byte vector of 1-byte elements widens to twice the fp32 registers
-    // (and pairs with two gamma vectors): hold half as many per thread.
-    if (elem_bytes == 1 && nv > 1) nv /= 2;
+    // A 16-byte vector of 1-byte elements widens to twice the fp32 registers:
+    // hold half as many per thread -- except for many wide rows, whose gamma
+    // is re-read per row instead of held (1-byte elements), which leaves room
+    // for the full count and halves the per-row work per vector.
+    if (elem_bytes == 1 && nv > 1 && !many) nv /= 2;
     int32_t threads = round32((units_max + nv - 1) / nv);
     while (threads > qknorm_register_max_threads(nv)) {
         nv *= 2;
@@ -1121,14 +1124,26 @@ qkn_status qknorm_combine_apply_launch(const void *q_in, void *q_out, const void
     return launch<qkn::kApply>(c, *launch_cfg, stream);
 }
 
-qkn_status qknorm_partial_stats_shards(int32_t P, const void *const *q_shards, int64_t q_stride, int32_t hq_shard,
-                                       float *q_sumsq_all, const void *const *k_shards, int64_t k_stride,
-                                       int32_t hk_shard, float *k_sumsq_all, int64_t T, qkn_dtype dtype,
-                                       void *stream) {
+}  // extern "C"
+
+namespace {
+
+qkn_status stats_shards(int32_t P, const void *const *q_shards, int64_t q_stride, int32_t hq_shard,
+                        float *q_sumsq_all, const void *const *k_shards, int64_t k_stride, int32_t hk_shard,
+                        float *k_sumsq_all, int64_t T, qkn_dtype dtype, void *stream, const qkn_launch *pinned) {
     ShardCall c;
     qkn_status st = prepare_stats_shards(P, q_shards, q_stride, hq_shard, q_sumsq_all, k_shards, k_stride, hk_shard,
                                          k_sumsq_all, T, dtype, c);
     if (st != QKN_OK) return st;
+    if (pinned) {
+        if (T > 0 && !one_launch(c))
+            return fail(QKN_ERR_INVALID_ARG, "a pinned launch needs 16-byte aligned shard rows of at most 32 KB");
+        if (T > 0 && (st = check_launch(c, *pinned)) != QKN_OK) return st;
+        if (T > 0 && pinned->kernel != QKN_KERNEL_REGISTER)
+            return fail(QKN_ERR_INVALID_ARG, "multi-shard calls run the register kernel only");
+        if (T == 0) return ok();
+        return launch<qkn::kStats>(c, *pinned, stream);
+    }
     if (T == 0) return ok();
     if (!one_launch(c)) {
         for (int p = 0; p < P; ++p)
@@ -1143,17 +1158,25 @@ qkn_status qknorm_partial_stats_shards(int32_t P, const void *const *q_shards, i
     return launch<qkn::kStats>(c, L, stream);
 }
 
-qkn_status qknorm_combine_apply_shards(int32_t P, const void *const *q_in, void *const *q_out,
-                                       const void *const *gamma_q_shards, int64_t q_stride, int32_t hq_shard,
-                                       const float *q_sumsq_all, int32_t Hq_full, const void *const *k_in,
-                                       void *const *k_out, const void *const *gamma_k_shards, int64_t k_stride,
-                                       int32_t hk_shard, const float *k_sumsq_all, int32_t Hk_full, int64_t T,
-                                       float eps, qkn_dtype dtype, void *stream) {
+qkn_status apply_shards(int32_t P, const void *const *q_in, void *const *q_out, const void *const *gamma_q_shards,
+                        int64_t q_stride, int32_t hq_shard, const float *q_sumsq_all, int32_t Hq_full,
+                        const void *const *k_in, void *const *k_out, const void *const *gamma_k_shards,
+                        int64_t k_stride, int32_t hk_shard, const float *k_sumsq_all, int32_t Hk_full, int64_t T,
+                        float eps, qkn_dtype dtype, void *stream, const qkn_launch *pinned) {
     ShardCall c;
     qkn_status st = prepare_apply_shards(P, q_in, q_out, gamma_q_shards, q_stride, hq_shard, q_sumsq_all, Hq_full,
                                          k_in, k_out, gamma_k_shards, k_stride, hk_shard, k_sumsq_all, Hk_full, T, eps,
                                          dtype, c);
     if (st != QKN_OK) return st;
+    if (pinned) {
+        if (T > 0 && !one_launch(c))
+            return fail(QKN_ERR_INVALID_ARG, "a pinned launch needs 16-byte aligned shard rows of at most 32 KB");
+        if (T > 0 && (st = check_launch(c, *pinned)) != QKN_OK) return st;
+        if (T > 0 && pinned->kernel != QKN_KERNEL_REGISTER)
+            return fail(QKN_ERR_INVALID_ARG, "multi-shard calls run the register kernel only");
+        if (T == 0) return ok();
+        return launch<qkn::kApply>(c, *pinned, stream);
+    }
     if (T == 0) return ok();
     if (!one_launch(c)) {
         for (int p = 0; p < P; ++p)
@@ -1166,6 +1189,49 @@ qkn_status qknorm_combine_apply_shards(int32_t P, const void *const *q_in, void 
     qkn_launch L;
     if ((st = plan_call<qkn::kApply>(c, L)) != QKN_OK) return st;
     return launch<qkn::kApply>(c, L, stream);
+}
+
+}  // namespace
+
+extern "C" {
+
+qkn_status qknorm_partial_stats_shards(int32_t P, const void *const *q_shards, int64_t q_stride, int32_t hq_shard,
+                                       float *q_sumsq_all, const void *const *k_shards, int64_t k_stride,
+                                       int32_t hk_shard, float *k_sumsq_all, int64_t T, qkn_dtype dtype,
+                                       void *stream) {
+    return stats_shards(P, q_shards, q_stride, hq_shard, q_sumsq_all, k_shards, k_stride, hk_shard, k_sumsq_all, T,
+                        dtype, stream, nullptr);
+}
+
+qkn_status qknorm_partial_stats_shards_launch(int32_t P, const void *const *q_shards, int64_t q_stride,
+                                              int32_t hq_shard, float *q_sumsq_all, const void *const *k_shards,
+                                              int64_t k_stride, int32_t hk_shard, float *k_sumsq_all, int64_t T,
+                                              qkn_dtype dtype, void *stream, const qkn_launch *launch_cfg) {
+    if (!launch_cfg) return fail(QKN_ERR_INVALID_ARG, "null launch");
+    return stats_shards(P, q_shards, q_stride, hq_shard, q_sumsq_all, k_shards, k_stride, hk_shard, k_sumsq_all, T,
+                        dtype, stream, launch_cfg);
+}
+
+qkn_status qknorm_combine_apply_shards(int32_t P, const void *const *q_in, void *const *q_out,
+                                       const void *const *gamma_q_shards, int64_t q_stride, int32_t hq_shard,
+                                       const float *q_sumsq_all, int32_t Hq_full, const void *const *k_in,
+                                       void *const *k_out, const void *const *gamma_k_shards, int64_t k_stride,
+                                       int32_t hk_shard, const float *k_sumsq_all, int32_t Hk_full, int64_t T,
+                                       float eps, qkn_dtype dtype, void *stream) {
+    return apply_shards(P, q_in, q_out, gamma_q_shards, q_stride, hq_shard, q_sumsq_all, Hq_full, k_in, k_out,
+                        gamma_k_shards, k_stride, hk_shard, k_sumsq_all, Hk_full, T, eps, dtype, stream, nullptr);
+}
+
+qkn_status qknorm_combine_apply_shards_launch(int32_t P, const void *const *q_in, void *const *q_out,
+                                              const void *const *gamma_q_shards, int64_t q_stride, int32_t hq_shard,
+                                              const float *q_sumsq_all, int32_t Hq_full, const void *const *k_in,
+                                              void *const *k_out, const void *const *gamma_k_shards,
+                                              int64_t k_stride, int32_t hk_shard, const float *k_sumsq_all,
+                                              int32_t Hk_full, int64_t T, float eps, qkn_dtype dtype, void *stream,
+                                              const qkn_launch *launch_cfg) {
+    if (!launch_cfg) return fail(QKN_ERR_INVALID_ARG, "null launch");
+    return apply_shards(P, q_in, q_out, gamma_q_shards, q_stride, hq_shard, q_sumsq_all, Hq_full, k_in, k_out,
+                        gamma_k_shards, k_stride, hk_shard, k_sumsq_all, Hk_full, T, eps, dtype, stream, launch_cfg);
 }
 
 qkn_status qknorm_qkv_gemm_stats(const void *x, int64_t x_stride, const void *w, int64_t w_stride, void *qkv,

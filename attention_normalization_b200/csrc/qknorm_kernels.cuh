@@ -470,6 +470,21 @@ __device__ __forceinline__ uint4 scale_vec(const uint4 &xv, const uint4 (&gv)[El
 // instead of each paying for a whole one.
 // TAIL: some row ends in a partial vector (otherwise the tail code is
 // compiled out).
+// Element types whose gamma vectors are re-read per row (through L1, where
+// they stay: the same few KB for every row of a tensor) instead of being
+// held in registers across rows.
+template <typename E>
+struct GammaPerRow {
+    static constexpr bool value = false;
+};
+#ifndef QKN_E4M3_GAMMA_PER_ROW
+#define QKN_E4M3_GAMMA_PER_ROW 1
+#endif
+template <>
+struct GammaPerRow<__nv_fp8_e4m3> {
+    static constexpr bool value = QKN_E4M3_GAMMA_PER_ROW != 0;
+};
+
 template <int NV>
 struct RegisterBounds {
     static constexpr int kMaxThreads = NV <= 2 ? 1024 : (NV == 4 ? 512 : 256);
@@ -497,7 +512,9 @@ __global__ void __launch_bounds__(RegisterBounds<NV>::kMaxThreads)
     int64_t stride = 0, head_bytes = 0, rows = 0;
     int nfull = 0, tail = 0, gsize = 32, rpi = 1, grp = 0, gl = 0, gwarps = 1, heads = 1, nparts = 1;
     float inv_div = 0.0f;
-    uint4 g[NV][KG];
+    constexpr int NG = GammaPerRow<E>::value ? 1 : NV;  // gamma vectors held across rows
+    uint4 g[NG][KG];
+    const char *gamma = nullptr;
 
     for (int64_t item = blockIdx.x; item < n_items; item += gridDim.x) {
         if (item >= set_end) {  // uniform across the CTA: on to the set holding this item
@@ -524,10 +541,11 @@ __global__ void __launch_bounds__(RegisterBounds<NV>::kMaxThreads)
             grp = tid / gsize;
             gl = tid - grp * gsize;
             gwarps = gsize >> 5;
-            if (MODE != kStats) {
+            if (MODE != kStats && !GammaPerRow<E>::value) {
 #pragma unroll
                 for (int i = 0; i < NV; ++i) ld_gamma_vec<E>(d.gamma, gl + i * gsize, nfull, tail, g[i]);
             }
+            gamma = d.gamma;
         }
         const int64_t t = (item - set_begin) * rpi + grp;  // row index within the set (= token when heads == 1)
         const bool active = t < rows;
@@ -577,7 +595,14 @@ __global__ void __launch_bounds__(RegisterBounds<NV>::kMaxThreads)
             const bool full = vi < nfull;
             const bool part = TAIL && vi == nfull && tail;
             if (full || part) {
-                const uint4 y = scale_vec<E>(v[i], g[i], r2);
+                uint4 y;
+                if constexpr (GammaPerRow<E>::value) {
+                    uint4 gv[KG];
+                    ld_gamma_vec<E>(gamma, vi, nfull, tail, gv);
+                    y = scale_vec<E>(v[i], gv, r2);
+                } else {
+                    y = scale_vec<E>(v[i], g[i < NG ? i : 0], r2);
+                }
                 if (full)
                     st_stream(orow + off, y);
                 else

@@ -372,6 +372,34 @@ class Workload:
             qk.qknorm_layerwise(s["q"], s["k"], s["gq"], s["gk"], b.eps, q_out=s["qo"], k_out=s["ko"])
 
 
+def roofline_record(wl: Workload, step_s: float, peaks: dict, digest: str, plan) -> dict:
+    """The line's roofline object: the step's effective bytes over the time of
+    the kernel that dominates it (the only kernel of the step, or -- for the
+    shard-decomposed GQA step -- the whole step), against the measured peak."""
+    kernel_s = step_s / wl.launches_per_step if wl.kind != "gqa" else step_s
+    if wl.kind == "gqa":
+        kernel = "whole step: " + wl.config()["form"]
+    elif wl.kind == "tp":
+        kernel = "tp_warp_kernel (one token per warp), all ranks in one launch (the only kernel of the step)"
+    else:
+        kernel = "qknorm rows kernel (the only kernel of the step)"
+    r = {"bound": "hbm", "achieved": round(wl.eff_bytes / kernel_s / 1e9, 1), "peak": peaks["hbm_gbs"],
+         "unit": "GB/s", "frac": round(wl.eff_bytes / kernel_s / 1e9 / peaks["hbm_gbs"], 4),
+         "traffic": profiled_traffic(wl.name, digest, launch_text(plan)),
+         "peak_source": f"{peaks['source']} copy bandwidth", "kernel": kernel,
+         "algorithmic_bytes_per_launch": wl.eff_bytes if wl.kind != "gqa" else None,
+         "source_digest": digest}
+    if wl.kind == "gqa":
+        # the decomposed form must read every shard twice (partial sums, then
+        # apply): its floor is 2 reads + 1 write of Q and K, gamma, and the
+        # [P][T] sums written once and read once
+        b = wl.batch
+        floor = 3 * wl.esz * (b.Hq + b.Hk) * b.T + 2 * (b.Hq + b.Hk) + 2 * 2 * b.P * b.T * 4
+        r.update({"floor_bytes_per_step": floor, "floor_achieved": round(floor / step_s / 1e9, 1),
+                  "floor_frac": round(floor / step_s / 1e9 / peaks["hbm_gbs"], 4)})
+    return r
+
+
 def graph_upload(graph: "torch.cuda.CUDAGraph", stream) -> bool:
     """Upload an instantiated CUDA graph to the device ahead of its first
     replay (cudaGraphUpload), so a timed replay does not pay the one-time
@@ -622,7 +650,6 @@ def native(args) -> int:
     per_rank_gbs = agg["per_rank_gbs"]
     peaks = load_peaks()
     digest = source_digest("tp" if wl.kind == "tp" else "rows")
-    kernel_s = step_s / wl.launches_per_step if wl.kind != "gqa" else step_s
     plan = None
     if wl.kind in ("prefill", "tiny", "decode", "packed"):
         s0 = sets[0]
@@ -631,24 +658,7 @@ def native(args) -> int:
         else:
             plan = qk.qknorm_layerwise_plan(s0["q"], s0["k"], s0["gq"], s0["gk"], q_out=s0["qo"], k_out=s0["ko"])
 
-    roofline = {"bound": "hbm", "achieved": round(wl.eff_bytes / kernel_s / 1e9, 1), "peak": peaks["hbm_gbs"],
-                "unit": "GB/s", "frac": round(wl.eff_bytes / kernel_s / 1e9 / peaks["hbm_gbs"], 4),
-                "traffic": profiled_traffic(wl.name, digest, launch_text(plan)),
-                "peak_source": f"{peaks['source']} copy bandwidth",
-                "kernel": {"gqa": "whole step: " + wl.config()["form"],
-                           "tp": "tp_warp_kernel (one token per warp), all ranks in one launch "
-                                 "(the only kernel of the step)"}.get(
-                               wl.kind, "qknorm rows kernel (the only kernel of the step)"),
-                "algorithmic_bytes_per_launch": wl.eff_bytes if wl.kind != "gqa" else None,
-                "source_digest": digest}
-    if wl.kind == "gqa":
-        # the decomposed form must read every shard twice (partial sums, then
-        # apply): its floor is 2 reads + 1 write of Q and K, gamma, and the
-        # [P][T] sums written once and read once
-        b = wl.batch
-        floor = 3 * wl.esz * (b.Hq + b.Hk) * b.T + 2 * (b.Hq + b.Hk) + 2 * 2 * b.P * b.T * 4
-        roofline.update({"floor_bytes_per_step": floor, "floor_achieved": round(floor / step_s / 1e9, 1),
-                         "floor_frac": round(floor / step_s / 1e9 / peaks["hbm_gbs"], 4)})
+    roofline = roofline_record(wl, step_s, peaks, digest, plan)
 
     timeouts = qk.device_timeouts()  # any bounded wait that ran out (tensor-parallel exchange)
 

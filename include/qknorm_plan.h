@@ -135,6 +135,24 @@ qkn_status qknorm_combine_apply_launch(const void *q_in, void *q_out, const void
                                        const qkn_launch *launch);
 
 /*
+ * qknorm_partial_stats_shards / qknorm_combine_apply_shards with a
+ * caller-chosen launch of the register kernel (the launch rules and checks of
+ * qknorm_layerwise_launch, with the widest shard row as the row); the shard
+ * rows must be 16-byte aligned and at most 32 KB, else QKN_ERR_INVALID_ARG.
+ */
+qkn_status qknorm_partial_stats_shards_launch(int32_t P, const void *const *q_shards, int64_t q_stride,
+                                              int32_t hq_shard, float *q_sumsq_all, const void *const *k_shards,
+                                              int64_t k_stride, int32_t hk_shard, float *k_sumsq_all, int64_t T,
+                                              qkn_dtype dtype, void *stream, const qkn_launch *launch);
+qkn_status qknorm_combine_apply_shards_launch(int32_t P, const void *const *q_in, void *const *q_out,
+                                              const void *const *gamma_q_shards, int64_t q_stride, int32_t hq_shard,
+                                              const float *q_sumsq_all, int32_t Hq_full, const void *const *k_in,
+                                              void *const *k_out, const void *const *gamma_k_shards,
+                                              int64_t k_stride, int32_t hk_shard, const float *k_sumsq_all,
+                                              int32_t Hk_full, int64_t T, float eps, qkn_dtype dtype, void *stream,
+                                              const qkn_launch *launch);
+
+/*
  * qknorm_tp_layerwise with the memory scope of the exchange chosen by the
  * caller.  scope 0: as qknorm_tp_layerwise (GPU-scope loads and stores when
  * every rank of the group runs in this call, system scope otherwise); scope

@@ -284,10 +284,17 @@ def test_plan_shape_covers_the_row(rows, units):
 
 
 def test_plan_shape_one_byte_elements_hold_half_the_vectors():
+    """1-byte elements widen to twice the registers: half the vectors per
+    thread for few rows and for narrow rows; many wide rows (gamma re-read per
+    row) keep the full count in half the threads."""
     two = qk.plan_shape(8192, 512, True, 148, 2)
-    one = qk.plan_shape(8192, 512, True, 148, 1)
-    assert one["vec_per_thread"] * 2 == two["vec_per_thread"]
-    assert one["vec_per_thread"] * one["threads"] >= 512
+    one = qk.plan_shape(8192, 256, True, 148, 1)   # the same rows in 1-byte elements: half the vectors
+    assert one["vec_per_thread"] == two["vec_per_thread"] == 4
+    assert one["threads"] * 2 == two["threads"]
+    for rows, units in ((100, 640), (8192, 16)):   # few rows; narrow rows
+        assert qk.plan_shape(rows, units, True, 148, 1)["vec_per_thread"] * 2 == \
+            qk.plan_shape(rows, units, True, 148, 2)["vec_per_thread"]
+    assert one["vec_per_thread"] * one["threads"] >= 256
     with pytest.raises(qk.QKNormError):
         qk.plan_shape(10, 10, True, 148, 3)
 
@@ -576,3 +583,20 @@ def test_multi_shard_apply_outputs_checked_across_shards(lib):
     assert b"shard" in lib.qknorm_last_error()
     assert _shards_call(lib, "apply", Hq=100) == INVALID        # full width below the shard width
     assert _shards_call(lib, "apply", eps=-1.0) == INVALID
+
+
+def test_multi_shard_launch_override_validation(lib):
+    P_ = ctypes.c_void_p
+    n = 4
+    arr = lambda base, step=0x100000: (P_ * n)(*[base + j * step for j in range(n)])
+
+    def stats(L):
+        # Q shard rows of 1024 bf16 = 128 vectors
+        return lib.qknorm_partial_stats_shards_launch(4, arr(0x10000000), 1024, 1024, 0x60000000, arr(0x20000000),
+                                                      128, 128, 0x61000000, 256, BF16, None,
+                                                      ctypes.byref(L) if L else None)
+    assert stats(None) == INVALID                                                   # no launch given
+    assert stats(_clib.QknLaunch(kernel=0, vec_per_thread=2, threads=100, grid=10)) == INVALID  # not a warp multiple
+    assert stats(_clib.QknLaunch(kernel=0, vec_per_thread=2, threads=32, grid=10)) == INVALID   # row not covered
+    assert stats(_clib.QknLaunch(kernel=1, vec_per_thread=0, threads=256, grid=10)) == INVALID  # not the register kernel
+    assert stats(_clib.QknLaunch(kernel=0, vec_per_thread=2, threads=64, grid=10)) == CUDA      # valid: launch fails here

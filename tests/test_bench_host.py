@@ -103,3 +103,24 @@ def test_launch_text_matches_the_summaries_form():
     assert bench.launch_text({"kernel": 0, "vec_per_thread": 4, "threads": 128, "grid": 1184}) == \
         "kernel=0 vec_per_thread=4 threads=128 grid=1184"
     assert bench.launch_text(None) is None
+
+
+@pytest.mark.parametrize("kind,tokens", [("prefill", None), ("tiny", None), ("decode", 8), ("packed", 1024),
+                                         ("gqa", None), ("headwise", 256), ("tp", None)])
+def test_roofline_record_for_every_workload(kind, tokens, fake_root):
+    """The roofline object of each workload's line builds on the host (no GPU):
+    achieved = effective bytes / the dominant kernel's time, frac against the
+    peak; the GQA line adds the decomposed form's double-read floor."""
+    wl = bench.Workload(kind, tokens, seed_offset=0)
+    peaks = {"hbm_gbs": 6000.0, "source": "test"}
+    step_s = 1e-3
+    r = bench.roofline_record(wl, step_s, peaks, "d0", None)
+    kernel_s = step_s if kind == "gqa" else step_s / wl.launches_per_step
+    assert r["achieved"] == pytest.approx(wl.eff_bytes / kernel_s / 1e9, abs=0.05)  # GB/s to one place
+    assert r["frac"] == pytest.approx(r["achieved"] / 6000.0, abs=1e-4)  # frac is rounded to 4 places
+    assert r["bound"] == "hbm" and r["traffic"] is None
+    if kind == "gqa":
+        assert "partial_stats_shards" in r["kernel"] and wl.launches_per_step == 2
+        assert r["floor_bytes_per_step"] > 1.49 * wl.eff_bytes
+    else:
+        assert "floor_bytes_per_step" not in r

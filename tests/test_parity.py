@@ -236,6 +236,32 @@ def test_multi_shard_calls_match_the_oracle(dtype, P, T, Hq, Hk, pad):
             assert torch.all(base_q[:, wq:].float() == 7.0)
 
 
+@pytest.mark.parametrize("launch", [{"kernel": 0, "vec_per_thread": 2, "threads": 96, "grid": 7},
+                                    {"kernel": 0, "vec_per_thread": 4, "threads": 128, "grid": 300},
+                                    {"kernel": 0, "vec_per_thread": 1, "threads": 160, "grid": 1184},
+                                    {"kernel": 0, "vec_per_thread": 8, "threads": 64, "grid": 50}])
+def test_multi_shard_pinned_launches_match_the_oracle(launch):
+    """Any valid launch of the multi-shard calls (rows grouped differently,
+    any grid) gives the oracle's results."""
+    P, T, Hq, Hk = 4, 333, 5120, 1024
+    b = workloads.random_rows(T, Hq, Hk, torch.bfloat16, seed=77, scale=1.5)
+    qs, ks = _split(b.q, P), _split(b.k, P)
+    wq, wk = Hq // P, Hk // P
+    gq, gk = b.gamma_q.to(DEV), b.gamma_k.to(DEV)
+    gqs = [gq[p * wq:(p + 1) * wq].contiguous() for p in range(P)]
+    gks = [gk[p * wk:(p + 1) * wk].contiguous() for p in range(P)]
+    q_all, k_all = qk.qknorm_partial_stats_shards(qs, ks, launch=launch)
+    qo, ko = qk.qknorm_combine_apply_shards(qs, ks, gqs, gks, q_all, k_all, Hq, Hk, b.eps, launch=launch)
+    torch.cuda.synchronize()
+    for p in range(P):
+        oq = oracle.partial_sumsq(to_np(b.q[:, p * wq:(p + 1) * wq]), wq, wq, T)
+        np.testing.assert_allclose(q_all[p].cpu().double().numpy(), oq, rtol=1e-5, atol=0)
+    yq, eq, _ = oracle_rows(b.q, b.gamma_q, b.eps)
+    yk, ek, _ = oracle_rows(b.k, b.gamma_k, b.eps)
+    assert_close(torch.cat([o.cpu() for o in qo], dim=1), yq, eq, f"pinned {launch} Q")
+    assert_close(torch.cat([o.cpu() for o in ko], dim=1), yk, ek, f"pinned {launch} K")
+
+
 def test_multi_shard_calls_reject_overlapping_shards():
     x = torch.zeros((8, 256), dtype=torch.bfloat16, device=DEV)
     g = torch.ones((128,), dtype=torch.bfloat16, device=DEV)
@@ -244,6 +270,51 @@ def test_multi_shard_calls_reject_overlapping_shards():
     with pytest.raises(qk.QKNormError, match="overlap"):  # shard 1's output on shard 0's input
         qk.qknorm_combine_apply_shards([x[:, :128], x[:, 128:]], [x[:, :128], x[:, 128:]], [g, g], [g, g], qa, ka,
                                        256, 256, q_out=[out[:, :128], x[:, :128]], k_out=[out[:, 128:], x[:, 128:]])
+
+
+def _e4m3_case(T, H, seed):
+    b = workloads.random_rows(T, H, H, torch.float8_e4m3fn, seed=seed, scale=1.5)
+    q, k = b.q.clone(), b.k.clone()
+    # rows 3, 10, ... hold one smallest subnormal (2^-9) and zeros: with eps = 0
+    # their factor is sqrt(H) / 2^-9 = 2^15.5 for H = 8192
+    tiny = torch.zeros((H,), dtype=torch.float32)
+    tiny[H // 3] = 2.0 ** -9
+    for t in range(3, T, 7):
+        q[t] = tiny.to(torch.float8_e4m3fn)
+        k[t] = (-tiny).to(torch.float8_e4m3fn)
+    return b, q, k
+
+
+@pytest.mark.parametrize("gamma_kind", ["ordinary", "one large", "tiny and zero"])
+def test_e4m3_extreme_gamma_and_factors(gamma_kind):
+    """E4M3 rows at the edges of the arithmetic: gamma entries far from 1
+    (200, where x * gamma exceeds f16's range; 2^-20, below it; exact zeros)
+    and, with eps = 0, rows holding a single 2^-9 among 8192 zeros, whose
+    factor 2^-9 * sqrt(8192) ~ 2^15.5 scales the lone element to ~90.  Every
+    output within one E4M3 unit of the oracle; zero gamma gives exact zeros."""
+    T, H = 64, 8192
+    b, q, k = _e4m3_case(T, H, seed=91)
+    gq, gk = b.gamma_q.clone(), b.gamma_k.clone()
+    if gamma_kind == "one large":
+        gq[17] = 200.0
+    elif gamma_kind == "tiny and zero":
+        gq[5] = 2.0 ** -20
+        gk[::9] = 0.0
+    eps = 0.0
+    qo, ko = qk.qknorm_layerwise(q.to(DEV), k.to(DEV), gq.to(DEV), gk.to(DEV), eps)
+    torch.cuda.synchronize()
+    yq, eq, _ = oracle_rows(q, gq, eps)
+    yk, ek, _ = oracle_rows(k, gk, eps)
+    assert_close(qo, yq, eq, f"E4M3 Q ({gamma_kind})")
+    assert_close(ko, yk, ek, f"E4M3 K ({gamma_kind})")
+    if gamma_kind == "tiny and zero":
+        assert torch.all(ko.cpu().float()[:, ::9] == 0)
+    # the same through combine/apply with one shard
+    sq, sk = qk.qknorm_partial_stats(q.to(DEV), k.to(DEV))
+    ao, bo = qk.qknorm_combine_apply(q.to(DEV), k.to(DEV), gq.to(DEV), gk.to(DEV), sq[None], sk[None], H, H, eps)
+    torch.cuda.synchronize()
+    assert_close(ao, yq, eq, f"E4M3 apply Q ({gamma_kind})")
+    assert_close(bo, yk, ek, f"E4M3 apply K ({gamma_kind})")
 
 
 @pytest.mark.parametrize("T", workloads.PACKED_TOKENS)
