@@ -256,7 +256,6 @@ void fill_rowset(qkn::RowSet &s, const void *in, void *out, const void *gamma, i
     s.out = static_cast<char *>(out);
     s.gamma = static_cast<const char *>(gamma);
     s.sumsq = nullptr;
-    s.sumsq_all = nullptr;
     s.stride_bytes = stride * esz;
     s.width = width;
     s.nfull = width / per_vec;
@@ -310,8 +309,7 @@ void set_groups(qkn::ParamsT<SETS> &p, int threads, int nv) {
             }
         d.group = group;
         d.rows_per_item = threads / group;
-        d.items = (d.rows + d.rows_per_item - 1) / d.rows_per_item;
-        end += d.items;
+        end += (d.rows + d.rows_per_item - 1) / d.rows_per_item;  // items: rows_per_item rows each
         d.item_end = end;
     }
     p.n_items = end;

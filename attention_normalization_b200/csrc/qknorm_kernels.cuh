@@ -32,27 +32,31 @@ enum Mode : int {
     kApply = 2   // combine P partial sums -> factor -> scale and store
 };
 
-// One tensor's rows (Q or K, or a shard of one).
+// One tensor's rows (Q or K, or a shard of one).  Kept compact (96 bytes):
+// every launch copies the row sets as kernel parameters, and the small,
+// latency-bound launches (decode, tiny batches) pay for each byte.
 struct RowSet {
     const char *in;          // row t starts at in + t * stride_bytes
     char *out;               // kFused / kApply
     const char *gamma;       // kFused / kApply, [width] of the gamma type
-    float *sumsq;            // kStats: [T]
-    const float *sumsq_all;  // kApply: [P][T]
-    int32_t P;               // kApply: partial sums per token in sumsq_all
+    union {
+        float *sumsq;            // kStats: [T]
+        const float *sumsq_all;  // kApply: [P][T]
+    };
     int64_t stride_bytes;
+    int64_t head_bytes;      // headwise: bytes from one head to the next within a token's row
+    int64_t rows;            // T * heads
+    int64_t item_end;        // register kernel: items of this set and of every set before it
+    int32_t P;               // kApply: partial sums per token in sumsq_all
     int32_t width;           // elements in this row (shard width for kStats / kApply)
     int32_t nfull;           // full 16-byte vectors of x in the row
     int32_t tail;            // elements after the last full vector
     float inv_div;           // 1 / (the FULL width), rounded to fp32 on the host
     int32_t heads;           // rows per token: 1 (layerwise) or the number of heads (headwise)
-    int64_t head_bytes;      // headwise: bytes from one head to the next within a token's row
-    int64_t rows;            // T * heads
     int32_t group;           // register kernel: threads that share one row (1..16, or a multiple of 32)
     int32_t rows_per_item;   // register kernel: blockDim / group rows handled per item
-    int64_t items;           // register kernel: ceil(rows / rows_per_item)
-    int64_t item_end;        // register kernel: items of this set and of every set before it
 };
+static_assert(sizeof(RowSet) == 96, "row set layout");
 
 // The row sets of one launch: Q then K (SETS = 2), or -- for the multi-shard
 // forms of Phase A's local step and of the combine/apply -- the P Q shards
@@ -381,6 +385,16 @@ __device__ __forceinline__ void fma_sq_half2(uint32_t w, float &even, float &odd
         : "r"(w));
 }
 
+// Two E4M3 values -> their exact f16 pair, converted where it is used: the
+// squared-sum pass converts each pair itself, so the compiler does not keep
+// the converted pairs alive until the scaling pass (which converts again)
+// and a thread can hold more vectors in flight.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2_here(uint16_t two) {
+    uint32_t h;
+    asm volatile("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(two));
+    return h;
+}
+
 template <typename E>
 struct HalfSquares {  // element types whose squares take fma_sq_half2
     static constexpr bool value = false;
@@ -407,12 +421,8 @@ __device__ __forceinline__ float sumsq_pairs(const uint4 (&v)[NV]) {
                 if constexpr (sizeof(typename Elem<E>::Bits) == 2) {
                     fma_sq_half2(w[j], even, odd);
                 } else {  // two E4M3 pairs per word, each widened exactly to f16x2
-                    const __half2_raw lo =
-                        __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w[j] & 0xFFFFu), __NV_E4M3);
-                    const __half2_raw hi =
-                        __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w[j] >> 16), __NV_E4M3);
-                    fma_sq_half2(*reinterpret_cast<const uint32_t *>(&lo), even, odd);
-                    fma_sq_half2(*reinterpret_cast<const uint32_t *>(&hi), even, odd);
+                    fma_sq_half2(e4m3x2_to_f16x2_here(static_cast<uint16_t>(w[j] & 0xFFFFu)), even, odd);
+                    fma_sq_half2(e4m3x2_to_f16x2_here(static_cast<uint16_t>(w[j] >> 16)), even, odd);
                 }
             }
         }
@@ -502,6 +512,7 @@ __global__ void __launch_bounds__(RegisterBounds<NV>::kMaxThreads)
     const int warp = tid >> 5;
     const int64_t T = p.T;
     const int64_t n_items = p.n_items;
+    const int64_t q_end = p.set[0].item_end;  // two sets (Q, K): the item where K starts
 
     int which = -1;
     int64_t set_begin = 0, set_end = 0;  // items of the current set: [set_begin, set_end)
@@ -517,12 +528,25 @@ __global__ void __launch_bounds__(RegisterBounds<NV>::kMaxThreads)
     const char *gamma = nullptr;
 
     for (int64_t item = blockIdx.x; item < n_items; item += gridDim.x) {
-        if (item >= set_end) {  // uniform across the CTA: on to the set holding this item
-            do {
-                ++which;
-                set_begin = set_end;
-                set_end = p.set[which].item_end;
-            } while (item >= set_end);
+        bool next_set;  // uniform across the CTA: this item lies in another set than the last one
+        if constexpr (SETS == 2) {
+            const int w = item >= q_end ? 1 : 0;
+            next_set = w != which;
+            if (next_set) {
+                which = w;
+                set_begin = w ? q_end : 0;
+            }
+        } else {
+            next_set = item >= set_end;
+            if (next_set) {
+                do {
+                    ++which;
+                    set_begin = set_end;
+                    set_end = p.set[which].item_end;
+                } while (item >= set_end);
+            }
+        }
+        if (next_set) {
             const RowSet &d = p.set[which];
             in = d.in;
             out = d.out;
