@@ -247,6 +247,10 @@ __device__ __forceinline__ uint4 scale8(uint4 x, uint4 g, float r) {
     return make_uint4(ys[0], ys[1], ys[2], ys[3]);
 }
 
+__device__ __forceinline__ void red_release_add(int *p, int v) {
+    asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
 __device__ __forceinline__ int ld_acquire(const int *p) {
     int v;
     asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
@@ -257,7 +261,9 @@ __device__ __forceinline__ int ld_acquire(const int *p) {
 // tile, run by the 256 epilogue threads once every tile of its 128-token
 // strip has been counted: r = rsqrt(S / H + eps) with S the strip's partial
 // sums added in order p = 0, 1, ...; then (x * gamma) * r over the tile, in
-// place.  Partial sums written by other CTAs are read through L2 (.cg).
+// place.  Tiles and partial sums written by other CTAs are read through L2
+// (.cg).  Each warp issues the loads of its rows of the tile first, so they
+// are in flight while the factors are formed.
 __device__ __noinline__ void scale_tile(const GemmParams &p, int tensor, int m_tile, int n_tile, float *s_r) {
     const int et = threadIdx.x - 64;  // 0 .. 255
     const int P = tensor ? p.k_tiles : p.q_tiles;
@@ -266,6 +272,18 @@ __device__ __noinline__ void scale_tile(const GemmParams &p, int tensor, int m_t
     const float inv = tensor ? p.inv_hk : p.inv_hq;
     const int64_t row0 = static_cast<int64_t>(m_tile) * kBM;
     const int rows = static_cast<int>(p.T - row0 < kBM ? p.T - row0 : kBM);
+    // warp e takes rows e, e + 8, ...; lane l the l-th 16-byte vector of each
+    // (a tile row is 32 vectors), so every load and store is one whole row
+    const int e = et >> 5, lane = et & 31;
+    char *base = p.qkv + row0 * p.qkv_stride_bytes + static_cast<int64_t>(n_tile) * kBN * 2 + lane * 16;
+    constexpr int kBatch = kBM / kEpiWarps;  // rows per warp: the whole tile in flight at once
+    uint4 xv[kBatch];
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i) {
+        const int rr = e + kEpiWarps * i;
+        xv[i] = rr < rows ? __ldcg(reinterpret_cast<const uint4 *>(base + rr * p.qkv_stride_bytes))
+                          : make_uint4(0u, 0u, 0u, 0u);
+    }
     if (et < kBM) {
         float r = 0.0f;
         if (et < rows) {
@@ -284,28 +302,13 @@ __device__ __noinline__ void scale_tile(const GemmParams &p, int tensor, int m_t
         }
         s_r[et] = r;
     }
-    epilogue_sync();
-    // warp e takes rows e, e + 8, ...; lane l the l-th 16-byte vector of each
-    // (a tile row is 32 vectors), so every load and store is one whole row
-    const int e = et >> 5, lane = et & 31;
     const uint4 *gamma = reinterpret_cast<const uint4 *>(tensor ? p.gamma_k : p.gamma_q);
     const uint4 g = __ldg(gamma + (n_tile - first) * (kBN / 8) + lane);
-    char *base = p.qkv + row0 * p.qkv_stride_bytes + static_cast<int64_t>(n_tile) * kBN * 2 + lane * 16;
-    constexpr int kBatch = 16;  // rows in flight per warp
-#pragma unroll 1
-    for (int r0 = e; r0 < rows; r0 += kEpiWarps * kBatch) {
-        uint4 xv[kBatch];
+    epilogue_sync();  // the factors are in s_r
 #pragma unroll
-        for (int i = 0; i < kBatch; ++i) {
-            const int rr = r0 + kEpiWarps * i;
-            xv[i] = rr < rows ? __ldcg(reinterpret_cast<const uint4 *>(base + rr * p.qkv_stride_bytes))
-                              : make_uint4(0u, 0u, 0u, 0u);
-        }
-#pragma unroll
-        for (int i = 0; i < kBatch; ++i) {
-            const int rr = r0 + kEpiWarps * i;
-            if (rr < rows) *reinterpret_cast<uint4 *>(base + rr * p.qkv_stride_bytes) = scale8(xv[i], g, s_r[rr]);
-        }
+    for (int i = 0; i < kBatch; ++i) {
+        const int rr = e + kEpiWarps * i;
+        if (rr < rows) *reinterpret_cast<uint4 *>(base + rr * p.qkv_stride_bytes) = scale8(xv[i], g, s_r[rr]);
     }
     epilogue_sync();  // s_r is reused by the next tile
 }
@@ -562,10 +565,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (p.k_sumsq) p.k_sumsq[static_cast<int64_t>(n_tile - p.q_tiles) * p.T + row] = total;
                     }
                 }
-                if (fused) __threadfence();  // this thread's stores of the tile, before the count
-                epilogue_sync();             // s_half[b] has been read
-                // Count the tile on its strip (after every thread's fence above).
-                if (fused && warp == 2 && lane == 0) atomicAdd(p.counters + tensor * p.m_tiles + m_tile, 1);
+                epilogue_sync();  // every epilogue thread's stores of the tile precede this; s_half[b] read
+                // Count the tile on its strip: one thread, after the barrier,
+                // adds with release semantics at GPU scope, which orders the
+                // whole tile's stores (made visible to it by the barrier)
+                // before the count for the CTA that acquires the counter.
+                if (fused && warp == 2 && lane == 0) red_release_add(p.counters + tensor * p.m_tiles + m_tile, 1);
             }
             // Scale earlier tiles of this CTA whose strips are complete (at
             // most two per tile, inside the MMAs' slack).

@@ -46,8 +46,9 @@
 //                    two accumulators the epilogue of one tile overlaps the
 //                    MMAs of the next.
 // Fused QK-Norm (when `counters` is set): after storing a Q or K tile and its
-// partial sums, the epilogue makes its writes visible (fence) and counts the
-// tile on its strip's counter (one per 128-token strip and tensor).  Between
+// partial sums, the epilogue warps meet at a barrier and one thread counts the
+// tile on its strip's counter (one per 128-token strip and tensor) with a
+// GPU-scope release add, which publishes the whole tile.  Between
 // tiles it scales, in order, those of its own earlier Q / K tiles whose strips
 // are complete (counter = the tensor's tile count, read with acquire): the
 // strip's partial sums are added in order p = 0, 1, ... (fp32), r = rsqrt(S /
