@@ -124,3 +124,22 @@ def test_roofline_record_for_every_workload(kind, tokens, fake_root):
         assert r["floor_bytes_per_step"] > 1.49 * wl.eff_bytes
     else:
         assert "floor_bytes_per_step" not in r
+
+
+@pytest.mark.parametrize("kind", ["tiny", "decode"])
+def test_reference_arm_line_on_the_host(kind, capsys):
+    """The reference arm (the oracle on the host cores) prints one JSON line
+    with the contract's keys and the native arm's config, so the two lines
+    name the same workload."""
+    rc = bench.main(["--impl", "reference", "--workload", kind, "--steps", "1", "--warmup", "3"])
+    assert rc == 0
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better", "scaling",
+                "vs_baseline", "dtype", "data", "config", "impl", "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["impl"] == "reference" and line["value"] > 0
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
+    want = bench.Workload(kind, None, seed_offset=0).config()
+    want["parallelism"] = bench.parallelism(1)
+    assert line["config"] == want
