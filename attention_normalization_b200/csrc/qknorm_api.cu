@@ -196,6 +196,9 @@ const void *register_kernel(int nv) {
         case 2: return (const void *)qkn::rows_register_kernel<E, 2, MODE, TAIL, SETS>;
         case 4: return (const void *)qkn::rows_register_kernel<E, 4, MODE, TAIL, SETS>;
         case 8: return (const void *)qkn::rows_register_kernel<E, 8, MODE, TAIL, SETS>;
+        case 5:  // one warp per row of 129..160 vectors (a partial-sum or apply pass over shards)
+            if constexpr (MODE == qkn::kFused) return nullptr;
+            else return (const void *)qkn::rows_register_kernel<E, 5, MODE, TAIL, SETS>;
         default: return nullptr;
     }
 }
@@ -410,6 +413,21 @@ qkn_status plan_call(const CallT<SETS> &c, qkn_launch &L) {
             L.threads = 128;
         }
     }
+    int oversubscribe = 1;  // CTAs per resident slot
+    if (MODE == qkn::kApply && L.kernel == QKN_KERNEL_REGISTER && items > sms && c.units_max > 128 &&
+        c.units_max <= 160) {
+        // Rows of 129..160 vectors (a hidden dimension split into shards):
+        // one warp per row with 5 vectors per lane covers it without idle
+        // lanes or a CTA barrier; 8 rows per CTA, and four CTAs per resident
+        // slot, so that CTAs finishing early take the next ones and the
+        // ragged end of the row list spreads over the SMs.  (One B200, the
+        // GQA step's apply pass over 4 + 4 shards of 1280 + 256 bf16 columns
+        // for 16384 tokens: 62.8 us against 68.0 us for 2 vectors per lane in
+        // 96-thread CTAs at one CTA per slot.)
+        L.vec_per_thread = 5;
+        L.threads = 256;
+        oversubscribe = 4;
+    }
     const void *fn = kernel_for<MODE, SETS>(c.dtype, L, c.tail);
     if (!fn) return fail(QKN_ERR_UNSUPPORTED, "no kernel for the planned launch");
     if ((st = blocks_per_sm(fn, dev, L.threads, 0, &bps)) != QKN_OK) return st;
@@ -419,11 +437,11 @@ qkn_status plan_call(const CallT<SETS> &c, qkn_launch &L) {
         set_groups(p, L.threads, L.vec_per_thread);
         work = p.n_items;
     }
-    L.grid = qknorm_plan_grid(work, bps, sms);
+    L.grid = qknorm_plan_grid(work, bps * oversubscribe, sms);
     return QKN_OK;
 }
 
-template <int SETS>
+template <int MODE, int SETS>
 qkn_status check_launch(const CallT<SETS> &c, const qkn_launch &L) {
     if (L.threads < 32 || L.threads > 1024 || (L.threads % 32) != 0)
         return fail(QKN_ERR_INVALID_ARG, "threads must be a multiple of 32 in [32, 1024], got %d", L.threads);
@@ -431,7 +449,9 @@ qkn_status check_launch(const CallT<SETS> &c, const qkn_launch &L) {
     switch (L.kernel) {
         case QKN_KERNEL_REGISTER: {
             const int mt = qknorm_register_max_threads(L.vec_per_thread);
-            if (mt == 0) return fail(QKN_ERR_INVALID_ARG, "vec_per_thread must be 1, 2, 4 or 8");
+            if (mt == 0 || (MODE == qkn::kFused && L.vec_per_thread == 5))
+                return fail(QKN_ERR_INVALID_ARG, MODE == qkn::kFused ? "vec_per_thread must be 1, 2, 4 or 8"
+                                                                     : "vec_per_thread must be 1, 2, 4, 5 or 8");
             if (L.threads > mt) return fail(QKN_ERR_INVALID_ARG, "threads above %d for vec_per_thread %d", mt, L.vec_per_thread);
             if (!c.vectorized) return fail(QKN_ERR_INVALID_ARG, "register kernel needs 16-byte aligned buffers");
             if ((int64_t)L.vec_per_thread * L.threads < c.units_max)
@@ -917,6 +937,7 @@ int32_t qknorm_register_max_threads(int32_t vec_per_thread) {
         case 2: return qkn::RegisterBounds<2>::kMaxThreads;
         case 4: return qkn::RegisterBounds<4>::kMaxThreads;
         case 8: return qkn::RegisterBounds<8>::kMaxThreads;
+        case 5: return qkn::RegisterBounds<5>::kMaxThreads;
         default: return 0;
     }
 }
@@ -1033,7 +1054,7 @@ qkn_status qknorm_layerwise_launch(const void *q_in, void *q_out, const void *ga
     qkn_status st = prepare_layerwise(q_in, q_out, gamma_q, q_stride, k_in, k_out, gamma_k, k_stride, T, Hq,
                                       Hk, eps, dtype, c);
     if (st != QKN_OK) return st;
-    if ((st = check_launch(c, *launch_cfg)) != QKN_OK) return st;
+    if ((st = check_launch<qkn::kFused>(c, *launch_cfg)) != QKN_OK) return st;
     if (T == 0) return ok();
     return launch<qkn::kFused>(c, *launch_cfg, stream);
 }
@@ -1060,7 +1081,7 @@ qkn_status qknorm_headwise_launch(const void *q_in, void *q_out, const void *gam
     qkn_status st = prepare_headwise(q_in, q_out, gamma_q, q_stride, q_heads, k_in, k_out, gamma_k, k_stride,
                                      k_heads, T, head_dim, eps, dtype, c);
     if (st != QKN_OK) return st;
-    if ((st = check_launch(c, *launch_cfg)) != QKN_OK) return st;
+    if ((st = check_launch<qkn::kFused>(c, *launch_cfg)) != QKN_OK) return st;
     if (T == 0) return ok();
     return launch<qkn::kFused>(c, *launch_cfg, stream);
 }
@@ -1086,7 +1107,7 @@ qkn_status qknorm_partial_stats_launch(const void *q_shard, int64_t q_stride, in
     qkn_status st = prepare_stats(q_shard, q_stride, hq_shard, q_sumsq, k_shard, k_stride, hk_shard, k_sumsq, T,
                                   dtype, c);
     if (st != QKN_OK) return st;
-    if ((st = check_launch(c, *launch_cfg)) != QKN_OK) return st;
+    if ((st = check_launch<qkn::kStats>(c, *launch_cfg)) != QKN_OK) return st;
     if (T == 0) return ok();
     return launch<qkn::kStats>(c, *launch_cfg, stream);
 }
@@ -1117,7 +1138,7 @@ qkn_status qknorm_combine_apply_launch(const void *q_in, void *q_out, const void
     qkn_status st = prepare_apply(q_in, q_out, gamma_q_shard, q_stride, hq_shard, q_sumsq_all, Hq_full, k_in, k_out,
                                   gamma_k_shard, k_stride, hk_shard, k_sumsq_all, Hk_full, P, T, eps, dtype, c);
     if (st != QKN_OK) return st;
-    if ((st = check_launch(c, *launch_cfg)) != QKN_OK) return st;
+    if ((st = check_launch<qkn::kApply>(c, *launch_cfg)) != QKN_OK) return st;
     if (T == 0) return ok();
     return launch<qkn::kApply>(c, *launch_cfg, stream);
 }
@@ -1136,7 +1157,7 @@ qkn_status stats_shards(int32_t P, const void *const *q_shards, int64_t q_stride
     if (pinned) {
         if (T > 0 && !one_launch(c))
             return fail(QKN_ERR_INVALID_ARG, "a pinned launch needs 16-byte aligned shard rows of at most 32 KB");
-        if (T > 0 && (st = check_launch(c, *pinned)) != QKN_OK) return st;
+        if (T > 0 && (st = check_launch<qkn::kStats>(c, *pinned)) != QKN_OK) return st;
         if (T > 0 && pinned->kernel != QKN_KERNEL_REGISTER)
             return fail(QKN_ERR_INVALID_ARG, "multi-shard calls run the register kernel only");
         if (T == 0) return ok();
@@ -1169,7 +1190,7 @@ qkn_status apply_shards(int32_t P, const void *const *q_in, void *const *q_out, 
     if (pinned) {
         if (T > 0 && !one_launch(c))
             return fail(QKN_ERR_INVALID_ARG, "a pinned launch needs 16-byte aligned shard rows of at most 32 KB");
-        if (T > 0 && (st = check_launch(c, *pinned)) != QKN_OK) return st;
+        if (T > 0 && (st = check_launch<qkn::kApply>(c, *pinned)) != QKN_OK) return st;
         if (T > 0 && pinned->kernel != QKN_KERNEL_REGISTER)
             return fail(QKN_ERR_INVALID_ARG, "multi-shard calls run the register kernel only");
         if (T == 0) return ok();

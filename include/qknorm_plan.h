@@ -46,13 +46,16 @@ typedef enum {
 
 typedef struct {
     int32_t kernel;          /* qkn_kernel_kind */
-    int32_t vec_per_thread;  /* QKN_KERNEL_REGISTER only: 1, 2, 4 or 8 */
+    int32_t vec_per_thread;  /* QKN_KERNEL_REGISTER only: 1, 2, 4 or 8; also 5 for the
+                                partial-sum and combine/apply passes (one warp per row
+                                of 129..160 vectors) */
     int32_t threads;         /* threads per CTA: a multiple of 32 in [32, 1024] */
     int64_t grid;            /* number of CTAs, >= 1 */
 } qkn_launch;
 
 /* Largest CTA the register kernel accepts for a given vec_per_thread
- * (1024 for 1 and 2, 512 for 4, 256 for 8); 0 for an unsupported value. */
+ * (1024 for 1 and 2, 512 for 4, 256 for 5 and 8); 0 for an unsupported
+ * value.  5 exists for the partial-sum and combine/apply passes only. */
 int32_t qknorm_register_max_threads(int32_t vec_per_thread);
 
 /*

@@ -186,6 +186,7 @@ def test_launch_override_validation(lib):
     assert st(0, 4, 128, 100) == OK  # T = 0: validated, nothing launched
     assert st(0, 4, 96, 100) == INVALID  # 4 * 96 < 512 vectors
     assert st(0, 3, 256, 100) == INVALID  # vec_per_thread
+    assert st(0, 5, 128, 100) == INVALID  # 5: the partial-sum and apply passes only
     assert st(0, 8, 512, 100) == INVALID  # above the NV=8 limit
     assert st(0, 4, 100, 100) == INVALID  # not a multiple of 32
     assert st(0, 4, 128, 0) == INVALID  # grid
@@ -215,6 +216,7 @@ def test_shard_launch_override_validation(lib):
         zero = list(args)
         zero[8 if f is lib.qknorm_partial_stats_launch else 15] = 0  # T = 0: validated, nothing launched
         assert f(*zero, ctypes.byref(_clib.QknLaunch(0, 2, 96, 10))) == OK
+        assert f(*zero, ctypes.byref(_clib.QknLaunch(0, 5, 32, 10))) == OK  # one warp per 160-vector shard row
         assert f(*zero, ctypes.byref(_clib.QknLaunch(0, 1, 96, 10))) == INVALID  # 96 < 160 vectors
         assert f(*zero, ctypes.byref(_clib.QknLaunch(0, 2, 100, 10))) == INVALID
         assert f(*zero, None) == INVALID

@@ -239,7 +239,8 @@ def test_multi_shard_calls_match_the_oracle(dtype, P, T, Hq, Hk, pad):
 @pytest.mark.parametrize("launch", [{"kernel": 0, "vec_per_thread": 2, "threads": 96, "grid": 7},
                                     {"kernel": 0, "vec_per_thread": 4, "threads": 128, "grid": 300},
                                     {"kernel": 0, "vec_per_thread": 1, "threads": 160, "grid": 1184},
-                                    {"kernel": 0, "vec_per_thread": 8, "threads": 64, "grid": 50}])
+                                    {"kernel": 0, "vec_per_thread": 8, "threads": 64, "grid": 50},
+                                    {"kernel": 0, "vec_per_thread": 5, "threads": 128, "grid": 592}])
 def test_multi_shard_pinned_launches_match_the_oracle(launch):
     """Any valid launch of the multi-shard calls (rows grouped differently,
     any grid) gives the oracle's results."""
