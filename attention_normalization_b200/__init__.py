@@ -29,7 +29,7 @@ __all__ = ["qknorm_layerwise", "qknorm_headwise", "qknorm_qkv_gemm_stats", "qkno
            "qknorm_partial_stats", "qknorm_combine_apply", "qknorm_partial_stats_shards",
            "qknorm_combine_apply_shards", "gamma_dtype",
            "qknorm_layerwise_plan", "qknorm_layerwise_host", "qknorm_packed_host",
-           "plan_shape", "plan_grid", "regions_overlap", "capi", "version", "QknLaunch", "QKNormError"]
+           "plan_shape", "plan_grid", "regions_overlap", "qkv_gemm_schedule", "qkv_gemm_plan", "capi", "version", "QknLaunch", "QKNormError"]
 
 _DTYPES = {torch.float32: _clib.QKN_F32, torch.bfloat16: _clib.QKN_BF16, torch.float16: _clib.QKN_F16,
            torch.float8_e4m3fn: _clib.QKN_FP8_E4M3}
@@ -389,6 +389,27 @@ def qknorm_layerwise_plan(q_in, k_in, gamma_q, gamma_k, eps: float = 1e-6, *, q_
         st = capi().qknorm_layerwise_plan(*args, ctypes.byref(L))
     _clib.check(st, "qknorm_layerwise_plan")
     return L.as_dict()
+
+
+def qkv_gemm_schedule(T: int, D: int, Hq: int, Hk: int, Hv: int, clusters: int, l2_bytes: int) -> dict:
+    """The projection GEMM's schedule for ``clusters`` resident CTA pairs and
+    an L2 of ``l2_bytes`` (pure; no GPU needed)."""
+    S = _clib.QknGemmSchedule()
+    st = capi().qknorm_qkv_gemm_schedule(int(T), int(D), int(Hq), int(Hk), int(Hv), int(clusters), int(l2_bytes),
+                                         ctypes.byref(S))
+    _clib.check(st, "qknorm_qkv_gemm_schedule")
+    return S.as_dict()
+
+
+def qkv_gemm_plan(T: int, D: int, Hq: int, Hk: int, Hv: int, device=None) -> dict:
+    """The schedule the projection entry points use for this shape on
+    ``device`` (default: the current CUDA device)."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    S = _clib.QknGemmSchedule()
+    with _on(dev):
+        st = capi().qknorm_qkv_gemm_plan(int(T), int(D), int(Hq), int(Hk), int(Hv), ctypes.byref(S))
+    _clib.check(st, "qknorm_qkv_gemm_plan")
+    return S.as_dict()
 
 
 def _launch_struct(launch):

@@ -36,6 +36,14 @@ class QknLaunch(ctypes.Structure):
                 "threads": self.threads, "grid": self.grid}
 
 
+class QknGemmSchedule(ctypes.Structure):
+    """Mirror of ``qkn_gemm_schedule``."""
+    _fields_ = [("clusters", ctypes.c_int32), ("units", ctypes.c_int32), ("group_units", ctypes.c_int32)]
+
+    def as_dict(self) -> dict:
+        return {f: getattr(self, f) for f, _ in self._fields_}
+
+
 # Every symbol the headers declare, with (restype, argtypes).
 _vp, _i64, _i32, _u64, _f32 = (ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32,
                                ctypes.c_uint64, ctypes.c_float)
@@ -45,6 +53,8 @@ _LAYERWISE_ARGS = [_vp, _vp, _vp, _i64, _vp, _vp, _vp, _i64, _i64, _i32, _i32, _
 _HEADWISE_ARGS = [_vp, _vp, _vp, _i64, _i32, _vp, _vp, _vp, _i64, _i32, _i64, _i32, _f32, _dt]
 
 PROTOTYPES = {
+    "qknorm_qkv_gemm_schedule": (_st, [_i64, _i32, _i32, _i32, _i32, _i32, _i64, ctypes.POINTER(QknGemmSchedule)]),
+    "qknorm_qkv_gemm_plan": (_st, [_i64, _i32, _i32, _i32, _i32, ctypes.POINTER(QknGemmSchedule)]),
     "qknorm_layerwise": (_st, _LAYERWISE_ARGS + [_vp]),
     "qknorm_partial_stats": (_st, [_vp, _i64, _i32, _vp, _vp, _i64, _i32, _vp, _i64, _dt, _vp]),
     "qknorm_headwise": (_st, _HEADWISE_ARGS + [_vp]),

@@ -828,6 +828,37 @@ struct FusedNorm {
 
 int64_t projection_m_tiles(int64_t T) { return (T + qkn::gemm::kBM - 1) / qkn::gemm::kBM; }
 
+// The tile counts of a projection of T tokens, D inputs and Hq + Hk + Hv
+// outputs (Hq, Hk, Hv multiples of kTileN).
+void gemm_tiles(int64_t T, int32_t D, int32_t Hq, int32_t Hk, int32_t Hv, qkn::gemm::GemmParams &gp) {
+    gp.T = T;
+    gp.k_blocks = (D + qkn::gemm::kBK - 1) / qkn::gemm::kBK;
+    gp.q_tiles = Hq / kTileN;
+    gp.k_tiles = Hk / kTileN;
+    gp.n_tiles = (Hq + Hk + Hv) / kTileN;
+    gp.m_tiles = (int32_t)((T + qkn::gemm::kBM - 1) / qkn::gemm::kBM);
+    gp.m_units = (int32_t)((T + qkn::gemm::kBM * qkn::gemm::kCta - 1) / (qkn::gemm::kBM * qkn::gemm::kCta));
+    gp.num_units = gp.m_units * gp.n_tiles;
+}
+
+qkn_status check_gemm_shape(int64_t T, int32_t D, int32_t Hq, int32_t Hk, int32_t Hv) {
+    if (T < 1 || T >= ((int64_t)1 << 31)) return fail(QKN_ERR_INVALID_ARG, "T must be in [1, 2^31)");
+    if (D <= 0 || Hq <= 0 || Hk <= 0 || Hv < 0) return fail(QKN_ERR_INVALID_ARG, "D, Hq, Hk must be positive, Hv >= 0");
+    if (Hq % kTileN || Hk % kTileN || Hv % kTileN)
+        return fail(QKN_ERR_UNSUPPORTED, "Hq, Hk and Hv must be multiples of %d (the output tile)", kTileN);
+    const int64_t N = (int64_t)Hq + Hk + Hv;
+    if (N > INT32_MAX) return fail(QKN_ERR_INVALID_ARG, "Hq + Hk + Hv overflows");
+    if (((T + 127) / 128) * (N / kTileN) > ((int64_t)1 << 30))
+        return fail(QKN_ERR_UNSUPPORTED, "more than 2^30 output tiles");
+    return QKN_OK;
+}
+
+void fill_schedule(const qkn::gemm::GemmParams &gp, int32_t clusters, qkn_gemm_schedule *out) {
+    out->clusters = gp.num_units < clusters ? gp.num_units : clusters;
+    out->units = gp.num_units;
+    out->group_units = gp.group_units;
+}
+
 qkn_status launch_projection_gemm(const Projection &pr, float *q_sums, float *k_sums, void *stream,
                                   const FusedNorm *fuse = nullptr) {
     qkn::gemm::GemmParams gp{};
@@ -835,14 +866,7 @@ qkn_status launch_projection_gemm(const Projection &pr, float *q_sums, float *k_
     gp.qkv_stride_bytes = pr.qkv_stride * 2;
     gp.q_sumsq = q_sums;
     gp.k_sumsq = k_sums;
-    gp.T = pr.T;
-    gp.k_blocks = (pr.D + qkn::gemm::kBK - 1) / qkn::gemm::kBK;
-    gp.q_tiles = pr.Hq / kTileN;
-    gp.k_tiles = pr.Hk / kTileN;
-    gp.n_tiles = pr.N / kTileN;
-    gp.m_tiles = (int32_t)((pr.T + qkn::gemm::kBM - 1) / qkn::gemm::kBM);
-    gp.m_units = (int32_t)((pr.T + qkn::gemm::kBM * qkn::gemm::kCta - 1) / (qkn::gemm::kBM * qkn::gemm::kCta));
-    gp.num_units = gp.m_units * gp.n_tiles;
+    gemm_tiles(pr.T, pr.D, pr.Hq, pr.Hk, pr.Hv, gp);
     gp.timeout_ns = kGemmTimeoutNs;
     if (fuse) {
         gp.counters = fuse->counters;
@@ -1281,6 +1305,33 @@ int64_t qknorm_qkv_projection_workspace_bytes(int64_t T, int32_t Hq, int32_t Hk)
     if (T < 0 || Hq <= 0 || Hk <= 0 || Hq % kTileN || Hk % kTileN) return -1;
     // partial sums [Hq/256][T] and [Hk/256][T], then two strip counters per 128 tokens
     return (int64_t)(Hq / kTileN + Hk / kTileN) * T * 4 + 2 * projection_m_tiles(T) * 4;
+}
+
+qkn_status qknorm_qkv_gemm_schedule(int64_t T, int32_t D, int32_t Hq, int32_t Hk, int32_t Hv, int32_t clusters,
+                                    int64_t l2_bytes, qkn_gemm_schedule *out) {
+    if (!out) return fail(QKN_ERR_INVALID_ARG, "null output");
+    qkn_status st = check_gemm_shape(T, D, Hq, Hk, Hv);
+    if (st != QKN_OK) return st;
+    if (clusters < 1 || l2_bytes < 0) return fail(QKN_ERR_INVALID_ARG, "clusters must be >= 1 and l2_bytes >= 0");
+    qkn::gemm::GemmParams gp{};
+    gemm_tiles(T, D, Hq, Hk, Hv, gp);
+    qkn::gemm::schedule_qkv_gemm(&gp, D, Hq + Hk + Hv, clusters, l2_bytes);
+    fill_schedule(gp, clusters, out);
+    return ok();
+}
+
+qkn_status qknorm_qkv_gemm_plan(int64_t T, int32_t D, int32_t Hq, int32_t Hk, int32_t Hv, qkn_gemm_schedule *out) {
+    if (!out) return fail(QKN_ERR_INVALID_ARG, "null output");
+    qkn_status st = check_gemm_shape(T, D, Hq, Hk, Hv);
+    if (st != QKN_OK) return st;
+    int clusters = 0, dev = 0, l2 = 0;
+    const char *what = "";
+    cudaError_t e = qkn::gemm::qkv_gemm_clusters(&clusters, &what);
+    if (e == cudaSuccess && (e = cudaGetDevice(&dev)) != cudaSuccess) what = "cudaGetDevice";
+    if (e == cudaSuccess && (e = cudaDeviceGetAttribute(&l2, cudaDevAttrL2CacheSize, dev)) != cudaSuccess)
+        what = "cudaDeviceGetAttribute(L2 cache size)";
+    if (e != cudaSuccess) return fail(QKN_ERR_CUDA, "projection plan (%s): %s", what, cudaGetErrorString(e));
+    return qknorm_qkv_gemm_schedule(T, D, Hq, Hk, Hv, clusters, l2, out);
 }
 
 qkn_status qknorm_qkv_projection(const void *x, int64_t x_stride, const void *w, int64_t w_stride, void *qkv,

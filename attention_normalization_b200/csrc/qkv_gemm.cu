@@ -49,6 +49,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return done != 0;
 }
 
+// Non-blocking: true if the phase of parity `parity` has completed.
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
 // True once the phase of parity `parity` has completed; false when
 // `timeout_ns` of global time passed first.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_t timeout_ns) {
@@ -217,15 +230,20 @@ __device__ __forceinline__ bool epilogue_all(bool ok) {
 struct TileRef {
     int m_tile, n_tile;
 };
-__device__ __forceinline__ TileRef cta_tile(const GemmParams &p, int j, int rank) {
-    const int clusters = static_cast<int>(gridDim.x) / kCta;
-    const int u = static_cast<int>(blockIdx.x) / kCta + j * clusters;
+__host__ __device__ __forceinline__ void unit_tile(const GemmParams &p, int u, int *m_unit, int *n_tile) {
     const int span = p.group_units * p.n_tiles;
     const int g = u / span;
     const int v = u - g * span;
     const int first = g * p.group_units;
-    const int rows = min(p.group_units, p.m_units - first);
-    return TileRef{(first + v % rows) * kCta + rank, v / rows};
+    const int rows = p.group_units < p.m_units - first ? p.group_units : p.m_units - first;
+    *m_unit = first + v % rows;
+    *n_tile = v / rows;
+}
+__device__ __forceinline__ TileRef cta_tile(const GemmParams &p, int j, int rank) {
+    const int clusters = static_cast<int>(gridDim.x) / kCta;
+    int m_unit, n_tile;
+    unit_tile(p, static_cast<int>(blockIdx.x) / kCta + j * clusters, &m_unit, &n_tile);
+    return TileRef{m_unit * kCta + rank, n_tile};
 }
 __device__ __forceinline__ int cta_tile_count(const GemmParams &p) {
     const int clusters = static_cast<int>(gridDim.x) / kCta;
@@ -287,15 +305,15 @@ __device__ __noinline__ void scale_tile(const GemmParams &p, int tensor, int m_t
     if (et < kBM) {
         float r = 0.0f;
         if (et < rows) {
-            // eight loads in flight at a time, added strictly in order p = 0, 1, ...
+            // sixteen loads in flight at a time, added strictly in order p = 0, 1, ...
             const float *col = sums + row0 + et;
             float S = 0.0f;
-            for (int q0 = 0; q0 < P; q0 += 8) {
-                float v[8];
+            for (int q0 = 0; q0 < P; q0 += 16) {
+                float v[16];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) v[i] = q0 + i < P ? __ldcg(col + static_cast<int64_t>(q0 + i) * p.T) : 0.0f;
+                for (int i = 0; i < 16; ++i) v[i] = q0 + i < P ? __ldcg(col + static_cast<int64_t>(q0 + i) * p.T) : 0.0f;
 #pragma unroll
-                for (int i = 0; i < 8; ++i)
+                for (int i = 0; i < 16; ++i)
                     if (q0 + i < P) S += v[i];
             }
             r = rsqrtf(__fmaf_rn(S, inv, p.eps));
@@ -315,14 +333,16 @@ __device__ __noinline__ void scale_tile(const GemmParams &p, int tensor, int m_t
 
 // Scales this CTA's stored Q / K tiles from sequence index `from` up to (not
 // including) `upto`, in order, while their strips are complete.  Without
-// `wait` it stops at the first incomplete strip or after `budget` tiles; with
-// `wait` (only once all of this CTA's own tiles are stored and counted, so
-// it never waits on itself) it waits, bounded, for each strip.  Returns the
-// next index to scale.
+// `wait` it stops at the first incomplete strip, or once `budget` tiles are
+// done and -- when `next_bar` is not 0 -- the phase `next_parity` of that
+// barrier (the next tile's accumulator) has completed; with `wait` (only
+// once all of this CTA's own tiles are stored and counted, so it never waits
+// on itself) it waits, bounded, for each strip.  Returns the next index to
+// scale.
 __device__ int scale_ready_tiles(const GemmParams &p, int from, int upto, bool wait, int budget, float *s_r,
-                                 int *abort_flag, int rank) {
+                                 int *abort_flag, int rank, uint32_t next_bar = 0, uint32_t next_parity = 0) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    while (from < upto && budget > 0) {
+    while (from < upto && (wait || budget > 0 || next_bar != 0)) {
         const TileRef tr = cta_tile(p, from, rank);
         const int m_tile = tr.m_tile, n_tile = tr.n_tile;
         if (m_tile >= p.m_tiles) {  // the pair's second token tile lies past T
@@ -336,10 +356,12 @@ __device__ int scale_ready_tiles(const GemmParams &p, int from, int upto, bool w
         }
         bool ready = true;
         if (warp == 2 && lane == 0) {
+            // past the budget, go on only while the next accumulator is not complete
+            const bool more = wait || budget > 0 || (next_bar != 0 && !mbar_test(next_bar, next_parity));
             const int *cnt = p.counters + tensor * p.m_tiles + m_tile;
             const int P = tensor ? p.k_tiles : p.q_tiles;
-            ready = ld_acquire(cnt) >= P;
-            if (!ready && wait) {
+            ready = more && ld_acquire(cnt) >= P;
+            if (more && !ready && wait) {
                 const uint64_t t0 = global_ns();
                 while (!(ready = ld_acquire(cnt) >= P)) {
                     if (global_ns() - t0 > p.timeout_ns) {
@@ -572,9 +594,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // before the count for the CTA that acquires the counter.
                 if (fused && warp == 2 && lane == 0) red_release_add(p.counters + tensor * p.m_tiles + m_tile, 1);
             }
-            // Scale earlier tiles of this CTA whose strips are complete (at
-            // most two per tile, inside the MMAs' slack).
-            if (fused) norm_next = scale_ready_tiles(p, norm_next, j + 1, false, 2, s_r, &s_abort, rank);
+            // Scale earlier tiles of this CTA whose strips are complete: two,
+            // and then more while the next tile's accumulator is not complete
+            // (the epilogue would only wait for it).
+            if (fused) {
+                const bool next = kAdaptiveRescale && j + 1 < n_tiles_cta;
+                norm_next = scale_ready_tiles(p, norm_next, j + 1, false, 2, s_r, &s_abort, rank,
+                                              next ? acc_full_bar((j + 1) & 1) : 0u,
+                                              static_cast<uint32_t>(((j + 1) >> 1) & 1));
+            }
         }
         if (fused && !timed_out)
             scale_ready_tiles(p, norm_next, j, true, 1 << 30, s_r, &s_abort, rank);
@@ -678,24 +706,34 @@ int raster_group_units(int m_units, int D, int N, int clusters, int l2_bytes) {
     return g < 1 ? 1 : (g > m_units ? m_units : g);
 }
 
+// The launch configuration shared by the launch and the occupancy query.
+void base_config(cudaLaunchConfig_t *cfg, cudaLaunchAttribute (&attr)[2], cudaStream_t stream) {
+    *cfg = cudaLaunchConfig_t{};
+    cfg->blockDim = dim3(kThreads);
+    cfg->dynamicSmemBytes = kSmemBytes;
+    cfg->stream = stream;
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = kCta;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg->attrs = attr;
+    cfg->numAttrs = kCta == 2 ? 2 : 1;
+}
+
 }  // namespace
 
-cudaError_t launch_qkv_gemm(const void *x, int64_t x_stride, const void *w, int64_t w_stride, int32_t D,
-                            int32_t N, const GemmParams &p, cudaStream_t stream, const char **what) {
-    PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    cudaError_t e = encoder(&fn);
-    if (e != cudaSuccess) {
-        *what = "cuTensorMapEncodeTiled entry point";
-        return e;
-    }
-    CUtensorMap tx, tw;
-    if (!encode_bf16_rows(fn, &tx, x, D, p.T, x_stride, kBM) ||
-        !encode_bf16_rows(fn, &tw, w, D, N, w_stride, kBNLocal)) {  // each CTA stages kBNLocal W rows
-        *what = "cuTensorMapEncodeTiled";
-        return cudaErrorInvalidValue;
-    }
+void schedule_qkv_gemm(GemmParams *p, int32_t D, int32_t N, int clusters, int64_t l2_bytes) {
+    const int units = p->num_units < clusters ? p->num_units : clusters;
+    p->group_units = raster_group_units(p->m_units, D, N, units > 0 ? units : 1,
+                                        static_cast<int>(l2_bytes > (int64_t(1) << 30) ? (int64_t(1) << 30) : l2_bytes));
+}
+
+cudaError_t qkv_gemm_clusters(int *clusters, const char **what) {
     int dev = 0;
-    if ((e = cudaGetDevice(&dev)) != cudaSuccess) {
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) {
         *what = "cudaGetDevice";
         return e;
     }
@@ -710,22 +748,12 @@ cudaError_t launch_qkv_gemm(const void *x, int64_t x_stride, const void *w, int6
             if (dev >= 0 && dev < kMaxDevices) g_smem_set[dev] = true;
         }
     }
-    cudaLaunchConfig_t cfg = {};
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = kSmemBytes;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[2];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    attr[1].id = cudaLaunchAttributeClusterDimension;
-    attr[1].val.clusterDim.x = kCta;
-    attr[1].val.clusterDim.y = 1;
-    attr[1].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = kCta == 2 ? 2 : 1;
     // Persistent: one CTA per SM (its shared memory allows no second one), as
     // many CTA groups as can be resident at once, so every group runs from
     // the start (a group that waited for a free SM would finish last).
+    cudaLaunchConfig_t cfg;
+    cudaLaunchAttribute attr[2];
+    base_config(&cfg, attr, nullptr);
     int groups = 0;
     {
         std::lock_guard<std::mutex> lk(g_smem_mu);
@@ -753,15 +781,42 @@ cudaError_t launch_qkv_gemm(const void *x, int64_t x_stride, const void *w, int6
         std::lock_guard<std::mutex> lk(g_smem_mu);
         if (dev >= 0 && dev < kMaxDevices) g_groups[dev] = groups;
     }
-    const int units = p.num_units < groups ? p.num_units : groups;
-    cfg.gridDim = dim3(static_cast<unsigned>((units > 0 ? units : 1) * kCta));
-    int l2 = 0;
+    *clusters = groups;
+    return cudaSuccess;
+}
+
+cudaError_t launch_qkv_gemm(const void *x, int64_t x_stride, const void *w, int64_t w_stride, int32_t D,
+                            int32_t N, const GemmParams &p, cudaStream_t stream, const char **what) {
+    PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    cudaError_t e = encoder(&fn);
+    if (e != cudaSuccess) {
+        *what = "cuTensorMapEncodeTiled entry point";
+        return e;
+    }
+    CUtensorMap tx, tw;
+    if (!encode_bf16_rows(fn, &tx, x, D, p.T, x_stride, kBM) ||
+        !encode_bf16_rows(fn, &tw, w, D, N, w_stride, kBNLocal)) {  // each CTA stages kBNLocal W rows
+        *what = "cuTensorMapEncodeTiled";
+        return cudaErrorInvalidValue;
+    }
+    int groups = 0;
+    if ((e = qkv_gemm_clusters(&groups, what)) != cudaSuccess) return e;
+    int dev = 0, l2 = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) {
+        *what = "cudaGetDevice";
+        return e;
+    }
     if ((e = cudaDeviceGetAttribute(&l2, cudaDevAttrL2CacheSize, dev)) != cudaSuccess) {
         *what = "cudaDeviceGetAttribute(L2 cache size)";
         return e;
     }
+    cudaLaunchConfig_t cfg;
+    cudaLaunchAttribute attr[2];
+    base_config(&cfg, attr, stream);
+    const int units = p.num_units < groups ? p.num_units : groups;
+    cfg.gridDim = dim3(static_cast<unsigned>((units > 0 ? units : 1) * kCta));
     GemmParams q = p;
-    q.group_units = raster_group_units(p.m_units, D, N, units, l2);
+    schedule_qkv_gemm(&q, D, N, groups, l2);
     void *args[] = {&tx, &tw, &q};
     e = cudaLaunchKernelExC(&cfg, reinterpret_cast<const void *>(qkv_gemm_stats_kernel), args);
     if (e != cudaSuccess) *what = "cudaLaunchKernelExC";

@@ -83,7 +83,13 @@ constexpr int kUmmaK = 16;         // K of one tcgen05.mma kind::f16
 // tile.
 constexpr int kCta = QKN_GEMM_CTA_GROUP;
 static_assert(kCta == 1 || kCta == 2, "one or two CTAs per MMA");
-constexpr int kStages = kCta == 2 ? 6 : 4;
+#ifndef QKN_GEMM_STAGES
+#define QKN_GEMM_STAGES 0
+#endif
+// Shared-memory ring depth: 6 x 32 KB for the pair form, 4 x 48 KB with one
+// CTA per tile.  (Measured on a B200: 7 x 32 KB, the most that fits, was 1-2%
+// slower than 6 at T = 4096.)
+constexpr int kStages = QKN_GEMM_STAGES > 0 ? QKN_GEMM_STAGES : (kCta == 2 ? 6 : 4);
 #ifndef QKN_GEMM_EPI_WARPS
 #define QKN_GEMM_EPI_WARPS 8
 #endif
@@ -106,6 +112,15 @@ constexpr int kTmemCols = 2 * kAccCols;
 // ring + barriers (2 * kStages + 4 mbarriers) + TMEM address slot + 1 KB
 // alignment slack for the 128-byte-swizzle atoms
 constexpr int kSmemBytes = kStages * kStageBytes + 1024 + 256;
+// the kernel's static shared memory (partial-sum halves, factors, flags) is
+// 1.5 KB; ring + static must stay within the 227 KB a CTA may use
+static_assert(kSmemBytes + 3 * kBM * 4 + 64 <= 232448, "ring + static shared memory within 227 KB");
+#ifndef QKN_GEMM_ADAPTIVE_RESCALE
+#define QKN_GEMM_ADAPTIVE_RESCALE 1
+#endif
+// Fused QK-Norm: between tiles, keep scaling ready tiles while the next
+// accumulator is not yet complete (1), or scale at most two per tile (0).
+constexpr bool kAdaptiveRescale = QKN_GEMM_ADAPTIVE_RESCALE != 0;
 
 struct GemmParams {
     char *qkv;               // [T][qkv_stride] bf16, columns [0, N)
@@ -147,6 +162,15 @@ namespace gemm {
 // step that failed (static storage).
 cudaError_t launch_qkv_gemm(const void *x, int64_t x_stride, const void *w, int64_t w_stride, int32_t D,
                             int32_t N, const GemmParams &p, cudaStream_t stream, const char **what);
+
+// Raster group (pure host function): sets p->group_units from p's tile
+// counts for a launch of min(num_units, clusters) CTA groups on a GPU with an
+// L2 of l2_bytes.
+void schedule_qkv_gemm(GemmParams *p, int32_t D, int32_t N, int clusters, int64_t l2_bytes);
+
+// CTA groups of the kernel resident at once on the current device (cached per
+// device); on failure *what names the step that failed.
+cudaError_t qkv_gemm_clusters(int *clusters, const char **what);
 
 // The device word a bounded wait writes when it runs out (0 = none); reading
 // synchronizes the current device and clears the word.

@@ -1060,7 +1060,7 @@ def native_projection(args) -> int:
                 "us_per_call": round(step_s * 1e6, 2), "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded; OLMo2-7B-shaped projection, "
                                                              "random weights)",
-                "config": cfg,
+                "config": cfg, "measurement": {"gemm_schedule": qk.qkv_gemm_plan(b.T, b.D, b.Hq, b.Hk, b.Hv)},
                 "roofline": {"bound": "tensor", "achieved": round(kernel_tflops, 1), "peak": peak["tflops"],
                              "unit": "TFLOP/s", "frac": round(kernel_tflops / peak["tflops"], 4),
                              "traffic": profiled_traffic(b.name, source_digest("projection")),

@@ -171,6 +171,40 @@ qkn_status qknorm_tp_layerwise_scope(int32_t R, int32_t first_rank, int32_t n_lo
                                      int64_t T, float eps, qkn_dtype dtype, void *const *recv, uint32_t epoch,
                                      int32_t blocks_per_rank, uint64_t timeout_ns, int32_t scope, void *stream);
 
+/*
+ * The schedule of the projection GEMM (qknorm_qkv_gemm_stats and the
+ * projection entry points; the QKV projection of the SwiftQK paper's
+ * Background section, with Phase A's partial sums in its epilogue).  A unit
+ * is one tensor-core tile of 256 tokens x 256 output columns; persistent CTA
+ * pairs take units c, c + clusters, ... in a grouped raster: within a group
+ * of group_units token blocks the token block runs fastest, then the column
+ * tile, then the group.  The group is sized by what fits in half of L2: all
+ * token blocks when X fits, one when W fits, else about sqrt(clusters).
+ */
+typedef struct {
+    int32_t clusters;    /* CTA groups launched: min(units, resident groups) */
+    int32_t units;       /* work units: ceil(T / 256) * (Hq + Hk + Hv) / 256 */
+    int32_t group_units; /* token blocks (of 256 tokens) per raster group */
+} qkn_gemm_schedule;
+
+/*
+ * The schedule for `clusters` resident CTA groups on a GPU with an L2 of
+ * `l2_bytes` bytes.  Pure function of its arguments; needs no GPU.
+ * QKN_ERR_INVALID_ARG for a null `out`, T outside [1, 2^31), D < 1, Hq < 1,
+ * Hk < 1, Hv < 0, clusters < 1 or l2_bytes < 0; QKN_ERR_UNSUPPORTED when Hq,
+ * Hk or Hv is not a multiple of 256 or the output has more than 2^30 tiles.
+ */
+qkn_status qknorm_qkv_gemm_schedule(int64_t T, int32_t D, int32_t Hq, int32_t Hk, int32_t Hv, int32_t clusters,
+                                    int64_t l2_bytes, qkn_gemm_schedule *out);
+
+/*
+ * The schedule the projection entry points use for this shape on the
+ * current device (queries the resident CTA pairs and the L2 size; needs a
+ * GPU).  Errors as qknorm_qkv_gemm_schedule, plus QKN_ERR_CUDA when a query
+ * fails.
+ */
+qkn_status qknorm_qkv_gemm_plan(int64_t T, int32_t D, int32_t Hq, int32_t Hk, int32_t Hv, qkn_gemm_schedule *out);
+
 #ifdef __cplusplus
 }
 #endif

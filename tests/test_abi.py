@@ -602,3 +602,52 @@ def test_multi_shard_launch_override_validation(lib):
     assert stats(_clib.QknLaunch(kernel=0, vec_per_thread=2, threads=32, grid=10)) == INVALID   # row not covered
     assert stats(_clib.QknLaunch(kernel=1, vec_per_thread=0, threads=256, grid=10)) == INVALID  # not the register kernel
     assert stats(_clib.QknLaunch(kernel=0, vec_per_thread=2, threads=64, grid=10)) == CUDA      # valid: launch fails here
+
+
+# --------------------------------------------------------------- GEMM schedule
+L2_B200 = 126 * 1024 * 1024
+
+
+def _group_rule(m_units: int, D: int, N: int, clusters: int, l2: int) -> int:
+    """The raster group, restated: all token blocks when X fits in half of L2,
+    one when W does, else the G minimising G + ceil(clusters / G)."""
+    half = l2 / 2
+    if m_units * 256 * D * 2 <= half:
+        return m_units
+    if N * D * 2 <= half:
+        return 1
+    return min(range(1, min(m_units, clusters) + 1), key=lambda g: (g + -(-clusters // g), g))
+
+
+@pytest.mark.parametrize("T,D,Hq,Hk,Hv,clusters,group", [
+    (4096, 4096, 4096, 1024, 1024, 74, 16),    # X 33.5 MB fits: one group of all 16 token blocks
+    (4096, 4096, 4096, 4096, 4096, 74, 16),
+    (16384, 4096, 4096, 1024, 1024, 74, 1),    # X 134 MB does not, W 50 MB does: one block per group
+    (16384, 4096, 4096, 4096, 4096, 74, 7),    # neither: G + ceil(74 / G) smallest at 7 (7 + 11)
+    (12000, 4096, 4096, 4096, 2048, 74, 7),
+    (512, 256, 512, 512, 512, 74, 2),          # fewer units (12) than clusters
+    (1, 64, 256, 256, 0, 74, 1),
+])
+def test_qkv_gemm_schedule(T, D, Hq, Hk, Hv, clusters, group):
+    s = qk.qkv_gemm_schedule(T, D, Hq, Hk, Hv, clusters, L2_B200)
+    m_units = -(-T // 256)
+    N = Hq + Hk + Hv
+    units = m_units * (N // 256)
+    assert s["units"] == units and s["clusters"] == min(units, clusters)
+    assert s["group_units"] == group == _group_rule(m_units, D, N, min(units, clusters), L2_B200)
+
+
+@pytest.mark.parametrize("args,want", [
+    ((0, 64, 256, 256, 0, 74, L2_B200), _clib.QKN_ERR_INVALID_ARG),
+    ((1 << 31, 64, 256, 256, 0, 74, L2_B200), _clib.QKN_ERR_INVALID_ARG),
+    ((16, 0, 256, 256, 0, 74, L2_B200), _clib.QKN_ERR_INVALID_ARG),
+    ((16, 64, 0, 256, 0, 74, L2_B200), _clib.QKN_ERR_INVALID_ARG),
+    ((16, 64, 256, 256, -256, 74, L2_B200), _clib.QKN_ERR_INVALID_ARG),
+    ((16, 64, 128, 256, 0, 74, L2_B200), _clib.QKN_ERR_UNSUPPORTED),
+    ((16, 64, 256, 256, 0, 0, L2_B200), _clib.QKN_ERR_INVALID_ARG),
+    ((16, 64, 256, 256, 0, 74, -1), _clib.QKN_ERR_INVALID_ARG),
+])
+def test_qkv_gemm_schedule_validation(lib, args, want):
+    S = _clib.QknGemmSchedule()
+    assert lib.qknorm_qkv_gemm_schedule(*args, ctypes.byref(S)) == want
+    assert lib.qknorm_qkv_gemm_schedule(16, 64, 256, 256, 0, 74, L2_B200, None) == _clib.QKN_ERR_INVALID_ARG

@@ -184,6 +184,9 @@ def test_projection_rasters_beyond_l2(T, D, Hq, Hk, Hv):
     the fused rescale must not depend on the order.  Checked on sampled rows
     against the oracle, with the ragged last strip among them, and bit for bit
     against the two-launch path."""
+    plan = qk.qkv_gemm_plan(T, D, Hq, Hk, Hv)
+    if plan["clusters"] == 74 and torch.cuda.get_device_properties(DEV).L2_cache_size >= 120 << 20:
+        assert plan["group_units"] == (1 if T == 16284 else 7), plan  # the raster the docstring names
     b = workloads.qkv_projection(T=T, D=D, Hq=Hq, Hk=Hk, Hv=Hv, seed=T + D)
     x, w = b.x.to(DEV), b.w.to(DEV)
     gq, gk = b.gamma_q.to(DEV), b.gamma_k.to(DEV)
@@ -249,3 +252,28 @@ def test_fused_norm_equals_the_two_launch_path(T, D, Hq, Hk, Hv):
     proj = check_projection(b, plain, rows)
     check_normalized(b, proj, fused, rows)
     assert qk.device_timeouts() == 0
+
+
+@pytest.mark.parametrize("T,D,Hq,Hk,Hv", [
+    (4096, 64, 4096, 1024, 1024),   # the GQA bench shape's tiling (384 units, a partial last wave of V tiles)
+    (4000, 72, 2048, 512, 2304),    # ragged last token block (160 tokens) and k-block
+])
+def test_projection_every_row(T, D, Hq, Hk, Hv):
+    """Every row and every column against the oracle (projection, tile sums
+    and the normalized Q and K), the fused call bit for bit against the
+    two-launch path, V equal to the plain projection."""
+    b = workloads.qkv_projection(T=T, D=D, Hq=Hq, Hk=Hk, Hv=Hv, seed=T + D + Hv)
+    x, w = b.x.to(DEV), b.w.to(DEV)
+    gq, gk = b.gamma_q.to(DEV), b.gamma_k.to(DEV)
+    plain, qs, ks = qk.qknorm_qkv_gemm_stats(x, w, Hq, Hk, Hv)
+    fused = qk.qknorm_qkv_projection(x, w, gq, gk, Hq, Hk, Hv, b.eps)
+    two = qk.qknorm_qkv_projection(x, w, _unaligned_copy(gq), _unaligned_copy(gk), Hq, Hk, Hv, b.eps)
+    torch.cuda.synchronize()
+    assert qk.device_timeouts() == 0
+    assert torch.equal(fused, two)
+    assert torch.equal(fused[:, Hq + Hk:], plain[:, Hq + Hk:])  # V keeps the projection
+    rows = np.arange(T)
+    proj = check_projection(b, plain, rows)
+    check_tile_sums(proj, qs, rows, 0, Hq // TILE)
+    check_tile_sums(proj, ks, rows, Hq, Hk // TILE)
+    check_normalized(b, proj, fused, rows)
