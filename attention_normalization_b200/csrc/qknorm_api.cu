@@ -438,14 +438,16 @@ qkn_status plan_call(const CallT<SETS> &c, qkn_launch &L) {
         work = p.n_items;
     }
     if (MODE == qkn::kFused && L.kernel == QKN_KERNEL_REGISTER && work >= 4 * (int64_t)bps * sms) {
-        // At least 4 items per resident slot: launch 4 CTAs per slot rather
-        // than one persistent CTA, so the hardware hands the remaining items
-        // to whichever CTAs finish first.  (One B200, graph replays: prefill
-        // T=4096 H=4096 bf16 22.2-22.3 us against 22.7-22.9; packed T=4096
-        // 15.1 against 15.5; headwise T=4096 14.6-14.9 against 15.1-15.2;
-        // with fewer items per slot -- E4M3 prefill, packed T=1024 -- it
-        // did not help.)
-        oversubscribe = 4;
+        // At least 4 items per resident slot: launch 3 (below 6 items per
+        // slot) or 4 CTAs per slot rather than one persistent CTA, so the
+        // hardware hands the remaining items to whichever CTAs finish first.
+        // (One B200, graph replays, CTAs per slot 1 / 3 / 4: prefill T=4096
+        // H=4096 bf16, 6.9 items per slot, 22.7-22.9 / 22.9 / 22.2-22.3 us;
+        // packed T=4096, 4.3 items per slot, 15.5 / 14.7 / 15.0-15.1;
+        // headwise T=4096, 4.3 items per slot, 15.1-15.2 / 14.6 / 14.9; with
+        // fewer items per slot -- E4M3 prefill, packed T=1024 -- it did not
+        // help.)
+        oversubscribe = work < 6 * (int64_t)bps * sms ? 3 : 4;
     }
     L.grid = qknorm_plan_grid(work, bps * oversubscribe, sms);
     return QKN_OK;
