@@ -415,6 +415,19 @@ def graph_upload(graph: "torch.cuda.CUDAGraph", stream) -> bool:
         return False
 
 
+HOLD_CYCLES = 200_000  # ~100 us at 1.9 GHz
+
+
+def hold_queue(stream) -> None:
+    """Queue a short device spin (torch's sleep kernel, ~100 us) on `stream`
+    before a timed region's start event, so that the start event and the
+    graph the host submits next are already queued when the GPU reaches
+    them: the timed region then holds the K steps' device time, not the
+    host's graph submission.  The spin itself ends before the start event."""
+    with torch.cuda.stream(stream):
+        torch.cuda._sleep(HOLD_CYCLES)
+
+
 MAX_SETS = 64
 
 
@@ -601,6 +614,7 @@ def native(args) -> int:
     # are also taken at its edges and while the replay is in flight
     sampler.sample_now()
     sampler.active.set()
+    hold_queue(stream)
     ev0.record(stream)
     g_timed.replay()
     ev1.record(stream)
@@ -628,6 +642,7 @@ def native(args) -> int:
         torch.cuda.synchronize()
         per_call = []
         for _ in range(20):
+            hold_queue(stream)
             ev0.record(stream)
             g_short.replay()
             ev1.record(stream)
@@ -679,7 +694,9 @@ def native(args) -> int:
                              f"{between / 1e6:.1f} MB touched between reuses "
                              + ("> 2 x" if between > 2 * l2 else "< 2 x (L2-warm)") + f" {l2 / 1e6:.0f} MB L2)",
                        "timing": "CUDA graph of K captured C-ABI calls (uploaded before timing: %s), "
-                                 "CUDA events on the launching stream" % ("yes" if uploaded else "no"),
+                                 "CUDA events on the launching stream, a ~100 us torch sleep kernel queued "
+                                 "ahead of the start event (the host's graph submission is not timed)"
+                                 % ("yes" if uploaded else "no"),
                        "launch_plan": plan}
         line = {"metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 6),
@@ -978,6 +995,7 @@ def native_projection(args) -> int:
         ranks.barrier()
         torch.cuda.synchronize()
         sampler.active.set()
+        hold_queue(stream)
         e0.record(stream)
         gt.replay()
         e1.record(stream)
@@ -1052,7 +1070,9 @@ def native_projection(args) -> int:
                "l2": f"rotating {R} sets of x, w, qkv, workspace ({R * set_bytes / 1e6:.1f} MB; "
                      f"{between / 1e6:.1f} MB touched between reuses "
                      + ("> 2 x" if between > 2 * l2 else "< 2 x") + f" {l2 / 1e6:.0f} MB L2)",
-               "timing": "CUDA graph of K captured C-ABI calls, CUDA events on the launching stream"}
+               "timing": "CUDA graph of K captured C-ABI calls, CUDA events on the launching stream, a ~100 us "
+                         "torch sleep kernel queued ahead of the start event (the host's graph submission is not "
+                         "timed)"}
         # the fused kernel is the step's only kernel (beside a 256-byte memset)
         kernel_tflops = flops / step_s / 1e12
         line = {"metric": PROJ_METRIC, "value": round(value, 1), "unit": PROJ_UNIT, "n_gpus": world,
