@@ -820,16 +820,6 @@ qkn_status check_projection_overlaps(const Projection &pr, const float *q_sums, 
     return QKN_OK;
 }
 
-// Fused QK-Norm inside the GEMM: per-strip completion counters (zeroed on
-// the stream before the launch) and the Q / K scales.
-struct FusedNorm {
-    int *counters;
-    const void *gamma_q, *gamma_k;
-    float eps;
-};
-
-int64_t projection_m_tiles(int64_t T) { return (T + qkn::gemm::kBM - 1) / qkn::gemm::kBM; }
-
 // The tile counts of a projection of T tokens, D inputs and Hq + Hk + Hv
 // outputs (Hq, Hk, Hv multiples of kTileN).
 void gemm_tiles(int64_t T, int32_t D, int32_t Hq, int32_t Hk, int32_t Hv, qkn::gemm::GemmParams &gp) {
@@ -861,8 +851,7 @@ void fill_schedule(const qkn::gemm::GemmParams &gp, int32_t clusters, qkn_gemm_s
     out->group_units = gp.group_units;
 }
 
-qkn_status launch_projection_gemm(const Projection &pr, float *q_sums, float *k_sums, void *stream,
-                                  const FusedNorm *fuse = nullptr) {
+qkn_status launch_projection_gemm(const Projection &pr, float *q_sums, float *k_sums, void *stream) {
     qkn::gemm::GemmParams gp{};
     gp.qkv = static_cast<char *>(pr.qkv);
     gp.qkv_stride_bytes = pr.qkv_stride * 2;
@@ -870,17 +859,6 @@ qkn_status launch_projection_gemm(const Projection &pr, float *q_sums, float *k_
     gp.k_sumsq = k_sums;
     gemm_tiles(pr.T, pr.D, pr.Hq, pr.Hk, pr.Hv, gp);
     gp.timeout_ns = kGemmTimeoutNs;
-    if (fuse) {
-        gp.counters = fuse->counters;
-        gp.gamma_q = static_cast<const char *>(fuse->gamma_q);
-        gp.gamma_k = static_cast<const char *>(fuse->gamma_k);
-        gp.inv_hq = static_cast<float>(1.0 / static_cast<double>(pr.Hq));
-        gp.inv_hk = static_cast<float>(1.0 / static_cast<double>(pr.Hk));
-        gp.eps = fuse->eps;
-        cudaError_t me = cudaMemsetAsync(fuse->counters, 0, (size_t)(2 * gp.m_tiles) * sizeof(int),
-                                         static_cast<cudaStream_t>(stream));
-        if (me != cudaSuccess) return fail(QKN_ERR_CUDA, "clearing the strip counters: %s", cudaGetErrorString(me));
-    }
     const char *what = "";
     cudaError_t e = qkn::gemm::launch_qkv_gemm(pr.x, pr.x_stride, pr.w, pr.w_stride, pr.D, pr.N, gp,
                                                static_cast<cudaStream_t>(stream), &what);
@@ -1305,8 +1283,8 @@ qkn_status qknorm_qkv_gemm_stats(const void *x, int64_t x_stride, const void *w,
 
 int64_t qknorm_qkv_projection_workspace_bytes(int64_t T, int32_t Hq, int32_t Hk) {
     if (T < 0 || Hq <= 0 || Hk <= 0 || Hq % kTileN || Hk % kTileN) return -1;
-    // partial sums [Hq/256][T] and [Hk/256][T], then two strip counters per 128 tokens
-    return (int64_t)(Hq / kTileN + Hk / kTileN) * T * 4 + 2 * projection_m_tiles(T) * 4;
+    // partial sums [Hq/256][T] and [Hk/256][T]
+    return (int64_t)(Hq / kTileN + Hk / kTileN) * T * 4;
 }
 
 qkn_status qknorm_qkv_gemm_schedule(int64_t T, int32_t D, int32_t Hq, int32_t Hk, int32_t Hv, int32_t clusters,
@@ -1362,15 +1340,12 @@ qkn_status qknorm_qkv_projection(const void *x, int64_t x_stride, const void *w,
             return fail(QKN_ERR_INVALID_ARG, "the workspace overlaps an operand");
     }
 
-    // 16-byte aligned gamma: QK-Norm runs inside the GEMM (the CTA that stores
-    // a strip's last Q or K tile combines the strip's partial sums and scales
-    // it in place).
-    if (aligned16(gamma_q) && aligned16(gamma_k)) {
-        FusedNorm fz{reinterpret_cast<int *>(k_sums + (int64_t)(Hk / kTileN) * T), gamma_q, gamma_k, eps};
-        return launch_projection_gemm(pr, q_sums, k_sums, stream, &fz);
-    }
-    // Otherwise a second launch: Phase A aggregation + Phase B over the Q and
-    // K columns of qkv, in place.
+    // The GEMM writes qkv and the partial sums; a second launch then runs
+    // Phase A's aggregation and Phase B over the Q and K columns of qkv, in
+    // place, while the freshly stored tiles are partly still in L2.  (Scaling
+    // the tiles inside the GEMM's epilogue once a strip was complete gave the
+    // same bits but was slower or equal: its read-modify-write competes with
+    // the GEMM's operand stream.)
     Call c;
     init_call(c, dtype, 2);
     char *kcols = static_cast<char *>(qkv) + (int64_t)Hq * 2;
@@ -1399,8 +1374,7 @@ qkn_status qknorm_qkv_projection_noalloc(const void *x, int64_t x_stride, const 
                                      eps, nullptr, 0, dtype, stream);
     if (need > kNoAllocScratchBytes)
         return fail(QKN_ERR_INVALID_ARG,
-                    "needs %lld bytes of workspace (partial sums and strip counters); the built-in scratch "
-                    "holds %lld",
+                    "needs %lld bytes of workspace for the partial sums; the built-in scratch holds %lld",
                     (long long)need, (long long)kNoAllocScratchBytes);
     void *ws = nullptr;
     qkn_status st = noalloc_scratch(&ws);

@@ -49,19 +49,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return done != 0;
 }
 
-// Non-blocking: true if the phase of parity `parity` has completed.
-__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
-    uint32_t done;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(done)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    return done != 0;
-}
-
 // True once the phase of parity `parity` has completed; false when
 // `timeout_ns` of global time passed first.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_t timeout_ns) {
@@ -224,9 +211,8 @@ __device__ __forceinline__ bool epilogue_all(bool ok) {
 // token blocks: within a group the token block runs fastest, then the column
 // tile, then the group (the last group may hold fewer token blocks).  One
 // group spanning all token blocks lets the units running at one time share a
-// few W tiles while X stays in L2; smaller groups complete each strip's Q and
-// K tiles sooner, so their rescale reads tiles still in L2 and overlaps the
-// next group's MMAs.
+// few W tiles while X stays in L2; smaller groups keep a wave's X blocks and
+// W tiles in L2 together when neither operand fits on its own.
 struct TileRef {
     int m_tile, n_tile;
 };
@@ -251,135 +237,6 @@ __device__ __forceinline__ int cta_tile_count(const GemmParams &p) {
     return c < p.num_units ? (p.num_units - c + clusters - 1) / clusters : 0;
 }
 
-// 8 bf16 (one 16-byte vector) -> (x * gamma) * r rounded to bf16, each
-// product in fp32 round-to-nearest.
-__device__ __forceinline__ uint4 scale8(uint4 x, uint4 g, float r) {
-    uint32_t xs[4] = {x.x, x.y, x.z, x.w}, gs[4] = {g.x, g.y, g.z, g.w}, ys[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const float x0 = __uint_as_float(xs[i] << 16), x1 = __uint_as_float(xs[i] & 0xFFFF0000u);
-        const float g0 = __uint_as_float(gs[i] << 16), g1 = __uint_as_float(gs[i] & 0xFFFF0000u);
-        const __nv_bfloat162 h = __floats2bfloat162_rn(__fmul_rn(__fmul_rn(x0, g0), r), __fmul_rn(__fmul_rn(x1, g1), r));
-        ys[i] = *reinterpret_cast<const uint32_t *>(&h);
-    }
-    return make_uint4(ys[0], ys[1], ys[2], ys[3]);
-}
-
-__device__ __forceinline__ void red_release_add(int *p, int v) {
-    asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-
-__device__ __forceinline__ int ld_acquire(const int *p) {
-    int v;
-    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-
-// Phase A aggregation + Phase B for one stored Q (tensor 0) or K (tensor 1)
-// tile, run by the 256 epilogue threads once every tile of its 128-token
-// strip has been counted: r = rsqrt(S / H + eps) with S the strip's partial
-// sums added in order p = 0, 1, ...; then (x * gamma) * r over the tile, in
-// place.  Tiles and partial sums written by other CTAs are read through L2
-// (.cg).  Each warp issues the loads of its rows of the tile first, so they
-// are in flight while the factors are formed.
-__device__ __noinline__ void scale_tile(const GemmParams &p, int tensor, int m_tile, int n_tile, float *s_r) {
-    const int et = threadIdx.x - 64;  // 0 .. 255
-    const int P = tensor ? p.k_tiles : p.q_tiles;
-    const int first = tensor ? p.q_tiles : 0;  // the tensor's first column tile
-    const float *sums = tensor ? p.k_sumsq : p.q_sumsq;
-    const float inv = tensor ? p.inv_hk : p.inv_hq;
-    const int64_t row0 = static_cast<int64_t>(m_tile) * kBM;
-    const int rows = static_cast<int>(p.T - row0 < kBM ? p.T - row0 : kBM);
-    // warp e takes rows e, e + 8, ...; lane l the l-th 16-byte vector of each
-    // (a tile row is 32 vectors), so every load and store is one whole row
-    const int e = et >> 5, lane = et & 31;
-    char *base = p.qkv + row0 * p.qkv_stride_bytes + static_cast<int64_t>(n_tile) * kBN * 2 + lane * 16;
-    constexpr int kBatch = kBM / kEpiWarps;  // rows per warp: the whole tile in flight at once
-    uint4 xv[kBatch];
-#pragma unroll
-    for (int i = 0; i < kBatch; ++i) {
-        const int rr = e + kEpiWarps * i;
-        xv[i] = rr < rows ? __ldcg(reinterpret_cast<const uint4 *>(base + rr * p.qkv_stride_bytes))
-                          : make_uint4(0u, 0u, 0u, 0u);
-    }
-    if (et < kBM) {
-        float r = 0.0f;
-        if (et < rows) {
-            // sixteen loads in flight at a time, added strictly in order p = 0, 1, ...
-            const float *col = sums + row0 + et;
-            float S = 0.0f;
-            for (int q0 = 0; q0 < P; q0 += 16) {
-                float v[16];
-#pragma unroll
-                for (int i = 0; i < 16; ++i) v[i] = q0 + i < P ? __ldcg(col + static_cast<int64_t>(q0 + i) * p.T) : 0.0f;
-#pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    if (q0 + i < P) S += v[i];
-            }
-            r = rsqrtf(__fmaf_rn(S, inv, p.eps));
-        }
-        s_r[et] = r;
-    }
-    const uint4 *gamma = reinterpret_cast<const uint4 *>(tensor ? p.gamma_k : p.gamma_q);
-    const uint4 g = __ldg(gamma + (n_tile - first) * (kBN / 8) + lane);
-    epilogue_sync();  // the factors are in s_r
-#pragma unroll
-    for (int i = 0; i < kBatch; ++i) {
-        const int rr = e + kEpiWarps * i;
-        if (rr < rows) *reinterpret_cast<uint4 *>(base + rr * p.qkv_stride_bytes) = scale8(xv[i], g, s_r[rr]);
-    }
-    epilogue_sync();  // s_r is reused by the next tile
-}
-
-// Scales this CTA's stored Q / K tiles from sequence index `from` up to (not
-// including) `upto`, in order, while their strips are complete.  Without
-// `wait` it stops at the first incomplete strip, or once `budget` tiles are
-// done and -- when `next_bar` is not 0 -- the phase `next_parity` of that
-// barrier (the next tile's accumulator) has completed; with `wait` (only
-// once all of this CTA's own tiles are stored and counted, so it never waits
-// on itself) it waits, bounded, for each strip.  Returns the next index to
-// scale.
-__device__ int scale_ready_tiles(const GemmParams &p, int from, int upto, bool wait, int budget, float *s_r,
-                                 int *abort_flag, int rank, uint32_t next_bar = 0, uint32_t next_parity = 0) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    while (from < upto && (wait || budget > 0 || next_bar != 0)) {
-        const TileRef tr = cta_tile(p, from, rank);
-        const int m_tile = tr.m_tile, n_tile = tr.n_tile;
-        if (m_tile >= p.m_tiles) {  // the pair's second token tile lies past T
-            ++from;
-            continue;
-        }
-        const int tensor = n_tile < p.q_tiles ? 0 : (n_tile < p.q_tiles + p.k_tiles ? 1 : -1);
-        if (tensor < 0) {  // V tile: nothing to scale
-            ++from;
-            continue;
-        }
-        bool ready = true;
-        if (warp == 2 && lane == 0) {
-            // past the budget, go on only while the next accumulator is not complete
-            const bool more = wait || budget > 0 || (next_bar != 0 && !mbar_test(next_bar, next_parity));
-            const int *cnt = p.counters + tensor * p.m_tiles + m_tile;
-            const int P = tensor ? p.k_tiles : p.q_tiles;
-            ready = more && ld_acquire(cnt) >= P;
-            if (more && !ready && wait) {
-                const uint64_t t0 = global_ns();
-                while (!(ready = ld_acquire(cnt) >= P)) {
-                    if (global_ns() - t0 > p.timeout_ns) {
-                        record_timeout(kErrEpilogue, abort_flag);
-                        break;
-                    }
-                    __nanosleep(256);
-                }
-            }
-        }
-        if (!epilogue_all(ready)) break;  // the leader's answer, in every epilogue thread;
-                                          // with `wait` a timeout (reported) leaves the rest unscaled
-        scale_tile(p, tensor, m_tile, n_tile, s_r);
-        ++from;
-        --budget;
-    }
-    return from;
-}
 }  // namespace
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -390,7 +247,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     __shared__ int s_consumed;   // k-blocks (over all tiles) whose MMAs were issued
     __shared__ int s_issued;     // k-blocks (over all tiles) whose TMA loads were issued
     __shared__ float s_half[2][kBM];  // second-half squared sums, by tile parity
-    __shared__ float s_r[kBM];        // RMS factors of the tile being scaled
 
     // 1024-byte aligned ring: A stages, then B stages, then the mbarriers:
     // full[kStages], empty[kStages], acc_full[2], acc_empty[2].  The layout
@@ -516,23 +372,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int quarter = warp & 3;          // TMEM lanes this warp may read
         const int half = (warp - 2) >> 2;      // which column range of the tile (0 with 4 warps)
         const int rl = quarter * 32 + lane;    // row within the tile
-        const bool fused = p.counters != nullptr;
         // the leader's acc_empty barriers: every epilogue warp of the group arrives there
         const uint32_t acc_empty_leader[2] = {kCta == 2 ? map_to_cta(acc_empty_bar(0), 0) : acc_empty_bar(0),
                                               kCta == 2 ? map_to_cta(acc_empty_bar(1), 0) : acc_empty_bar(1)};
-        int norm_next = 0;  // next of this CTA's tiles to scale (fused QK-Norm)
-        bool timed_out = false;
-        int j = 0;
-        for (; j < n_tiles_cta; ++j) {
+        for (int j = 0; j < n_tiles_cta; ++j) {
             const int b = j & 1;
             const int use = j >> 1;
             bool ok = mbar_wait(acc_full_bar(b), use & 1, p.timeout_ns);
             if (!ok) record_timeout(kErrEpilogue, &s_abort);
             // the same decision in every epilogue warp, so the named barriers below always match
-            if (!epilogue_all(ok && p.k_blocks > 0)) {
-                timed_out = true;
-                break;
-            }
+            if (!epilogue_all(ok && p.k_blocks > 0)) break;
             fence_after_sync();
             const TileRef tr = cta_tile(p, j, rank);
             const int m_tile = tr.m_tile, n_tile = tr.n_tile;
@@ -587,25 +436,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (p.k_sumsq) p.k_sumsq[static_cast<int64_t>(n_tile - p.q_tiles) * p.T + row] = total;
                     }
                 }
-                epilogue_sync();  // every epilogue thread's stores of the tile precede this; s_half[b] read
-                // Count the tile on its strip: one thread, after the barrier,
-                // adds with release semantics at GPU scope, which orders the
-                // whole tile's stores (made visible to it by the barrier)
-                // before the count for the CTA that acquires the counter.
-                if (fused && warp == 2 && lane == 0) red_release_add(p.counters + tensor * p.m_tiles + m_tile, 1);
-            }
-            // Scale earlier tiles of this CTA whose strips are complete: two,
-            // and then more while the next tile's accumulator is not complete
-            // (the epilogue would only wait for it).
-            if (fused) {
-                const bool next = kAdaptiveRescale && j + 1 < n_tiles_cta;
-                norm_next = scale_ready_tiles(p, norm_next, j + 1, false, 2, s_r, &s_abort, rank,
-                                              next ? acc_full_bar((j + 1) & 1) : 0u,
-                                              static_cast<uint32_t>(((j + 1) >> 1) & 1));
+                epilogue_sync();  // s_half[b] has been read before the tile after next reuses it
             }
         }
-        if (fused && !timed_out)
-            scale_ready_tiles(p, norm_next, j, true, 1 << 30, s_r, &s_abort, rank);
     }
 
     fence_before_sync();
@@ -670,7 +503,7 @@ std::mutex g_smem_mu;
 
 // Token blocks per raster group (1 .. m_units) for `clusters` CTA groups
 // running at once, by what must stay in L2 (half of it, leaving room for the
-// stored tiles the fused rescale reads back):
+// stored tiles):
 //   * X fits: one group -- the token blocks run fastest, X stays resident and
 //     each W tile is read by the units of about one wave;
 //   * else W fits: one token block per group -- each X block is read once by
@@ -678,10 +511,10 @@ std::mutex g_smem_mu;
 //   * else the G that makes a wave's distinct X blocks + W tiles, G +
 //     ceil(clusters / G), smallest (about sqrt(clusters)), so a wave's
 //     operands fit in L2 together.
-// (One B200, fused projection, D = 4096: at T = 16384 this order took 597 us
-// against 731 us for one group with Hq = 4096, Hk = Hv = 1024, and 1235 us
-// against 1391 us with Hq = Hk = Hv = 4096; at T = 4096 one group was best or
-// equal.)
+// (One B200, projection + QK-Norm, D = 4096: at T = 16384 this order took
+// 597 us against 731 us for one group with Hq = 4096, Hk = Hv = 1024, and
+// 1235 us against 1391 us with Hq = Hk = Hv = 4096; at T = 4096 one group was
+// best or equal.)
 int raster_group_units(int m_units, int D, int N, int clusters, int l2_bytes) {
     int g = m_units;
     if (kGroupM >= 0) {

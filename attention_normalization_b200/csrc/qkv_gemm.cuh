@@ -45,18 +45,6 @@
 //                    Then the accumulator goes back to the MMA thread.  With
 //                    two accumulators the epilogue of one tile overlaps the
 //                    MMAs of the next.
-// Fused QK-Norm (when `counters` is set): after storing a Q or K tile and its
-// partial sums, the epilogue warps meet at a barrier and one thread counts the
-// tile on its strip's counter (one per 128-token strip and tensor) with a
-// GPU-scope release add, which publishes the whole tile.  Between
-// tiles it scales, in order, those of its own earlier Q / K tiles whose strips
-// are complete (counter = the tensor's tile count, read with acquire): the
-// strip's partial sums are added in order p = 0, 1, ... (fp32), r = rsqrt(S /
-// H + eps) per token, and the tile is rewritten in place as (x * gamma) * r
-// rounded to bf16, read back through L2 -- Phase A's aggregation and Phase B's
-// scaling without a second pass over HBM.  Once all of its own tiles are
-// counted it waits (bounded) for its remaining strips; it never waits while
-// it still owes tiles, so no CTA waits on one that waits on it.
 // Every mbarrier wait is bounded by the global timer; on expiry the kernel
 // records a code in a device word, skips the rest of its work, lets its
 // in-flight loads land, frees its TMEM and returns, so the context stays
@@ -112,15 +100,9 @@ constexpr int kTmemCols = 2 * kAccCols;
 // ring + barriers (2 * kStages + 4 mbarriers) + TMEM address slot + 1 KB
 // alignment slack for the 128-byte-swizzle atoms
 constexpr int kSmemBytes = kStages * kStageBytes + 1024 + 256;
-// the kernel's static shared memory (partial-sum halves, factors, flags) is
-// 1.5 KB; ring + static must stay within the 227 KB a CTA may use
-static_assert(kSmemBytes + 3 * kBM * 4 + 64 <= 232448, "ring + static shared memory within 227 KB");
-#ifndef QKN_GEMM_ADAPTIVE_RESCALE
-#define QKN_GEMM_ADAPTIVE_RESCALE 1
-#endif
-// Fused QK-Norm: between tiles, keep scaling ready tiles while the next
-// accumulator is not yet complete (1), or scale at most two per tile (0).
-constexpr bool kAdaptiveRescale = QKN_GEMM_ADAPTIVE_RESCALE != 0;
+// the kernel's static shared memory (partial-sum halves, flags) is about
+// 1 KB; ring + static must stay within the 227 KB a CTA may use
+static_assert(kSmemBytes + 2 * kBM * 4 + 64 <= 232448, "ring + static shared memory within 227 KB");
 
 struct GemmParams {
     char *qkv;               // [T][qkv_stride] bf16, columns [0, N)
@@ -132,18 +114,11 @@ struct GemmParams {
     int32_t q_tiles;         // Hq / kBN
     int32_t k_tiles;         // Hk / kBN
     int32_t n_tiles;         // N / kBN
-    int32_t m_tiles;         // ceil(T / kBM): 128-token tiles (= strips)
+    int32_t m_tiles;         // ceil(T / kBM): 128-token tiles
     int32_t m_units;         // ceil(T / (kBM * kCta)): token blocks of one MMA
     int32_t num_units;       // m_units * n_tiles: work units (one per CTA group)
     int32_t group_units;     // token blocks per raster group, 1 .. m_units
     uint64_t timeout_ns;     // bound on every mbarrier wait
-    // Fused QK-Norm (all null / unused when counters is null).
-    int *counters;           // [2][m_tiles] tiles stored per strip, zero at launch
-    const char *gamma_q;     // [Hq] bf16
-    const char *gamma_k;     // [Hk] bf16
-    float inv_hq;            // fl(1 / Hq)
-    float inv_hk;            // fl(1 / Hk)
-    float eps;
 };
 
 // Error codes written to the device word when a wait runs out.

@@ -300,16 +300,15 @@ qkn_status qknorm_qkv_projection(const void *x, int64_t x_stride, const void *w,
  * another one (after cudaDeviceReset, say): the first call after such a
  * change should also come before any capture.
  * Limits: the call's workspace, qknorm_qkv_projection_workspace_bytes(T, Hq,
- * Hk) = (Hq/256 + Hk/256) * T * 4 + 8 * ceil(T / 128) bytes, must fit in the
- * 4 MiB (e.g. T = 32000 with Hq = Hk = 4096); larger calls return
- * QKN_ERR_INVALID_ARG before any launch.
+ * Hk) = (Hq/256 + Hk/256) * T * 4 bytes, must fit in the 4 MiB (e.g. T up to
+ * 32768 with Hq = Hk = 4096); larger calls return QKN_ERR_INVALID_ARG before
+ * any launch.
  * Sharing: all calls on a device use the same array, and it keeps the last
- * call's contents.  Each call clears the strip counters it uses on its
- * stream (cudaMemsetAsync, which allocates nothing) and writes every partial
- * sum before reading it; but two calls that can run at the same time on the
- * GPU (different streams without ordering between them, or different host
- * threads) race on the array and may corrupt each other's results.  Order
- * such calls on one stream or with events.
+ * call's contents.  Each call writes every partial sum before reading it;
+ * but two calls that can run at the same time on the GPU (different streams
+ * without ordering between them, or different host threads) race on the
+ * array and may corrupt each other's results.  Order such calls on one
+ * stream or with events.
  * The paper has no counterpart: this is a deployment variant of this library.
  */
 qkn_status qknorm_qkv_projection_noalloc(const void *x, int64_t x_stride, const void *w, int64_t w_stride,

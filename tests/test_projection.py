@@ -181,9 +181,10 @@ def test_projection_full_size_sampled_rows():
 def test_projection_rasters_beyond_l2(T, D, Hq, Hk, Hv):
     """Shapes whose operands do not fit in half of L2 run the GEMM in smaller
     raster groups (on a B200: 148 SMs, 126 MB L2); the tiles, their sums and
-    the fused rescale must not depend on the order.  Checked on sampled rows
-    against the oracle, with the ragged last strip among them, and bit for bit
-    against the two-launch path."""
+    the normalized Q and K must not depend on the order.  Checked on sampled
+    rows against the oracle, with the ragged last token tile among them, and
+    bit for bit between the vector and the scalar apply pass (16-byte aligned
+    and unaligned gamma)."""
     plan = qk.qkv_gemm_plan(T, D, Hq, Hk, Hv)
     if plan["clusters"] == 74 and torch.cuda.get_device_properties(DEV).L2_cache_size >= 120 << 20:
         assert plan["group_units"] == (1 if T == 16284 else 7), plan  # the raster the docstring names
@@ -230,16 +231,16 @@ def _unaligned_copy(t: torch.Tensor) -> torch.Tensor:
 
 
 @pytest.mark.parametrize("T,D,Hq,Hk,Hv", [
-    (1000, 136, 1024, 512, 512),    # ragged last strip; Q and K with different tile counts
-    (4096, 64, 2048, 512, 512),     # many strips finishing at once
-    (129, 64, 256, 256, 0),         # one tile per strip and tensor
+    (1000, 136, 1024, 512, 512),    # ragged last token tile; Q and K with different tile counts
+    (4096, 64, 2048, 512, 512),     # 8 and 2 partial sums per row
+    (129, 64, 256, 256, 0),         # one partial sum per row and tensor
     (2048, 320, 512, 1536, 256),    # K wider than Q
 ])
-def test_fused_norm_equals_the_two_launch_path(T, D, Hq, Hk, Hv):
-    """With 16-byte aligned gamma the strip that stores its last tile scales
-    itself inside the GEMM; with unaligned gamma a second kernel does it.
-    Both combine the same partial sums in the same order, so they agree bit
-    for bit; sampled rows are also checked against the oracle."""
+def test_aligned_and_unaligned_gamma_agree(T, D, Hq, Hk, Hv):
+    """The apply pass after the GEMM runs the 16-byte vector kernel with
+    aligned gamma and the scalar-access kernel with unaligned gamma.  Both
+    combine the same partial sums in the same order, so they agree bit for
+    bit; sampled rows are also checked against the oracle."""
     b = workloads.qkv_projection(T=T, D=D, Hq=Hq, Hk=Hk, Hv=Hv, seed=T + Hk)
     x, w = b.x.to(DEV), b.w.to(DEV)
     gq, gk = b.gamma_q.to(DEV), b.gamma_k.to(DEV)
@@ -260,8 +261,8 @@ def test_fused_norm_equals_the_two_launch_path(T, D, Hq, Hk, Hv):
 ])
 def test_projection_every_row(T, D, Hq, Hk, Hv):
     """Every row and every column against the oracle (projection, tile sums
-    and the normalized Q and K), the fused call bit for bit against the
-    two-launch path, V equal to the plain projection."""
+    and the normalized Q and K), the vector apply pass bit for bit against
+    the scalar one (unaligned gamma), V equal to the plain projection."""
     b = workloads.qkv_projection(T=T, D=D, Hq=Hq, Hk=Hk, Hv=Hv, seed=T + D + Hv)
     x, w = b.x.to(DEV), b.w.to(DEV)
     gq, gk = b.gamma_q.to(DEV), b.gamma_k.to(DEV)
