@@ -651,3 +651,17 @@ def test_qkv_gemm_schedule_validation(lib, args, want):
     S = _clib.QknGemmSchedule()
     assert lib.qknorm_qkv_gemm_schedule(*args, ctypes.byref(S)) == want
     assert lib.qknorm_qkv_gemm_schedule(16, 64, 256, 256, 0, 74, L2_B200, None) == _clib.QKN_ERR_INVALID_ARG
+
+
+def test_noalloc_scratch_limit_on_the_host(lib):
+    """The allocation-free projection's scratch holds the partial sums of
+    T = 32768 tokens at Hq = Hk = 4096 (the header's example) and refuses one
+    token more before touching the device."""
+    cap = lib.qknorm_qkv_projection_noalloc_max_bytes()
+    assert cap == 4 << 20
+    assert lib.qknorm_qkv_projection_workspace_bytes(32768, 4096, 4096) == cap
+    assert lib.qknorm_qkv_projection_workspace_bytes(32769, 4096, 4096) > cap
+    st = lib.qknorm_qkv_projection_noalloc(0x10000, 64, 0x20000000, 64, 0x40000000, 8192, 0x60000000, 0x60010000,
+                                           32769, 64, 4096, 4096, 0, 1e-6, _clib.QKN_BF16, None)
+    assert st == _clib.QKN_ERR_INVALID_ARG
+    assert b"scratch" in lib.qknorm_last_error()
