@@ -4,12 +4,17 @@
  * shape (benchmark sweeps, per-variant tests).  Include after qknorm.h.
  *
  * Execution model (the single-GPU form of the paper's "deadlock-safe
- * persistent execution"): a kernel launches a bounded grid — at most as many
- * CTAs as can be resident at once — and each CTA loops over row items
- * blockIdx.x, blockIdx.x + grid, ...  Items 0..T-1 are the Q rows and items
- * T..2T-1 the K rows, so every CTA gets a near-equal share of each tensor's
- * rows whatever the grid.  A CTA works on one row at a time.  No CTA ever
- * waits on another, so any grid is safe.
+ * persistent execution"): a kernel launches a bounded grid and each CTA loops
+ * over items blockIdx.x, blockIdx.x + grid, ...  An item is a group of rows
+ * of one tensor (a CTA of `threads` threads holds threads / group rows); the
+ * items of the Q rows come first, then those of the K rows, so every CTA
+ * gets a near-equal share of each tensor's rows whatever the grid.  The
+ * planner launches as many CTAs as can be resident at once, except where a
+ * fused launch has at least 4 items per resident slot -- then 3 (below 6
+ * items per slot) or 4 CTAs per slot, so that the hardware hands the
+ * remaining items to the CTAs that finish first -- and the combine/apply
+ * pass over rows of 129..160 vectors, which also runs 4 per slot.  No CTA
+ * ever waits on another, so any grid is safe.
  *
  * Kernel kinds:
  *   QKN_KERNEL_REGISTER  one pass; the row (or head) is held in registers by
